@@ -1,0 +1,185 @@
+"""CPU oracle for the fine-grained MoE layer forward -- TEST INFRASTRUCTURE.
+
+Only the tests, the package smoke check and the bench's CPU-baseline leg may
+import this module.  The CUDA library never calls it and shares no code with it.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, double accumulation); this
+module only builds it with gcc and marshals numpy arrays.  bf16 tensors are
+passed as ``uint16`` arrays holding the raw bf16 bits.
+
+Sources, by page title and section:
+  * "DeepSeek V3 From Scratch" -- "The idea", "Worked example", "In code".
+  * "Scaling Efficiency: A Deep Dive into the DeepSeek-V3 Architecture" --
+    the DeepSeekMoE module sketch.
+  * kbwen.com DeepSeek tag page -- "A bias term for each expert".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32 = 0
+BF16 = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into liboracle.so next to it (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC",
+             "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i = ctypes.c_int
+        lib.orc_affinity.argtypes = [P, P, i, i, i, i, P]
+        lib.orc_select.argtypes = [P, P, i, i, i, P, P]
+        lib.orc_select.restype = i
+        lib.orc_histogram.argtypes = [P, i, i, i, P]
+        lib.orc_histogram.restype = i
+        lib.orc_bias_update.argtypes = [P, i, i, i, ctypes.c_float, P, P, P]
+        lib.orc_permute.argtypes = [P, i, i, i, P, P, P]
+        lib.orc_permute.restype = i
+        lib.orc_expert_accumulate.argtypes = [P, i, P, P, P, P, P, i, i, i, P]
+        lib.orc_finalize.argtypes = [P, ctypes.c_size_t, i, P]
+        lib.orc_layer_output.argtypes = [P, P, P, P, P, P, P, P, P, i, i, i, i, i, i, i, i, P]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.float32:
+        return F32
+    if a.dtype == np.uint16:
+        return BF16
+    raise TypeError(f"oracle takes float32 or bf16-as-uint16 arrays, got {a.dtype}")
+
+
+def _c(a, dtype=None):
+    a = np.ascontiguousarray(a if dtype is None else a.astype(dtype, copy=False))
+    return a
+
+
+def affinity(x: np.ndarray, w_gate: np.ndarray) -> np.ndarray:
+    """s = sigmoid(x @ W_g^T), double inside, fp32 out.  x [T][d], W_g [E][d]."""
+    x, w_gate = _c(x), _c(w_gate)
+    dt = _dtype_code(x)
+    assert _dtype_code(w_gate) == dt
+    T, d = x.shape
+    E = w_gate.shape[0]
+    s = np.empty((T, E), np.float32)
+    _load().orc_affinity(_ptr(x), _ptr(w_gate), dt, T, d, E, _ptr(s))
+    return s
+
+
+def select(s: np.ndarray, bias: np.ndarray, k: int):
+    """Top-k of fl32(s + b) by rank counting; weights from the unbiased s.
+
+    Returns (idx int32 [T][k], w float32 [T][k])."""
+    s, bias = _c(s, np.float32), _c(bias, np.float32)
+    T, E = s.shape
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float32)
+    rc = _load().orc_select(_ptr(s), _ptr(bias), T, E, k, _ptr(idx), _ptr(w))
+    if rc != 0:
+        raise ValueError("oracle select: a row did not fill k slots (non-finite scores)")
+    return idx, w
+
+
+def histogram(idx: np.ndarray, E: int) -> np.ndarray:
+    idx = _c(idx, np.int32)
+    T, k = idx.shape
+    counts = np.empty(E, np.int32)
+    if _load().orc_histogram(_ptr(idx), T, k, E, _ptr(counts)) != 0:
+        raise ValueError("oracle histogram: expert index out of range")
+    return counts
+
+
+def bias_update(counts: np.ndarray, bias: np.ndarray, T: int, k: int, step: float = 1e-3, target=None):
+    """Returns (new_bias, load) -- the sign-step update, fp32 throughout."""
+    counts = _c(counts, np.int32)
+    E = counts.shape[0]
+    b = np.array(bias, np.float32, copy=True)
+    load = np.empty(E, np.float32)
+    tgt = None if target is None else _c(target, np.float32)
+    _load().orc_bias_update(_ptr(counts), T, E, k, ctypes.c_float(step), _ptr(tgt), _ptr(b), _ptr(load))
+    return b, load
+
+
+def permute(idx: np.ndarray, E: int):
+    """Returns (offsets [E+1], perm_tok [T*k], inv_row [T*k]), all int32."""
+    idx = _c(idx, np.int32)
+    T, k = idx.shape
+    offsets = np.empty(E + 1, np.int32)
+    perm = np.empty(T * k, np.int32)
+    inv = np.empty(T * k, np.int32)
+    if _load().orc_permute(_ptr(idx), T, k, E, _ptr(offsets), _ptr(perm), _ptr(inv)) != 0:
+        raise ValueError("oracle permute: expert index out of range")
+    return offsets, perm, inv
+
+
+def expert_accumulate(x_rows, dest, wts, w1, w3, w2, yacc):
+    """yacc[dest[r]] += wts[r] * W2 (round(silu(W1 x) * W3 x)) for each row r."""
+    x_rows = _c(x_rows)
+    dt = _dtype_code(x_rows)
+    n, d = x_rows.shape
+    I = w1.shape[0]
+    dest = _c(dest, np.int32)
+    wts = _c(wts, np.float64)
+    w1, w3, w2 = _c(w1), _c(w3), _c(w2)
+    assert yacc.dtype == np.float64 and yacc.flags.c_contiguous
+    _load().orc_expert_accumulate(_ptr(x_rows), n, _ptr(dest), _ptr(wts), _ptr(w1), _ptr(w3), _ptr(w2),
+                                  d, I, dt, _ptr(yacc))
+
+
+def finalize(yacc: np.ndarray, like_dtype) -> np.ndarray:
+    out = np.empty(yacc.shape, like_dtype)
+    _load().orc_finalize(_ptr(np.ascontiguousarray(yacc)), yacc.size, _dtype_code(out), _ptr(out))
+    return out
+
+
+def layer_output(x, idx, w, w1, w3, w2, ws1, ws3, ws2) -> np.ndarray:
+    """Whole layer output y [T][d] (same dtype as x) for given routing."""
+    x = _c(x)
+    dt = _dtype_code(x)
+    T, d = x.shape
+    E, I, _ = w1.shape
+    S, Is, _ = ws1.shape
+    k = idx.shape[1]
+    idx = _c(idx, np.int32)
+    w = _c(w, np.float32)
+    arrs = [_c(a) for a in (w1, w3, w2, ws1, ws3, ws2)]
+    for a in arrs:
+        assert _dtype_code(a) == dt
+    y = np.empty((T, d), x.dtype)
+    _load().orc_layer_output(_ptr(x), _ptr(idx), _ptr(w), *[_ptr(a) for a in arrs], T, d, E, k, I, S, Is, dt,
+                             _ptr(y))
+    return y
+
+
+def route(x, w_gate, bias, k):
+    """The pages' route(): returns (weights, idx, s) computed entirely here."""
+    s = affinity(x, w_gate)
+    idx, w = select(s, bias, k)
+    return w, idx, s

@@ -1,0 +1,288 @@
+/*
+ * Reference oracle for the fine-grained MoE layer forward.  TEST
+ * INFRASTRUCTURE ONLY: the tests, the package's smoke check and the bench's
+ * CPU-baseline leg may call it; the product path never does.
+ *
+ * Plain, slow, obviously correct C.  Dot products accumulate in double over the
+ * exact input values (bf16 inputs are widened losslessly).  The router's fp32
+ * quantities (affinity, biased score, weights, load, bias) are rounded to fp32
+ * at the points the method defines them, so that integer decisions (top-k,
+ * counts, signs) are taken in fp32, the precision of the GPU path.
+ *
+ * It shares no code, header or constant with the CUDA library.
+ *
+ * Sources (web pages on DeepSeek-V3, cited by title and section):
+ *   [P1] "DeepSeek V3 From Scratch": "The idea", "Worked example", "In code"
+ *        (the route() and update_bias() sketches).
+ *   [P2] "Scaling Efficiency: A Deep Dive into the DeepSeek-V3 Architecture":
+ *        the DeepSeekMoE module sketch (shared + routed experts, weighted
+ *        combine loop).
+ *   [P3] kbwen.com DeepSeek tag page: "A bias term for each expert".
+ *
+ * Parity pins: every function below is pinned by the CPU tests against
+ * brute force, closed forms, invariants the pages state, or library
+ * routines on special cases -- except the general layer output for
+ * arbitrary shapes, which the pages pin only through its formula and the
+ * special cases (E = k = 1, W2 = 0, k = E).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_F32 0
+#define ORC_BF16 1
+
+/* ---- element access ---------------------------------------------------- */
+
+static double bf16_bits_to_double(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a float to bf16, round-to-nearest-even (NaN kept quiet). */
+static uint16_t float_to_bf16_bits(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) return (uint16_t)((u >> 16) | 0x40);
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+static double load_elem(const void* base, int dtype, size_t i) {
+    if (dtype == ORC_BF16) return bf16_bits_to_double(((const uint16_t*)base)[i]);
+    return (double)((const float*)base)[i];
+}
+
+static void store_elem(void* base, int dtype, size_t i, double v) {
+    float f = (float)v;
+    if (dtype == ORC_BF16)
+        ((uint16_t*)base)[i] = float_to_bf16_bits(f);
+    else
+        ((float*)base)[i] = f;
+}
+
+/* Value after the storage rounding of dtype (used for the documented bf16
+ * rounding of the SwiGLU intermediate h). */
+static double round_to_dtype(double v, int dtype) {
+    float f = (float)v;
+    if (dtype == ORC_BF16) return bf16_bits_to_double(float_to_bf16_bits(f));
+    return (double)f;
+}
+
+static double dot_rows(const void* a, size_t a_off, const void* b, size_t b_off, int dtype, int n) {
+    double acc = 0.0;
+    for (int c = 0; c < n; ++c) acc += load_elem(a, dtype, a_off + c) * load_elem(b, dtype, b_off + c);
+    return acc;
+}
+
+/* ---- router ------------------------------------------------------------ */
+
+/* Gate affinities [P1 "In code", route: sigmoid(x @ gate_w.T)].
+ * s[t][i] = fl32( 1 / (1 + exp(-sum_c x[t][c] * W_g[i][c])) ), the sum and the
+ * sigmoid in double.  x is [T][d], W_g is [E][d], both row-major in dtype. */
+void orc_affinity(const void* x, const void* w_gate, int dtype, int T, int d, int E, float* s_out) {
+    #pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        for (int i = 0; i < E; ++i) {
+            double z = dot_rows(x, (size_t)t * d, w_gate, (size_t)i * d, dtype, d);
+            s_out[(size_t)t * E + i] = (float)(1.0 / (1.0 + exp(-z)));
+        }
+    }
+}
+
+/* Bias-shifted top-k and unbiased, renormalised weights
+ * [P1 "In code", route; P1 "The idea"; P3 "A bias term for each expert"].
+ *
+ * v_i = fl32(s_i + b_i).  Selection by rank counting:
+ *   rank_i = #{ j : v_j > v_i  or  (v_j == v_i and j < i) }
+ * expert i is chosen iff rank_i < k, and it occupies slot rank_i, so slots are
+ * ordered by descending v with ties going to the lower expert index.
+ * Weights use the UNBIASED s: den = fl32 sum of s over slots 0..k-1 in slot
+ * order, w_j = fl32(s_idx_j / den).
+ * Returns 0, or -1 if a row does not fill k slots (NaN scores). */
+int orc_select(const float* s, const float* bias, int T, int E, int k, int32_t* idx, float* w) {
+    int bad = 0;
+    #pragma omp parallel for schedule(static) reduction(| : bad)
+    for (int t = 0; t < T; ++t) {
+        const float* st = s + (size_t)t * E;
+        float* v = (float*)malloc(sizeof(float) * (size_t)E);
+        for (int i = 0; i < E; ++i) {
+            volatile float vi = st[i] + bias[i]; /* one fp32 add, no contraction */
+            v[i] = vi;
+        }
+        int filled = 0;
+        for (int i = 0; i < E; ++i) {
+            int rank = 0;
+            for (int j = 0; j < E; ++j)
+                if (v[j] > v[i] || (v[j] == v[i] && j < i)) ++rank;
+            if (rank < k && v[i] == v[i]) {
+                idx[(size_t)t * k + rank] = i;
+                ++filled;
+            }
+        }
+        free(v);
+        if (filled != k) { bad = 1; continue; }
+        float den = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            volatile float nd = den + st[idx[(size_t)t * k + j]];
+            den = nd;
+        }
+        for (int j = 0; j < k; ++j) {
+            volatile float q = st[idx[(size_t)t * k + j]] / den;
+            w[(size_t)t * k + j] = q;
+        }
+    }
+    return bad ? -1 : 0;
+}
+
+/* Per-expert load histogram over the whole batch of the step
+ * [P1 "In code", update_bias comment "load: fraction of tokens per expert";
+ *  P3 "A bias term for each expert"].  c_i = #{(t, j) : idx[t][j] = i}.
+ * Returns -1 if an index is out of range. */
+int orc_histogram(const int32_t* idx, int T, int k, int E, int32_t* counts) {
+    for (int i = 0; i < E; ++i) counts[i] = 0;
+    for (size_t a = 0; a < (size_t)T * k; ++a) {
+        int e = idx[a];
+        if (e < 0 || e >= E) return -1;
+        counts[e] += 1;
+    }
+    return 0;
+}
+
+/* Auxiliary-loss-free bias update, applied once at the end of the step
+ * [P1 "In code", update_bias: bias + step * sign(target - load);
+ *  P3 "A bias term for each expert": fixed amount, down for overloaded,
+ *  up for underloaded].
+ * load_i = fl32(c_i / T), target_i = target ? target[i] : fl32(k / E),
+ * delta_i = sign(fl32(target_i - load_i)) in {-1, 0, +1},
+ * b_i = fl32(b_i + delta_i * fl32(step)).  load_out may be NULL. */
+void orc_bias_update(const int32_t* counts, int T, int E, int k, float step, const float* target,
+                     float* bias, float* load_out) {
+    for (int i = 0; i < E; ++i) {
+        volatile float load = (float)counts[i] / (float)T;
+        volatile float tgt = target ? target[i] : (float)k / (float)E;
+        volatile float diff = tgt - load;
+        float sgn = diff > 0.0f ? 1.0f : (diff < 0.0f ? -1.0f : 0.0f);
+        volatile float nb = bias[i] + sgn * step;
+        bias[i] = nb;
+        if (load_out) load_out[i] = load;
+    }
+}
+
+/* ---- permutation ------------------------------------------------------- */
+
+/* Expert-contiguous order ["Tokens routed to the same expert can be batched
+ * together", locionic.com DeepSeek V3 Architecture Deep Dive, "Throughput on
+ * NVIDIA H100/H800"].  Rows are ordered by (expert ascending, token
+ * ascending); offsets[e] = first row of expert e, offsets[E] = T*k;
+ * perm_tok[row] = t*k + j (the assignment held by that row);
+ * inv_row[t*k + j] = row.  Returns -1 on an out-of-range index. */
+int orc_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_t* perm_tok, int32_t* inv_row) {
+    int32_t* counts = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+    if (orc_histogram(idx, T, k, E, counts) != 0) { free(counts); return -1; }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t* cursor = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+    for (int e = 0; e < E; ++e) cursor[e] = offsets[e];
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int e = idx[(size_t)t * k + j];
+            int row = cursor[e]++;
+            perm_tok[row] = t * k + j;
+            inv_row[(size_t)t * k + j] = row;
+        }
+    }
+    free(cursor);
+    free(counts);
+    return 0;
+}
+
+/* ---- experts and combine ----------------------------------------------- */
+
+/* One SwiGLU expert applied to n token rows, accumulated into a double buffer
+ * [P2 DeepSeekMoE sketch: routed_out[mask] += w * expert(x[mask]); the expert
+ *  MLP is SwiGLU without biases]:
+ *   a = W1 x,  g = W3 x            (W1, W3: [I][d], row-major, dtype)
+ *   h = round_dtype( a / (1 + exp(-a)) * g )   (h stored in dtype once)
+ *   o = W2 h                       (W2: [d][I], row-major, dtype)
+ *   yacc[dest[r]][:] += wts[r] * o
+ * x_rows is [n][d] in dtype.  W2 may be addressed with a row stride (ld2)
+ * and W1/W3 likewise (ld1) so a shared expert of a stacked tensor can be
+ * passed without copying. */
+void orc_expert_accumulate(const void* x_rows, int n, const int32_t* dest, const double* wts,
+                           const void* w1, const void* w3, const void* w2, int d, int I, int dtype,
+                           double* yacc) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < n; ++r) {
+        double* h = (double*)malloc(sizeof(double) * (size_t)I);
+        for (int c = 0; c < I; ++c) {
+            double a = dot_rows(w1, (size_t)c * d, x_rows, (size_t)r * d, dtype, d);
+            double g = dot_rows(w3, (size_t)c * d, x_rows, (size_t)r * d, dtype, d);
+            double silu = a / (1.0 + exp(-a));
+            h[c] = round_to_dtype(silu * g, dtype);
+        }
+        double* yr = yacc + (size_t)dest[r] * d;
+        for (int o = 0; o < d; ++o) {
+            double acc = 0.0;
+            for (int c = 0; c < I; ++c) acc += load_elem(w2, dtype, (size_t)o * I + c) * h[c];
+            /* rows of one call never share a destination (one expert per
+             * token), so the update is race-free */
+            yr[o] += wts[r] * acc;
+        }
+        free(h);
+    }
+}
+
+/* Round the double accumulator to the output dtype once
+ * [P2 DeepSeekMoE sketch: shared_out + routed_out]. */
+void orc_finalize(const double* yacc, size_t n, int dtype, void* y_out) {
+    for (size_t i = 0; i < n; ++i) store_elem(y_out, dtype, i, yacc[i]);
+}
+
+/* Whole layer for small cases, in the order of the pages' forward:
+ * shared expert(s) on every token, then for each routed expert e the tokens
+ * routed to it, weighted by the unbiased weight of that slot.
+ * idx/w are the routing decisions (from orc_select, or injected).
+ * Natural layouts: W1, W3 [E][I][d]; W2 [E][d][I]; Ws1, Ws3 [S][Is][d];
+ * Ws2 [S][d][Is].  y is [T][d] in dtype. */
+void orc_layer_output(const void* x, const int32_t* idx, const float* w, const void* w1, const void* w3,
+                      const void* w2, const void* ws1, const void* ws3, const void* ws2, int T, int d, int E,
+                      int k, int I, int S, int Is, int dtype, void* y) {
+    size_t esz = dtype == ORC_BF16 ? 2 : 4;
+    double* yacc = (double*)calloc((size_t)T * d, sizeof(double));
+    int32_t* dest = (int32_t*)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1));
+    double* wts = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    char* rows = (char*)malloc(esz * (size_t)(T > 0 ? T : 1) * d);
+    /* shared experts: weight 1 on every token */
+    for (int s = 0; s < S; ++s) {
+        for (int t = 0; t < T; ++t) { dest[t] = t; wts[t] = 1.0; }
+        orc_expert_accumulate(x, T, dest, wts, (const char*)ws1 + esz * (size_t)s * Is * d,
+                              (const char*)ws3 + esz * (size_t)s * Is * d, (const char*)ws2 + esz * (size_t)s * d * Is,
+                              d, Is, dtype, yacc);
+    }
+    /* routed experts: the tokens whose top-k holds e */
+    for (int e = 0; e < E; ++e) {
+        int n = 0;
+        for (int t = 0; t < T; ++t)
+            for (int j = 0; j < k; ++j)
+                if (idx[(size_t)t * k + j] == e) {
+                    memcpy(rows + esz * (size_t)n * d, (const char*)x + esz * (size_t)t * d, esz * (size_t)d);
+                    dest[n] = t;
+                    wts[n] = (double)w[(size_t)t * k + j];
+                    ++n;
+                }
+        if (n == 0) continue;
+        orc_expert_accumulate(rows, n, dest, wts, (const char*)w1 + esz * (size_t)e * I * d,
+                              (const char*)w3 + esz * (size_t)e * I * d, (const char*)w2 + esz * (size_t)e * d * I, d, I,
+                              dtype, yacc);
+    }
+    orc_finalize(yacc, (size_t)T * d, dtype, y);
+    free(rows);
+    free(wts);
+    free(dest);
+    free(yacc);
+}
