@@ -1,0 +1,179 @@
+"""B200 (sm_100a) fine-grained MoE layer forward -- Python binding.
+
+A thin ctypes binding over ``libmoe_gate.so`` (the C ABI in
+``include/moe_gate.h``): each function has the C entry point's name and
+arguments, takes torch tensors (or raw device pointers as ints) and raises
+``MoEError`` on a non-OK status.  Every step of the layer runs in the
+library's CUDA kernels; PyTorch only provides device memory and streams.
+There is no CPU fallback: if the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_gate.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+
+STATUS = {
+    0: "MOE_OK",
+    1: "MOE_ERR_INVALID_ARG",
+    2: "MOE_ERR_UNSUPPORTED",
+    3: "MOE_ERR_ALIGNMENT",
+    4: "MOE_ERR_WORKSPACE",
+    5: "MOE_ERR_CUDA",
+    6: "MOE_ERR_DEVICE_CHECK",
+    7: "MOE_ERR_TIMEOUT",
+}
+
+EXPORTS = (
+    "moe_route", "moe_load_and_bias_update", "moe_permute", "moe_permute_workspace_size", "moe_grouped_swiglu",
+    "moe_grouped_swiglu_workspace_size", "moe_combine", "moe_layer_forward", "moe_workspace_size",
+    "moe_get_last_error", "moe_status_string", "moe_abi_version",
+)
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class MoEShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("I", ctypes.c_int32), ("S", ctypes.c_int32), ("Is", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "MoEShape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def shape_of(cfg, T: int | None = None) -> MoEShape:
+    """MoEShape from a workload config (``inputs.MoEConfig``)."""
+    return MoEShape(cfg.T if T is None else T, cfg.d, cfg.E, cfg.k, cfg.I, cfg.S, cfg.Is,
+                    MOE_BF16 if cfg.dtype == "bf16" else MOE_F32)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises MoEError-free ImportError if it is not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m fine_grained_moe_gate_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S, F = ctypes.c_void_p, MoEShape, ctypes.c_float
+        sz = ctypes.c_size_t
+        sig = {
+            "moe_route": [P, P, P, S, P, P, P, P, P],
+            "moe_load_and_bias_update": [P, S, F, P, P, P, P],
+            "moe_permute": [P, P, P, S, P, P, P, P, P, sz, P],
+            "moe_grouped_swiglu": [P, P, P, P, P, P, P, P, P, S, P, P, P, sz, P],
+            "moe_combine": [P, P, P, P, S, P, P],
+            "moe_layer_forward": [P, P, P, P, P, P, P, P, P, S, P, P, P, P, P, sz, P],
+            "moe_get_last_error": [P],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        for name in ("moe_workspace_size", "moe_permute_workspace_size", "moe_grouped_swiglu_workspace_size"):
+            fn = getattr(L, name)
+            fn.argtypes = [S]
+            fn.restype = sz
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_abi_version.argtypes = []
+        L.moe_abi_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    """Device pointer of a tensor (None -> NULL; an int is taken as a pointer)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise MoEError(status, where)
+
+
+def _nbytes(t) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+# ---- entry points (same names and argument order as moe_gate.h) -----------
+
+def moe_route(x, w_gate, bias, shape, topk_idx, topk_w, counts, affinity_out=None, stream=None):
+    _check(lib().moe_route(_p(x), _p(w_gate), _p(bias), shape, _p(topk_idx), _p(topk_w), _p(counts),
+                           _p(affinity_out), _stream(stream)), "moe_route")
+
+
+def moe_load_and_bias_update(counts, shape, step, target, bias, load_out=None, stream=None):
+    _check(lib().moe_load_and_bias_update(_p(counts), shape, ctypes.c_float(step), _p(target), _p(bias), _p(load_out),
+                                          _stream(stream)), "moe_load_and_bias_update")
+
+
+def moe_permute(x, topk_idx, counts, shape, x_perm, offsets, perm_tok, inv_row, workspace, stream=None):
+    _check(lib().moe_permute(_p(x), _p(topk_idx), _p(counts), shape, _p(x_perm), _p(offsets), _p(perm_tok),
+                             _p(inv_row), _p(workspace), _nbytes(workspace), _stream(stream)), "moe_permute")
+
+
+def moe_grouped_swiglu(x_perm, offsets, w1, w3, w2, x, ws1, ws3, ws2, shape, y_perm, shared_out, workspace,
+                       stream=None):
+    _check(lib().moe_grouped_swiglu(_p(x_perm), _p(offsets), _p(w1), _p(w3), _p(w2), _p(x), _p(ws1), _p(ws3),
+                                    _p(ws2), shape, _p(y_perm), _p(shared_out), _p(workspace), _nbytes(workspace),
+                                    _stream(stream)), "moe_grouped_swiglu")
+
+
+def moe_combine(y_perm, topk_w, inv_row, shared_out, shape, y, stream=None):
+    _check(lib().moe_combine(_p(y_perm), _p(topk_w), _p(inv_row), _p(shared_out), shape, _p(y), _stream(stream)),
+           "moe_combine")
+
+
+def moe_layer_forward(x, w_gate, bias, w1, w3, w2, ws1, ws3, ws2, shape, y, topk_idx, topk_w, counts, workspace,
+                      stream=None):
+    _check(lib().moe_layer_forward(_p(x), _p(w_gate), _p(bias), _p(w1), _p(w3), _p(w2), _p(ws1), _p(ws3), _p(ws2),
+                                   shape, _p(y), _p(topk_idx), _p(topk_w), _p(counts), _p(workspace),
+                                   _nbytes(workspace), _stream(stream)), "moe_layer_forward")
+
+
+def moe_workspace_size(shape) -> int:
+    return lib().moe_workspace_size(shape)
+
+
+def moe_permute_workspace_size(shape) -> int:
+    return lib().moe_permute_workspace_size(shape)
+
+
+def moe_grouped_swiglu_workspace_size(shape) -> int:
+    return lib().moe_grouped_swiglu_workspace_size(shape)
+
+
+def moe_get_last_error(stream=None) -> int:
+    return lib().moe_get_last_error(_stream(stream))
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+def moe_abi_version() -> int:
+    return lib().moe_abi_version()

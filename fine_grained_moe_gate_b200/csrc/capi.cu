@@ -1,0 +1,337 @@
+// C ABI entry points (moe_gate.h): host-side validation, workspace carving
+// and kernel launches.  Nothing here allocates device memory.
+#include "../../include/moe_gate.h"
+#include "kernels.h"
+
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+namespace {
+
+// Per-device status word written by kernels on an anomaly.
+__device__ int g_status_word;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices];
+int g_num_sms[kMaxDevices];
+std::mutex g_setup_mu;
+
+// Per-device set-up, once: the status word's device address and SM count.
+moe_status device_setup(int* dev_out, int** status_out, int* sms_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_setup_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return MOE_ERR_CUDA;
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+        g_num_sms[dev] = sms;
+        g_status_ptr[dev] = static_cast<int*>(p);
+    }
+    *dev_out = dev;
+    *status_out = g_status_ptr[dev];
+    *sms_out = g_num_sms[dev];
+    return MOE_OK;
+}
+
+inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+inline size_t esize(const moe_shape& sh) { return sh.dtype == MOE_BF16 ? 2 : 4; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status validate_shape(const moe_shape& sh) {
+    if (sh.dtype != MOE_F32 && sh.dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (sh.T < 0 || sh.d <= 0 || sh.E <= 0 || sh.k <= 0 || sh.I <= 0 || sh.S < 0) return MOE_ERR_INVALID_ARG;
+    if (sh.S > 0 && sh.Is <= 0) return MOE_ERR_INVALID_ARG;
+    if (sh.k > sh.E) return MOE_ERR_INVALID_ARG;
+    if (sh.k > 16 || sh.E > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    if (sh.d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    // 32-bit row coordinates (tensor maps, row indices)
+    if ((long long)sh.T * sh.k >= (1ll << 31) || (long long)sh.E * sh.I >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+    if (sh.dtype == MOE_BF16) {
+        if (sh.d % 64 != 0 || sh.I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+        if (sh.S > 0 && sh.Is % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    }
+    return MOE_OK;
+}
+
+#define MOE_REQUIRE(cond, code) \
+    do {                        \
+        if (!(cond)) return (code); \
+    } while (0)
+
+#define MOE_CUDA(call)                                   \
+    do {                                                 \
+        if ((call) != cudaSuccess) return MOE_ERR_CUDA;  \
+    } while (0)
+
+size_t permute_ws(const moe_shape& sh) { return align256(moe::permute_scratch_bytes(sh.T, sh.E)); }
+size_t swiglu_ws(const moe_shape& sh) {
+    const size_t eb = esize(sh);
+    return align256((size_t)sh.T * sh.k * sh.I * eb) + align256((size_t)sh.T * sh.S * (size_t)sh.Is * eb);
+}
+
+// ---- internal stages (arguments already validated) -----------------------
+
+moe_status do_route(const void* x, const void* w_gate, const float* bias, const moe_shape& sh, int32_t* idx,
+                    float* w, int32_t* counts, float* aff, int* status, int sms, cudaStream_t st) {
+    MOE_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * sh.E, st));
+    if (sh.T == 0) return MOE_OK;
+    cudaError_t err;
+    if (sh.dtype == MOE_BF16)
+        err = moe::launch_router_tc(x, w_gate, bias, sh.T, sh.d, sh.E, sh.k, idx, w, counts, aff, status, sms, st);
+    else
+        err = moe::launch_router_simt(x, w_gate, bias, sh.T, sh.d, sh.E, sh.k, false, idx, w, counts, aff, status,
+                                      st);
+    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status do_permute(const void* x, const int32_t* idx, const int32_t* counts, const moe_shape& sh, void* x_perm,
+                      int32_t* offsets, int32_t* perm, int32_t* inv, void* ws, int* status, cudaStream_t st) {
+    cudaError_t err = moe::launch_permute(x, idx, counts, sh.T, sh.d, sh.E, sh.k, esize(sh), x_perm, offsets, perm,
+                                          inv, static_cast<int32_t*>(ws), status, st);
+    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3, const void* w2,
+                     const void* x, const void* ws1, const void* ws3, const void* ws2, const moe_shape& sh,
+                     void* y_perm, void* shared_out, void* ws, int* status, int sms, cudaStream_t st) {
+    const size_t eb = esize(sh);
+    const long long rows = (long long)sh.T * sh.k;
+    char* h = static_cast<char*>(ws);
+    char* hs = h + align256((size_t)rows * sh.I * eb);
+    const bool shared = x && sh.S > 0 && shared_out;
+    const int Ks = sh.S * sh.Is;
+    if (sh.T == 0) return MOE_OK;
+    if (sh.dtype == MOE_BF16) {
+        moe::TcUpArgs up{x_perm, rows, w1, w3, (long long)sh.E * sh.I, h, sh.d, sh.I, offsets, sh.E, 0};
+        if (moe::launch_tc_up(up, status, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+        if (shared) {
+            moe::TcUpArgs su{x, sh.T, ws1, ws3, (long long)Ks, hs, sh.d, Ks, nullptr, 1, sh.T};
+            if (moe::launch_tc_up(su, status, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+        }
+        moe::TcDownArgs dn{h, rows, w2, 1, sh.I, y_perm, sh.d, sh.I, offsets, sh.E, 0};
+        if (moe::launch_tc_down(dn, status, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+        if (shared) {
+            moe::TcDownArgs sd{hs, sh.T, ws2, sh.S, sh.Is, shared_out, sh.d, Ks, nullptr, 1, sh.T};
+            if (moe::launch_tc_down(sd, status, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+        }
+        return MOE_OK;
+    }
+    // fp32: SIMT grouped GEMMs
+    moe::GemmArgs up{x_perm, sh.d, w1, w3, (long long)sh.I * sh.d, sh.d, sh.d, 0, h, sh.I, sh.I, sh.d,
+                     offsets, sh.E, (int)rows};
+    if (moe::launch_simt_gemm(up, false, true, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+    moe::GemmArgs dn{h, sh.I, w2, nullptr, (long long)sh.d * sh.I, sh.I, sh.I, 0, y_perm, sh.d, sh.d, sh.I,
+                     offsets, sh.E, (int)rows};
+    if (moe::launch_simt_gemm(dn, false, false, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (shared) {
+        // S stacked [Is][d] blocks are one [S*Is][d] matrix for the up side
+        moe::GemmArgs su{x, sh.d, ws1, ws3, 0, sh.d, sh.d, 0, hs, Ks, Ks, sh.d, nullptr, 1, sh.T};
+        if (moe::launch_simt_gemm(su, false, true, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+        moe::GemmArgs sd{hs, Ks, ws2, nullptr, 0, sh.Is, sh.Is, (long long)sh.d * sh.Is, shared_out, sh.d, sh.d, Ks,
+                         nullptr, 1, sh.T};
+        if (moe::launch_simt_gemm(sd, false, false, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return 100; }
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case MOE_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_DEVICE_CHECK: return "device-side consistency check failed";
+        case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+size_t moe_permute_workspace_size(moe_shape sh) {
+    if (validate_shape(sh) != MOE_OK) return 0;
+    return permute_ws(sh);
+}
+
+size_t moe_grouped_swiglu_workspace_size(moe_shape sh) {
+    if (validate_shape(sh) != MOE_OK) return 0;
+    return swiglu_ws(sh);
+}
+
+size_t moe_workspace_size(moe_shape sh) {
+    if (validate_shape(sh) != MOE_OK) return 0;
+    const size_t rows = (size_t)sh.T * sh.k;
+    return align256((sh.E + 1) * sizeof(int32_t)) + 2 * align256(rows * sizeof(int32_t)) + permute_ws(sh) +
+           align256(rows * sh.d * esize(sh)) + swiglu_ws(sh) + align256((size_t)sh.T * sh.d * esize(sh));
+}
+
+moe_status moe_route(const void* x, const void* w_gate, const float* bias, moe_shape sh, int32_t* topk_idx,
+                     float* topk_w, int32_t* counts, float* affinity_out, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(w_gate && bias && counts, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (x && topk_idx && topk_w), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x) && aligned16(w_gate) && aligned16(bias) && aligned16(topk_idx) && aligned16(topk_w) &&
+                    aligned16(counts) && aligned16(affinity_out),
+                MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_route(x, w_gate, bias, sh, topk_idx, topk_w, counts, affinity_out, status, sms,
+                    static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_load_and_bias_update(const int32_t* counts, moe_shape sh, float step, const float* target, float* bias,
+                                    float* load_out, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(sh.T > 0, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(counts && bias, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(step == step, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(counts) && aligned16(bias) && aligned16(target) && aligned16(load_out), MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return moe::launch_bias_update(counts, sh.T, sh.E, sh.k, step, target, bias, load_out,
+                                   static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_permute(const void* x, const int32_t* topk_idx, const int32_t* counts, moe_shape sh, void* x_perm,
+                       int32_t* offsets, int32_t* perm_tok, int32_t* inv_row, void* workspace, size_t ws_bytes,
+                       void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(offsets, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (x && topk_idx && x_perm && perm_tok && inv_row), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x) && aligned16(topk_idx) && aligned16(counts) && aligned16(x_perm) && aligned16(offsets) &&
+                    aligned16(perm_tok) && aligned16(inv_row),
+                MOE_ERR_ALIGNMENT);
+    MOE_REQUIRE(ws_bytes >= permute_ws(sh) && (workspace || permute_ws(sh) == 0), MOE_ERR_WORKSPACE);
+    MOE_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_permute(x, topk_idx, counts, sh, x_perm, offsets, perm_tok, inv_row, workspace, status,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_grouped_swiglu(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3,
+                              const void* w2, const void* x, const void* ws1, const void* ws3, const void* ws2,
+                              moe_shape sh, void* y_perm, void* shared_out, void* workspace, size_t ws_bytes,
+                              void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(offsets && w1 && w3 && w2, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (x_perm && y_perm), MOE_ERR_INVALID_ARG);
+    const bool shared = x != nullptr && sh.S > 0;
+    MOE_REQUIRE(!shared || (ws1 && ws3 && ws2 && shared_out), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x_perm) && aligned16(offsets) && aligned16(w1) && aligned16(w3) && aligned16(w2) &&
+                    aligned16(x) && aligned16(ws1) && aligned16(ws3) && aligned16(ws2) && aligned16(y_perm) &&
+                    aligned16(shared_out),
+                MOE_ERR_ALIGNMENT);
+    MOE_REQUIRE(ws_bytes >= swiglu_ws(sh) && (workspace || swiglu_ws(sh) == 0), MOE_ERR_WORKSPACE);
+    MOE_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_swiglu(x_perm, offsets, w1, w3, w2, shared ? x : nullptr, ws1, ws3, ws2, sh, y_perm, shared_out,
+                     workspace, status, sms, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine(const void* y_perm, const float* topk_w, const int32_t* inv_row, const void* shared_out,
+                       moe_shape sh, void* y, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(sh.T == 0 || (y_perm && topk_w && inv_row && y), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(y_perm) && aligned16(topk_w) && aligned16(inv_row) && aligned16(shared_out) && aligned16(y),
+                MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return moe::launch_combine(y_perm, topk_w, inv_row, shared_out, sh.T, sh.d, sh.k, sh.dtype == MOE_BF16, y, status,
+                               static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bias, const void* w1, const void* w3,
+                             const void* w2, const void* ws1, const void* ws3, const void* ws2, moe_shape sh, void* y,
+                             int32_t* topk_idx, float* topk_w, int32_t* counts, void* workspace, size_t ws_bytes,
+                             void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(w_gate && bias && w1 && w3 && w2 && counts, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.S == 0 || (ws1 && ws3 && ws2), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (x && y && topk_idx && topk_w), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x) && aligned16(w_gate) && aligned16(bias) && aligned16(w1) && aligned16(w3) &&
+                    aligned16(w2) && aligned16(ws1) && aligned16(ws3) && aligned16(ws2) && aligned16(y) &&
+                    aligned16(topk_idx) && aligned16(topk_w) && aligned16(counts),
+                MOE_ERR_ALIGNMENT);
+    const size_t need = moe_workspace_size(sh);
+    MOE_REQUIRE(workspace && ws_bytes >= need, MOE_ERR_WORKSPACE);
+    MOE_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    const size_t rows = (size_t)sh.T * sh.k;
+    const size_t eb = esize(sh);
+    char* p = static_cast<char*>(workspace);
+    int32_t* offsets = reinterpret_cast<int32_t*>(p);
+    p += align256((sh.E + 1) * sizeof(int32_t));
+    int32_t* perm = reinterpret_cast<int32_t*>(p);
+    p += align256(rows * sizeof(int32_t));
+    int32_t* inv = reinterpret_cast<int32_t*>(p);
+    p += align256(rows * sizeof(int32_t));
+    void* pws = p;
+    p += permute_ws(sh);
+    void* x_perm = p;  // reused for y_perm once the up projection has read it
+    p += align256(rows * sh.d * eb);
+    void* gws = p;
+    p += swiglu_ws(sh);
+    void* shared_out = sh.S > 0 ? p : nullptr;
+
+    if ((v = do_route(x, w_gate, bias, sh, topk_idx, topk_w, counts, nullptr, status, sms, st)) != MOE_OK) return v;
+    if (sh.T == 0) return MOE_OK;
+    if ((v = do_permute(x, topk_idx, counts, sh, x_perm, offsets, perm, inv, pws, status, st)) != MOE_OK) return v;
+    if ((v = do_swiglu(x_perm, offsets, w1, w3, w2, sh.S > 0 ? x : nullptr, ws1, ws3, ws2, sh, x_perm, shared_out, gws,
+                       status, sms, st)) != MOE_OK)
+        return v;
+    return moe::launch_combine(x_perm, topk_w, inv, shared_out, sh.T, sh.d, sh.k, sh.dtype == MOE_BF16, y, status,
+                               st) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_get_last_error(void* stream) {
+    int dev, sms;
+    int* status;
+    moe_status v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    MOE_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    int h = 0;
+    MOE_CUDA(cudaMemcpy(&h, status, sizeof(int), cudaMemcpyDeviceToHost));
+    const int zero = 0;
+    MOE_CUDA(cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice));
+    return static_cast<moe_status>(h);
+}
+
+}  // extern "C"

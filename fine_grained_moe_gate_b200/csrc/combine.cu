@@ -1,0 +1,100 @@
+// Weighted combine back into token order ("Scaling Efficiency: A Deep Dive
+// into the DeepSeek-V3 Architecture", DeepSeekMoE sketch: each routed
+// expert's output scaled by its gate weight and added to the token, plus the
+// shared experts' output):
+//   y[t] = shared[t] + sum_j w[t][j] * y_perm[inv_row[t*k + j]]
+// fp32 accumulation in that fixed order (deterministic), one rounding to the
+// output type.  One CTA per token, 16-byte vector loads.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+template <typename T>
+struct Vec;
+template <>
+struct Vec<float> {
+    static constexpr int n = 4;
+    __device__ static void unpack(const uint4& u, float* f) {
+        f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+        f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+    }
+    __device__ static uint4 pack(const float* f) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
+    }
+};
+template <>
+struct Vec<__nv_bfloat16> {
+    static constexpr int n = 8;
+    __device__ static void unpack(const uint4& u, float* f) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ static uint4 pack(const float* f) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 b = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+template <typename T>
+__global__ void combine_kernel(const uint4* __restrict__ y_perm, const float* __restrict__ w,
+                               const int32_t* __restrict__ inv_row, const uint4* __restrict__ shared, int k,
+                               int vec_per_row, int total_rows, uint4* __restrict__ y, int* status) {
+    constexpr int n = Vec<T>::n;
+    const int t = blockIdx.x;
+    __shared__ int rows[16];
+    __shared__ float ws[16];
+    if (threadIdx.x < k) {
+        const int r = inv_row[(size_t)t * k + threadIdx.x];
+        if ((unsigned)r >= (unsigned)total_rows) report(status, kStDeviceCheck);
+        rows[threadIdx.x] = r;
+        ws[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) {
+        float acc[n], tmp[n];
+        if (shared) {
+            Vec<T>::unpack(shared[(size_t)t * vec_per_row + v], acc);
+        } else {
+#pragma unroll
+            for (int i = 0; i < n; ++i) acc[i] = 0.f;
+        }
+        for (int j = 0; j < k; ++j) {
+            const int r = rows[j];
+            if ((unsigned)r >= (unsigned)total_rows) continue;
+            Vec<T>::unpack(y_perm[(size_t)r * vec_per_row + v], tmp);
+            const float wj = ws[j];
+#pragma unroll
+            for (int i = 0; i < n; ++i) acc[i] = fmaf(wj, tmp[i], acc[i]);
+        }
+        y[(size_t)t * vec_per_row + v] = Vec<T>::pack(acc);
+    }
+}
+
+cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* inv_row, const void* shared, int T,
+                           int d, int k, bool bf16, void* y, int* status, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const size_t eb = bf16 ? 2 : 4;
+    const int vec = (int)((size_t)d * eb / 16);
+    const int threads = vec >= 256 ? 256 : ((vec + 31) / 32) * 32;
+    if (bf16)
+        combine_kernel<__nv_bfloat16><<<T, threads, 0, st>>>(static_cast<const uint4*>(y_perm), w, inv_row,
+                                                              static_cast<const uint4*>(shared), k, vec, T * k,
+                                                              static_cast<uint4*>(y), status);
+    else
+        combine_kernel<float><<<T, threads, 0, st>>>(static_cast<const uint4*>(y_perm), w, inv_row,
+                                                      static_cast<const uint4*>(shared), k, vec, T * k,
+                                                      static_cast<uint4*>(y), status);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,95 @@
+// Internal launchers of the MoE kernels (host side).  Not part of the ABI;
+// the entry points in capi.cu validate arguments before calling these.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxExperts = 256;
+constexpr int kMaxGroups = kMaxExperts;
+
+// One grouped GEMM C = A . B^T (optionally with the SwiGLU pair B0/B1).
+// Group g: rows [offsets[g], offsets[g+1]) of A and C, all inside [0, M)
+// (or [0, M) itself when offsets is null and G == 1); B block g starts b_gstride elements after
+// block g-1.  Element (n, kk) of a B block sits at
+//   (kk / kseg) * seg_stride + n * ldb + (kk % kseg)
+// which covers both a plain [N][K] matrix (kseg = K) and S stacked
+// [N][Is] matrices contracted over their concatenated K (kseg = Is).
+struct GemmArgs {
+    const void* A;
+    int lda;
+    const void* B0;
+    const void* B1;
+    long long b_gstride;
+    int ldb;
+    int kseg;
+    long long seg_stride;
+    void* C;
+    int ldc;
+    int N, K;
+    const int32_t* offsets;
+    int G;
+    int M;
+};
+
+// router.cu
+cudaError_t launch_router_simt(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
+                               bool bf16, int32_t* idx, float* w, int32_t* counts, float* aff, int* status,
+                               cudaStream_t st);
+size_t router_simt_smem(int E);
+cudaError_t launch_bias_update(const int32_t* counts, int T, int E, int k, float step, const float* target,
+                               float* bias, float* load_out, cudaStream_t st);
+
+// router_tc.cu (bf16, tensor cores)
+cudaError_t launch_router_tc(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
+                             int32_t* idx, float* w, int32_t* counts, float* aff, int* status, int num_sms,
+                             cudaStream_t st);
+
+// permute.cu
+size_t permute_scratch_bytes(int T, int E);
+cudaError_t launch_permute(const void* x, const int32_t* idx, const int32_t* counts, int T, int d, int E, int k,
+                           size_t elem_bytes, void* x_perm, int32_t* offsets, int32_t* perm_tok, int32_t* inv_row,
+                           int32_t* scratch, int* status, cudaStream_t st);
+
+// gemm_simt.cu
+cudaError_t launch_simt_gemm(const GemmArgs& p, bool bf16, bool swiglu, int num_sms, cudaStream_t st);
+
+// gemm_tc.cu (bf16, tensor cores)
+// Up projection with fused SwiGLU: h[r][n] = silu(A W1^T) * (A W3^T).
+//   A: [rows][d] (x_perm, or x for the shared group), W1/W3 row blocks of I
+//   rows per group, h: [rows][I].
+struct TcUpArgs {
+    const void* A;          // [A_rows][d] bf16
+    long long A_rows;
+    const void* W1;         // [G * I][d] bf16 (groups stacked)
+    const void* W3;
+    long long W_rows;       // G * I
+    void* H;                // [A_rows][I] bf16
+    int d, I;
+    const int32_t* offsets; // group rows; null: one group of M rows
+    int G, M;
+};
+// Down projection: Y[r][:] = H[r] . W2_g^T, W2_g = [d][K] (K = I), or for
+// the shared group S stacked [d][Is] blocks contracted over K = S * Is.
+struct TcDownArgs {
+    const void* H;          // [H_rows][K] bf16
+    long long H_rows;
+    const void* W2;         // [G][d][kseg] bf16 (G = groups, or S for shared)
+    int nseg;               // K / kseg segments (1 routed, S shared)
+    int kseg;
+    void* Y;                // [H_rows][d] bf16
+    int d, K;
+    const int32_t* offsets;
+    int G, M;
+};
+cudaError_t launch_tc_up(const TcUpArgs& a, int* status, int num_sms, cudaStream_t st);
+cudaError_t launch_tc_down(const TcDownArgs& a, int* status, int num_sms, cudaStream_t st);
+
+// combine.cu
+cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* inv_row, const void* shared, int T,
+                           int d, int k, bool bf16, void* y, int* status, cudaStream_t st);
+
+}  // namespace moe

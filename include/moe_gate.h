@@ -1,0 +1,187 @@
+/*
+ * moe_gate.h -- C ABI of the B200 (sm_100a) fine-grained MoE layer forward.
+ *
+ * The layer is the DeepSeek-V3 MoE feed-forward as the following web pages
+ * state it (cited by page title and section):
+ *   [P1] "DeepSeek V3 From Scratch": "The idea" (256 routed + 1 shared
+ *        expert, top-8; bias acts on selection only, weights from the
+ *        unbiased affinity), "Worked example", "In code" (route() and
+ *        update_bias()).
+ *   [P2] "Scaling Efficiency: A Deep Dive into the DeepSeek-V3
+ *        Architecture": DeepSeekMoE module sketch (shared experts on every
+ *        token, routed experts combined with their gate weights).
+ *   [P3] kbwen.com DeepSeek tag page: "A bias term for each expert"
+ *        (per-step load over the whole batch, fixed +-0.001 bias step).
+ *   [P4] "DeepSeek V3 Architecture Deep Dive: Multi-Head Latent Attention
+ *        (MLA), DeepSeekMoE & FP8 Mixed Precision": "Throughput on NVIDIA
+ *        H100/H800" (tokens routed to the same expert batched together).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library allocates no device memory on any call.  Scratch space is
+ *     passed in as `workspace` (size from the matching *_workspace_size).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Arguments are validated on the host before
+ *     anything is enqueued; on an error nothing is launched.
+ *   - Layouts are row-major and contiguous.  Weights use nn.Linear's
+ *     [out][in] layout: W_gate [E][d]; W1, W3 [E][I][d]; W2 [E][d][I];
+ *     shared Ws1, Ws3 [S][Is][d]; Ws2 [S][d][Is].  x and y are [T][d].
+ *   - dtype MOE_F32: x, weights, y, intermediates fp32.  MOE_BF16: x,
+ *     weights, y, intermediates bf16; every contraction accumulates in
+ *     fp32; affinities, router weights and the bias are always fp32.
+ *   - Every tensor pointer must be 16-byte aligned (MOE_ERR_ALIGNMENT).
+ *   - Anomalies found on the device (an expert index out of range, counts
+ *     that disagree with the routing table, a pipeline wait that timed
+ *     out) are recorded in a per-device status word and returned by
+ *     moe_get_last_error().  Kernels never trap.
+ *   - Not thread-safe across host threads for the same device status word
+ *     (moe_get_last_error reads and clears it).
+ */
+#ifndef MOE_GATE_H
+#define MOE_GATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* bad size, null required pointer, k > E ... */
+    MOE_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels cover  */
+    MOE_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned          */
+    MOE_ERR_WORKSPACE = 4,     /* workspace missing or smaller than needed  */
+    MOE_ERR_CUDA = 5,          /* a CUDA runtime call failed                */
+    MOE_ERR_DEVICE_CHECK = 6,  /* a device-side consistency check failed    */
+    MOE_ERR_TIMEOUT = 7        /* a device-side wait gave up (bounded spin) */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Problem sizes.  T tokens of width d; E routed experts, k chosen per
+ * token; routed SwiGLU intermediate I; S shared experts of intermediate Is
+ * (S may be 0). */
+typedef struct {
+    int32_t T, d, E, k, I, S, Is;
+    int32_t dtype; /* moe_dtype */
+} moe_shape;
+
+/* Limits (validated): 1 <= k <= min(E, 16); E <= 256; d % 8 == 0.
+ * MOE_BF16 additionally needs d % 64 == 0, I % 128 == 0 and Is % 128 == 0
+ * (tensor-core tiles), else MOE_ERR_UNSUPPORTED. */
+
+/* ---------------------------------------------------------------------------
+ * moe_route -- gate affinities, bias-shifted top-k, unbiased weights and the
+ * load histogram  [P1 "In code", route(); P1 "The idea"; P3 "A bias term for
+ * each expert"].
+ *   s[t][i]   = sigmoid( x[t] . W_gate[i] )            fp32 (fp32 accumulate)
+ *   v[t][i]   = s[t][i] + bias[i]                        fp32
+ *   topk_idx[t][0..k)  the k largest v, descending; equal v -> lower index
+ *   topk_w[t][j]       = s[t][idx_j] / sum_{j'} s[t][idx_j'] (sum in slot
+ *                        order, fp32, IEEE division)
+ *   counts[i] = #{(t, j) : topk_idx[t][j] == i}   (overwritten, not added)
+ * x [T][d] dtype; W_gate [E][d] dtype; bias [E] fp32 (read only);
+ * topk_idx [T][k] int32; topk_w [T][k] fp32; counts [E] int32;
+ * affinity_out: NULL, or [T][E] fp32 receiving s.
+ * -------------------------------------------------------------------------*/
+MOE_API moe_status moe_route(const void* x, const void* w_gate, const float* bias, moe_shape sh,
+                     int32_t* topk_idx, float* topk_w, int32_t* counts, float* affinity_out,
+                     void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_load_and_bias_update -- auxiliary-loss-free balancing step, applied
+ * once at the end of a training step  [P1 "In code", update_bias();
+ * P3 "A bias term for each expert"].
+ *   load[i] = counts[i] / T                      fp32, T = sh.T, the tokens
+ *                                                the counts were taken over
+ *   bias[i] = bias[i] + step * sign(target[i] - load[i])  (sign(0) = 0)
+ * target: NULL means the uniform load k/E for every expert.  bias [E] fp32
+ * is updated in place; load_out: NULL or [E] fp32.  step 0 leaves the bias
+ * unchanged (the pages' final 0.0 phase).
+ * -------------------------------------------------------------------------*/
+MOE_API moe_status moe_load_and_bias_update(const int32_t* counts, moe_shape sh, float step, const float* target,
+                                    float* bias, float* load_out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_permute -- expert-contiguous token order  [P4 "Throughput on NVIDIA
+ * H100/H800": tokens routed to the same expert are batched together].
+ * Rows are ordered by (expert ascending, token ascending):
+ *   offsets[e]       first row of expert e; offsets[E] = T*k   int32 [E+1]
+ *   perm_tok[row]    = t*k + j, the assignment held by that row int32 [T*k]
+ *   inv_row[t*k + j] = row                                     int32 [T*k]
+ *   x_perm[row]      = x[t]                                    [T*k][d] dtype
+ * counts: the histogram from moe_route; it is cross-checked on the device
+ * (MOE_ERR_DEVICE_CHECK via moe_get_last_error on a mismatch).
+ * Out-of-range expert indices are reported the same way and skipped.
+ * workspace: >= moe_permute_workspace_size(sh) bytes, 256-byte aligned.
+ * -------------------------------------------------------------------------*/
+MOE_API moe_status moe_permute(const void* x, const int32_t* topk_idx, const int32_t* counts, moe_shape sh, void* x_perm,
+                       int32_t* offsets, int32_t* perm_tok, int32_t* inv_row, void* workspace, size_t ws_bytes,
+                       void* stream);
+MOE_API size_t moe_permute_workspace_size(moe_shape sh);
+
+/* ---------------------------------------------------------------------------
+ * moe_grouped_swiglu -- the routed experts as one grouped SwiGLU GEMM pair,
+ * and optionally the always-on shared experts  [P2 DeepSeekMoE sketch:
+ * per-expert MLPs on the tokens routed to them; shared experts on every
+ * token; the MLP is SwiGLU without biases].
+ *   for expert e, rows r in [offsets[e], offsets[e+1]):
+ *     h        = silu(x_perm[r] . W1[e]^T) * (x_perm[r] . W3[e]^T)
+ *                (stored once in dtype)
+ *     y_perm[r] = h . W2[e]^T                          [T*k][d] dtype
+ *   if x != NULL and S > 0, for every token t:
+ *     shared_out[t] = sum_s SwiGLU_s(x[t])             [T][d] dtype
+ * workspace: >= moe_grouped_swiglu_workspace_size(sh) bytes.
+ * -------------------------------------------------------------------------*/
+MOE_API moe_status moe_grouped_swiglu(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3,
+                              const void* w2, const void* x, const void* ws1, const void* ws3, const void* ws2,
+                              moe_shape sh, void* y_perm, void* shared_out, void* workspace, size_t ws_bytes,
+                              void* stream);
+MOE_API size_t moe_grouped_swiglu_workspace_size(moe_shape sh);
+
+/* ---------------------------------------------------------------------------
+ * moe_combine -- weighted combine back into token order  [P2 DeepSeekMoE
+ * sketch: routed_out[mask] += w * expert(x[mask]); shared_out + routed_out].
+ *   y[t] = shared_out[t] + sum_{j=0..k-1} topk_w[t][j] * y_perm[inv_row[t*k+j]]
+ * accumulated in fp32 in that order, rounded once to dtype.
+ * shared_out may be NULL (no shared term).
+ * -------------------------------------------------------------------------*/
+MOE_API moe_status moe_combine(const void* y_perm, const float* topk_w, const int32_t* inv_row, const void* shared_out,
+                       moe_shape sh, void* y, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_layer_forward -- the whole layer: route, permute, grouped SwiGLU for
+ * routed and shared experts, combine.  Same semantics as the five calls in
+ * sequence.  The bias is read, not updated (call moe_load_and_bias_update
+ * with the returned counts at the end of a training step).
+ * Outputs: y [T][d] dtype; topk_idx [T][k]; topk_w [T][k]; counts [E].
+ * workspace: >= moe_workspace_size(sh) bytes.  No host synchronisation.
+ * -------------------------------------------------------------------------*/
+MOE_API moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bias, const void* w1, const void* w3,
+                             const void* w2, const void* ws1, const void* ws3, const void* ws2, moe_shape sh, void* y,
+                             int32_t* topk_idx, float* topk_w, int32_t* counts, void* workspace, size_t ws_bytes,
+                             void* stream);
+MOE_API size_t moe_workspace_size(moe_shape sh);
+
+/* Synchronises `stream`, then returns and clears the current device's
+ * status word (MOE_OK if no kernel reported an anomaly). */
+MOE_API moe_status moe_get_last_error(void* stream);
+
+/* Static description of a status code. */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* ABI version of this header (major * 100 + minor). */
+MOE_API int moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_GATE_H */

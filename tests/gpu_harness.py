@@ -1,0 +1,157 @@
+"""Helpers shared by the GPU parity tests: run the C-ABI stages on device
+tensors and compute the oracle's answer from the very same tensors."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import fine_grained_moe_gate_b200 as moe
+import oracle
+from fine_grained_moe_gate_b200.inputs import MoEConfig, make_layer, make_tokens, to_numpy
+
+DEV = "cuda"
+
+
+def rel_fro(a, b) -> float:
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
+
+
+def as_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def check_status():
+    st = moe.moe_get_last_error()
+    assert st == 0, f"device status {moe.STATUS.get(st, st)}"
+
+
+def route(sh, x, wg, bias, with_aff=True):
+    T, E, k = sh.T, sh.E, sh.k
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    aff = torch.empty((T, E), dtype=torch.float32, device=DEV) if with_aff else None
+    moe.moe_route(x, wg, bias, sh, idx, w, counts, aff)
+    torch.cuda.synchronize()
+    return idx, w, counts, aff
+
+
+def affinity_tolerance(s_orc: np.ndarray, K: int, tensor_cores: bool) -> np.ndarray:
+    """Per-element bound on |s_kernel - s_oracle| from the arithmetic.
+
+    The kernel accumulates z = x . W_g in fp32; the oracle in double (exact
+    enough to count as exact).  Worst-case (n * u) rounding bound on z:
+      SIMT path:        K fused multiply-adds, each rounded to nearest:
+                        |dz| <= K * 2^-24 * (|z| + 1)
+      tensor-core path: K/16 additions of a block of 16 products into the
+                        fp32 accumulator, each may lose up to one ulp:
+                        |dz| <= (K / 16) * 2^-23 * (|z| + 1)
+    (|z| + 1 bounds the partial sums for these inputs).  The sigmoid scales
+    dz by s (1 - s); rounding s to fp32 adds 2^-24."""
+    s = s_orc.astype(np.float64)
+    z = np.log(s / (1.0 - s))
+    dsig = s * (1.0 - s)
+    if tensor_cores:
+        dz = (K / 16.0) * 2.0 ** -23 * (np.abs(z) + 1.0)
+    else:
+        dz = K * 2.0 ** -24 * (np.abs(z) + 1.0)
+    return dsig * dz + 2.0 ** -24
+
+
+def check_route_parity(x, wg, bias, k, idx, w, counts, aff, s_tol, self_rows=None):
+    """Injected mode: the oracle's selection on the kernel's fp32 affinities
+    must match idx, w and counts bit for bit.  Self mode: the oracle's own
+    affinities on ``self_rows`` within s_tol ("auto": the bound
+    ``affinity_tolerance`` derives for the input dtype)."""
+    aff_np = aff.cpu().numpy()
+    b_np = bias.cpu().numpy()
+    o_idx, o_w = oracle.select(aff_np, b_np, k)
+    g_idx, g_w = idx.cpu().numpy(), w.cpu().numpy()
+    assert (g_idx == o_idx).all(), f"idx mismatch at {np.argwhere(g_idx != o_idx)[:5]}"
+    assert (g_w.view(np.uint32) == o_w.view(np.uint32)).all(), "weights not bit-exact"
+    E = aff_np.shape[1]
+    assert (counts.cpu().numpy() == oracle.histogram(o_idx, E)).all()
+    rows = np.arange(aff_np.shape[0]) if self_rows is None else np.asarray(self_rows)
+    s_orc = oracle.affinity(to_numpy(x[torch.as_tensor(rows, device=x.device)]), to_numpy(wg))
+    diff = np.abs(s_orc.astype(np.float64) - aff_np[rows].astype(np.float64))
+    if s_tol == "auto":
+        tol = affinity_tolerance(s_orc, x.shape[1], x.dtype == torch.bfloat16)
+    else:
+        tol = np.full(diff.shape, float(s_tol))
+    worst = np.unravel_index(np.argmax(diff / tol), diff.shape)
+    assert (diff <= tol).all(), f"affinity error {diff[worst]} > bound {tol[worst]} at {worst}"
+    return o_idx, o_w
+
+
+def permute(sh, x, idx, counts):
+    T, k, d, E = sh.T, sh.k, sh.d, sh.E
+    x_perm = torch.empty((T * k, d), dtype=x.dtype, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    ws = torch.empty(max(moe.moe_permute_workspace_size(sh), 256), dtype=torch.uint8, device=DEV)
+    moe.moe_permute(x, idx, counts, sh, x_perm, offsets, perm, inv, ws)
+    torch.cuda.synchronize()
+    return x_perm, offsets, perm, inv
+
+
+def grouped_swiglu(sh, x_perm, offsets, p, x=None):
+    T, k, d = sh.T, sh.k, sh.d
+    y_perm = torch.empty((T * k, d), dtype=x_perm.dtype, device=DEV)
+    shared_out = torch.empty((T, d), dtype=x_perm.dtype, device=DEV) if x is not None else None
+    ws = torch.empty(max(moe.moe_grouped_swiglu_workspace_size(sh), 256), dtype=torch.uint8, device=DEV)
+    moe.moe_grouped_swiglu(x_perm, offsets, p["w1"], p["w3"], p["w2"], x, p["ws1"], p["ws3"], p["ws2"], sh, y_perm,
+                           shared_out, ws)
+    torch.cuda.synchronize()
+    return y_perm, shared_out
+
+
+def layer_forward(sh, p, x, ws=None, stream=None):
+    T, k, d, E = sh.T, sh.k, sh.d, sh.E
+    y = torch.empty((T, d), dtype=x.dtype, device=DEV)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    if ws is None:
+        ws = torch.empty(moe.moe_workspace_size(sh), dtype=torch.uint8, device=DEV)
+    moe.moe_layer_forward(x, p["w_gate"], p["bias"], p["w1"], p["w3"], p["w2"], p["ws1"], p["ws3"], p["ws2"], sh, y,
+                          idx, w, counts, ws, stream)
+    torch.cuda.synchronize()
+    return y, idx, w, counts
+
+
+def oracle_rows(p, x, idx, w, tokens, S):
+    """The oracle's layer output for the given token rows, built expert by
+    expert from the routing (idx, w) -- the weights of one expert at a time
+    come back from the device."""
+    tokens = np.asarray(tokens)
+    n = len(tokens)
+    d = x.shape[1]
+    xs = to_numpy(x[torch.as_tensor(tokens, device=x.device)])
+    yacc = np.zeros((n, d), np.float64)
+    for s in range(S):
+        oracle.expert_accumulate(xs, np.arange(n, dtype=np.int32), np.ones(n), to_numpy(p["ws1"][s]),
+                                 to_numpy(p["ws3"][s]), to_numpy(p["ws2"][s]), yacc)
+    idx_np = idx.cpu().numpy()[tokens]
+    w_np = w.cpu().numpy()[tokens]
+    for e in np.unique(idx_np):
+        ii, jj = np.nonzero(idx_np == e)
+        oracle.expert_accumulate(xs[ii], ii.astype(np.int32), w_np[ii, jj].astype(np.float64), to_numpy(p["w1"][e]),
+                                 to_numpy(p["w3"][e]), to_numpy(p["w2"][e]), yacc)
+    return oracle.finalize(yacc, xs.dtype)
+
+
+def to_f64_rows(arr_np) -> np.ndarray:
+    """numpy oracle output (float32 or bf16 bits) -> float64."""
+    if arr_np.dtype == np.uint16:
+        return (arr_np.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return arr_np.astype(np.float64)
+
+
+def setup(cfg: MoEConfig, step: int = 0):
+    p = make_layer(cfg, DEV)
+    x = make_tokens(cfg, DEV, step)
+    return moe.shape_of(cfg), p, x

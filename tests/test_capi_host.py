@@ -1,0 +1,132 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, it
+exports every entry point include/moe_gate.h declares, and argument
+validation rejects bad calls before anything reaches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fine_grained_moe_gate_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_gate.h")
+
+INVALID, UNSUPPORTED, ALIGN, WORKSPACE = 1, 2, 3, 4
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(moe.LIB_PATH):
+        from fine_grained_moe_gate_b200 import build
+        build.build()
+    return moe.lib()
+
+
+def test_header_declares_the_abi():
+    names = declared_entry_points()
+    for required in ("moe_route", "moe_load_and_bias_update", "moe_permute", "moe_grouped_swiglu", "moe_combine",
+                     "moe_layer_forward", "moe_workspace_size", "moe_get_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_entry_points():
+        assert hasattr(L, name), name
+    assert set(moe.EXPORTS) == set(declared_entry_points())
+
+
+def test_abi_version_and_strings(L):
+    assert moe.moe_abi_version() == 100
+    assert moe.moe_status_string(0) == "ok"
+    assert "workspace" in moe.moe_status_string(WORKSPACE)
+
+
+def shape(**kw):
+    base = dict(T=128, d=256, E=16, k=4, I=64, S=1, Is=64, dtype=moe.MOE_F32)
+    base.update(kw)
+    return moe.MoEShape(*[base[n] for n, _ in moe.MoEShape._fields_])
+
+
+def test_workspace_sizes(L):
+    sh = shape()
+    ws = moe.moe_workspace_size(sh)
+    assert ws > 0 and ws % 256 == 0
+    assert moe.moe_permute_workspace_size(sh) == 256          # one chunk x 16 experts x int32, rounded
+    eb = 4
+    swg = ((128 * 4 * 64 * eb + 255) // 256 * 256) + ((128 * 1 * 64 * eb + 255) // 256 * 256)
+    assert moe.moe_grouped_swiglu_workspace_size(sh) == swg
+    # invalid shapes report 0
+    assert moe.moe_workspace_size(shape(k=17, E=16)) == 0
+    # bf16 needs tensor-core friendly sizes
+    assert moe.moe_workspace_size(shape(dtype=moe.MOE_BF16, d=256, I=128, Is=128)) > 0
+    assert moe.moe_workspace_size(shape(dtype=moe.MOE_BF16, d=96, I=128, Is=128)) == 0
+    assert moe.moe_workspace_size(shape(dtype=moe.MOE_BF16, d=256, I=96, Is=128)) == 0
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null "pointer" never dereferenced
+
+
+def _route(L, sh, **ptr):
+    p = dict(x=FAKE, wg=FAKE, bias=FAKE, idx=FAKE, w=FAKE, counts=FAKE, aff=None)
+    p.update(ptr)
+    c = lambda v: None if v is None else ctypes.c_void_p(v)
+    return L.moe_route(c(p["x"]), c(p["wg"]), c(p["bias"]), sh, c(p["idx"]), c(p["w"]), c(p["counts"]), c(p["aff"]),
+                       None)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(k=0), INVALID), (dict(k=17, E=32), UNSUPPORTED), (dict(k=5, E=4), INVALID), (dict(E=300), UNSUPPORTED),
+    (dict(T=-1), INVALID), (dict(d=12), UNSUPPORTED), (dict(dtype=7), INVALID), (dict(S=1, Is=0), INVALID),
+    (dict(dtype=moe.MOE_BF16, d=256, I=64), UNSUPPORTED),
+])
+def test_route_rejects_bad_shapes(L, bad, code):
+    assert _route(L, shape(**bad)) == code
+
+
+def test_route_rejects_null_and_misaligned(L):
+    assert _route(L, shape(), wg=None) == INVALID
+    assert _route(L, shape(), counts=None) == INVALID
+    assert _route(L, shape(), x=FAKE + 4) == ALIGN
+    assert _route(L, shape(), aff=FAKE + 8) == ALIGN
+
+
+def test_permute_workspace_checks(L):
+    sh = shape()
+    c = ctypes.c_void_p
+    ws_need = moe.moe_permute_workspace_size(sh)
+    r = L.moe_permute(c(FAKE), c(FAKE), c(FAKE), sh, c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), ws_need - 1, None)
+    assert r == WORKSPACE
+    r = L.moe_permute(c(FAKE), c(FAKE), c(FAKE), sh, c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE + 16), ws_need, None)
+    assert r == ALIGN
+
+
+def test_layer_forward_checks(L):
+    sh = shape()
+    c = ctypes.c_void_p
+    need = moe.moe_workspace_size(sh)
+    args = [c(FAKE)] * 9
+    r = L.moe_layer_forward(*args, sh, c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), need - 256, None)
+    assert r == WORKSPACE
+    args_noshared = [c(FAKE)] * 6 + [None, None, None]
+    r = L.moe_layer_forward(*args_noshared, sh, c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), need, None)
+    assert r == INVALID  # S = 1 needs the shared weights
+
+
+def test_bias_update_checks(L):
+    c = ctypes.c_void_p
+    assert L.moe_load_and_bias_update(c(FAKE), shape(T=0), ctypes.c_float(1e-3), None, c(FAKE), None, None) == INVALID
+    assert L.moe_load_and_bias_update(None, shape(), ctypes.c_float(1e-3), None, c(FAKE), None, None) == INVALID
+    assert L.moe_load_and_bias_update(c(FAKE), shape(), ctypes.c_float(float("nan")), None, c(FAKE), None,
+                                      None) == INVALID
+
+
+def test_binding_raises_on_error(L):
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_route(FAKE, None, FAKE, shape(), FAKE, FAKE, FAKE, stream=0)
+    assert ei.value.status == INVALID
