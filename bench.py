@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the fine-grained MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch held in HBM:
+gate GEMM + sigmoid + bias-shifted top-k + weights + load histogram
+(moe_route), expert-contiguous permutation (moe_permute), the routed and
+shared grouped SwiGLU GEMMs (moe_expert_up / moe_expert_down), the weighted
+combine (moe_combine) and the bias update at the end of the step
+(moe_load_and_bias_update; with N > 1 the counts are first summed over the
+ranks with an NCCL all-reduce -- the one exchange the method has).  Each rank
+processes its own T tokens (weak scaling, token-sharded data parallel with
+replicated weights).
+
+Timing: W warm-up steps, then K steps bracketed by a barrier and a device
+synchronize, measured with CUDA events on the launching stream; the slowest
+rank's time is reported.  CUDA events between the stages give each kernel's
+duration inside the timed region (roofline of the dominant kernel).  The
+layer weights (22.6 GB for the DeepSeek-V3 shape) are far larger than the
+126 MB L2, so no flush is needed between steps.
+
+The e2e leg runs the same steps through moe_layer_forward with the tokens
+copied from pinned host memory each step and the output copied back.
+
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd tokens/s (V3-shaped, bf16) and % of BF16 tensor / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+STAGES = ["route", "permute", "up_routed", "up_shared", "down_routed", "down_shared", "combine", "bias_update"]
+DOMINANT = "up_routed"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="v3_prefill",
+                    choices=["v3_prefill", "v3_decode", "small_bf16", "skew_stress", "tiny_fp32"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0: per-workload default)")
+    ap.add_argument("--T", type=int, default=0, help="override tokens per GPU (profiling slices)")
+    ap.add_argument("--E", type=int, default=0, help="override routed experts (profiling slices)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while the
+    timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        sm, smax = [], []
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ oracle leg
+
+DEFAULT_CPU_TOKENS = {"v3_prefill": 12, "v3_decode": 12, "skew_stress": 12, "small_bf16": 48, "tiny_fp32": 128}
+
+
+def oracle_sample(cfg, p, x, n_tok):
+    """Times the CPU oracle on the first n_tok tokens of x: routing
+    (affinities + top-k + weights), then every routed expert those tokens
+    use and the shared experts.  Expert weights are copied to the host
+    before the clock starts; only oracle arithmetic is timed.
+    Returns (seconds, tokens, threads)."""
+    import numpy as np
+    import oracle
+    from fine_grained_moe_gate_b200.inputs import to_numpy
+
+    oracle.build()
+    xs = to_numpy(x[:n_tok])
+    wg = to_numpy(p["w_gate"])
+    bias = p["bias"].detach().cpu().numpy()
+    t0 = time.perf_counter()
+    s = oracle.affinity(xs, wg)
+    idx, w = oracle.select(s, bias, cfg.k)
+    secs = time.perf_counter() - t0
+    yacc = np.zeros((n_tok, cfg.d), np.float64)
+    for sidx in range(cfg.S):
+        a, b, c = to_numpy(p["ws1"][sidx]), to_numpy(p["ws3"][sidx]), to_numpy(p["ws2"][sidx])
+        t0 = time.perf_counter()
+        oracle.expert_accumulate(xs, np.arange(n_tok, dtype=np.int32), np.ones(n_tok), a, b, c, yacc)
+        secs += time.perf_counter() - t0
+    for e in np.unique(idx):
+        ii, jj = np.nonzero(idx == e)
+        a, b, c = to_numpy(p["w1"][e]), to_numpy(p["w3"][e]), to_numpy(p["w2"][e])
+        t0 = time.perf_counter()
+        oracle.expert_accumulate(xs[ii], ii.astype(np.int32), w[ii, jj].astype(np.float64), a, b, c, yacc)
+        secs += time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.finalize(yacc, xs.dtype)
+    secs += time.perf_counter() - t0
+    threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or len(os.sched_getaffinity(0))
+    return secs, n_tok, threads
+
+
+def cpu_baseline_record(cfg, secs, n_tok, threads, label):
+    return {"value": n_tok / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": (f"{label}: {n_tok} of {cfg.T} tokens of the {cfg.name} batch through the whole layer "
+                       f"(routing over all {cfg.E} experts, every routed expert those tokens use, "
+                       f"{cfg.S} shared); {secs:.2f} s of oracle arithmetic, scaled to tokens/s; "
+                       f"OpenMP over tokens/rows, up to {threads} threads")}
+
+
+# ------------------------------------------------------------ our leg
+
+def traffic_record(kernel_file: str):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
+    summary, if the kernel source is unchanged since it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(kernel_file, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+        ent = rec.get(DOMINANT)
+        if ent and ent.get("source_sha256_16") == digest:
+            return ent.get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+def workload(args):
+    from fine_grained_moe_gate_b200.inputs import CONFIGS
+    cfg = CONFIGS[args.workload]
+    over = {}
+    if args.T:
+        over["T"] = args.T
+    if args.E:
+        over["E"] = args.E
+    if over:
+        tag = ",".join(f"{k}={v}" for k, v in over.items())
+        cfg = cfg.scaled(name=f"{cfg.name}[{tag}]", **over)
+    return cfg
+
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import fine_grained_moe_gate_b200 as moe
+    from fine_grained_moe_gate_b200.inputs import make_layer, make_tokens
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    cfg = workload(args)
+    sh = moe.shape_of(cfg)
+    sh_global = moe.shape_of(cfg, T=cfg.T * world)   # the step's batch for the bias update
+    stream = torch.cuda.current_stream()
+
+    p = make_layer(cfg, dev)
+    n_x = max(1, min(4, args.steps + args.warmup))
+    xs = [make_tokens(cfg, dev, step=i * world + rank) for i in range(n_x)]
+
+    T, k, d, E = cfg.T, cfg.k, cfg.d, cfg.E
+    dt = cfg.torch_dtype
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+    pws = torch.empty(max(moe.moe_permute_workspace_size(sh), 256), dtype=torch.uint8, device=dev)
+    x_perm = torch.empty((T * k, d), dtype=dt, device=dev)   # also holds y_perm after the up projection
+    h = torch.empty((T * k, cfg.I), dtype=dt, device=dev)
+    hs = torch.empty((T, max(1, cfg.S * cfg.Is)), dtype=dt, device=dev)
+    shared_out = torch.empty((T, d), dtype=dt, device=dev) if cfg.S > 0 else None
+    y = torch.empty((T, d), dtype=dt, device=dev)
+
+    def step(i, ev=None):
+        x = xs[i % n_x]
+        rec = (lambda j: ev[j].record(stream)) if ev is not None else (lambda j: None)
+        rec(0)
+        moe.moe_route(x, p["w_gate"], p["bias"], sh, idx, w, counts, None, stream)
+        rec(1)
+        moe.moe_permute(x, idx, counts, sh, x_perm, offsets, perm, inv, pws, stream)
+        rec(2)
+        moe.moe_expert_up(x_perm, offsets, p["w1"], p["w3"], sh, moe.MOE_ROUTED, h, stream)
+        rec(3)
+        if cfg.S > 0:
+            moe.moe_expert_up(x, None, p["ws1"], p["ws3"], sh, moe.MOE_SHARED, hs, stream)
+        rec(4)
+        moe.moe_expert_down(h, offsets, p["w2"], sh, moe.MOE_ROUTED, x_perm, stream)
+        rec(5)
+        if cfg.S > 0:
+            moe.moe_expert_down(hs, None, p["ws2"], sh, moe.MOE_SHARED, shared_out, stream)
+        rec(6)
+        moe.moe_combine(x_perm, w, inv, shared_out, sh, y, stream)
+        rec(7)
+        if world > 1:
+            dist.all_reduce(counts)
+        moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
+        rec(8)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        step(i)
+    st = moe.moe_get_last_error(stream)
+    if st != 0:
+        raise moe.MoEError(st, "warm-up steps")
+
+    gpu_id = str(local)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        gpu_id = vis.split(",")[local].strip()
+    clocks = ClockSampler(gpu_id)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    clocks.start()
+    launches0 = moe.moe_kernel_launch_count()
+    start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+    end.record(stream)
+    launches = moe.moe_kernel_launch_count() - launches0
+    barrier()
+    clk = clocks.stop()
+    st = moe.moe_get_last_error(stream)
+    if st != 0:
+        raise moe.MoEError(st, "timed steps")
+    ms_local = start.elapsed_time(end)
+    stage_ms = {}
+    for j, name in enumerate(STAGES):
+        stage_ms[name] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+    t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_per_step = ms_total / args.steps
+    tokens_per_s = world * T * args.steps / (ms_total / 1e3)
+
+    # ---- e2e: public call, host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        ws = torch.empty(moe.moe_workspace_size(sh), dtype=torch.uint8, device=dev)
+        x_dev = torch.empty((T, d), dtype=dt, device=dev)
+        x_host = [xx.cpu().pin_memory() for xx in xs]
+        y_host = torch.empty((T, d), dtype=dt).pin_memory()
+
+        def e2e_step(i):
+            x_dev.copy_(x_host[i % n_x], non_blocking=True)
+            moe.moe_layer_forward(x_dev, p["w_gate"], p["bias"], p["w1"], p["w3"], p["w2"], p["ws1"], p["ws3"],
+                                  p["ws2"], sh, y, idx, w, counts, ws, stream)
+            if world > 1:
+                dist.all_reduce(counts)
+            moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
+            y_host.copy_(y, non_blocking=True)
+
+        for i in range(args.warmup):
+            e2e_step(i)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(args.steps):
+            e2e_step(i)
+        b.record(stream)
+        barrier()
+        te = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * T * args.steps / (float(te.item()) / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": x_dev.numel() * x_dev.element_size(),
+               "d2h_bytes_per_step": y_host.numel() * y_host.element_size(),
+               "ms_per_step": float(te.item()) / args.steps}
+        st = moe.moe_get_last_error(stream)
+        if st != 0:
+            raise moe.MoEError(st, "e2e steps")
+
+    # ---- roofline of the dominant kernel (routed gate/up grouped GEMM)
+    peaks, peak_src = load_peaks()
+    flops_per_launch = T * k * 4 * d * cfg.I   # gate + up, real rows only
+    dom_ms = stage_ms[DOMINANT]
+    achieved = flops_per_launch / (dom_ms / 1e3) / 1e12
+    if cfg.dtype == "bf16":
+        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        roof = {"bound": "tensor", "kernel": "tc_grouped_gemm_kernel<up> (routed experts, SwiGLU epilogue)",
+                "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": traffic_record(os.path.join(ROOT, "fine_grained_moe_gate_b200", "csrc", "gemm_tc.cu")),
+                "peak_kind": f"bf16_tflops_sustained ({peak_src}): the kernel is timed inside a long step",
+                "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
+    else:
+        roof = {"bound": "alu", "kernel": "simt_grouped_gemm_kernel (fp32 FFMA)", "achieved": round(achieved, 3),
+                "peak": None, "unit": "TFLOP/s", "frac": None, "traffic": None,
+                "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
+    layer_flops = cfg.flops()
+    step_tflops = layer_flops / (ms_per_step / 1e3) / 1e12
+
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        n_tok = args.cpu_tokens or DEFAULT_CPU_TOKENS[args.workload]
+        secs, n, threads = oracle_sample(cfg, p, xs[0], min(n_tok, T))
+        cpu = cpu_baseline_record(cfg, secs, n, threads, "oracle sample")
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+            "data": "synthetic (seeded N(0,1) tokens, N(0,std) weights of the stated shape)",
+            "config": {"workload": cfg.name, "T_per_gpu": T, "global_batch": T * world, "d": d, "E": E, "k": k,
+                       "I": cfg.I, "S": cfg.S, "Is": cfg.Is, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2: layer weights read every step "
+                             f"({(p['w1'].numel() * 3 + p['ws1'].numel() * 3) * p['w1'].element_size() / 1e9:.1f} GB)",
+                       "bias_update": "every step"},
+            "roofline": roof,
+            "layer_tflops": round(step_tflops, 2),
+            "layer_frac_of_peak": round(step_tflops / float(peaks.get("bf16_tflops_sustained", 1400.0)), 4)
+            if cfg.dtype == "bf16" else None,
+            "stages_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "impl": "ours",
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args, world, rank, local):
+    """The oracle as the reference arm: rank 0 times it on the host cores on
+    a bounded token sample per step; other ranks exit without work."""
+    if rank != 0:
+        return
+    import torch
+    from fine_grained_moe_gate_b200.inputs import make_layer, make_tokens
+
+    cfg = workload(args)
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    if dev.type == "cuda":
+        torch.cuda.set_device(local)
+    p = make_layer(cfg, dev)
+    x = make_tokens(cfg, dev, 0)
+    n_tok = args.cpu_tokens or max(2, DEFAULT_CPU_TOKENS[args.workload] // 3)
+    n_tok = min(n_tok, cfg.T)
+    for _ in range(args.warmup):
+        oracle_sample(cfg, p, x, n_tok)
+    total, threads = 0.0, 1
+    for _ in range(args.steps):
+        secs, n, threads = oracle_sample(cfg, p, x, n_tok)
+        total += secs
+    value = n_tok * args.steps / total
+    rec = cpu_baseline_record(cfg, total, n_tok * args.steps, threads, "reference arm (oracle)")
+    rec["value"] = value
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic (seeded N(0,1) tokens, N(0,std) weights of the stated shape)",
+        "config": {"workload": cfg.name, "T_per_gpu": cfg.T, "global_batch": cfg.T * world, "d": cfg.d, "E": cfg.E,
+                   "k": cfg.k, "I": cfg.I, "S": cfg.S, "Is": cfg.Is, "parallelism": f"dp{world}",
+                   "sample_tokens_per_step": n_tok},
+        "impl": "reference",
+        "cpu_baseline": rec,
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, world, rank, local)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

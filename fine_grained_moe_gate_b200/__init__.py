@@ -30,9 +30,11 @@ STATUS = {
 
 EXPORTS = (
     "moe_route", "moe_load_and_bias_update", "moe_permute", "moe_permute_workspace_size", "moe_grouped_swiglu",
-    "moe_grouped_swiglu_workspace_size", "moe_combine", "moe_layer_forward", "moe_workspace_size",
-    "moe_get_last_error", "moe_status_string", "moe_abi_version",
+    "moe_grouped_swiglu_workspace_size", "moe_expert_up", "moe_expert_down", "moe_combine", "moe_layer_forward",
+    "moe_workspace_size", "moe_get_last_error", "moe_kernel_launch_count", "moe_status_string", "moe_abi_version",
 )
+
+MOE_ROUTED, MOE_SHARED = 0, 1
 
 
 class MoEError(RuntimeError):
@@ -72,6 +74,8 @@ def lib() -> ctypes.CDLL:
             "moe_load_and_bias_update": [P, S, F, P, P, P, P],
             "moe_permute": [P, P, P, S, P, P, P, P, P, sz, P],
             "moe_grouped_swiglu": [P, P, P, P, P, P, P, P, P, S, P, P, P, sz, P],
+            "moe_expert_up": [P, P, P, P, S, ctypes.c_int32, P, P],
+            "moe_expert_down": [P, P, P, S, ctypes.c_int32, P, P],
             "moe_combine": [P, P, P, P, S, P, P],
             "moe_layer_forward": [P, P, P, P, P, P, P, P, P, S, P, P, P, P, P, sz, P],
             "moe_get_last_error": [P],
@@ -84,6 +88,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.argtypes = [S]
             fn.restype = sz
+        L.moe_kernel_launch_count.argtypes = []
+        L.moe_kernel_launch_count.restype = ctypes.c_uint64
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_abi_version.argtypes = []
@@ -143,6 +149,16 @@ def moe_grouped_swiglu(x_perm, offsets, w1, w3, w2, x, ws1, ws3, ws2, shape, y_p
                                     _stream(stream)), "moe_grouped_swiglu")
 
 
+def moe_expert_up(a, offsets, w1, w3, shape, expert_set, h, stream=None):
+    _check(lib().moe_expert_up(_p(a), _p(offsets), _p(w1), _p(w3), shape, expert_set, _p(h), _stream(stream)),
+           "moe_expert_up")
+
+
+def moe_expert_down(h, offsets, w2, shape, expert_set, y, stream=None):
+    _check(lib().moe_expert_down(_p(h), _p(offsets), _p(w2), shape, expert_set, _p(y), _stream(stream)),
+           "moe_expert_down")
+
+
 def moe_combine(y_perm, topk_w, inv_row, shared_out, shape, y, stream=None):
     _check(lib().moe_combine(_p(y_perm), _p(topk_w), _p(inv_row), _p(shared_out), shape, _p(y), _stream(stream)),
            "moe_combine")
@@ -169,6 +185,10 @@ def moe_grouped_swiglu_workspace_size(shape) -> int:
 
 def moe_get_last_error(stream=None) -> int:
     return lib().moe_get_last_error(_stream(stream))
+
+
+def moe_kernel_launch_count() -> int:
+    return lib().moe_kernel_launch_count()
 
 
 def moe_status_string(status: int) -> str:

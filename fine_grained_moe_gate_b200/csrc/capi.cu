@@ -5,6 +5,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 namespace {
@@ -13,6 +14,7 @@ namespace {
 __device__ int g_status_word;
 
 constexpr int kMaxDevices = 64;
+std::atomic<unsigned long long> g_launches{0};
 int* g_status_ptr[kMaxDevices];
 int g_num_sms[kMaxDevices];
 std::mutex g_setup_mu;
@@ -94,6 +96,45 @@ moe_status do_permute(const void* x, const int32_t* idx, const int32_t* counts, 
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+moe_status do_expert_up(const void* a, const int32_t* offsets, const void* w1, const void* w3, const moe_shape& sh,
+                        bool shared, void* h, int* status, int sms, cudaStream_t st) {
+    if (sh.T == 0) return MOE_OK;
+    const long long rows = shared ? sh.T : (long long)sh.T * sh.k;
+    const int Ig = shared ? sh.S * sh.Is : sh.I;  // S stacked [Is][d] blocks = one [S*Is][d] matrix
+    cudaError_t err;
+    if (sh.dtype == MOE_BF16) {
+        moe::TcUpArgs up{a, rows, w1, w3, shared ? (long long)Ig : (long long)sh.E * sh.I, h, sh.d, Ig,
+                         shared ? nullptr : offsets, shared ? 1 : sh.E, shared ? sh.T : 0};
+        err = moe::launch_tc_up(up, status, sms, st);
+    } else {
+        moe::GemmArgs up{a, sh.d, w1, w3, shared ? 0 : (long long)sh.I * sh.d, sh.d, sh.d, 0, h, Ig, Ig, sh.d,
+                         shared ? nullptr : offsets, shared ? 1 : sh.E, (int)rows};
+        err = moe::launch_simt_gemm(up, false, true, sms, st);
+    }
+    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status do_expert_down(const void* h, const int32_t* offsets, const void* w2, const moe_shape& sh, bool shared,
+                          void* y, int* status, int sms, cudaStream_t st) {
+    if (sh.T == 0) return MOE_OK;
+    const long long rows = shared ? sh.T : (long long)sh.T * sh.k;
+    const int kseg = shared ? sh.Is : sh.I;
+    const int K = shared ? sh.S * sh.Is : sh.I;
+    cudaError_t err;
+    if (sh.dtype == MOE_BF16) {
+        moe::TcDownArgs dn{h, rows, w2, shared ? sh.S : 1, kseg, y, sh.d, K, shared ? nullptr : offsets,
+                           shared ? 1 : sh.E, shared ? sh.T : 0};
+        err = moe::launch_tc_down(dn, status, sms, st);
+    } else {
+        // element (n, kk) of W2 block g: (kk / kseg) * d * kseg + n * kseg + kk % kseg
+        moe::GemmArgs dn{h, K, w2, nullptr, shared ? 0 : (long long)sh.d * sh.I, kseg, kseg,
+                         (long long)sh.d * kseg, y, sh.d, sh.d, K, shared ? nullptr : offsets, shared ? 1 : sh.E,
+                         (int)rows};
+        err = moe::launch_simt_gemm(dn, false, false, sms, st);
+    }
+    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3, const void* w2,
                      const void* x, const void* ws1, const void* ws3, const void* ws2, const moe_shape& sh,
                      void* y_perm, void* shared_out, void* ws, int* status, int sms, cudaStream_t st) {
@@ -102,44 +143,23 @@ moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1,
     char* h = static_cast<char*>(ws);
     char* hs = h + align256((size_t)rows * sh.I * eb);
     const bool shared = x && sh.S > 0 && shared_out;
-    const int Ks = sh.S * sh.Is;
-    if (sh.T == 0) return MOE_OK;
-    if (sh.dtype == MOE_BF16) {
-        moe::TcUpArgs up{x_perm, rows, w1, w3, (long long)sh.E * sh.I, h, sh.d, sh.I, offsets, sh.E, 0};
-        if (moe::launch_tc_up(up, status, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
-        if (shared) {
-            moe::TcUpArgs su{x, sh.T, ws1, ws3, (long long)Ks, hs, sh.d, Ks, nullptr, 1, sh.T};
-            if (moe::launch_tc_up(su, status, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
-        }
-        moe::TcDownArgs dn{h, rows, w2, 1, sh.I, y_perm, sh.d, sh.I, offsets, sh.E, 0};
-        if (moe::launch_tc_down(dn, status, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
-        if (shared) {
-            moe::TcDownArgs sd{hs, sh.T, ws2, sh.S, sh.Is, shared_out, sh.d, Ks, nullptr, 1, sh.T};
-            if (moe::launch_tc_down(sd, status, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
-        }
-        return MOE_OK;
-    }
-    // fp32: SIMT grouped GEMMs
-    moe::GemmArgs up{x_perm, sh.d, w1, w3, (long long)sh.I * sh.d, sh.d, sh.d, 0, h, sh.I, sh.I, sh.d,
-                     offsets, sh.E, (int)rows};
-    if (moe::launch_simt_gemm(up, false, true, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
-    moe::GemmArgs dn{h, sh.I, w2, nullptr, (long long)sh.d * sh.I, sh.I, sh.I, 0, y_perm, sh.d, sh.d, sh.I,
-                     offsets, sh.E, (int)rows};
-    if (moe::launch_simt_gemm(dn, false, false, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (shared) {
-        // S stacked [Is][d] blocks are one [S*Is][d] matrix for the up side
-        moe::GemmArgs su{x, sh.d, ws1, ws3, 0, sh.d, sh.d, 0, hs, Ks, Ks, sh.d, nullptr, 1, sh.T};
-        if (moe::launch_simt_gemm(su, false, true, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
-        moe::GemmArgs sd{hs, Ks, ws2, nullptr, 0, sh.Is, sh.Is, (long long)sh.d * sh.Is, shared_out, sh.d, sh.d, Ks,
-                         nullptr, 1, sh.T};
-        if (moe::launch_simt_gemm(sd, false, false, sms, st) != cudaSuccess) return MOE_ERR_CUDA;
-    }
+    moe_status v;
+    if ((v = do_expert_up(x_perm, offsets, w1, w3, sh, false, h, status, sms, st)) != MOE_OK) return v;
+    if (shared && (v = do_expert_up(x, nullptr, ws1, ws3, sh, true, hs, status, sms, st)) != MOE_OK) return v;
+    if ((v = do_expert_down(h, offsets, w2, sh, false, y_perm, status, sms, st)) != MOE_OK) return v;
+    if (shared && (v = do_expert_down(hs, nullptr, ws2, sh, true, shared_out, status, sms, st)) != MOE_OK) return v;
     return MOE_OK;
 }
 
 }  // namespace
 
+namespace moe {
+void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+}  // namespace moe
+
 extern "C" {
+
+uint64_t moe_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int moe_abi_version(void) { return 100; }
 
@@ -251,6 +271,41 @@ moe_status moe_grouped_swiglu(const void* x_perm, const int32_t* offsets, const 
     if (v != MOE_OK) return v;
     return do_swiglu(x_perm, offsets, w1, w3, w2, shared ? x : nullptr, ws1, ws3, ws2, sh, y_perm, shared_out,
                      workspace, status, sms, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_up(const void* a, const int32_t* offsets, const void* w1, const void* w3, moe_shape sh,
+                         int32_t set, void* h, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(set == MOE_ROUTED || set == MOE_SHARED, MOE_ERR_INVALID_ARG);
+    const bool shared = set == MOE_SHARED;
+    MOE_REQUIRE(!shared || sh.S > 0, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(w1 && w3 && (shared || offsets), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (a && h), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(a) && aligned16(offsets) && aligned16(w1) && aligned16(w3) && aligned16(h),
+                MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_expert_up(a, offsets, w1, w3, sh, shared, h, status, sms, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_down(const void* h, const int32_t* offsets, const void* w2, moe_shape sh, int32_t set, void* y,
+                           void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(set == MOE_ROUTED || set == MOE_SHARED, MOE_ERR_INVALID_ARG);
+    const bool shared = set == MOE_SHARED;
+    MOE_REQUIRE(!shared || sh.S > 0, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(w2 && (shared || offsets), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (h && y), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(h) && aligned16(offsets) && aligned16(w2) && aligned16(y), MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_expert_down(h, offsets, w2, sh, shared, y, status, sms, static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_combine(const void* y_perm, const float* topk_w, const int32_t* inv_row, const void* shared_out,

@@ -94,6 +94,7 @@ cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* in
         combine_kernel<float><<<T, threads, 0, st>>>(static_cast<const uint4*>(y_perm), w, inv_row,
                                                       static_cast<const uint4*>(shared), k, vec, T * k,
                                                       static_cast<uint4*>(y), status);
+    note_launches(1);
     return cudaGetLastError();
 }
 

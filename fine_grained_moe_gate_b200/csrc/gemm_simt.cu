@@ -134,6 +134,7 @@ cudaError_t launch_simt_gemm(const GemmArgs& p, bool bf16, bool swiglu, int num_
         if (swiglu) simt_grouped_gemm_kernel<float, true><<<grid, 256, 0, st>>>(p);
         else simt_grouped_gemm_kernel<float, false><<<grid, 256, 0, st>>>(p);
     }
+    note_launches(1);
     return cudaGetLastError();
 }
 

@@ -4,27 +4,36 @@
 // routed to it; "DeepSeek V3 Architecture Deep Dive ...", "Throughput on
 // NVIDIA H100/H800": tokens of one expert batched together).
 //
-//   up:   h[r][n]  = silu(A[r] . W1_g[n]) * (A[r] . W3_g[n])   (SwiGLU fused)
-//   down: Y[r][n]  = h[r] . W2_g[n]
+//   up:   h[t][f] = silu(W1_g[f] . a[t]) * (W3_g[f] . a[t])   (SwiGLU fused)
+//   down: y[t][o] = W2_g[o] . h[t]
+//
+// Weights are the MMA's M operand (128 output features per tile) and the
+// expert's tokens the N operand.  N only has to be a multiple of 16, so the
+// last token tile of an expert is trimmed to its real rows rounded up to 16
+// instead of padding a 128-row M tile: with ~256 rows per expert the
+// padded MMA work drops from ~25% to ~3%.
+//
+//   up tile:   128 features of W1 and the same 128 of W3 x up to 128 tokens;
+//              two MMAs per K step into TMEM columns [0,128) (gate) and
+//              [128,256) (up), so one thread holds gate and up of its feature
+//              and SwiGLU is an epilogue over the accumulator.
+//   down tile: 128 features of W2 x up to 256 tokens, one MMA per K step.
+// Both use 48 KB smem stages (4-stage TMA ring, 128-byte swizzle) and two
+// 256-column TMEM accumulators, so the epilogue of one tile overlaps the
+// main loop of the next.  Weights stay in their natural [out][in] layout.
 //
 // One persistent CTA per SM walks a device-side tile list built from the
-// expert offsets (no host read-back).  Tile = 128 rows x 256 accumulator
-// columns; for the up projection the 256 columns are 128 gate rows of W1
-// and the matching 128 rows of W3, loaded by two TMA boxes into one
-// 256-row operand so gate and up land side by side in TMEM and the SwiGLU
-// is an epilogue over one accumulator.  Weights stay in their natural
-// [out][in] layout; no packing pass.
+// expert offsets (no host read-back); per expert, token tiles are walked
+// fastest so the CTAs working on one weight tile at the same time share it
+// in L2, and the expert's token rows stay in L2 across its feature tiles.
 //
 // Warp roles (192 threads):
-//   warp 0      TMA producer (one lane): A box 64x128, B boxes into a
-//               4-stage ring of 48 KB stages, 128-byte swizzle.
-//   warp 1      TMEM owner; one lane issues tcgen05.mma (M=128, N=256,
-//               K=16, bf16 -> fp32) and commits to the ring / accumulator
-//               barriers.
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 16 columns, SwiGLU or
-//               plain bf16 conversion, stores.  Two TMEM accumulators
-//               (2 x 256 columns) let the epilogue of tile i overlap the
-//               main loop of tile i+1.
+//   warp 0      TMA producer (one lane)
+//   warp 1      TMEM owner; one lane issues tcgen05.mma (kind::f16, M=128,
+//               N = trimmed token count) and commits to the barriers
+//   warps 2..5  epilogue: tcgen05.ld (32 lanes = 32 features x 16 tokens),
+//               SwiGLU / bf16 conversion, transpose through a 1 KB per-warp
+//               shared buffer into token-major rows, 32-byte vector stores.
 // Every wait is bounded (common.cuh); on a timeout the CTA raises its abort
 // flag, drains the copies and MMAs it issued, frees TMEM and exits.
 #include "common.cuh"
@@ -34,12 +43,24 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int BF = 128;  // weight rows (output features) per tile = MMA M
+constexpr int BK = 64;   // K per stage: one 128-byte swizzle row of bf16
+constexpr int STAGES = 4;
+constexpr int W_BYTES = BF * BK * 2;  // 16 KB per weight operand
+constexpr int STAGE_BYTES = 48 * 1024;
+constexpr int SMALL_ROWS = 32;        // token box for tiles of <= 32 tokens
+constexpr uint32_t ACC_COLS = 256;    // one accumulator buffer
+constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
 constexpr int NTHREADS = 192;
+constexpr int EPI_BUF = 16 * 32 * 2;  // per-warp transpose buffer: 16 tokens x 32 features
+
+template <bool UP>
+struct Geo {
+    static constexpr int NT = UP ? 128 : 256;              // tokens per tile
+    static constexpr int A_BYTES = UP ? 2 * W_BYTES : W_BYTES;
+    static constexpr int B_BYTES = NT * BK * 2;
+    static_assert(A_BYTES + B_BYTES == STAGE_BYTES, "stage layout");
+};
 
 struct Ctl {
     uint64_t full[STAGES];
@@ -53,57 +74,56 @@ struct Ctl {
 struct Tables {
     int rowstart[kMaxGroups];
     int rows[kMaxGroups];
-    int mtiles[kMaxGroups];
+    int ttiles[kMaxGroups];  // token tiles per group
     int prefix[kMaxGroups + 1];
 };
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctl) + sizeof(Tables);
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 4 * EPI_BUF + sizeof(Ctl) + sizeof(Tables);
 
 struct Params {
     const int32_t* offsets;
     int G, M;
-    int n_tiles, k_blocks;
-    int w_rows;     // up: rows of W1/W3 per group (I)
-    int kseg, nseg; // down: W2 block geometry along K
+    int f_tiles;       // feature tiles per group
+    int k_blocks;
+    int w_rows;        // up: rows of W1/W3 per group (I)
+    int kseg, nseg;    // down: W2 block geometry along K
     void* out;
-    int ldo, n_limit;
-    int n_fastest;
-    long long a_rows;  // rows of A and of the output; every group must lie inside
+    int ldo;           // output row pitch (elements)
+    int f_limit;       // valid output features
+    long long a_rows;  // rows of the token operand and of the output
     int* status;
 };
 
-__device__ __forceinline__ void tile_coords(const Tables* tb, int G, int n_tiles, bool n_fastest, int tile, int& g,
-                                            int& mt, int& nt) {
+struct TileCoord {
+    int g, ft, tt;
+};
+
+__device__ __forceinline__ TileCoord tile_coords(const Tables* tb, int G, int tile) {
     int lo = 0, hi = G - 1;
     while (lo < hi) {  // last group whose first tile is <= tile (never an empty one)
         const int mid = (lo + hi + 1) >> 1;
         if (tb->prefix[mid] <= tile) lo = mid; else hi = mid - 1;
     }
-    g = lo;
-    const int q = tile - tb->prefix[g];
-    if (n_fastest) {
-        mt = q / n_tiles;
-        nt = q - mt * n_tiles;
-    } else {
-        const int m = tb->mtiles[g];
-        nt = q / m;
-        mt = q - nt * m;
-    }
+    const int q = tile - tb->prefix[lo];
+    const int nt = tb->ttiles[lo];
+    return {lo, q / nt, q - (q / nt) * nt};
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&b);
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+    const __nv_bfloat16 b = __float2bfloat16_rn(v);
+    return *reinterpret_cast<const uint16_t*>(&b);
 }
 
 template <bool UP>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                           const __grid_constant__ CUtensorMap tmB1, const Params p) {
+    tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
+                           const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXs,
+                           const Params p) {
+    using GE = Geo<UP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* sA = base;
-    uint8_t* sB = base + STAGES * A_BYTES;
-    Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES);
+    uint8_t* ring = base;
+    uint8_t* epi = base + STAGES * STAGE_BYTES;
+    Ctl* ctl = reinterpret_cast<Ctl*>(epi + 4 * EPI_BUF);
     Tables* tb = reinterpret_cast<Tables*>(ctl + 1);
 
     const int tid = threadIdx.x;
@@ -120,7 +140,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         tb->rowstart[g] = rows > 0 ? rs : 0;
         tb->rows[g] = rows;
-        tb->mtiles[g] = (rows + BM - 1) / BM;
+        tb->ttiles[g] = (rows + GE::NT - 1) / GE::NT;
     }
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -144,7 +164,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int carry = 0;
         for (int b = 0; b < G; b += 32) {
             const int g = b + lane;
-            const int v = g < G ? tb->mtiles[g] * p.n_tiles : 0;
+            const int v = g < G ? tb->ttiles[g] * p.f_tiles : 0;
             int incl = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -161,39 +181,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
     const int total = tb->prefix[G];
-    const bool n_fastest = p.n_fastest != 0;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (elect_one()) {
-            tma_prefetch_desc(&tmA);
-            tma_prefetch_desc(&tmB0);
-            if (UP) tma_prefetch_desc(&tmB1);
+            tma_prefetch_desc(&tmW0);
+            if (UP) tma_prefetch_desc(&tmW1);
+            tma_prefetch_desc(&tmX);
+            tma_prefetch_desc(&tmXs);
             int stage = 0;
             uint32_t phase = 0, issued = 0, iss_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                int g, mt, nt;
-                tile_coords(tb, G, p.n_tiles, n_fastest, tile, g, mt, nt);
-                const int arow = tb->rowstart[g] + mt * BM;
+                const TileCoord tc = tile_coords(tb, G, tile);
+                const int tok0 = tb->rowstart[tc.g] + tc.tt * GE::NT;
+                const int ntok = min(GE::NT, tb->rows[tc.g] - tc.tt * GE::NT);
+                const bool small = ntok <= SMALL_ROWS;
+                const uint32_t tx = GE::A_BYTES + (small ? SMALL_ROWS : GE::NT) * BK * 2;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, p.status)) {
                         ok = false;
                         break;
                     }
                     uint64_t* fb = &ctl->full[stage];
-                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                    tma_load_2d(sA + stage * A_BYTES, &tmA, fb, kb * BK, arow, kEvictNormal);
+                    uint8_t* sa = ring + stage * STAGE_BYTES;
+                    uint8_t* sb = sa + GE::A_BYTES;
+                    mbar_arrive_expect_tx(fb, tx);
                     if (UP) {
-                        const int brow = g * p.w_rows + nt * (BN / 2);
-                        tma_load_2d(sB + stage * B_BYTES, &tmB0, fb, kb * BK, brow, kEvictNormal);
-                        tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, &tmB1, fb, kb * BK, brow, kEvictNormal);
+                        const int wrow = tc.g * p.w_rows + tc.ft * BF;
+                        tma_load_2d(sa, &tmW0, fb, kb * BK, wrow, kEvictNormal);
+                        tma_load_2d(sa + W_BYTES, &tmW1, fb, kb * BK, wrow, kEvictNormal);
                     } else {
                         const int kk = kb * BK;
                         const int seg = kk / p.kseg;
-                        tma_load_3d(sB + stage * B_BYTES, &tmB0, fb, kk - seg * p.kseg, nt * BN, g * p.nseg + seg,
-                                    kEvictNormal);
+                        tma_load_3d(sa, &tmW0, fb, kk - seg * p.kseg, tc.ft * BF, tc.g * p.nseg + seg, kEvictNormal);
                     }
+                    tma_load_2d(sb, small ? &tmXs : &tmX, fb, kb * BK, tok0, kEvictNormal);
                     issued |= 1u << stage;
                     iss_phase = (iss_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -211,29 +234,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (elect_one()) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const TileCoord tc = tile_coords(tb, G, tile);
+                const int ntok = min(GE::NT, tb->rows[tc.g] - tc.tt * GE::NT);
+                const int n_mma = (ntok + 15) & ~15;
+                const uint32_t idesc = idesc_bf16_f32(BF, n_mma);
                 if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                const uint32_t d_tmem = tmem_base + (uint32_t)acc * ACC_COLS;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!mbar_wait(&ctl->full[stage], phase, &ctl->abort, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t ad = smem_desc_sw128(smem_u32(sA + stage * A_BYTES));
-                    const uint64_t bd = smem_desc_sw128(smem_u32(sB + stage * B_BYTES));
+                    uint8_t* sa = ring + stage * STAGE_BYTES;
+                    const uint64_t ad0 = smem_desc_sw128(smem_u32(sa));
+                    const uint64_t bd = smem_desc_sw128(smem_u32(sa + GE::A_BYTES));
+                    if (UP) {
+                        const uint64_t ad1 = smem_desc_sw128(smem_u32(sa + W_BYTES));
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per step
-                        tc_mma_bf16(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
-                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < BK / 16; ++kk) {  // +32 bytes along K per step
+                            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+                            tc_mma_bf16(d_tmem, ad0 + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, accum);
+                            tc_mma_bf16(d_tmem + GE::NT, ad1 + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+                                        accum);
+                        }
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            tc_mma_bf16(d_tmem, ad0 + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+                                        (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
                     tc_commit(&ctl->empty[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
@@ -253,58 +291,51 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int r = q * 32 + lane;
+        const int q = warp & 3;  // TMEM lane quarter: features 32q .. 32q+31 of the tile
+        uint16_t* buf = reinterpret_cast<uint16_t*>(epi + q * EPI_BUF);  // [16 tokens][32 features]
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
         int acc = 0;
         uint32_t acc_phase = 0;
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            int g, mt, nt;
-            tile_coords(tb, G, p.n_tiles, n_fastest, tile, g, mt, nt);
+            const TileCoord tc = tile_coords(tb, G, tile);
+            const int tok0 = tb->rowstart[tc.g] + tc.tt * GE::NT;
+            const int ntok = min(GE::NT, tb->rows[tc.g] - tc.tt * GE::NT);
+            const int f0 = tc.ft * BF + q * 32;  // first feature of this warp
             if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, p.status)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            const int mrow = mt * BM + r;
-            const bool valid = mrow < tb->rows[g];
-            const size_t grow = (size_t)(tb->rowstart[g] + mrow);
-            if (UP) {
-                __nv_bfloat16* dst = out + grow * p.ldo + nt * (BN / 2);
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACC_COLS;
+            // this lane's share of a 16-token x 32-feature block: token lane/2, 16 features
+            const int my_tok = lane >> 1;
+            const int my_half = (lane & 1) * 16;
+            const bool feat_ok = f0 + my_half < p.f_limit;  // f_limit is a multiple of 16
 #pragma unroll 1
-                for (int c = 0; c < BN / 2; c += 16) {
+            for (int c = 0; c < ntok; c += 16) {
+                float v[16];
+                if (UP) {
                     uint32_t gv[16], uv[16];
-                    tmem_ld16(taddr + c, gv);
-                    tmem_ld16(taddr + BN / 2 + c, uv);
+                    tmem_ld16(taddr + (uint32_t)c, gv);
+                    tmem_ld16(taddr + (uint32_t)(GE::NT + c), uv);
                     tmem_ld_wait();
-                    if (valid) {
-                        uint32_t pk[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float h0 = silu_f32(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]);
-                            const float h1 =
-                                silu_f32(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
-                            pk[i] = pack_bf16x2(h0, h1);
-                        }
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-                        d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                    }
-                }
-            } else {
-                __nv_bfloat16* dst = out + grow * p.ldo + nt * BN;
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(taddr + c, v);
+                    for (int i = 0; i < 16; ++i) v[i] = silu_f32(__uint_as_float(gv[i])) * __uint_as_float(uv[i]);
+                } else {
+                    uint32_t r[16];
+                    tmem_ld16(taddr + (uint32_t)c, r);
                     tmem_ld_wait();
-                    if (valid && nt * BN + c < p.n_limit) {
-                        uint32_t pk[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-                        d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                    }
+                    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
                 }
+                // transpose: buf[token i][feature lane]
+#pragma unroll
+                for (int i = 0; i < 16; ++i) buf[i * 32 + lane] = bf16_bits(v[i]);
+                __syncwarp();
+                if (c + my_tok < ntok && feat_ok) {
+                    const uint4* src = reinterpret_cast<const uint4*>(buf + my_tok * 32 + my_half);
+                    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * p.ldo + f0 + my_half);
+                    dst[0] = src[0];
+                    dst[1] = src[1];
+                }
+                __syncwarp();
             }
             tc_fence_before();
             mbar_arrive(&ctl->tempty[acc]);
@@ -322,66 +353,65 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 template <bool UP>
-cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const Params& p, int num_sms,
-                   cudaStream_t st) {
+cudaError_t launch(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x, const CUtensorMap& xs,
+                   const Params& p, int num_sms, cudaStream_t st) {
     auto kern = tc_grouped_gemm_kernel<UP>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    kern<<<num_sms, NTHREADS, SMEM_BYTES, st>>>(a, b0, b1, p);
+    kern<<<num_sms, NTHREADS, SMEM_BYTES, st>>>(w0, w1, x, xs, p);
+    note_launches(1);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_tc_up(const TcUpArgs& a, int* status, int num_sms, cudaStream_t st) {
-    if (a.G <= 0 || a.G > kMaxGroups || a.d % BK != 0 || a.I % (BN / 2) != 0) return cudaErrorInvalidValue;
-    CUtensorMap tA, tB0, tB1;
-    if (!make_tmap_2d(&tA, a.A, a.d, a.A_rows, a.d, BK, BM) || !make_tmap_2d(&tB0, a.W1, a.d, a.W_rows, a.d, BK, BN / 2) ||
-        !make_tmap_2d(&tB1, a.W3, a.d, a.W_rows, a.d, BK, BN / 2))
+    if (a.G <= 0 || a.G > kMaxGroups || a.d % BK != 0 || a.I % BF != 0) return cudaErrorInvalidValue;
+    CUtensorMap tW1, tW3, tX, tXs;
+    if (!make_tmap_2d(&tW1, a.W1, a.d, a.W_rows, a.d, BK, BF) || !make_tmap_2d(&tW3, a.W3, a.d, a.W_rows, a.d, BK, BF) ||
+        !make_tmap_2d(&tX, a.A, a.d, a.A_rows, a.d, BK, Geo<true>::NT) ||
+        !make_tmap_2d(&tXs, a.A, a.d, a.A_rows, a.d, BK, SMALL_ROWS))
         return cudaErrorInvalidValue;
     Params p{};
     p.offsets = a.offsets;
     p.G = a.G;
     p.M = a.M;
-    p.n_tiles = a.I / (BN / 2);
+    p.f_tiles = a.I / BF;
     p.k_blocks = a.d / BK;
     p.w_rows = a.I;
     p.kseg = a.d;
     p.nseg = 1;
     p.out = a.H;
     p.ldo = a.I;
-    p.n_limit = a.I;
-    // one large group (the shared experts): walk N fastest so a band of A
-    // rows stays in L2 while every weight tile passes over it
-    p.n_fastest = (a.offsets == nullptr && a.M > 8 * BM) ? 1 : 0;
+    p.f_limit = a.I;
     p.a_rows = a.A_rows;
     p.status = status;
-    return launch<true>(tA, tB0, tB1, p, num_sms, st);
+    return launch<true>(tW1, tW3, tX, tXs, p, num_sms, st);
 }
 
 cudaError_t launch_tc_down(const TcDownArgs& a, int* status, int num_sms, cudaStream_t st) {
-    if (a.G <= 0 || a.G > kMaxGroups || a.K % BK != 0 || a.kseg % BK != 0 || a.d % BK != 0)
+    if (a.G <= 0 || a.G > kMaxGroups || a.K % BK != 0 || a.kseg % BK != 0 || a.d % 16 != 0)
         return cudaErrorInvalidValue;
-    CUtensorMap tA, tB;
-    if (!make_tmap_2d(&tA, a.H, a.K, a.H_rows, a.K, BK, BM) ||
-        !make_tmap_3d(&tB, a.W2, a.kseg, a.d, (unsigned long long)a.G * a.nseg, BK, BN))
+    CUtensorMap tW2, tX, tXs;
+    if (!make_tmap_3d(&tW2, a.W2, a.kseg, a.d, (unsigned long long)a.G * a.nseg, BK, BF) ||
+        !make_tmap_2d(&tX, a.H, a.K, a.H_rows, a.K, BK, Geo<false>::NT) ||
+        !make_tmap_2d(&tXs, a.H, a.K, a.H_rows, a.K, BK, SMALL_ROWS))
         return cudaErrorInvalidValue;
     Params p{};
     p.offsets = a.offsets;
     p.G = a.G;
     p.M = a.M;
-    p.n_tiles = (a.d + BN - 1) / BN;
+    p.f_tiles = (a.d + BF - 1) / BF;
     p.k_blocks = a.K / BK;
     p.w_rows = 0;
     p.kseg = a.kseg;
     p.nseg = a.nseg;
     p.out = a.Y;
     p.ldo = a.d;
-    p.n_limit = a.d;
-    p.n_fastest = (a.offsets == nullptr && a.M > 8 * BM) ? 1 : 0;
+    p.f_limit = a.d;
     p.a_rows = a.H_rows;
     p.status = status;
-    return launch<false>(tA, tB, tB, p, num_sms, st);
+    return launch<false>(tW2, tW2, tX, tXs, p, num_sms, st);
 }
 
 }  // namespace moe

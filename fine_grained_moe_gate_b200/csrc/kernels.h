@@ -9,6 +9,9 @@
 namespace moe {
 
 constexpr int kMaxExperts = 256;
+
+// Adds n to the library's kernel-launch counter (moe_kernel_launch_count).
+void note_launches(int n);
 constexpr int kMaxGroups = kMaxExperts;
 
 // One grouped GEMM C = A . B^T (optionally with the SwiGLU pair B0/B1).

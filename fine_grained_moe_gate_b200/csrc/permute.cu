@@ -148,20 +148,26 @@ cudaError_t launch_permute(const void* x, const int32_t* idx, const int32_t* cou
                            size_t elem_bytes, void* x_perm, int32_t* offsets, int32_t* perm_tok, int32_t* inv_row,
                            int32_t* scratch, int* status, cudaStream_t st) {
     const int C = (T + kChunk - 1) / kChunk;
+    int launched = 0;
     if (C > 0) {
         permute_hist_kernel<<<C, 256, E * sizeof(int), st>>>(idx, T, k, E, scratch, status);
+        ++launched;
     }
     const int nthr = ((E + 31) / 32) * 32;
     permute_scan_kernel<<<1, nthr < 32 ? 32 : nthr, 0, st>>>(scratch, C, E, counts, offsets, status);
+    ++launched;
     if (C > 0) {
         permute_rank_kernel<<<C, 256, (size_t)E * kChunkWords * sizeof(uint32_t), st>>>(idx, T, k, E, scratch,
                                                                                           perm_tok, inv_row);
+        ++launched;
         if (x && x_perm) {
             const int vec = (int)((size_t)d * elem_bytes / 16);
             permute_scatter_kernel<<<T, 128, 0, st>>>(static_cast<const uint4*>(x), vec, k, inv_row, T * k,
                                                        static_cast<uint4*>(x_perm));
+            ++launched;
         }
     }
+    note_launches(launched);
     return cudaGetLastError();
 }
 

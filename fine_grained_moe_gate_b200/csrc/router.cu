@@ -116,6 +116,7 @@ static cudaError_t launch_router_simt_t(const void* x, const void* wg, const flo
     const int grid = (T + kRtTok - 1) / kRtTok;
     kern<<<grid, 256, smem, st>>>(static_cast<const Tin*>(x), static_cast<const Tin*>(wg), bias, T, d, E, k, idx,
                                   w, counts, aff, status);
+    note_launches(1);
     return cudaGetLastError();
 }
 
@@ -152,6 +153,7 @@ __global__ void bias_update_kernel(const int32_t* __restrict__ counts, int T, in
 cudaError_t launch_bias_update(const int32_t* counts, int T, int E, int k, float step, const float* target,
                                float* bias, float* load_out, cudaStream_t st) {
     bias_update_kernel<<<(E + 255) / 256, 256, 0, st>>>(counts, T, E, k, step, target, bias, load_out);
+    note_launches(1);
     return cudaGetLastError();
 }
 

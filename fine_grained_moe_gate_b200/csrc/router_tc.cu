@@ -177,6 +177,7 @@ cudaError_t launch_k(const CUtensorMap& tx, const CUtensorMap& tw, const float* 
     if (err != cudaSuccess) return err;
     const int grid = (T + BM - 1) / BM;
     kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status);
+    note_launches(1);
     return cudaGetLastError();
 }
 

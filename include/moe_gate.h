@@ -148,6 +148,28 @@ MOE_API moe_status moe_grouped_swiglu(const void* x_perm, const int32_t* offsets
 MOE_API size_t moe_grouped_swiglu_workspace_size(moe_shape sh);
 
 /* ---------------------------------------------------------------------------
+ * moe_expert_up / moe_expert_down -- the two grouped GEMMs moe_grouped_swiglu
+ * is made of, callable one at a time (to keep h, or to time each launch).
+ * `set` picks the expert set:
+ *   MOE_ROUTED: a = x_perm [T*k][d], offsets [E+1] (group e owns rows
+ *               [offsets[e], offsets[e+1])), W1/W3 [E][I][d], W2 [E][d][I],
+ *               h [T*k][I], y = y_perm [T*k][d];
+ *   MOE_SHARED: a = x [T][d] (offsets ignored, may be NULL), W1/W3 = Ws1/Ws3
+ *               [S][Is][d], W2 = Ws2 [S][d][Is], h [T][S*Is] (shared expert s
+ *               in columns [s*Is, (s+1)*Is)), y = shared_out [T][d] = the
+ *               sum over the S shared experts.
+ *   up:   h[r] = silu(a[r] . W1_g^T) * (a[r] . W3_g^T)   stored once in dtype
+ *   down: y[r] = h[r] . W2_g^T                            fp32 accumulate
+ * Same sources as moe_grouped_swiglu.  Invalid for MOE_SHARED when S == 0.
+ * -------------------------------------------------------------------------*/
+typedef enum { MOE_ROUTED = 0, MOE_SHARED = 1 } moe_expert_set;
+
+MOE_API moe_status moe_expert_up(const void* a, const int32_t* offsets, const void* w1, const void* w3, moe_shape sh,
+                                 int32_t set, void* h, void* stream);
+MOE_API moe_status moe_expert_down(const void* h, const int32_t* offsets, const void* w2, moe_shape sh, int32_t set,
+                                   void* y, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_combine -- weighted combine back into token order  [P2 DeepSeekMoE
  * sketch: routed_out[mask] += w * expert(x[mask]); shared_out + routed_out].
  *   y[t] = shared_out[t] + sum_{j=0..k-1} topk_w[t][j] * y_perm[inv_row[t*k+j]]
@@ -174,6 +196,11 @@ MOE_API size_t moe_workspace_size(moe_shape sh);
 /* Synchronises `stream`, then returns and clears the current device's
  * status word (MOE_OK if no kernel reported an anomaly). */
 MOE_API moe_status moe_get_last_error(void* stream);
+
+/* Number of CUDA kernels this library has launched in this process (all
+ * devices, all streams); a tracing aid, e.g. to count the kernels of one
+ * step.  Host-side counter, no synchronisation. */
+MOE_API uint64_t moe_kernel_launch_count(void);
 
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
