@@ -29,7 +29,8 @@ STATUS = {
 }
 
 EXPORTS = (
-    "moe_route", "moe_load_and_bias_update", "moe_permute", "moe_permute_workspace_size", "moe_grouped_swiglu",
+    "moe_route", "moe_load_and_bias_update", "moe_permute", "moe_permute_workspace_size", "moe_permute_noalloc",
+    "moe_grouped_swiglu",
     "moe_grouped_swiglu_workspace_size", "moe_expert_up", "moe_expert_down", "moe_combine", "moe_layer_forward",
     "moe_workspace_size", "moe_get_last_error", "moe_kernel_launch_count", "moe_status_string", "moe_abi_version",
 )
@@ -73,6 +74,7 @@ def lib() -> ctypes.CDLL:
             "moe_route": [P, P, P, S, P, P, P, P, P],
             "moe_load_and_bias_update": [P, S, F, P, P, P, P],
             "moe_permute": [P, P, P, S, P, P, P, P, P, sz, P],
+            "moe_permute_noalloc": [P, P, P, S, P, P, P, P, P],
             "moe_grouped_swiglu": [P, P, P, P, P, P, P, P, P, S, P, P, P, sz, P],
             "moe_expert_up": [P, P, P, P, S, ctypes.c_int32, P, P],
             "moe_expert_down": [P, P, P, S, ctypes.c_int32, P, P],
@@ -140,6 +142,14 @@ def moe_load_and_bias_update(counts, shape, step, target, bias, load_out=None, s
 def moe_permute(x, topk_idx, counts, shape, x_perm, offsets, perm_tok, inv_row, workspace, stream=None):
     _check(lib().moe_permute(_p(x), _p(topk_idx), _p(counts), shape, _p(x_perm), _p(offsets), _p(perm_tok),
                              _p(inv_row), _p(workspace), _nbytes(workspace), _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(x, topk_idx, counts, shape, x_perm, offsets, perm_tok, inv_row, stream=None):
+    """moe_permute for callers that cannot provide scratch memory: the
+    library uses a fixed array in its own device image instead (see
+    moe_gate.h for the size limit and the sharing rules)."""
+    _check(lib().moe_permute_noalloc(_p(x), _p(topk_idx), _p(counts), shape, _p(x_perm), _p(offsets), _p(perm_tok),
+                                     _p(inv_row), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_grouped_swiglu(x_perm, offsets, w1, w3, w2, x, ws1, ws3, ws2, shape, y_perm, shared_out, workspace,

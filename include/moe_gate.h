@@ -129,6 +129,29 @@ MOE_API moe_status moe_permute(const void* x, const int32_t* topk_idx, const int
 MOE_API size_t moe_permute_workspace_size(moe_shape sh);
 
 /* ---------------------------------------------------------------------------
+ * moe_permute_noalloc -- moe_permute without a workspace argument.  The pages
+ * have no counterpart: this is an interface for callers that cannot give the
+ * library scratch memory (a host framework that owns all device memory and
+ * offers its plugins no allocator, or a deployment that reserves a fixed
+ * device-memory budget up front and forbids allocation at run time).
+ * Same arguments, results and errors as moe_permute, minus workspace.  The
+ * scratch lives in a fixed 256 KiB array inside the library's device image,
+ * which every GPU that loads the library keeps until the process exits; it
+ * holds ceil(T / 128) * E int32 counters, so problems needing more than
+ * 65536 (e.g. T > 32768 with E = 256) are rejected with MOE_ERR_UNSUPPORTED
+ * before anything is launched.  Nothing is allocated: no cudaMalloc, no
+ * cudaFree.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  All calls share the one array and
+ * it keeps the last call's contents (this permutation overwrites every
+ * counter it reads, so nothing needs clearing); calls that overlap on the
+ * GPU -- on different streams, or from different host threads -- race on it.
+ * -------------------------------------------------------------------------*/
+MOE_API moe_status moe_permute_noalloc(const void* x, const int32_t* topk_idx, const int32_t* counts, moe_shape sh,
+                                       void* x_perm, int32_t* offsets, int32_t* perm_tok, int32_t* inv_row,
+                                       void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_grouped_swiglu -- the routed experts as one grouped SwiGLU GEMM pair,
  * and optionally the always-on shared experts  [P2 DeepSeekMoE sketch:
  * per-expert MLPs on the tokens routed to them; shared experts on every
