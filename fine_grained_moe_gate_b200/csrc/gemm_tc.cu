@@ -1,41 +1,48 @@
-// Grouped expert GEMMs on the sm_100a tensor cores (tcgen05 + TMEM + TMA)
-// for the bf16 layer ("Scaling Efficiency: A Deep Dive into the DeepSeek-V3
-// Architecture", DeepSeekMoE sketch: one MLP per expert over the tokens
-// routed to it; "DeepSeek V3 Architecture Deep Dive ...", "Throughput on
-// NVIDIA H100/H800": tokens of one expert batched together).
+// Grouped expert GEMMs on the sm_100a tensor cores (2-SM tcgen05 MMA, TMEM,
+// TMA) for the bf16 layer ("Scaling Efficiency: A Deep Dive into the
+// DeepSeek-V3 Architecture", DeepSeekMoE sketch: one MLP per expert over the
+// tokens routed to it; "DeepSeek V3 Architecture Deep Dive ...", "Throughput
+// on NVIDIA H100/H800": tokens of one expert batched together).
 //
 //   up:   h[t][f] = silu(W1_g[f] . a[t]) * (W3_g[f] . a[t])   (SwiGLU fused)
 //   down: y[t][o] = W2_g[o] . h[t]
 //
-// Weights are the MMA's M operand (128 output features per tile) and the
-// expert's tokens the N operand.  N only has to be a multiple of 16, so the
-// last token tile of an expert is trimmed to its real rows rounded up to 16
-// instead of padding a 128-row M tile: with ~256 rows per expert the
-// padded MMA work drops from ~25% to ~3%.
+// Swap-AB: the expert's weights are the MMA's M operand and its tokens the N
+// operand.  N only has to be a multiple of 16, so an expert's tokens are cut
+// into ceil(rows / 256) tiles of equal size, each rounded up to 16, instead
+// of padding 128-row M tiles (padded MMA work on the V3 routing drops from
+// ~25% to a few percent).
 //
-//   up tile:   128 features of W1 and the same 128 of W3 x up to 128 tokens;
-//              two MMAs per K step into TMEM columns [0,128) (gate) and
-//              [128,256) (up), so one thread holds gate and up of its feature
-//              and SwiGLU is an epilogue over the accumulator.
-//   down tile: 128 features of W2 x up to 256 tokens, one MMA per K step.
-// Both use 48 KB smem stages (4-stage TMA ring, 128-byte swizzle) and two
-// 256-column TMEM accumulators, so the epilogue of one tile overlaps the
-// main loop of the next.  Weights stay in their natural [out][in] layout.
+// Each tile runs on a cluster of two CTAs (two SMs) sharing one
+// cta_group::2 MMA of M = 256 weight rows (128 in each CTA's shared memory)
+// by N <= 256 tokens (N/2 rows in each CTA); each CTA's TMEM receives its 128
+// rows of the result.  Per SM and K step that is 16 KB of weights + 16 KB of
+// tokens for 128 x 256 x 64 MMA work -- a third fewer operand bytes per FLOP
+// than a one-SM 128 x 256 tile, and 32 KB stages allow a 6-deep TMA ring.
 //
-// One persistent CTA per SM walks a device-side tile list built from the
-// expert offsets (no host read-back); per expert, token tiles are walked
-// fastest so the CTAs working on one weight tile at the same time share it
-// in L2, and the expert's token rows stay in L2 across its feature tiles.
+//   up tile:   each CTA holds 64 rows of W1 and the same 64 rows of W3, so
+//              its TMEM lanes 0-63 hold gate and 64-127 up of its 64 output
+//              features; the epilogue pairs them through shared memory.
+//   down tile: each CTA holds 128 rows of W2 (its 128 output features).
+// The weights stay in their natural [out][in] layout (no packing pass).
 //
-// Warp roles (192 threads):
-//   warp 0      TMA producer (one lane)
-//   warp 1      TMEM owner; one lane issues tcgen05.mma (kind::f16, M=128,
-//               N = trimmed token count) and commits to the barriers
-//   warps 2..5  epilogue: tcgen05.ld (32 lanes = 32 features x 16 tokens),
-//               SwiGLU / bf16 conversion, transpose through a 1 KB per-warp
-//               shared buffer into token-major rows, 32-byte vector stores.
+// One persistent cluster per SM pair walks a device-side tile list built
+// from the expert offsets (no host read-back); per expert, token tiles are
+// walked fastest so clusters working on one weight tile at the same time
+// share it in L2, and the expert's tokens stay in L2 across feature tiles.
+//
+// Warp roles (192 threads per CTA):
+//   warp 0      TMA producer (one lane), both CTAs: loads its own halves,
+//               completion counted on the leader CTA's barrier.
+//   warp 1      TMEM owner (paired allocation); in the leader (even) CTA one
+//               lane issues the MMAs and commits to both CTAs' barriers.
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 16 tokens into shared memory,
+//               SwiGLU / bf16 conversion, token-major vector stores.  Two
+//               256-column TMEM accumulators let the epilogue of one tile
+//               overlap the main loop of the next.
 // Every wait is bounded (common.cuh); on a timeout the CTA raises its abort
-// flag, drains the copies and MMAs it issued, frees TMEM and exits.
+// flag, drains what it issued, frees TMEM and exits (the peer then times out
+// on its next wait and does the same).
 #include "common.cuh"
 #include "kernels.h"
 #include "tmap.h"
@@ -43,24 +50,19 @@
 namespace moe {
 namespace {
 
-constexpr int BF = 128;  // weight rows (output features) per tile = MMA M
-constexpr int BK = 64;   // K per stage: one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
-constexpr int W_BYTES = BF * BK * 2;  // 16 KB per weight operand
-constexpr int STAGE_BYTES = 48 * 1024;
-constexpr int SMALL_ROWS = 32;        // token box for tiles of <= 32 tokens
-constexpr uint32_t ACC_COLS = 256;    // one accumulator buffer
+constexpr int BK = 64;                  // K per stage: one 128-byte swizzle row of bf16
+constexpr int STAGES = 6;
+constexpr int A_BYTES = 128 * BK * 2;   // this CTA's 128 weight rows
+constexpr int B_ROWS = 128;             // this CTA's half of <= 256 tokens
+constexpr int B_BYTES = B_ROWS * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
+constexpr int NT = 256;                 // tokens per tile (MMA N <= 256)
+constexpr int SMALL_ROWS = 16;          // per-CTA token box for tiles of <= 32 tokens
+constexpr uint32_t ACC_COLS = 256;      // one accumulator buffer
 constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
 constexpr int NTHREADS = 192;
-constexpr int EPI_BUF = 16 * 32 * 2;  // per-warp transpose buffer: 16 tokens x 32 features
-
-template <bool UP>
-struct Geo {
-    static constexpr int NT = UP ? 128 : 256;              // tokens per tile
-    static constexpr int A_BYTES = UP ? 2 * W_BYTES : W_BYTES;
-    static constexpr int B_BYTES = NT * BK * 2;
-    static_assert(A_BYTES + B_BYTES == STAGE_BYTES, "stage layout");
-};
+constexpr int XS = 132;                 // row stride (floats) of the epilogue exchange buffer
+constexpr int XBUF_BYTES = 16 * XS * 4; // 16 tokens x 128 lanes (+pad), fp32
 
 struct Ctl {
     uint64_t full[STAGES];
@@ -77,12 +79,13 @@ struct Tables {
     int ttiles[kMaxGroups];  // token tiles per group
     int prefix[kMaxGroups + 1];
 };
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 4 * EPI_BUF + sizeof(Ctl) + sizeof(Tables);
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 2 * XBUF_BYTES + sizeof(Ctl) + sizeof(Tables);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 struct Params {
     const int32_t* offsets;
     int G, M;
-    int f_tiles;       // feature tiles per group
+    int f_tiles;       // feature tiles (per CTA pair) per group
     int k_blocks;
     int w_rows;        // up: rows of W1/W3 per group (I)
     int kseg, nseg;    // down: W2 block geometry along K
@@ -108,26 +111,62 @@ __device__ __forceinline__ TileCoord tile_coords(const Tables* tb, int G, int ti
     return {lo, q / nt, q - (q / nt) * nt};
 }
 
-__device__ __forceinline__ uint16_t bf16_bits(float v) {
-    const __nv_bfloat16 b = __float2bfloat16_rn(v);
-    return *reinterpret_cast<const uint16_t*>(&b);
+// Token tile tt of a group with `rows` tokens split into `ntt` tiles of
+// near-equal size (<= NT each).  Equal sizes keep the clusters that share a
+// weight tile at the same pace, so the weight tile is still in L2 when the
+// slower one reads it (a small tail tile would run ahead and let L2 evict).
+__device__ __forceinline__ void token_tile(int rows, int ntt, int tt, int& start, int& len) {
+    const int q = rows / ntt, r = rows - q * ntt;
+    start = tt * q + min(tt, r);
+    len = q + (tt < r ? 1 : 0);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// Bounded wait with cluster-scope acquire (for barriers the peer CTA arrives on).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  int* status) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if ((it & 63u) == 63u) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                report(status, kStTimeout);
+                return false;
+            }
+        }
+    }
 }
 
 template <bool UP>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
                            const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXs,
                            const Params p) {
-    using GE = Geo<UP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = base;
-    uint8_t* epi = base + STAGES * STAGE_BYTES;
-    Ctl* ctl = reinterpret_cast<Ctl*>(epi + 4 * EPI_BUF);
+    float* xbuf = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
+    Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + 2 * XBUF_BYTES);
     Tables* tb = reinterpret_cast<Tables*>(ctl + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();  // 0 = leader (issues the MMAs)
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const int G = p.G;
 
     for (int g = tid; g < G; g += NTHREADS) {
@@ -140,7 +179,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         tb->rowstart[g] = rows > 0 ? rs : 0;
         tb->rows[g] = rows;
-        tb->ttiles[g] = (rows + GE::NT - 1) / GE::NT;
+        tb->ttiles[g] = (rows + NT - 1) / NT;
     }
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -149,15 +188,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&ctl->tfull[a], 1);
-            mbar_init(&ctl->tempty[a], 128);
+            mbar_init(&ctl->tempty[a], 8);  // 4 epilogue warps x 2 CTAs
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(&ctl->tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     __syncthreads();
     if (warp == 0) {  // exclusive prefix of per-group tile counts
@@ -177,72 +216,77 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) tb->prefix[G] = carry;
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
     const int total = tb->prefix[G];
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (both CTAs)
         if (elect_one()) {
             tma_prefetch_desc(&tmW0);
             if (UP) tma_prefetch_desc(&tmW1);
             tma_prefetch_desc(&tmX);
             tma_prefetch_desc(&tmXs);
+            const uint32_t leader_full = mapa_shared(smem_u32(&ctl->full[0]), 0);
             int stage = 0;
-            uint32_t phase = 0, issued = 0, iss_phase = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            uint32_t phase = 0;
+            bool ok = true, issued_any = false;
+            for (int tile = pair; tile < total && ok; tile += npairs) {
                 const TileCoord tc = tile_coords(tb, G, tile);
-                const int tok0 = tb->rowstart[tc.g] + tc.tt * GE::NT;
-                const int ntok = min(GE::NT, tb->rows[tc.g] - tc.tt * GE::NT);
-                const bool small = ntok <= SMALL_ROWS;
-                const uint32_t tx = GE::A_BYTES + (small ? SMALL_ROWS : GE::NT) * BK * 2;
+                int tstart, ntok;
+                token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
+                const int half = ((ntok + 15) & ~15) >> 1;
+                const int tok0 = tb->rowstart[tc.g] + tstart + (int)rank * half;
+                const bool small = half <= SMALL_ROWS;
+                const uint32_t tx = 2u * (A_BYTES + (small ? SMALL_ROWS : B_ROWS) * BK * 2);
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, p.status)) {
                         ok = false;
                         break;
                     }
-                    uint64_t* fb = &ctl->full[stage];
+                    const uint32_t fb = leader_full + 8u * (uint32_t)stage;
                     uint8_t* sa = ring + stage * STAGE_BYTES;
-                    uint8_t* sb = sa + GE::A_BYTES;
-                    mbar_arrive_expect_tx(fb, tx);
+                    uint8_t* sb = sa + A_BYTES;
+                    if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], tx);
                     if (UP) {
-                        const int wrow = tc.g * p.w_rows + tc.ft * BF;
-                        tma_load_2d(sa, &tmW0, fb, kb * BK, wrow, kEvictNormal);
-                        tma_load_2d(sa + W_BYTES, &tmW1, fb, kb * BK, wrow, kEvictNormal);
+                        const int wrow = tc.g * p.w_rows + tc.ft * 128 + (int)rank * 64;
+                        tma_load_2d_pair(sa, &tmW0, fb, kb * BK, wrow, kEvictNormal);
+                        tma_load_2d_pair(sa + A_BYTES / 2, &tmW1, fb, kb * BK, wrow, kEvictNormal);
                     } else {
                         const int kk = kb * BK;
                         const int seg = kk / p.kseg;
-                        tma_load_3d(sa, &tmW0, fb, kk - seg * p.kseg, tc.ft * BF, tc.g * p.nseg + seg, kEvictNormal);
+                        tma_load_3d_pair(sa, &tmW0, fb, kk - seg * p.kseg, tc.ft * 256 + (int)rank * 128,
+                                         tc.g * p.nseg + seg, kEvictNormal);
                     }
-                    tma_load_2d(sb, small ? &tmXs : &tmX, fb, kb * BK, tok0, kEvictNormal);
-                    issued |= 1u << stage;
-                    iss_phase = (iss_phase & ~(1u << stage)) | (phase << stage);
+                    tma_load_2d_pair(sb, small ? &tmXs : &tmX, fb, kb * BK, tok0, kEvictNormal);
+                    issued_any = true;
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            if (!ok) {
-                for (int s = 0; s < STAGES; ++s)
-                    if ((issued >> s) & 1u) mbar_wait_drain(&ctl->full[s], (iss_phase >> s) & 1u);
+            if (!ok && issued_any) {  // let copies already in flight land before the CTA exits
+                const uint64_t t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 200000ull) {
+                }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (elect_one()) {
+        // ------------------------------------------------ MMA issuer (leader CTA only)
+        if (rank == 0 && elect_one()) {
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            for (int tile = pair; tile < total && ok; tile += npairs) {
                 const TileCoord tc = tile_coords(tb, G, tile);
-                const int ntok = min(GE::NT, tb->rows[tc.g] - tc.tt * GE::NT);
+                int tstart, ntok;
+                token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
                 const int n_mma = (ntok + 15) & ~15;
-                const uint32_t idesc = idesc_bf16_f32(BF, n_mma);
-                if (!mbar_wait(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, p.status)) {
+                const uint32_t idesc = idesc_bf16_f32(256, n_mma);
+                if (!mbar_wait_cluster(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, p.status)) {
                     ok = false;
                     break;
                 }
@@ -255,100 +299,108 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     tc_fence_after();
                     uint8_t* sa = ring + stage * STAGE_BYTES;
-                    const uint64_t ad0 = smem_desc_sw128(smem_u32(sa));
-                    const uint64_t bd = smem_desc_sw128(smem_u32(sa + GE::A_BYTES));
-                    if (UP) {
-                        const uint64_t ad1 = smem_desc_sw128(smem_u32(sa + W_BYTES));
+                    const uint64_t ad = smem_desc_sw128(smem_u32(sa));
+                    const uint64_t bd = smem_desc_sw128(smem_u32(sa + A_BYTES));
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk) {  // +32 bytes along K per step
-                            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
-                            tc_mma_bf16(d_tmem, ad0 + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, accum);
-                            tc_mma_bf16(d_tmem + GE::NT, ad1 + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
-                                        accum);
-                        }
-                    } else {
-#pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            tc_mma_bf16(d_tmem, ad0 + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
-                                        (kb > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    tc_commit(&ctl->empty[stage]);
+                    for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per step
+                        tc_mma_bf16_pair(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+                                         (kb > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit_pair(&ctl->empty[stage], 0x3);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit(&ctl->tfull[acc]);
+                tc_commit_pair(&ctl->tfull[acc], 0x3);
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
             }
-            if (!ok) {
-                tc_commit(&ctl->drain);
+            if (!ok) {  // wait for the pair MMAs already issued (same cta_group as the MMAs)
+                tc_commit_pair(&ctl->drain, 0x1);
                 mbar_wait_drain(&ctl->drain, 0);
             }
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter: features 32q .. 32q+31 of the tile
-        uint16_t* buf = reinterpret_cast<uint16_t*>(epi + q * EPI_BUF);  // [16 tokens][32 features]
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;           // TMEM lane quarter this warp may read
+        const int e = tid - 64;           // 0..127 among the epilogue threads
+        const int my_tok = e >> 3;        // token (0..15) of a 16-token chunk this thread stores
+        const int part = e & 7;
+        const uint32_t leader_tempty = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-        int acc = 0;
+        int acc = 0, xb = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        for (int tile = pair; tile < total; tile += npairs) {
             const TileCoord tc = tile_coords(tb, G, tile);
-            const int tok0 = tb->rowstart[tc.g] + tc.tt * GE::NT;
-            const int ntok = min(GE::NT, tb->rows[tc.g] - tc.tt * GE::NT);
-            const int f0 = tc.ft * BF + q * 32;  // first feature of this warp
+            int tstart, ntok;
+            token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
+            const int tok0 = tb->rowstart[tc.g] + tstart;
+            // first output feature of this CTA
+            const int fcta = UP ? tc.ft * 128 + (int)rank * 64 : tc.ft * 256 + (int)rank * 128;
             if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, p.status)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACC_COLS;
-            // this lane's share of a 16-token x 32-feature block: token lane/2, 16 features
-            const int my_tok = lane >> 1;
-            const int my_half = (lane & 1) * 16;
-            const bool feat_ok = f0 + my_half < p.f_limit;  // f_limit is a multiple of 16
 #pragma unroll 1
             for (int c = 0; c < ntok; c += 16) {
-                float v[16];
-                if (UP) {
-                    uint32_t gv[16], uv[16];
-                    tmem_ld16(taddr + (uint32_t)c, gv);
-                    tmem_ld16(taddr + (uint32_t)(GE::NT + c), uv);
-                    tmem_ld_wait();
+                uint32_t r[16];
+                tmem_ld16(taddr + (uint32_t)c, r);
+                tmem_ld_wait();
+                float* xs = xbuf + xb * (XBUF_BYTES / 4);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = silu_f32(__uint_as_float(gv[i])) * __uint_as_float(uv[i]);
+                for (int i = 0; i < 16; ++i) xs[i * XS + q * 32 + lane] = __uint_as_float(r[i]);
+                named_bar_sync(1, 128);
+                const bool tok_ok = c + my_tok < ntok;
+                const float* row = xs + my_tok * XS;
+                if (UP) {  // lanes 0-63: gate, 64-127: up of the same 64 features
+                    const int fj = part * 8;
+                    const float4 g0 = *reinterpret_cast<const float4*>(row + fj);
+                    const float4 g1 = *reinterpret_cast<const float4*>(row + fj + 4);
+                    const float4 u0 = *reinterpret_cast<const float4*>(row + 64 + fj);
+                    const float4 u1 = *reinterpret_cast<const float4*>(row + 64 + fj + 4);
+                    if (tok_ok) {
+                        uint4 v;
+                        v.x = pack_bf16x2(silu_f32(g0.x) * u0.x, silu_f32(g0.y) * u0.y);
+                        v.y = pack_bf16x2(silu_f32(g0.z) * u0.z, silu_f32(g0.w) * u0.w);
+                        v.z = pack_bf16x2(silu_f32(g1.x) * u1.x, silu_f32(g1.y) * u1.y);
+                        v.w = pack_bf16x2(silu_f32(g1.z) * u1.z, silu_f32(g1.w) * u1.w);
+                        *reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * p.ldo + fcta + fj) = v;
+                    }
                 } else {
-                    uint32_t r[16];
-                    tmem_ld16(taddr + (uint32_t)c, r);
-                    tmem_ld_wait();
+                    const int fj = part * 16;
+                    if (tok_ok && fcta + fj < p.f_limit) {
+                        float f[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 t = *reinterpret_cast<const float4*>(row + fj + 4 * i);
+                            f[4 * i] = t.x;
+                            f[4 * i + 1] = t.y;
+                            f[4 * i + 2] = t.z;
+                            f[4 * i + 3] = t.w;
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * p.ldo + fcta + fj);
+                        dst[0] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                                            pack_bf16x2(f[6], f[7]));
+                        dst[1] = make_uint4(pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
+                                            pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
+                    }
                 }
-                // transpose: buf[token i][feature lane]
-#pragma unroll
-                for (int i = 0; i < 16; ++i) buf[i * 32 + lane] = bf16_bits(v[i]);
-                __syncwarp();
-                if (c + my_tok < ntok && feat_ok) {
-                    const uint4* src = reinterpret_cast<const uint4*>(buf + my_tok * 32 + my_half);
-                    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * p.ldo + f0 + my_half);
-                    dst[0] = src[0];
-                    dst[1] = src[1];
-                }
-                __syncwarp();
+                xb ^= 1;  // the next chunk writes the other buffer; its barrier orders the reuse
             }
             tc_fence_before();
-            mbar_arrive(&ctl->tempty[acc]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_tempty + 8u * (uint32_t)acc);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
     }
 
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while its peer's MMAs may still read its shared memory
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
 }
 
@@ -358,7 +410,8 @@ cudaError_t launch(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorM
     auto kern = tc_grouped_gemm_kernel<UP>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    kern<<<num_sms, NTHREADS, SMEM_BYTES, st>>>(w0, w1, x, xs, p);
+    const int grid = (num_sms / 2) * 2;  // whole CTA pairs, one CTA per SM
+    kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(w0, w1, x, xs, p);
     note_launches(1);
     return cudaGetLastError();
 }
@@ -366,17 +419,17 @@ cudaError_t launch(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorM
 }  // namespace
 
 cudaError_t launch_tc_up(const TcUpArgs& a, int* status, int num_sms, cudaStream_t st) {
-    if (a.G <= 0 || a.G > kMaxGroups || a.d % BK != 0 || a.I % BF != 0) return cudaErrorInvalidValue;
+    if (a.G <= 0 || a.G > kMaxGroups || a.d % BK != 0 || a.I % 128 != 0) return cudaErrorInvalidValue;
     CUtensorMap tW1, tW3, tX, tXs;
-    if (!make_tmap_2d(&tW1, a.W1, a.d, a.W_rows, a.d, BK, BF) || !make_tmap_2d(&tW3, a.W3, a.d, a.W_rows, a.d, BK, BF) ||
-        !make_tmap_2d(&tX, a.A, a.d, a.A_rows, a.d, BK, Geo<true>::NT) ||
+    if (!make_tmap_2d(&tW1, a.W1, a.d, a.W_rows, a.d, BK, 64) || !make_tmap_2d(&tW3, a.W3, a.d, a.W_rows, a.d, BK, 64) ||
+        !make_tmap_2d(&tX, a.A, a.d, a.A_rows, a.d, BK, B_ROWS) ||
         !make_tmap_2d(&tXs, a.A, a.d, a.A_rows, a.d, BK, SMALL_ROWS))
         return cudaErrorInvalidValue;
     Params p{};
     p.offsets = a.offsets;
     p.G = a.G;
     p.M = a.M;
-    p.f_tiles = a.I / BF;
+    p.f_tiles = a.I / 128;
     p.k_blocks = a.d / BK;
     p.w_rows = a.I;
     p.kseg = a.d;
@@ -393,15 +446,15 @@ cudaError_t launch_tc_down(const TcDownArgs& a, int* status, int num_sms, cudaSt
     if (a.G <= 0 || a.G > kMaxGroups || a.K % BK != 0 || a.kseg % BK != 0 || a.d % 16 != 0)
         return cudaErrorInvalidValue;
     CUtensorMap tW2, tX, tXs;
-    if (!make_tmap_3d(&tW2, a.W2, a.kseg, a.d, (unsigned long long)a.G * a.nseg, BK, BF) ||
-        !make_tmap_2d(&tX, a.H, a.K, a.H_rows, a.K, BK, Geo<false>::NT) ||
+    if (!make_tmap_3d(&tW2, a.W2, a.kseg, a.d, (unsigned long long)a.G * a.nseg, BK, 128) ||
+        !make_tmap_2d(&tX, a.H, a.K, a.H_rows, a.K, BK, B_ROWS) ||
         !make_tmap_2d(&tXs, a.H, a.K, a.H_rows, a.K, BK, SMALL_ROWS))
         return cudaErrorInvalidValue;
     Params p{};
     p.offsets = a.offsets;
     p.G = a.G;
     p.M = a.M;
-    p.f_tiles = (a.d + BF - 1) / BF;
+    p.f_tiles = (a.d + 255) / 256;
     p.k_blocks = a.K / BK;
     p.w_rows = 0;
     p.kseg = a.kseg;
