@@ -222,6 +222,7 @@ def run_ours(args, world, rank, local):
     import torch.distributed as dist
 
     import fine_grained_moe_gate_b200 as moe
+    from fine_grained_moe_gate_b200 import dist as mdist
     from fine_grained_moe_gate_b200.inputs import make_layer, make_tokens
 
     torch.cuda.set_device(local)
@@ -230,12 +231,12 @@ def run_ours(args, world, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     cfg = workload(args)
     sh = moe.shape_of(cfg)
-    sh_global = moe.shape_of(cfg, T=cfg.T * world)   # the step's batch for the bias update
+    sh_global = moe.shape_of(cfg, T=mdist.global_token_count(cfg.T, world))  # the step's batch, all ranks
     stream = torch.cuda.current_stream()
 
     p = make_layer(cfg, dev)
     n_x = max(1, min(4, args.steps + args.warmup))
-    xs = [make_tokens(cfg, dev, step=i * world + rank) for i in range(n_x)]
+    xs = [make_tokens(cfg, dev, step=mdist.shard_step(i, rank, world)) for i in range(n_x)]
 
     T, k, d, E = cfg.T, cfg.k, cfg.d, cfg.E
     dt = cfg.torch_dtype
@@ -272,8 +273,7 @@ def run_ours(args, world, rank, local):
         rec(6)
         moe.moe_combine(x_perm, w, inv, shared_out, sh, y, stream)
         rec(7)
-        if world > 1:
-            dist.all_reduce(counts)
+        mdist.allreduce_counts(counts)
         moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
         rec(8)
 
@@ -331,8 +331,7 @@ def run_ours(args, world, rank, local):
             x_dev.copy_(x_host[i % n_x], non_blocking=True)
             moe.moe_layer_forward(x_dev, p["w_gate"], p["bias"], p["w1"], p["w3"], p["w2"], p["ws1"], p["ws3"],
                                   p["ws2"], sh, y, idx, w, counts, ws, stream)
-            if world > 1:
-                dist.all_reduce(counts)
+            mdist.allreduce_counts(counts)
             moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
             y_host.copy_(y, non_blocking=True)
 

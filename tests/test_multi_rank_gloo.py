@@ -1,0 +1,101 @@
+"""The multi-GPU path's host logic on CPU with world size 2 (gloo): token
+shards per rank, the one exchange (per-expert counts summed over ranks) and
+the bias update with the global token count ("A bias term for each expert":
+the load is taken over the whole batch of the step).  The oracle stands in
+for the per-rank kernels, which need a GPU."""
+import datetime
+import json
+import os
+import socket
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+WORLD = 2
+STEPS = 3
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _cfg():
+    from fine_grained_moe_gate_b200.inputs import CONFIGS
+    return CONFIGS["tiny_fp32"].scaled(T=48, d=64, E=32, k=4, I=8, Is=8)
+
+
+def _worker(rank, port, out_dir, fail_rank):
+    import torch.distributed as dist
+
+    import oracle
+    from fine_grained_moe_gate_b200 import dist as mdist
+    from fine_grained_moe_gate_b200.inputs import make_layer, make_tokens, to_numpy
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD, timeout=datetime.timedelta(seconds=10))
+    cfg = _cfg()
+    p = make_layer(cfg, "cpu")                      # same seed on every rank: replicated weights
+    wg = to_numpy(p["w_gate"])
+    bias = p["bias"].numpy().copy()
+    result = {"rank": rank, "biases": [], "error": None}
+    try:
+        for step in range(STEPS):
+            x = make_tokens(cfg, "cpu", step=mdist.shard_step(step, rank, WORLD))
+            s = oracle.affinity(to_numpy(x), wg)
+            idx, _ = oracle.select(s, bias, cfg.k)
+            counts = torch.from_numpy(oracle.histogram(idx, cfg.E))
+            if rank == fail_rank:
+                raise RuntimeError("injected host-side failure before the exchange")
+            mdist.allreduce_counts(counts)
+            bias, _ = oracle.bias_update(counts.numpy(), bias, mdist.global_token_count(cfg.T, WORLD), cfg.k,
+                                         cfg.step_size)
+            result["biases"].append(bias.view(np.uint32).tolist())
+    except Exception as e:  # reported to the parent, never hangs the test
+        result["error"] = f"{type(e).__name__}: {e}"
+    with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+        json.dump(result, f)
+    try:
+        dist.destroy_process_group()
+    except Exception:
+        pass
+
+
+def _run(fail_rank):
+    out_dir = tempfile.mkdtemp(prefix="gloo_")
+    mp.start_processes(_worker, args=(_free_port(), out_dir, fail_rank), nprocs=WORLD, join=True,
+                       start_method="spawn")
+    return [json.load(open(os.path.join(out_dir, f"rank{r}.json"))) for r in range(WORLD)]
+
+
+def test_two_ranks_keep_identical_bias_equal_to_single_process():
+    import oracle
+    from fine_grained_moe_gate_b200 import dist as mdist
+    from fine_grained_moe_gate_b200.inputs import make_layer, make_tokens, to_numpy
+
+    res = _run(fail_rank=-1)
+    for r in res:
+        assert r["error"] is None, r["error"]
+    assert res[0]["biases"] == res[1]["biases"]     # bit-identical on every rank, every step
+    # single process over the concatenated batch of each step
+    cfg = _cfg()
+    p = make_layer(cfg, "cpu")
+    wg = to_numpy(p["w_gate"])
+    bias = p["bias"].numpy().copy()
+    for step in range(STEPS):
+        x = torch.cat([make_tokens(cfg, "cpu", step=mdist.shard_step(step, r, WORLD)) for r in range(WORLD)])
+        idx, _ = oracle.select(oracle.affinity(to_numpy(x), wg), bias, cfg.k)
+        bias, _ = oracle.bias_update(oracle.histogram(idx, cfg.E), bias, x.shape[0], cfg.k, cfg.step_size)
+        assert bias.view(np.uint32).tolist() == res[0]["biases"][step], f"step {step}"
+
+
+def test_a_failed_rank_ends_the_exchange_with_an_error_not_a_hang():
+    res = _run(fail_rank=1)
+    assert "injected" in res[1]["error"]
+    assert res[0]["error"] is not None             # the survivor's all-reduce errored out within the timeout
+    assert len(res[0]["biases"]) == 0
