@@ -247,7 +247,7 @@ def run_ours(args, world, rank, local):
     perm = torch.empty(T * k, dtype=torch.int32, device=dev)
     inv = torch.empty(T * k, dtype=torch.int32, device=dev)
     pws = torch.empty(max(moe.moe_permute_workspace_size(sh), 256), dtype=torch.uint8, device=dev)
-    x_perm = torch.empty((T * k, d), dtype=dt, device=dev)   # also holds y_perm after the up projection
+    x_perm = torch.empty((T * k, d), dtype=dt, device=dev)   # x_perm, then y_perm
     h = torch.empty((T * k, cfg.I), dtype=dt, device=dev)
     hs = torch.empty((T, max(1, cfg.S * cfg.Is)), dtype=dt, device=dev)
     shared_out = torch.empty((T, d), dtype=dt, device=dev) if cfg.S > 0 else None
@@ -261,10 +261,10 @@ def run_ours(args, world, rank, local):
         rec(1)
         moe.moe_permute(x, idx, counts, sh, x_perm, offsets, perm, inv, pws, stream)
         rec(2)
-        moe.moe_expert_up(x_perm, offsets, p["w1"], p["w3"], sh, moe.MOE_ROUTED, h, stream)
+        moe.moe_expert_up(x_perm, None, offsets, p["w1"], p["w3"], sh, moe.MOE_ROUTED, h, stream)
         rec(3)
         if cfg.S > 0:
-            moe.moe_expert_up(x, None, p["ws1"], p["ws3"], sh, moe.MOE_SHARED, hs, stream)
+            moe.moe_expert_up(x, None, None, p["ws1"], p["ws3"], sh, moe.MOE_SHARED, hs, stream)
         rec(4)
         moe.moe_expert_down(h, offsets, p["w2"], sh, moe.MOE_ROUTED, x_perm, stream)
         rec(5)
@@ -360,6 +360,23 @@ def run_ours(args, world, rank, local):
     flops_per_launch = T * k * 4 * d * cfg.I   # gate + up, real rows only
     dom_ms = stage_ms[DOMINANT]
     achieved = flops_per_launch / (dom_ms / 1e3) / 1e12
+    # algorithmic bytes of that launch: W1 + W3 of the experts that got rows
+    # (counted by routing each input once more, outside the timed region),
+    # the token rows read and h written
+    touched = []
+    for xx in xs:
+        moe.moe_route(xx, p["w_gate"], p["bias"], sh, idx, w, counts, None, stream)
+        touched.append(int((counts > 0).sum().item()))
+    n_touched = statistics.mean(touched)
+    esz = 2 if cfg.dtype == "bf16" else 4
+    bytes_per_launch = n_touched * 2 * cfg.I * d * esz + T * k * (d + cfg.I) * esz
+    hbm_gbs = bytes_per_launch / (dom_ms / 1e3) / 1e9
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    roof_hbm = {"bound": "hbm", "kernel": "routed up projection", "achieved": round(hbm_gbs, 1), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(hbm_gbs / hbm_peak, 4),
+                "frac_of_nominal_8000": round(hbm_gbs / 8000.0, 4),
+                "traffic": None, "bytes_per_launch": int(bytes_per_launch), "experts_touched": n_touched,
+                "peak_kind": f"hbm_gbs ({peak_src}, copy bandwidth)"}
     if cfg.dtype == "bf16":
         peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         roof = {"bound": "tensor", "kernel": "tc_grouped_gemm_kernel<up> (routed experts, SwiGLU epilogue)",
@@ -371,6 +388,9 @@ def run_ours(args, world, rank, local):
         roof = {"bound": "alu", "kernel": "simt_grouped_gemm_kernel (fp32 FFMA)", "achieved": round(achieved, 3),
                 "peak": None, "unit": "TFLOP/s", "frac": None, "traffic": None,
                 "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
+    if cfg.name.startswith("v3_decode"):
+        # a few tokens per expert: the launch streams the touched experts' weights
+        roof, roof_hbm = roof_hbm, roof
     layer_flops = cfg.flops()
     step_tflops = layer_flops / (ms_per_step / 1e3) / 1e12
 
@@ -392,6 +412,7 @@ def run_ours(args, world, rank, local):
                              f"({(p['w1'].numel() * 3 + p['ws1'].numel() * 3) * p['w1'].element_size() / 1e9:.1f} GB)",
                        "bias_update": "every step"},
             "roofline": roof,
+            "roofline_alt": roof_hbm,
             "layer_tflops": round(step_tflops, 2),
             "layer_frac_of_peak": round(step_tflops / float(peaks.get("bf16_tflops_sustained", 1400.0)), 4)
             if cfg.dtype == "bf16" else None,

@@ -76,7 +76,7 @@ def lib() -> ctypes.CDLL:
             "moe_permute": [P, P, P, S, P, P, P, P, P, sz, P],
             "moe_permute_noalloc": [P, P, P, S, P, P, P, P, P],
             "moe_grouped_swiglu": [P, P, P, P, P, P, P, P, P, S, P, P, P, sz, P],
-            "moe_expert_up": [P, P, P, P, S, ctypes.c_int32, P, P],
+            "moe_expert_up": [P, P, P, P, P, S, ctypes.c_int32, P, P],
             "moe_expert_down": [P, P, P, S, ctypes.c_int32, P, P],
             "moe_combine": [P, P, P, P, S, P, P],
             "moe_layer_forward": [P, P, P, P, P, P, P, P, P, S, P, P, P, P, P, sz, P],
@@ -159,9 +159,9 @@ def moe_grouped_swiglu(x_perm, offsets, w1, w3, w2, x, ws1, ws3, ws2, shape, y_p
                                     _stream(stream)), "moe_grouped_swiglu")
 
 
-def moe_expert_up(a, offsets, w1, w3, shape, expert_set, h, stream=None):
-    _check(lib().moe_expert_up(_p(a), _p(offsets), _p(w1), _p(w3), shape, expert_set, _p(h), _stream(stream)),
-           "moe_expert_up")
+def moe_expert_up(a, gather_idx, offsets, w1, w3, shape, expert_set, h, stream=None):
+    _check(lib().moe_expert_up(_p(a), _p(gather_idx), _p(offsets), _p(w1), _p(w3), shape, expert_set, _p(h),
+                               _stream(stream)), "moe_expert_up")
 
 
 def moe_expert_down(h, offsets, w2, shape, expert_set, y, stream=None):

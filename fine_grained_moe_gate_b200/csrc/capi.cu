@@ -96,19 +96,23 @@ moe_status do_permute(const void* x, const int32_t* idx, const int32_t* counts, 
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-moe_status do_expert_up(const void* a, const int32_t* offsets, const void* w1, const void* w3, const moe_shape& sh,
-                        bool shared, void* h, int* status, int sms, cudaStream_t st) {
+// gather (routed set only, may be null): group row r reads row gather[r] / k
+// of `a` (= x, unpermuted); without it `a` is x_perm itself.
+moe_status do_expert_up(const void* a, const int32_t* gather, const int32_t* offsets, const void* w1, const void* w3,
+                        const moe_shape& sh, bool shared, void* h, int* status, int sms, cudaStream_t st) {
     if (sh.T == 0) return MOE_OK;
-    const long long rows = shared ? sh.T : (long long)sh.T * sh.k;
+    const long long rows = shared ? sh.T : (long long)sh.T * sh.k;  // rows the groups index (= rows of h)
     const int Ig = shared ? sh.S * sh.Is : sh.I;  // S stacked [Is][d] blocks = one [S*Is][d] matrix
+    if (shared) gather = nullptr;
+    const long long a_rows = gather ? sh.T : rows;
     cudaError_t err;
     if (sh.dtype == MOE_BF16) {
-        moe::TcUpArgs up{a, rows, w1, w3, shared ? (long long)Ig : (long long)sh.E * sh.I, h, sh.d, Ig,
-                         shared ? nullptr : offsets, shared ? 1 : sh.E, shared ? sh.T : 0};
+        moe::TcUpArgs up{a, a_rows, gather, sh.k, rows, w1, w3, shared ? (long long)Ig : (long long)sh.E * sh.I, h,
+                         sh.d, Ig, shared ? nullptr : offsets, shared ? 1 : sh.E, shared ? sh.T : 0};
         err = moe::launch_tc_up(up, status, sms, st);
     } else {
         moe::GemmArgs up{a, sh.d, w1, w3, shared ? 0 : (long long)sh.I * sh.d, sh.d, sh.d, 0, h, Ig, Ig, sh.d,
-                         shared ? nullptr : offsets, shared ? 1 : sh.E, (int)rows};
+                         shared ? nullptr : offsets, shared ? 1 : sh.E, (int)rows, gather, sh.k};
         err = moe::launch_simt_gemm(up, false, true, sms, st);
     }
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -129,7 +133,7 @@ moe_status do_expert_down(const void* h, const int32_t* offsets, const void* w2,
         // element (n, kk) of W2 block g: (kk / kseg) * d * kseg + n * kseg + kk % kseg
         moe::GemmArgs dn{h, K, w2, nullptr, shared ? 0 : (long long)sh.d * sh.I, kseg, kseg,
                          (long long)sh.d * kseg, y, sh.d, sh.d, K, shared ? nullptr : offsets, shared ? 1 : sh.E,
-                         (int)rows};
+                         (int)rows, nullptr, 1};
         err = moe::launch_simt_gemm(dn, false, false, sms, st);
     }
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -144,8 +148,8 @@ moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1,
     char* hs = h + align256((size_t)rows * sh.I * eb);
     const bool shared = x && sh.S > 0 && shared_out;
     moe_status v;
-    if ((v = do_expert_up(x_perm, offsets, w1, w3, sh, false, h, status, sms, st)) != MOE_OK) return v;
-    if (shared && (v = do_expert_up(x, nullptr, ws1, ws3, sh, true, hs, status, sms, st)) != MOE_OK) return v;
+    if ((v = do_expert_up(x_perm, nullptr, offsets, w1, w3, sh, false, h, status, sms, st)) != MOE_OK) return v;
+    if (shared && (v = do_expert_up(x, nullptr, nullptr, ws1, ws3, sh, true, hs, status, sms, st)) != MOE_OK) return v;
     if ((v = do_expert_down(h, offsets, w2, sh, false, y_perm, status, sms, st)) != MOE_OK) return v;
     if (shared && (v = do_expert_down(hs, nullptr, ws2, sh, true, shared_out, status, sms, st)) != MOE_OK) return v;
     return MOE_OK;
@@ -235,7 +239,8 @@ moe_status moe_permute(const void* x, const int32_t* topk_idx, const int32_t* co
     moe_status v = validate_shape(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(offsets, MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(sh.T == 0 || (x && topk_idx && x_perm && perm_tok && inv_row), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (topk_idx && perm_tok && inv_row), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(!x_perm || sh.T == 0 || x, MOE_ERR_INVALID_ARG);  // x_perm null: index outputs only
     MOE_REQUIRE(aligned16(x) && aligned16(topk_idx) && aligned16(counts) && aligned16(x_perm) && aligned16(offsets) &&
                     aligned16(perm_tok) && aligned16(inv_row),
                 MOE_ERR_ALIGNMENT);
@@ -273,8 +278,8 @@ moe_status moe_grouped_swiglu(const void* x_perm, const int32_t* offsets, const 
                      workspace, status, sms, static_cast<cudaStream_t>(stream));
 }
 
-moe_status moe_expert_up(const void* a, const int32_t* offsets, const void* w1, const void* w3, moe_shape sh,
-                         int32_t set, void* h, void* stream) {
+moe_status moe_expert_up(const void* a, const int32_t* gather_idx, const int32_t* offsets, const void* w1,
+                         const void* w3, moe_shape sh, int32_t set, void* h, void* stream) {
     moe_status v = validate_shape(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(set == MOE_ROUTED || set == MOE_SHARED, MOE_ERR_INVALID_ARG);
@@ -282,13 +287,16 @@ moe_status moe_expert_up(const void* a, const int32_t* offsets, const void* w1, 
     MOE_REQUIRE(!shared || sh.S > 0, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(w1 && w3 && (shared || offsets), MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(sh.T == 0 || (a && h), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(aligned16(a) && aligned16(offsets) && aligned16(w1) && aligned16(w3) && aligned16(h),
+    MOE_REQUIRE(!shared || !gather_idx, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(a) && aligned16(gather_idx) && aligned16(offsets) && aligned16(w1) && aligned16(w3) &&
+                    aligned16(h),
                 MOE_ERR_ALIGNMENT);
     int dev, sms;
     int* status;
     v = device_setup(&dev, &status, &sms);
     if (v != MOE_OK) return v;
-    return do_expert_up(a, offsets, w1, w3, sh, shared, h, status, sms, static_cast<cudaStream_t>(stream));
+    return do_expert_up(a, gather_idx, offsets, w1, w3, sh, shared, h, status, sms,
+                        static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_expert_down(const void* h, const int32_t* offsets, const void* w2, moe_shape sh, int32_t set, void* y,
@@ -358,19 +366,27 @@ moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bia
     p += align256(rows * sizeof(int32_t));
     void* pws = p;
     p += permute_ws(sh);
-    void* x_perm = p;  // reused for y_perm once the up projection has read it
+    void* x_perm = p;  // x_perm, then y_perm
     p += align256(rows * sh.d * eb);
     void* gws = p;
     p += swiglu_ws(sh);
     void* shared_out = sh.S > 0 ? p : nullptr;
 
+    // route; permute (token rows copied into expert order: a row gather
+    // inside the GEMM's loads, tile::gather4, measured 2x slower for the
+    // routed up projection than this copy plus whole-tile loads)
+    void* y_perm = x_perm;  // the down projection overwrites x_perm once the up projection has read it
+    char* h = static_cast<char*>(gws);
+    char* hs = h + align256(rows * sh.I * eb);
     if ((v = do_route(x, w_gate, bias, sh, topk_idx, topk_w, counts, nullptr, status, sms, st)) != MOE_OK) return v;
     if (sh.T == 0) return MOE_OK;
     if ((v = do_permute(x, topk_idx, counts, sh, x_perm, offsets, perm, inv, pws, status, st)) != MOE_OK) return v;
-    if ((v = do_swiglu(x_perm, offsets, w1, w3, w2, sh.S > 0 ? x : nullptr, ws1, ws3, ws2, sh, x_perm, shared_out, gws,
-                       status, sms, st)) != MOE_OK)
+    if ((v = do_expert_up(x_perm, nullptr, offsets, w1, w3, sh, false, h, status, sms, st)) != MOE_OK) return v;
+    if (sh.S > 0 && (v = do_expert_up(x, nullptr, nullptr, ws1, ws3, sh, true, hs, status, sms, st)) != MOE_OK)
         return v;
-    return moe::launch_combine(x_perm, topk_w, inv, shared_out, sh.T, sh.d, sh.k, sh.dtype == MOE_BF16, y, status,
+    if ((v = do_expert_down(h, offsets, w2, sh, false, y_perm, status, sms, st)) != MOE_OK) return v;
+    if (sh.S > 0 && (v = do_expert_down(hs, nullptr, ws2, sh, true, shared_out, status, sms, st)) != MOE_OK) return v;
+    return moe::launch_combine(y_perm, topk_w, inv, shared_out, sh.T, sh.d, sh.k, sh.dtype == MOE_BF16, y, status,
                                st) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;

@@ -238,6 +238,19 @@ __device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const void* des
         "l"(reinterpret_cast<uint64_t>(desc)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "l"(cache_hint)
         : "memory");
 }
+// Four arbitrary rows (r0..r3) of a 2-D tensor map whose box is one row
+// high, columns [c0, c0 + box width), into four consecutive rows of this
+// CTA's shared memory (the map's swizzle applied); completion bytes counted
+// on the pair leader's barrier.
+__device__ __forceinline__ void tma_gather4_pair(void* smem_dst, const void* desc, uint32_t bar_cluster, int32_t c0,
+                                                 int32_t r0, int32_t r1, int32_t r2, int32_t r3, uint64_t cache_hint) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(desc)), "r"(bar_cluster), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+        "l"(cache_hint)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_slot, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_slot)),
                  "r"(ncols)

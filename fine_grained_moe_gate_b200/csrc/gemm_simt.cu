@@ -77,7 +77,10 @@ __global__ void __launch_bounds__(256) simt_grouped_gemm_kernel(GemmArgs p) {
                 const int kg = k0 + kk;
                 float va = 0.f, vb = 0.f, v3 = 0.f;
                 if (kg < p.K) {
-                    if (m0 + r < Mg) va = to_f32(A[(size_t)(row0 + m0 + r) * p.lda + kg]);
+                    if (m0 + r < Mg) {
+                        const int ar = p.gather ? p.gather[row0 + m0 + r] / p.gather_div : row0 + m0 + r;
+                        va = to_f32(A[(size_t)ar * p.lda + kg]);
+                    }
                     if (n0 + r < p.N) {
                         const size_t boff = (size_t)(kg / p.kseg) * p.seg_stride + (size_t)(n0 + r) * p.ldb +
                                             (size_t)(kg % p.kseg);

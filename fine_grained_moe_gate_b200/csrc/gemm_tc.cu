@@ -92,7 +92,9 @@ struct Params {
     void* out;
     int ldo;           // output row pitch (elements)
     int f_limit;       // valid output features
-    long long a_rows;  // rows of the token operand and of the output
+    long long a_rows;  // rows the groups index (token operand rows, or gathered rows) and output rows
+    const int32_t* gather;  // up, optional: row r of the groups reads token row gather[r] / gather_div
+    int gather_div;
     int* status;
 };
 
@@ -155,7 +157,7 @@ template <bool UP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
                            const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXs,
-                           const Params p) {
+                           const __grid_constant__ CUtensorMap tmXg, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = base;
@@ -223,31 +225,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
-        if (elect_one()) {
+        // Lane 0 waits for free stages and loads the weights; with a gather
+        // index every lane also fetches four token rows (tile::gather4), so
+        // the token operand is read straight from x in expert order.
+        const bool gather = UP && p.gather != nullptr;
+        if (lane == 0) {
             tma_prefetch_desc(&tmW0);
             if (UP) tma_prefetch_desc(&tmW1);
-            tma_prefetch_desc(&tmX);
-            tma_prefetch_desc(&tmXs);
-            const uint32_t leader_full = mapa_shared(smem_u32(&ctl->full[0]), 0);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true, issued_any = false;
-            for (int tile = pair; tile < total && ok; tile += npairs) {
-                const TileCoord tc = tile_coords(tb, G, tile);
-                int tstart, ntok;
-                token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
-                const int half = ((ntok + 15) & ~15) >> 1;
-                const int tok0 = tb->rowstart[tc.g] + tstart + (int)rank * half;
-                const bool small = half <= SMALL_ROWS;
-                const uint32_t tx = 2u * (A_BYTES + (small ? SMALL_ROWS : B_ROWS) * BK * 2);
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fb = leader_full + 8u * (uint32_t)stage;
-                    uint8_t* sa = ring + stage * STAGE_BYTES;
-                    uint8_t* sb = sa + A_BYTES;
+            if (gather) {
+                tma_prefetch_desc(&tmXg);
+            } else {
+                tma_prefetch_desc(&tmX);
+                tma_prefetch_desc(&tmXs);
+            }
+        }
+        const uint32_t leader_full = mapa_shared(smem_u32(&ctl->full[0]), 0);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true, issued_any = false;
+        for (int tile = pair; tile < total && ok; tile += npairs) {
+            const TileCoord tc = tile_coords(tb, G, tile);
+            int tstart, ntok;
+            token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
+            const int half = ((ntok + 15) & ~15) >> 1;
+            const int row0 = tb->rowstart[tc.g] + tstart;  // first row of the tile
+            const int tok0 = row0 + (int)rank * half;      // first row of this CTA's half
+            int src[4] = {0, 0, 0, 0};
+            if (gather) {  // this lane's four rows; rows past the tile's tokens repeat its first row
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int jr = (int)rank * half + 4 * lane + j;
+                    src[j] = p.gather[row0 + (jr < ntok ? jr : 0)] / p.gather_div;
+                }
+            }
+            const bool small = !gather && half <= SMALL_ROWS;
+            const uint32_t brows = gather ? (uint32_t)half : (uint32_t)(small ? SMALL_ROWS : B_ROWS);
+            const uint32_t tx = 2u * ((uint32_t)A_BYTES + brows * BK * 2);
+            for (int kb = 0; kb < p.k_blocks; ++kb) {
+                int got = 1;
+                if (lane == 0) got = mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, p.status) ? 1 : 0;
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = leader_full + 8u * (uint32_t)stage;
+                uint8_t* sa = ring + stage * STAGE_BYTES;
+                uint8_t* sb = sa + A_BYTES;
+                if (lane == 0) {
                     if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], tx);
                     if (UP) {
                         const int wrow = tc.g * p.w_rows + tc.ft * 128 + (int)rank * 64;
@@ -259,18 +284,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                         tma_load_3d_pair(sa, &tmW0, fb, kk - seg * p.kseg, tc.ft * 256 + (int)rank * 128,
                                          tc.g * p.nseg + seg, kEvictNormal);
                     }
-                    tma_load_2d_pair(sb, small ? &tmXs : &tmX, fb, kb * BK, tok0, kEvictNormal);
-                    issued_any = true;
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    if (!gather) tma_load_2d_pair(sb, small ? &tmXs : &tmX, fb, kb * BK, tok0, kEvictNormal);
+                }
+                if (gather && 4 * lane < half)
+                    tma_gather4_pair(sb + 4 * lane * BK * 2, &tmXg, fb, kb * BK, src[0], src[1], src[2], src[3],
+                                     kEvictNormal);
+                issued_any = true;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
-            if (!ok && issued_any) {  // let copies already in flight land before the CTA exits
-                const uint64_t t0 = globaltimer_ns();
-                while (globaltimer_ns() - t0 < 200000ull) {
-                }
+        }
+        if (!ok && issued_any && lane == 0) {  // let copies already in flight land before the CTA exits
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < 200000ull) {
             }
         }
         __syncwarp();
@@ -406,12 +434,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 
 template <bool UP>
 cudaError_t launch(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x, const CUtensorMap& xs,
-                   const Params& p, int num_sms, cudaStream_t st) {
+                   const CUtensorMap& xg, const Params& p, int num_sms, cudaStream_t st) {
     auto kern = tc_grouped_gemm_kernel<UP>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;  // whole CTA pairs, one CTA per SM
-    kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(w0, w1, x, xs, p);
+    kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(w0, w1, x, xs, xg, p);
     note_launches(1);
     return cudaGetLastError();
 }
@@ -420,10 +448,11 @@ cudaError_t launch(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorM
 
 cudaError_t launch_tc_up(const TcUpArgs& a, int* status, int num_sms, cudaStream_t st) {
     if (a.G <= 0 || a.G > kMaxGroups || a.d % BK != 0 || a.I % 128 != 0) return cudaErrorInvalidValue;
-    CUtensorMap tW1, tW3, tX, tXs;
+    CUtensorMap tW1, tW3, tX, tXs, tXg;
     if (!make_tmap_2d(&tW1, a.W1, a.d, a.W_rows, a.d, BK, 64) || !make_tmap_2d(&tW3, a.W3, a.d, a.W_rows, a.d, BK, 64) ||
         !make_tmap_2d(&tX, a.A, a.d, a.A_rows, a.d, BK, B_ROWS) ||
-        !make_tmap_2d(&tXs, a.A, a.d, a.A_rows, a.d, BK, SMALL_ROWS))
+        !make_tmap_2d(&tXs, a.A, a.d, a.A_rows, a.d, BK, SMALL_ROWS) ||
+        !make_tmap_2d(&tXg, a.A, a.d, a.A_rows, a.d, BK, 1))  // one-row box for tile::gather4
         return cudaErrorInvalidValue;
     Params p{};
     p.offsets = a.offsets;
@@ -437,9 +466,11 @@ cudaError_t launch_tc_up(const TcUpArgs& a, int* status, int num_sms, cudaStream
     p.out = a.H;
     p.ldo = a.I;
     p.f_limit = a.I;
-    p.a_rows = a.A_rows;
+    p.a_rows = a.gather ? a.gather_rows : a.A_rows;
+    p.gather = a.gather;
+    p.gather_div = a.gather_div > 0 ? a.gather_div : 1;
     p.status = status;
-    return launch<true>(tW1, tW3, tX, tXs, p, num_sms, st);
+    return launch<true>(tW1, tW3, tX, tXs, tXg, p, num_sms, st);
 }
 
 cudaError_t launch_tc_down(const TcDownArgs& a, int* status, int num_sms, cudaStream_t st) {
@@ -463,8 +494,10 @@ cudaError_t launch_tc_down(const TcDownArgs& a, int* status, int num_sms, cudaSt
     p.ldo = a.d;
     p.f_limit = a.d;
     p.a_rows = a.H_rows;
+    p.gather = nullptr;
+    p.gather_div = 1;
     p.status = status;
-    return launch<false>(tW2, tW2, tX, tXs, p, num_sms, st);
+    return launch<false>(tW2, tW2, tX, tXs, tXs, p, num_sms, st);
 }
 
 }  // namespace moe

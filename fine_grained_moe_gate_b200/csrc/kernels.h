@@ -36,6 +36,8 @@ struct GemmArgs {
     const int32_t* offsets;
     int G;
     int M;
+    const int32_t* gather;  // optional: A row of group row r is gather[r] / gather_div
+    int gather_div;
 };
 
 // router.cu
@@ -67,6 +69,9 @@ cudaError_t launch_simt_gemm(const GemmArgs& p, bool bf16, bool swiglu, int num_
 struct TcUpArgs {
     const void* A;          // [A_rows][d] bf16
     long long A_rows;
+    const int32_t* gather;  // optional: group row r reads A row gather[r] / gather_div (A = x, unpermuted)
+    int gather_div;
+    long long gather_rows;  // rows the groups index when gathering (T * k)
     const void* W1;         // [G * I][d] bf16 (groups stacked)
     const void* W3;
     long long W_rows;       // G * I

@@ -118,6 +118,7 @@ MOE_API moe_status moe_load_and_bias_update(const int32_t* counts, moe_shape sh,
  *   perm_tok[row]    = t*k + j, the assignment held by that row int32 [T*k]
  *   inv_row[t*k + j] = row                                     int32 [T*k]
  *   x_perm[row]      = x[t]                                    [T*k][d] dtype
+ *                      (x_perm may be NULL: only the index outputs)
  * counts: the histogram from moe_route; it is cross-checked on the device
  * (MOE_ERR_DEVICE_CHECK via moe_get_last_error on a mismatch).
  * Out-of-range expert indices are reported the same way and skipped.
@@ -181,14 +182,19 @@ MOE_API size_t moe_grouped_swiglu_workspace_size(moe_shape sh);
  *               [S][Is][d], W2 = Ws2 [S][d][Is], h [T][S*Is] (shared expert s
  *               in columns [s*Is, (s+1)*Is)), y = shared_out [T][d] = the
  *               sum over the S shared experts.
+ * gather_idx (MOE_ROUTED only, may be NULL): when given, `a` is the
+ *   unpermuted x [T][d] and row r reads x[gather_idx[r] / k] -- pass
+ *   moe_permute's perm_tok to skip the x_perm copy (saves T*k*d elements
+ *   of memory; on B200 the row gather in the GEMM's loads is slower than
+ *   the copy, so moe_layer_forward copies).
  *   up:   h[r] = silu(a[r] . W1_g^T) * (a[r] . W3_g^T)   stored once in dtype
  *   down: y[r] = h[r] . W2_g^T                            fp32 accumulate
  * Same sources as moe_grouped_swiglu.  Invalid for MOE_SHARED when S == 0.
  * -------------------------------------------------------------------------*/
 typedef enum { MOE_ROUTED = 0, MOE_SHARED = 1 } moe_expert_set;
 
-MOE_API moe_status moe_expert_up(const void* a, const int32_t* offsets, const void* w1, const void* w3, moe_shape sh,
-                                 int32_t set, void* h, void* stream);
+MOE_API moe_status moe_expert_up(const void* a, const int32_t* gather_idx, const int32_t* offsets, const void* w1,
+                                 const void* w3, moe_shape sh, int32_t set, void* h, void* stream);
 MOE_API moe_status moe_expert_down(const void* h, const int32_t* offsets, const void* w2, moe_shape sh, int32_t set,
                                    void* y, void* stream);
 

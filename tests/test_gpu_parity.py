@@ -353,3 +353,24 @@ def test_layer_is_deterministic():
         assert torch.equal(u.view(torch.uint8) if u.dtype != torch.int32 else u,
                            v.view(torch.uint8) if v.dtype != torch.int32 else v)
     check_status()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_expert_up_gather_equals_permuted_rows(dtype):
+    """moe_expert_up reading token rows through perm_tok (no x_perm copy)
+    gives the same h, bit for bit, as reading the permuted copy."""
+    cfg = V3.scaled(T=700, d=256 if dtype == "bf16" else 96, E=16, k=4, I=256 if dtype == "bf16" else 40, S=0,
+                    dtype=dtype, w_std=0.05)
+    sh = moe.shape_of(cfg)
+    p = make_layer(cfg, DEV)
+    x = make_tokens(cfg, DEV)
+    idx, w, counts, _ = route(sh, x, p["w_gate"], p["bias"], with_aff=False)
+    x_perm, offsets, perm, inv = permute(sh, x, idx, counts)
+    h1 = torch.empty((cfg.T * cfg.k, cfg.I), dtype=x.dtype, device=DEV)
+    h2 = torch.empty_like(h1)
+    moe.moe_expert_up(x_perm, None, offsets, p["w1"], p["w3"], sh, moe.MOE_ROUTED, h1)
+    moe.moe_expert_up(x, perm, offsets, p["w1"], p["w3"], sh, moe.MOE_ROUTED, h2)
+    torch.cuda.synchronize()
+    check_status()
+    bits = torch.int16 if dtype == "bf16" else torch.int32
+    assert torch.equal(h1.view(bits), h2.view(bits))
