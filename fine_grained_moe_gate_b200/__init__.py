@@ -32,7 +32,8 @@ EXPORTS = (
     "moe_route", "moe_load_and_bias_update", "moe_permute", "moe_permute_workspace_size", "moe_permute_noalloc",
     "moe_grouped_swiglu",
     "moe_grouped_swiglu_workspace_size", "moe_expert_up", "moe_expert_down", "moe_combine", "moe_layer_forward",
-    "moe_workspace_size", "moe_get_last_error", "moe_kernel_launch_count", "moe_status_string", "moe_abi_version",
+    "moe_workspace_size", "moe_get_last_error", "moe_kernel_launch_count", "moe_selftest_bounded_wait",
+    "moe_status_string", "moe_abi_version",
 )
 
 MOE_ROUTED, MOE_SHARED = 0, 1
@@ -81,6 +82,7 @@ def lib() -> ctypes.CDLL:
             "moe_combine": [P, P, P, P, S, P, P],
             "moe_layer_forward": [P, P, P, P, P, P, P, P, P, S, P, P, P, P, P, sz, P],
             "moe_get_last_error": [P],
+            "moe_selftest_bounded_wait": [ctypes.c_uint32, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -195,6 +197,10 @@ def moe_grouped_swiglu_workspace_size(shape) -> int:
 
 def moe_get_last_error(stream=None) -> int:
     return lib().moe_get_last_error(_stream(stream))
+
+
+def moe_selftest_bounded_wait(limit_us: int, stream=None):
+    _check(lib().moe_selftest_bounded_wait(limit_us, _stream(stream)), "moe_selftest_bounded_wait")
 
 
 def moe_kernel_launch_count() -> int:

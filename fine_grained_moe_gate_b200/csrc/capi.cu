@@ -392,6 +392,18 @@ moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bia
                : MOE_ERR_CUDA;
 }
 
+moe_status moe_selftest_bounded_wait(uint32_t limit_us, void* stream) {
+    MOE_REQUIRE(limit_us > 0 && limit_us <= 5000000u, MOE_ERR_INVALID_ARG);
+    int dev, sms;
+    int* status;
+    moe_status v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return moe::launch_bounded_wait_selftest((uint64_t)limit_us * 1000ull, status,
+                                             static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
 moe_status moe_get_last_error(void* stream) {
     int dev, sms;
     int* status;

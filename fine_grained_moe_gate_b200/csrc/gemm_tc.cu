@@ -63,6 +63,13 @@ constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
 constexpr int NTHREADS = 192;
 constexpr int XS = 132;                 // row stride (floats) of the epilogue exchange buffer
 constexpr int XBUF_BYTES = 16 * XS * 4; // 16 tokens x 128 lanes (+pad), fp32
+// L2 policy of the two operands' loads.  Marking the weights evict-first
+// (each weight box is read by at most two clusters) and the token rows
+// evict-last (re-read by every feature tile of the expert) measured 3.5%
+// slower on the V3 step than the normal policy for both.
+constexpr uint64_t W_HINT = kEvictNormal;
+constexpr uint64_t X_HINT = kEvictNormal;
+
 
 struct Ctl {
     uint64_t full[STAGES];
@@ -276,19 +283,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], tx);
                     if (UP) {
                         const int wrow = tc.g * p.w_rows + tc.ft * 128 + (int)rank * 64;
-                        tma_load_2d_pair(sa, &tmW0, fb, kb * BK, wrow, kEvictNormal);
-                        tma_load_2d_pair(sa + A_BYTES / 2, &tmW1, fb, kb * BK, wrow, kEvictNormal);
+                        tma_load_2d_pair(sa, &tmW0, fb, kb * BK, wrow, W_HINT);
+                        tma_load_2d_pair(sa + A_BYTES / 2, &tmW1, fb, kb * BK, wrow, W_HINT);
                     } else {
                         const int kk = kb * BK;
                         const int seg = kk / p.kseg;
                         tma_load_3d_pair(sa, &tmW0, fb, kk - seg * p.kseg, tc.ft * 256 + (int)rank * 128,
-                                         tc.g * p.nseg + seg, kEvictNormal);
+                                         tc.g * p.nseg + seg, W_HINT);
                     }
-                    if (!gather) tma_load_2d_pair(sb, small ? &tmXs : &tmX, fb, kb * BK, tok0, kEvictNormal);
+                    if (!gather) tma_load_2d_pair(sb, small ? &tmXs : &tmX, fb, kb * BK, tok0, X_HINT);
                 }
                 if (gather && 4 * lane < half)
                     tma_gather4_pair(sb + 4 * lane * BK * 2, &tmXg, fb, kb * BK, src[0], src[1], src[2], src[3],
-                                     kEvictNormal);
+                                     X_HINT);
                 issued_any = true;
                 if (++stage == STAGES) {
                     stage = 0;
@@ -370,14 +377,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, p.status)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACC_COLS;
+            // TMEM reads run one 16-token chunk ahead of the exchange below
+            uint32_t r[16];
+            tmem_ld16(taddr, r);
 #pragma unroll 1
             for (int c = 0; c < ntok; c += 16) {
-                uint32_t r[16];
-                tmem_ld16(taddr + (uint32_t)c, r);
                 tmem_ld_wait();
+                float v16[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v16[i] = __uint_as_float(r[i]);
+                if (c + 16 < ntok) tmem_ld16(taddr + (uint32_t)(c + 16), r);
                 float* xs = xbuf + xb * (XBUF_BYTES / 4);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) xs[i * XS + q * 32 + lane] = __uint_as_float(r[i]);
+                for (int i = 0; i < 16; ++i) xs[i * XS + q * 32 + lane] = v16[i];
                 named_bar_sync(1, 128);
                 const bool tok_ok = c + my_tok < ntok;
                 const float* row = xs + my_tok * XS;

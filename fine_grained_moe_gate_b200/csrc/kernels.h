@@ -96,6 +96,9 @@ struct TcDownArgs {
 cudaError_t launch_tc_up(const TcUpArgs& a, int* status, int num_sms, cudaStream_t st);
 cudaError_t launch_tc_down(const TcDownArgs& a, int* status, int num_sms, cudaStream_t st);
 
+// selftest.cu
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int* status, cudaStream_t st);
+
 // combine.cu
 cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* inv_row, const void* shared, int T,
                            int d, int k, bool bf16, void* y, int* status, cudaStream_t st);

@@ -226,6 +226,14 @@ MOE_API size_t moe_workspace_size(moe_shape sh);
  * status word (MOE_OK if no kernel reported an anomaly). */
 MOE_API moe_status moe_get_last_error(void* stream);
 
+/* Failure-detection self-test (no counterpart in the pages): launches one
+ * kernel that waits, with the same bounded mbarrier wait the pipelined
+ * kernels use, on a barrier nothing arrives on.  After limit_us
+ * microseconds (1 .. 5e6) the wait gives up and records MOE_ERR_TIMEOUT in
+ * the device status word, which moe_get_last_error then returns; the
+ * context stays usable.  Returns MOE_OK when the kernel was launched. */
+MOE_API moe_status moe_selftest_bounded_wait(uint32_t limit_us, void* stream);
+
 /* Number of CUDA kernels this library has launched in this process (all
  * devices, all streams); a tracing aid, e.g. to count the kernels of one
  * step.  Host-side counter, no synchronisation. */

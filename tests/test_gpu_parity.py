@@ -374,3 +374,23 @@ def test_expert_up_gather_equals_permuted_rows(dtype):
     check_status()
     bits = torch.int16 if dtype == "bf16" else torch.int32
     assert torch.equal(h1.view(bits), h2.view(bits))
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """Failure detection without a fault: a device wait that nothing ends
+    gives up after its limit, reports MOE_ERR_TIMEOUT through the status
+    word, and the next layer call runs normally."""
+    import time
+    t0 = time.perf_counter()
+    moe.moe_selftest_bounded_wait(50_000)          # 50 ms limit
+    assert moe.moe_get_last_error() == 7           # MOE_ERR_TIMEOUT (read and cleared)
+    assert time.perf_counter() - t0 < 5.0
+    assert moe.moe_get_last_error() == 0
+    cfg = SMALL.scaled(T=128, d=256, E=16, k=2, I=128, S=1, Is=128)
+    sh = moe.shape_of(cfg)
+    p = make_layer(cfg, DEV)
+    x = make_tokens(cfg, DEV)
+    y, idx, w, counts = layer_forward(sh, p, x)
+    check_status()
+    assert int(counts.sum()) == cfg.T * cfg.k
+    assert torch.isfinite(y.float()).all()
