@@ -6,7 +6,8 @@
 One step = one pass of the whole hot path over one batch held in HBM:
 gate GEMM + sigmoid + bias-shifted top-k + weights + load histogram
 (moe_route), expert-contiguous permutation (moe_permute), the routed and
-shared grouped SwiGLU GEMMs (moe_expert_up / moe_expert_down), the weighted
+shared grouped SwiGLU GEMMs (moe_ffn_up / moe_ffn_down: one launch each for
+both expert sets), the weighted
 combine (moe_combine) and the bias update at the end of the step
 (moe_load_and_bias_update; with N > 1 the counts are first summed over the
 ranks with an NCCL all-reduce -- the one exchange the method has).  Each rank
@@ -44,8 +45,8 @@ if ROOT not in sys.path:
 
 METRIC = "MoE layer fwd tokens/s (V3-shaped, bf16) and % of BF16 tensor / HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-STAGES = ["route", "permute", "up_routed", "up_shared", "down_routed", "down_shared", "combine", "bias_update"]
-DOMINANT = "up_routed"
+STAGES = ["route", "permute", "ffn_up", "ffn_down", "combine", "bias_update"]
+DOMINANT = "ffn_up"
 
 
 def parse_args():
@@ -261,21 +262,16 @@ def run_ours(args, world, rank, local):
         rec(1)
         moe.moe_permute(x, idx, counts, sh, x_perm, offsets, perm, inv, pws, stream)
         rec(2)
-        moe.moe_expert_up(x_perm, None, offsets, p["w1"], p["w3"], sh, moe.MOE_ROUTED, h, stream)
+        xs_ = x if cfg.S > 0 else None
+        moe.moe_ffn_up(x_perm, offsets, p["w1"], p["w3"], xs_, p["ws1"], p["ws3"], sh, h, hs, stream)
         rec(3)
-        if cfg.S > 0:
-            moe.moe_expert_up(x, None, None, p["ws1"], p["ws3"], sh, moe.MOE_SHARED, hs, stream)
+        moe.moe_ffn_down(h, offsets, p["w2"], hs if cfg.S > 0 else None, p["ws2"], sh, x_perm, shared_out, stream)
         rec(4)
-        moe.moe_expert_down(h, offsets, p["w2"], sh, moe.MOE_ROUTED, x_perm, stream)
-        rec(5)
-        if cfg.S > 0:
-            moe.moe_expert_down(hs, None, p["ws2"], sh, moe.MOE_SHARED, shared_out, stream)
-        rec(6)
         moe.moe_combine(x_perm, w, inv, shared_out, sh, y, stream)
-        rec(7)
+        rec(5)
         mdist.allreduce_counts(counts)
         moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
-        rec(8)
+        rec(6)
 
     def barrier():
         if world > 1:
@@ -293,7 +289,7 @@ def run_ours(args, world, rank, local):
     if vis:
         gpu_id = vis.split(",")[local].strip()
     clocks = ClockSampler(gpu_id)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     clocks.start()
@@ -355,37 +351,38 @@ def run_ours(args, world, rank, local):
         if st != 0:
             raise moe.MoEError(st, "e2e steps")
 
-    # ---- roofline of the dominant kernel (routed gate/up grouped GEMM)
+    # ---- roofline of the dominant kernel (gate/up grouped GEMM, routed + shared sets)
     peaks, peak_src = load_peaks()
-    flops_per_launch = T * k * 4 * d * cfg.I   # gate + up, real rows only
+    SIs = cfg.S * cfg.Is
+    flops_per_launch = T * k * 4 * d * cfg.I + T * 4 * d * SIs   # gate + up, real rows only
     dom_ms = stage_ms[DOMINANT]
     achieved = flops_per_launch / (dom_ms / 1e3) / 1e12
-    # algorithmic bytes of that launch: W1 + W3 of the experts that got rows
-    # (counted by routing each input once more, outside the timed region),
-    # the token rows read and h written
+    # algorithmic bytes of that launch: W1 + W3 of the routed experts that got
+    # rows (counted by routing each input once more, outside the timed region)
+    # and of the shared experts, the token rows read and h written
     touched = []
     for xx in xs:
         moe.moe_route(xx, p["w_gate"], p["bias"], sh, idx, w, counts, None, stream)
         touched.append(int((counts > 0).sum().item()))
     n_touched = statistics.mean(touched)
     esz = 2 if cfg.dtype == "bf16" else 4
-    bytes_per_launch = n_touched * 2 * cfg.I * d * esz + T * k * (d + cfg.I) * esz
+    bytes_per_launch = (n_touched * 2 * cfg.I * d + T * k * (d + cfg.I) + 2 * SIs * d + T * (d + SIs)) * esz
     hbm_gbs = bytes_per_launch / (dom_ms / 1e3) / 1e9
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    roof_hbm = {"bound": "hbm", "kernel": "routed up projection", "achieved": round(hbm_gbs, 1), "peak": hbm_peak,
+    roof_hbm = {"bound": "hbm", "kernel": "gate/up projection (routed + shared)", "achieved": round(hbm_gbs, 1), "peak": hbm_peak,
                 "unit": "GB/s", "frac": round(hbm_gbs / hbm_peak, 4),
                 "frac_of_nominal_8000": round(hbm_gbs / 8000.0, 4),
                 "traffic": None, "bytes_per_launch": int(bytes_per_launch), "experts_touched": n_touched,
                 "peak_kind": f"hbm_gbs ({peak_src}, copy bandwidth)"}
     if cfg.dtype == "bf16":
         peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-        roof = {"bound": "tensor", "kernel": "tc_grouped_gemm_kernel<up> (routed experts, SwiGLU epilogue)",
+        roof = {"bound": "tensor", "kernel": "tc_grouped_gemm_kernel<up> (routed + shared experts, SwiGLU epilogue)",
                 "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "traffic": traffic_record(os.path.join(ROOT, "fine_grained_moe_gate_b200", "csrc", "gemm_tc.cu")),
                 "peak_kind": f"bf16_tflops_sustained ({peak_src}): the kernel is timed inside a long step",
                 "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
     else:
-        roof = {"bound": "alu", "kernel": "simt_grouped_gemm_kernel (fp32 FFMA)", "achieved": round(achieved, 3),
+        roof = {"bound": "alu", "kernel": "simt_grouped_gemm_kernel (fp32 FFMA; routed and shared launches)", "achieved": round(achieved, 3),
                 "peak": None, "unit": "TFLOP/s", "frac": None, "traffic": None,
                 "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
     if cfg.name.startswith("v3_decode"):

@@ -30,10 +30,9 @@ STATUS = {
 
 EXPORTS = (
     "moe_route", "moe_load_and_bias_update", "moe_permute", "moe_permute_workspace_size", "moe_permute_noalloc",
-    "moe_grouped_swiglu",
-    "moe_grouped_swiglu_workspace_size", "moe_expert_up", "moe_expert_down", "moe_combine", "moe_layer_forward",
-    "moe_workspace_size", "moe_get_last_error", "moe_kernel_launch_count", "moe_selftest_bounded_wait",
-    "moe_status_string", "moe_abi_version",
+    "moe_grouped_swiglu", "moe_grouped_swiglu_workspace_size", "moe_expert_up", "moe_expert_down", "moe_ffn_up",
+    "moe_ffn_down", "moe_combine", "moe_layer_forward", "moe_workspace_size", "moe_get_last_error",
+    "moe_kernel_launch_count", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
 )
 
 MOE_ROUTED, MOE_SHARED = 0, 1
@@ -79,6 +78,8 @@ def lib() -> ctypes.CDLL:
             "moe_grouped_swiglu": [P, P, P, P, P, P, P, P, P, S, P, P, P, sz, P],
             "moe_expert_up": [P, P, P, P, P, S, ctypes.c_int32, P, P],
             "moe_expert_down": [P, P, P, S, ctypes.c_int32, P, P],
+            "moe_ffn_up": [P, P, P, P, P, P, P, S, P, P, P],
+            "moe_ffn_down": [P, P, P, P, P, S, P, P, P],
             "moe_combine": [P, P, P, P, S, P, P],
             "moe_layer_forward": [P, P, P, P, P, P, P, P, P, S, P, P, P, P, P, sz, P],
             "moe_get_last_error": [P],
@@ -169,6 +170,16 @@ def moe_expert_up(a, gather_idx, offsets, w1, w3, shape, expert_set, h, stream=N
 def moe_expert_down(h, offsets, w2, shape, expert_set, y, stream=None):
     _check(lib().moe_expert_down(_p(h), _p(offsets), _p(w2), shape, expert_set, _p(y), _stream(stream)),
            "moe_expert_down")
+
+
+def moe_ffn_up(x_perm, offsets, w1, w3, x, ws1, ws3, shape, h, hs, stream=None):
+    _check(lib().moe_ffn_up(_p(x_perm), _p(offsets), _p(w1), _p(w3), _p(x), _p(ws1), _p(ws3), shape, _p(h), _p(hs),
+                            _stream(stream)), "moe_ffn_up")
+
+
+def moe_ffn_down(h, offsets, w2, hs, ws2, shape, y_perm, shared_out, stream=None):
+    _check(lib().moe_ffn_down(_p(h), _p(offsets), _p(w2), _p(hs), _p(ws2), shape, _p(y_perm), _p(shared_out),
+                              _stream(stream)), "moe_ffn_down")
 
 
 def moe_combine(y_perm, topk_w, inv_row, shared_out, shape, y, stream=None):

@@ -96,6 +96,27 @@ moe_status do_permute(const void* x, const int32_t* idx, const int32_t* counts, 
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Tensor-core argument blocks of one expert set: the routed set has a group
+// per expert (rows from offsets), the shared set is one group of T rows whose
+// S weight blocks are stacked into one [S*Is][d] matrix.
+moe::TcUpArgs tc_up_args(const void* a, const int32_t* gather, const int32_t* offsets, const void* w1,
+                         const void* w3, const moe_shape& sh, bool shared, void* h) {
+    const long long rows = shared ? sh.T : (long long)sh.T * sh.k;
+    const int Ig = shared ? sh.S * sh.Is : sh.I;
+    if (shared) gather = nullptr;
+    return moe::TcUpArgs{a, gather ? sh.T : rows, gather, sh.k, rows, w1, w3,
+                         shared ? (long long)Ig : (long long)sh.E * sh.I, h, sh.d, Ig, shared ? nullptr : offsets,
+                         shared ? 1 : sh.E, shared ? sh.T : 0};
+}
+
+moe::TcDownArgs tc_down_args(const void* h, const int32_t* offsets, const void* w2, const moe_shape& sh, bool shared,
+                             void* y) {
+    const long long rows = shared ? sh.T : (long long)sh.T * sh.k;
+    return moe::TcDownArgs{h, rows, w2, shared ? sh.S : 1, shared ? sh.Is : sh.I, y, sh.d,
+                           shared ? sh.S * sh.Is : sh.I, shared ? nullptr : offsets, shared ? 1 : sh.E,
+                           shared ? sh.T : 0};
+}
+
 // gather (routed set only, may be null): group row r reads row gather[r] / k
 // of `a` (= x, unpermuted); without it `a` is x_perm itself.
 moe_status do_expert_up(const void* a, const int32_t* gather, const int32_t* offsets, const void* w1, const void* w3,
@@ -104,12 +125,10 @@ moe_status do_expert_up(const void* a, const int32_t* gather, const int32_t* off
     const long long rows = shared ? sh.T : (long long)sh.T * sh.k;  // rows the groups index (= rows of h)
     const int Ig = shared ? sh.S * sh.Is : sh.I;  // S stacked [Is][d] blocks = one [S*Is][d] matrix
     if (shared) gather = nullptr;
-    const long long a_rows = gather ? sh.T : rows;
     cudaError_t err;
     if (sh.dtype == MOE_BF16) {
-        moe::TcUpArgs up{a, a_rows, gather, sh.k, rows, w1, w3, shared ? (long long)Ig : (long long)sh.E * sh.I, h,
-                         sh.d, Ig, shared ? nullptr : offsets, shared ? 1 : sh.E, shared ? sh.T : 0};
-        err = moe::launch_tc_up(up, status, sms, st);
+        const moe::TcUpArgs up = tc_up_args(a, gather, offsets, w1, w3, sh, shared, h);
+        err = moe::launch_tc_up(shared ? nullptr : &up, shared ? &up : nullptr, status, sms, st);
     } else {
         moe::GemmArgs up{a, sh.d, w1, w3, shared ? 0 : (long long)sh.I * sh.d, sh.d, sh.d, 0, h, Ig, Ig, sh.d,
                          shared ? nullptr : offsets, shared ? 1 : sh.E, (int)rows, gather, sh.k};
@@ -126,9 +145,8 @@ moe_status do_expert_down(const void* h, const int32_t* offsets, const void* w2,
     const int K = shared ? sh.S * sh.Is : sh.I;
     cudaError_t err;
     if (sh.dtype == MOE_BF16) {
-        moe::TcDownArgs dn{h, rows, w2, shared ? sh.S : 1, kseg, y, sh.d, K, shared ? nullptr : offsets,
-                           shared ? 1 : sh.E, shared ? sh.T : 0};
-        err = moe::launch_tc_down(dn, status, sms, st);
+        const moe::TcDownArgs dn = tc_down_args(h, offsets, w2, sh, shared, y);
+        err = moe::launch_tc_down(shared ? nullptr : &dn, shared ? &dn : nullptr, status, sms, st);
     } else {
         // element (n, kk) of W2 block g: (kk / kseg) * d * kseg + n * kseg + kk % kseg
         moe::GemmArgs dn{h, K, w2, nullptr, shared ? 0 : (long long)sh.d * sh.I, kseg, kseg,
@@ -139,6 +157,38 @@ moe_status do_expert_down(const void* h, const int32_t* offsets, const void* w2,
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Both expert sets, one launch per projection on the tensor-core path.
+moe_status do_ffn_up(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3, const void* x,
+                     const void* ws1, const void* ws3, const moe_shape& sh, void* h, void* hs, int* status, int sms,
+                     cudaStream_t st) {
+    if (sh.T == 0) return MOE_OK;
+    const bool shared = x && sh.S > 0;
+    if (sh.dtype == MOE_BF16) {
+        const moe::TcUpArgs ur = tc_up_args(x_perm, nullptr, offsets, w1, w3, sh, false, h);
+        const moe::TcUpArgs us = tc_up_args(x, nullptr, nullptr, ws1, ws3, sh, true, hs);
+        return moe::launch_tc_up(&ur, shared ? &us : nullptr, status, sms, st) == cudaSuccess ? MOE_OK
+                                                                                                : MOE_ERR_CUDA;
+    }
+    moe_status v = do_expert_up(x_perm, nullptr, offsets, w1, w3, sh, false, h, status, sms, st);
+    if (v == MOE_OK && shared) v = do_expert_up(x, nullptr, nullptr, ws1, ws3, sh, true, hs, status, sms, st);
+    return v;
+}
+
+moe_status do_ffn_down(const void* h, const int32_t* offsets, const void* w2, const void* hs, const void* ws2,
+                       const moe_shape& sh, void* y_perm, void* shared_out, int* status, int sms, cudaStream_t st) {
+    if (sh.T == 0) return MOE_OK;
+    const bool shared = hs && sh.S > 0;
+    if (sh.dtype == MOE_BF16) {
+        const moe::TcDownArgs dr = tc_down_args(h, offsets, w2, sh, false, y_perm);
+        const moe::TcDownArgs ds = tc_down_args(hs, nullptr, ws2, sh, true, shared_out);
+        return moe::launch_tc_down(&dr, shared ? &ds : nullptr, status, sms, st) == cudaSuccess ? MOE_OK
+                                                                                                  : MOE_ERR_CUDA;
+    }
+    moe_status v = do_expert_down(h, offsets, w2, sh, false, y_perm, status, sms, st);
+    if (v == MOE_OK && shared) v = do_expert_down(hs, nullptr, ws2, sh, true, shared_out, status, sms, st);
+    return v;
+}
+
 moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3, const void* w2,
                      const void* x, const void* ws1, const void* ws3, const void* ws2, const moe_shape& sh,
                      void* y_perm, void* shared_out, void* ws, int* status, int sms, cudaStream_t st) {
@@ -147,12 +197,9 @@ moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1,
     char* h = static_cast<char*>(ws);
     char* hs = h + align256((size_t)rows * sh.I * eb);
     const bool shared = x && sh.S > 0 && shared_out;
-    moe_status v;
-    if ((v = do_expert_up(x_perm, nullptr, offsets, w1, w3, sh, false, h, status, sms, st)) != MOE_OK) return v;
-    if (shared && (v = do_expert_up(x, nullptr, nullptr, ws1, ws3, sh, true, hs, status, sms, st)) != MOE_OK) return v;
-    if ((v = do_expert_down(h, offsets, w2, sh, false, y_perm, status, sms, st)) != MOE_OK) return v;
-    if (shared && (v = do_expert_down(hs, nullptr, ws2, sh, true, shared_out, status, sms, st)) != MOE_OK) return v;
-    return MOE_OK;
+    moe_status v = do_ffn_up(x_perm, offsets, w1, w3, shared ? x : nullptr, ws1, ws3, sh, h, hs, status, sms, st);
+    if (v != MOE_OK) return v;
+    return do_ffn_down(h, offsets, w2, shared ? hs : nullptr, ws2, sh, y_perm, shared_out, status, sms, st);
 }
 
 }  // namespace
@@ -316,6 +363,44 @@ moe_status moe_expert_down(const void* h, const int32_t* offsets, const void* w2
     return do_expert_down(h, offsets, w2, sh, shared, y, status, sms, static_cast<cudaStream_t>(stream));
 }
 
+moe_status moe_ffn_up(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3, const void* x,
+                      const void* ws1, const void* ws3, moe_shape sh, void* h, void* hs, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    const bool shared = x != nullptr && sh.S > 0;
+    MOE_REQUIRE(offsets && w1 && w3, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (x_perm && h), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(!shared || (ws1 && ws3 && (sh.T == 0 || hs)), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x_perm) && aligned16(offsets) && aligned16(w1) && aligned16(w3) && aligned16(x) &&
+                    aligned16(ws1) && aligned16(ws3) && aligned16(h) && aligned16(hs),
+                MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_ffn_up(x_perm, offsets, w1, w3, shared ? x : nullptr, ws1, ws3, sh, h, hs, status, sms,
+                     static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_ffn_down(const void* h, const int32_t* offsets, const void* w2, const void* hs, const void* ws2,
+                        moe_shape sh, void* y_perm, void* shared_out, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    const bool shared = hs != nullptr && sh.S > 0;
+    MOE_REQUIRE(offsets && w2, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (h && y_perm), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(!shared || (ws2 && (sh.T == 0 || shared_out)), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(h) && aligned16(offsets) && aligned16(w2) && aligned16(hs) && aligned16(ws2) &&
+                    aligned16(y_perm) && aligned16(shared_out),
+                MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_ffn_down(h, offsets, w2, shared ? hs : nullptr, ws2, sh, y_perm, shared_out, status, sms,
+                       static_cast<cudaStream_t>(stream));
+}
+
 moe_status moe_combine(const void* y_perm, const float* topk_w, const int32_t* inv_row, const void* shared_out,
                        moe_shape sh, void* y, void* stream) {
     moe_status v = validate_shape(sh);
@@ -376,16 +461,12 @@ moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bia
     // inside the GEMM's loads, tile::gather4, measured 2x slower for the
     // routed up projection than this copy plus whole-tile loads)
     void* y_perm = x_perm;  // the down projection overwrites x_perm once the up projection has read it
-    char* h = static_cast<char*>(gws);
-    char* hs = h + align256(rows * sh.I * eb);
     if ((v = do_route(x, w_gate, bias, sh, topk_idx, topk_w, counts, nullptr, status, sms, st)) != MOE_OK) return v;
     if (sh.T == 0) return MOE_OK;
     if ((v = do_permute(x, topk_idx, counts, sh, x_perm, offsets, perm, inv, pws, status, st)) != MOE_OK) return v;
-    if ((v = do_expert_up(x_perm, nullptr, offsets, w1, w3, sh, false, h, status, sms, st)) != MOE_OK) return v;
-    if (sh.S > 0 && (v = do_expert_up(x, nullptr, nullptr, ws1, ws3, sh, true, hs, status, sms, st)) != MOE_OK)
+    if ((v = do_swiglu(x_perm, offsets, w1, w3, w2, sh.S > 0 ? x : nullptr, ws1, ws3, ws2, sh, y_perm, shared_out,
+                       gws, status, sms, st)) != MOE_OK)
         return v;
-    if ((v = do_expert_down(h, offsets, w2, sh, false, y_perm, status, sms, st)) != MOE_OK) return v;
-    if (sh.S > 0 && (v = do_expert_down(hs, nullptr, ws2, sh, true, shared_out, status, sms, st)) != MOE_OK) return v;
     return moe::launch_combine(y_perm, topk_w, inv, shared_out, sh.T, sh.d, sh.k, sh.dtype == MOE_BF16, y, status,
                                st) == cudaSuccess
                ? MOE_OK

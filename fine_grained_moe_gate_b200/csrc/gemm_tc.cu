@@ -70,7 +70,6 @@ constexpr int XBUF_BYTES = 16 * XS * 4; // 16 tokens x 128 lanes (+pad), fp32
 constexpr uint64_t W_HINT = kEvictNormal;
 constexpr uint64_t X_HINT = kEvictNormal;
 
-
 struct Ctl {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
@@ -80,18 +79,19 @@ struct Ctl {
     uint32_t tmem_base;
     int abort;
 };
+constexpr int kMaxTcGroups = kMaxGroups + 1;  // routed experts + the shared set
 struct Tables {
-    int rowstart[kMaxGroups];
-    int rows[kMaxGroups];
-    int ttiles[kMaxGroups];  // token tiles per group
-    int prefix[kMaxGroups + 1];
+    int rowstart[kMaxTcGroups];
+    int rows[kMaxTcGroups];
+    int ttiles[kMaxTcGroups];  // token tiles per group
+    int prefix[kMaxTcGroups + 1];
 };
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 2 * XBUF_BYTES + sizeof(Ctl) + sizeof(Tables);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-struct Params {
-    const int32_t* offsets;
-    int G, M;
+// One expert set in a launch: set 0 = the routed experts (groups [0, G0),
+// rows from offsets), set 1 = the shared experts (group G0, rows [0, M)).
+struct SetParams {
     int f_tiles;       // feature tiles (per CTA pair) per group
     int k_blocks;
     int w_rows;        // up: rows of W1/W3 per group (I)
@@ -99,8 +99,15 @@ struct Params {
     void* out;
     int ldo;           // output row pitch (elements)
     int f_limit;       // valid output features
-    long long a_rows;  // rows the groups index (token operand rows, or gathered rows) and output rows
-    const int32_t* gather;  // up, optional: row r of the groups reads token row gather[r] / gather_div
+    long long a_rows;  // rows the groups may index (token operand rows, or gathered rows) = output rows
+};
+struct Params {
+    const int32_t* offsets;
+    int G0;            // routed groups
+    int has_shared;    // 1: group G0 is the shared set
+    int M;             // rows of the shared set
+    SetParams set[2];
+    const int32_t* gather;  // up, routed set, optional: row r reads token row gather[r] / gather_div
     int gather_div;
     int* status;
 };
@@ -162,8 +169,10 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 
 template <bool UP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
-    tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmW1,
-                           const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXs,
+    tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW0a, const __grid_constant__ CUtensorMap tmW1a,
+                           const __grid_constant__ CUtensorMap tmXa, const __grid_constant__ CUtensorMap tmXsa,
+                           const __grid_constant__ CUtensorMap tmW0b, const __grid_constant__ CUtensorMap tmW1b,
+                           const __grid_constant__ CUtensorMap tmXb, const __grid_constant__ CUtensorMap tmXsb,
                            const __grid_constant__ CUtensorMap tmXg, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -176,13 +185,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();  // 0 = leader (issues the MMAs)
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-    const int G = p.G;
+    const int G = p.G0 + p.has_shared;
 
     for (int g = tid; g < G; g += NTHREADS) {
-        const int rs = p.offsets ? p.offsets[g] : 0;
-        const int re = p.offsets ? p.offsets[g + 1] : p.M;
+        const bool sh = g >= p.G0;
+        const int rs = sh ? 0 : p.offsets[g];
+        const int re = sh ? p.M : p.offsets[g + 1];
         int rows = re - rs;
-        if (rs < 0 || rows < 0 || (long long)re > p.a_rows) {  // corrupt offsets: skip the group
+        if (rs < 0 || rows < 0 || (long long)re > p.set[sh ? 1 : 0].a_rows) {  // corrupt offsets: skip the group
             report(p.status, kStDeviceCheck);
             rows = 0;
         }
@@ -212,7 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         int carry = 0;
         for (int b = 0; b < G; b += 32) {
             const int g = b + lane;
-            const int v = g < G ? tb->ttiles[g] * p.f_tiles : 0;
+            const int v = g < G ? tb->ttiles[g] * p.set[g >= p.G0 ? 1 : 0].f_tiles : 0;
             int incl = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -235,15 +245,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // Lane 0 waits for free stages and loads the weights; with a gather
         // index every lane also fetches four token rows (tile::gather4), so
         // the token operand is read straight from x in expert order.
-        const bool gather = UP && p.gather != nullptr;
+        const bool gather = UP && p.gather != nullptr;  // routed set only
         if (lane == 0) {
-            tma_prefetch_desc(&tmW0);
-            if (UP) tma_prefetch_desc(&tmW1);
-            if (gather) {
-                tma_prefetch_desc(&tmXg);
-            } else {
-                tma_prefetch_desc(&tmX);
-                tma_prefetch_desc(&tmXs);
+            if (p.G0 > 0) {
+                tma_prefetch_desc(&tmW0a);
+                if (UP) tma_prefetch_desc(&tmW1a);
+                tma_prefetch_desc(gather ? &tmXg : &tmXa);
+            }
+            if (p.has_shared) {
+                tma_prefetch_desc(&tmW0b);
+                if (UP) tma_prefetch_desc(&tmW1b);
+                tma_prefetch_desc(&tmXb);
             }
         }
         const uint32_t leader_full = mapa_shared(smem_u32(&ctl->full[0]), 0);
@@ -252,23 +264,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         bool ok = true, issued_any = false;
         for (int tile = pair; tile < total && ok; tile += npairs) {
             const TileCoord tc = tile_coords(tb, G, tile);
+            const int si = tc.g >= p.G0 ? 1 : 0;
+            const SetParams& sp = p.set[si];
+            const CUtensorMap* mW0 = si ? &tmW0b : &tmW0a;
+            const CUtensorMap* mW1 = si ? &tmW1b : &tmW1a;
+            const CUtensorMap* mX = si ? &tmXb : &tmXa;
+            const CUtensorMap* mXs = si ? &tmXsb : &tmXsa;
+            const int wg = si ? 0 : tc.g;  // weight block index of the group inside its set
+            const bool gat = gather && si == 0;
             int tstart, ntok;
             token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
             const int half = ((ntok + 15) & ~15) >> 1;
             const int row0 = tb->rowstart[tc.g] + tstart;  // first row of the tile
             const int tok0 = row0 + (int)rank * half;      // first row of this CTA's half
             int src[4] = {0, 0, 0, 0};
-            if (gather) {  // this lane's four rows; rows past the tile's tokens repeat its first row
+            if (gat) {  // this lane's four rows; rows past the tile's tokens repeat its first row
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int jr = (int)rank * half + 4 * lane + j;
                     src[j] = p.gather[row0 + (jr < ntok ? jr : 0)] / p.gather_div;
                 }
             }
-            const bool small = !gather && half <= SMALL_ROWS;
-            const uint32_t brows = gather ? (uint32_t)half : (uint32_t)(small ? SMALL_ROWS : B_ROWS);
+            const bool small = !gat && half <= SMALL_ROWS;
+            const uint32_t brows = gat ? (uint32_t)half : (uint32_t)(small ? SMALL_ROWS : B_ROWS);
             const uint32_t tx = 2u * ((uint32_t)A_BYTES + brows * BK * 2);
-            for (int kb = 0; kb < p.k_blocks; ++kb) {
+            for (int kb = 0; kb < sp.k_blocks; ++kb) {
                 int got = 1;
                 if (lane == 0) got = mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, p.status) ? 1 : 0;
                 got = __shfl_sync(0xffffffffu, got, 0);
@@ -282,18 +302,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 if (lane == 0) {
                     if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], tx);
                     if (UP) {
-                        const int wrow = tc.g * p.w_rows + tc.ft * 128 + (int)rank * 64;
-                        tma_load_2d_pair(sa, &tmW0, fb, kb * BK, wrow, W_HINT);
-                        tma_load_2d_pair(sa + A_BYTES / 2, &tmW1, fb, kb * BK, wrow, W_HINT);
+                        const int wrow = wg * sp.w_rows + tc.ft * 128 + (int)rank * 64;
+                        tma_load_2d_pair(sa, mW0, fb, kb * BK, wrow, W_HINT);
+                        tma_load_2d_pair(sa + A_BYTES / 2, mW1, fb, kb * BK, wrow, W_HINT);
                     } else {
                         const int kk = kb * BK;
-                        const int seg = kk / p.kseg;
-                        tma_load_3d_pair(sa, &tmW0, fb, kk - seg * p.kseg, tc.ft * 256 + (int)rank * 128,
-                                         tc.g * p.nseg + seg, W_HINT);
+                        const int seg = kk / sp.kseg;
+                        tma_load_3d_pair(sa, mW0, fb, kk - seg * sp.kseg, tc.ft * 256 + (int)rank * 128,
+                                         wg * sp.nseg + seg, W_HINT);
                     }
-                    if (!gather) tma_load_2d_pair(sb, small ? &tmXs : &tmX, fb, kb * BK, tok0, X_HINT);
+                    if (!gat) tma_load_2d_pair(sb, small ? mXs : mX, fb, kb * BK, tok0, X_HINT);
                 }
-                if (gather && 4 * lane < half)
+                if (gat && 4 * lane < half)
                     tma_gather4_pair(sb + 4 * lane * BK * 2, &tmXg, fb, kb * BK, src[0], src[1], src[2], src[3],
                                      X_HINT);
                 issued_any = true;
@@ -317,6 +337,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             bool ok = true;
             for (int tile = pair; tile < total && ok; tile += npairs) {
                 const TileCoord tc = tile_coords(tb, G, tile);
+                const int kblocks = p.set[tc.g >= p.G0 ? 1 : 0].k_blocks;
                 int tstart, ntok;
                 token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
                 const int n_mma = (ntok + 15) & ~15;
@@ -327,7 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * ACC_COLS;
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&ctl->full[stage], phase, &ctl->abort, p.status)) {
                         ok = false;
                         break;
@@ -364,11 +385,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int my_tok = e >> 3;        // token (0..15) of a 16-token chunk this thread stores
         const int part = e & 7;
         const uint32_t leader_tempty = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
         int acc = 0, xb = 0;
         uint32_t acc_phase = 0;
         for (int tile = pair; tile < total; tile += npairs) {
             const TileCoord tc = tile_coords(tb, G, tile);
+            const SetParams& sp = p.set[tc.g >= p.G0 ? 1 : 0];
+            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(sp.out);
             int tstart, ntok;
             token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
             const int tok0 = tb->rowstart[tc.g] + tstart;
@@ -405,11 +427,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                         v.y = pack_bf16x2(silu_f32(g0.z) * u0.z, silu_f32(g0.w) * u0.w);
                         v.z = pack_bf16x2(silu_f32(g1.x) * u1.x, silu_f32(g1.y) * u1.y);
                         v.w = pack_bf16x2(silu_f32(g1.z) * u1.z, silu_f32(g1.w) * u1.w);
-                        *reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * p.ldo + fcta + fj) = v;
+                        *reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * sp.ldo + fcta + fj) = v;
                     }
                 } else {
                     const int fj = part * 16;
-                    if (tok_ok && fcta + fj < p.f_limit) {
+                    if (tok_ok && fcta + fj < sp.f_limit) {
                         float f[16];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
@@ -419,7 +441,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                             f[4 * i + 2] = t.z;
                             f[4 * i + 3] = t.w;
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * p.ldo + fcta + fj);
+                        uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * sp.ldo + fcta + fj);
                         dst[0] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
                                             pack_bf16x2(f[6], f[7]));
                         dst[1] = make_uint4(pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
@@ -444,72 +466,112 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
 }
 
+struct Maps {
+    CUtensorMap w0, w1, x, xs;
+};
+
 template <bool UP>
-cudaError_t launch(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x, const CUtensorMap& xs,
-                   const CUtensorMap& xg, const Params& p, int num_sms, cudaStream_t st) {
+cudaError_t launch(const Maps& a, const Maps& b, const CUtensorMap& xg, const Params& p, int num_sms,
+                   cudaStream_t st) {
     auto kern = tc_grouped_gemm_kernel<UP>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;  // whole CTA pairs, one CTA per SM
-    kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(w0, w1, x, xs, xg, p);
+    kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(a.w0, a.w1, a.x, a.xs, b.w0, b.w1, b.x, b.xs, xg, p);
     note_launches(1);
     return cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_tc_up(const TcUpArgs& a, int* status, int num_sms, cudaStream_t st) {
-    if (a.G <= 0 || a.G > kMaxGroups || a.d % BK != 0 || a.I % 128 != 0) return cudaErrorInvalidValue;
-    CUtensorMap tW1, tW3, tX, tXs, tXg;
-    if (!make_tmap_2d(&tW1, a.W1, a.d, a.W_rows, a.d, BK, 64) || !make_tmap_2d(&tW3, a.W3, a.d, a.W_rows, a.d, BK, 64) ||
-        !make_tmap_2d(&tX, a.A, a.d, a.A_rows, a.d, BK, B_ROWS) ||
-        !make_tmap_2d(&tXs, a.A, a.d, a.A_rows, a.d, BK, SMALL_ROWS) ||
-        !make_tmap_2d(&tXg, a.A, a.d, a.A_rows, a.d, BK, 1))  // one-row box for tile::gather4
-        return cudaErrorInvalidValue;
-    Params p{};
-    p.offsets = a.offsets;
-    p.G = a.G;
-    p.M = a.M;
-    p.f_tiles = a.I / 128;
-    p.k_blocks = a.d / BK;
-    p.w_rows = a.I;
-    p.kseg = a.d;
-    p.nseg = 1;
-    p.out = a.H;
-    p.ldo = a.I;
-    p.f_limit = a.I;
-    p.a_rows = a.gather ? a.gather_rows : a.A_rows;
-    p.gather = a.gather;
-    p.gather_div = a.gather_div > 0 ? a.gather_div : 1;
-    p.status = status;
-    return launch<true>(tW1, tW3, tX, tXs, tXg, p, num_sms, st);
+bool up_set(const TcUpArgs& a, Maps& m, SetParams& sp) {
+    if (a.d % BK != 0 || a.I % 128 != 0) return false;
+    if (!make_tmap_2d(&m.w0, a.W1, a.d, a.W_rows, a.d, BK, 64) || !make_tmap_2d(&m.w1, a.W3, a.d, a.W_rows, a.d, BK, 64) ||
+        !make_tmap_2d(&m.x, a.A, a.d, a.A_rows, a.d, BK, B_ROWS) ||
+        !make_tmap_2d(&m.xs, a.A, a.d, a.A_rows, a.d, BK, SMALL_ROWS))
+        return false;
+    sp.f_tiles = a.I / 128;
+    sp.k_blocks = a.d / BK;
+    sp.w_rows = a.I;
+    sp.kseg = a.d;
+    sp.nseg = 1;
+    sp.out = a.H;
+    sp.ldo = a.I;
+    sp.f_limit = a.I;
+    sp.a_rows = a.gather ? a.gather_rows : a.A_rows;
+    return true;
 }
 
-cudaError_t launch_tc_down(const TcDownArgs& a, int* status, int num_sms, cudaStream_t st) {
-    if (a.G <= 0 || a.G > kMaxGroups || a.K % BK != 0 || a.kseg % BK != 0 || a.d % 16 != 0)
-        return cudaErrorInvalidValue;
-    CUtensorMap tW2, tX, tXs;
-    if (!make_tmap_3d(&tW2, a.W2, a.kseg, a.d, (unsigned long long)a.G * a.nseg, BK, 128) ||
-        !make_tmap_2d(&tX, a.H, a.K, a.H_rows, a.K, BK, B_ROWS) ||
-        !make_tmap_2d(&tXs, a.H, a.K, a.H_rows, a.K, BK, SMALL_ROWS))
-        return cudaErrorInvalidValue;
+bool down_set(const TcDownArgs& a, Maps& m, SetParams& sp) {
+    if (a.K % BK != 0 || a.kseg % BK != 0 || a.d % 16 != 0) return false;
+    if (!make_tmap_3d(&m.w0, a.W2, a.kseg, a.d, (unsigned long long)a.G * a.nseg, BK, 128) ||
+        !make_tmap_2d(&m.x, a.H, a.K, a.H_rows, a.K, BK, B_ROWS) ||
+        !make_tmap_2d(&m.xs, a.H, a.K, a.H_rows, a.K, BK, SMALL_ROWS))
+        return false;
+    m.w1 = m.w0;
+    sp.f_tiles = (a.d + 255) / 256;
+    sp.k_blocks = a.K / BK;
+    sp.w_rows = 0;
+    sp.kseg = a.kseg;
+    sp.nseg = a.nseg;
+    sp.out = a.Y;
+    sp.ldo = a.d;
+    sp.f_limit = a.d;
+    sp.a_rows = a.H_rows;
+    return true;
+}
+
+}  // namespace
+
+// routed: groups from offsets (may be null to launch the shared set alone);
+// shared: one group of M rows (may be null).  Both sets share one launch.
+cudaError_t launch_tc_up(const TcUpArgs* routed, const TcUpArgs* shared, int* status, int num_sms, cudaStream_t st) {
+    if (!routed && !shared) return cudaSuccess;
+    Maps ma{}, mb{};
     Params p{};
-    p.offsets = a.offsets;
-    p.G = a.G;
-    p.M = a.M;
-    p.f_tiles = (a.d + 255) / 256;
-    p.k_blocks = a.K / BK;
-    p.w_rows = 0;
-    p.kseg = a.kseg;
-    p.nseg = a.nseg;
-    p.out = a.Y;
-    p.ldo = a.d;
-    p.f_limit = a.d;
-    p.a_rows = a.H_rows;
+    CUtensorMap xg{};
+    if (routed) {
+        if (routed->G <= 0 || routed->G > kMaxGroups || !routed->offsets || !up_set(*routed, ma, p.set[0]))
+            return cudaErrorInvalidValue;
+        if (!make_tmap_2d(&xg, routed->A, routed->d, routed->A_rows, routed->d, BK, 1))  // one-row box, tile::gather4
+            return cudaErrorInvalidValue;
+        p.offsets = routed->offsets;
+        p.G0 = routed->G;
+        p.gather = routed->gather;
+        p.gather_div = routed->gather_div > 0 ? routed->gather_div : 1;
+    }
+    if (shared) {
+        if (shared->M <= 0 || !up_set(*shared, mb, p.set[1])) return cudaErrorInvalidValue;
+        p.has_shared = 1;
+        p.M = shared->M;
+        if (!routed) xg = mb.x;
+    }
+    if (!routed) ma = mb;
+    if (!shared) mb = ma;
+    p.status = status;
+    return launch<true>(ma, mb, xg, p, num_sms, st);
+}
+
+cudaError_t launch_tc_down(const TcDownArgs* routed, const TcDownArgs* shared, int* status, int num_sms,
+                           cudaStream_t st) {
+    if (!routed && !shared) return cudaSuccess;
+    Maps ma{}, mb{};
+    Params p{};
+    if (routed) {
+        if (routed->G <= 0 || routed->G > kMaxGroups || !routed->offsets || !down_set(*routed, ma, p.set[0]))
+            return cudaErrorInvalidValue;
+        p.offsets = routed->offsets;
+        p.G0 = routed->G;
+    }
+    if (shared) {
+        if (shared->M <= 0 || !down_set(*shared, mb, p.set[1])) return cudaErrorInvalidValue;
+        p.has_shared = 1;
+        p.M = shared->M;
+    }
+    if (!routed) ma = mb;
+    if (!shared) mb = ma;
     p.gather = nullptr;
     p.gather_div = 1;
     p.status = status;
-    return launch<false>(tW2, tW2, tX, tXs, tXs, p, num_sms, st);
+    return launch<false>(ma, mb, ma.x, p, num_sms, st);
 }
 
 }  // namespace moe

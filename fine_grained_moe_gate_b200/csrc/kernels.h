@@ -93,8 +93,11 @@ struct TcDownArgs {
     const int32_t* offsets;
     int G, M;
 };
-cudaError_t launch_tc_up(const TcUpArgs& a, int* status, int num_sms, cudaStream_t st);
-cudaError_t launch_tc_down(const TcDownArgs& a, int* status, int num_sms, cudaStream_t st);
+// One launch for the routed set (offsets) and/or the shared set (M rows);
+// either pointer may be null.
+cudaError_t launch_tc_up(const TcUpArgs* routed, const TcUpArgs* shared, int* status, int num_sms, cudaStream_t st);
+cudaError_t launch_tc_down(const TcDownArgs* routed, const TcDownArgs* shared, int* status, int num_sms,
+                           cudaStream_t st);
 
 // selftest.cu
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int* status, cudaStream_t st);

@@ -199,6 +199,26 @@ MOE_API moe_status moe_expert_down(const void* h, const int32_t* offsets, const 
                                    void* y, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_ffn_up / moe_ffn_down -- the routed AND the shared experts' projection
+ * in one launch each: the shared set is one more group of the same
+ * persistent grouped GEMM (bf16), so its tiles fill the SMs the routed
+ * groups leave idle.  moe_grouped_swiglu is moe_ffn_up then moe_ffn_down.
+ *   moe_ffn_up:   h  = moe_expert_up(x_perm; MOE_ROUTED)   [T*k][I]
+ *                 hs = moe_expert_up(x;      MOE_SHARED)   [T][S*Is]
+ *   moe_ffn_down: y_perm     = moe_expert_down(h;  MOE_ROUTED)  [T*k][d]
+ *                 shared_out = moe_expert_down(hs; MOE_SHARED)  [T][d]
+ * x == NULL (up), hs == NULL (down) or S == 0 leaves the shared set out
+ * (hs / shared_out and the shared weights are then ignored).  Results are
+ * bit-identical to the separate calls.  h must not alias x_perm or x; y_perm
+ * may alias x_perm (moe_ffn_down does not read it).
+ * -------------------------------------------------------------------------*/
+MOE_API moe_status moe_ffn_up(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3,
+                              const void* x, const void* ws1, const void* ws3, moe_shape sh, void* h, void* hs,
+                              void* stream);
+MOE_API moe_status moe_ffn_down(const void* h, const int32_t* offsets, const void* w2, const void* hs,
+                                const void* ws2, moe_shape sh, void* y_perm, void* shared_out, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_combine -- weighted combine back into token order  [P2 DeepSeekMoE
  * sketch: routed_out[mask] += w * expert(x[mask]); shared_out + routed_out].
  *   y[t] = shared_out[t] + sum_{j=0..k-1} topk_w[t][j] * y_perm[inv_row[t*k+j]]

@@ -118,6 +118,25 @@ def test_layer_forward_checks(L):
     assert r == INVALID  # S = 1 needs the shared weights
 
 
+def test_ffn_checks(L):
+    sh = shape()
+    c = ctypes.c_void_p
+    # up: x_perm, offsets, w1, w3, x, ws1, ws3, sh, h, hs
+    assert L.moe_ffn_up(c(FAKE), None, c(FAKE), c(FAKE), None, None, None, sh, c(FAKE), None, None) == INVALID
+    assert L.moe_ffn_up(c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), None, c(FAKE), sh, c(FAKE), c(FAKE),
+                        None) == INVALID                                    # x given: shared weights needed
+    assert L.moe_ffn_up(c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), sh, c(FAKE), None,
+                        None) == INVALID                                    # ... and hs
+    assert L.moe_ffn_up(c(FAKE), c(FAKE), c(FAKE), c(FAKE), None, None, None, sh, c(FAKE + 4), None,
+                        None) == ALIGN
+    # down: h, offsets, w2, hs, ws2, sh, y_perm, shared_out
+    assert L.moe_ffn_down(c(FAKE), c(FAKE), None, None, None, sh, c(FAKE), None, None) == INVALID
+    assert L.moe_ffn_down(c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), sh, c(FAKE), None, None) == INVALID
+    assert L.moe_ffn_down(c(FAKE), c(FAKE), c(FAKE), c(FAKE), None, sh, c(FAKE), c(FAKE), None) == INVALID
+    assert L.moe_ffn_down(c(FAKE), c(FAKE), c(FAKE), None, None, shape(k=17, E=32), c(FAKE), None,
+                          None) == UNSUPPORTED
+
+
 def test_bias_update_checks(L):
     c = ctypes.c_void_p
     assert L.moe_load_and_bias_update(c(FAKE), shape(T=0), ctypes.c_float(1e-3), None, c(FAKE), None, None) == INVALID

@@ -376,6 +376,45 @@ def test_expert_up_gather_equals_permuted_rows(dtype):
     assert torch.equal(h1.view(bits), h2.view(bits))
 
 
+@pytest.mark.parametrize("dtype,S", [("bf16", 2), ("bf16", 0), ("f32", 2)])
+def test_ffn_one_launch_per_projection_equals_separate_sets(dtype, S):
+    """moe_ffn_up / moe_ffn_down run the routed and the shared set in one
+    launch each; every output equals, bit for bit, the per-set calls.  The
+    shared set is wider than a routed expert (S*Is = 4 I) and contracts over
+    a longer K on the way down, so per-set tile counts and K blocks differ."""
+    bf = dtype == "bf16"
+    cfg = V3.scaled(T=700, d=256 if bf else 96, E=16, k=4, I=128 if bf else 16, S=S, Is=256 if bf else 24,
+                    dtype=dtype, w_std=0.05)
+    sh = moe.shape_of(cfg)
+    p = make_layer(cfg, DEV)
+    x = make_tokens(cfg, DEV)
+    idx, w, counts, _ = route(sh, x, p["w_gate"], p["bias"], with_aff=False)
+    x_perm, offsets, perm, inv = permute(sh, x, idx, counts)
+    rows, SIs = cfg.T * cfg.k, max(1, cfg.S * cfg.Is)
+    new = lambda *shape: torch.full(shape, float("nan"), dtype=x.dtype, device=DEV)
+    h1, h2 = new(rows, cfg.I), new(rows, cfg.I)
+    hs1, hs2 = new(cfg.T, SIs), new(cfg.T, SIs)
+    y1, y2 = new(rows, cfg.d), new(rows, cfg.d)
+    so1, so2 = new(cfg.T, cfg.d), new(cfg.T, cfg.d)
+    xs_ = x if S > 0 else None
+    moe.moe_ffn_up(x_perm, offsets, p["w1"], p["w3"], xs_, p["ws1"], p["ws3"], sh, h1, hs1)
+    moe.moe_ffn_down(h1, offsets, p["w2"], hs1 if S > 0 else None, p["ws2"], sh, y1, so1)
+    moe.moe_expert_up(x_perm, None, offsets, p["w1"], p["w3"], sh, moe.MOE_ROUTED, h2)
+    moe.moe_expert_down(h2, offsets, p["w2"], sh, moe.MOE_ROUTED, y2)
+    if S > 0:
+        moe.moe_expert_up(x, None, None, p["ws1"], p["ws3"], sh, moe.MOE_SHARED, hs2)
+        moe.moe_expert_down(hs2, None, p["ws2"], sh, moe.MOE_SHARED, so2)
+    torch.cuda.synchronize()
+    check_status()
+    bits = torch.int16 if bf else torch.int32
+    pairs = [(h1, h2), (y1, y2)] + ([(hs1, hs2), (so1, so2)] if S > 0 else [])
+    for a, b in pairs:
+        assert torch.isfinite(a.float()).all()
+        assert torch.equal(a.view(bits), b.view(bits))
+    if S == 0:  # the shared buffers are left alone
+        assert torch.isnan(hs1.float()).all() and torch.isnan(so1.float()).all()
+
+
 def test_bounded_wait_times_out_and_context_survives():
     """Failure detection without a fault: a device wait that nothing ends
     gives up after its limit, reports MOE_ERR_TIMEOUT through the status
