@@ -186,16 +186,17 @@ def cpu_baseline_record(cfg, secs, n_tok, threads, label):
 
 # ------------------------------------------------------------ our leg
 
-def traffic_record(kernel_file: str):
-    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
-    summary, if the kernel source is unchanged since it was captured."""
+def traffic_record(kernel_file: str, workload_name: str):
+    """Per-launch DRAM bytes of the dominant kernel on this workload from the
+    committed ncu summary, if the kernel source is unchanged since it was
+    captured."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
         with open(kernel_file, "rb") as f:
             digest = hashlib.sha256(f.read()).hexdigest()[:16]
-        ent = rec.get(DOMINANT)
+        ent = rec.get(workload_name, {}).get(DOMINANT)
         if ent and ent.get("source_sha256_16") == digest:
             return ent.get("dram_bytes_per_launch")
     except (OSError, ValueError):
@@ -369,16 +370,17 @@ def run_ours(args, world, rank, local):
     bytes_per_launch = (n_touched * 2 * cfg.I * d + T * k * (d + cfg.I) + 2 * SIs * d + T * (d + SIs)) * esz
     hbm_gbs = bytes_per_launch / (dom_ms / 1e3) / 1e9
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    traffic = traffic_record(os.path.join(ROOT, "fine_grained_moe_gate_b200", "csrc", "gemm_tc.cu"), cfg.name)
     roof_hbm = {"bound": "hbm", "kernel": "gate/up projection (routed + shared)", "achieved": round(hbm_gbs, 1), "peak": hbm_peak,
                 "unit": "GB/s", "frac": round(hbm_gbs / hbm_peak, 4),
                 "frac_of_nominal_8000": round(hbm_gbs / 8000.0, 4),
-                "traffic": None, "bytes_per_launch": int(bytes_per_launch), "experts_touched": n_touched,
+                "traffic": traffic, "bytes_per_launch": int(bytes_per_launch), "experts_touched": n_touched,
                 "peak_kind": f"hbm_gbs ({peak_src}, copy bandwidth)"}
     if cfg.dtype == "bf16":
         peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         roof = {"bound": "tensor", "kernel": "tc_grouped_gemm_kernel<up> (routed + shared experts, SwiGLU epilogue)",
                 "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": traffic_record(os.path.join(ROOT, "fine_grained_moe_gate_b200", "csrc", "gemm_tc.cu")),
+                "traffic": traffic,
                 "peak_kind": f"bf16_tflops_sustained ({peak_src}): the kernel is timed inside a long step",
                 "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
     else:

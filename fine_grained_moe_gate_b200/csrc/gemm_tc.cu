@@ -26,14 +26,21 @@
 //   down tile: each CTA holds 128 rows of W2 (its 128 output features).
 // The weights stay in their natural [out][in] layout (no packing pass).
 //
-// One persistent cluster per SM pair walks a device-side tile list built
-// from the expert offsets (no host read-back); per expert, token tiles are
-// walked fastest so clusters working on one weight tile at the same time
-// share it in L2, and the expert's tokens stay in L2 across feature tiles.
+// One persistent cluster per SM pair takes tiles from a device-side tile list
+// built from the expert offsets (no host read-back), in list order, through
+// a global atomic counter: the tiles in flight are always a window of about
+// one tile per cluster, so the clusters sharing an expert's token rows (its
+// feature tiles) or a weight tile (its token tiles) run at the same time and
+// find them in L2, and the last tiles spread over the clusters that are free.
+// Per expert, token tiles are walked fastest, then feature tiles.
 //
 // Warp roles (192 threads per CTA):
 //   warp 0      TMA producer (one lane), both CTAs: loads its own halves,
-//               completion counted on the leader CTA's barrier.
+//               completion counted on the leader CTA's barrier.  The
+//               leader's producer takes tiles from the counter and posts
+//               them in a small tile queue in both CTAs' shared memory for
+//               every other role, one tile ahead of its own loads (the
+//               atomic's round trip overlaps the current tile's loads).
 //   warp 1      TMEM owner (paired allocation); in the leader (even) CTA one
 //               lane issues the MMAs and commits to both CTAs' barriers.
 //   warps 2..5  epilogue: tcgen05.ld 32 lanes x 16 tokens into shared memory,
@@ -43,6 +50,8 @@
 // Every wait is bounded (common.cuh); on a timeout the CTA raises its abort
 // flag, drains what it issued, frees TMEM and exits (the peer then times out
 // on its next wait and does the same).
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tmap.h"
@@ -69,13 +78,28 @@ constexpr int XBUF_BYTES = 16 * XS * 4; // 16 tokens x 128 lanes (+pad), fp32
 // slower on the V3 step than the normal policy for both.
 constexpr uint64_t W_HINT = kEvictNormal;
 constexpr uint64_t X_HINT = kEvictNormal;
+constexpr int TQ = 8;                   // tile queue slots
+// readers of a queue slot: leader MMA issuer + 4 epilogue warps, peer producer + 4 epilogue warps
+constexpr uint32_t TQ_READERS = 10;
+
+// Tile counters: one {next, done} pair per launch slot.  A launch takes the
+// next slot round-robin on the host; the last cluster to finish resets its
+// pair to zero, so every launch starts from a zero counter without a memset.
+// Two launches share a pair only if 1024 launches were enqueued in between
+// while the first is still running.
+constexpr int kSchedSlots = 1024;
+__device__ unsigned int g_tile_sched[kSchedSlots][2];
+
 
 struct Ctl {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t tfull[2];
     uint64_t tempty[2];
+    uint64_t tq_full[TQ];   // in both CTAs: slot holds the next tile
+    uint64_t tq_empty[TQ];  // leader only: every reader has taken the slot's tile
     uint64_t drain;
+    int tq[TQ];             // tile index, or -1 when the list is exhausted
     uint32_t tmem_base;
     int abort;
 };
@@ -109,6 +133,7 @@ struct Params {
     SetParams set[2];
     const int32_t* gather;  // up, routed set, optional: row r reads token row gather[r] / gather_div
     int gather_div;
+    int sched_slot;         // this launch's tile counter pair
     int* status;
 };
 
@@ -167,6 +192,37 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     }
 }
 
+// Tile queue signalling.  No cluster-scope release is issued by the TMA
+// producer or the MMA issuer: on B200 one such arrive per tile measured about
+// 1 us of producer stall per tile (the loads of the next tile start late).
+// The peer's slot is written with st.async, whose byte count completes the
+// peer's barrier (armed by a relaxed remote expect-tx arrive), and readers
+// free a slot with a relaxed arrive issued after the tile index was consumed.
+__device__ __forceinline__ void st_async_u32(uint32_t cluster_addr, int v, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(cluster_addr),
+                 "r"(v), "r"(cluster_bar)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+// Reader side of the tile queue: wait for slot j, take its tile, free the
+// slot for the leader's producer.  Returns false on a timeout or abort.
+__device__ __forceinline__ bool tq_take(Ctl* ctl, int j, uint32_t ph, uint32_t leader_tq_empty, int* tile,
+                                        int* status) {
+    if (!mbar_wait_cluster(&ctl->tq_full[j], ph, &ctl->abort, status)) return false;
+    const int t = reinterpret_cast<volatile int*>(ctl->tq)[j];
+    *tile = t;
+    mbar_arrive_relaxed_cluster(leader_tq_empty + 8u * (uint32_t)j);
+    return true;
+}
+
 template <bool UP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW0a, const __grid_constant__ CUtensorMap tmW1a,
@@ -184,7 +240,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();  // 0 = leader (issues the MMAs)
-    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int npairs = gridDim.x >> 1;
     const int G = p.G0 + p.has_shared;
 
     for (int g = tid; g < G; g += NTHREADS) {
@@ -208,6 +264,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         for (int a = 0; a < 2; ++a) {
             mbar_init(&ctl->tfull[a], 1);
             mbar_init(&ctl->tempty[a], 8);  // 4 epilogue warps x 2 CTAs
+        }
+        for (int j = 0; j < TQ; ++j) {
+            mbar_init(&ctl->tq_full[j], 1);
+            mbar_init(&ctl->tq_empty[j], TQ_READERS);
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -239,6 +299,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
     const int total = tb->prefix[G];
+    const uint32_t leader_tq_empty = mapa_shared(smem_u32(&ctl->tq_empty[0]), 0);
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
@@ -259,10 +320,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             }
         }
         const uint32_t leader_full = mapa_shared(smem_u32(&ctl->full[0]), 0);
-        int stage = 0;
-        uint32_t phase = 0;
+        const uint32_t peer_tq = mapa_shared(smem_u32(&ctl->tq[0]), 1);
+        const uint32_t peer_tq_full = mapa_shared(smem_u32(&ctl->tq_full[0]), 1);
+        unsigned int* sched = g_tile_sched[p.sched_slot];
+        int stage = 0, tq_j = 0, post_j = 0;
+        uint32_t phase = 0, tq_ph = 0, post_ph = 0;
         bool ok = true, issued_any = false;
-        for (int tile = pair; tile < total && ok; tile += npairs) {
+        // leader, lane 0: post a tile (index, or -1 = no more) to both CTAs' queue slot post_j
+        auto post = [&](int t) -> bool {
+            if (!mbar_wait_cluster(&ctl->tq_empty[post_j], post_ph ^ 1u, &ctl->abort, p.status)) return false;
+            ctl->tq[post_j] = t;
+            mbar_arrive(&ctl->tq_full[post_j]);  // CTA-scope release of the store above
+            mbar_arrive_expect_tx_remote(peer_tq_full + 8u * (uint32_t)post_j, 4u);
+            st_async_u32(peer_tq + 4u * (uint32_t)post_j, t, peer_tq_full + 8u * (uint32_t)post_j);
+            if (++post_j == TQ) {
+                post_j = 0;
+                post_ph ^= 1u;
+            }
+            return true;
+        };
+        const auto take = [&](unsigned int t) { return t < (unsigned int)total ? (int)t : -1; };
+        int cur = -1;
+        unsigned int t_next = 0;
+        if (rank == 0 && lane == 0) {
+            cur = take(atomicAdd(&sched[0], 1u));
+            ok = post(cur);
+            if (ok && cur >= 0) t_next = atomicAdd(&sched[0], 1u);
+        }
+        for (;;) {
+            int tile = -1;
+            if (lane == 0) {
+                if (rank == 0) {  // cur is posted; post the next one before loading cur
+                    tile = ok ? cur : -1;
+                    if (ok && cur >= 0) {
+                        cur = take(t_next);
+                        ok = post(cur);
+                        if (ok && cur >= 0) t_next = atomicAdd(&sched[0], 1u);
+                    }
+                } else {
+                    ok = tq_take(ctl, tq_j, tq_ph, leader_tq_empty, &tile, p.status);
+                    if (++tq_j == TQ) {
+                        tq_j = 0;
+                        tq_ph ^= 1u;
+                    }
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            tile = __shfl_sync(0xffffffffu, tile, 0);
+            if (!ok || tile < 0) break;
             const TileCoord tc = tile_coords(tb, G, tile);
             const int si = tc.g >= p.G0 ? 1 : 0;
             const SetParams& sp = p.set[si];
@@ -322,6 +427,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     phase ^= 1u;
                 }
             }
+            if (!ok) break;
+        }
+        if (rank == 0 && lane == 0) {  // this cluster takes no more tiles; the last one resets the counter
+            __threadfence();
+            if (atomicAdd(&sched[1], 1u) == (unsigned int)npairs - 1u) {
+                __threadfence();
+                atomicExch(&sched[0], 0u);
+                atomicExch(&sched[1], 0u);
+            }
         }
         if (!ok && issued_any && lane == 0) {  // let copies already in flight land before the CTA exits
             const uint64_t t0 = globaltimer_ns();
@@ -332,10 +446,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (leader CTA only)
         if (rank == 0 && elect_one()) {
-            int stage = 0, acc = 0;
-            uint32_t phase = 0, acc_phase = 0;
+            int stage = 0, acc = 0, j = 0;
+            uint32_t phase = 0, acc_phase = 0, tq_ph = 0;
             bool ok = true;
-            for (int tile = pair; tile < total && ok; tile += npairs) {
+            for (;;) {
+                int tile;
+                if (!tq_take(ctl, j, tq_ph, leader_tq_empty, &tile, p.status)) {
+                    ok = false;
+                    break;
+                }
+                if (++j == TQ) {
+                    j = 0;
+                    tq_ph ^= 1u;
+                }
+                if (tile < 0) break;
                 const TileCoord tc = tile_coords(tb, G, tile);
                 const int kblocks = p.set[tc.g >= p.G0 ? 1 : 0].k_blocks;
                 int tstart, ntok;
@@ -385,9 +509,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const int my_tok = e >> 3;        // token (0..15) of a 16-token chunk this thread stores
         const int part = e & 7;
         const uint32_t leader_tempty = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
-        int acc = 0, xb = 0;
-        uint32_t acc_phase = 0;
-        for (int tile = pair; tile < total; tile += npairs) {
+        int acc = 0, xb = 0, j = 0;
+        uint32_t acc_phase = 0, tq_ph = 0;
+        for (;;) {
+            int tile = -1, got = 1;
+            if (lane == 0) got = tq_take(ctl, j, tq_ph, leader_tq_empty, &tile, p.status) ? 1 : 0;
+            got = __shfl_sync(0xffffffffu, got, 0);
+            tile = __shfl_sync(0xffffffffu, tile, 0);
+            if (!got || tile < 0) break;
+            if (++j == TQ) {
+                j = 0;
+                tq_ph ^= 1u;
+            }
             const TileCoord tc = tile_coords(tb, G, tile);
             const SetParams& sp = p.set[tc.g >= p.G0 ? 1 : 0];
             __nv_bfloat16* out = static_cast<__nv_bfloat16*>(sp.out);
@@ -470,10 +603,12 @@ struct Maps {
     CUtensorMap w0, w1, x, xs;
 };
 
+std::atomic<unsigned int> g_sched_seq{0};
+
 template <bool UP>
-cudaError_t launch(const Maps& a, const Maps& b, const CUtensorMap& xg, const Params& p, int num_sms,
-                   cudaStream_t st) {
+cudaError_t launch(const Maps& a, const Maps& b, const CUtensorMap& xg, Params p, int num_sms, cudaStream_t st) {
     auto kern = tc_grouped_gemm_kernel<UP>;
+    p.sched_slot = (int)(g_sched_seq.fetch_add(1u, std::memory_order_relaxed) % (unsigned int)kSchedSlots);
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;  // whole CTA pairs, one CTA per SM
