@@ -64,9 +64,13 @@ constexpr int STAGES = 6;
 constexpr int A_BYTES = 128 * BK * 2;   // this CTA's 128 weight rows
 constexpr int B_ROWS = 128;             // this CTA's half of <= 256 tokens
 constexpr int B_BYTES = B_ROWS * BK * 2;
+// Token rows are loaded with one box per K step whose height is the CTA's
+// half of the tile rounded up to 16 rows (16, 32, ..., 128: one tensor map
+// each); a fixed 128-row box would bring in up to 60% rows of no use on
+// balanced tiles.
+constexpr int NXBOX = B_ROWS / 16;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
 constexpr int NT = 256;                 // tokens per tile (MMA N <= 256)
-constexpr int SMALL_ROWS = 16;          // per-CTA token box for tiles of <= 32 tokens
 constexpr uint32_t ACC_COLS = 256;      // one accumulator buffer
 constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
 constexpr int NTHREADS = 192;
@@ -115,6 +119,13 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // One expert set in a launch: set 0 = the routed experts (groups [0, G0),
 // rows from offsets), set 1 = the shared experts (group G0, rows [0, M)).
+// Tensor maps of one expert set: weights (w1 only for the up projection) and
+// the token operand with box heights 16 * (i + 1) rows.
+struct SetMaps {
+    CUtensorMap w0, w1;
+    CUtensorMap x[NXBOX];
+};
+
 struct SetParams {
     int f_tiles;       // feature tiles (per CTA pair) per group
     int k_blocks;
@@ -225,10 +236,7 @@ __device__ __forceinline__ bool tq_take(Ctl* ctl, int j, uint32_t ph, uint32_t l
 
 template <bool UP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
-    tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW0a, const __grid_constant__ CUtensorMap tmW1a,
-                           const __grid_constant__ CUtensorMap tmXa, const __grid_constant__ CUtensorMap tmXsa,
-                           const __grid_constant__ CUtensorMap tmW0b, const __grid_constant__ CUtensorMap tmW1b,
-                           const __grid_constant__ CUtensorMap tmXb, const __grid_constant__ CUtensorMap tmXsb,
+    tc_grouped_gemm_kernel(const __grid_constant__ SetMaps ma, const __grid_constant__ SetMaps mb,
                            const __grid_constant__ CUtensorMap tmXg, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -309,14 +317,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const bool gather = UP && p.gather != nullptr;  // routed set only
         if (lane == 0) {
             if (p.G0 > 0) {
-                tma_prefetch_desc(&tmW0a);
-                if (UP) tma_prefetch_desc(&tmW1a);
-                tma_prefetch_desc(gather ? &tmXg : &tmXa);
+                tma_prefetch_desc(&ma.w0);
+                if (UP) tma_prefetch_desc(&ma.w1);
+                tma_prefetch_desc(gather ? &tmXg : &ma.x[NXBOX - 1]);
             }
             if (p.has_shared) {
-                tma_prefetch_desc(&tmW0b);
-                if (UP) tma_prefetch_desc(&tmW1b);
-                tma_prefetch_desc(&tmXb);
+                tma_prefetch_desc(&mb.w0);
+                if (UP) tma_prefetch_desc(&mb.w1);
+                tma_prefetch_desc(&mb.x[NXBOX - 1]);
             }
         }
         const uint32_t leader_full = mapa_shared(smem_u32(&ctl->full[0]), 0);
@@ -371,10 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const TileCoord tc = tile_coords(tb, G, tile);
             const int si = tc.g >= p.G0 ? 1 : 0;
             const SetParams& sp = p.set[si];
-            const CUtensorMap* mW0 = si ? &tmW0b : &tmW0a;
-            const CUtensorMap* mW1 = si ? &tmW1b : &tmW1a;
-            const CUtensorMap* mX = si ? &tmXb : &tmXa;
-            const CUtensorMap* mXs = si ? &tmXsb : &tmXsa;
+            const SetMaps& M = si ? mb : ma;
             const int wg = si ? 0 : tc.g;  // weight block index of the group inside its set
             const bool gat = gather && si == 0;
             int tstart, ntok;
@@ -390,9 +395,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     src[j] = p.gather[row0 + (jr < ntok ? jr : 0)] / p.gather_div;
                 }
             }
-            const bool small = !gat && half <= SMALL_ROWS;
-            const uint32_t brows = gat ? (uint32_t)half : (uint32_t)(small ? SMALL_ROWS : B_ROWS);
-            const uint32_t tx = 2u * ((uint32_t)A_BYTES + brows * BK * 2);
+            const int xrows = gat ? half : (half + 15) & ~15;  // token rows this CTA loads per K step
+            const uint32_t tx = 2u * ((uint32_t)A_BYTES + (uint32_t)xrows * BK * 2);  // both CTAs' bytes
             for (int kb = 0; kb < sp.k_blocks; ++kb) {
                 int got = 1;
                 if (lane == 0) got = mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, p.status) ? 1 : 0;
@@ -408,15 +412,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], tx);
                     if (UP) {
                         const int wrow = wg * sp.w_rows + tc.ft * 128 + (int)rank * 64;
-                        tma_load_2d_pair(sa, mW0, fb, kb * BK, wrow, W_HINT);
-                        tma_load_2d_pair(sa + A_BYTES / 2, mW1, fb, kb * BK, wrow, W_HINT);
+                        tma_load_2d_pair(sa, &M.w0, fb, kb * BK, wrow, W_HINT);
+                        tma_load_2d_pair(sa + A_BYTES / 2, &M.w1, fb, kb * BK, wrow, W_HINT);
                     } else {
                         const int kk = kb * BK;
                         const int seg = kk / sp.kseg;
-                        tma_load_3d_pair(sa, mW0, fb, kk - seg * sp.kseg, tc.ft * 256 + (int)rank * 128,
+                        tma_load_3d_pair(sa, &M.w0, fb, kk - seg * sp.kseg, tc.ft * 256 + (int)rank * 128,
                                          wg * sp.nseg + seg, W_HINT);
                     }
-                    if (!gat) tma_load_2d_pair(sb, small ? mXs : mX, fb, kb * BK, tok0, X_HINT);
+                    if (!gat) tma_load_2d_pair(sb, &M.x[xrows / 16 - 1], fb, kb * BK, tok0, X_HINT);
                 }
                 if (gat && 4 * lane < half)
                     tma_gather4_pair(sb + 4 * lane * BK * 2, &tmXg, fb, kb * BK, src[0], src[1], src[2], src[3],
@@ -599,29 +603,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
 }
 
-struct Maps {
-    CUtensorMap w0, w1, x, xs;
-};
-
 std::atomic<unsigned int> g_sched_seq{0};
 
 template <bool UP>
-cudaError_t launch(const Maps& a, const Maps& b, const CUtensorMap& xg, Params p, int num_sms, cudaStream_t st) {
+cudaError_t launch(const SetMaps& a, const SetMaps& b, const CUtensorMap& xg, Params p, int num_sms, cudaStream_t st) {
     auto kern = tc_grouped_gemm_kernel<UP>;
     p.sched_slot = (int)(g_sched_seq.fetch_add(1u, std::memory_order_relaxed) % (unsigned int)kSchedSlots);
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;  // whole CTA pairs, one CTA per SM
-    kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(a.w0, a.w1, a.x, a.xs, b.w0, b.w1, b.x, b.xs, xg, p);
+    kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(a, b, xg, p);
     note_launches(1);
     return cudaGetLastError();
 }
 
-bool up_set(const TcUpArgs& a, Maps& m, SetParams& sp) {
+bool token_maps(SetMaps& m, const void* base, int cols, long long rows) {
+    for (int b = 0; b < NXBOX; ++b)
+        if (!make_tmap_2d(&m.x[b], base, cols, rows, cols, BK, 16 * (b + 1))) return false;
+    return true;
+}
+
+bool up_set(const TcUpArgs& a, SetMaps& m, SetParams& sp) {
     if (a.d % BK != 0 || a.I % 128 != 0) return false;
     if (!make_tmap_2d(&m.w0, a.W1, a.d, a.W_rows, a.d, BK, 64) || !make_tmap_2d(&m.w1, a.W3, a.d, a.W_rows, a.d, BK, 64) ||
-        !make_tmap_2d(&m.x, a.A, a.d, a.A_rows, a.d, BK, B_ROWS) ||
-        !make_tmap_2d(&m.xs, a.A, a.d, a.A_rows, a.d, BK, SMALL_ROWS))
+        !token_maps(m, a.A, a.d, a.A_rows))
         return false;
     sp.f_tiles = a.I / 128;
     sp.k_blocks = a.d / BK;
@@ -635,11 +640,10 @@ bool up_set(const TcUpArgs& a, Maps& m, SetParams& sp) {
     return true;
 }
 
-bool down_set(const TcDownArgs& a, Maps& m, SetParams& sp) {
+bool down_set(const TcDownArgs& a, SetMaps& m, SetParams& sp) {
     if (a.K % BK != 0 || a.kseg % BK != 0 || a.d % 16 != 0) return false;
     if (!make_tmap_3d(&m.w0, a.W2, a.kseg, a.d, (unsigned long long)a.G * a.nseg, BK, 128) ||
-        !make_tmap_2d(&m.x, a.H, a.K, a.H_rows, a.K, BK, B_ROWS) ||
-        !make_tmap_2d(&m.xs, a.H, a.K, a.H_rows, a.K, BK, SMALL_ROWS))
+        !token_maps(m, a.H, a.K, a.H_rows))
         return false;
     m.w1 = m.w0;
     sp.f_tiles = (a.d + 255) / 256;
@@ -660,7 +664,7 @@ bool down_set(const TcDownArgs& a, Maps& m, SetParams& sp) {
 // shared: one group of M rows (may be null).  Both sets share one launch.
 cudaError_t launch_tc_up(const TcUpArgs* routed, const TcUpArgs* shared, int* status, int num_sms, cudaStream_t st) {
     if (!routed && !shared) return cudaSuccess;
-    Maps ma{}, mb{};
+    SetMaps ma{}, mb{};
     Params p{};
     CUtensorMap xg{};
     if (routed) {
@@ -677,7 +681,7 @@ cudaError_t launch_tc_up(const TcUpArgs* routed, const TcUpArgs* shared, int* st
         if (shared->M <= 0 || !up_set(*shared, mb, p.set[1])) return cudaErrorInvalidValue;
         p.has_shared = 1;
         p.M = shared->M;
-        if (!routed) xg = mb.x;
+        if (!routed) xg = mb.x[NXBOX - 1];
     }
     if (!routed) ma = mb;
     if (!shared) mb = ma;
@@ -688,7 +692,7 @@ cudaError_t launch_tc_up(const TcUpArgs* routed, const TcUpArgs* shared, int* st
 cudaError_t launch_tc_down(const TcDownArgs* routed, const TcDownArgs* shared, int* status, int num_sms,
                            cudaStream_t st) {
     if (!routed && !shared) return cudaSuccess;
-    Maps ma{}, mb{};
+    SetMaps ma{}, mb{};
     Params p{};
     if (routed) {
         if (routed->G <= 0 || routed->G > kMaxGroups || !routed->offsets || !down_set(*routed, ma, p.set[0]))
@@ -706,7 +710,7 @@ cudaError_t launch_tc_down(const TcDownArgs* routed, const TcDownArgs* shared, i
     p.gather = nullptr;
     p.gather_div = 1;
     p.status = status;
-    return launch<false>(ma, mb, ma.x, p, num_sms, st);
+    return launch<false>(ma, mb, ma.x[NXBOX - 1], p, num_sms, st);
 }
 
 }  // namespace moe
