@@ -286,3 +286,126 @@ void orc_layer_output(const void* x, const int32_t* idx, const float* w, const v
     free(dest);
     free(yacc);
 }
+
+/* ---- FP8 (E4M3) experts ------------------------------------------------- */
+/* [P4] "DeepSeek V3 Architecture Deep Dive ...", "FP8 Formats": E4M3 (4
+ * exponent, 3 mantissa bits) for weights and activations; "Per-Tensor/
+ * Per-Axis Quantization": a scaling factor per row/channel.  Read here as:
+ * weights quantized per output row (channel), activations per token row;
+ * products accumulated wider than fp8 and the two scales applied after the
+ * sum, which is exact because both factor out of the dot product.
+ *
+ * E4M3 values, from the format's definition (the "fn" variant with no
+ * infinities): exponent bias 7; field e in 1..15 gives (1 + m/8) * 2^(e-7),
+ * e = 0 gives subnormals (m/8) * 2^-6; S.1111.111 is NaN; the largest finite
+ * magnitude is 1.75 * 2^8 = 448. */
+
+double orc_e4m3_decode(uint8_t c) {
+    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Nearest E4M3 value, ties to the even mantissa; magnitudes at or above 448
+ * give +-448 (saturating conversion).  Exact: every step is a multiplication
+ * by a power of two or an integer rounding in double. */
+uint8_t orc_e4m3_encode(float x) {
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0;
+    double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;
+    int e;
+    frexp(a, &e);            /* a = f * 2^e with f in [0.5, 1): the binade is 2^(e-1) */
+    int be = e - 1;
+    if (be < -6) be = -6;    /* below 2^-6 the grid is the subnormal one, step 2^-9 */
+    double step = ldexp(1.0, be - 3);
+    double n = a / step;
+    double r = floor(n);
+    double frac = n - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    double v = r * step;
+    if (v >= 448.0) return sign | 0x7E;
+    if (v == 0.0) return sign;
+    int e2;
+    frexp(v, &e2);
+    int vbe = e2 - 1;
+    if (vbe < -6) return sign | (uint8_t)(v / ldexp(1.0, -9));              /* subnormal: m * 2^-9 */
+    int m = (int)((v / ldexp(1.0, vbe) - 1.0) * 8.0);
+    return sign | (uint8_t)(((vbe + 7) << 3) | m);
+}
+
+void orc_e4m3_encode_array(const float* x, size_t n, uint8_t* q) {
+    for (size_t i = 0; i < n; ++i) q[i] = orc_e4m3_encode(x[i]);
+}
+void orc_e4m3_decode_array(const uint8_t* q, size_t n, double* x) {
+    for (size_t i = 0; i < n; ++i) x[i] = orc_e4m3_decode(q[i]);
+}
+
+/* Element (r, c) of a matrix with `rows` rows stored as nseg column blocks of
+ * kseg columns each ([nseg][rows][kseg], the layout of stacked experts whose
+ * blocks are joined along the contraction); nseg = 1 is plain row major. */
+static size_t seg_index(long r, int c, long rows, int kseg) {
+    return (size_t)(c / kseg) * (size_t)rows * kseg + (size_t)r * kseg + (size_t)(c % kseg);
+}
+
+/* Per-row quantization: amax_r = max |v| (fp32), scale_r = fl32(amax_r / 448),
+ * or 1 for an all-zero row; q = e4m3(fl32(v / scale_r)).  q has src's layout. */
+void orc_quantize_rows_fp8(const void* src, int dtype, long rows, int kseg, int nseg, uint8_t* q, float* scale) {
+    int K = kseg * nseg;
+    #pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int c = 0; c < K; ++c) {
+            float v = fabsf((float)load_elem(src, dtype, seg_index(r, c, rows, kseg)));
+            if (v > amax) amax = v;
+        }
+        float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scale[r] = sc;
+        for (int c = 0; c < K; ++c) {
+            size_t i = seg_index(r, c, rows, kseg);
+            float v = (float)load_elem(src, dtype, i);
+            q[i] = orc_e4m3_encode(v / sc);
+        }
+    }
+}
+
+/* Gate/up of one FP8 expert on n quantized token rows:
+ *   a[c] = xs[r] * w1s[c] * sum_i dec(xq[r][i]) dec(w1q[c][i])   (double)
+ *   g[c] = xs[r] * w3s[c] * sum_i dec(xq[r][i]) dec(w3q[c][i])
+ *   h[r][c] = bf16(silu(a) * g)                 (h stored in bf16, as the bf16 path)
+ * xq [n][d], w1q/w3q [I][d] row major. */
+void orc_expert_up_fp8(const uint8_t* xq, const float* xs, int n, const uint8_t* w1q, const float* w1s,
+                       const uint8_t* w3q, const float* w3s, int d, int I, uint16_t* h) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < n; ++r) {
+        for (int c = 0; c < I; ++c) {
+            double sa = 0.0, sg = 0.0;
+            for (int i = 0; i < d; ++i) {
+                double xv = orc_e4m3_decode(xq[(size_t)r * d + i]);
+                sa += xv * orc_e4m3_decode(w1q[(size_t)c * d + i]);
+                sg += xv * orc_e4m3_decode(w3q[(size_t)c * d + i]);
+            }
+            double a = (double)xs[r] * (double)w1s[c] * sa;
+            double g = (double)xs[r] * (double)w3s[c] * sg;
+            h[(size_t)r * I + c] = float_to_bf16_bits((float)(a / (1.0 + exp(-a)) * g));
+        }
+    }
+}
+
+/* Down projection of one FP8 expert on n quantized rows of h:
+ *   o[r][j] = hs[r] * w2s[j] * sum_c dec(hq[r][c]) dec(w2q(j, c))   (double)
+ * hq [n][K]; w2q is [d][K] stored as nseg blocks of kseg columns (K = nseg*kseg). */
+void orc_expert_down_fp8(const uint8_t* hq, const float* hs, int n, const uint8_t* w2q, const float* w2s, int d,
+                         int kseg, int nseg, double* o) {
+    int K = kseg * nseg;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < n; ++r) {
+        for (int j = 0; j < d; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < K; ++c)
+                acc += orc_e4m3_decode(hq[(size_t)r * K + c]) * orc_e4m3_decode(w2q[seg_index(j, c, d, kseg)]);
+            o[(size_t)r * d + j] = (double)hs[r] * (double)w2s[j] * acc;
+        }
+    }
+}
