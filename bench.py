@@ -46,7 +46,11 @@ if ROOT not in sys.path:
 METRIC = "MoE layer fwd tokens/s (V3-shaped, bf16) and % of BF16 tensor / HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES = ["route", "permute", "ffn_up", "ffn_down", "combine", "bias_update"]
+# E4M3 expert workloads: token rows and h are quantized per row in the step
+STAGES_FP8 = ["route", "quant_x", "permute", "ffn_up", "quant_h", "ffn_down", "combine", "bias_update"]
 DOMINANT = "ffn_up"
+WORKLOADS = ["v3_prefill", "v3_decode", "small_bf16", "skew_stress", "tiny_fp32", "v3_prefill_fp8",
+             "v3_decode_fp8", "small_fp8"]
 
 
 def parse_args():
@@ -54,8 +58,7 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="v3_prefill",
-                    choices=["v3_prefill", "v3_decode", "small_bf16", "skew_stress", "tiny_fp32"])
+    ap.add_argument("--workload", default="v3_prefill", choices=WORKLOADS)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -136,7 +139,8 @@ class ClockSampler:
 
 # ------------------------------------------------------------ oracle leg
 
-DEFAULT_CPU_TOKENS = {"v3_prefill": 12, "v3_decode": 12, "skew_stress": 12, "small_bf16": 48, "tiny_fp32": 128}
+DEFAULT_CPU_TOKENS = {"v3_prefill": 12, "v3_decode": 12, "skew_stress": 12, "small_bf16": 48, "tiny_fp32": 128,
+                      "v3_prefill_fp8": 12, "v3_decode_fp8": 12, "small_fp8": 48}
 
 
 def oracle_sample(cfg, p, x, n_tok):
@@ -174,6 +178,55 @@ def oracle_sample(cfg, p, x, n_tok):
     secs += time.perf_counter() - t0
     threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or len(os.sched_getaffinity(0))
     return secs, n_tok, threads
+
+
+def oracle_sample_fp8(cfg, p, x, n_tok):
+    """oracle_sample for the E4M3 expert workloads: routing, per-token
+    quantization of x, and for every expert the tokens use (and the shared
+    experts) the FP8 gate/up, per-row quantization of h and the FP8 down.
+    The expert weights are quantized by the oracle itself, expert by expert,
+    before the clock starts; only the forward's oracle arithmetic is timed."""
+    import numpy as np
+    import oracle
+    from fine_grained_moe_gate_b200.inputs import to_numpy
+
+    oracle.build()
+    xs = to_numpy(x[:n_tok])
+    wg = to_numpy(p["w_gate"])
+    bias = p["bias"].detach().cpu().numpy()
+    d, I, S, Is = cfg.d, cfg.I, cfg.S, cfg.Is
+    t0 = time.perf_counter()
+    s = oracle.affinity(xs, wg)
+    idx, w = oracle.select(s, bias, cfg.k)
+    xq, xsc = oracle.quantize_rows_fp8(xs)
+    secs = time.perf_counter() - t0
+    yacc = np.zeros((n_tok, d), np.float64)
+    if S > 0:
+        q1, s1 = oracle.quantize_rows_fp8(to_numpy(p["ws1"]).reshape(S * Is, d))
+        q3, s3 = oracle.quantize_rows_fp8(to_numpy(p["ws3"]).reshape(S * Is, d))
+        q2, s2 = oracle.quantize_rows_fp8(to_numpy(p["ws2"]), nseg=S)
+        t0 = time.perf_counter()
+        hq, hsc = oracle.quantize_rows_fp8(oracle.expert_up_fp8(xq, xsc, q1, s1, q3, s3))
+        yacc += oracle.expert_down_fp8(hq, hsc, q2, s2)
+        secs += time.perf_counter() - t0
+    for e in np.unique(idx):
+        ii, jj = np.nonzero(idx == e)
+        q1, s1 = oracle.quantize_rows_fp8(to_numpy(p["w1"][e]))
+        q3, s3 = oracle.quantize_rows_fp8(to_numpy(p["w3"][e]))
+        q2, s2 = oracle.quantize_rows_fp8(to_numpy(p["w2"][e]))
+        t0 = time.perf_counter()
+        hq, hsc = oracle.quantize_rows_fp8(oracle.expert_up_fp8(xq[ii], xsc[ii], q1, s1, q3, s3))
+        yacc[ii] += w[ii, jj].astype(np.float64)[:, None] * oracle.expert_down_fp8(hq, hsc, q2, s2)
+        secs += time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.finalize(yacc, xs.dtype)
+    secs += time.perf_counter() - t0
+    threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or len(os.sched_getaffinity(0))
+    return secs, n_tok, threads
+
+
+def run_oracle_sample(cfg, p, x, n_tok):
+    return (oracle_sample_fp8 if cfg.dtype == "fp8" else oracle_sample)(cfg, p, x, n_tok)
 
 
 def cpu_baseline_record(cfg, secs, n_tok, threads, label):
@@ -237,6 +290,12 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream()
 
     p = make_layer(cfg, dev)
+    fp8 = cfg.dtype == "fp8"
+    stages = STAGES_FP8 if fp8 else STAGES
+    if fp8:  # E4M3 expert weights, quantized once per output row before timing
+        q8 = moe.quantize_experts_fp8(p)
+        w8 = moe.fp8_experts(q8)
+        torch.cuda.synchronize()
     n_x = max(1, min(4, args.steps + args.warmup))
     xs = [make_tokens(cfg, dev, step=mdist.shard_step(i, rank, world)) for i in range(n_x)]
 
@@ -254,6 +313,40 @@ def run_ours(args, world, rank, local):
     hs = torch.empty((T, max(1, cfg.S * cfg.Is)), dtype=dt, device=dev)
     shared_out = torch.empty((T, d), dtype=dt, device=dev) if cfg.S > 0 else None
     y = torch.empty((T, d), dtype=dt, device=dev)
+    if fp8:
+        SIs = max(1, cfg.S * cfg.Is)
+        xq = torch.empty((T, d), dtype=torch.uint8, device=dev)
+        xsc = torch.empty(T, dtype=torch.float32, device=dev)
+        xq_perm = torch.empty((T * k, d), dtype=torch.uint8, device=dev)
+        hq = torch.empty((T * k, cfg.I), dtype=torch.uint8, device=dev)
+        h_sc = torch.empty(T * k, dtype=torch.float32, device=dev)
+        hsq = torch.empty((T, SIs), dtype=torch.uint8, device=dev)
+        hs_sc = torch.empty(T, dtype=torch.float32, device=dev)
+
+    def step_fp8(i, ev=None):
+        x = xs[i % n_x]
+        rec = (lambda j: ev[j].record(stream)) if ev is not None else (lambda j: None)
+        sh_ = cfg.S > 0
+        rec(0)
+        moe.moe_route(x, p["w_gate"], p["bias"], sh, idx, w, counts, None, stream)
+        rec(1)
+        moe.moe_quantize_fp8(x, T, d, 1, xq, xsc, stream)
+        rec(2)
+        moe.moe_permute(xq, idx, counts, sh, xq_perm, offsets, perm, inv, pws, stream)
+        rec(3)
+        moe.moe_ffn_up_fp8(xq_perm, perm, xsc, offsets, xq if sh_ else None, w8, sh, h, hs if sh_ else None, stream)
+        rec(4)
+        moe.moe_quantize_fp8(h, T * k, cfg.I, 1, hq, h_sc, stream)
+        if sh_:
+            moe.moe_quantize_fp8(hs, T, cfg.S * cfg.Is, 1, hsq, hs_sc, stream)
+        rec(5)
+        moe.moe_ffn_down_fp8(hq, h_sc, offsets, hsq if sh_ else None, hs_sc, w8, sh, x_perm, shared_out, stream)
+        rec(6)
+        moe.moe_combine(x_perm, w, inv, shared_out, sh, y, stream)
+        rec(7)
+        mdist.allreduce_counts(counts)
+        moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
+        rec(8)
 
     def step(i, ev=None):
         x = xs[i % n_x]
@@ -274,6 +367,9 @@ def run_ours(args, world, rank, local):
         moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
         rec(6)
 
+    if fp8:
+        step = step_fp8
+
     def barrier():
         if world > 1:
             dist.barrier()
@@ -290,7 +386,7 @@ def run_ours(args, world, rank, local):
     if vis:
         gpu_id = vis.split(",")[local].strip()
     clocks = ClockSampler(gpu_id)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     clocks.start()
@@ -307,7 +403,7 @@ def run_ours(args, world, rank, local):
         raise moe.MoEError(st, "timed steps")
     ms_local = start.elapsed_time(end)
     stage_ms = {}
-    for j, name in enumerate(STAGES):
+    for j, name in enumerate(stages):
         stage_ms[name] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
     t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
     if world > 1:
@@ -326,8 +422,11 @@ def run_ours(args, world, rank, local):
 
         def e2e_step(i):
             x_dev.copy_(x_host[i % n_x], non_blocking=True)
-            moe.moe_layer_forward(x_dev, p["w_gate"], p["bias"], p["w1"], p["w3"], p["w2"], p["ws1"], p["ws3"],
-                                  p["ws2"], sh, y, idx, w, counts, ws, stream)
+            if fp8:
+                moe.moe_layer_forward_fp8(x_dev, p["w_gate"], p["bias"], w8, sh, y, idx, w, counts, ws, stream)
+            else:
+                moe.moe_layer_forward(x_dev, p["w_gate"], p["bias"], p["w1"], p["w3"], p["w2"], p["ws1"], p["ws3"],
+                                      p["ws2"], sh, y, idx, w, counts, ws, stream)
             mdist.allreduce_counts(counts)
             moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
             y_host.copy_(y, non_blocking=True)
@@ -366,8 +465,12 @@ def run_ours(args, world, rank, local):
         moe.moe_route(xx, p["w_gate"], p["bias"], sh, idx, w, counts, None, stream)
         touched.append(int((counts > 0).sum().item()))
     n_touched = statistics.mean(touched)
-    esz = 2 if cfg.dtype == "bf16" else 4
-    bytes_per_launch = (n_touched * 2 * cfg.I * d + T * k * (d + cfg.I) + 2 * SIs * d + T * (d + SIs)) * esz
+    esz = {"bf16": 2, "fp8": 1}.get(cfg.dtype, 4)
+    if fp8:  # E4M3 weights and token rows in, bf16 h out
+        bytes_per_launch = (n_touched * 2 * cfg.I * d + 2 * SIs * d + T * k * d + T * d) + \
+            (T * k * cfg.I + T * SIs) * 2
+    else:
+        bytes_per_launch = (n_touched * 2 * cfg.I * d + T * k * (d + cfg.I) + 2 * SIs * d + T * (d + SIs)) * esz
     hbm_gbs = bytes_per_launch / (dom_ms / 1e3) / 1e9
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     traffic = traffic_record(os.path.join(ROOT, "fine_grained_moe_gate_b200", "csrc", "gemm_tc.cu"), cfg.name)
@@ -376,12 +479,20 @@ def run_ours(args, world, rank, local):
                 "frac_of_nominal_8000": round(hbm_gbs / 8000.0, 4),
                 "traffic": traffic, "bytes_per_launch": int(bytes_per_launch), "experts_touched": n_touched,
                 "peak_kind": f"hbm_gbs ({peak_src}, copy bandwidth)"}
+    bf16_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     if cfg.dtype == "bf16":
-        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        peak = bf16_sus
         roof = {"bound": "tensor", "kernel": "tc_grouped_gemm_kernel<up> (routed + shared experts, SwiGLU epilogue)",
                 "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "traffic": traffic,
                 "peak_kind": f"bf16_tflops_sustained ({peak_src}): the kernel is timed inside a long step",
+                "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
+    elif fp8:
+        peak = 2.0 * bf16_sus  # nominal dense E4M3 / bf16 ratio 4.5 / 2.25 times the measured bf16 figure
+        roof = {"bound": "tensor", "kernel": "tc_grouped_gemm_kernel<up, E4M3> (routed + shared experts)",
+                "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": traffic,
+                "peak_kind": f"2 x bf16_tflops_sustained ({peak_src}; nominal fp8/bf16 dense ratio 4.5/2.25)",
                 "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
     else:
         roof = {"bound": "alu", "kernel": "simt_grouped_gemm_kernel (fp32 FFMA; routed and shared launches)", "achieved": round(achieved, 3),
@@ -396,7 +507,7 @@ def run_ours(args, world, rank, local):
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         n_tok = args.cpu_tokens or DEFAULT_CPU_TOKENS[args.workload]
-        secs, n, threads = oracle_sample(cfg, p, xs[0], min(n_tok, T))
+        secs, n, threads = run_oracle_sample(cfg, p, xs[0], min(n_tok, T))
         cpu = cpu_baseline_record(cfg, secs, n, threads, "oracle sample")
 
     if rank == 0:
@@ -404,17 +515,18 @@ def run_ours(args, world, rank, local):
             "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
-            "data": "synthetic (seeded N(0,1) tokens, N(0,std) weights of the stated shape)",
+            "data": "synthetic (seeded N(0,1) tokens, N(0,std) weights of the stated shape"
+                    + ("; expert weights quantized to E4M3 per output row before timing)" if fp8 else ")"),
             "config": {"workload": cfg.name, "T_per_gpu": T, "global_batch": T * world, "d": d, "E": E, "k": k,
                        "I": cfg.I, "S": cfg.S, "Is": cfg.Is, "parallelism": f"dp{world}",
                        "l2": "inputs larger than L2: layer weights read every step "
-                             f"({(p['w1'].numel() * 3 + p['ws1'].numel() * 3) * p['w1'].element_size() / 1e9:.1f} GB)",
+                             f"({(p['w1'].numel() * 3 + p['ws1'].numel() * 3) * esz / 1e9:.1f} GB)",
                        "bias_update": "every step"},
             "roofline": roof,
             "roofline_alt": roof_hbm,
             "layer_tflops": round(step_tflops, 2),
-            "layer_frac_of_peak": round(step_tflops / float(peaks.get("bf16_tflops_sustained", 1400.0)), 4)
-            if cfg.dtype == "bf16" else None,
+            "layer_frac_of_peak": round(step_tflops / (bf16_sus * (2.0 if fp8 else 1.0)), 4)
+            if cfg.dtype in ("bf16", "fp8") else None,
             "stages_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -445,10 +557,10 @@ def run_reference(args, world, rank, local):
     n_tok = args.cpu_tokens or max(2, DEFAULT_CPU_TOKENS[args.workload] // 3)
     n_tok = min(n_tok, cfg.T)
     for _ in range(args.warmup):
-        oracle_sample(cfg, p, x, n_tok)
+        run_oracle_sample(cfg, p, x, n_tok)
     total, threads = 0.0, 1
     for _ in range(args.steps):
-        secs, n, threads = oracle_sample(cfg, p, x, n_tok)
+        secs, n, threads = run_oracle_sample(cfg, p, x, n_tok)
         total += secs
     value = n_tok * args.steps / total
     rec = cpu_baseline_record(cfg, total, n_tok * args.steps, threads, "reference arm (oracle)")

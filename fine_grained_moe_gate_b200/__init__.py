@@ -33,9 +33,11 @@ EXPORTS = (
     "moe_grouped_swiglu", "moe_grouped_swiglu_workspace_size", "moe_expert_up", "moe_expert_down", "moe_ffn_up",
     "moe_ffn_down", "moe_combine", "moe_layer_forward", "moe_workspace_size", "moe_get_last_error",
     "moe_kernel_launch_count", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
+    "moe_quantize_fp8", "moe_ffn_up_fp8", "moe_ffn_down_fp8", "moe_layer_forward_fp8",
 )
 
 MOE_ROUTED, MOE_SHARED = 0, 1
+MOE_F32, MOE_BF16, MOE_FP8_E4M3 = 0, 1, 2
 
 
 class MoEError(RuntimeError):
@@ -55,7 +57,23 @@ class MoEShape(ctypes.Structure):
 def shape_of(cfg, T: int | None = None) -> MoEShape:
     """MoEShape from a workload config (``inputs.MoEConfig``)."""
     return MoEShape(cfg.T if T is None else T, cfg.d, cfg.E, cfg.k, cfg.I, cfg.S, cfg.Is,
-                    MOE_BF16 if cfg.dtype == "bf16" else MOE_F32)
+                    {"bf16": MOE_BF16, "fp8": MOE_FP8_E4M3}.get(cfg.dtype, MOE_F32))
+
+
+class MoEFp8Experts(ctypes.Structure):
+    """moe_fp8_experts: E4M3 expert weights and their per-row fp32 scales."""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "w1_scale", "w3", "w3_scale", "w2", "w2_scale",
+                                               "ws1", "ws1_scale", "ws3", "ws3_scale", "ws2", "ws2_scale")]
+
+
+def fp8_experts(q: dict) -> MoEFp8Experts:
+    """MoEFp8Experts from a dict of device tensors with keys w1q, w1s, ... (the
+    layout of ``quantize_experts_fp8``).  The tensors must outlive its use."""
+    f = {}
+    for n in ("w1", "w3", "w2", "ws1", "ws3", "ws2"):
+        f[n] = _p(q.get(n + "q"))
+        f[n + "_scale"] = _p(q.get(n + "s"))
+    return MoEFp8Experts(**f)
 
 
 _lib = None
@@ -83,6 +101,10 @@ def lib() -> ctypes.CDLL:
             "moe_combine": [P, P, P, P, S, P, P],
             "moe_layer_forward": [P, P, P, P, P, P, P, P, P, S, P, P, P, P, P, sz, P],
             "moe_get_last_error": [P],
+            "moe_quantize_fp8": [P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, P, P, P],
+            "moe_ffn_up_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
+            "moe_ffn_down_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
+            "moe_layer_forward_fp8": [P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P, P, P, sz, P],
             "moe_selftest_bounded_wait": [ctypes.c_uint32, P],
         }
         for name, args in sig.items():
@@ -224,3 +246,51 @@ def moe_status_string(status: int) -> str:
 
 def moe_abi_version() -> int:
     return lib().moe_abi_version()
+
+
+# ---- FP8 experts -------------------------------------------------------------
+
+def moe_quantize_fp8(src, rows, kseg, nseg, q, scale, stream=None):
+    _check(lib().moe_quantize_fp8(_p(src), rows, kseg, nseg, _p(q), _p(scale), _stream(stream)), "moe_quantize_fp8")
+
+
+def moe_ffn_up_fp8(xq_perm, perm_tok, x_scale, offsets, xq, experts, shape, h, hs, stream=None):
+    _check(lib().moe_ffn_up_fp8(_p(xq_perm), _p(perm_tok), _p(x_scale), _p(offsets), _p(xq), ctypes.byref(experts),
+                                shape, _p(h), _p(hs), _stream(stream)), "moe_ffn_up_fp8")
+
+
+def moe_ffn_down_fp8(hq, h_scale, offsets, hsq, hs_scale, experts, shape, y_perm, shared_out, stream=None):
+    _check(lib().moe_ffn_down_fp8(_p(hq), _p(h_scale), _p(offsets), _p(hsq), _p(hs_scale), ctypes.byref(experts),
+                                  shape, _p(y_perm), _p(shared_out), _stream(stream)), "moe_ffn_down_fp8")
+
+
+def moe_layer_forward_fp8(x, w_gate, bias, experts, shape, y, topk_idx, topk_w, counts, workspace, stream=None):
+    _check(lib().moe_layer_forward_fp8(_p(x), _p(w_gate), _p(bias), ctypes.byref(experts), shape, _p(y),
+                                       _p(topk_idx), _p(topk_w), _p(counts), _p(workspace), _nbytes(workspace),
+                                       _stream(stream)), "moe_layer_forward_fp8")
+
+
+def quantize_experts_fp8(p: dict, stream=None) -> dict:
+    """E4M3 copies of a layer's bf16 expert weights (device tensors) through
+    moe_quantize_fp8: per output row for W1/W3/W2 and the shared Ws1/Ws3; the
+    shared Ws2 [S][d][Is] per output row across its S blocks.  Returns uint8
+    codes and fp32 scales under w1q, w1s, ... (the weights' own shapes)."""
+    import torch
+    out = {}
+    for n in ("w1", "w3", "w2", "ws1", "ws3"):
+        w = p[n]
+        if w.numel() == 0:
+            continue
+        rows, K = w.numel() // w.shape[-1], w.shape[-1]
+        q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+        sc = torch.empty(rows, dtype=torch.float32, device=w.device)
+        moe_quantize_fp8(w, rows, K, 1, q, sc, stream)
+        out[n + "q"], out[n + "s"] = q, sc
+    w = p["ws2"]
+    if w.numel() > 0:
+        S, d, Is = w.shape
+        q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+        sc = torch.empty(d, dtype=torch.float32, device=w.device)
+        moe_quantize_fp8(w, d, Is, S, q, sc, stream)
+        out["ws2q"], out["ws2s"] = q, sc
+    return out

@@ -39,11 +39,13 @@ moe_status device_setup(int* dev_out, int** status_out, int* sms_out) {
 }
 
 inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
-inline size_t esize(const moe_shape& sh) { return sh.dtype == MOE_BF16 ? 2 : 4; }
+// bytes per element of the token rows moe_permute moves (E4M3 rows for MOE_FP8_E4M3)
+inline size_t esize(const moe_shape& sh) { return sh.dtype == MOE_F32 ? 4 : sh.dtype == MOE_BF16 ? 2 : 1; }
+inline bool is_fp8(const moe_shape& sh) { return sh.dtype == MOE_FP8_E4M3; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 moe_status validate_shape(const moe_shape& sh) {
-    if (sh.dtype != MOE_F32 && sh.dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (sh.dtype != MOE_F32 && sh.dtype != MOE_BF16 && sh.dtype != MOE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
     if (sh.T < 0 || sh.d <= 0 || sh.E <= 0 || sh.k <= 0 || sh.I <= 0 || sh.S < 0) return MOE_ERR_INVALID_ARG;
     if (sh.S > 0 && sh.Is <= 0) return MOE_ERR_INVALID_ARG;
     if (sh.k > sh.E) return MOE_ERR_INVALID_ARG;
@@ -51,11 +53,18 @@ moe_status validate_shape(const moe_shape& sh) {
     if (sh.d % 8 != 0) return MOE_ERR_UNSUPPORTED;
     // 32-bit row coordinates (tensor maps, row indices)
     if ((long long)sh.T * sh.k >= (1ll << 31) || (long long)sh.E * sh.I >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
-    if (sh.dtype == MOE_BF16) {
-        if (sh.d % 64 != 0 || sh.I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (sh.dtype != MOE_F32) {
+        if (sh.d % (is_fp8(sh) ? 128 : 64) != 0 || sh.I % 128 != 0) return MOE_ERR_UNSUPPORTED;
         if (sh.S > 0 && sh.Is % 128 != 0) return MOE_ERR_UNSUPPORTED;
     }
     return MOE_OK;
+}
+
+// Calls that take bf16 (or fp32) expert weights.
+moe_status validate_dense_weights(const moe_shape& sh) {
+    const moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    return is_fp8(sh) ? MOE_ERR_UNSUPPORTED : MOE_OK;
 }
 
 #define MOE_REQUIRE(cond, code) \
@@ -81,7 +90,7 @@ moe_status do_route(const void* x, const void* w_gate, const float* bias, const 
     MOE_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * sh.E, st));
     if (sh.T == 0) return MOE_OK;
     cudaError_t err;
-    if (sh.dtype == MOE_BF16)
+    if (sh.dtype != MOE_F32)  // x and W_gate are bf16 for MOE_FP8_E4M3 too
         err = moe::launch_router_tc(x, w_gate, bias, sh.T, sh.d, sh.E, sh.k, idx, w, counts, aff, status, sms, st);
     else
         err = moe::launch_router_simt(x, w_gate, bias, sh.T, sh.d, sh.E, sh.k, false, idx, w, counts, aff, status,
@@ -202,6 +211,109 @@ moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1,
     return do_ffn_down(h, offsets, w2, shared ? hs : nullptr, ws2, sh, y_perm, shared_out, status, sms, st);
 }
 
+// ---- FP8 experts -----------------------------------------------------------
+
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+moe_status do_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const float* xs, const int32_t* offsets,
+                         const uint8_t* xq, const moe_fp8_experts* w, const moe_shape& sh, void* h, void* hs,
+                         int* status, int sms, cudaStream_t st) {
+    if (sh.T == 0) return MOE_OK;
+    const bool shared = xq && sh.S > 0;
+    moe::TcUpArgs ur = tc_up_args(xq_perm, nullptr, offsets, w->w1, w->w3, sh, false, h);
+    ur.f8 = true;
+    ur.w1s = w->w1_scale;
+    ur.w3s = w->w3_scale;
+    ur.xs = xs;
+    ur.xs_idx = perm_tok;  // row r holds token perm_tok[r] / k
+    ur.xs_div = sh.k;
+    moe::TcUpArgs us = tc_up_args(xq, nullptr, nullptr, w->ws1, w->ws3, sh, true, hs);
+    us.f8 = true;
+    us.w1s = w->ws1_scale;
+    us.w3s = w->ws3_scale;
+    us.xs = xs;
+    return moe::launch_tc_up(&ur, shared ? &us : nullptr, status, sms, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status do_ffn_down_fp8(const uint8_t* hq, const float* h_scale, const int32_t* offsets, const uint8_t* hsq,
+                           const float* hs_scale, const moe_fp8_experts* w, const moe_shape& sh, void* y_perm,
+                           void* shared_out, int* status, int sms, cudaStream_t st) {
+    if (sh.T == 0) return MOE_OK;
+    const bool shared = hsq && sh.S > 0;
+    moe::TcDownArgs dr = tc_down_args(hq, offsets, w->w2, sh, false, y_perm);
+    dr.f8 = true;
+    dr.w2s = w->w2_scale;
+    dr.hs = h_scale;
+    moe::TcDownArgs ds = tc_down_args(hsq, nullptr, w->ws2, sh, true, shared_out);
+    ds.f8 = true;
+    ds.w2s = w->ws2_scale;
+    ds.hs = hs_scale;
+    return moe::launch_tc_down(&dr, shared ? &ds : nullptr, status, sms, st) == cudaSuccess ? MOE_OK
+                                                                                              : MOE_ERR_CUDA;
+}
+
+bool fp8_weights_ok(const moe_fp8_experts* w, const moe_shape& sh) {
+    if (!w || !w->w1 || !w->w3 || !w->w2 || !w->w1_scale || !w->w3_scale || !w->w2_scale) return false;
+    if (sh.S > 0 && (!w->ws1 || !w->ws3 || !w->ws2 || !w->ws1_scale || !w->ws3_scale || !w->ws2_scale)) return false;
+    return true;
+}
+
+bool fp8_weights_aligned(const moe_fp8_experts* w) {
+    return aligned16(w->w1) && aligned16(w->w3) && aligned16(w->w2) && aligned16(w->ws1) && aligned16(w->ws3) &&
+           aligned16(w->ws2) && aligned4(w->w1_scale) && aligned4(w->w3_scale) && aligned4(w->w2_scale) &&
+           aligned4(w->ws1_scale) && aligned4(w->ws3_scale) && aligned4(w->ws2_scale);
+}
+
+// Workspace of moe_layer_forward_fp8, carved in this order.
+struct Fp8Work {
+    int32_t* offsets;
+    int32_t* perm;
+    int32_t* inv;
+    void* pws;
+    uint8_t* xq;
+    float* xs;
+    uint8_t* xq_perm;
+    void* h;
+    void* hs;
+    uint8_t* hq;
+    float* h_scale;
+    uint8_t* hsq;
+    float* hs_scale;
+    void* y_perm;
+    void* shared_out;
+};
+
+size_t fp8_work(const moe_shape& sh, char* base, Fp8Work* o) {
+    const size_t T = (size_t)sh.T, rows = T * sh.k, SI = (size_t)sh.S * sh.Is, d = (size_t)sh.d, I = (size_t)sh.I;
+    const size_t sizes[15] = {(size_t)(sh.E + 1) * 4, rows * 4, rows * 4, permute_ws(sh), T * d, T * 4,
+                              rows * d, rows * I * 2, T * SI * 2, rows * I, rows * 4, T * SI, T * 4,
+                              rows * d * 2, T * d * 2};
+    void* ptrs[15];
+    size_t off = 0;
+    for (int i = 0; i < 15; ++i) {
+        ptrs[i] = base ? base + off : nullptr;
+        off += align256(sizes[i]);
+    }
+    if (o) {
+        o->offsets = static_cast<int32_t*>(ptrs[0]);
+        o->perm = static_cast<int32_t*>(ptrs[1]);
+        o->inv = static_cast<int32_t*>(ptrs[2]);
+        o->pws = ptrs[3];
+        o->xq = static_cast<uint8_t*>(ptrs[4]);
+        o->xs = static_cast<float*>(ptrs[5]);
+        o->xq_perm = static_cast<uint8_t*>(ptrs[6]);
+        o->h = ptrs[7];
+        o->hs = ptrs[8];
+        o->hq = static_cast<uint8_t*>(ptrs[9]);
+        o->h_scale = static_cast<float*>(ptrs[10]);
+        o->hsq = static_cast<uint8_t*>(ptrs[11]);
+        o->hs_scale = static_cast<float*>(ptrs[12]);
+        o->y_perm = ptrs[13];
+        o->shared_out = ptrs[14];
+    }
+    return off;
+}
+
 }  // namespace
 
 namespace moe {
@@ -234,12 +346,13 @@ size_t moe_permute_workspace_size(moe_shape sh) {
 }
 
 size_t moe_grouped_swiglu_workspace_size(moe_shape sh) {
-    if (validate_shape(sh) != MOE_OK) return 0;
+    if (validate_dense_weights(sh) != MOE_OK) return 0;
     return swiglu_ws(sh);
 }
 
 size_t moe_workspace_size(moe_shape sh) {
     if (validate_shape(sh) != MOE_OK) return 0;
+    if (is_fp8(sh)) return fp8_work(sh, nullptr, nullptr);
     const size_t rows = (size_t)sh.T * sh.k;
     return align256((sh.E + 1) * sizeof(int32_t)) + 2 * align256(rows * sizeof(int32_t)) + permute_ws(sh) +
            align256(rows * sh.d * esize(sh)) + swiglu_ws(sh) + align256((size_t)sh.T * sh.d * esize(sh));
@@ -305,7 +418,7 @@ moe_status moe_grouped_swiglu(const void* x_perm, const int32_t* offsets, const 
                               const void* w2, const void* x, const void* ws1, const void* ws3, const void* ws2,
                               moe_shape sh, void* y_perm, void* shared_out, void* workspace, size_t ws_bytes,
                               void* stream) {
-    moe_status v = validate_shape(sh);
+    moe_status v = validate_dense_weights(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(offsets && w1 && w3 && w2, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(sh.T == 0 || (x_perm && y_perm), MOE_ERR_INVALID_ARG);
@@ -327,7 +440,7 @@ moe_status moe_grouped_swiglu(const void* x_perm, const int32_t* offsets, const 
 
 moe_status moe_expert_up(const void* a, const int32_t* gather_idx, const int32_t* offsets, const void* w1,
                          const void* w3, moe_shape sh, int32_t set, void* h, void* stream) {
-    moe_status v = validate_shape(sh);
+    moe_status v = validate_dense_weights(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(set == MOE_ROUTED || set == MOE_SHARED, MOE_ERR_INVALID_ARG);
     const bool shared = set == MOE_SHARED;
@@ -348,7 +461,7 @@ moe_status moe_expert_up(const void* a, const int32_t* gather_idx, const int32_t
 
 moe_status moe_expert_down(const void* h, const int32_t* offsets, const void* w2, moe_shape sh, int32_t set, void* y,
                            void* stream) {
-    moe_status v = validate_shape(sh);
+    moe_status v = validate_dense_weights(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(set == MOE_ROUTED || set == MOE_SHARED, MOE_ERR_INVALID_ARG);
     const bool shared = set == MOE_SHARED;
@@ -365,7 +478,7 @@ moe_status moe_expert_down(const void* h, const int32_t* offsets, const void* w2
 
 moe_status moe_ffn_up(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3, const void* x,
                       const void* ws1, const void* ws3, moe_shape sh, void* h, void* hs, void* stream) {
-    moe_status v = validate_shape(sh);
+    moe_status v = validate_dense_weights(sh);
     if (v != MOE_OK) return v;
     const bool shared = x != nullptr && sh.S > 0;
     MOE_REQUIRE(offsets && w1 && w3, MOE_ERR_INVALID_ARG);
@@ -384,7 +497,7 @@ moe_status moe_ffn_up(const void* x_perm, const int32_t* offsets, const void* w1
 
 moe_status moe_ffn_down(const void* h, const int32_t* offsets, const void* w2, const void* hs, const void* ws2,
                         moe_shape sh, void* y_perm, void* shared_out, void* stream) {
-    moe_status v = validate_shape(sh);
+    moe_status v = validate_dense_weights(sh);
     if (v != MOE_OK) return v;
     const bool shared = hs != nullptr && sh.S > 0;
     MOE_REQUIRE(offsets && w2, MOE_ERR_INVALID_ARG);
@@ -412,7 +525,7 @@ moe_status moe_combine(const void* y_perm, const float* topk_w, const int32_t* i
     int* status;
     v = device_setup(&dev, &status, &sms);
     if (v != MOE_OK) return v;
-    return moe::launch_combine(y_perm, topk_w, inv_row, shared_out, sh.T, sh.d, sh.k, sh.dtype == MOE_BF16, y, status,
+    return moe::launch_combine(y_perm, topk_w, inv_row, shared_out, sh.T, sh.d, sh.k, sh.dtype != MOE_F32, y, status,
                                static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
@@ -422,7 +535,7 @@ moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bia
                              const void* w2, const void* ws1, const void* ws3, const void* ws2, moe_shape sh, void* y,
                              int32_t* topk_idx, float* topk_w, int32_t* counts, void* workspace, size_t ws_bytes,
                              void* stream) {
-    moe_status v = validate_shape(sh);
+    moe_status v = validate_dense_weights(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(w_gate && bias && w1 && w3 && w2 && counts, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(sh.S == 0 || (ws1 && ws3 && ws2), MOE_ERR_INVALID_ARG);
@@ -467,8 +580,110 @@ moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bia
     if ((v = do_swiglu(x_perm, offsets, w1, w3, w2, sh.S > 0 ? x : nullptr, ws1, ws3, ws2, sh, y_perm, shared_out,
                        gws, status, sms, st)) != MOE_OK)
         return v;
-    return moe::launch_combine(y_perm, topk_w, inv, shared_out, sh.T, sh.d, sh.k, sh.dtype == MOE_BF16, y, status,
+    return moe::launch_combine(y_perm, topk_w, inv, shared_out, sh.T, sh.d, sh.k, sh.dtype != MOE_F32, y, status,
                                st) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t kseg, int32_t nseg, uint8_t* q, float* scale,
+                            void* stream) {
+    MOE_REQUIRE(rows >= 0 && kseg > 0 && nseg >= 1, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(kseg % 8 == 0, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE((long long)kseg * nseg < (1ll << 31), MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(rows == 0 || (src && q && scale), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(src) && aligned16(q) && aligned4(scale), MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    moe_status v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return moe::launch_quantize_e4m3(src, rows, kseg, nseg, q, scale, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const float* x_scale,
+                          const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w, moe_shape sh, void* h,
+                          void* hs, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(is_fp8(sh), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(offsets && fp8_weights_ok(w, sh), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (xq_perm && perm_tok && x_scale && h), MOE_ERR_INVALID_ARG);
+    const bool shared = xq != nullptr && sh.S > 0;
+    MOE_REQUIRE(!shared || sh.T == 0 || hs, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(xq_perm) && aligned16(perm_tok) && aligned4(x_scale) && aligned16(offsets) &&
+                    aligned16(xq) && aligned16(h) && aligned16(hs) && fp8_weights_aligned(w),
+                MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_ffn_up_fp8(xq_perm, perm_tok, x_scale, offsets, shared ? xq : nullptr, w, sh, h, hs, status, sms,
+                         static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_ffn_down_fp8(const uint8_t* hq, const float* h_scale, const int32_t* offsets, const uint8_t* hsq,
+                            const float* hs_scale, const moe_fp8_experts* w, moe_shape sh, void* y_perm,
+                            void* shared_out, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(is_fp8(sh), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(offsets && fp8_weights_ok(w, sh), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (hq && h_scale && y_perm), MOE_ERR_INVALID_ARG);
+    const bool shared = hsq != nullptr && sh.S > 0;
+    MOE_REQUIRE(!shared || sh.T == 0 || (hs_scale && shared_out), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(hq) && aligned4(h_scale) && aligned16(offsets) && aligned16(hsq) && aligned4(hs_scale) &&
+                    aligned16(y_perm) && aligned16(shared_out) && fp8_weights_aligned(w),
+                MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_ffn_down_fp8(hq, h_scale, offsets, shared ? hsq : nullptr, hs_scale, w, sh, y_perm, shared_out, status,
+                           sms, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float* bias, const moe_fp8_experts* w,
+                                 moe_shape sh, void* y, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(is_fp8(sh), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(w_gate && bias && counts && fp8_weights_ok(w, sh), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (x && y && topk_idx && topk_w), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x) && aligned16(w_gate) && aligned16(bias) && aligned16(y) && aligned16(topk_idx) &&
+                    aligned16(topk_w) && aligned16(counts) && fp8_weights_aligned(w),
+                MOE_ERR_ALIGNMENT);
+    MOE_REQUIRE(workspace && ws_bytes >= fp8_work(sh, nullptr, nullptr), MOE_ERR_WORKSPACE);
+    MOE_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Fp8Work k8;
+    fp8_work(sh, static_cast<char*>(workspace), &k8);
+    const bool shared = sh.S > 0;
+    if ((v = do_route(x, w_gate, bias, sh, topk_idx, topk_w, counts, nullptr, status, sms, st)) != MOE_OK) return v;
+    if (sh.T == 0) return MOE_OK;
+    if (moe::launch_quantize_e4m3(x, sh.T, sh.d, 1, k8.xq, k8.xs, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((v = do_permute(k8.xq, topk_idx, counts, sh, k8.xq_perm, k8.offsets, k8.perm, k8.inv, k8.pws, status, st)) !=
+        MOE_OK)
+        return v;
+    if ((v = do_ffn_up_fp8(k8.xq_perm, k8.perm, k8.xs, k8.offsets, shared ? k8.xq : nullptr, w, sh, k8.h, k8.hs,
+                           status, sms, st)) != MOE_OK)
+        return v;
+    if (moe::launch_quantize_e4m3(k8.h, (long long)sh.T * sh.k, sh.I, 1, k8.hq, k8.h_scale, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (shared && moe::launch_quantize_e4m3(k8.hs, sh.T, sh.S * sh.Is, 1, k8.hsq, k8.hs_scale, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if ((v = do_ffn_down_fp8(k8.hq, k8.h_scale, k8.offsets, shared ? k8.hsq : nullptr, k8.hs_scale, w, sh, k8.y_perm,
+                             k8.shared_out, status, sms, st)) != MOE_OK)
+        return v;
+    return moe::launch_combine(k8.y_perm, topk_w, k8.inv, shared ? k8.shared_out : nullptr, sh.T, sh.d, sh.k, true, y,
+                               status, st) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }

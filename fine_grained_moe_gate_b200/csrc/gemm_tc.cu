@@ -59,7 +59,10 @@
 namespace moe {
 namespace {
 
-constexpr int BK = 64;                  // K per stage: one 128-byte swizzle row of bf16
+constexpr int BK = 64;                  // bf16 K per stage: one 128-byte swizzle row
+// K elements per stage for the operand type: 64 bf16 or 128 E4M3 (128 bytes either way)
+template <bool F8>
+__host__ __device__ constexpr int bk_elems() { return F8 ? 128 : 64; }
 constexpr int STAGES = 6;
 constexpr int A_BYTES = 128 * BK * 2;   // this CTA's 128 weight rows
 constexpr int B_ROWS = 128;             // this CTA's half of <= 256 tokens
@@ -117,8 +120,6 @@ struct Tables {
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 2 * XBUF_BYTES + sizeof(Ctl) + sizeof(Tables);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// One expert set in a launch: set 0 = the routed experts (groups [0, G0),
-// rows from offsets), set 1 = the shared experts (group G0, rows [0, M)).
 // Tensor maps of one expert set: weights (w1 only for the up projection) and
 // the token operand with box heights 16 * (i + 1) rows.
 struct SetMaps {
@@ -126,6 +127,8 @@ struct SetMaps {
     CUtensorMap x[NXBOX];
 };
 
+// One expert set in a launch: set 0 = the routed experts (groups [0, G0),
+// rows from offsets), set 1 = the shared experts (group G0, rows [0, M)).
 struct SetParams {
     int f_tiles;       // feature tiles (per CTA pair) per group
     int k_blocks;
@@ -135,6 +138,15 @@ struct SetParams {
     int ldo;           // output row pitch (elements)
     int f_limit;       // valid output features
     long long a_rows;  // rows the groups may index (token operand rows, or gathered rows) = output rows
+    // E4M3 operands only: per-row scales.  Weight row scales (up: W1 rows in
+    // ws0, W3 rows in ws1; down: W2 rows in ws0), srows scale rows per group;
+    // token-row scale of operand row r: xscale[xidx ? xidx[r] / xdiv : r].
+    const float* ws0;
+    const float* ws1;
+    int srows;
+    const float* xscale;
+    const int32_t* xidx;
+    int xdiv;
 };
 struct Params {
     const int32_t* offsets;
@@ -171,6 +183,13 @@ __device__ __forceinline__ void token_tile(int rows, int ntt, int tt, int& start
     const int q = rows / ntt, r = rows - q * ntt;
     start = tt * q + min(tt, r);
     len = q + (tt < r ? 1 : 0);
+}
+
+__device__ __forceinline__ void scale4(float4& v, float s) {
+    v.x *= s;
+    v.y *= s;
+    v.z *= s;
+    v.w *= s;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -234,7 +253,7 @@ __device__ __forceinline__ bool tq_take(Ctl* ctl, int j, uint32_t ph, uint32_t l
     return true;
 }
 
-template <bool UP>
+template <bool UP, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ SetMaps ma, const __grid_constant__ SetMaps mb,
                            const __grid_constant__ CUtensorMap tmXg, const Params p) {
@@ -245,6 +264,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + 2 * XBUF_BYTES);
     Tables* tb = reinterpret_cast<Tables*>(ctl + 1);
 
+    constexpr int BKE = bk_elems<F8>();
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();  // 0 = leader (issues the MMAs)
@@ -396,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 }
             }
             const int xrows = gat ? half : (half + 15) & ~15;  // token rows this CTA loads per K step
-            const uint32_t tx = 2u * ((uint32_t)A_BYTES + (uint32_t)xrows * BK * 2);  // both CTAs' bytes
+            const uint32_t tx = 2u * ((uint32_t)A_BYTES + (uint32_t)xrows * 128u);  // both CTAs' bytes
             for (int kb = 0; kb < sp.k_blocks; ++kb) {
                 int got = 1;
                 if (lane == 0) got = mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, p.status) ? 1 : 0;
@@ -412,18 +432,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], tx);
                     if (UP) {
                         const int wrow = wg * sp.w_rows + tc.ft * 128 + (int)rank * 64;
-                        tma_load_2d_pair(sa, &M.w0, fb, kb * BK, wrow, W_HINT);
-                        tma_load_2d_pair(sa + A_BYTES / 2, &M.w1, fb, kb * BK, wrow, W_HINT);
+                        tma_load_2d_pair(sa, &M.w0, fb, kb * BKE, wrow, W_HINT);
+                        tma_load_2d_pair(sa + A_BYTES / 2, &M.w1, fb, kb * BKE, wrow, W_HINT);
                     } else {
-                        const int kk = kb * BK;
+                        const int kk = kb * BKE;
                         const int seg = kk / sp.kseg;
                         tma_load_3d_pair(sa, &M.w0, fb, kk - seg * sp.kseg, tc.ft * 256 + (int)rank * 128,
                                          wg * sp.nseg + seg, W_HINT);
                     }
-                    if (!gat) tma_load_2d_pair(sb, &M.x[xrows / 16 - 1], fb, kb * BK, tok0, X_HINT);
+                    if (!gat) tma_load_2d_pair(sb, &M.x[xrows / 16 - 1], fb, kb * BKE, tok0, X_HINT);
                 }
                 if (gat && 4 * lane < half)
-                    tma_gather4_pair(sb + 4 * lane * BK * 2, &tmXg, fb, kb * BK, src[0], src[1], src[2], src[3],
+                    tma_gather4_pair(sb + 4 * lane * 128, &tmXg, fb, kb * BKE, src[0], src[1], src[2], src[3],
                                      X_HINT);
                 issued_any = true;
                 if (++stage == STAGES) {
@@ -469,7 +489,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 int tstart, ntok;
                 token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
                 const int n_mma = (ntok + 15) & ~15;
-                const uint32_t idesc = idesc_bf16_f32(256, n_mma);
+                const uint32_t idesc = F8 ? idesc_e4m3_f32(256, n_mma) : idesc_bf16_f32(256, n_mma);
                 if (!mbar_wait_cluster(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, p.status)) {
                     ok = false;
                     break;
@@ -486,9 +506,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     const uint64_t ad = smem_desc_sw128(smem_u32(sa));
                     const uint64_t bd = smem_desc_sw128(smem_u32(sa + A_BYTES));
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per step
-                        tc_mma_bf16_pair(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
-                                         (kb > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {  // 4 MMAs of 32 bytes along K (16 bf16 or 32 E4M3)
+                        if (F8)
+                            tc_mma_e4m3_pair(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+                                             (kb > 0 || kk > 0) ? 1u : 0u);
+                        else
+                            tc_mma_bf16_pair(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+                                             (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
                     tc_commit_pair(&ctl->empty[stage], 0x3);
                     if (++stage == STAGES) {
                         stage = 0;
@@ -533,6 +558,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const int tok0 = tb->rowstart[tc.g] + tstart;
             // first output feature of this CTA
             const int fcta = UP ? tc.ft * 128 + (int)rank * 64 : tc.ft * 256 + (int)rank * 128;
+            // E4M3: scale of the weight row held in this thread's TMEM lane
+            float wsc = 1.0f;
+            if (F8) {
+                const int tl = q * 32 + lane;
+                const int wg = tc.g >= p.G0 ? 0 : tc.g;
+                if (UP) {
+                    const int f = tc.ft * 128 + (int)rank * 64 + (tl & 63);
+                    wsc = (tl < 64 ? sp.ws0 : sp.ws1)[(size_t)wg * sp.srows + f];
+                } else {
+                    const int f = fcta + tl;
+                    wsc = f < sp.f_limit ? sp.ws0[(size_t)wg * sp.srows + f] : 0.0f;
+                }
+            }
             if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, p.status)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACC_COLS;
@@ -544,7 +582,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 tmem_ld_wait();
                 float v16[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v16[i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 16; ++i) v16[i] = F8 ? __uint_as_float(r[i]) * wsc : __uint_as_float(r[i]);
                 if (c + 16 < ntok) tmem_ld16(taddr + (uint32_t)(c + 16), r);
                 float* xs = xbuf + xb * (XBUF_BYTES / 4);
 #pragma unroll
@@ -552,12 +590,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 named_bar_sync(1, 128);
                 const bool tok_ok = c + my_tok < ntok;
                 const float* row = xs + my_tok * XS;
+                float tsc = 1.0f;  // E4M3: scale of this token row
+                if (F8 && tok_ok) {
+                    const int orow = tok0 + c + my_tok;
+                    tsc = sp.xscale[sp.xidx ? sp.xidx[orow] / sp.xdiv : orow];
+                }
                 if (UP) {  // lanes 0-63: gate, 64-127: up of the same 64 features
                     const int fj = part * 8;
-                    const float4 g0 = *reinterpret_cast<const float4*>(row + fj);
-                    const float4 g1 = *reinterpret_cast<const float4*>(row + fj + 4);
-                    const float4 u0 = *reinterpret_cast<const float4*>(row + 64 + fj);
-                    const float4 u1 = *reinterpret_cast<const float4*>(row + 64 + fj + 4);
+                    float4 g0 = *reinterpret_cast<const float4*>(row + fj);
+                    float4 g1 = *reinterpret_cast<const float4*>(row + fj + 4);
+                    float4 u0 = *reinterpret_cast<const float4*>(row + 64 + fj);
+                    float4 u1 = *reinterpret_cast<const float4*>(row + 64 + fj + 4);
+                    if (F8) {
+                        scale4(g0, tsc);
+                        scale4(g1, tsc);
+                        scale4(u0, tsc);
+                        scale4(u1, tsc);
+                    }
                     if (tok_ok) {
                         uint4 v;
                         v.x = pack_bf16x2(silu_f32(g0.x) * u0.x, silu_f32(g0.y) * u0.y);
@@ -572,7 +621,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                         float f[16];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const float4 t = *reinterpret_cast<const float4*>(row + fj + 4 * i);
+                            float4 t = *reinterpret_cast<const float4*>(row + fj + 4 * i);
+                            if (F8) scale4(t, tsc);
                             f[4 * i] = t.x;
                             f[4 * i + 1] = t.y;
                             f[4 * i + 2] = t.z;
@@ -605,9 +655,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 
 std::atomic<unsigned int> g_sched_seq{0};
 
-template <bool UP>
+template <bool UP, bool F8>
 cudaError_t launch(const SetMaps& a, const SetMaps& b, const CUtensorMap& xg, Params p, int num_sms, cudaStream_t st) {
-    auto kern = tc_grouped_gemm_kernel<UP>;
+    auto kern = tc_grouped_gemm_kernel<UP, F8>;
     p.sched_slot = (int)(g_sched_seq.fetch_add(1u, std::memory_order_relaxed) % (unsigned int)kSchedSlots);
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
@@ -617,19 +667,28 @@ cudaError_t launch(const SetMaps& a, const SetMaps& b, const CUtensorMap& xg, Pa
     return cudaGetLastError();
 }
 
-bool token_maps(SetMaps& m, const void* base, int cols, long long rows) {
+bool token_maps(SetMaps& m, const void* base, int cols, long long rows, unsigned eb) {
     for (int b = 0; b < NXBOX; ++b)
-        if (!make_tmap_2d(&m.x[b], base, cols, rows, cols, BK, 16 * (b + 1))) return false;
+        if (!make_tmap_2d(&m.x[b], base, cols, rows, cols, 128 / eb, 16 * (b + 1), eb)) return false;
     return true;
 }
 
 bool up_set(const TcUpArgs& a, SetMaps& m, SetParams& sp) {
-    if (a.d % BK != 0 || a.I % 128 != 0) return false;
-    if (!make_tmap_2d(&m.w0, a.W1, a.d, a.W_rows, a.d, BK, 64) || !make_tmap_2d(&m.w1, a.W3, a.d, a.W_rows, a.d, BK, 64) ||
-        !token_maps(m, a.A, a.d, a.A_rows))
+    const unsigned eb = a.f8 ? 1 : 2;
+    const int bke = 128 / (int)eb;
+    if (a.d % bke != 0 || a.I % 128 != 0) return false;
+    if (a.f8 && (!a.w1s || !a.w3s || !a.xs)) return false;
+    if (!make_tmap_2d(&m.w0, a.W1, a.d, a.W_rows, a.d, bke, 64, eb) ||
+        !make_tmap_2d(&m.w1, a.W3, a.d, a.W_rows, a.d, bke, 64, eb) || !token_maps(m, a.A, a.d, a.A_rows, eb))
         return false;
     sp.f_tiles = a.I / 128;
-    sp.k_blocks = a.d / BK;
+    sp.k_blocks = a.d / bke;
+    sp.ws0 = a.w1s;
+    sp.ws1 = a.w3s;
+    sp.srows = a.I;
+    sp.xscale = a.xs;
+    sp.xidx = a.xs_idx;
+    sp.xdiv = a.xs_div > 0 ? a.xs_div : 1;
     sp.w_rows = a.I;
     sp.kseg = a.d;
     sp.nseg = 1;
@@ -641,13 +700,22 @@ bool up_set(const TcUpArgs& a, SetMaps& m, SetParams& sp) {
 }
 
 bool down_set(const TcDownArgs& a, SetMaps& m, SetParams& sp) {
-    if (a.K % BK != 0 || a.kseg % BK != 0 || a.d % 16 != 0) return false;
-    if (!make_tmap_3d(&m.w0, a.W2, a.kseg, a.d, (unsigned long long)a.G * a.nseg, BK, 128) ||
-        !token_maps(m, a.H, a.K, a.H_rows))
+    const unsigned eb = a.f8 ? 1 : 2;
+    const int bke = 128 / (int)eb;
+    if (a.K % bke != 0 || a.kseg % bke != 0 || a.d % 16 != 0) return false;
+    if (a.f8 && (!a.w2s || !a.hs)) return false;
+    if (!make_tmap_3d(&m.w0, a.W2, a.kseg, a.d, (unsigned long long)a.G * a.nseg, bke, 128, eb) ||
+        !token_maps(m, a.H, a.K, a.H_rows, eb))
         return false;
     m.w1 = m.w0;
     sp.f_tiles = (a.d + 255) / 256;
-    sp.k_blocks = a.K / BK;
+    sp.k_blocks = a.K / bke;
+    sp.ws0 = a.w2s;
+    sp.ws1 = nullptr;
+    sp.srows = a.d;
+    sp.xscale = a.hs;
+    sp.xidx = nullptr;
+    sp.xdiv = 1;
     sp.w_rows = 0;
     sp.kseg = a.kseg;
     sp.nseg = a.nseg;
@@ -670,7 +738,8 @@ cudaError_t launch_tc_up(const TcUpArgs* routed, const TcUpArgs* shared, int* st
     if (routed) {
         if (routed->G <= 0 || routed->G > kMaxGroups || !routed->offsets || !up_set(*routed, ma, p.set[0]))
             return cudaErrorInvalidValue;
-        if (!make_tmap_2d(&xg, routed->A, routed->d, routed->A_rows, routed->d, BK, 1))  // one-row box, tile::gather4
+        const unsigned eb = routed->f8 ? 1 : 2;
+        if (!make_tmap_2d(&xg, routed->A, routed->d, routed->A_rows, routed->d, 128 / eb, 1, eb))  // tile::gather4 box
             return cudaErrorInvalidValue;
         p.offsets = routed->offsets;
         p.G0 = routed->G;
@@ -683,10 +752,12 @@ cudaError_t launch_tc_up(const TcUpArgs* routed, const TcUpArgs* shared, int* st
         p.M = shared->M;
         if (!routed) xg = mb.x[NXBOX - 1];
     }
+    if (routed && shared && routed->f8 != shared->f8) return cudaErrorInvalidValue;
     if (!routed) ma = mb;
     if (!shared) mb = ma;
     p.status = status;
-    return launch<true>(ma, mb, xg, p, num_sms, st);
+    const bool f8 = routed ? routed->f8 : shared->f8;
+    return f8 ? launch<true, true>(ma, mb, xg, p, num_sms, st) : launch<true, false>(ma, mb, xg, p, num_sms, st);
 }
 
 cudaError_t launch_tc_down(const TcDownArgs* routed, const TcDownArgs* shared, int* status, int num_sms,
@@ -705,12 +776,15 @@ cudaError_t launch_tc_down(const TcDownArgs* routed, const TcDownArgs* shared, i
         p.has_shared = 1;
         p.M = shared->M;
     }
+    if (routed && shared && routed->f8 != shared->f8) return cudaErrorInvalidValue;
     if (!routed) ma = mb;
     if (!shared) mb = ma;
     p.gather = nullptr;
     p.gather_div = 1;
     p.status = status;
-    return launch<false>(ma, mb, ma.x[NXBOX - 1], p, num_sms, st);
+    const bool f8 = routed ? routed->f8 : shared->f8;
+    return f8 ? launch<false, true>(ma, mb, ma.x[NXBOX - 1], p, num_sms, st)
+              : launch<false, false>(ma, mb, ma.x[NXBOX - 1], p, num_sms, st);
 }
 
 }  // namespace moe

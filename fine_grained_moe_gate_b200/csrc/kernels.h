@@ -79,6 +79,14 @@ struct TcUpArgs {
     int d, I;
     const int32_t* offsets; // group rows; null: one group of M rows
     int G, M;
+    // E4M3 operands (A, W1, W3 one byte per element) with per-row scales:
+    // w1s/w3s [W_rows]; token row r's scale xs[xs_idx ? xs_idx[r] / xs_div : r].
+    bool f8 = false;
+    const float* w1s = nullptr;
+    const float* w3s = nullptr;
+    const float* xs = nullptr;
+    const int32_t* xs_idx = nullptr;
+    int xs_div = 1;
 };
 // Down projection: Y[r][:] = H[r] . W2_g^T, W2_g = [d][K] (K = I), or for
 // the shared group S stacked [d][Is] blocks contracted over K = S * Is.
@@ -92,7 +100,17 @@ struct TcDownArgs {
     int d, K;
     const int32_t* offsets;
     int G, M;
+    // E4M3 operands (H, W2 one byte per element): w2s [G][d] per output row
+    // (one scale per row across the nseg blocks), hs [H_rows] per token row.
+    bool f8 = false;
+    const float* w2s = nullptr;
+    const float* hs = nullptr;
 };
+// quant.cu: per-row E4M3 quantization of a bf16 matrix with `rows` rows
+// stored as nseg column blocks of kseg columns (kseg % 8 == 0).
+cudaError_t launch_quantize_e4m3(const void* src, long long rows, int kseg, int nseg, uint8_t* q, float* scale,
+                                 cudaStream_t st);
+
 // One launch for the routed set (offsets) and/or the shared set (M rows);
 // either pointer may be null.
 cudaError_t launch_tc_up(const TcUpArgs* routed, const TcUpArgs* shared, int* status, int num_sms, cudaStream_t st);

@@ -1,6 +1,7 @@
-// Host helper: encode TMA tensor maps (CUtensorMap) for bf16 row-major
-// matrices, loaded in boxes whose inner extent is 64 elements (128 bytes)
-// with the 128-byte swizzle the tcgen05 shared-memory descriptors expect.
+// Host helper: encode TMA tensor maps (CUtensorMap) for bf16 or 8-bit
+// row-major matrices, loaded in boxes whose inner extent is 128 bytes (64
+// bf16 or 128 one-byte elements) with the 128-byte swizzle the tcgen05
+// shared-memory descriptors expect.
 // The driver entry point is fetched through the runtime, so the library
 // links only against cudart.
 #pragma once
@@ -27,32 +28,37 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
     return fn;
 }
 
-// rank-2 map over a [rows][cols] bf16 matrix with row pitch `ld` elements;
-// box = box_cols (innermost, 64) x box_rows.  Out-of-bounds reads fill 0.
+inline CUtensorMapDataType tmap_type(unsigned elem_bytes) {
+    return elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+}
+
+// rank-2 map over a [rows][cols] matrix of elem_bytes-wide elements (2: bf16,
+// 1: an 8-bit format) with row pitch `ld` elements; box = box_cols
+// (innermost, 128 bytes) x box_rows.  Out-of-bounds reads fill 0.
 inline bool make_tmap_2d(CUtensorMap* m, const void* base, unsigned long long cols, unsigned long long rows,
-                         unsigned long long ld, unsigned box_cols, unsigned box_rows) {
+                         unsigned long long ld, unsigned box_cols, unsigned box_rows, unsigned elem_bytes = 2) {
     auto enc = tmap_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {ld * 2};
+    cuuint64_t strides[1] = {ld * elem_bytes};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t es[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+    return enc(m, tmap_type(elem_bytes), 2, const_cast<void*>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// rank-3 map over [n2][rows][cols] bf16 (contiguous); box box_cols x
-// box_rows x 1.
+// rank-3 map over [n2][rows][cols] (contiguous, elem_bytes-wide elements);
+// box box_cols x box_rows x 1.
 inline bool make_tmap_3d(CUtensorMap* m, const void* base, unsigned long long cols, unsigned long long rows,
-                         unsigned long long n2, unsigned box_cols, unsigned box_rows) {
+                         unsigned long long n2, unsigned box_cols, unsigned box_rows, unsigned elem_bytes = 2) {
     auto enc = tmap_encoder();
     if (!enc) return false;
     cuuint64_t dims[3] = {cols, rows, n2};
-    cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+    cuuint64_t strides[2] = {cols * elem_bytes, cols * rows * elem_bytes};
     cuuint32_t box[3] = {box_cols, box_rows, 1};
     cuuint32_t es[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+    return enc(m, tmap_type(elem_bytes), 3, const_cast<void*>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

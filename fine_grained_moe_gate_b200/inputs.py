@@ -12,6 +12,8 @@ from the stated distributions):
   v3_prefill   T=8192,  d=7168, E=256, k=8, 1 shared, I=Is=2048,   bf16
                x~N(0,1), W~N(0,0.006), bias~U(-0.01,0.01)
   v3_decode    T=64 per call, V3 shape and distributions, fresh x per call
+  *_fp8        small_fp8, v3_prefill_fp8, v3_decode_fp8: the same tensors,
+               expert GEMMs in E4M3 (weights quantized per output row)
   skew_stress  T=32768, V3 shape; x[:,0]=1 and W_g[i][0]=o_i, a per-expert
                logit offset that ranks expert popularity by a seeded
                permutation with Zipf exponent 1.2 (see ``zipf_offsets``);
@@ -40,7 +42,7 @@ class MoEConfig:
     I: int
     S: int
     Is: int
-    dtype: str            # "f32" or "bf16"
+    dtype: str            # "f32", "bf16" or "fp8" (bf16 tokens, E4M3 expert GEMMs)
     w_std: float
     bias_kind: str        # "uniform" or "zero"
     bias_range: float
@@ -69,6 +71,12 @@ CONFIGS = {
     "skew_stress": MoEConfig("skew_stress", 32768, 7168, 256, 8, 2048, 1, 2048, "bf16", 0.006, "uniform", 0.01, 4,
                              steps=200, zipf_s=1.2),
 }
+# The same workloads with E4M3 expert GEMMs (same seeds, so the same bf16
+# tensors before quantization).
+for _n in ("small_bf16", "v3_prefill", "v3_decode"):
+    _c = CONFIGS[_n]
+    _fp8 = _n.replace("_bf16", "") + "_fp8"
+    CONFIGS[_fp8] = _c.scaled(name=_fp8, dtype="fp8")
 
 
 def _gen(device, seed: int) -> torch.Generator:

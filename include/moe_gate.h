@@ -64,7 +64,10 @@ typedef enum {
     MOE_ERR_TIMEOUT = 7        /* a device-side wait gave up (bounded spin) */
 } moe_status;
 
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+/* MOE_FP8_E4M3: x, W_gate, y and the bf16 intermediates as MOE_BF16; the
+ * expert GEMM operands (expert weights, token rows, h) in E4M3 with fp32
+ * per-row scales -- see the FP8 section below. */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_FP8_E4M3 = 2 } moe_dtype;
 
 /* Problem sizes.  T tokens of width d; E routed experts, k chosen per
  * token; routed SwiGLU intermediate I; S shared experts of intermediate Is
@@ -76,7 +79,11 @@ typedef struct {
 
 /* Limits (validated): 1 <= k <= min(E, 16); E <= 256; d % 8 == 0.
  * MOE_BF16 additionally needs d % 64 == 0, I % 128 == 0 and Is % 128 == 0
- * (tensor-core tiles), else MOE_ERR_UNSUPPORTED. */
+ * (tensor-core tiles), MOE_FP8_E4M3 d % 128 == 0 as well, else
+ * MOE_ERR_UNSUPPORTED.  With MOE_FP8_E4M3, moe_route, moe_load_and_bias_update
+ * and moe_combine behave as with MOE_BF16 and moe_permute moves E4M3 rows (one
+ * byte per element); the bf16-weight calls (moe_grouped_swiglu, moe_ffn_*,
+ * moe_expert_*, moe_layer_forward) return MOE_ERR_UNSUPPORTED. */
 
 /* ---------------------------------------------------------------------------
  * moe_route -- gate affinities, bias-shifted top-k, unbiased weights and the
@@ -240,7 +247,67 @@ MOE_API moe_status moe_layer_forward(const void* x, const void* w_gate, const fl
                              const void* w2, const void* ws1, const void* ws3, const void* ws2, moe_shape sh, void* y,
                              int32_t* topk_idx, float* topk_w, int32_t* counts, void* workspace, size_t ws_bytes,
                              void* stream);
-MOE_API size_t moe_workspace_size(moe_shape sh);
+MOE_API size_t moe_workspace_size(moe_shape sh);  /* moe_layer_forward, or moe_layer_forward_fp8 for MOE_FP8_E4M3 */
+
+/* ---------------------------------------------------------------------------
+ * FP8 experts  ["DeepSeek V3 Architecture Deep Dive ...", "FP8 Formats": E4M3
+ * for weights and activations; "Per-Tensor/Per-Axis Quantization": a scale
+ * per row/channel].  Read as: each weight matrix quantized per output row,
+ * token rows and h per row; both scales factor out of every dot product and
+ * are applied to the fp32 tensor-core accumulator:
+ *   out[t][f] = sx[t] * sw[f] * sum_c e4m3(xq[t][c]) * e4m3(wq[f][c])
+ * E4M3: 1 sign, 4 exponent (bias 7), 3 mantissa bits, no infinities, largest
+ * finite 448.
+ * -------------------------------------------------------------------------*/
+
+/* moe_quantize_fp8 -- per-row E4M3 quantization of a bf16 matrix with `rows`
+ * rows stored as nseg column blocks of kseg columns ([nseg][rows][kseg];
+ * nseg = 1 is plain row major; a row spans all blocks):
+ *   scale[r] = max_c |src[r][c]| / 448  (fp32, IEEE division; 1 if the row is 0)
+ *   q[r][c]  = E4M3(src[r][c] / scale[r]), nearest, ties to even, saturating
+ * q has src's layout, one byte per element.  Needs kseg % 8 == 0, nseg >= 1,
+ * 16-byte aligned src and q.  Used once per weight tensor (W2 [E][d][I] is
+ * rows = E*d, kseg = I; the shared Ws2 [S][d][Is] is rows = d, kseg = Is,
+ * nseg = S) and per step for the token rows and h. */
+MOE_API moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t kseg, int32_t nseg, uint8_t* q,
+                                    float* scale, void* stream);
+
+/* E4M3 expert weights and their per-row fp32 scales (all device pointers). */
+typedef struct {
+    const uint8_t* w1;  const float* w1_scale;   /* [E][I][d],  [E*I]  */
+    const uint8_t* w3;  const float* w3_scale;   /* [E][I][d],  [E*I]  */
+    const uint8_t* w2;  const float* w2_scale;   /* [E][d][I],  [E*d]  */
+    const uint8_t* ws1; const float* ws1_scale;  /* [S][Is][d], [S*Is] (NULL if S == 0) */
+    const uint8_t* ws3; const float* ws3_scale;  /* [S][Is][d], [S*Is] */
+    const uint8_t* ws2; const float* ws2_scale;  /* [S][d][Is], [d]: one scale per output row across the S blocks */
+} moe_fp8_experts;
+
+/* moe_ffn_up_fp8 / moe_ffn_down_fp8 -- moe_ffn_up / moe_ffn_down on E4M3
+ * operands (sh.dtype == MOE_FP8_E4M3), routed and shared experts in one
+ * launch each.
+ *   up:   xq_perm [T*k][d] E4M3 token rows in expert order (moe_permute of
+ *         xq), perm_tok from moe_permute, x_scale [T] the token scales;
+ *         xq [T][d] the unpermuted quantized tokens (shared experts; NULL
+ *         leaves them out).  h = bf16(silu(a) * g) with a, g the scaled sums
+ *         [T*k][I]; hs likewise [T][S*Is].
+ *   down: hq [T*k][I] E4M3 with h_scale [T*k] (moe_quantize_fp8 of h), hsq
+ *         [T][S*Is] with hs_scale [T] (NULL leaves the shared set out);
+ *         y_perm [T*k][d] and shared_out [T][d] in bf16. */
+MOE_API moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const float* x_scale,
+                                  const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w, moe_shape sh,
+                                  void* h, void* hs, void* stream);
+MOE_API moe_status moe_ffn_down_fp8(const uint8_t* hq, const float* h_scale, const int32_t* offsets,
+                                    const uint8_t* hsq, const float* hs_scale, const moe_fp8_experts* w,
+                                    moe_shape sh, void* y_perm, void* shared_out, void* stream);
+
+/* moe_layer_forward_fp8 -- the layer with FP8 experts: route (bf16 x),
+ * quantize x per token, permute the E4M3 rows, gate/up, quantize h and hs
+ * per row, down, combine into y [T][d] bf16.  sh.dtype == MOE_FP8_E4M3;
+ * workspace >= moe_workspace_size(sh). */
+MOE_API moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float* bias,
+                                         const moe_fp8_experts* w, moe_shape sh, void* y, int32_t* topk_idx,
+                                         float* topk_w, int32_t* counts, void* workspace, size_t ws_bytes,
+                                         void* stream);
 
 /* Synchronises `stream`, then returns and clears the current device's
  * status word (MOE_OK if no kernel reported an anomaly). */
