@@ -76,7 +76,17 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
 constexpr int NT = 256;                 // tokens per tile (MMA N <= 256)
 constexpr uint32_t ACC_COLS = 256;      // one accumulator buffer
 constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
-constexpr int NTHREADS = 192;
+// Epilogue warps come in groups of four (one per TMEM lane quarter); groups
+// take the tile's 16-token chunks in turn.  The gate/up epilogue (SwiGLU on
+// every element) runs two groups with one exchange buffer each; the down
+// epilogue, a plain conversion, one group with two buffers.  On short-K
+// tiles (d = 2048, E4M3) the single group paced the whole kernel.
+template <bool UP>
+__host__ __device__ constexpr int n_epi_warps() { return UP ? 8 : 4; }
+template <bool UP>
+__host__ __device__ constexpr int n_xbuf_per_group() { return UP ? 1 : 2; }
+template <bool UP>
+__host__ __device__ constexpr int n_threads() { return 64 + 32 * n_epi_warps<UP>(); }
 constexpr int XS = 132;                 // row stride (floats) of the epilogue exchange buffer
 constexpr int XBUF_BYTES = 16 * XS * 4; // 16 tokens x 128 lanes (+pad), fp32
 // L2 policy of the two operands' loads.  Marking the weights evict-first
@@ -86,8 +96,9 @@ constexpr int XBUF_BYTES = 16 * XS * 4; // 16 tokens x 128 lanes (+pad), fp32
 constexpr uint64_t W_HINT = kEvictNormal;
 constexpr uint64_t X_HINT = kEvictNormal;
 constexpr int TQ = 8;                   // tile queue slots
-// readers of a queue slot: leader MMA issuer + 4 epilogue warps, peer producer + 4 epilogue warps
-constexpr uint32_t TQ_READERS = 10;
+// readers of a queue slot: leader MMA issuer + its epilogue warps, peer producer + its epilogue warps
+template <bool UP>
+__host__ __device__ constexpr uint32_t tq_readers() { return 2u * (1u + (uint32_t)n_epi_warps<UP>()); }
 
 // Tile counters: one {next, done} pair per launch slot.  A launch takes the
 // next slot round-robin on the host; the last cluster to finish resets its
@@ -117,7 +128,10 @@ struct Tables {
     int ttiles[kMaxTcGroups];  // token tiles per group
     int prefix[kMaxTcGroups + 1];
 };
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 2 * XBUF_BYTES + sizeof(Ctl) + sizeof(Tables);
+constexpr size_t XBUF_TOTAL = 2 * (size_t)XBUF_BYTES;  // groups x buffers per group = 2 either way
+static_assert(n_epi_warps<true>() / 4 * n_xbuf_per_group<true>() == 2, "exchange buffers");
+static_assert(n_epi_warps<false>() / 4 * n_xbuf_per_group<false>() == 2, "exchange buffers");
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + XBUF_TOTAL + sizeof(Ctl) + sizeof(Tables);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // Tensor maps of one expert set: weights (w1 only for the up projection) and
@@ -184,6 +198,11 @@ __device__ __forceinline__ void token_tile(int rows, int ntt, int tt, int& start
     start = tt * q + min(tt, r);
     len = q + (tt < r ? 1 : 0);
 }
+
+// silu(a) = a / (1 + e^-a) with the hardware exponential and division: the
+// result is rounded to bf16 right after, so their few-ulp fp32 error is far
+// below the output's own rounding.
+__device__ __forceinline__ float silu_fast(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
 __device__ __forceinline__ void scale4(float4& v, float s) {
     v.x *= s;
@@ -254,14 +273,17 @@ __device__ __forceinline__ bool tq_take(Ctl* ctl, int j, uint32_t ph, uint32_t l
 }
 
 template <bool UP, bool F8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
     tc_grouped_gemm_kernel(const __grid_constant__ SetMaps ma, const __grid_constant__ SetMaps mb,
                            const __grid_constant__ CUtensorMap tmXg, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = base;
     float* xbuf = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
-    Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + 2 * XBUF_BYTES);
+    Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + XBUF_TOTAL);
+    constexpr int NEPI = n_epi_warps<UP>();
+    constexpr int NXB = n_xbuf_per_group<UP>();
+    constexpr int NTHREADS = n_threads<UP>();
     Tables* tb = reinterpret_cast<Tables*>(ctl + 1);
 
     constexpr int BKE = bk_elems<F8>();
@@ -291,11 +313,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&ctl->tfull[a], 1);
-            mbar_init(&ctl->tempty[a], 8);  // 4 epilogue warps x 2 CTAs
+            mbar_init(&ctl->tempty[a], 2 * NEPI);  // every epilogue warp of both CTAs
         }
         for (int j = 0; j < TQ; ++j) {
             mbar_init(&ctl->tq_full[j], 1);
-            mbar_init(&ctl->tq_empty[j], TQ_READERS);
+            mbar_init(&ctl->tq_empty[j], tq_readers<UP>());
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -533,8 +555,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue (both CTAs)
+        // Two groups of four warps (one per TMEM lane quarter each) take the
+        // tile's 16-token chunks in turn: group eg handles chunks eg, eg+2, ...
         const int q = warp & 3;           // TMEM lane quarter this warp may read
-        const int e = tid - 64;           // 0..127 among the epilogue threads
+        const int eg = (warp - 2) >> 2;   // epilogue group
+        const int e = tid - 64 - 128 * eg;  // 0..127 within the group
         const int my_tok = e >> 3;        // token (0..15) of a 16-token chunk this thread stores
         const int part = e & 7;
         const uint32_t leader_tempty = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
@@ -574,20 +599,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, p.status)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACC_COLS;
-            // TMEM reads run one 16-token chunk ahead of the exchange below
+            // TMEM reads run one chunk ahead of the exchange below
+            constexpr int CSTEP = 16 * (NEPI / 4);
             uint32_t r[16];
-            tmem_ld16(taddr, r);
+            if (16 * eg < ntok) tmem_ld16(taddr + (uint32_t)(16 * eg), r);
 #pragma unroll 1
-            for (int c = 0; c < ntok; c += 16) {
+            for (int c = 16 * eg; c < ntok; c += CSTEP) {
                 tmem_ld_wait();
                 float v16[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) v16[i] = F8 ? __uint_as_float(r[i]) * wsc : __uint_as_float(r[i]);
-                if (c + 16 < ntok) tmem_ld16(taddr + (uint32_t)(c + 16), r);
-                float* xs = xbuf + xb * (XBUF_BYTES / 4);
+                if (c + CSTEP < ntok) tmem_ld16(taddr + (uint32_t)(c + CSTEP), r);
+                float* xs = xbuf + (NXB * eg + xb) * (XBUF_BYTES / 4);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) xs[i * XS + q * 32 + lane] = v16[i];
-                named_bar_sync(1, 128);
+                named_bar_sync(1 + eg, 128);
                 const bool tok_ok = c + my_tok < ntok;
                 const float* row = xs + my_tok * XS;
                 float tsc = 1.0f;  // E4M3: scale of this token row
@@ -601,6 +627,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     float4 g1 = *reinterpret_cast<const float4*>(row + fj + 4);
                     float4 u0 = *reinterpret_cast<const float4*>(row + 64 + fj);
                     float4 u1 = *reinterpret_cast<const float4*>(row + 64 + fj + 4);
+                    if (NXB == 1) named_bar_sync(1 + eg, 128);  // the single buffer is free for the next chunk
                     if (F8) {
                         scale4(g0, tsc);
                         scale4(g1, tsc);
@@ -609,10 +636,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     }
                     if (tok_ok) {
                         uint4 v;
-                        v.x = pack_bf16x2(silu_f32(g0.x) * u0.x, silu_f32(g0.y) * u0.y);
-                        v.y = pack_bf16x2(silu_f32(g0.z) * u0.z, silu_f32(g0.w) * u0.w);
-                        v.z = pack_bf16x2(silu_f32(g1.x) * u1.x, silu_f32(g1.y) * u1.y);
-                        v.w = pack_bf16x2(silu_f32(g1.z) * u1.z, silu_f32(g1.w) * u1.w);
+                        v.x = pack_bf16x2(silu_fast(g0.x) * u0.x, silu_fast(g0.y) * u0.y);
+                        v.y = pack_bf16x2(silu_fast(g0.z) * u0.z, silu_fast(g0.w) * u0.w);
+                        v.z = pack_bf16x2(silu_fast(g1.x) * u1.x, silu_fast(g1.y) * u1.y);
+                        v.w = pack_bf16x2(silu_fast(g1.z) * u1.z, silu_fast(g1.w) * u1.w);
                         *reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * sp.ldo + fcta + fj) = v;
                     }
                 } else {
@@ -635,7 +662,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                                             pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
                     }
                 }
-                xb ^= 1;  // the next chunk writes the other buffer; its barrier orders the reuse
+                if (NXB == 2) xb ^= 1;  // the next chunk writes the other buffer; its barrier orders the reuse
             }
             tc_fence_before();
             __syncwarp();
@@ -660,6 +687,7 @@ cudaError_t launch(const SetMaps& a, const SetMaps& b, const CUtensorMap& xg, Pa
     auto kern = tc_grouped_gemm_kernel<UP, F8>;
     p.sched_slot = (int)(g_sched_seq.fetch_add(1u, std::memory_order_relaxed) % (unsigned int)kSchedSlots);
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    constexpr int NTHREADS = n_threads<UP>();
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;  // whole CTA pairs, one CTA per SM
     kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(a, b, xg, p);
