@@ -2,8 +2,9 @@
 // "FP8 Formats": E4M3 for weights and activations; "Per-Tensor/Per-Axis
 // Quantization": one scale per row/channel).
 //
-//   scale_r = amax_r / 448 (fp32, IEEE division; 1 for an all-zero row)
-//   q[r][c] = E4M3(src[r][c] / scale_r), round to nearest even, saturating
+//   scale_r = amax_r / 448, inv_r = 448 / amax_r (fp32, IEEE division, once
+//   per row; an all-zero row gets scale 1 and codes 0)
+//   q[r][c] = E4M3(src[r][c] * inv_r), round to nearest even, saturating
 //
 // A matrix with `rows` rows may be stored as nseg column blocks of kseg
 // columns ([nseg][rows][kseg], stacked experts joined along the contraction);
@@ -50,6 +51,7 @@ __global__ void __launch_bounds__(kWarps * 32) quantize_e4m3_kernel(const uint16
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
     if (lane == 0) scale[r] = sc;
     for (int c = lane * 8; c < K; c += 256) {
         const size_t off = seg_offset(r, c, rows, kseg);
@@ -58,7 +60,7 @@ __global__ void __launch_bounds__(kWarps * 32) quantize_e4m3_kernel(const uint16
         uint32_t p[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            p[i] = e4m3x2(__fdiv_rn(bf16_lo(w[i]), sc), __fdiv_rn(bf16_hi(w[i]), sc));
+            p[i] = e4m3x2(__fmul_rn(bf16_lo(w[i]), inv), __fmul_rn(bf16_hi(w[i]), inv));
         // element order in memory: low byte first
         *reinterpret_cast<uint2*>(q + off) = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
     }

@@ -263,8 +263,9 @@ MOE_API size_t moe_workspace_size(moe_shape sh);  /* moe_layer_forward, or moe_l
 /* moe_quantize_fp8 -- per-row E4M3 quantization of a bf16 matrix with `rows`
  * rows stored as nseg column blocks of kseg columns ([nseg][rows][kseg];
  * nseg = 1 is plain row major; a row spans all blocks):
- *   scale[r] = max_c |src[r][c]| / 448  (fp32, IEEE division; 1 if the row is 0)
- *   q[r][c]  = E4M3(src[r][c] / scale[r]), nearest, ties to even, saturating
+ *   scale[r] = amax_r / 448, inv_r = 448 / amax_r  (amax_r = max_c |src[r][c]|;
+ *              fp32, IEEE division; a zero row gets scale 1 and codes 0)
+ *   q[r][c]  = E4M3(src[r][c] * inv_r), nearest, ties to even, saturating
  * q has src's layout, one byte per element.  Needs kseg % 8 == 0, nseg >= 1,
  * 16-byte aligned src and q.  Used once per weight tensor (W2 [E][d][I] is
  * rows = E*d, kseg = I; the shared Ws2 [S][d][Is] is rows = d, kseg = Is,

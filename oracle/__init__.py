@@ -214,7 +214,8 @@ def quantize_rows_fp8(a: np.ndarray, nseg: int = 1):
     """Per-row E4M3 quantization.  ``a`` is [rows][K] (bf16 bits as uint16, or
     float32), or [nseg][rows][kseg] for a matrix stored as column blocks (the
     rows then span all nseg blocks).  Returns (codes with a's shape, scale fp32
-    [rows]) with scale = amax / 448 and codes = e4m3(v / scale)."""
+    [rows]) with scale = amax / 448 and codes = e4m3(v * (448 / amax)), both
+    factors rounded to fp32."""
     a = _c(a)
     dt = _dtype_code(a)
     if a.ndim == 3:

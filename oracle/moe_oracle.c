@@ -349,8 +349,10 @@ static size_t seg_index(long r, int c, long rows, int kseg) {
     return (size_t)(c / kseg) * (size_t)rows * kseg + (size_t)r * kseg + (size_t)(c % kseg);
 }
 
-/* Per-row quantization: amax_r = max |v| (fp32), scale_r = fl32(amax_r / 448),
- * or 1 for an all-zero row; q = e4m3(fl32(v / scale_r)).  q has src's layout. */
+/* Per-row quantization: amax_r = max |v| (fp32); the dequantization scale is
+ * scale_r = fl32(amax_r / 448) and the codes use its reciprocal taken the
+ * other way round, inv_r = fl32(448 / amax_r): q = e4m3(fl32(v * inv_r)).
+ * An all-zero row has scale 1 and codes 0.  q has src's layout. */
 void orc_quantize_rows_fp8(const void* src, int dtype, long rows, int kseg, int nseg, uint8_t* q, float* scale) {
     int K = kseg * nseg;
     #pragma omp parallel for schedule(static)
@@ -361,11 +363,12 @@ void orc_quantize_rows_fp8(const void* src, int dtype, long rows, int kseg, int 
             if (v > amax) amax = v;
         }
         float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+        float inv = amax > 0.0f ? 448.0f / amax : 0.0f;
         scale[r] = sc;
         for (int c = 0; c < K; ++c) {
             size_t i = seg_index(r, c, rows, kseg);
             float v = (float)load_elem(src, dtype, i);
-            q[i] = orc_e4m3_encode(v / sc);
+            q[i] = orc_e4m3_encode(v * inv);
         }
     }
 }

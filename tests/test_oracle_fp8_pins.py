@@ -89,8 +89,9 @@ def test_quantize_rows_scale_and_codes(oracle_lib):
     want_sc = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
     assert np.array_equal(sc, want_sc)
     assert np.all(q[5] == 0) and sc[5] == 1.0
-    # codes = encode(v / scale) element by element, and the row max maps to +-448
-    assert np.array_equal(q, oracle.fp8_encode((af / sc[:, None]).astype(np.float32)))
+    # codes = encode(v * (448 / amax)) element by element, and the row max maps to +-448
+    inv = np.where(amax > 0, np.float32(448.0) / np.where(amax > 0, amax, 1), np.float32(0)).astype(np.float32)
+    assert np.array_equal(q, oracle.fp8_encode((af * inv[:, None]).astype(np.float32)))
     dec = oracle.fp8_decode(q)
     nz = amax > 0
     assert np.all(np.abs(dec[nz]).max(axis=1) == 448.0)
