@@ -21,8 +21,10 @@ duration inside the timed region (roofline of the dominant kernel).  The
 layer weights (22.6 GB for the DeepSeek-V3 shape) are far larger than the
 126 MB L2, so no flush is needed between steps.
 
-The e2e leg runs the same steps through moe_layer_forward with the tokens
-copied from pinned host memory each step and the output copied back.
+The e2e leg runs the same steps through moe_layer_forward (or
+moe_layer_forward_fp8) with each step's tokens copied from pinned host memory
+and its output copied back, double-buffered on two copy streams so that the
+copies of one step overlap the compute of the next.
 
 Rank 0 prints one JSON line.
 """
@@ -415,38 +417,73 @@ def run_ours(args, world, rank, local):
     # ---- e2e: public call, host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
+        # Double-buffered: the tokens of step i+1 go up (copy stream) and the
+        # output of step i comes down (another copy stream) while step i+1
+        # computes; every step still copies its own x in and its y out, all
+        # inside the timed region.
         ws = torch.empty(moe.moe_workspace_size(sh), dtype=torch.uint8, device=dev)
-        x_dev = torch.empty((T, d), dtype=dt, device=dev)
+        nb = 2
+        x_dev = [torch.empty((T, d), dtype=dt, device=dev) for _ in range(nb)]
+        y_dev = [torch.empty((T, d), dtype=dt, device=dev) for _ in range(nb)]
         x_host = [xx.cpu().pin_memory() for xx in xs]
-        y_host = torch.empty((T, d), dtype=dt).pin_memory()
+        y_host = [torch.empty((T, d), dtype=dt).pin_memory() for _ in range(nb)]
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(nb)]     # x_dev[b] holds the step's tokens
+        ev_done = [torch.cuda.Event() for _ in range(nb)]   # the step using buffer b has computed
+        ev_out = [torch.cuda.Event() for _ in range(nb)]    # y_dev[b] has reached the host
 
-        def e2e_step(i):
-            x_dev.copy_(x_host[i % n_x], non_blocking=True)
+        def issue_h2d(i):
+            bb = i % nb
+            s_in.wait_event(ev_done[bb])                    # the step that last read x_dev[bb] is done
+            with torch.cuda.stream(s_in):
+                x_dev[bb].copy_(x_host[i % n_x], non_blocking=True)
+            ev_in[bb].record(s_in)
+
+        def e2e_step(i, last):
+            bb = i % nb
+            stream.wait_event(ev_in[bb])
+            stream.wait_event(ev_out[bb])                   # y_dev[bb] is no longer being copied out
             if fp8:
-                moe.moe_layer_forward_fp8(x_dev, p["w_gate"], p["bias"], w8, sh, y, idx, w, counts, ws, stream)
+                moe.moe_layer_forward_fp8(x_dev[bb], p["w_gate"], p["bias"], w8, sh, y_dev[bb], idx, w, counts, ws,
+                                          stream)
             else:
-                moe.moe_layer_forward(x_dev, p["w_gate"], p["bias"], p["w1"], p["w3"], p["w2"], p["ws1"], p["ws3"],
-                                      p["ws2"], sh, y, idx, w, counts, ws, stream)
+                moe.moe_layer_forward(x_dev[bb], p["w_gate"], p["bias"], p["w1"], p["w3"], p["w2"], p["ws1"],
+                                      p["ws3"], p["ws2"], sh, y_dev[bb], idx, w, counts, ws, stream)
             mdist.allreduce_counts(counts)
             moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
-            y_host.copy_(y, non_blocking=True)
+            ev_done[bb].record(stream)
+            if not last:
+                issue_h2d(i + 1)
+            s_out.wait_event(ev_done[bb])
+            with torch.cuda.stream(s_out):
+                y_host[bb].copy_(y_dev[bb], non_blocking=True)
+            ev_out[bb].record(s_out)
 
-        for i in range(args.warmup):
-            e2e_step(i)
+        def e2e_run(n):
+            s_in.wait_event(start_ev)
+            issue_h2d(0)
+            for i in range(n):
+                e2e_step(i, i == n - 1)
+            stream.wait_event(ev_out[(n - 1) % nb])
+
+        start_ev = torch.cuda.Event()
+        start_ev.record(stream)
+        e2e_run(args.warmup)
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for i in range(args.steps):
-            e2e_step(i)
+        start_ev = a
+        e2e_run(args.steps)
         b.record(stream)
         barrier()
         te = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
         if world > 1:
             dist.all_reduce(te, op=dist.ReduceOp.MAX)
         e2e = {"value": world * T * args.steps / (float(te.item()) / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": x_dev.numel() * x_dev.element_size(),
-               "d2h_bytes_per_step": y_host.numel() * y_host.element_size(),
-               "ms_per_step": float(te.item()) / args.steps}
+               "h2d_bytes_per_step": x_dev[0].numel() * x_dev[0].element_size(),
+               "d2h_bytes_per_step": y_host[0].numel() * y_host[0].element_size(),
+               "ms_per_step": float(te.item()) / args.steps,
+               "pipelining": "copy-in of step i+1 and copy-out of step i overlap step i+1's compute (2 buffers)"}
         st = moe.moe_get_last_error(stream)
         if st != 0:
             raise moe.MoEError(st, "e2e steps")
