@@ -335,6 +335,22 @@ uint8_t orc_e4m3_encode(float x) {
     return sign | (uint8_t)(((vbe + 7) << 3) | m);
 }
 
+/* The 256 code values, from orc_e4m3_decode, for the expert sums below. */
+static double e4m3_table[256];
+static int e4m3_table_ready = 0;
+static const double* e4m3_values(void) {
+    if (!e4m3_table_ready) {
+        #pragma omp critical(e4m3_table)
+        {
+            if (!e4m3_table_ready) {
+                for (int c = 0; c < 256; ++c) e4m3_table[c] = orc_e4m3_decode((uint8_t)c);
+                e4m3_table_ready = 1;
+            }
+        }
+    }
+    return e4m3_table;
+}
+
 void orc_e4m3_encode_array(const float* x, size_t n, uint8_t* q) {
     for (size_t i = 0; i < n; ++i) q[i] = orc_e4m3_encode(x[i]);
 }
@@ -380,14 +396,15 @@ void orc_quantize_rows_fp8(const void* src, int dtype, long rows, int kseg, int 
  * xq [n][d], w1q/w3q [I][d] row major. */
 void orc_expert_up_fp8(const uint8_t* xq, const float* xs, int n, const uint8_t* w1q, const float* w1s,
                        const uint8_t* w3q, const float* w3s, int d, int I, uint16_t* h) {
-    #pragma omp parallel for schedule(dynamic, 1)
+    const double* val = e4m3_values();
+    #pragma omp parallel for schedule(dynamic, 8) collapse(2)
     for (int r = 0; r < n; ++r) {
         for (int c = 0; c < I; ++c) {
             double sa = 0.0, sg = 0.0;
             for (int i = 0; i < d; ++i) {
-                double xv = orc_e4m3_decode(xq[(size_t)r * d + i]);
-                sa += xv * orc_e4m3_decode(w1q[(size_t)c * d + i]);
-                sg += xv * orc_e4m3_decode(w3q[(size_t)c * d + i]);
+                double xv = val[xq[(size_t)r * d + i]];
+                sa += xv * val[w1q[(size_t)c * d + i]];
+                sg += xv * val[w3q[(size_t)c * d + i]];
             }
             double a = (double)xs[r] * (double)w1s[c] * sa;
             double g = (double)xs[r] * (double)w3s[c] * sg;
@@ -402,12 +419,12 @@ void orc_expert_up_fp8(const uint8_t* xq, const float* xs, int n, const uint8_t*
 void orc_expert_down_fp8(const uint8_t* hq, const float* hs, int n, const uint8_t* w2q, const float* w2s, int d,
                          int kseg, int nseg, double* o) {
     int K = kseg * nseg;
-    #pragma omp parallel for schedule(dynamic, 1)
+    const double* val = e4m3_values();
+    #pragma omp parallel for schedule(dynamic, 8) collapse(2)
     for (int r = 0; r < n; ++r) {
         for (int j = 0; j < d; ++j) {
             double acc = 0.0;
-            for (int c = 0; c < K; ++c)
-                acc += orc_e4m3_decode(hq[(size_t)r * K + c]) * orc_e4m3_decode(w2q[seg_index(j, c, d, kseg)]);
+            for (int c = 0; c < K; ++c) acc += val[hq[(size_t)r * K + c]] * val[w2q[seg_index(j, c, d, kseg)]];
             o[(size_t)r * d + j] = (double)hs[r] * (double)w2s[j] * acc;
         }
     }

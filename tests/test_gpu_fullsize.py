@@ -104,3 +104,76 @@ def test_skew_stress_routing_and_sampled_output():
         bias_orc, _ = oracle.bias_update(oracle.histogram(o_idx, cfg.E), bias_orc, cfg.T, cfg.k, cfg.step_size)
         assert (p["bias"].cpu().numpy().view(np.uint32) == bias_orc.view(np.uint32)).all()
     check_status()
+
+
+# ------------------------------------------------------------------ FP8 experts
+
+def _oracle_rows_fp8(q, x, idx, w, tokens, cfg):
+    """The oracle's FP8 layer output for the sampled tokens (page: "DeepSeek
+    V3 Architecture Deep Dive ...", "FP8 Formats"): tokens quantized per row,
+    every expert they use run from its E4M3 codes (brought back one expert at
+    a time), h quantized per assignment row, outputs summed in double."""
+    from fine_grained_moe_gate_b200.inputs import to_numpy
+    d, I, S, Is = cfg.d, cfg.I, cfg.S, cfg.Is
+    tokens = np.asarray(tokens)
+    xq, xs = oracle.quantize_rows_fp8(to_numpy(x[torch.as_tensor(tokens, device=DEV)]))
+    yacc = np.zeros((len(tokens), d), np.float64)
+    if S > 0:
+        h = oracle.expert_up_fp8(xq, xs, q["ws1q"].reshape(S * Is, d).cpu().numpy(), q["ws1s"].cpu().numpy(),
+                                 q["ws3q"].reshape(S * Is, d).cpu().numpy(), q["ws3s"].cpu().numpy())
+        hq, hs = oracle.quantize_rows_fp8(h)
+        yacc += oracle.expert_down_fp8(hq, hs, q["ws2q"].cpu().numpy(), q["ws2s"].cpu().numpy())
+    idx_np, w_np = idx.cpu().numpy()[tokens], w.cpu().numpy()[tokens]
+    for e in np.unique(idx_np):
+        ii, jj = np.nonzero(idx_np == e)
+        h = oracle.expert_up_fp8(xq[ii], xs[ii], q["w1q"][e].cpu().numpy(), q["w1s"][e * I:(e + 1) * I].cpu().numpy(),
+                                 q["w3q"][e].cpu().numpy(), q["w3s"][e * I:(e + 1) * I].cpu().numpy())
+        hq, hs = oracle.quantize_rows_fp8(h)
+        o = oracle.expert_down_fp8(hq, hs, q["w2q"][e].cpu().numpy(), q["w2s"][e * d:(e + 1) * d].cpu().numpy())
+        yacc[ii] += w_np[ii, jj].astype(np.float64)[:, None] * o
+    return oracle.finalize(yacc, np.uint16)
+
+
+def _fp8_check(cfg, p, q, w8, x, n_sample, seed):
+    sh = moe.shape_of(cfg)
+    T, k, d, E = cfg.T, cfg.k, cfg.d, cfg.E
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    ws = torch.empty(moe.moe_workspace_size(sh), dtype=torch.uint8, device=DEV)
+    moe.moe_layer_forward_fp8(x, p["w_gate"], p["bias"], w8, sh, y, idx, w, counts, ws)
+    torch.cuda.synchronize()
+    check_status()
+    ridx, rw, rcounts, _ = route(sh, x, p["w_gate"], p["bias"], with_aff=False)   # routing is the bf16 path's
+    assert torch.equal(ridx, idx) and torch.equal(rw, w) and torch.equal(rcounts, counts)
+    tokens = np.sort(np.random.default_rng(seed).choice(T, size=n_sample, replace=False))
+    ref = to_f64_rows(_oracle_rows_fp8(q, x, idx, w, tokens, cfg))
+    got = as_f64(y[torch.as_tensor(tokens, device=DEV)])
+    err = rel_fro(got, ref)
+    assert err <= 5e-3, err
+
+
+def test_v3_fp8_prefill_and_decode(v3_layer):
+    """V3 prefill (T=8192) and decode calls with E4M3 experts through
+    moe_layer_forward_fp8 (what the bench times); the weights are quantized on
+    the device and checked bit for bit on three sampled experts."""
+    _, p = v3_layer
+    q = moe.quantize_experts_fp8(p)
+    w8 = moe.fp8_experts(q)
+    torch.cuda.synchronize()
+    check_status()
+    from fine_grained_moe_gate_b200.inputs import to_numpy
+    for e in (0, 77, 255):
+        for n in ("w1", "w2"):
+            qo, so = oracle.quantize_rows_fp8(to_numpy(p[n][e]))
+            rows = p[n].shape[1]
+            assert np.array_equal(q[n + "q"][e].cpu().numpy(), qo)
+            assert np.array_equal(q[n + "s"][e * rows:(e + 1) * rows].cpu().numpy(), so)
+    cfg = CONFIGS["v3_prefill_fp8"]
+    _fp8_check(cfg, p, q, w8, make_tokens(cfg, DEV), n_sample=4, seed=12)
+    cfg = CONFIGS["v3_decode_fp8"]
+    for call in (0, 999):
+        _fp8_check(cfg, p, q, w8, make_tokens(cfg, DEV, call), n_sample=3, seed=call)
+    del q, w8
+    torch.cuda.empty_cache()
