@@ -2,12 +2,12 @@
 // "In code", route(); "The idea"): gate GEMM + sigmoid + bias-shifted top-k
 // + unbiased renormalised weights + load histogram in one kernel.
 //
-// One CTA = 128 tokens.  All E (<= 256) experts fit one tcgen05 MMA: the
+// A tile = 128 tokens.  All E (<= 256) experts fit one tcgen05 MMA: the
 // accumulator is 128 TMEM lanes (tokens) x E columns (experts), fp32.  The
-// K loop over d streams x and W_gate through a 4-stage TMA ring.  Epilogue
-// thread r owns token r: it reads its E scores from TMEM 16 at a time and
-// runs the shared top-k (topk.cuh) in registers, so no score matrix is
-// written unless the caller asks for the affinities.
+// K loop over d streams x and W_gate through a 4-stage TMA ring.  Small
+// batches split K over a cluster of up to 8 CTAs per tile (one CTA per tile
+// read all of W_gate alone, 3.7 MB at V3 through one SM); the scores only
+// leave shared memory for the caller's optional affinity output.
 #include "common.cuh"
 #include "kernels.h"
 #include "tmap.h"
@@ -20,6 +20,9 @@ constexpr int BM = 128, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_STRIDE = 256 * BK * 2;  // room for N <= 256 rows
 constexpr int NTHREADS = 192;
+constexpr int RING_BYTES = STAGES * (A_BYTES + B_STRIDE);
+constexpr int PS = kMaxExperts + 4;  // row stride (floats) of the score buffers
+constexpr int PART_BYTES = BM * PS * 4;
 
 struct Ctl {
     uint64_t full[STAGES];
@@ -31,9 +34,25 @@ struct Ctl {
     float bias[kMaxExperts];
     int hist[kMaxExperts];
 };
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * (A_BYTES + B_STRIDE) + sizeof(Ctl);
+// After the K loop the ring is reused for the partial scores of the CTA's K
+// slice ([128 tokens][E], fp32) and, with a split K, the reduced scores of the
+// tokens this CTA finishes.
+constexpr int SCORE_BYTES = PART_BYTES + BM / 2 * PS * 4;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)(RING_BYTES > SCORE_BYTES ? RING_BYTES : SCORE_BYTES) + sizeof(Ctl);
 
-template <int KMAX>
+__device__ __forceinline__ float ld_cluster_f32(uint32_t cluster_addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
+// Split K: the C CTAs of a cluster share one 128-token tile, CTA c running
+// the MMA over its slice of d; the slices' fp32 partial scores are summed in
+// the fixed order c = 0..C-1 through distributed shared memory (deterministic
+// for a given C), CTA c then finishes tokens [c*128/C, (c+1)*128/C) with C
+// threads per token, each taking every C-th expert, whose top-k lists are
+// merged with warp shuffles.  C = 1 is the plain one-CTA tile.
+template <int KMAX, int C>
 __global__ void __launch_bounds__(NTHREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ bias, int T, int E, int n_pad, uint32_t tmem_cols, int k_blocks,
@@ -43,9 +62,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sA = base;
     uint8_t* sB = base + STAGES * A_BYTES;
-    Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * (A_BYTES + B_STRIDE));
+    float* part = reinterpret_cast<float*>(base);                 // after the K loop
+    float* red = reinterpret_cast<float*>(base + PART_BYTES);     // split K only
+    const size_t ring_or_scores = RING_BYTES > SCORE_BYTES ? RING_BYTES : SCORE_BYTES;
+    Ctl* ctl = reinterpret_cast<Ctl*>(base + ring_or_scores);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int t0 = blockIdx.x * BM;
+    const int crank = C > 1 ? (int)cluster_ctarank() : 0;
+    const int t0 = (blockIdx.x / C) * BM;
+    const int kb0 = crank * k_blocks / C, kb1 = (crank + 1) * k_blocks / C;
 
     for (int e = tid; e < E; e += NTHREADS) {
         ctl->bias[e] = bias[e];
@@ -78,7 +102,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int stage = 0;
             uint32_t phase = 0, issued = 0, iss_phase = 0;
             bool ok = true;
-            for (int kb = 0; kb < k_blocks; ++kb) {
+            for (int kb = kb0; kb < kb1; ++kb) {
                 if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, status)) {
                     ok = false;
                     break;
@@ -106,7 +130,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int kb = 0; kb < k_blocks; ++kb) {
+            for (int kb = kb0; kb < kb1; ++kb) {
                 if (!mbar_wait(&ctl->full[stage], phase, &ctl->abort, status)) {
                     ok = false;
                     break;
@@ -117,7 +141,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
                     tc_mma_bf16(tmem_base, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
-                                (kb > 0 || kk > 0) ? 1u : 0u);
+                                (kb > kb0 || kk > 0) ? 1u : 0u);
                 tc_commit(&ctl->empty[stage]);
                 if (++stage == STAGES) {
                     stage = 0;
@@ -132,7 +156,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
         }
         __syncwarp();
-    } else {
+    } else if (C == 1) {
+        // whole K in this CTA: thread r owns token r and streams its scores
+        // from TMEM straight into the top-k
         const int q = warp & 3;
         const int r = q * 32 + lane;
         const int t = t0 + r;
@@ -157,28 +183,139 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (t < T) emit_route<KMAX>(tk, k, idx + (size_t)t * k, w + (size_t)t * k, ctl->hist, status);
         }
+    } else {
+        // partial scores of this K slice: TMEM lane r (token r) -> part[r][0..n_pad)
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        if (mbar_wait(&ctl->tfull, 0, &ctl->abort, status)) {
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
+            for (int c = 0; c < n_pad; c += 16) {
+                uint32_t v[16];
+                tmem_ld16(taddr + (uint32_t)c, v);
+                tmem_ld_wait();
+                float4* dst = reinterpret_cast<float4*>(part + r * PS + c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                         __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            }
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (C > 1) cluster_sync_all();  // every CTA's partial scores are complete and visible
+
+    if (C > 1 && warp >= 2) {
+        const int u = tid - 64;             // 0..127
+        constexpr int TPC = BM / C;         // tokens this CTA finishes
+        const int tl0 = crank * TPC;        // its first token within the tile
+        // scores s = sigmoid(sum of the C partials in CTA order), for this CTA's tokens
+        float* sc = red;
+        for (int it = u; it < TPC * E; it += 128) {
+            const int rl = it / E, e = it - rl * E;
+            const int r = tl0 + rl;
+            const uint32_t a = smem_u32(part + r * PS + e);
+            float z = ld_cluster_f32(mapa_shared(a, 0));
+#pragma unroll
+            for (int c = 1; c < C; ++c) z = __fadd_rn(z, ld_cluster_f32(mapa_shared(a, c)));
+            const float s = sigmoid_f32(z);
+            sc[rl * PS + e] = s;
+            if (aff && t0 + r < T) aff[(size_t)(t0 + r) * E + e] = s;
+        }
+        named_bar_sync(1, 128);
+        // top-k: C threads per token, thread `sub` pushes experts sub, sub + C, ...
+        const int rl = u / C, sub = u - rl * C;
+        const int t = t0 + tl0 + rl;
+        TopK<KMAX> tk;
+        tk.init();
+        for (int e = sub; e < E; e += C) {
+            const float s = sc[rl * PS + e];
+            tk.push(__fadd_rn(s, ctl->bias[e]), s, e);
+        }
+        {  // merge the C lists in (v desc, index asc) order
+            TopK<KMAX> m;
+            m.init();
+            int pos = 0;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                float hv = -FLT_MAX, hs = 0.f;
+                int hid = 0x7fffffff;
+#pragma unroll
+                for (int i = 0; i < KMAX; ++i)
+                    if (i == pos && tk.id[i] >= 0) {
+                        hv = tk.v[i];
+                        hs = tk.s[i];
+                        hid = tk.id[i];
+                    }
+                float bv = hv, bs = hs;
+                int bid = hid;
+#pragma unroll
+                for (int o = C / 2; o > 0; o >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+                    const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+                    if (ov > bv || (ov == bv && oid < bid)) {
+                        bv = ov;
+                        bs = os;
+                        bid = oid;
+                    }
+                }
+                if (bid != 0x7fffffff) {
+                    m.v[j] = bv;
+                    m.s[j] = bs;
+                    m.id[j] = bid;
+                    if (bid == hid) ++pos;
+                }
+            }
+            tk = m;
+        }
+        if (sub == 0 && t < T) emit_route<KMAX>(tk, k, idx + (size_t)t * k, w + (size_t)t * k, ctl->hist, status);
+    }
+    __syncthreads();
     for (int e = tid; e < E; e += NTHREADS)
         if (ctl->hist[e]) atomicAdd(&counts[e], ctl->hist[e]);
+    if (C > 1) cluster_sync_all();  // no CTA leaves while its partial scores may still be read
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, tmem_cols);
     }
 }
 
+template <int KMAX, int C>
+cudaError_t launch_kc(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int E, int n_pad,
+                      uint32_t cols, int kb, int k, int32_t* idx, float* w, int32_t* counts, float* aff, int* status,
+                      cudaStream_t st) {
+    auto kern = router_tc_kernel<KMAX, C>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(((T + BM - 1) / BM) * C));
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, kern, tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status);
+    note_launches(1);
+    return err == cudaSuccess ? cudaGetLastError() : err;
+}
+
 template <int KMAX>
 cudaError_t launch_k(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int E, int n_pad,
                      uint32_t cols, int kb, int k, int32_t* idx, float* w, int32_t* counts, float* aff, int* status,
-                     cudaStream_t st) {
-    auto kern = router_tc_kernel<KMAX>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    if (err != cudaSuccess) return err;
-    const int grid = (T + BM - 1) / BM;
-    kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status);
-    note_launches(1);
-    return cudaGetLastError();
+                     int split, cudaStream_t st) {
+    switch (split) {
+        case 8: return launch_kc<KMAX, 8>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
+        case 4: return launch_kc<KMAX, 4>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
+        case 2: return launch_kc<KMAX, 2>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
+        default: return launch_kc<KMAX, 1>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
+    }
 }
 
 }  // namespace
@@ -186,7 +323,6 @@ cudaError_t launch_k(const CUtensorMap& tx, const CUtensorMap& tw, const float* 
 cudaError_t launch_router_tc(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
                              int32_t* idx, float* w, int32_t* counts, float* aff, int* status, int num_sms,
                              cudaStream_t st) {
-    (void)num_sms;
     if (T == 0) return cudaSuccess;
     if (d % BK != 0 || E > kMaxExperts || E <= 0) return cudaErrorInvalidValue;
     const int n_pad = (E + 15) / 16 * 16;  // MMA N: multiple of 16 for M = 128
@@ -195,8 +331,12 @@ cudaError_t launch_router_tc(const void* x, const void* wg, const float* bias, i
     CUtensorMap tx, tw;
     if (!make_tmap_2d(&tx, x, d, T, d, BK, BM) || !make_tmap_2d(&tw, wg, d, E, d, BK, n_pad))
         return cudaErrorInvalidValue;
-    return k <= 8 ? launch_k<8>(tx, tw, bias, T, E, n_pad, cols, d / BK, k, idx, w, counts, aff, status, st)
-                  : launch_k<16>(tx, tw, bias, T, E, n_pad, cols, d / BK, k, idx, w, counts, aff, status, st);
+    // K split: as many CTAs per token tile as keep the grid within one wave of SMs
+    const int tiles = (T + BM - 1) / BM, kb = d / BK;
+    int split = 8;
+    while (split > 1 && (tiles * split > num_sms || split > kb)) split >>= 1;
+    return k <= 8 ? launch_k<8>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, split, st)
+                  : launch_k<16>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, split, st);
 }
 
 }  // namespace moe
