@@ -34,6 +34,7 @@ EXPORTS = (
     "moe_ffn_down", "moe_combine", "moe_layer_forward", "moe_workspace_size", "moe_get_last_error",
     "moe_kernel_launch_count", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
     "moe_quantize_fp8", "moe_ffn_up_fp8", "moe_ffn_down_fp8", "moe_layer_forward_fp8",
+    "moe_ep_plan_size", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_return",
 )
 
 MOE_ROUTED, MOE_SHARED = 0, 1
@@ -105,6 +106,9 @@ def lib() -> ctypes.CDLL:
             "moe_ffn_up_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_ffn_down_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_layer_forward_fp8": [P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P, P, P, sz, P],
+            "moe_ep_plan": [P, ctypes.c_int32, ctypes.c_int32, S, P, P, P],
+            "moe_ep_dispatch": [P, P, P, ctypes.c_int32, ctypes.c_int32, S, P, P],
+            "moe_ep_return": [P, P, ctypes.c_int32, ctypes.c_int32, S, P, P],
             "moe_selftest_bounded_wait": [ctypes.c_uint32, P],
         }
         for name, args in sig.items():
@@ -115,6 +119,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.argtypes = [S]
             fn.restype = sz
+        L.moe_ep_plan_size.argtypes = [ctypes.c_int32, S]
+        L.moe_ep_plan_size.restype = sz
         L.moe_kernel_launch_count.argtypes = []
         L.moe_kernel_launch_count.restype = ctypes.c_uint64
         L.moe_status_string.argtypes = [ctypes.c_int]
@@ -294,3 +300,33 @@ def quantize_experts_fp8(p: dict, stream=None) -> dict:
         moe_quantize_fp8(w, d, Is, S, q, sc, stream)
         out["ws2q"], out["ws2s"] = q, sc
     return out
+
+
+# ---- expert parallelism --------------------------------------------------------
+
+def _ptr_array(bufs):
+    arr = (ctypes.c_void_p * len(bufs))()
+    for i, b in enumerate(bufs):
+        arr[i] = b if isinstance(b, int) else b.data_ptr()
+    return arr
+
+
+def moe_ep_plan_size(world, shape) -> int:
+    return lib().moe_ep_plan_size(world, shape)
+
+
+def moe_ep_plan(counts_all, world, rank, shape, plan, recv_offsets, stream=None):
+    _check(lib().moe_ep_plan(_p(counts_all), world, rank, shape, _p(plan), _p(recv_offsets), _stream(stream)),
+           "moe_ep_plan")
+
+
+def moe_ep_dispatch(x, perm_tok, plan, world, rank, shape, recv_bufs, stream=None):
+    """recv_bufs: per rank, its receive buffer (tensor or device pointer valid here)."""
+    _check(lib().moe_ep_dispatch(_p(x), _p(perm_tok), _p(plan), world, rank, shape, _ptr_array(recv_bufs),
+                                 _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_return(y_recv, plan, world, rank, shape, back_bufs, stream=None):
+    """back_bufs: per rank, its return buffer (tensor or device pointer valid here)."""
+    _check(lib().moe_ep_return(_p(y_recv), _p(plan), world, rank, shape, _ptr_array(back_bufs), _stream(stream)),
+           "moe_ep_return")

@@ -688,6 +688,89 @@ moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float*
                : MOE_ERR_CUDA;
 }
 
+size_t moe_ep_plan_size(int32_t world, moe_shape sh) {
+    if (validate_shape(sh) != MOE_OK || world < 1 || world > moe::kMaxRanks || sh.E % world != 0) return 0;
+    return align256(moe::ep_plan_ints(world, sh.E) * sizeof(int32_t));
+}
+
+moe_status moe_ep_plan(const int32_t* counts_all, int32_t world, int32_t rank, moe_shape sh, int32_t* plan,
+                       int32_t* recv_offsets, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(world >= 1 && world <= moe::kMaxRanks && sh.E % world == 0 && rank >= 0 && rank < world,
+                MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(counts_all && plan, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(counts_all) && aligned16(plan) && aligned16(recv_offsets), MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (moe::launch_ep_plan(counts_all, world, sh.E, plan, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (recv_offsets) {
+        const int Epr = sh.E / world;
+        const size_t at = (size_t)sh.E * world + (size_t)world * (sh.E + 1) + (size_t)rank * (Epr + 1);
+        MOE_CUDA(cudaMemcpyAsync(recv_offsets, plan + at, sizeof(int32_t) * (Epr + 1), cudaMemcpyDeviceToDevice, st));
+    }
+    return MOE_OK;
+}
+
+namespace {
+moe_status ep_peers(void* const* bufs, int32_t world, moe::EpPeers* out) {
+    MOE_REQUIRE(bufs, MOE_ERR_INVALID_ARG);
+    for (int i = 0; i < moe::kMaxRanks; ++i) out->p[i] = nullptr;
+    for (int i = 0; i < world; ++i) {
+        MOE_REQUIRE(bufs[i], MOE_ERR_INVALID_ARG);
+        MOE_REQUIRE(aligned16(bufs[i]), MOE_ERR_ALIGNMENT);
+        out->p[i] = bufs[i];
+    }
+    return MOE_OK;
+}
+}  // namespace
+
+moe_status moe_ep_dispatch(const void* x, const int32_t* perm_tok, const int32_t* plan, int32_t world, int32_t rank,
+                           moe_shape sh, void* const* recv_bufs, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(!is_fp8(sh), MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(world >= 1 && world <= moe::kMaxRanks && sh.E % world == 0 && rank >= 0 && rank < world,
+                MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(plan && (sh.T == 0 || (x && perm_tok)), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x) && aligned16(perm_tok) && aligned16(plan), MOE_ERR_ALIGNMENT);
+    moe::EpPeers peers;
+    if ((v = ep_peers(recv_bufs, world, &peers)) != MOE_OK) return v;
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    if (sh.T == 0) return MOE_OK;
+    return moe::launch_ep_dispatch(x, perm_tok, plan, world, sh.E, sh.k, rank, sh.T, (size_t)sh.d * esize(sh), peers,
+                                   sms, status, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_return(const void* y_recv, const int32_t* plan, int32_t world, int32_t rank, moe_shape sh,
+                         void* const* back_bufs, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(!is_fp8(sh), MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(world >= 1 && world <= moe::kMaxRanks && sh.E % world == 0 && rank >= 0 && rank < world,
+                MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(plan && y_recv, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(y_recv) && aligned16(plan), MOE_ERR_ALIGNMENT);
+    moe::EpPeers peers;
+    if ((v = ep_peers(back_bufs, world, &peers)) != MOE_OK) return v;
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return moe::launch_ep_return(y_recv, plan, world, sh.E, sh.k, rank, sh.T, (size_t)sh.d * esize(sh), peers, sms,
+                                 status, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
 moe_status moe_selftest_bounded_wait(uint32_t limit_us, void* stream) {
     MOE_REQUIRE(limit_us > 0 && limit_us <= 5000000u, MOE_ERR_INVALID_ARG);
     int dev, sms;

@@ -106,6 +106,21 @@ struct TcDownArgs {
     const float* w2s = nullptr;
     const float* hs = nullptr;
 };
+// ep.cu: expert-parallel dispatch / return over peer memory.  Plan layout
+// (int32): base [E][W], src_off [W][E+1], recv_off [W][E/W+1].
+constexpr int kMaxRanks = 64;
+struct EpPeers {
+    void* p[kMaxRanks];  // per rank: a device pointer valid in this process (peer memory)
+};
+size_t ep_plan_ints(int W, int E);
+cudaError_t launch_ep_plan(const int32_t* counts_all, int W, int E, int32_t* plan, cudaStream_t st);
+// Every rank holds T tokens: receive buffers W*T*k rows, return buffers T*k.
+cudaError_t launch_ep_dispatch(const void* x, const int32_t* perm_tok, const int32_t* plan, int W, int E, int k,
+                               int rank, int T, size_t row_bytes, const EpPeers& recv, int num_sms, int* status,
+                               cudaStream_t st);
+cudaError_t launch_ep_return(const void* y, const int32_t* plan, int W, int E, int k, int rank, int T,
+                             size_t row_bytes, const EpPeers& back, int num_sms, int* status, cudaStream_t st);
+
 // quant.cu: per-row E4M3 quantization of a bf16 matrix with `rows` rows
 // stored as nseg column blocks of kseg columns (kseg % 8 == 0).
 cudaError_t launch_quantize_e4m3(const void* src, long long rows, int kseg, int nseg, uint8_t* q, float* scale,

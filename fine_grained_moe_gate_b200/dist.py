@@ -30,3 +30,134 @@ def allreduce_counts(counts: torch.Tensor, group=None) -> torch.Tensor:
     if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
         dist.all_reduce(counts, op=dist.ReduceOp.SUM, group=group)
     return counts
+
+
+# ---- expert parallelism ---------------------------------------------------------
+#
+# Experts sharded over the ranks (rank o owns experts [o*E/W, (o+1)*E/W)),
+# tokens kept where they are: each rank routes its own tokens, the step's
+# counts are gathered (a few KB), and the token rows travel to the experts'
+# owners and the expert outputs back through the library's peer-store
+# kernels (moe_ep_dispatch / moe_ep_return) -- no NCCL data all-to-all.
+
+def exchange_counts(counts: torch.Tensor, world: int, group=None) -> torch.Tensor:
+    """All ranks' per-expert counts [W][E] (int32), gathered in rank order."""
+    import torch.distributed as dist
+    out = torch.empty((world, counts.numel()), dtype=counts.dtype, device=counts.device)
+    if world == 1:
+        out[0].copy_(counts)
+        return out
+    dist.all_gather_into_tensor(out, counts.reshape(1, -1).contiguous(), group=group)
+    return out
+
+
+def local_experts(p: dict, rank: int, world: int) -> dict:
+    """Views of the expert weights rank `rank` owns (contiguous slices)."""
+    E = p["w1"].shape[0]
+    e0, e1 = rank * E // world, (rank + 1) * E // world
+    return {"w1": p["w1"][e0:e1], "w3": p["w3"][e0:e1], "w2": p["w2"][e0:e1]}
+
+
+class EPBuffers:
+    """One rank's per-step device buffers for ep_forward_steps.  `recv` and
+    `back` are the buffers peers store into: allocate them where peers can
+    reach them (symmetric memory across GPUs; any allocation on one GPU)."""
+
+    def __init__(self, cfg, world: int, device, recv=None, back=None):
+        T, k, d, E, I = cfg.T, cfg.k, cfg.d, cfg.E, cfg.I
+        dt = cfg.torch_dtype
+        cap = world * T * k                          # receive capacity: every rank sends all its rows here
+        i32 = torch.int32
+        self.recv = recv if recv is not None else torch.empty((cap, d), dtype=dt, device=device)
+        self.back = back if back is not None else torch.empty((T * k, d), dtype=dt, device=device)
+        self.h_recv = torch.empty((cap, I), dtype=dt, device=device)
+        self.y_recv = torch.empty((cap, d), dtype=dt, device=device)
+        self.idx = torch.empty((T, k), dtype=i32, device=device)
+        self.w = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.counts = torch.empty(E, dtype=i32, device=device)
+        self.offsets = torch.empty(E + 1, dtype=i32, device=device)
+        self.perm = torch.empty(T * k, dtype=i32, device=device)
+        self.inv = torch.empty(T * k, dtype=i32, device=device)
+        self.recv_offsets = torch.empty(E // world + 1, dtype=i32, device=device)
+        self.hs = torch.empty((T, max(1, cfg.S * cfg.Is)), dtype=dt, device=device)
+        self.shared_out = torch.empty((T, d), dtype=dt, device=device) if cfg.S > 0 else None
+        self.y = torch.empty((T, d), dtype=dt, device=device)
+        self.flag = torch.zeros(1, dtype=torch.float32, device=device)
+        self._pws = None
+        self._plan = None
+
+    def scratch(self, moe, sh, world):
+        if self._pws is None:
+            self._pws = torch.empty(max(moe.moe_permute_workspace_size(sh), 256), dtype=torch.uint8,
+                                    device=self.y.device)
+            self._plan = torch.empty(max(moe.moe_ep_plan_size(world, sh), 256) // 4, dtype=torch.int32,
+                                     device=self.y.device)
+        return self._pws, self._plan
+
+
+def ep_forward_steps(moe, cfg, rank: int, world: int, x, p: dict, bufs: EPBuffers, recv_ptrs, back_ptrs,
+                     stream=None):
+    """One rank's expert-parallel layer forward, as a generator.
+
+    Yields ("counts", counts) and expects the step's counts of all ranks
+    [W][E] to be sent back; yields ("barrier",) where every rank's peer
+    stores must be complete before it is resumed.  Returns y [T][d] (the
+    generator's value).  p holds the replicated router weights and shared
+    experts plus this rank's experts (``local_experts``); recv_ptrs[o] is
+    rank o's receive buffer, back_ptrs[s] rank s's return buffer."""
+    from . import MoEShape, MOE_SHARED, shape_of
+    sh = shape_of(cfg)
+    Epr = cfg.E // world
+    # the GEMMs on the receive buffer: this rank's experts, rows by offsets,
+    # capacity W*T*k rows (k = 1 so that the local expert count may be < k)
+    sh_local = MoEShape(world * cfg.T * cfg.k, cfg.d, Epr, 1, cfg.I, 0, cfg.Is, sh.dtype)
+    pws, plan = bufs.scratch(moe, sh, world)
+    moe.moe_route(x, p["w_gate"], p["bias"], sh, bufs.idx, bufs.w, bufs.counts, None, stream)
+    counts_all = yield ("counts", bufs.counts)
+    moe.moe_permute(x, bufs.idx, bufs.counts, sh, None, bufs.offsets, bufs.perm, bufs.inv, pws, stream)
+    moe.moe_ep_plan(counts_all, world, rank, sh, plan, bufs.recv_offsets, stream)
+    moe.moe_ep_dispatch(x, bufs.perm, plan, world, rank, sh, recv_ptrs, stream)
+    yield ("barrier",)
+    moe.moe_ffn_up(bufs.recv, bufs.recv_offsets, p["w1"], p["w3"], None, None, None, sh_local, bufs.h_recv, None,
+                   stream)
+    moe.moe_ffn_down(bufs.h_recv, bufs.recv_offsets, p["w2"], None, None, sh_local, bufs.y_recv, None, stream)
+    if cfg.S > 0:
+        moe.moe_expert_up(x, None, None, p["ws1"], p["ws3"], sh, MOE_SHARED, bufs.hs, stream)
+        moe.moe_expert_down(bufs.hs, None, p["ws2"], sh, MOE_SHARED, bufs.shared_out, stream)
+    moe.moe_ep_return(bufs.y_recv, plan, world, rank, sh, back_ptrs, stream)
+    yield ("barrier",)
+    moe.moe_combine(bufs.back, bufs.w, bufs.inv, bufs.shared_out, sh, bufs.y, stream)
+    return bufs.y
+
+
+def ep_forward(moe, cfg, rank: int, world: int, x, p: dict, bufs: EPBuffers, recv_ptrs, back_ptrs, group=None):
+    """ep_forward_steps driven across processes: counts gathered with
+    all_gather, barriers as a stream-ordered all-reduce of one float (it
+    completes on every rank only after every rank's earlier kernels, so the
+    peer stores have landed).  Not run on more than one GPU in this build."""
+    import torch.distributed as dist
+    gen = ep_forward_steps(moe, cfg, rank, world, x, p, bufs, recv_ptrs, back_ptrs)
+    msg = next(gen)
+    while True:
+        try:
+            if msg[0] == "counts":
+                msg = gen.send(exchange_counts(msg[1], world, group))
+            else:
+                dist.all_reduce(bufs.flag, group=group)
+                msg = gen.send(None)
+        except StopIteration as stop:
+            return stop.value
+
+
+def ep_symmetric_buffers(cfg, world: int, device, group_name: str):
+    """Receive and return buffers in symmetric memory, with every rank's
+    device pointers (torch.distributed._symmetric_memory; NVLink peers).
+    Returns (recv, back, recv_ptrs, back_ptrs).  Not run on more than one GPU
+    in this build."""
+    import torch.distributed._symmetric_memory as symm_mem
+    T, k, d = cfg.T, cfg.k, cfg.d
+    recv = symm_mem.empty((world * T * k, d), dtype=cfg.torch_dtype, device=device)
+    back = symm_mem.empty((T * k, d), dtype=cfg.torch_dtype, device=device)
+    hr = symm_mem.rendezvous(recv, group_name)
+    hb = symm_mem.rendezvous(back, group_name)
+    return recv, back, list(hr.buffer_ptrs), list(hb.buffer_ptrs)

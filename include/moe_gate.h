@@ -310,6 +310,40 @@ MOE_API moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, cons
                                          float* topk_w, int32_t* counts, void* workspace, size_t ws_bytes,
                                          void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Expert parallelism (no counterpart in the pages' code; their "custom
+ * all-to-all kernels for MoE dispatch/combine", crackai.dev "DeepSeek-V3",
+ * "How It Works").  W ranks, one per GPU; rank o owns experts
+ * [o*E/W, (o+1)*E/W) (E % W == 0, W <= 64) and keeps its own T tokens.  Per
+ * step, on every rank:
+ *   1. moe_route and moe_permute (x_perm may be NULL) on the local tokens;
+ *   2. gather all ranks' counts into counts_all [W][E] (any collective);
+ *   3. moe_ep_plan: the receive layout, identical on every rank;
+ *   4. moe_ep_dispatch: this rank's permuted rows go straight into the
+ *      owners' receive buffers (peer stores); then a barrier across ranks;
+ *   5. the grouped GEMMs (moe_ffn_up / moe_ffn_down, shape with E/W experts)
+ *      on the receive buffer with recv_offsets; the shared experts on the
+ *      local tokens (moe_expert_up / moe_expert_down, MOE_SHARED);
+ *   6. moe_ep_return: each output row goes straight back into its source
+ *      rank's return buffer, at the row's place in that rank's own
+ *      permutation; then a barrier;
+ *   7. moe_combine on the return buffer with the local inv_row.
+ * A receive buffer holds its experts in order, each expert's rows by source
+ * rank, each source's rows by token: the rows, and so the results, of the
+ * single-GPU layer over the ranks' concatenated batch (same routing).
+ * Receive buffers need W*T*k rows of capacity at most; return buffers T*k.
+ * recv_bufs / back_bufs: host arrays of W device pointers valid in the
+ * calling process (peer memory, e.g. IPC or symmetric memory; on one GPU
+ * plain allocations).  bf16 and fp32 rows; MOE_FP8_E4M3 is unsupported.
+ * -------------------------------------------------------------------------*/
+MOE_API size_t moe_ep_plan_size(int32_t world, moe_shape sh);  /* bytes; 0 if invalid */
+MOE_API moe_status moe_ep_plan(const int32_t* counts_all, int32_t world, int32_t rank, moe_shape sh, int32_t* plan,
+                               int32_t* recv_offsets, void* stream);  /* recv_offsets [E/W+1]: this rank's */
+MOE_API moe_status moe_ep_dispatch(const void* x, const int32_t* perm_tok, const int32_t* plan, int32_t world,
+                                   int32_t rank, moe_shape sh, void* const* recv_bufs, void* stream);
+MOE_API moe_status moe_ep_return(const void* y_recv, const int32_t* plan, int32_t world, int32_t rank,
+                                 moe_shape sh, void* const* back_bufs, void* stream);
+
 /* Synchronises `stream`, then returns and clears the current device's
  * status word (MOE_OK if no kernel reported an anomaly). */
 MOE_API moe_status moe_get_last_error(void* stream);

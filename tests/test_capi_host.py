@@ -137,6 +137,22 @@ def test_ffn_checks(L):
                           None) == UNSUPPORTED
 
 
+def test_ep_checks(L):
+    c = ctypes.c_void_p
+    sh = shape(E=16, k=4)
+    peers = (ctypes.c_void_p * 4)(FAKE, FAKE, FAKE, FAKE)
+    assert moe.moe_ep_plan_size(4, sh) > 0 and moe.moe_ep_plan_size(3, sh) == 0        # E % W != 0
+    assert L.moe_ep_dispatch(c(FAKE), c(FAKE), c(FAKE), 3, 0, sh, peers, None) == INVALID
+    assert L.moe_ep_dispatch(c(FAKE), c(FAKE), c(FAKE), 4, 4, sh, peers, None) == INVALID   # rank out of range
+    assert L.moe_ep_dispatch(c(FAKE), c(FAKE), c(FAKE), 4, 0, shape(E=16, k=4, dtype=moe.MOE_FP8_E4M3, d=256,
+                                                                          I=128, Is=128), peers, None) == UNSUPPORTED
+    bad = (ctypes.c_void_p * 4)(FAKE, None, FAKE, FAKE)
+    assert L.moe_ep_dispatch(c(FAKE), c(FAKE), c(FAKE), 4, 0, sh, bad, None) == INVALID
+    odd = (ctypes.c_void_p * 4)(FAKE, FAKE + 8, FAKE, FAKE)
+    assert L.moe_ep_return(c(FAKE), c(FAKE), 4, 1, sh, odd, None) == ALIGN
+    assert L.moe_ep_plan(c(FAKE), 4, 5, sh, c(FAKE), None, None) == INVALID
+
+
 def test_bias_update_checks(L):
     c = ctypes.c_void_p
     assert L.moe_load_and_bias_update(c(FAKE), shape(T=0), ctypes.c_float(1e-3), None, c(FAKE), None, None) == INVALID

@@ -99,3 +99,40 @@ def test_a_failed_rank_ends_the_exchange_with_an_error_not_a_hang():
     assert "injected" in res[1]["error"]
     assert res[0]["error"] is not None             # the survivor's all-reduce errored out within the timeout
     assert len(res[0]["biases"]) == 0
+
+
+def _ep_worker(rank, port, out_dir):
+    import torch.distributed as dist
+
+    import oracle
+    from fine_grained_moe_gate_b200 import dist as mdist
+    from fine_grained_moe_gate_b200.inputs import make_layer, make_tokens, to_numpy
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD, timeout=datetime.timedelta(seconds=10))
+    cfg = _cfg()
+    p = make_layer(cfg, "cpu")
+    x = make_tokens(cfg, "cpu", step=mdist.shard_step(0, rank, WORLD))
+    idx, _ = oracle.select(oracle.affinity(to_numpy(x), to_numpy(p["w_gate"])), p["bias"].numpy(), cfg.k)
+    counts = torch.from_numpy(oracle.histogram(idx, cfg.E))
+    allc = mdist.exchange_counts(counts, WORLD)
+    with open(os.path.join(out_dir, f"ep{rank}.json"), "w") as f:
+        json.dump({"counts_all": allc.tolist(), "own": counts.tolist()}, f)
+    dist.destroy_process_group()
+
+
+def test_expert_parallel_counts_exchange():
+    """Expert parallelism's one host-side exchange: every rank ends with the
+    same [W][E] counts in rank order, from which each owner's receive size
+    (its experts' columns summed over the sources) follows."""
+    out_dir = tempfile.mkdtemp(prefix="gloo_ep_")
+    mp.start_processes(_ep_worker, args=(_free_port(), out_dir), nprocs=WORLD, join=True, start_method="spawn")
+    res = [json.load(open(os.path.join(out_dir, f"ep{r}.json"))) for r in range(WORLD)]
+    assert res[0]["counts_all"] == res[1]["counts_all"]
+    assert res[0]["counts_all"] == [res[r]["own"] for r in range(WORLD)]
+    cfg = _cfg()
+    allc = np.array(res[0]["counts_all"])
+    Epr = cfg.E // WORLD
+    recv = [allc[:, o * Epr:(o + 1) * Epr].sum() for o in range(WORLD)]
+    assert sum(recv) == WORLD * cfg.T * cfg.k
