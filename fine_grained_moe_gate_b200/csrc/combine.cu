@@ -4,7 +4,8 @@
 // shared experts' output):
 //   y[t] = shared[t] + sum_j w[t][j] * y_perm[inv_row[t*k + j]]
 // fp32 accumulation in that fixed order (deterministic), one rounding to the
-// output type.  One CTA per token, 16-byte vector loads.
+// output type.  One CTA per token, 16-byte vector loads.  HBM bound:
+// (k + 1) rows read and one written per token.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -45,22 +46,31 @@ struct Vec<__nv_bfloat16> {
     }
 };
 
-template <typename T>
+// The k rows' vectors are all loaded before the sum (KMAX-wide, predicated),
+// so each thread keeps k loads in flight instead of one.
+template <typename T, int KMAX>
 __global__ void combine_kernel(const uint4* __restrict__ y_perm, const float* __restrict__ w,
                                const int32_t* __restrict__ inv_row, const uint4* __restrict__ shared, int k,
                                int vec_per_row, int total_rows, uint4* __restrict__ y, int* status) {
     constexpr int n = Vec<T>::n;
     const int t = blockIdx.x;
-    __shared__ int rows[16];
-    __shared__ float ws[16];
+    __shared__ int rows[KMAX];
+    __shared__ float ws[KMAX];
     if (threadIdx.x < k) {
-        const int r = inv_row[(size_t)t * k + threadIdx.x];
-        if ((unsigned)r >= (unsigned)total_rows) report(status, kStDeviceCheck);
+        int r = inv_row[(size_t)t * k + threadIdx.x];
+        if ((unsigned)r >= (unsigned)total_rows) {
+            report(status, kStDeviceCheck);
+            r = -1;
+        }
         rows[threadIdx.x] = r;
         ws[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
     }
     __syncthreads();
     for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) {
+        uint4 in[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            if (j < k && rows[j] >= 0) in[j] = y_perm[(size_t)rows[j] * vec_per_row + v];
         float acc[n], tmp[n];
         if (shared) {
             Vec<T>::unpack(shared[(size_t)t * vec_per_row + v], acc);
@@ -68,16 +78,37 @@ __global__ void combine_kernel(const uint4* __restrict__ y_perm, const float* __
 #pragma unroll
             for (int i = 0; i < n; ++i) acc[i] = 0.f;
         }
-        for (int j = 0; j < k; ++j) {
-            const int r = rows[j];
-            if ((unsigned)r >= (unsigned)total_rows) continue;
-            Vec<T>::unpack(y_perm[(size_t)r * vec_per_row + v], tmp);
-            const float wj = ws[j];
 #pragma unroll
-            for (int i = 0; i < n; ++i) acc[i] = fmaf(wj, tmp[i], acc[i]);
+        for (int j = 0; j < KMAX; ++j) {
+            if (j < k && rows[j] >= 0) {
+                Vec<T>::unpack(in[j], tmp);
+                const float wj = ws[j];
+#pragma unroll
+                for (int i = 0; i < n; ++i) acc[i] = fmaf(wj, tmp[i], acc[i]);
+            }
         }
         y[(size_t)t * vec_per_row + v] = Vec<T>::pack(acc);
     }
+}
+
+template <typename T>
+void launch_t(const void* y_perm, const float* w, const int32_t* inv_row, const void* shared, int T_, int k, int vec,
+              void* y, int* status, cudaStream_t st) {
+    // threads: a multiple of 32 that divides the row's vectors when one does (no idle tail pass)
+    int threads = 256;
+    for (int c = 256; c >= 96; c -= 32)
+        if (vec % c == 0) {
+            threads = c;
+            break;
+        }
+    if (vec < 256) threads = ((vec + 31) / 32) * 32;
+    const uint4* yp = static_cast<const uint4*>(y_perm);
+    const uint4* sh = static_cast<const uint4*>(shared);
+    uint4* out = static_cast<uint4*>(y);
+    if (k <= 8)
+        combine_kernel<T, 8><<<T_, threads, 0, st>>>(yp, w, inv_row, sh, k, vec, T_ * k, out, status);
+    else
+        combine_kernel<T, 16><<<T_, threads, 0, st>>>(yp, w, inv_row, sh, k, vec, T_ * k, out, status);
 }
 
 cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* inv_row, const void* shared, int T,
@@ -85,15 +116,10 @@ cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* in
     if (T == 0) return cudaSuccess;
     const size_t eb = bf16 ? 2 : 4;
     const int vec = (int)((size_t)d * eb / 16);
-    const int threads = vec >= 256 ? 256 : ((vec + 31) / 32) * 32;
     if (bf16)
-        combine_kernel<__nv_bfloat16><<<T, threads, 0, st>>>(static_cast<const uint4*>(y_perm), w, inv_row,
-                                                              static_cast<const uint4*>(shared), k, vec, T * k,
-                                                              static_cast<uint4*>(y), status);
+        launch_t<__nv_bfloat16>(y_perm, w, inv_row, shared, T, k, vec, y, status, st);
     else
-        combine_kernel<float><<<T, threads, 0, st>>>(static_cast<const uint4*>(y_perm), w, inv_row,
-                                                      static_cast<const uint4*>(shared), k, vec, T * k,
-                                                      static_cast<uint4*>(y), status);
+        launch_t<float>(y_perm, w, inv_row, shared, T, k, vec, y, status, st);
     note_launches(1);
     return cudaGetLastError();
 }
