@@ -49,12 +49,15 @@ __global__ void permute_scan_kernel(int32_t* __restrict__ hist, int C, int E, co
     __shared__ int tot[256];
     __shared__ int warp_sum[8];
     const int e = threadIdx.x;
+    constexpr int U = 8;  // chunk counts loaded per batch: independent loads in flight
     int running = 0;
     if (e < E) {
-        for (int c = 0; c < C; ++c) {
-            const int h = hist[(size_t)c * E + e];
-            hist[(size_t)c * E + e] = running;
-            running += h;
+        for (int c0 = 0; c0 < C; c0 += U) {
+            int h[U];
+#pragma unroll
+            for (int i = 0; i < U; ++i) h[i] = c0 + i < C ? hist[(size_t)(c0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < U; ++i) running += h[i];
         }
         if (counts && counts[e] != running) report(status, kStDeviceCheck);
     }
@@ -82,9 +85,19 @@ __global__ void permute_scan_kernel(int32_t* __restrict__ hist, int C, int E, co
         offsets[E] = all;
     }
     __syncthreads();
-    if (e < E) {
-        const int base = tot[e];
-        for (int c = 0; c < C; ++c) hist[(size_t)c * E + e] += base;
+    if (e < E) {  // base[c][e] = offsets[e] + counts of expert e in chunks before c
+        int acc = tot[e];
+        for (int c0 = 0; c0 < C; c0 += U) {
+            int h[U];
+#pragma unroll
+            for (int i = 0; i < U; ++i) h[i] = c0 + i < C ? hist[(size_t)(c0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < U; ++i)
+                if (c0 + i < C) {
+                    hist[(size_t)(c0 + i) * E + e] = acc;
+                    acc += h[i];
+                }
+        }
     }
 }
 
@@ -129,12 +142,23 @@ __global__ void permute_scatter_kernel(const uint4* __restrict__ x, int vec_per_
     if (threadIdx.x < k) rows[threadIdx.x] = inv_row[(size_t)t * k + threadIdx.x];
     __syncthreads();
     const uint4* src = x + (size_t)t * vec_per_row;
-    for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) {
-        const uint4 val = src[v];
-#pragma unroll 4
+    constexpr int U = 4;  // vectors loaded per thread before the k stores of each
+    for (int v0 = threadIdx.x; v0 < vec_per_row; v0 += blockDim.x * U) {
+        uint4 val[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int v = v0 + u * blockDim.x;
+            if (v < vec_per_row) val[u] = src[v];
+        }
         for (int j = 0; j < k; ++j) {
             const int r = rows[j];
-            if ((unsigned)r < (unsigned)total_rows) xp[(size_t)r * vec_per_row + v] = val;
+            if ((unsigned)r >= (unsigned)total_rows) continue;
+            uint4* dst = xp + (size_t)r * vec_per_row;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + u * blockDim.x;
+                if (v < vec_per_row) dst[v] = val[u];
+            }
         }
     }
 }
@@ -162,8 +186,15 @@ cudaError_t launch_permute(const void* x, const int32_t* idx, const int32_t* cou
         ++launched;
         if (x && x_perm) {
             const int vec = (int)((size_t)d * elem_bytes / 16);
-            permute_scatter_kernel<<<T, 128, 0, st>>>(static_cast<const uint4*>(x), vec, k, inv_row, T * k,
-                                                       static_cast<uint4*>(x_perm));
+            // a block size that divides the row's vectors in U = 4 passes when one does
+            int threads = 128;
+            for (int c = 256; c >= 64; c -= 32)
+                if (vec % (4 * c) == 0) {
+                    threads = c;
+                    break;
+                }
+            permute_scatter_kernel<<<T, threads, 0, st>>>(static_cast<const uint4*>(x), vec, k, inv_row, T * k,
+                                                           static_cast<uint4*>(x_perm));
             ++launched;
         }
     }
