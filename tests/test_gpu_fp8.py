@@ -45,7 +45,8 @@ def _quant(src: torch.Tensor, rows, kseg, nseg=1):
     return q, sc
 
 
-@pytest.mark.parametrize("rows,K,std", [(37, 200, 0.05), (9, 7168, 1.0), (300, 2048, 3e-3), (1, 8, 100.0)])
+@pytest.mark.parametrize("rows,K,std", [(37, 200, 0.05), (9, 7168, 1.0), (300, 2048, 3e-3), (1, 8, 100.0),
+                                        (5, 10240, 0.5), (3, 4104, 2.0)])
 def test_quantize_rows_bit_exact(rows, K, std):
     g = torch.Generator(device=DEV).manual_seed(rows * 31 + K)
     a = (torch.randn((rows, K), generator=g, device=DEV) * std).to(torch.bfloat16)
