@@ -34,19 +34,28 @@
 // find them in L2, and the last tiles spread over the clusters that are free.
 // Per expert, token tiles are walked fastest, then feature tiles.
 //
-// Warp roles (192 threads per CTA):
-//   warp 0      TMA producer (one lane), both CTAs: loads its own halves,
-//               completion counted on the leader CTA's barrier.  The
-//               leader's producer takes tiles from the counter and posts
-//               them in a small tile queue in both CTAs' shared memory for
-//               every other role, one tile ahead of its own loads (the
-//               atomic's round trip overlaps the current tile's loads).
+// Warp roles per CTA (up: 12 warps, down: 7):
+//   warp 0      weight producer (one lane), both CTAs: loads this CTA's
+//               weight rows (up: the W1 half), completion counted on the
+//               leader CTA's stage barrier, which the leader's lane arms with
+//               both CTAs' bytes.  The leader's warp 0 also takes tiles from
+//               the counter and posts them in a small tile queue in both
+//               CTAs' shared memory for every other role, one tile ahead of
+//               its own loads (the atomic's round trip overlaps the current
+//               tile's loads).
 //   warp 1      TMEM owner (paired allocation); in the leader (even) CTA one
 //               lane issues the MMAs and commits to both CTAs' barriers.
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 16 tokens into shared memory,
-//               SwiGLU / bf16 conversion, token-major vector stores.  Two
-//               256-column TMEM accumulators let the epilogue of one tile
-//               overlap the main loop of the next.
+//   warps 2..   epilogue (up: 8 warps, down: 4): tcgen05.ld 32 lanes x 16
+//               tokens into shared memory, SwiGLU / bf16 conversion,
+//               token-major vector stores.  Two 256-column TMEM accumulators
+//               let the epilogue of one tile overlap the main loop of the next.
+//   then        the token-operand producer, and for up the W3-half producer:
+//               they follow the tile queue and fill their part of each stage.
+//               A thread that issues a TMA tile load stalls for roughly as
+//               long as the unit takes to accept its bytes, so one thread
+//               issuing all of a stage's loads left the tensor pipe waiting;
+//               spreading a stage's loads over warps measured the up
+//               projection 13-15% and the V3 step 7% faster.
 // Every wait is bounded (common.cuh); on a timeout the CTA raises its abort
 // flag, drains what it issued, frees TMEM and exits (the peer then times out
 // on its next wait and does the same).
@@ -85,8 +94,11 @@ template <bool UP>
 __host__ __device__ constexpr int n_epi_warps() { return UP ? 8 : 4; }
 template <bool UP>
 __host__ __device__ constexpr int n_xbuf_per_group() { return UP ? 1 : 2; }
+// producer warps after the epilogue warps: the token operand (both), the W3 half (up)
 template <bool UP>
-__host__ __device__ constexpr int n_threads() { return 64 + 32 * n_epi_warps<UP>(); }
+__host__ __device__ constexpr int n_extra_producers() { return UP ? 2 : 1; }
+template <bool UP>
+__host__ __device__ constexpr int n_threads() { return 32 * (2 + n_epi_warps<UP>() + n_extra_producers<UP>()); }
 constexpr int XS = 132;                 // row stride (floats) of the epilogue exchange buffer
 constexpr int XBUF_BYTES = 16 * XS * 4; // 16 tokens x 128 lanes (+pad), fp32
 // L2 policy of the two operands' loads.  Marking the weights evict-first
@@ -96,9 +108,12 @@ constexpr int XBUF_BYTES = 16 * XS * 4; // 16 tokens x 128 lanes (+pad), fp32
 constexpr uint64_t W_HINT = kEvictNormal;
 constexpr uint64_t X_HINT = kEvictNormal;
 constexpr int TQ = 8;                   // tile queue slots
-// readers of a queue slot: leader MMA issuer + its epilogue warps, peer producer + its epilogue warps
+// readers of a queue slot, in each CTA: the epilogue warps, the extra producers, and
+// the MMA issuer (leader) or the weight producer (peer)
 template <bool UP>
-__host__ __device__ constexpr uint32_t tq_readers() { return 2u * (1u + (uint32_t)n_epi_warps<UP>()); }
+__host__ __device__ constexpr uint32_t tq_readers() {
+    return 2u * (1u + (uint32_t)n_epi_warps<UP>() + (uint32_t)n_extra_producers<UP>());
+}
 
 // Tile counters: one {next, done} pair per launch slot.  A launch takes the
 // next slot round-robin on the host; the last cluster to finish resets its
@@ -272,6 +287,62 @@ __device__ __forceinline__ bool tq_take(Ctl* ctl, int j, uint32_t ph, uint32_t l
     return true;
 }
 
+// After an abort, wait (bounded) for TMA loads this thread issued to land
+// before the CTA releases its shared memory.
+__device__ __forceinline__ void settle_inflight_loads() {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+}
+
+// A producer warp other than warp 0: follows the tile queue; per tile,
+// begin(tc) returns the tile's K steps; per K step it waits until the stage
+// is free and load(kb, stage, leader_full_bar) issues this warp's part.  The
+// stage barrier may see these bytes land before warp 0 arms it: its
+// transaction count then stays negative until the arming, and the phase
+// cannot complete before the arrive that comes with it.
+template <typename Begin, typename Load>
+__device__ __forceinline__ void follow_tiles(Ctl* ctl, const Tables* tb, int G, uint32_t leader_tq_empty, int* status,
+                                             uint8_t* ring, int lane, Begin&& begin, Load&& load) {
+    const uint32_t leader_full = mapa_shared(smem_u32(&ctl->full[0]), 0);
+    int stage = 0, j = 0;
+    uint32_t phase = 0, tq_ph = 0;
+    bool ok = true, issued_any = false;
+    for (;;) {
+        int tile = -1, got = 1;
+        if (lane == 0) got = tq_take(ctl, j, tq_ph, leader_tq_empty, &tile, status) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        tile = __shfl_sync(0xffffffffu, tile, 0);
+        if (!got) {
+            ok = false;
+            break;
+        }
+        if (tile < 0) break;
+        if (++j == TQ) {
+            j = 0;
+            tq_ph ^= 1u;
+        }
+        const int k_blocks = begin(tile_coords(tb, G, tile));
+        for (int kb = 0; kb < k_blocks; ++kb) {
+            int free_ = 1;
+            if (lane == 0) free_ = mbar_wait(&ctl->empty[stage], phase ^ 1u, &ctl->abort, status) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, free_, 0)) {
+                ok = false;
+                break;
+            }
+            load(kb, ring + stage * STAGE_BYTES, leader_full + 8u * (uint32_t)stage);
+            issued_any = true;
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (!ok) break;
+    }
+    if (!ok && issued_any && lane == 0) settle_inflight_loads();
+    __syncwarp();
+}
+
 template <bool UP, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
     tc_grouped_gemm_kernel(const __grid_constant__ SetMaps ma, const __grid_constant__ SetMaps mb,
@@ -351,23 +422,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
     const int total = tb->prefix[G];
     const uint32_t leader_tq_empty = mapa_shared(smem_u32(&ctl->tq_empty[0]), 0);
 
+    constexpr int kTokWarp = 2 + NEPI;  // token-operand producer
+    constexpr int kW3Warp = 3 + NEPI;   // up: W3-half producer
+    const bool gather = UP && p.gather != nullptr;  // routed set only
+
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer (both CTAs)
-        // Lane 0 waits for free stages and loads the weights; with a gather
-        // index every lane also fetches four token rows (tile::gather4), so
-        // the token operand is read straight from x in expert order.
-        const bool gather = UP && p.gather != nullptr;  // routed set only
+        // ------------------------------------------------ weight producer (both CTAs)
         if (lane == 0) {
-            if (p.G0 > 0) {
-                tma_prefetch_desc(&ma.w0);
-                if (UP) tma_prefetch_desc(&ma.w1);
-                tma_prefetch_desc(gather ? &tmXg : &ma.x[NXBOX - 1]);
-            }
-            if (p.has_shared) {
-                tma_prefetch_desc(&mb.w0);
-                if (UP) tma_prefetch_desc(&mb.w1);
-                tma_prefetch_desc(&mb.x[NXBOX - 1]);
-            }
+            if (p.G0 > 0) tma_prefetch_desc(&ma.w0);
+            if (p.has_shared) tma_prefetch_desc(&mb.w0);
         }
         const uint32_t leader_full = mapa_shared(smem_u32(&ctl->full[0]), 0);
         const uint32_t peer_tq = mapa_shared(smem_u32(&ctl->tq[0]), 1);
@@ -427,17 +490,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
             int tstart, ntok;
             token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
             const int half = ((ntok + 15) & ~15) >> 1;
-            const int row0 = tb->rowstart[tc.g] + tstart;  // first row of the tile
-            const int tok0 = row0 + (int)rank * half;      // first row of this CTA's half
-            int src[4] = {0, 0, 0, 0};
-            if (gat) {  // this lane's four rows; rows past the tile's tokens repeat its first row
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int jr = (int)rank * half + 4 * lane + j;
-                    src[j] = p.gather[row0 + (jr < ntok ? jr : 0)] / p.gather_div;
-                }
-            }
-            const int xrows = gat ? half : (half + 15) & ~15;  // token rows this CTA loads per K step
+            const int xrows = gat ? half : (half + 15) & ~15;  // token rows a CTA loads per K step
             const uint32_t tx = 2u * ((uint32_t)A_BYTES + (uint32_t)xrows * 128u);  // both CTAs' bytes
             for (int kb = 0; kb < sp.k_blocks; ++kb) {
                 int got = 1;
@@ -449,24 +502,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                 }
                 const uint32_t fb = leader_full + 8u * (uint32_t)stage;
                 uint8_t* sa = ring + stage * STAGE_BYTES;
-                uint8_t* sb = sa + A_BYTES;
                 if (lane == 0) {
                     if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], tx);
                     if (UP) {
                         const int wrow = wg * sp.w_rows + tc.ft * 128 + (int)rank * 64;
                         tma_load_2d_pair(sa, &M.w0, fb, kb * BKE, wrow, W_HINT);
-                        tma_load_2d_pair(sa + A_BYTES / 2, &M.w1, fb, kb * BKE, wrow, W_HINT);
                     } else {
                         const int kk = kb * BKE;
                         const int seg = kk / sp.kseg;
                         tma_load_3d_pair(sa, &M.w0, fb, kk - seg * sp.kseg, tc.ft * 256 + (int)rank * 128,
                                          wg * sp.nseg + seg, W_HINT);
                     }
-                    if (!gat) tma_load_2d_pair(sb, &M.x[xrows / 16 - 1], fb, kb * BKE, tok0, X_HINT);
                 }
-                if (gat && 4 * lane < half)
-                    tma_gather4_pair(sb + 4 * lane * 128, &tmXg, fb, kb * BKE, src[0], src[1], src[2], src[3],
-                                     X_HINT);
                 issued_any = true;
                 if (++stage == STAGES) {
                     stage = 0;
@@ -483,12 +530,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                 atomicExch(&sched[1], 0u);
             }
         }
-        if (!ok && issued_any && lane == 0) {  // let copies already in flight land before the CTA exits
-            const uint64_t t0 = globaltimer_ns();
-            while (globaltimer_ns() - t0 < 200000ull) {
-            }
-        }
+        if (!ok && issued_any && lane == 0) settle_inflight_loads();
         __syncwarp();
+    } else if (warp == kTokWarp) {
+        // ------------------------------------------------ token-operand producer (both CTAs)
+        // One lane loads this CTA's half of the tile's token rows per K step;
+        // with a gather index every lane fetches four token rows
+        // (tile::gather4), so the operand is read straight from x in expert order.
+        if (lane == 0) {
+            if (p.G0 > 0) tma_prefetch_desc(gather ? &tmXg : &ma.x[NXBOX - 1]);
+            if (p.has_shared) tma_prefetch_desc(&mb.x[NXBOX - 1]);
+        }
+        const CUtensorMap* xmap = nullptr;
+        bool gat = false;
+        int half = 0, tok0 = 0;
+        int src[4] = {0, 0, 0, 0};
+        follow_tiles(
+            ctl, tb, G, leader_tq_empty, p.status, ring, lane,
+            [&](const TileCoord& tc) {
+                const int si = tc.g >= p.G0 ? 1 : 0;
+                gat = gather && si == 0;
+                int tstart, ntok;
+                token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
+                half = ((ntok + 15) & ~15) >> 1;
+                const int row0 = tb->rowstart[tc.g] + tstart;  // first row of the tile
+                tok0 = row0 + (int)rank * half;                // first row of this CTA's half
+                xmap = &(si ? mb : ma).x[((half + 15) & ~15) / 16 - 1];
+                if (gat) {  // this lane's four rows; rows past the tile's tokens repeat its first row
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int jr = (int)rank * half + 4 * lane + i;
+                        src[i] = p.gather[row0 + (jr < ntok ? jr : 0)] / p.gather_div;
+                    }
+                }
+                return p.set[si].k_blocks;
+            },
+            [&](int kb, uint8_t* stage, uint32_t fb) {
+                uint8_t* sb = stage + A_BYTES;
+                if (!gat && lane == 0) tma_load_2d_pair(sb, xmap, fb, kb * BKE, tok0, X_HINT);
+                if (gat && 4 * lane < half)
+                    tma_gather4_pair(sb + 4 * lane * 128, &tmXg, fb, kb * BKE, src[0], src[1], src[2], src[3],
+                                     X_HINT);
+            });
+    } else if (UP && warp == kW3Warp) {
+        // ------------------------------------------------ W3-half producer (up, both CTAs)
+        if (lane == 0) {
+            if (p.G0 > 0) tma_prefetch_desc(&ma.w1);
+            if (p.has_shared) tma_prefetch_desc(&mb.w1);
+        }
+        const CUtensorMap* wmap = nullptr;
+        int wrow = 0;
+        follow_tiles(
+            ctl, tb, G, leader_tq_empty, p.status, ring, lane,
+            [&](const TileCoord& tc) {
+                const int si = tc.g >= p.G0 ? 1 : 0;
+                wmap = &(si ? mb : ma).w1;
+                wrow = (si ? 0 : tc.g) * p.set[si].w_rows + tc.ft * 128 + (int)rank * 64;
+                return p.set[si].k_blocks;
+            },
+            [&](int kb, uint8_t* stage, uint32_t fb) {
+                if (lane == 0) tma_load_2d_pair(stage + A_BYTES / 2, wmap, fb, kb * BKE, wrow, W_HINT);
+            });
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (leader CTA only)
         if (rank == 0 && elect_one()) {
