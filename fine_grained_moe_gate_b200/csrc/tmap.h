@@ -48,19 +48,4 @@ inline bool make_tmap_2d(CUtensorMap* m, const void* base, unsigned long long co
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// rank-3 map over [n2][rows][cols] (contiguous, elem_bytes-wide elements);
-// box box_cols x box_rows x 1.
-inline bool make_tmap_3d(CUtensorMap* m, const void* base, unsigned long long cols, unsigned long long rows,
-                         unsigned long long n2, unsigned box_cols, unsigned box_rows, unsigned elem_bytes = 2) {
-    auto enc = tmap_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[3] = {cols, rows, n2};
-    cuuint64_t strides[2] = {cols * elem_bytes, cols * rows * elem_bytes};
-    cuuint32_t box[3] = {box_cols, box_rows, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    return enc(m, tmap_type(elem_bytes), 3, const_cast<void*>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace moe
