@@ -40,9 +40,12 @@ struct Ctl {
 constexpr int SCORE_BYTES = PART_BYTES + BM / 2 * PS * 4;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)(RING_BYTES > SCORE_BYTES ? RING_BYTES : SCORE_BYTES) + sizeof(Ctl);
 
-__device__ __forceinline__ float ld_cluster_f32(uint32_t cluster_addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t cluster_addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(cluster_addr)
+                 : "memory");
     return v;
 }
 
@@ -210,18 +213,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int u = tid - 64;             // 0..127
         constexpr int TPC = BM / C;         // tokens this CTA finishes
         const int tl0 = crank * TPC;        // its first token within the tile
-        // scores s = sigmoid(sum of the C partials in CTA order), for this CTA's tokens
+        // scores s = sigmoid(sum of the C partials in CTA order), for this CTA's
+        // tokens: 128 / TPC threads per token row, four experts per DSMEM load
+        // (rows are 16-byte aligned; columns up to n_pad >= E hold MMA results)
         float* sc = red;
-        for (int it = u; it < TPC * E; it += 128) {
-            const int rl = it / E, e = it - rl * E;
+        {
+            constexpr int TPR = 128 / TPC;
+            const int rl = u / TPR, q4 = u - rl * TPR;
             const int r = tl0 + rl;
-            const uint32_t a = smem_u32(part + r * PS + e);
-            float z = ld_cluster_f32(mapa_shared(a, 0));
+            const bool keep_aff = aff && t0 + r < T;
+#pragma unroll 4
+            for (int e = 4 * q4; e < E; e += 4 * TPR) {
+                const uint32_t a = smem_u32(part + r * PS + e);
+                float4 z = ld_cluster_f32x4(mapa_shared(a, 0));
 #pragma unroll
-            for (int c = 1; c < C; ++c) z = __fadd_rn(z, ld_cluster_f32(mapa_shared(a, c)));
-            const float s = sigmoid_f32(z);
-            sc[rl * PS + e] = s;
-            if (aff && t0 + r < T) aff[(size_t)(t0 + r) * E + e] = s;
+                for (int c = 1; c < C; ++c) {
+                    const float4 o = ld_cluster_f32x4(mapa_shared(a, c));
+                    z.x = __fadd_rn(z.x, o.x);
+                    z.y = __fadd_rn(z.y, o.y);
+                    z.z = __fadd_rn(z.z, o.z);
+                    z.w = __fadd_rn(z.w, o.w);
+                }
+                const float zs[4] = {z.x, z.y, z.z, z.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (e + i < E) {
+                        const float s = sigmoid_f32(zs[i]);
+                        sc[rl * PS + e + i] = s;
+                        if (keep_aff) aff[(size_t)(t0 + r) * E + e + i] = s;
+                    }
+                }
+            }
         }
         named_bar_sync(1, 128);
         // top-k: C threads per token, thread `sub` pushes experts sub, sub + C, ...
