@@ -35,6 +35,7 @@ EXPORTS = (
     "moe_kernel_launch_count", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
     "moe_quantize_fp8", "moe_ffn_up_fp8", "moe_ffn_down_fp8", "moe_layer_forward_fp8",
     "moe_ep_plan_size", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_return",
+    "moe_layer_backward", "moe_backward_workspace_size",
 )
 
 MOE_ROUTED, MOE_SHARED = 0, 1
@@ -110,6 +111,8 @@ def lib() -> ctypes.CDLL:
             "moe_ep_dispatch": [P, P, P, ctypes.c_int32, ctypes.c_int32, S, P, P],
             "moe_ep_return": [P, P, ctypes.c_int32, ctypes.c_int32, S, P, P],
             "moe_selftest_bounded_wait": [ctypes.c_uint32, P],
+            "moe_layer_backward": [P, P, P, P, P, P, P, P, S, P, P, P, P, P, F, ctypes.c_int32, P, P, P, P, P, P, P,
+                                   P, P, P, sz, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -119,6 +122,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.argtypes = [S]
             fn.restype = sz
+        L.moe_backward_workspace_size.argtypes = [S, ctypes.c_int32]
+        L.moe_backward_workspace_size.restype = sz
         L.moe_ep_plan_size.argtypes = [ctypes.c_int32, S]
         L.moe_ep_plan_size.restype = sz
         L.moe_kernel_launch_count.argtypes = []
@@ -224,6 +229,19 @@ def moe_layer_forward(x, w_gate, bias, w1, w3, w2, ws1, ws3, ws2, shape, y, topk
 
 def moe_workspace_size(shape) -> int:
     return lib().moe_workspace_size(shape)
+
+
+def moe_layer_backward(x, w_gate, w1, w3, w2, ws1, ws3, ws2, shape, topk_idx, topk_w, counts, affinity, dy, alpha,
+                       seq_len, dx, dw_gate, dw1, dw3, dw2, dws1, dws3, dws2, balance_loss, workspace, stream=None):
+    _check(lib().moe_layer_backward(_p(x), _p(w_gate), _p(w1), _p(w3), _p(w2), _p(ws1), _p(ws3), _p(ws2), shape,
+                                    _p(topk_idx), _p(topk_w), _p(counts), _p(affinity), _p(dy), float(alpha),
+                                    int(seq_len), _p(dx), _p(dw_gate), _p(dw1), _p(dw3), _p(dw2), _p(dws1), _p(dws3),
+                                    _p(dws2), _p(balance_loss), _p(workspace), _nbytes(workspace), _stream(stream)),
+           "moe_layer_backward")
+
+
+def moe_backward_workspace_size(shape, seq_len: int = 0) -> int:
+    return lib().moe_backward_workspace_size(shape, int(seq_len))
 
 
 def moe_permute_workspace_size(shape) -> int:

@@ -1,0 +1,583 @@
+// Backward of the MoE layer forward: gradients of <dy, y> (+ the sequence-wise
+// balance loss) with respect to x, the gate weights and the routed and shared
+// expert weights, for the selection the forward made.
+//
+// What is differentiated (page title, section):
+//   "DeepSeek V3 From Scratch", "In code" (route): s = sigmoid(x W_g^T); the
+//     top-k is chosen on s + b; w_j = s_{idx_j} / sum_j' s_{idx_j'} from the
+//     unbiased scores.  The bias and the choice carry no gradient.
+//   "Scaling Efficiency: A Deep Dive into the DeepSeek-V3 Architecture",
+//     DeepSeekMoE sketch: y_t = sum_s shared_s(x_t) + sum_j w_j expert_{idx_j}(x_t),
+//     every expert W2 (silu(W1 x) * (W3 x)).
+//   kbwen.com DeepSeek tag page, "A bias term for each expert": a small
+//     complementary sequence-wise balance loss is kept; its formula is not
+//     on the pages -- the DeepSeek-V3 report's is used: per sequence of L
+//     tokens, f_i = E/(kL) #{t : i chosen}, P_i = 1/L sum_t s_ti / sum_j s_tj,
+//     loss = alpha sum_i f_i P_i, averaged over the sequences.
+//
+// Gradients (per routed assignment r = (t, j) of expert e, h recomputed and
+// rounded like the forward's):
+//   dw_tj = <dy_t, o_r>,  o_r = W2_e h_r;   do_r = w_tj dy_t
+//   dW2_e = sum_r do_r h_r^T;   dh_r = W2_e^T do_r
+//   da = dh g sigma(a) (1 + a (1 - sigma(a))),   dg = dh a sigma(a)
+//   dW1_e = sum_r da_r x_t^T,  dW3_e likewise;  dx_t += W1_e^T da_r + W3_e^T dg_r
+//   shared experts the same with weight 1;  router: ds_{t,idx_j} =
+//   (dw_tj - sum_j' dw_tj' w_tj') / sum_j' s_{t,idx_j'} (+ the balance term),
+//   dz = ds s (1 - s),  dx += dz W_g,  dW_g = dz^T x.
+//
+// Every contraction runs through two fp32 SIMT kernels over strided operand
+// views (no transposed copies): a "rows" GEMM (C[r][n] = sum_k A(r,k) B_g(n,k)
+// for the rows r of group g) and a weight-gradient GEMM whose contraction runs
+// over a group's rows (C_g[m][n] = sum_r A(r,m) B(r,n)).  Groups and tiles are
+// resolved on the device from the routing offsets.  fp32 FFMA throughout:
+// the backward is a first, exact-in-fp32 path, not yet on the tensor cores.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 64, BN = 64, BK = 16;
+
+// Element (r, c) of group g: base + g*gs + row(r)*rs + c*cs, where row(r) =
+// gather[r] / gdiv when a gather index is given, else r.
+struct Opnd {
+    const void* p;
+    int bf16;
+    long long rs, cs, gs;
+    const int32_t* gather;
+    int gdiv;
+};
+
+__device__ __forceinline__ float opnd_ld(const Opnd& o, int r, int c, int g) {
+    const long long row = o.gather ? (long long)(o.gather[r] / o.gdiv) : (long long)r;
+    const long long off = (long long)g * o.gs + row * o.rs + (long long)c * o.cs;
+    if (o.bf16) return __uint_as_float((uint32_t)static_cast<const uint16_t*>(o.p)[off] << 16);
+    return static_cast<const float*>(o.p)[off];
+}
+
+// Rows r of group g: [offsets[g], offsets[g+1]) or, without offsets, [0, M).
+// A corrupt range is skipped and reported.
+__device__ __forceinline__ void group_rows(const int32_t* offsets, int g, int M, int* status, int& rs, int& re) {
+    if (!offsets) {
+        rs = 0;
+        re = M;
+        return;
+    }
+    rs = offsets[g];
+    re = offsets[g + 1];
+    if (rs < 0 || re < rs || re > M) {
+        report(status, kStDeviceCheck);
+        rs = re = 0;
+    }
+}
+
+struct RowsGemm {
+    Opnd A, B;          // A(r, k) (no group), B(n, k) of group g
+    float* C;           // C[r * c_rs + n]
+    long long c_rs;
+    int M, N, K;
+    const int32_t* offsets;
+    int G;
+    int accumulate;
+    int* status;
+};
+
+// C[r][n] (+)= sum_k A(r, k) B_g(n, k) for every row r of every group g.
+// 64 x 64 output tiles, 256 threads with 4 x 4 outputs each, K in steps of 16
+// through shared memory; tiles of all groups in one grid-stride list.
+__global__ void __launch_bounds__(256) rows_gemm_kernel(RowsGemm p) {
+    __shared__ float As[BK][BM + 4];
+    __shared__ float Bs[BK][BN + 4];
+    __shared__ int prefix[kMaxGroups + 1];
+    __shared__ int gstart[kMaxGroups], grows[kMaxGroups];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int n_tiles = (p.N + BN - 1) / BN;
+    for (int g = tid; g < p.G; g += blockDim.x) {
+        int rs, re;
+        group_rows(p.offsets, g, p.M, p.status, rs, re);
+        gstart[g] = rs;
+        grows[g] = re - rs;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int acc = 0;
+        for (int g = 0; g < p.G; ++g) {
+            prefix[g] = acc;
+            acc += (grows[g] + BM - 1) / BM * n_tiles;
+        }
+        prefix[p.G] = acc;
+    }
+    __syncthreads();
+    const bool a_kfast = p.A.cs == 1, b_kfast = p.B.cs == 1;
+    for (int tile = blockIdx.x; tile < prefix[p.G]; tile += gridDim.x) {
+        int lo = 0, hi = p.G - 1;
+        while (lo < hi) {  // last group whose first tile is <= tile
+            const int mid = (lo + hi + 1) >> 1;
+            if (prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+        }
+        const int g = lo;
+        const int mt = (grows[g] + BM - 1) / BM;
+        const int q = tile - prefix[g];
+        const int m0 = (q % mt) * BM, n0 = (q / mt) * BN;
+        const int row0 = gstart[g] + m0;
+        const int nrows = min(BM, grows[g] - m0);
+        float acc[4][4] = {};
+        for (int k0 = 0; k0 < p.K; k0 += BK) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int e = tid + 256 * i;
+                const int m = a_kfast ? e / BK : e % BM, kk = a_kfast ? e % BK : e / BM;
+                As[kk][m] = (m < nrows && k0 + kk < p.K) ? opnd_ld(p.A, row0 + m, k0 + kk, 0) : 0.0f;
+                const int n = b_kfast ? e / BK : e % BN, kb = b_kfast ? e % BK : e / BN;
+                Bs[kb][n] = (n0 + n < p.N && k0 + kb < p.K) ? opnd_ld(p.B, n0 + n, k0 + kb, g) : 0.0f;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int kk = 0; kk < BK; ++kk) {
+                float a[4], b[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    a[i] = As[kk][ty * 4 + i];
+                    b[i] = Bs[kk][tx * 4 + i];
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+            }
+            __syncthreads();
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int m = ty * 4 + i;
+            if (m >= nrows) continue;
+            float* crow = p.C + (long long)(row0 + m) * p.c_rs;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int n = n0 + tx * 4 + j;
+                if (n < p.N) crow[n] = p.accumulate ? crow[n] + acc[i][j] : acc[i][j];
+            }
+        }
+    }
+}
+
+struct WgradGemm {
+    Opnd A, B;          // A(r, m), B(r, n) over the group's rows r
+    float* C;           // C_g[m][n] at C + g * c_gs + m * c_rs + n
+    long long c_rs, c_gs;
+    int M, N;
+    const int32_t* offsets;
+    int G;
+    int rows;           // rows of the single group without offsets
+    int accumulate;
+    int* status;
+};
+
+// C_g[m][n] (+)= sum over the rows r of group g of A(r, m) B(r, n).  Grid:
+// x = output tiles of one group, y = group.  An empty group writes zeros.
+__global__ void __launch_bounds__(256) wgrad_gemm_kernel(WgradGemm p) {
+    __shared__ float As[BK][BM + 4];
+    __shared__ float Bs[BK][BN + 4];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int g = blockIdx.y;
+    const int m_tiles = (p.M + BM - 1) / BM;
+    const int m0 = (blockIdx.x % m_tiles) * BM, n0 = (blockIdx.x / m_tiles) * BN;
+    int rs, re;
+    group_rows(p.offsets, g, p.rows, p.status, rs, re);
+    const bool a_mfast = p.A.cs == 1, b_nfast = p.B.cs == 1;
+    float acc[4][4] = {};
+    for (int r0 = rs; r0 < re; r0 += BK) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + 256 * i;
+            const int m = a_mfast ? e % BM : e / BK, kk = a_mfast ? e / BM : e % BK;
+            As[kk][m] = (r0 + kk < re && m0 + m < p.M) ? opnd_ld(p.A, r0 + kk, m0 + m, 0) : 0.0f;
+            const int n = b_nfast ? e % BN : e / BK, kb = b_nfast ? e / BN : e % BK;
+            Bs[kb][n] = (r0 + kb < re && n0 + n < p.N) ? opnd_ld(p.B, r0 + kb, n0 + n, 0) : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < BK; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                a[i] = As[kk][ty * 4 + i];
+                b[i] = Bs[kk][tx * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+    float* cg = p.C + (long long)g * p.c_gs;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int m = m0 + ty * 4 + i;
+        if (m >= p.M) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + tx * 4 + j;
+            if (n < p.N) {
+                float* c = cg + (long long)m * p.c_rs + n;
+                *c = p.accumulate ? *c + acc[i][j] : acc[i][j];
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ float sigmoid_acc(float a) { return 1.0f / (1.0f + expf(-a)); }
+
+// h = silu(a) * g, rounded to bf16 when the layer is bf16 (the forward's rounding point).
+__global__ void swiglu_fwd_kernel(const float* __restrict__ a, const float* __restrict__ g, float* __restrict__ h,
+                                  long long n, int bf16) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const float av = a[i];
+        float v = av * sigmoid_acc(av) * g[i];
+        if (bf16) v = __bfloat162float(__float2bfloat16_rn(v));
+        h[i] = v;
+    }
+}
+
+// In place: dh_da <- dh g s (1 + a (1 - s)),  g_dg <- dh a s,  s = sigmoid(a).
+__global__ void swiglu_bwd_kernel(const float* __restrict__ a, float* __restrict__ g_dg, float* __restrict__ dh_da,
+                                  long long n) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const float av = a[i], gv = g_dg[i], dh = dh_da[i];
+        const float s = sigmoid_acc(av);
+        dh_da[i] = dh * gv * s * (1.0f + av * (1.0f - s));
+        g_dg[i] = dh * av * s;
+    }
+}
+
+// Fixed-order block sum (warp shuffles, then warp 0 over the warp partials).
+__device__ float block_sum(float v, float* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[w] = v;
+    __syncthreads();
+    if (w == 0) {
+        v = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[0] = v;
+    }
+    __syncthreads();
+    const float r = red[0];
+    __syncthreads();
+    return r;
+}
+
+// One block per assignment q = t*k + j, row r = inv[q] of the permuted
+// buffers: dw[q] = <dy_t, o_r>, then o_r <- do_r = w[q] dy_t (in place).
+__global__ void __launch_bounds__(256) combine_bwd_kernel(const float* __restrict__ dy, const float* __restrict__ w,
+                                                          const int32_t* __restrict__ inv, float* o_do,
+                                                          float* __restrict__ dw, int d, int k, int rows,
+                                                          int* status) {
+    __shared__ float red[32];
+    const int q = blockIdx.x, t = q / k;
+    const int r = inv[q];
+    if (r < 0 || r >= rows) {
+        if (threadIdx.x == 0) report(status, kStDeviceCheck);
+        return;
+    }
+    const float* dyt = dy + (long long)t * d;
+    float* orow = o_do + (long long)r * d;
+    float part = 0.0f;
+    for (int c = threadIdx.x; c < d; c += blockDim.x) part = fmaf(dyt[c], orow[c], part);
+    const float tot = block_sum(part, red);  // every read of the row is done past this point
+    if (threadIdx.x == 0) dw[q] = tot;
+    const float wq = w[q];
+    for (int c = threadIdx.x; c < d; c += blockDim.x) orow[c] = wq * dyt[c];
+}
+
+// dx[t] = sum_j dxp[inv[t*k + j]] (overwrite), one block per token.
+__global__ void unpermute_sum_kernel(const float* __restrict__ dxp, const int32_t* __restrict__ inv, float* dx, int d,
+                                     int k, int rows, int* status) {
+    const int t = blockIdx.x;
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+        float v = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int r = inv[(long long)t * k + j];
+            if (r < 0 || r >= rows) {
+                report(status, kStDeviceCheck);
+                continue;
+            }
+            v += dxp[(long long)r * d + c];
+        }
+        dx[(long long)t * d + c] = v;
+    }
+}
+
+// Per-sequence choice counts: cnt[b][i] = #{(t in sequence b, j) : idx[t][j] = i}.
+__global__ void seq_counts_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int L, int32_t* cnt,
+                                  int* status) {
+    for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < (long long)T * k;
+         q += (long long)gridDim.x * blockDim.x) {
+        const int e = idx[q];
+        if (e < 0 || e >= E) {
+            report(status, kStDeviceCheck);
+            continue;
+        }
+        atomicAdd(&cnt[(q / k) / L * E + e], 1);
+    }
+}
+
+// One warp per token: ds over all experts (the renormalised gate's part on
+// the chosen ones, plus the balance term), dz = ds s (1 - s); tot[t] = sum_i s_ti.
+__global__ void router_bwd_kernel(const float* __restrict__ s, const int32_t* __restrict__ idx,
+                                  const float* __restrict__ dw, const int32_t* __restrict__ cnt, float alpha, int L,
+                                  int nb, int T, int E, int k, float* __restrict__ dz, float* __restrict__ tot,
+                                  int* status) {
+    const int warps = blockDim.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * warps + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float* st = s + (long long)t * E;
+    const int32_t* it = idx + (long long)t * k;
+    const float* dwt = dw + (long long)t * k;
+    bool bad = false;
+    for (int j = 0; j < k; ++j) bad |= it[j] < 0 || it[j] >= E;
+    if (bad) {  // corrupt selection: report, no gradient for this token
+        if (lane == 0) report(status, kStDeviceCheck);
+        for (int i = lane; i < E; i += 32) dz[(long long)t * E + i] = 0.0f;
+        if (lane == 0 && tot) tot[t] = 1.0f;
+        return;
+    }
+    float ssel = 0.0f;
+    for (int j = 0; j < k; ++j) ssel += st[it[j]];
+    float dot = 0.0f;  // sum_j dw_j w_j with w_j = s_{idx_j} / ssel
+    for (int j = 0; j < k; ++j) dot += dwt[j] * (st[it[j]] / ssel);
+    float sum_s = 0.0f, sum_fs = 0.0f;
+    const float fscale = (float)E / ((float)k * (float)L);
+    const int32_t* cb = cnt ? cnt + (long long)(t / L) * E : nullptr;
+    if (alpha > 0.0f) {
+        for (int i = lane; i < E; i += 32) {
+            sum_s += st[i];
+            sum_fs += fscale * (float)cb[i] * st[i];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            sum_s += __shfl_xor_sync(0xffffffffu, sum_s, o);
+            sum_fs += __shfl_xor_sync(0xffffffffu, sum_fs, o);
+        }
+        if (lane == 0) tot[t] = sum_s;
+    }
+    for (int i = lane; i < E; i += 32) {
+        float ds = 0.0f;
+        for (int j = 0; j < k; ++j)
+            if (it[j] == i) ds += (dwt[j] - dot) / ssel;
+        if (alpha > 0.0f) ds += alpha / ((float)nb * (float)L) * (fscale * (float)cb[i] - sum_fs / sum_s) / sum_s;
+        const float sv = st[i];
+        dz[(long long)t * E + i] = ds * sv * (1.0f - sv);
+    }
+}
+
+// One block per sequence b: part[b] = alpha * sum_i f_bi P_bi.
+__global__ void balance_part_kernel(const float* __restrict__ s, const float* __restrict__ tot,
+                                    const int32_t* __restrict__ cnt, float alpha, int L, int E, int k,
+                                    float* __restrict__ part) {
+    __shared__ float red[32];
+    const int b = blockIdx.x;
+    const float fscale = (float)E / ((float)k * (float)L);
+    float v = 0.0f;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        float P = 0.0f;
+        for (int t = b * L; t < (b + 1) * L; ++t) P += s[(long long)t * E + i] / tot[t];
+        v += fscale * (float)cnt[(long long)b * E + i] * (P / (float)L);
+    }
+    v = block_sum(v, red);
+    if (threadIdx.x == 0) part[b] = alpha * v;
+}
+
+__global__ void balance_sum_kernel(const float* __restrict__ part, int nb, float* loss) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    float v = 0.0f;
+    for (int b = 0; b < nb; ++b) v += part[b];
+    *loss = v / (float)nb;
+}
+
+// ------------------------------------------------------------------ launch helpers
+
+Opnd view(const void* p, bool bf16, long long rs, long long cs, long long gs = 0, const int32_t* gather = nullptr,
+          int gdiv = 1) {
+    return Opnd{p, bf16 ? 1 : 0, rs, cs, gs, gather, gdiv};
+}
+
+cudaError_t rows_gemm(const Opnd& A, const Opnd& B, float* C, long long c_rs, int M, int N, int K,
+                      const int32_t* offsets, int G, bool accumulate, int* status, int num_sms, cudaStream_t st) {
+    if (M <= 0 || N <= 0) return cudaSuccess;
+    RowsGemm p{A, B, C, c_rs, M, N, K, offsets, G, accumulate ? 1 : 0, status};
+    // an upper bound of the tile count: every group adds at most one partial m-tile
+    const long long tiles = ((long long)(M + BM - 1) / BM + G) * ((N + BN - 1) / BN);
+    const int grid = (int)(tiles < (long long)num_sms * 8 ? tiles : (long long)num_sms * 8);
+    rows_gemm_kernel<<<grid, 256, 0, st>>>(p);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t wgrad_gemm(const Opnd& A, const Opnd& B, float* C, long long c_rs, long long c_gs, int M, int N,
+                       const int32_t* offsets, int G, int rows, bool accumulate, int* status, cudaStream_t st) {
+    if (M <= 0 || N <= 0 || G <= 0) return cudaSuccess;
+    WgradGemm p{A, B, C, c_rs, c_gs, M, N, offsets, G, rows, accumulate ? 1 : 0, status};
+    const dim3 grid((unsigned)(((M + BM - 1) / BM) * ((N + BN - 1) / BN)), (unsigned)G);
+    wgrad_gemm_kernel<<<grid, 256, 0, st>>>(p);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+int ew_grid(long long n) {
+    const long long b = (n + 255) / 256;
+    return (int)(b < 4096 ? (b > 0 ? b : 1) : 4096);
+}
+
+}  // namespace
+
+size_t backward_scratch_bytes(int T, int d, int E, int k, int I, int S, int Is, int seq_len) {
+    auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
+    const size_t R = (size_t)T * k;
+    const size_t nb = seq_len > 0 ? (size_t)T / seq_len : 0;
+    return al((E + 1) * 4) + 2 * al(R * 4) + al(permute_scratch_bytes(T, E)) + 4 * al(R * I * 4) + al(R * d * 4) +
+           al(R * 4) + 4 * al((size_t)T * S * Is * 4) + al((size_t)T * E * 4) + al((size_t)T * 4) + al(nb * E * 4) +
+           al(nb * 4);
+}
+
+cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sms, cudaStream_t st) {
+    const int T = a.T, d = a.d, E = a.E, k = a.k, I = a.I, S = a.S, Is = a.Is;
+    const bool bf = a.bf16;
+    const int R = T * k;
+    const int nb = a.alpha > 0.0f ? T / a.seq_len : 0;
+    auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
+    char* p = static_cast<char*>(a.workspace);
+    auto take = [&](size_t bytes) {
+        char* q = p;
+        p += al(bytes);
+        return q;
+    };
+    int32_t* offsets = reinterpret_cast<int32_t*>(take((E + 1) * 4));
+    int32_t* perm = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    int32_t* inv = reinterpret_cast<int32_t*>(take((size_t)R * 4));
+    int32_t* pscratch = reinterpret_cast<int32_t*>(take(permute_scratch_bytes(T, E)));
+    float* abuf = reinterpret_cast<float*>(take((size_t)R * I * 4));
+    float* gbuf = reinterpret_cast<float*>(take((size_t)R * I * 4));
+    float* hbuf = reinterpret_cast<float*>(take((size_t)R * I * 4));
+    float* dhbuf = reinterpret_cast<float*>(take((size_t)R * I * 4));
+    float* obuf = reinterpret_cast<float*>(take((size_t)R * d * 4));
+    float* dw = reinterpret_cast<float*>(take((size_t)R * 4));
+    const int SI = S * Is;
+    float* as = reinterpret_cast<float*>(take((size_t)T * SI * 4));
+    float* gs = reinterpret_cast<float*>(take((size_t)T * SI * 4));
+    float* hs = reinterpret_cast<float*>(take((size_t)T * SI * 4));
+    float* dhs = reinterpret_cast<float*>(take((size_t)T * SI * 4));
+    float* dz = reinterpret_cast<float*>(take((size_t)T * E * 4));
+    float* tot = reinterpret_cast<float*>(take((size_t)T * 4));
+    int32_t* cnt = reinterpret_cast<int32_t*>(take((size_t)nb * E * 4));
+    float* part = reinterpret_cast<float*>(take((size_t)nb * 4));
+
+    cudaError_t err;
+#define BWD_TRY(x)                          \
+    do {                                    \
+        if ((err = (x)) != cudaSuccess) return err; \
+    } while (0)
+
+    // routing layout of the forward: offsets, perm_tok, inv_row (no row copy)
+    BWD_TRY(launch_permute(nullptr, a.idx, a.counts, T, d, E, k, bf ? 2 : 4, nullptr, offsets, perm, inv, pscratch,
+                           status, st));
+
+    // ---- routed experts
+    const Opnd xg = view(a.x, bf, d, 1, 0, perm, k);  // x row of permuted row r
+    BWD_TRY(rows_gemm(xg, view(a.w1, bf, d, 1, (long long)I * d), abuf, I, R, I, d, offsets, E, false, status,
+                      a.num_sms, st));
+    BWD_TRY(rows_gemm(xg, view(a.w3, bf, d, 1, (long long)I * d), gbuf, I, R, I, d, offsets, E, false, status,
+                      a.num_sms, st));
+    swiglu_fwd_kernel<<<ew_grid((long long)R * I), 256, 0, st>>>(abuf, gbuf, hbuf, (long long)R * I, bf ? 1 : 0);
+    note_launches(1);
+    // o = h W2_e^T
+    BWD_TRY(rows_gemm(view(hbuf, false, I, 1), view(a.w2, bf, I, 1, (long long)d * I), obuf, d, R, d, I, offsets, E,
+                      false, status, a.num_sms, st));
+    if (R > 0) {
+        combine_bwd_kernel<<<R, 256, 0, st>>>(a.dy, a.w, inv, obuf, dw, d, k, R, status);
+        note_launches(1);
+    }
+    // dW2_e[c][i] = sum_r do[r][c] h[r][i]
+    BWD_TRY(wgrad_gemm(view(obuf, false, d, 1), view(hbuf, false, I, 1), a.dw2, I, (long long)d * I, d, I, offsets, E,
+                       R, false, status, st));
+    // dh[r][i] = sum_c do[r][c] W2_e[c][i]
+    BWD_TRY(rows_gemm(view(obuf, false, d, 1), view(a.w2, bf, 1, I, (long long)d * I), dhbuf, I, R, I, d, offsets, E,
+                      false, status, a.num_sms, st));
+    swiglu_bwd_kernel<<<ew_grid((long long)R * I), 256, 0, st>>>(abuf, gbuf, dhbuf, (long long)R * I);
+    note_launches(1);
+    // dW1_e = da^T x, dW3_e = dg^T x
+    BWD_TRY(wgrad_gemm(view(dhbuf, false, I, 1), xg, a.dw1, d, (long long)I * d, I, d, offsets, E, R, false, status,
+                       st));
+    BWD_TRY(wgrad_gemm(view(gbuf, false, I, 1), xg, a.dw3, d, (long long)I * d, I, d, offsets, E, R, false, status,
+                       st));
+    // dx_perm = da W1_e + dg W3_e  (into the do buffer, no longer needed)
+    BWD_TRY(rows_gemm(view(dhbuf, false, I, 1), view(a.w1, bf, 1, d, (long long)I * d), obuf, d, R, d, I, offsets, E,
+                      false, status, a.num_sms, st));
+    BWD_TRY(rows_gemm(view(gbuf, false, I, 1), view(a.w3, bf, 1, d, (long long)I * d), obuf, d, R, d, I, offsets, E,
+                      true, status, a.num_sms, st));
+    if (T > 0) {
+        unpermute_sum_kernel<<<T, 256, 0, st>>>(obuf, inv, a.dx, d, k, R, status);
+        note_launches(1);
+    }
+
+    // ---- shared experts: one group of T rows, the S blocks stacked along the features
+    if (S > 0) {
+        const Opnd x = view(a.x, bf, d, 1);
+        BWD_TRY(rows_gemm(x, view(a.ws1, bf, d, 1), as, SI, T, SI, d, nullptr, 1, false, status, a.num_sms, st));
+        BWD_TRY(rows_gemm(x, view(a.ws3, bf, d, 1), gs, SI, T, SI, d, nullptr, 1, false, status, a.num_sms, st));
+        swiglu_fwd_kernel<<<ew_grid((long long)T * SI), 256, 0, st>>>(as, gs, hs, (long long)T * SI, bf ? 1 : 0);
+        note_launches(1);
+        const Opnd dyv = view(a.dy, false, d, 1);
+        const size_t eb = bf ? 2 : 4;
+        for (int s = 0; s < S; ++s) {
+            const char* w2s = static_cast<const char*>(a.ws2) + eb * (size_t)s * d * Is;
+            // dWs2_s[c][i] = sum_t dy[t][c] hs[t][s*Is + i]
+            BWD_TRY(wgrad_gemm(dyv, view(hs + (size_t)s * Is, false, SI, 1), a.dws2 + (size_t)s * d * Is, Is, 0, d,
+                               Is, nullptr, 1, T, false, status, st));
+            // dhs[t][s*Is + i] = sum_c dy[t][c] Ws2_s[c][i]
+            BWD_TRY(rows_gemm(dyv, view(w2s, bf, 1, Is), dhs + (size_t)s * Is, SI, T, Is, d, nullptr, 1, false, status,
+                              a.num_sms, st));
+        }
+        swiglu_bwd_kernel<<<ew_grid((long long)T * SI), 256, 0, st>>>(as, gs, dhs, (long long)T * SI);
+        note_launches(1);
+        BWD_TRY(wgrad_gemm(view(dhs, false, SI, 1), x, a.dws1, d, 0, SI, d, nullptr, 1, T, false, status, st));
+        BWD_TRY(wgrad_gemm(view(gs, false, SI, 1), x, a.dws3, d, 0, SI, d, nullptr, 1, T, false, status, st));
+        BWD_TRY(rows_gemm(view(dhs, false, SI, 1), view(a.ws1, bf, 1, d), a.dx, d, T, d, SI, nullptr, 1, true, status,
+                          a.num_sms, st));
+        BWD_TRY(rows_gemm(view(gs, false, SI, 1), view(a.ws3, bf, 1, d), a.dx, d, T, d, SI, nullptr, 1, true, status,
+                          a.num_sms, st));
+    }
+
+    // ---- router and balance loss
+    if (T > 0) {
+        if (nb > 0) {
+            BWD_TRY(cudaMemsetAsync(cnt, 0, (size_t)nb * E * 4, st));
+            seq_counts_kernel<<<ew_grid((long long)R), 256, 0, st>>>(a.idx, T, k, E, a.seq_len, cnt, status);
+            note_launches(1);
+        }
+        router_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(a.s, a.idx, dw, nb > 0 ? cnt : nullptr, a.alpha, a.seq_len,
+                                                        nb, T, E, k, dz, tot, status);
+        note_launches(1);
+        if (nb > 0 && a.loss) {
+            balance_part_kernel<<<nb, 256, 0, st>>>(a.s, tot, cnt, a.alpha, a.seq_len, E, k, part);
+            balance_sum_kernel<<<1, 32, 0, st>>>(part, nb, a.loss);
+            note_launches(2);
+        }
+        // dx += dz W_g;  dW_g = dz^T x
+        BWD_TRY(rows_gemm(view(dz, false, E, 1), view(a.w_gate, bf, 1, d), a.dx, d, T, d, E, nullptr, 1, true, status,
+                          a.num_sms, st));
+    }
+    BWD_TRY(wgrad_gemm(view(dz, false, E, 1), view(a.x, bf, d, 1), a.dw_gate, d, 0, E, d, nullptr, 1, T, false, status,
+                       st));
+    if (a.loss && nb == 0) BWD_TRY(cudaMemsetAsync(a.loss, 0, sizeof(float), st));
+#undef BWD_TRY
+    return cudaSuccess;
+}
+
+}  // namespace moe

@@ -531,6 +531,78 @@ moe_status moe_combine(const void* y_perm, const float* topk_w, const int32_t* i
                : MOE_ERR_CUDA;
 }
 
+size_t moe_backward_workspace_size(moe_shape sh, int32_t seq_len) {
+    if (validate_dense_weights(sh) != MOE_OK) return 0;
+    return moe::backward_scratch_bytes(sh.T, sh.d, sh.E, sh.k, sh.I, sh.S, sh.Is, seq_len > 0 ? seq_len : 0);
+}
+
+moe_status moe_layer_backward(const void* x, const void* w_gate, const void* w1, const void* w3, const void* w2,
+                              const void* ws1, const void* ws3, const void* ws2, moe_shape sh, const int32_t* topk_idx,
+                              const float* topk_w, const int32_t* counts, const float* affinity, const float* dy,
+                              float alpha, int32_t seq_len, float* dx, float* dw_gate, float* dw1, float* dw3,
+                              float* dw2, float* dws1, float* dws3, float* dws2, float* balance_loss, void* workspace,
+                              size_t ws_bytes, void* stream) {
+    moe_status v = validate_dense_weights(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(w_gate && w1 && w3 && w2 && counts && dw_gate && dw1 && dw3 && dw2, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (x && topk_idx && topk_w && affinity && dy && dx), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.S == 0 || (ws1 && ws3 && ws2 && dws1 && dws3 && dws2), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(alpha == alpha && alpha >= 0.0f && alpha < 3.0e38f, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(alpha == 0.0f || (seq_len > 0 && sh.T % seq_len == 0), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x) && aligned16(w_gate) && aligned16(w1) && aligned16(w3) && aligned16(w2) &&
+                    aligned16(ws1) && aligned16(ws3) && aligned16(ws2) && aligned16(topk_idx) && aligned16(topk_w) &&
+                    aligned16(counts) && aligned16(affinity) && aligned16(dy) && aligned16(dx) &&
+                    aligned16(dw_gate) && aligned16(dw1) && aligned16(dw3) && aligned16(dw2) && aligned16(dws1) &&
+                    aligned16(dws3) && aligned16(dws2),
+                MOE_ERR_ALIGNMENT);
+    const int32_t L = alpha > 0.0f ? seq_len : 0;
+    const size_t need = moe::backward_scratch_bytes(sh.T, sh.d, sh.E, sh.k, sh.I, sh.S, sh.Is, L);
+    MOE_REQUIRE(workspace && ws_bytes >= need, MOE_ERR_WORKSPACE);
+    MOE_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    moe::BackwardArgs a{};
+    a.x = x;
+    a.w_gate = w_gate;
+    a.w1 = w1;
+    a.w3 = w3;
+    a.w2 = w2;
+    a.ws1 = ws1;
+    a.ws3 = ws3;
+    a.ws2 = ws2;
+    a.T = sh.T;
+    a.d = sh.d;
+    a.E = sh.E;
+    a.k = sh.k;
+    a.I = sh.I;
+    a.S = sh.S;
+    a.Is = sh.Is;
+    a.bf16 = sh.dtype == MOE_BF16;
+    a.idx = topk_idx;
+    a.w = topk_w;
+    a.counts = counts;
+    a.s = affinity;
+    a.dy = dy;
+    a.alpha = alpha;
+    a.seq_len = L;
+    a.dx = dx;
+    a.dw_gate = dw_gate;
+    a.dw1 = dw1;
+    a.dw3 = dw3;
+    a.dw2 = dw2;
+    a.dws1 = dws1;
+    a.dws3 = dws3;
+    a.dws2 = dws2;
+    a.loss = balance_loss;
+    a.workspace = workspace;
+    a.num_sms = sms;
+    return moe::launch_layer_backward(a, status, sms, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
 moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bias, const void* w1, const void* w3,
                              const void* w2, const void* ws1, const void* ws3, const void* ws2, moe_shape sh, void* y,
                              int32_t* topk_idx, float* topk_w, int32_t* counts, void* workspace, size_t ws_bytes,

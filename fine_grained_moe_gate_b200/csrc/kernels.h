@@ -59,6 +59,26 @@ cudaError_t launch_permute(const void* x, const int32_t* idx, const int32_t* cou
                            size_t elem_bytes, void* x_perm, int32_t* offsets, int32_t* perm_tok, int32_t* inv_row,
                            int32_t* scratch, int* status, cudaStream_t st);
 
+// backward.cu: the layer backward (fp32 SIMT contractions).  Pointers as in
+// moe_layer_backward; x and the weights bf16 when bf16, else fp32.
+struct BackwardArgs {
+    const void *x, *w_gate, *w1, *w3, *w2, *ws1, *ws3, *ws2;
+    int T, d, E, k, I, S, Is;
+    bool bf16;
+    const int32_t* idx;
+    const float* w;
+    const int32_t* counts;
+    const float* s;
+    const float* dy;
+    float alpha;
+    int seq_len;
+    float *dx, *dw_gate, *dw1, *dw3, *dw2, *dws1, *dws3, *dws2, *loss;
+    void* workspace;
+    int num_sms;
+};
+size_t backward_scratch_bytes(int T, int d, int E, int k, int I, int S, int Is, int seq_len);
+cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sms, cudaStream_t st);
+
 // gemm_simt.cu
 cudaError_t launch_simt_gemm(const GemmArgs& p, bool bf16, bool swiglu, int num_sms, cudaStream_t st);
 

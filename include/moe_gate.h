@@ -250,6 +250,40 @@ MOE_API moe_status moe_layer_forward(const void* x, const void* w_gate, const fl
 MOE_API size_t moe_workspace_size(moe_shape sh);  /* moe_layer_forward, or moe_layer_forward_fp8 for MOE_FP8_E4M3 */
 
 /* ---------------------------------------------------------------------------
+ * moe_layer_backward -- gradients of the layer forward for the selection the
+ * forward made  [P1 "In code", route(): the weights renormalised over the
+ * chosen unbiased scores; P2 DeepSeekMoE sketch: shared + weighted routed
+ * SwiGLU experts; P3 "A bias term for each expert": the bias enters only the
+ * choice, so it and the choice carry no gradient, and a small complementary
+ * sequence-wise balance loss is kept].
+ * The balance loss is not defined on the pages; the DeepSeek-V3 report's
+ * form is used: for each sequence of seq_len consecutive tokens,
+ *   f_i = E / (k L) * #{t : i in topk_idx[t]},  P_i = 1/L sum_t s_ti / sum_j s_tj
+ *   L_seq = alpha * sum_i f_i P_i,   balance_loss = mean over the T / L sequences.
+ * Computes, for the objective <dy, y> + balance_loss:
+ *   dx [T][d], dw_gate [E][d], dw1 / dw3 [E][I][d], dw2 [E][d][I],
+ *   dws1 / dws3 [S][Is][d], dws2 [S][d][Is]   -- all fp32, overwritten;
+ *   balance_loss: NULL or one fp32 (0 when alpha == 0).
+ * Inputs: x, w_gate, w1, w3, w2, ws1, ws3, ws2 as in moe_layer_forward
+ * (dtype MOE_F32 or MOE_BF16); topk_idx, topk_w and counts as moe_route
+ * returned them; affinity [T][E] fp32, moe_route's affinity_out; dy [T][d]
+ * fp32.  alpha >= 0; with alpha > 0, seq_len > 0 must divide T.  h is
+ * recomputed and rounded like the forward's (bf16 layers); the output
+ * rounding of y is treated as identity.  fp32 accumulation throughout.
+ * dws1 / dws3 / dws2 and ws1 / ws3 / ws2 may be NULL when S == 0.
+ * workspace: >= moe_backward_workspace_size(sh, seq_len) bytes, 256-byte
+ * aligned.  MOE_FP8_E4M3: MOE_ERR_UNSUPPORTED.  No host synchronisation.
+ * -------------------------------------------------------------------------*/
+MOE_API moe_status moe_layer_backward(const void* x, const void* w_gate, const void* w1, const void* w3,
+                                      const void* w2, const void* ws1, const void* ws3, const void* ws2, moe_shape sh,
+                                      const int32_t* topk_idx, const float* topk_w, const int32_t* counts,
+                                      const float* affinity, const float* dy, float alpha, int32_t seq_len, float* dx,
+                                      float* dw_gate, float* dw1, float* dw3, float* dw2, float* dws1, float* dws3,
+                                      float* dws2, float* balance_loss, void* workspace, size_t ws_bytes,
+                                      void* stream);
+MOE_API size_t moe_backward_workspace_size(moe_shape sh, int32_t seq_len);
+
+/* ---------------------------------------------------------------------------
  * FP8 experts  ["DeepSeek V3 Architecture Deep Dive ...", "FP8 Formats": E4M3
  * for weights and activations; "Per-Tensor/Per-Axis Quantization": a scale
  * per row/channel].  Read as: each weight matrix quantized per output row,

@@ -165,3 +165,32 @@ def test_binding_raises_on_error(L):
     with pytest.raises(moe.MoEError) as ei:
         moe.moe_route(FAKE, None, FAKE, shape(), FAKE, FAKE, FAKE, stream=0)
     assert ei.value.status == INVALID
+
+
+def test_backward_checks(L):
+    """moe_layer_backward validates before touching the device."""
+    c = ctypes.c_void_p
+    F = ctypes.c_float
+    sh = shape()
+    need = moe.moe_backward_workspace_size(sh, 0)
+    assert need > 0 and need % 256 == 0
+    assert moe.moe_backward_workspace_size(sh, 32) > need          # per-sequence buffers
+    assert moe.moe_backward_workspace_size(shape(dtype=moe.MOE_FP8_E4M3, d=256, I=128, Is=128), 0) == 0
+
+    def call(sh=sh, x=FAKE, ws1=FAKE, dy=FAKE, dx=FAKE, alpha=0.0, L_=0, ws=FAKE, nbytes=None):
+        w = [c(x), c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(ws1), c(FAKE), c(FAKE)]
+        return L.moe_layer_backward(*w, sh, c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(dy), F(alpha), L_, c(dx), c(FAKE),
+                                    c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), None, c(ws),
+                                    need if nbytes is None else nbytes, None)
+
+    assert call(sh=shape(dtype=moe.MOE_FP8_E4M3, d=256, I=128, Is=128)) == UNSUPPORTED
+    assert call(dy=None) == INVALID
+    assert call(ws1=None) == INVALID                  # S = 1 needs the shared weights
+    assert call(alpha=-1.0) == INVALID
+    assert call(alpha=float("nan")) == INVALID
+    assert call(alpha=0.01, L_=0) == INVALID          # a balance loss needs a sequence length
+    assert call(alpha=0.01, L_=48) == INVALID         # that divides T = 128
+    assert call(dx=FAKE + 4) == ALIGN
+    assert call(nbytes=need - 256) == WORKSPACE
+    assert call(alpha=0.01, L_=32) == WORKSPACE       # the sequences' buffers are not in `need`
+    assert call(ws=FAKE + 128) == ALIGN
