@@ -67,6 +67,8 @@ def parse_args():
     ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0: per-workload default)")
     ap.add_argument("--T", type=int, default=0, help="override tokens per GPU (profiling slices)")
     ap.add_argument("--E", type=int, default=0, help="override routed experts (profiling slices)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time moe_layer_backward (one GPU) instead of the forward step; prints its own line")
     return ap.parse_args()
 
 
@@ -617,6 +619,94 @@ def run_reference(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# fp32 FFMA peak for the SIMT backward: 148 SMs x 128 fp32 lanes x 2 FLOP per
+# cycle at the 1965 MHz maximum SM clock
+FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_backward(args, world, rank, local):
+    """One step = moe_layer_backward over the workload's batch: gradients of
+    x, the gate and all expert weights plus the sequence-wise balance loss
+    (alpha 1e-4, one sequence per 4096 tokens or the whole batch), for a
+    routing computed once before timing."""
+    import torch
+
+    import fine_grained_moe_gate_b200 as moe
+    from fine_grained_moe_gate_b200.inputs import make_layer, make_tokens
+
+    if world > 1:
+        if rank == 0:
+            print(json.dumps({"metric": "MoE layer backward", "unavailable": "--backward runs on one GPU"}))
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = workload(args)
+    if cfg.dtype == "fp8":
+        raise SystemExit("--backward: E4M3 layers have no backward")
+    sh = moe.shape_of(cfg)
+    p = make_layer(cfg, dev)
+    x = make_tokens(cfg, dev)
+    T, d, E, k, I, S, Is = cfg.T, cfg.d, cfg.E, cfg.k, cfg.I, cfg.S, cfg.Is
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    aff = torch.empty((T, E), dtype=torch.float32, device=dev)
+    moe.moe_route(x, p["w_gate"], p["bias"], sh, idx, w, counts, aff)
+    g = torch.Generator(device=dev).manual_seed(cfg.seed + 101)
+    dy = torch.randn((T, d), generator=g, device=dev)
+    f32 = lambda *shp: torch.empty(shp, dtype=torch.float32, device=dev)
+    out = [f32(T, d), f32(E, d), f32(E, I, d), f32(E, I, d), f32(E, d, I)]
+    sh_out = [f32(S, Is, d), f32(S, Is, d), f32(S, d, Is)] if S else [None, None, None]
+    loss = f32(1)
+    L = 4096 if T % 4096 == 0 else T
+    ws = torch.empty(moe.moe_backward_workspace_size(sh, L), dtype=torch.uint8, device=dev)
+    shw = [p["ws1"], p["ws3"], p["ws2"]] if S else [None, None, None]
+
+    def step():
+        moe.moe_layer_backward(x, p["w_gate"], p["w1"], p["w3"], p["w2"], *shw, sh, idx, w, counts, aff, dy, 1e-4, L,
+                               *out, *sh_out, loss, ws)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, args.steps)
+    clocks = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
+    clocks.start()
+    n0 = moe.moe_kernel_launch_count()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ck = clocks.stop()
+    launches = moe.moe_kernel_launch_count() - n0
+    st = moe.moe_get_last_error()
+    if st != 0:
+        raise SystemExit(f"device status {moe.STATUS.get(st, st)}")
+    ms = a.elapsed_time(b) / steps
+    # FLOPs (2 per multiply-add): per routed row the recomputed a, g and o (6 d I), dh (2 d I), dx_perm
+    # (4 d I) and dW1, dW3, dW2 (6 d I) = 18 d I; per token the shared experts 16 d S Is (no o) and the
+    # router's dx and dW_g 4 d E
+    flop = T * k * 18 * d * I + T * 16 * d * S * Is + T * 4 * d * E
+    tflops = flop / (ms * 1e-3) / 1e12
+    line = {
+        "metric": "MoE layer backward tokens/s (fp32 SIMT contractions)", "value": round(T / (ms * 1e-3), 2),
+        "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) tokens and dy, N(0,std) weights of the stated shape)",
+        "config": {"workload": cfg.name + " backward", "T": T, "d": d, "E": E, "k": k, "I": I, "S": S, "Is": Is,
+                   "balance_alpha": 1e-4, "seq_len": L,
+                   "l2": "weights and activations far larger than L2 at these shapes; no flush"},
+        "roofline": {"bound": "alu", "achieved": round(tflops, 3), "peak": round(FP32_SIMT_PEAK_TFLOPS, 1),
+                     "unit": "TFLOP/s", "frac": round(tflops / FP32_SIMT_PEAK_TFLOPS, 4), "traffic": None,
+                     "peak_kind": "derived: 148 SMs x 128 fp32 FMA lanes x 2 FLOP x 1965 MHz"},
+        "gpu_launches": int(launches), "clocks": ck,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -624,7 +714,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
-    if args.impl == "reference":
+    if args.backward:
+        run_backward(args, world, rank, local)
+    elif args.impl == "reference":
         run_reference(args, world, rank, local)
     else:
         run_ours(args, world, rank, local)
