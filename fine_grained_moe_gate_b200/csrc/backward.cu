@@ -39,7 +39,7 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 64, BN = 64, BK = 16;
+constexpr int TB = 128, TK = 16;  // block tile (both output dimensions), contraction slab
 
 // Element (r, c) of group g: base + g*gs + row(r)*rs + c*cs, where row(r) =
 // gather[r] / gdiv when a gather index is given, else r.
@@ -51,9 +51,11 @@ struct Opnd {
     int gdiv;
 };
 
-__device__ __forceinline__ float opnd_ld(const Opnd& o, int r, int c, int g) {
+__device__ __forceinline__ long long row_off(const Opnd& o, int r) {
     const long long row = o.gather ? (long long)(o.gather[r] / o.gdiv) : (long long)r;
-    const long long off = (long long)g * o.gs + row * o.rs + (long long)c * o.cs;
+    return row * o.rs;
+}
+__device__ __forceinline__ float ld_at(const Opnd& o, long long off) {
     if (o.bf16) return __uint_as_float((uint32_t)static_cast<const uint16_t*>(o.p)[off] << 16);
     return static_cast<const float*>(o.p)[off];
 }
@@ -74,6 +76,24 @@ __device__ __forceinline__ void group_rows(const int32_t* offsets, int g, int M,
     }
 }
 
+// acc[i][j] += As[kk][ty*8 + i] * Bs[kk][tx*8 + j] over one slab (float4 reads).
+__device__ __forceinline__ void slab_fma(const float (*As)[TB + 4], const float (*Bs)[TB + 4], int ty, int tx,
+                                         float (&acc)[8][8]) {
+#pragma unroll
+    for (int kk = 0; kk < TK; ++kk) {
+        const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 8]);
+        const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][ty * 8 + 4]);
+        const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8]);
+        const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8 + 4]);
+        const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+}
+
 struct RowsGemm {
     Opnd A, B;          // A(r, k) (no group), B(n, k) of group g
     float* C;           // C[r * c_rs + n]
@@ -86,15 +106,17 @@ struct RowsGemm {
 };
 
 // C[r][n] (+)= sum_k A(r, k) B_g(n, k) for every row r of every group g.
-// 64 x 64 output tiles, 256 threads with 4 x 4 outputs each, K in steps of 16
-// through shared memory; tiles of all groups in one grid-stride list.
-__global__ void __launch_bounds__(256) rows_gemm_kernel(RowsGemm p) {
-    __shared__ float As[BK][BM + 4];
-    __shared__ float Bs[BK][BN + 4];
+// 128 x 128 output tiles, 256 threads with 8 x 8 outputs each, K in slabs of
+// 16 through shared memory; the tile's row offsets (the gather resolved) are
+// computed once per tile.  Tiles of all groups in one grid-stride list.
+__global__ void __launch_bounds__(256, 2) rows_gemm_kernel(RowsGemm p) {
+    __shared__ __align__(16) float As[TK][TB + 4];
+    __shared__ __align__(16) float Bs[TK][TB + 4];
+    __shared__ long long arow[TB], brow[TB];
     __shared__ int prefix[kMaxGroups + 1];
     __shared__ int gstart[kMaxGroups], grows[kMaxGroups];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-    const int n_tiles = (p.N + BN - 1) / BN;
+    const int n_tiles = (p.N + TB - 1) / TB;
     for (int g = tid; g < p.G; g += blockDim.x) {
         int rs, re;
         group_rows(p.offsets, g, p.M, p.status, rs, re);
@@ -106,7 +128,7 @@ __global__ void __launch_bounds__(256) rows_gemm_kernel(RowsGemm p) {
         int acc = 0;
         for (int g = 0; g < p.G; ++g) {
             prefix[g] = acc;
-            acc += (grows[g] + BM - 1) / BM * n_tiles;
+            acc += (grows[g] + TB - 1) / TB * n_tiles;
         }
         prefix[p.G] = acc;
     }
@@ -119,45 +141,45 @@ __global__ void __launch_bounds__(256) rows_gemm_kernel(RowsGemm p) {
             if (prefix[mid] <= tile) lo = mid; else hi = mid - 1;
         }
         const int g = lo;
-        const int mt = (grows[g] + BM - 1) / BM;
+        const int mt = (grows[g] + TB - 1) / TB;
         const int q = tile - prefix[g];
-        const int m0 = (q % mt) * BM, n0 = (q / mt) * BN;
+        const int m0 = (q % mt) * TB, n0 = (q / mt) * TB;
         const int row0 = gstart[g] + m0;
-        const int nrows = min(BM, grows[g] - m0);
-        float acc[4][4] = {};
-        for (int k0 = 0; k0 < p.K; k0 += BK) {
+        const int nrows = min(TB, grows[g] - m0);
+        __syncthreads();  // the previous tile's readers of arow / brow are done
+        if (tid < TB) {
+            arow[tid] = tid < nrows ? row_off(p.A, row0 + tid) : -1;
+        } else {
+            const int n = tid - TB;
+            brow[n] = n0 + n < p.N ? (long long)g * p.B.gs + (long long)(n0 + n) * p.B.rs : -1;
+        }
+        __syncthreads();
+        // each thread loads one row of each operand per slab: 8 consecutive k
+        // (k contiguous in memory) or every other k (rows contiguous)
+        const int am = a_kfast ? tid >> 1 : tid & (TB - 1), bn = b_kfast ? tid >> 1 : tid & (TB - 1);
+        const long long ra = arow[am], rb = brow[bn];
+        float acc[8][8] = {};
+#pragma unroll 1
+        for (int k0 = 0; k0 < p.K; k0 += TK) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int e = tid + 256 * i;
-                const int m = a_kfast ? e / BK : e % BM, kk = a_kfast ? e % BK : e / BM;
-                As[kk][m] = (m < nrows && k0 + kk < p.K) ? opnd_ld(p.A, row0 + m, k0 + kk, 0) : 0.0f;
-                const int n = b_kfast ? e / BK : e % BN, kb = b_kfast ? e % BK : e / BN;
-                Bs[kb][n] = (n0 + n < p.N && k0 + kb < p.K) ? opnd_ld(p.B, n0 + n, k0 + kb, g) : 0.0f;
+            for (int i = 0; i < 8; ++i) {
+                const int ka = a_kfast ? (tid & 1) * 8 + i : (tid >> 7) + 2 * i;
+                As[ka][am] = (ra >= 0 && k0 + ka < p.K) ? ld_at(p.A, ra + (long long)(k0 + ka) * p.A.cs) : 0.0f;
+                const int kb = b_kfast ? (tid & 1) * 8 + i : (tid >> 7) + 2 * i;
+                Bs[kb][bn] = (rb >= 0 && k0 + kb < p.K) ? ld_at(p.B, rb + (long long)(k0 + kb) * p.B.cs) : 0.0f;
             }
             __syncthreads();
-#pragma unroll
-            for (int kk = 0; kk < BK; ++kk) {
-                float a[4], b[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    a[i] = As[kk][ty * 4 + i];
-                    b[i] = Bs[kk][tx * 4 + i];
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-            }
+            slab_fma(As, Bs, ty, tx, acc);
             __syncthreads();
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int m = ty * 4 + i;
+        for (int i = 0; i < 8; ++i) {
+            const int m = ty * 8 + i;
             if (m >= nrows) continue;
             float* crow = p.C + (long long)(row0 + m) * p.c_rs;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int n = n0 + tx * 4 + j;
+            for (int j = 0; j < 8; ++j) {
+                const int n = n0 + tx * 8 + j;
                 if (n < p.N) crow[n] = p.accumulate ? crow[n] + acc[i][j] : acc[i][j];
             }
         }
@@ -177,51 +199,50 @@ struct WgradGemm {
 };
 
 // C_g[m][n] (+)= sum over the rows r of group g of A(r, m) B(r, n).  Grid:
-// x = output tiles of one group, y = group.  An empty group writes zeros.
-__global__ void __launch_bounds__(256) wgrad_gemm_kernel(WgradGemm p) {
-    __shared__ float As[BK][BM + 4];
-    __shared__ float Bs[BK][BN + 4];
+// x = 128 x 128 output tiles of one group, y = group; the slab's 16 row
+// offsets of each operand are resolved once per slab.  An empty group writes
+// zeros.
+__global__ void __launch_bounds__(256, 2) wgrad_gemm_kernel(WgradGemm p) {
+    __shared__ __align__(16) float As[TK][TB + 4];
+    __shared__ __align__(16) float Bs[TK][TB + 4];
+    __shared__ long long arow[TK], brow[TK];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int g = blockIdx.y;
-    const int m_tiles = (p.M + BM - 1) / BM;
-    const int m0 = (blockIdx.x % m_tiles) * BM, n0 = (blockIdx.x / m_tiles) * BN;
+    const int m_tiles = (p.M + TB - 1) / TB;
+    const int m0 = (blockIdx.x % m_tiles) * TB, n0 = (blockIdx.x / m_tiles) * TB;
     int rs, re;
     group_rows(p.offsets, g, p.rows, p.status, rs, re);
     const bool a_mfast = p.A.cs == 1, b_nfast = p.B.cs == 1;
-    float acc[4][4] = {};
-    for (int r0 = rs; r0 < re; r0 += BK) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int e = tid + 256 * i;
-            const int m = a_mfast ? e % BM : e / BK, kk = a_mfast ? e / BM : e % BK;
-            As[kk][m] = (r0 + kk < re && m0 + m < p.M) ? opnd_ld(p.A, r0 + kk, m0 + m, 0) : 0.0f;
-            const int n = b_nfast ? e % BN : e / BK, kb = b_nfast ? e / BN : e % BK;
-            Bs[kb][n] = (r0 + kb < re && n0 + n < p.N) ? opnd_ld(p.B, r0 + kb, n0 + n, 0) : 0.0f;
+    float acc[8][8] = {};
+    for (int r0 = rs; r0 < re; r0 += TK) {
+        if (tid < TK) {
+            arow[tid] = r0 + tid < re ? row_off(p.A, r0 + tid) : -1;
+        } else if (tid < 2 * TK) {
+            brow[tid - TK] = r0 + tid - TK < re ? row_off(p.B, r0 + tid - TK) : -1;
         }
         __syncthreads();
 #pragma unroll
-        for (int kk = 0; kk < BK; ++kk) {
-            float a[4], b[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                a[i] = As[kk][ty * 4 + i];
-                b[i] = Bs[kk][tx * 4 + i];
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int i = 0; i < 8; ++i) {
+            const int e = tid + 256 * i;
+            const int m = a_mfast ? e % TB : e / TK, kk = a_mfast ? e / TB : e % TK;
+            const long long ra = arow[kk];
+            As[kk][m] = (ra >= 0 && m0 + m < p.M) ? ld_at(p.A, ra + (long long)(m0 + m) * p.A.cs) : 0.0f;
+            const int n = b_nfast ? e % TB : e / TK, kb = b_nfast ? e / TB : e % TK;
+            const long long rb = brow[kb];
+            Bs[kb][n] = (rb >= 0 && n0 + n < p.N) ? ld_at(p.B, rb + (long long)(n0 + n) * p.B.cs) : 0.0f;
         }
+        __syncthreads();
+        slab_fma(As, Bs, ty, tx, acc);
         __syncthreads();
     }
     float* cg = p.C + (long long)g * p.c_gs;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int m = m0 + ty * 4 + i;
+    for (int i = 0; i < 8; ++i) {
+        const int m = m0 + ty * 8 + i;
         if (m >= p.M) continue;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int n = n0 + tx * 4 + j;
+        for (int j = 0; j < 8; ++j) {
+            const int n = n0 + tx * 8 + j;
             if (n < p.N) {
                 float* c = cg + (long long)m * p.c_rs + n;
                 *c = p.accumulate ? *c + acc[i][j] : acc[i][j];
@@ -413,8 +434,8 @@ cudaError_t rows_gemm(const Opnd& A, const Opnd& B, float* C, long long c_rs, in
     if (M <= 0 || N <= 0) return cudaSuccess;
     RowsGemm p{A, B, C, c_rs, M, N, K, offsets, G, accumulate ? 1 : 0, status};
     // an upper bound of the tile count: every group adds at most one partial m-tile
-    const long long tiles = ((long long)(M + BM - 1) / BM + G) * ((N + BN - 1) / BN);
-    const int grid = (int)(tiles < (long long)num_sms * 8 ? tiles : (long long)num_sms * 8);
+    const long long tiles = ((long long)(M + TB - 1) / TB + G) * ((N + TB - 1) / TB);
+    const int grid = (int)(tiles < (long long)num_sms * 2 ? tiles : (long long)num_sms * 2);
     rows_gemm_kernel<<<grid, 256, 0, st>>>(p);
     note_launches(1);
     return cudaGetLastError();
@@ -424,7 +445,7 @@ cudaError_t wgrad_gemm(const Opnd& A, const Opnd& B, float* C, long long c_rs, l
                        const int32_t* offsets, int G, int rows, bool accumulate, int* status, cudaStream_t st) {
     if (M <= 0 || N <= 0 || G <= 0) return cudaSuccess;
     WgradGemm p{A, B, C, c_rs, c_gs, M, N, offsets, G, rows, accumulate ? 1 : 0, status};
-    const dim3 grid((unsigned)(((M + BM - 1) / BM) * ((N + BN - 1) / BN)), (unsigned)G);
+    const dim3 grid((unsigned)(((M + TB - 1) / TB) * ((N + TB - 1) / TB)), (unsigned)G);
     wgrad_gemm_kernel<<<grid, 256, 0, st>>>(p);
     note_launches(1);
     return cudaGetLastError();
