@@ -32,6 +32,39 @@ def allreduce_counts(counts: torch.Tensor, group=None) -> torch.Tensor:
     return counts
 
 
+# ---- backward under token-sharded data parallelism ---------------------------------
+#
+# Each rank runs moe_layer_backward on its own tokens.  x's gradient stays
+# per rank; the weight gradients of the replicated layer are sums over the
+# tokens of all ranks, so they are summed over the ranks (the backward's one
+# exchange).  The balance loss is a mean over the batch's sequences: with
+# every rank holding whole sequences, a rank runs its backward with its share
+# of the weight, alpha * (its sequences / all sequences), and the summed
+# gradients and losses are then exactly those of the whole batch.
+
+WEIGHT_GRADS = ("dw_gate", "dw1", "dw3", "dw2", "dws1", "dws3", "dws2")
+
+
+def local_balance_alpha(alpha: float, tokens_per_rank: int, world: int) -> float:
+    """The balance-loss weight one rank's backward uses so that the sum over
+    the ranks is the batch's loss (equal, whole-sequence shards)."""
+    return alpha * tokens_per_rank / global_token_count(tokens_per_rank, world)
+
+
+def allreduce_grads(grads: dict, group=None) -> dict:
+    """Sum the weight gradients (and the balance loss, key 'balance_loss',
+    a 1-element tensor) over the ranks in place; other entries (dx) are left
+    per rank.  No-op on one rank."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1):
+        return grads
+    for name in WEIGHT_GRADS + ("balance_loss",):
+        t = grads.get(name)
+        if t is not None:
+            dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+    return grads
+
+
 # ---- expert parallelism ---------------------------------------------------------
 #
 # Experts sharded over the ranks (rank o owns experts [o*E/W, (o+1)*E/W)),

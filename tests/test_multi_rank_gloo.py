@@ -136,3 +136,80 @@ def test_expert_parallel_counts_exchange():
     Epr = cfg.E // WORLD
     recv = [allc[:, o * Epr:(o + 1) * Epr].sum() for o in range(WORLD)]
     assert sum(recv) == WORLD * cfg.T * cfg.k
+
+
+# ---- backward under token-sharded data parallelism
+
+def _bwd_cfg():
+    from fine_grained_moe_gate_b200.inputs import CONFIGS
+    return CONFIGS["tiny_fp32"].scaled(T=12, d=16, E=8, k=2, I=8, S=1, Is=8)
+
+
+BWD_ALPHA, BWD_SEQ = 0.05, 4
+
+
+def _bwd_grads(cfg, x, p, alpha):
+    """Oracle backward (stands in for moe_layer_backward) of one rank's tokens."""
+    import oracle
+    from oracle import backward as ob
+    from fine_grained_moe_gate_b200.inputs import to_numpy
+
+    xn = to_numpy(x)
+    s = oracle.affinity(xn, to_numpy(p["w_gate"]))
+    idx, w = oracle.select(s, p["bias"].numpy(), cfg.k)
+    g = torch.Generator().manual_seed(int(x.sum().abs().item() * 1000) % (1 << 31))
+    dy = torch.randn((x.shape[0], cfg.d), generator=g, dtype=torch.float64).numpy()
+    out = ob.layer_backward(xn, to_numpy(p["w_gate"]), idx, w, s, *[to_numpy(p[n]) for n in
+                            ("w1", "w3", "w2", "ws1", "ws3", "ws2")], dy, alpha=alpha, seq_len=BWD_SEQ)
+    return out, dy
+
+
+def _bwd_worker(rank, port, out_dir):
+    import torch.distributed as dist
+
+    from fine_grained_moe_gate_b200 import dist as mdist
+    from fine_grained_moe_gate_b200.inputs import make_layer, make_tokens
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD, timeout=datetime.timedelta(seconds=10))
+    cfg = _bwd_cfg()
+    p = make_layer(cfg, "cpu")
+    x = make_tokens(cfg, "cpu", step=mdist.shard_step(0, rank, WORLD))
+    out, _ = _bwd_grads(cfg, x, p, mdist.local_balance_alpha(BWD_ALPHA, cfg.T, WORLD))
+    grads = {n: torch.from_numpy(np.ascontiguousarray(out[n])) for n in mdist.WEIGHT_GRADS}
+    grads["balance_loss"] = torch.tensor([out["balance_loss"]], dtype=torch.float64)
+    mdist.allreduce_grads(grads)
+    np.savez(os.path.join(out_dir, f"bwd{rank}.npz"), dx=out["dx"], **{n: t.numpy() for n, t in grads.items()})
+    dist.destroy_process_group()
+
+
+def test_backward_data_parallel_equals_whole_batch():
+    """Two ranks, each with its own tokens: after the weight-gradient
+    all-reduce every rank holds the whole batch's weight gradients and
+    balance loss, and each rank's dx is the whole batch's dx for its rows."""
+    from fine_grained_moe_gate_b200 import dist as mdist
+    from fine_grained_moe_gate_b200.inputs import make_layer, make_tokens
+
+    out_dir = tempfile.mkdtemp(prefix="gloo_bwd_")
+    mp.start_processes(_bwd_worker, args=(_free_port(), out_dir), nprocs=WORLD, join=True, start_method="spawn")
+    res = [dict(np.load(os.path.join(out_dir, f"bwd{r}.npz"))) for r in range(WORLD)]
+    cfg = _bwd_cfg()
+    p = make_layer(cfg, "cpu")
+    xs = [make_tokens(cfg, "cpu", step=mdist.shard_step(0, r, WORLD)) for r in range(WORLD)]
+    # the whole batch in one process: same tokens, same per-rank dy, the batch's alpha
+    import oracle
+    from oracle import backward as ob
+    from fine_grained_moe_gate_b200.inputs import to_numpy
+    dys = [_bwd_grads(cfg, x, p, 0.0)[1] for x in xs]
+    x = torch.cat(xs)
+    s = oracle.affinity(to_numpy(x), to_numpy(p["w_gate"]))
+    idx, w = oracle.select(s, p["bias"].numpy(), cfg.k)
+    ref = ob.layer_backward(to_numpy(x), to_numpy(p["w_gate"]), idx, w, s, *[to_numpy(p[n]) for n in
+                            ("w1", "w3", "w2", "ws1", "ws3", "ws2")], np.concatenate(dys), alpha=BWD_ALPHA,
+                            seq_len=BWD_SEQ)
+    for r in range(WORLD):
+        for n in mdist.WEIGHT_GRADS:
+            assert np.allclose(res[r][n], ref[n], rtol=1e-12, atol=1e-14), (r, n)
+        assert abs(float(res[r]["balance_loss"][0]) - ref["balance_loss"]) < 1e-14
+        assert np.allclose(res[r]["dx"], ref["dx"][r * cfg.T:(r + 1) * cfg.T], rtol=1e-12, atol=1e-14)
