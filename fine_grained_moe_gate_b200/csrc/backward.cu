@@ -60,6 +60,32 @@ __device__ __forceinline__ float ld_at(const Opnd& o, long long off) {
     return static_cast<const float*>(o.p)[off];
 }
 
+// Eight consecutive elements from element offset off (16-byte aligned for
+// bf16, 32-byte aligned for fp32: one or two vector loads).
+__device__ __forceinline__ void ld8(const Opnd& o, long long off, float (&v)[8]) {
+    if (o.bf16) {
+        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(o.p) + off);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    } else {
+        const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(o.p) + off);
+        const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(o.p) + off + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+// A k-contiguous operand whose row and group strides keep every run of eight
+// elements starting at a multiple of 8 on a 16-byte (bf16) / 32-byte (fp32)
+// boundary: the rows GEMM then loads its eight k per thread with ld8.
+bool vec8_ok(const void* p, int bf16, long long rs, long long cs, long long gs) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return cs == 1 && rs % 8 == 0 && gs % 8 == 0 && (a % (bf16 ? 16u : 32u)) == 0;
+}
+
 // Rows r of group g: [offsets[g], offsets[g+1]) or, without offsets, [0, M).
 // A corrupt range is skipped and reported.
 __device__ __forceinline__ void group_rows(const int32_t* offsets, int g, int M, int* status, int& rs, int& re) {
@@ -102,6 +128,7 @@ struct RowsGemm {
     const int32_t* offsets;
     int G;
     int accumulate;
+    int a_vec, b_vec;   // operand loads eight k at a time (vec8_ok)
     int* status;
 };
 
@@ -161,12 +188,30 @@ __global__ void __launch_bounds__(256, 2) rows_gemm_kernel(RowsGemm p) {
         float acc[8][8] = {};
 #pragma unroll 1
         for (int k0 = 0; k0 < p.K; k0 += TK) {
+            const int kh = k0 + (tid & 1) * 8;  // first of this thread's eight k (k-contiguous operands)
+            if (p.a_vec && ra >= 0 && kh + 8 <= p.K) {
+                float v[8];
+                ld8(p.A, ra + kh, v);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int ka = a_kfast ? (tid & 1) * 8 + i : (tid >> 7) + 2 * i;
-                As[ka][am] = (ra >= 0 && k0 + ka < p.K) ? ld_at(p.A, ra + (long long)(k0 + ka) * p.A.cs) : 0.0f;
-                const int kb = b_kfast ? (tid & 1) * 8 + i : (tid >> 7) + 2 * i;
-                Bs[kb][bn] = (rb >= 0 && k0 + kb < p.K) ? ld_at(p.B, rb + (long long)(k0 + kb) * p.B.cs) : 0.0f;
+                for (int i = 0; i < 8; ++i) As[(tid & 1) * 8 + i][am] = v[i];
+            } else {
+#pragma unroll 1
+                for (int i = 0; i < 8; ++i) {
+                    const int ka = a_kfast ? (tid & 1) * 8 + i : (tid >> 7) + 2 * i;
+                    As[ka][am] = (ra >= 0 && k0 + ka < p.K) ? ld_at(p.A, ra + (long long)(k0 + ka) * p.A.cs) : 0.0f;
+                }
+            }
+            if (p.b_vec && rb >= 0 && kh + 8 <= p.K) {
+                float v[8];
+                ld8(p.B, rb + kh, v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) Bs[(tid & 1) * 8 + i][bn] = v[i];
+            } else {
+#pragma unroll 1
+                for (int i = 0; i < 8; ++i) {
+                    const int kb = b_kfast ? (tid & 1) * 8 + i : (tid >> 7) + 2 * i;
+                    Bs[kb][bn] = (rb >= 0 && k0 + kb < p.K) ? ld_at(p.B, rb + (long long)(k0 + kb) * p.B.cs) : 0.0f;
+                }
             }
             __syncthreads();
             slab_fma(As, Bs, ty, tx, acc);
@@ -398,17 +443,30 @@ __global__ void router_bwd_kernel(const float* __restrict__ s, const int32_t* __
     }
 }
 
-// One block per sequence b: part[b] = alpha * sum_i f_bi P_bi.
-__global__ void balance_part_kernel(const float* __restrict__ s, const float* __restrict__ tot,
-                                    const int32_t* __restrict__ cnt, float alpha, int L, int E, int k,
-                                    float* __restrict__ part) {
+constexpr int kLossChunk = 64;  // tokens per partial sum of the balance loss
+
+// Block (c, b): chunk[b][c][i] = sum over tokens t of chunk c of sequence b of s_ti / tot_t.
+__global__ void balance_chunk_kernel(const float* __restrict__ s, const float* __restrict__ tot, int L, int E,
+                                     int C, float* __restrict__ chunk) {
+    const int b = blockIdx.y, c = blockIdx.x;
+    const int t0 = b * L + c * kLossChunk, t1 = min((b + 1) * L, t0 + kLossChunk);
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        float P = 0.0f;
+        for (int t = t0; t < t1; ++t) P += s[(long long)t * E + i] / tot[t];
+        chunk[((long long)b * C + c) * E + i] = P;
+    }
+}
+
+// One block per sequence b: part[b] = alpha * sum_i f_bi P_bi, the chunks summed in order.
+__global__ void balance_part_kernel(const float* __restrict__ chunk, const int32_t* __restrict__ cnt, float alpha,
+                                    int L, int E, int k, int C, float* __restrict__ part) {
     __shared__ float red[32];
     const int b = blockIdx.x;
     const float fscale = (float)E / ((float)k * (float)L);
     float v = 0.0f;
     for (int i = threadIdx.x; i < E; i += blockDim.x) {
         float P = 0.0f;
-        for (int t = b * L; t < (b + 1) * L; ++t) P += s[(long long)t * E + i] / tot[t];
+        for (int c = 0; c < C; ++c) P += chunk[((long long)b * C + c) * E + i];
         v += fscale * (float)cnt[(long long)b * E + i] * (P / (float)L);
     }
     v = block_sum(v, red);
@@ -432,7 +490,9 @@ Opnd view(const void* p, bool bf16, long long rs, long long cs, long long gs = 0
 cudaError_t rows_gemm(const Opnd& A, const Opnd& B, float* C, long long c_rs, int M, int N, int K,
                       const int32_t* offsets, int G, bool accumulate, int* status, int num_sms, cudaStream_t st) {
     if (M <= 0 || N <= 0) return cudaSuccess;
-    RowsGemm p{A, B, C, c_rs, M, N, K, offsets, G, accumulate ? 1 : 0, status};
+    RowsGemm p{A, B, C, c_rs, M, N, K, offsets, G, accumulate ? 1 : 0,
+               vec8_ok(A.p, A.bf16, A.rs, A.cs, A.gs) ? 1 : 0, vec8_ok(B.p, B.bf16, B.rs, B.cs, B.gs) ? 1 : 0,
+               status};
     // an upper bound of the tile count: every group adds at most one partial m-tile
     const long long tiles = ((long long)(M + TB - 1) / TB + G) * ((N + TB - 1) / TB);
     const int grid = (int)(tiles < (long long)num_sms * 2 ? tiles : (long long)num_sms * 2);
@@ -462,9 +522,10 @@ size_t backward_scratch_bytes(int T, int d, int E, int k, int I, int S, int Is, 
     auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
     const size_t R = (size_t)T * k;
     const size_t nb = seq_len > 0 ? (size_t)T / seq_len : 0;
+    const size_t C = seq_len > 0 ? ((size_t)seq_len + kLossChunk - 1) / kLossChunk : 0;
     return al((E + 1) * 4) + 2 * al(R * 4) + al(permute_scratch_bytes(T, E)) + 4 * al(R * I * 4) + al(R * d * 4) +
            al(R * 4) + 4 * al((size_t)T * S * Is * 4) + al((size_t)T * E * 4) + al((size_t)T * 4) + al(nb * E * 4) +
-           al(nb * 4);
+           al(nb * 4) + al(nb * C * E * 4);
 }
 
 cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sms, cudaStream_t st) {
@@ -498,6 +559,8 @@ cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sm
     float* tot = reinterpret_cast<float*>(take((size_t)T * 4));
     int32_t* cnt = reinterpret_cast<int32_t*>(take((size_t)nb * E * 4));
     float* part = reinterpret_cast<float*>(take((size_t)nb * 4));
+    const int C = nb > 0 ? (a.seq_len + kLossChunk - 1) / kLossChunk : 0;
+    float* chunk = reinterpret_cast<float*>(take((size_t)nb * C * E * 4));
 
     cudaError_t err;
 #define BWD_TRY(x)                          \
@@ -586,9 +649,10 @@ cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sm
                                                         nb, T, E, k, dz, tot, status);
         note_launches(1);
         if (nb > 0 && a.loss) {
-            balance_part_kernel<<<nb, 256, 0, st>>>(a.s, tot, cnt, a.alpha, a.seq_len, E, k, part);
+            balance_chunk_kernel<<<dim3((unsigned)C, (unsigned)nb), 256, 0, st>>>(a.s, tot, a.seq_len, E, C, chunk);
+            balance_part_kernel<<<nb, 256, 0, st>>>(chunk, cnt, a.alpha, a.seq_len, E, k, C, part);
             balance_sum_kernel<<<1, 32, 0, st>>>(part, nb, a.loss);
-            note_launches(2);
+            note_launches(3);
         }
         // dx += dz W_g;  dW_g = dz^T x
         BWD_TRY(rows_gemm(view(dz, false, E, 1), view(a.w_gate, bf, 1, d), a.dx, d, T, d, E, nullptr, 1, true, status,
