@@ -549,6 +549,7 @@ moe_status moe_layer_backward(const void* x, const void* w_gate, const void* w1,
     MOE_REQUIRE(sh.S == 0 || (ws1 && ws3 && ws2 && dws1 && dws3 && dws2), MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(alpha == alpha && alpha >= 0.0f && alpha < 3.0e38f, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(alpha == 0.0f || (seq_len > 0 && sh.T % seq_len == 0), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(alpha == 0.0f || sh.T / seq_len <= 65535, MOE_ERR_UNSUPPORTED);  // sequences per launch
     MOE_REQUIRE(aligned16(x) && aligned16(w_gate) && aligned16(w1) && aligned16(w3) && aligned16(w2) &&
                     aligned16(ws1) && aligned16(ws3) && aligned16(ws2) && aligned16(topk_idx) && aligned16(topk_w) &&
                     aligned16(counts) && aligned16(affinity) && aligned16(dy) && aligned16(dx) &&

@@ -267,7 +267,8 @@ MOE_API size_t moe_workspace_size(moe_shape sh);  /* moe_layer_forward, or moe_l
  * Inputs: x, w_gate, w1, w3, w2, ws1, ws3, ws2 as in moe_layer_forward
  * (dtype MOE_F32 or MOE_BF16); topk_idx, topk_w and counts as moe_route
  * returned them; affinity [T][E] fp32, moe_route's affinity_out; dy [T][d]
- * fp32.  alpha >= 0; with alpha > 0, seq_len > 0 must divide T.  h is
+ * fp32.  alpha >= 0; with alpha > 0, seq_len > 0 must divide T (at most
+ * 65535 sequences per call, else MOE_ERR_UNSUPPORTED).  h is
  * recomputed and rounded like the forward's (bf16 layers); the output
  * rounding of y is treated as identity.  fp32 accumulation throughout.
  * dws1 / dws3 / dws2 and ws1 / ws3 / ws2 may be NULL when S == 0.

@@ -190,6 +190,7 @@ def test_backward_checks(L):
     assert call(alpha=float("nan")) == INVALID
     assert call(alpha=0.01, L_=0) == INVALID          # a balance loss needs a sequence length
     assert call(alpha=0.01, L_=48) == INVALID         # that divides T = 128
+    assert call(sh=shape(T=65536 * 2), alpha=0.01, L_=1) == UNSUPPORTED   # more than 65535 sequences
     assert call(dx=FAKE + 4) == ALIGN
     assert call(nbytes=need - 256) == WORKSPACE
     assert call(alpha=0.01, L_=32) == WORKSPACE       # the sequences' buffers are not in `need`
