@@ -27,6 +27,10 @@ and its output copied back, double-buffered on two copy streams so that the
 copies of one step overlap the compute of the next.
 
 Rank 0 prints one JSON line.
+
+--backward times moe_layer_backward instead (one GPU, its own JSON line): the
+gradients of x, the gate and every expert weight plus the sequence-wise
+balance loss for a routing computed once before timing.
 """
 from __future__ import annotations
 

@@ -195,3 +195,19 @@ def test_backward_checks(L):
     assert call(nbytes=need - 256) == WORKSPACE
     assert call(alpha=0.01, L_=32) == WORKSPACE       # the sequences' buffers are not in `need`
     assert call(ws=FAKE + 128) == ALIGN
+
+
+def test_backward_binding_marshals_and_raises(L):
+    """The Python wrapper passes its 28 arguments in header order: a call
+    whose only fault is a missing dy comes back as MOE_ERR_INVALID_ARG."""
+    import torch
+    sh = shape()
+    ws = torch.empty(256, dtype=torch.uint8)   # never reached: validation fails first
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_layer_backward(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, sh, FAKE, FAKE, FAKE, FAKE, None, 0.0,
+                               0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, ws, stream=0)
+    assert ei.value.status == INVALID
+    with pytest.raises(moe.MoEError) as ei:   # every pointer given, alpha negative
+        moe.moe_layer_backward(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, sh, FAKE, FAKE, FAKE, FAKE, FAKE, -1.0,
+                               0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, ws, stream=0)
+    assert ei.value.status == INVALID
