@@ -106,6 +106,28 @@ def test_skew_stress_routing_and_sampled_output():
     check_status()
 
 
+def test_skew_stress_bias_trajectory_200_steps():
+    """The skew workload's load trajectory ("A bias term for each expert":
+    the bias moves by the fixed step at the end of every step): 200 steps of
+    routing and bias update, a fresh batch per step; every step's choices
+    and bias bit-exact against the oracle taking the kernel's affinities."""
+    cfg = CONFIGS["skew_stress"]
+    sh = moe.shape_of(cfg)
+    p = make_layer(cfg, DEV)
+    bias_orc = p["bias"].cpu().numpy().copy()
+    for step in range(200):
+        x = make_tokens(cfg, DEV, step)
+        idx, _, counts, aff = route(sh, x, p["w_gate"], p["bias"])
+        o_idx, _ = oracle.select(aff.cpu().numpy(), bias_orc, cfg.k)
+        assert (o_idx == idx.cpu().numpy()).all(), f"step {step}"
+        assert (oracle.histogram(o_idx, cfg.E) == counts.cpu().numpy()).all(), f"step {step}"
+        moe.moe_load_and_bias_update(counts, sh, cfg.step_size, None, p["bias"])
+        torch.cuda.synchronize()
+        bias_orc, _ = oracle.bias_update(oracle.histogram(o_idx, cfg.E), bias_orc, cfg.T, cfg.k, cfg.step_size)
+        assert (p["bias"].cpu().numpy().view(np.uint32) == bias_orc.view(np.uint32)).all(), f"step {step}"
+    check_status()
+
+
 # ------------------------------------------------------------------ FP8 experts
 
 def _oracle_rows_fp8(q, x, idx, w, tokens, cfg):
