@@ -1,5 +1,7 @@
 /*
- * moe_gate.h -- C ABI of the B200 (sm_100a) fine-grained MoE layer forward.
+ * moe_gate.h -- C ABI of the B200 (sm_100a) fine-grained MoE layer: the
+ * forward (bf16 / fp32, and E4M3 experts), expert-parallel dispatch and
+ * return, and the layer backward with the sequence-wise balance loss.
  *
  * The layer is the DeepSeek-V3 MoE feed-forward as the following web pages
  * state it (cited by page title and section):
@@ -14,7 +16,10 @@
  *        (per-step load over the whole batch, fixed +-0.001 bias step).
  *   [P4] "DeepSeek V3 Architecture Deep Dive: Multi-Head Latent Attention
  *        (MLA), DeepSeekMoE & FP8 Mixed Precision": "Throughput on NVIDIA
- *        H100/H800" (tokens routed to the same expert batched together).
+ *        H100/H800" (tokens routed to the same expert batched together),
+ *        "FP8 Formats" and "Per-Tensor/Per-Axis Quantization".
+ *   [P5] crackai.dev "DeepSeek-V3": "How It Works" (all-to-all dispatch /
+ *        combine kernels for expert parallelism).
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the
