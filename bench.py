@@ -26,7 +26,12 @@ moe_layer_forward_fp8) with each step's tokens copied from pinned host memory
 and its output copied back, double-buffered on two copy streams so that the
 copies of one step overlap the compute of the next.
 
-Rank 0 prints one JSON line.
+Rank 0 prints one JSON line.  With the default workload (v3_prefill) the
+line also carries, under "workloads", the decode-shaped workload (T=64 per
+call, 1000 calls with fresh tokens each) and the skewed-routing workload
+(T=32768, Zipf(1.2) popularity, 200 steps with the bias updated every step,
+reporting the most-loaded expert's rows over the mean per step), each timed
+the same way with its own roofline (HBM for decode, tensor for skew).
 
 --backward times moe_layer_backward instead (one GPU, its own JSON line): the
 gradients of x, the gate and every expert weight plus the sequence-wise
@@ -71,6 +76,10 @@ def parse_args():
     ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0: per-workload default)")
     ap.add_argument("--T", type=int, default=0, help="override tokens per GPU (profiling slices)")
     ap.add_argument("--E", type=int, default=0, help="override routed experts (profiling slices)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="v3_prefill only: skip the decode and skew workloads of the default line")
+    ap.add_argument("--decode-calls", type=int, default=1000, help="decode workload: timed calls (fresh x each)")
+    ap.add_argument("--skew-steps", type=int, default=200, help="skew workload: timed steps")
     ap.add_argument("--backward", action="store_true",
                     help="time moe_layer_backward (one GPU) instead of the forward step; prints its own line")
     return ap.parse_args()
@@ -89,18 +98,38 @@ def load_peaks():
 # --------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples of the SM clock and throttle reasons while the
-    timed region runs."""
+    """SM clock, power and throttle reasons sampled while the timed region
+    runs: NVML polled from a thread every 5 ms (nvidia-smi at 50 ms if NVML
+    is unavailable)."""
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id: str):
+    def __init__(self, gpu_id: str, period_s: float = 0.005):
         self.gpu_id = gpu_id
+        self.period = period_s
+        self.samples = []
         self.proc = None
-        self.path = None
+        self.thread = None
+        self.nvml = None
 
     def start(self):
+        import threading
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid_or_idx = self.gpu_id
+            h = (pynvml.nvmlDeviceGetHandleByUUID(uuid_or_idx) if not uuid_or_idx.isdigit()
+                 else pynvml.nvmlDeviceGetHandleByIndex(int(uuid_or_idx)))
+            self.nvml = (pynvml, h)
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            self.stop_evt = threading.Event()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
         os.close(fd)
         try:
@@ -111,38 +140,56 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.out.close()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = set()
-        sm, smax, pw = [], [], []
-        for r in rows:
+    def _poll(self):
+        pynvml, h = self.nvml
+        bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+        smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.stop_evt.is_set():
             try:
-                sm.append(float(r[1]))
-                smax.append(float(r[2]))
-                pw.append(float(r[3]))
-            except ValueError:
-                continue
-            for n, v in zip(names, r[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm),
-                "power_w_median": statistics.median(pw) if pw else None}
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(smax), pw, [n for n, b in bits.items() if rs & b]))
+            except Exception:
+                pass
+            self.stop_evt.wait(self.period)
+
+    def stop(self):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            rows = self.samples
+            src = "nvml 5 ms"
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.close()
+            rows = []
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) < 9:
+                        continue
+                    try:
+                        rows.append((float(parts[1]), float(parts[2]), float(parts[3]),
+                                     [n for n, v in zip(self.REASONS, parts[5:9]) if v.lower() == "active"]))
+                    except ValueError:
+                        continue
+            os.unlink(self.path)
+            src = "nvidia-smi 50 ms"
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"], "samples": 0}
+        sm = [r[0] for r in rows]
+        reasons = sorted({n for r in rows for n in r[3]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(r[1] for r in rows) if rows else None,
+                "reasons": reasons, "samples": len(rows), "source": src,
+                "power_w_median": statistics.median(r[2] for r in rows) if rows else None}
 
 
 # ------------------------------------------------------------ oracle leg
@@ -279,8 +326,255 @@ def workload(args):
     return cfg
 
 
+class LayerStep:
+    """Device buffers and the step of one workload on one rank: route,
+    (quantize x,) permute, gate/up, (quantize h,) down, combine, counts
+    all-reduce when N > 1, bias update.  ``xs`` are the step inputs, cycled."""
+
+    def __init__(self, cfg, dev, world, p, xs, stream):
+        import torch
+        import fine_grained_moe_gate_b200 as moe
+        from fine_grained_moe_gate_b200 import dist as mdist
+        self.moe, self.mdist, self.torch = moe, mdist, torch
+        self.cfg, self.p, self.xs, self.stream = cfg, p, xs, stream
+        self.sh = moe.shape_of(cfg)
+        self.sh_global = moe.shape_of(cfg, T=mdist.global_token_count(cfg.T, world))  # the step's batch
+        self.fp8 = cfg.dtype == "fp8"
+        self.stages = STAGES_FP8 if self.fp8 else STAGES
+        T, k, d, E = cfg.T, cfg.k, cfg.d, cfg.E
+        dt = cfg.torch_dtype
+        e = lambda *s, dtype=torch.int32: torch.empty(s, dtype=dtype, device=dev)
+        self.idx, self.w, self.counts = e(T, k), e(T, k, dtype=torch.float32), e(E)
+        self.offsets, self.perm, self.inv = e(E + 1), e(T * k), e(T * k)
+        self.pws = e(max(moe.moe_permute_workspace_size(self.sh), 256), dtype=torch.uint8)
+        self.x_perm = e(T * k, d, dtype=dt)   # x_perm, then y_perm
+        self.h = e(T * k, cfg.I, dtype=dt)
+        self.hs = e(T, max(1, cfg.S * cfg.Is), dtype=dt)
+        self.shared_out = e(T, d, dtype=dt) if cfg.S > 0 else None
+        self.y = e(T, d, dtype=dt)
+        if self.fp8:  # E4M3 expert weights, quantized once per output row before timing
+            self.q8 = moe.quantize_experts_fp8(p)
+            self.w8 = moe.fp8_experts(self.q8)
+            SIs = max(1, cfg.S * cfg.Is)
+            self.xq, self.xsc = e(T, d, dtype=torch.uint8), e(T, dtype=torch.float32)
+            self.xq_perm = e(T * k, d, dtype=torch.uint8)
+            self.hq, self.h_sc = e(T * k, cfg.I, dtype=torch.uint8), e(T * k, dtype=torch.float32)
+            self.hsq, self.hs_sc = e(T, SIs, dtype=torch.uint8), e(T, dtype=torch.float32)
+            torch.cuda.synchronize()
+
+    def __call__(self, i, ev=None):
+        moe, cfg, p, st, sh = self.moe, self.cfg, self.p, self.stream, self.sh
+        x = self.xs[i % len(self.xs)]
+        rec = (lambda j: ev[j].record(st)) if ev is not None else (lambda j: None)
+        sh_ = cfg.S > 0
+        T, k = cfg.T, cfg.k
+        rec(0)
+        moe.moe_route(x, p["w_gate"], p["bias"], sh, self.idx, self.w, self.counts, None, st)
+        rec(1)
+        if self.fp8:
+            moe.moe_quantize_fp8(x, T, cfg.d, 1, self.xq, self.xsc, st)
+            rec(2)
+            moe.moe_permute(self.xq, self.idx, self.counts, sh, self.xq_perm, self.offsets, self.perm, self.inv,
+                            self.pws, st)
+            rec(3)
+            moe.moe_ffn_up_fp8(self.xq_perm, self.perm, self.xsc, self.offsets, self.xq if sh_ else None, self.w8, sh,
+                               self.h, self.hs if sh_ else None, st)
+            rec(4)
+            moe.moe_quantize_fp8(self.h, T * k, cfg.I, 1, self.hq, self.h_sc, st)
+            if sh_:
+                moe.moe_quantize_fp8(self.hs, T, cfg.S * cfg.Is, 1, self.hsq, self.hs_sc, st)
+            rec(5)
+            moe.moe_ffn_down_fp8(self.hq, self.h_sc, self.offsets, self.hsq if sh_ else None, self.hs_sc, self.w8,
+                                 sh, self.x_perm, self.shared_out, st)
+            j = 6
+        else:
+            moe.moe_permute(x, self.idx, self.counts, sh, self.x_perm, self.offsets, self.perm, self.inv, self.pws, st)
+            rec(2)
+            moe.moe_ffn_up(self.x_perm, self.offsets, p["w1"], p["w3"], x if sh_ else None, p["ws1"], p["ws3"], sh,
+                           self.h, self.hs, st)
+            rec(3)
+            moe.moe_ffn_down(self.h, self.offsets, p["w2"], self.hs if sh_ else None, p["ws2"], sh, self.x_perm,
+                             self.shared_out, st)
+            j = 4
+        rec(j)
+        moe.moe_combine(self.x_perm, self.w, self.inv, self.shared_out, sh, self.y, st)
+        rec(j + 1)
+        self.mdist.allreduce_counts(self.counts)
+        moe.moe_load_and_bias_update(self.counts, self.sh_global, cfg.step_size, None, p["bias"], None, st)
+        rec(j + 2)
+
+
+def _gpu_id(local):
+    gpu_id = str(local)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        gpu_id = vis.split(",")[local].strip()
+    return gpu_id
+
+
+def timed_steps(step, steps, warmup, world, local, dev, on_step=None):
+    """W untimed steps, then K steps between a barrier + synchronize on both
+    sides, CUDA events on the launching stream (and between the stages);
+    max over ranks.  Returns (ms_total, stage_ms, launches, clocks)."""
+    import torch
+    import torch.distributed as dist
+    import fine_grained_moe_gate_b200 as moe
+    stream = step.stream
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(warmup):
+        step(i)
+    st = moe.moe_get_last_error(stream)
+    if st != 0:
+        raise moe.MoEError(st, f"{step.cfg.name}: warm-up steps")
+    clocks = ClockSampler(_gpu_id(local))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(step.stages) + 1)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    clocks.start()
+    launches0 = moe.moe_kernel_launch_count()
+    start.record(stream)
+    for i in range(steps):
+        step(warmup + i, evs[i])
+        if on_step is not None:
+            on_step(i)
+    end.record(stream)
+    launches = moe.moe_kernel_launch_count() - launches0
+    barrier()
+    clk = clocks.stop()
+    st = moe.moe_get_last_error(stream)
+    if st != 0:
+        raise moe.MoEError(st, f"{step.cfg.name}: timed steps")
+    stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+                for j, name in enumerate(step.stages)}
+    t = torch.tensor([start.elapsed_time(end)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item()), stage_ms, launches, clk
+
+
+def roofline_records(step, stage_ms, peaks, peak_src, dominant_ms=None):
+    """Roofline of the dominant kernel (the gate/up launch, routed + shared
+    sets): tensor FLOP/s against the measured burst bf16 peak (the kernel is
+    timed in a sub-second region; the sustained figure is the seconds-long
+    power-capped one) and the HBM bytes it must move against the measured
+    copy bandwidth.  Returns (primary, alternate, touched experts)."""
+    moe, cfg, p, sh = step.moe, step.cfg, step.p, step.sh
+    T, k, d = cfg.T, cfg.k, cfg.d
+    SIs = cfg.S * cfg.Is
+    flops_per_launch = T * k * 4 * d * cfg.I + T * 4 * d * SIs   # gate + up, real rows only
+    dom_ms = stage_ms[DOMINANT] if dominant_ms is None else dominant_ms
+    achieved = flops_per_launch / (dom_ms / 1e3) / 1e12
+    # algorithmic bytes of that launch: W1 + W3 of the routed experts that got
+    # rows (counted by routing each input once more, outside the timed region)
+    # and of the shared experts, the token rows read and h written
+    touched = []
+    for xx in step.xs[:8]:
+        moe.moe_route(xx, p["w_gate"], p["bias"], sh, step.idx, step.w, step.counts, None, step.stream)
+        touched.append(int((step.counts > 0).sum().item()))
+    n_touched = statistics.mean(touched)
+    esz = {"bf16": 2, "fp8": 1}.get(cfg.dtype, 4)
+    if step.fp8:  # E4M3 weights and token rows in, bf16 h out
+        bytes_per_launch = (n_touched * 2 * cfg.I * d + 2 * SIs * d + T * k * d + T * d) + \
+            (T * k * cfg.I + T * SIs) * 2
+    else:
+        bytes_per_launch = (n_touched * 2 * cfg.I * d + T * k * (d + cfg.I) + 2 * SIs * d + T * (d + SIs)) * esz
+    hbm_gbs = bytes_per_launch / (dom_ms / 1e3) / 1e9
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    traffic = traffic_record(os.path.join(ROOT, "fine_grained_moe_gate_b200", "csrc", "gemm_tc.cu"), cfg.name)
+    roof_hbm = {"bound": "hbm", "kernel": "gate/up projection (routed + shared)", "achieved": round(hbm_gbs, 1),
+                "peak": hbm_peak, "unit": "GB/s", "frac": round(hbm_gbs / hbm_peak, 4),
+                "frac_of_nominal_8000": round(hbm_gbs / 8000.0, 4),
+                "traffic": traffic, "bytes_per_launch": int(bytes_per_launch), "experts_touched": n_touched,
+                "ms_per_launch": round(dom_ms, 4), "peak_kind": f"hbm_gbs ({peak_src}, copy bandwidth)"}
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    if cfg.dtype in ("bf16", "fp8"):
+        mult = 2.0 if step.fp8 else 1.0  # nominal dense E4M3 / bf16 ratio 4.5 / 2.25
+        peak = mult * burst
+        roof = {"bound": "tensor",
+                "kernel": "tc_grouped_gemm_kernel<up%s> (routed + shared experts, SwiGLU epilogue)"
+                          % (", E4M3" if step.fp8 else ""),
+                "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "frac_of_sustained": round(achieved / (mult * sus), 4), "traffic": traffic,
+                "peak_kind": ("%sbf16_tflops (%s, burst): the kernel is timed in a sub-second region"
+                              % ("2 x " if step.fp8 else "", peak_src)),
+                "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
+    else:
+        roof = {"bound": "alu", "kernel": "simt_grouped_gemm_kernel (fp32 FFMA; routed and shared launches)",
+                "achieved": round(achieved, 3), "peak": None, "unit": "TFLOP/s", "frac": None, "traffic": None,
+                "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
+    if cfg.name.startswith("v3_decode"):
+        # a few tokens per expert: the launch streams the touched experts' weights
+        roof, roof_hbm = roof_hbm, roof
+    return roof, roof_hbm, n_touched
+
+
+def layer_weight_bytes(cfg, n_touched):
+    """HBM bytes of the weights one layer step must read: W1, W3, W2 of the
+    touched experts, the shared experts and W_gate (the decode workload's
+    bound)."""
+    esz = {"bf16": 2, "fp8": 1}.get(cfg.dtype, 4)
+    gate = cfg.E * cfg.d * (2 if cfg.dtype == "fp8" else esz)
+    return int((n_touched * 3 * cfg.I * cfg.d + 3 * cfg.S * cfg.Is * cfg.d) * esz + gate)
+
+
+def measure_extra(name, args, world, rank, local, dev, peaks, peak_src, n_steps, n_x):
+    """One more workload of the default line (decode, skew): its own layer
+    and inputs, timed like the main line; returns its record."""
+    import torch
+    from fine_grained_moe_gate_b200 import dist as mdist
+    from fine_grained_moe_gate_b200.inputs import CONFIGS, make_layer, make_tokens
+    cfg = CONFIGS[name]
+    stream = torch.cuda.current_stream()
+    p = make_layer(cfg, dev)
+    xs = [make_tokens(cfg, dev, step=mdist.shard_step(i, rank, world)) for i in range(n_x)]
+    step = LayerStep(cfg, dev, world, p, xs, stream)
+    loads = None
+    if cfg.zipf_s > 0:
+        loads = torch.empty((n_steps, cfg.E), dtype=torch.int32, device=dev)
+        on_step = lambda i: loads[i].copy_(step.counts, non_blocking=True)  # 1 KB device copy per step
+    else:
+        on_step = None
+    ms_total, stage_ms, launches, clk = timed_steps(step, n_steps, max(3, args.warmup), world, local, dev, on_step)
+    roof, roof_alt, n_touched = roofline_records(step, stage_ms, peaks, peak_src)
+    ms = ms_total / n_steps
+    rec = {"value": round(world * cfg.T * n_steps / (ms_total / 1e3), 1), "unit": "tokens/s",
+           "ms_per_step": round(ms, 4), "steps": n_steps, "warmup": max(3, args.warmup),
+           "config": {"workload": cfg.name, "T_per_gpu": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "I": cfg.I,
+                      "S": cfg.S, "Is": cfg.Is, "inputs": f"{n_x} pre-drawn batches, cycled"
+                      + (" (fresh x every call)" if n_x >= n_steps else "")},
+           "roofline": roof, "roofline_alt": roof_alt,
+           "stages_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
+           "gpu_launches": int(launches), "clocks": clk}
+    if cfg.name.startswith("v3_decode"):
+        wb = layer_weight_bytes(cfg, n_touched)
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        gbs = wb / (ms / 1e3) / 1e9
+        rec["layer_hbm"] = {"bytes_per_step": wb, "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                            "frac_of_nominal_8000": round(gbs / 8000.0, 4),
+                            "what": "weights of the touched experts (W1, W3, W2), the shared expert and W_gate "
+                                    "per step / step time, against the measured copy bandwidth"}
+    else:
+        rec["layer_tflops"] = round(cfg.flops() / (ms / 1e3) / 1e12, 2)
+    if loads is not None:
+        c = loads.double()
+        ratio = (c.max(1).values / c.mean(1)).cpu().tolist()
+        rec["load_max_over_mean"] = {"first": round(ratio[0], 3), "last": round(ratio[-1], 3),
+                                     "min": round(min(ratio), 3), "median": round(statistics.median(ratio), 3),
+                                     "max": round(max(ratio), 3),
+                                     "what": "per timed step: the most-loaded expert's rows / mean rows per expert "
+                                             "(counts summed over ranks), bias updated every step"}
+    del step, p, xs
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_ours(args, world, rank, local):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -294,131 +588,23 @@ def run_ours(args, world, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     cfg = workload(args)
     sh = moe.shape_of(cfg)
-    sh_global = moe.shape_of(cfg, T=mdist.global_token_count(cfg.T, world))  # the step's batch, all ranks
     stream = torch.cuda.current_stream()
 
     p = make_layer(cfg, dev)
     fp8 = cfg.dtype == "fp8"
-    stages = STAGES_FP8 if fp8 else STAGES
-    if fp8:  # E4M3 expert weights, quantized once per output row before timing
-        q8 = moe.quantize_experts_fp8(p)
-        w8 = moe.fp8_experts(q8)
-        torch.cuda.synchronize()
     n_x = max(1, min(4, args.steps + args.warmup))
     xs = [make_tokens(cfg, dev, step=mdist.shard_step(i, rank, world)) for i in range(n_x)]
-
+    step = LayerStep(cfg, dev, world, p, xs, stream)
     T, k, d, E = cfg.T, cfg.k, cfg.d, cfg.E
     dt = cfg.torch_dtype
-    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
-    w = torch.empty((T, k), dtype=torch.float32, device=dev)
-    counts = torch.empty(E, dtype=torch.int32, device=dev)
-    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
-    inv = torch.empty(T * k, dtype=torch.int32, device=dev)
-    pws = torch.empty(max(moe.moe_permute_workspace_size(sh), 256), dtype=torch.uint8, device=dev)
-    x_perm = torch.empty((T * k, d), dtype=dt, device=dev)   # x_perm, then y_perm
-    h = torch.empty((T * k, cfg.I), dtype=dt, device=dev)
-    hs = torch.empty((T, max(1, cfg.S * cfg.Is)), dtype=dt, device=dev)
-    shared_out = torch.empty((T, d), dtype=dt, device=dev) if cfg.S > 0 else None
-    y = torch.empty((T, d), dtype=dt, device=dev)
-    if fp8:
-        SIs = max(1, cfg.S * cfg.Is)
-        xq = torch.empty((T, d), dtype=torch.uint8, device=dev)
-        xsc = torch.empty(T, dtype=torch.float32, device=dev)
-        xq_perm = torch.empty((T * k, d), dtype=torch.uint8, device=dev)
-        hq = torch.empty((T * k, cfg.I), dtype=torch.uint8, device=dev)
-        h_sc = torch.empty(T * k, dtype=torch.float32, device=dev)
-        hsq = torch.empty((T, SIs), dtype=torch.uint8, device=dev)
-        hs_sc = torch.empty(T, dtype=torch.float32, device=dev)
-
-    def step_fp8(i, ev=None):
-        x = xs[i % n_x]
-        rec = (lambda j: ev[j].record(stream)) if ev is not None else (lambda j: None)
-        sh_ = cfg.S > 0
-        rec(0)
-        moe.moe_route(x, p["w_gate"], p["bias"], sh, idx, w, counts, None, stream)
-        rec(1)
-        moe.moe_quantize_fp8(x, T, d, 1, xq, xsc, stream)
-        rec(2)
-        moe.moe_permute(xq, idx, counts, sh, xq_perm, offsets, perm, inv, pws, stream)
-        rec(3)
-        moe.moe_ffn_up_fp8(xq_perm, perm, xsc, offsets, xq if sh_ else None, w8, sh, h, hs if sh_ else None, stream)
-        rec(4)
-        moe.moe_quantize_fp8(h, T * k, cfg.I, 1, hq, h_sc, stream)
-        if sh_:
-            moe.moe_quantize_fp8(hs, T, cfg.S * cfg.Is, 1, hsq, hs_sc, stream)
-        rec(5)
-        moe.moe_ffn_down_fp8(hq, h_sc, offsets, hsq if sh_ else None, hs_sc, w8, sh, x_perm, shared_out, stream)
-        rec(6)
-        moe.moe_combine(x_perm, w, inv, shared_out, sh, y, stream)
-        rec(7)
-        mdist.allreduce_counts(counts)
-        moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
-        rec(8)
-
-    def step(i, ev=None):
-        x = xs[i % n_x]
-        rec = (lambda j: ev[j].record(stream)) if ev is not None else (lambda j: None)
-        rec(0)
-        moe.moe_route(x, p["w_gate"], p["bias"], sh, idx, w, counts, None, stream)
-        rec(1)
-        moe.moe_permute(x, idx, counts, sh, x_perm, offsets, perm, inv, pws, stream)
-        rec(2)
-        xs_ = x if cfg.S > 0 else None
-        moe.moe_ffn_up(x_perm, offsets, p["w1"], p["w3"], xs_, p["ws1"], p["ws3"], sh, h, hs, stream)
-        rec(3)
-        moe.moe_ffn_down(h, offsets, p["w2"], hs if cfg.S > 0 else None, p["ws2"], sh, x_perm, shared_out, stream)
-        rec(4)
-        moe.moe_combine(x_perm, w, inv, shared_out, sh, y, stream)
-        rec(5)
-        mdist.allreduce_counts(counts)
-        moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
-        rec(6)
-
-    if fp8:
-        step = step_fp8
+    ms_total, stage_ms, launches, clk = timed_steps(step, args.steps, args.warmup, world, local, dev)
+    ms_per_step = ms_total / args.steps
+    tokens_per_s = world * T * args.steps / (ms_total / 1e3)
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-
-    for i in range(args.warmup):
-        step(i)
-    st = moe.moe_get_last_error(stream)
-    if st != 0:
-        raise moe.MoEError(st, "warm-up steps")
-
-    gpu_id = str(local)
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    if vis:
-        gpu_id = vis.split(",")[local].strip()
-    clocks = ClockSampler(gpu_id)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    clocks.start()
-    launches0 = moe.moe_kernel_launch_count()
-    start.record(stream)
-    for i in range(args.steps):
-        step(args.warmup + i, evs[i])
-    end.record(stream)
-    launches = moe.moe_kernel_launch_count() - launches0
-    barrier()
-    clk = clocks.stop()
-    st = moe.moe_get_last_error(stream)
-    if st != 0:
-        raise moe.MoEError(st, "timed steps")
-    ms_local = start.elapsed_time(end)
-    stage_ms = {}
-    for j, name in enumerate(stages):
-        stage_ms[name] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
-    t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
-    ms_per_step = ms_total / args.steps
-    tokens_per_s = world * T * args.steps / (ms_total / 1e3)
 
     # ---- e2e: public call, host buffers, copies inside the timed region
     e2e = None
@@ -437,6 +623,7 @@ def run_ours(args, world, rank, local):
         ev_in = [torch.cuda.Event() for _ in range(nb)]     # x_dev[b] holds the step's tokens
         ev_done = [torch.cuda.Event() for _ in range(nb)]   # the step using buffer b has computed
         ev_out = [torch.cuda.Event() for _ in range(nb)]    # y_dev[b] has reached the host
+        idx, w, counts = step.idx, step.w, step.counts
 
         def issue_h2d(i):
             bb = i % nb
@@ -450,13 +637,13 @@ def run_ours(args, world, rank, local):
             stream.wait_event(ev_in[bb])
             stream.wait_event(ev_out[bb])                   # y_dev[bb] is no longer being copied out
             if fp8:
-                moe.moe_layer_forward_fp8(x_dev[bb], p["w_gate"], p["bias"], w8, sh, y_dev[bb], idx, w, counts, ws,
-                                          stream)
+                moe.moe_layer_forward_fp8(x_dev[bb], p["w_gate"], p["bias"], step.w8, sh, y_dev[bb], idx, w, counts,
+                                          ws, stream)
             else:
                 moe.moe_layer_forward(x_dev[bb], p["w_gate"], p["bias"], p["w1"], p["w3"], p["w2"], p["ws1"],
                                       p["ws3"], p["ws2"], sh, y_dev[bb], idx, w, counts, ws, stream)
             mdist.allreduce_counts(counts)
-            moe.moe_load_and_bias_update(counts, sh_global, cfg.step_size, None, p["bias"], None, stream)
+            moe.moe_load_and_bias_update(counts, step.sh_global, cfg.step_size, None, p["bias"], None, stream)
             ev_done[bb].record(stream)
             if not last:
                 issue_h2d(i + 1)
@@ -493,65 +680,32 @@ def run_ours(args, world, rank, local):
         st = moe.moe_get_last_error(stream)
         if st != 0:
             raise moe.MoEError(st, "e2e steps")
+        del ws, x_dev, y_dev, x_host, y_host
 
-    # ---- roofline of the dominant kernel (gate/up grouped GEMM, routed + shared sets)
     peaks, peak_src = load_peaks()
-    SIs = cfg.S * cfg.Is
-    flops_per_launch = T * k * 4 * d * cfg.I + T * 4 * d * SIs   # gate + up, real rows only
-    dom_ms = stage_ms[DOMINANT]
-    achieved = flops_per_launch / (dom_ms / 1e3) / 1e12
-    # algorithmic bytes of that launch: W1 + W3 of the routed experts that got
-    # rows (counted by routing each input once more, outside the timed region)
-    # and of the shared experts, the token rows read and h written
-    touched = []
-    for xx in xs:
-        moe.moe_route(xx, p["w_gate"], p["bias"], sh, idx, w, counts, None, stream)
-        touched.append(int((counts > 0).sum().item()))
-    n_touched = statistics.mean(touched)
+    roof, roof_hbm, n_touched = roofline_records(step, stage_ms, peaks, peak_src)
     esz = {"bf16": 2, "fp8": 1}.get(cfg.dtype, 4)
-    if fp8:  # E4M3 weights and token rows in, bf16 h out
-        bytes_per_launch = (n_touched * 2 * cfg.I * d + 2 * SIs * d + T * k * d + T * d) + \
-            (T * k * cfg.I + T * SIs) * 2
-    else:
-        bytes_per_launch = (n_touched * 2 * cfg.I * d + T * k * (d + cfg.I) + 2 * SIs * d + T * (d + SIs)) * esz
-    hbm_gbs = bytes_per_launch / (dom_ms / 1e3) / 1e9
-    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    traffic = traffic_record(os.path.join(ROOT, "fine_grained_moe_gate_b200", "csrc", "gemm_tc.cu"), cfg.name)
-    roof_hbm = {"bound": "hbm", "kernel": "gate/up projection (routed + shared)", "achieved": round(hbm_gbs, 1), "peak": hbm_peak,
-                "unit": "GB/s", "frac": round(hbm_gbs / hbm_peak, 4),
-                "frac_of_nominal_8000": round(hbm_gbs / 8000.0, 4),
-                "traffic": traffic, "bytes_per_launch": int(bytes_per_launch), "experts_touched": n_touched,
-                "peak_kind": f"hbm_gbs ({peak_src}, copy bandwidth)"}
-    bf16_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    if cfg.dtype == "bf16":
-        peak = bf16_sus
-        roof = {"bound": "tensor", "kernel": "tc_grouped_gemm_kernel<up> (routed + shared experts, SwiGLU epilogue)",
-                "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": traffic,
-                "peak_kind": f"bf16_tflops_sustained ({peak_src}): the kernel is timed inside a long step",
-                "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
-    elif fp8:
-        peak = 2.0 * bf16_sus  # nominal dense E4M3 / bf16 ratio 4.5 / 2.25 times the measured bf16 figure
-        roof = {"bound": "tensor", "kernel": "tc_grouped_gemm_kernel<up, E4M3> (routed + shared experts)",
-                "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": traffic,
-                "peak_kind": f"2 x bf16_tflops_sustained ({peak_src}; nominal fp8/bf16 dense ratio 4.5/2.25)",
-                "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
-    else:
-        roof = {"bound": "alu", "kernel": "simt_grouped_gemm_kernel (fp32 FFMA; routed and shared launches)", "achieved": round(achieved, 3),
-                "peak": None, "unit": "TFLOP/s", "frac": None, "traffic": None,
-                "flops_per_launch": flops_per_launch, "ms_per_launch": round(dom_ms, 4)}
-    if cfg.name.startswith("v3_decode"):
-        # a few tokens per expert: the launch streams the touched experts' weights
-        roof, roof_hbm = roof_hbm, roof
     layer_flops = cfg.flops()
     step_tflops = layer_flops / (ms_per_step / 1e3) / 1e12
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    weights_gb = (p["w1"].numel() * 3 + p["ws1"].numel() * 3) * esz / 1e9
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         n_tok = args.cpu_tokens or DEFAULT_CPU_TOKENS[args.workload]
         secs, n, threads = run_oracle_sample(cfg, p, xs[0], min(n_tok, T))
         cpu = cpu_baseline_record(cfg, secs, n, threads, "oracle sample")
+
+    # ---- the other workloads of the default line (decode-shaped, skewed routing)
+    extras = {}
+    if not args.no_extra and args.workload == "v3_prefill" and not (args.T or args.E):
+        del step, xs
+        p.clear()
+        torch.cuda.empty_cache()
+        extras["v3_decode"] = measure_extra("v3_decode", args, world, rank, local, dev, peaks, peak_src,
+                                            args.decode_calls, args.decode_calls)
+        extras["skew_stress"] = measure_extra("skew_stress", args, world, rank, local, dev, peaks, peak_src,
+                                              args.skew_steps, 8)
 
     if rank == 0:
         line = {
@@ -562,14 +716,14 @@ def run_ours(args, world, rank, local):
                     + ("; expert weights quantized to E4M3 per output row before timing)" if fp8 else ")"),
             "config": {"workload": cfg.name, "T_per_gpu": T, "global_batch": T * world, "d": d, "E": E, "k": k,
                        "I": cfg.I, "S": cfg.S, "Is": cfg.Is, "parallelism": f"dp{world}",
-                       "l2": "inputs larger than L2: layer weights read every step "
-                             f"({(p['w1'].numel() * 3 + p['ws1'].numel() * 3) * esz / 1e9:.1f} GB)",
+                       "l2": f"inputs larger than L2: layer weights read every step ({weights_gb:.1f} GB)",
                        "bias_update": "every step"},
             "roofline": roof,
             "roofline_alt": roof_hbm,
             "layer_tflops": round(step_tflops, 2),
-            "layer_frac_of_peak": round(step_tflops / (bf16_sus * (2.0 if fp8 else 1.0)), 4)
+            "layer_frac_of_peak": round(step_tflops / (burst * (2.0 if fp8 else 1.0)), 4)
             if cfg.dtype in ("bf16", "fp8") else None,
+            "layer_peak_kind": "bf16_tflops burst (x2 for E4M3)",
             "stages_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -577,6 +731,8 @@ def run_ours(args, world, rank, local):
             "clocks": clk,
             "impl": "ours",
         }
+        if extras:
+            line["workloads"] = extras
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -107,7 +107,7 @@ def lib() -> ctypes.CDLL:
             "moe_ffn_up_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_ffn_down_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_layer_forward_fp8": [P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P, P, P, sz, P],
-            "moe_ep_plan": [P, ctypes.c_int32, ctypes.c_int32, S, P, P, P],
+            "moe_ep_plan": [P, ctypes.c_int32, ctypes.c_int32, S, ctypes.c_int64, P, P, P],
             "moe_ep_dispatch": [P, P, P, ctypes.c_int32, ctypes.c_int32, S, P, P],
             "moe_ep_return": [P, P, ctypes.c_int32, ctypes.c_int32, S, P, P],
             "moe_selftest_bounded_wait": [ctypes.c_uint32, P],
@@ -333,8 +333,9 @@ def moe_ep_plan_size(world, shape) -> int:
     return lib().moe_ep_plan_size(world, shape)
 
 
-def moe_ep_plan(counts_all, world, rank, shape, plan, recv_offsets, stream=None):
-    _check(lib().moe_ep_plan(_p(counts_all), world, rank, shape, _p(plan), _p(recv_offsets), _stream(stream)),
+def moe_ep_plan(counts_all, world, rank, shape, recv_capacity, plan, recv_offsets, stream=None):
+    _check(lib().moe_ep_plan(_p(counts_all), world, rank, shape, recv_capacity, _p(plan), _p(recv_offsets),
+                             _stream(stream)),
            "moe_ep_plan")
 
 

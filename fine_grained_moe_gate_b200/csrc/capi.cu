@@ -766,20 +766,22 @@ size_t moe_ep_plan_size(int32_t world, moe_shape sh) {
     return align256(moe::ep_plan_ints(world, sh.E) * sizeof(int32_t));
 }
 
-moe_status moe_ep_plan(const int32_t* counts_all, int32_t world, int32_t rank, moe_shape sh, int32_t* plan,
-                       int32_t* recv_offsets, void* stream) {
+moe_status moe_ep_plan(const int32_t* counts_all, int32_t world, int32_t rank, moe_shape sh, int64_t recv_capacity,
+                       int32_t* plan, int32_t* recv_offsets, void* stream) {
     moe_status v = validate_shape(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(world >= 1 && world <= moe::kMaxRanks && sh.E % world == 0 && rank >= 0 && rank < world,
                 MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(counts_all && plan, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(recv_capacity > 0 && recv_capacity <= 0x7fffffffLL, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(aligned16(counts_all) && aligned16(plan) && aligned16(recv_offsets), MOE_ERR_ALIGNMENT);
     int dev, sms;
     int* status;
     v = device_setup(&dev, &status, &sms);
     if (v != MOE_OK) return v;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (moe::launch_ep_plan(counts_all, world, sh.E, plan, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe::launch_ep_plan(counts_all, world, sh.E, (long long)recv_capacity, plan, status, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
     if (recv_offsets) {
         const int Epr = sh.E / world;
         const size_t at = (size_t)sh.E * world + (size_t)world * (sh.E + 1) + (size_t)rank * (Epr + 1);

@@ -24,13 +24,15 @@
 namespace moe {
 namespace {
 
-__global__ void ep_plan_kernel(const int32_t* __restrict__ C, int W, int E, int32_t* __restrict__ plan) {
+__global__ void ep_plan_kernel(const int32_t* __restrict__ C, int W, int E, long long cap, int32_t* __restrict__ plan,
+                               int* status) {
     // one thread: E * W <= 16K additions
     if (threadIdx.x != 0 || blockIdx.x != 0) return;
     const int Epr = E / W;
     int32_t* base = plan;
     int32_t* src_off = plan + E * W;
     int32_t* recv_off = src_off + W * (E + 1);
+    int32_t* tail = recv_off + W * (Epr + 1);  // [receive capacity (rows, clamped to int32), overflow flag]
     for (int s = 0; s < W; ++s) {
         int acc = 0;
         for (int e = 0; e < E; ++e) {
@@ -39,18 +41,23 @@ __global__ void ep_plan_kernel(const int32_t* __restrict__ C, int W, int E, int3
         }
         src_off[s * (E + 1) + E] = acc;
     }
+    int overflow = 0;
     for (int o = 0; o < W; ++o) {
-        int row = 0;
+        long long row = 0;
         for (int i = 0; i < Epr; ++i) {
             const int e = o * Epr + i;
-            recv_off[o * (Epr + 1) + i] = row;
+            recv_off[o * (Epr + 1) + i] = (int)row;
             for (int s = 0; s < W; ++s) {
-                base[e * W + s] = row;
+                base[e * W + s] = (int)row;
                 row += C[s * E + e];
             }
         }
-        recv_off[o * (Epr + 1) + Epr] = row;
+        recv_off[o * (Epr + 1) + Epr] = (int)row;
+        if (row > cap) overflow = 1;  // some owner would receive more rows than its buffer holds
     }
+    tail[0] = (int)(cap < 0x7fffffffLL ? cap : 0x7fffffffLL);
+    tail[1] = overflow;
+    if (overflow) report(status, kStDeviceCheck);
 }
 
 // last index i in [0, n) with a[i] <= v (a non-decreasing, a[0] <= v)
@@ -72,8 +79,11 @@ __device__ __forceinline__ void copy_row(const uint4* __restrict__ src, uint4* d
 __global__ void __launch_bounds__(kWarps * 32)
     ep_dispatch_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_tok,
                        const int32_t* __restrict__ plan, int W, int E, int k, int rank, int vec, int T,
-                       long long cap_recv, EpPeers recv, int* status) {
+                       EpPeers recv, int* status) {
     const int32_t* base = plan;
+    const int32_t* tail = plan + E * W + W * (E + 1) + W * (E / W + 1);
+    if (tail[1]) return;  // the plan found a receive buffer too small: nothing is sent (status already set)
+    const long long cap_recv = tail[0];
     const int32_t* off = plan + E * W + rank * (E + 1);  // this rank's permutation offsets
     const int rows = min(off[E], T * k);  // this rank's rows (the plan must agree with the permutation)
     const int Epr = E / W;
@@ -94,8 +104,11 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 __global__ void __launch_bounds__(kWarps * 32)
     ep_return_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ plan, int W, int E, int rank, int vec,
-                     long long cap_recv, int cap_back, EpPeers back, int* status) {
+                     int cap_back, EpPeers back, int* status) {
     const int Epr = E / W;
+    const int32_t* tail = plan + E * W + W * (E + 1) + W * (Epr + 1);
+    if (tail[1]) return;
+    const long long cap_recv = tail[0];
     const int32_t* base = plan;
     const int32_t* src_off = plan + E * W;
     const int32_t* roff = src_off + W * (E + 1) + rank * (Epr + 1);
@@ -116,10 +129,11 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 }  // namespace
 
-size_t ep_plan_ints(int W, int E) { return (size_t)E * W + (size_t)W * (E + 1) + (size_t)W * (E / W + 1); }
+size_t ep_plan_ints(int W, int E) { return (size_t)E * W + (size_t)W * (E + 1) + (size_t)W * (E / W + 1) + 2; }
 
-cudaError_t launch_ep_plan(const int32_t* counts_all, int W, int E, int32_t* plan, cudaStream_t st) {
-    ep_plan_kernel<<<1, 32, 0, st>>>(counts_all, W, E, plan);
+cudaError_t launch_ep_plan(const int32_t* counts_all, int W, int E, long long recv_capacity, int32_t* plan,
+                           int* status, cudaStream_t st) {
+    ep_plan_kernel<<<1, 32, 0, st>>>(counts_all, W, E, recv_capacity, plan, status);
     note_launches(1);
     return cudaGetLastError();
 }
@@ -127,9 +141,8 @@ cudaError_t launch_ep_plan(const int32_t* counts_all, int W, int E, int32_t* pla
 cudaError_t launch_ep_dispatch(const void* x, const int32_t* perm_tok, const int32_t* plan, int W, int E, int k,
                                int rank, int T, size_t row_bytes, const EpPeers& recv, int num_sms, int* status,
                                cudaStream_t st) {
-    const long long cap_recv = (long long)W * T * k;  // every rank's receive buffer holds W*T*k rows
     ep_dispatch_kernel<<<num_sms * 4, kWarps * 32, 0, st>>>(static_cast<const uint4*>(x), perm_tok, plan, W, E, k,
-                                                            rank, (int)(row_bytes / 16), T, cap_recv, recv, status);
+                                                            rank, (int)(row_bytes / 16), T, recv, status);
     note_launches(1);
     return cudaGetLastError();
 }
@@ -137,8 +150,7 @@ cudaError_t launch_ep_dispatch(const void* x, const int32_t* perm_tok, const int
 cudaError_t launch_ep_return(const void* y, const int32_t* plan, int W, int E, int k, int rank, int T,
                              size_t row_bytes, const EpPeers& back, int num_sms, int* status, cudaStream_t st) {
     ep_return_kernel<<<num_sms * 4, kWarps * 32, 0, st>>>(static_cast<const uint4*>(y), plan, W, E, rank,
-                                                          (int)(row_bytes / 16), (long long)W * T * k, T * k, back,
-                                                          status);
+                                                          (int)(row_bytes / 16), T * k, back, status);
     note_launches(1);
     return cudaGetLastError();
 }

@@ -133,7 +133,8 @@ struct EpPeers {
     void* p[kMaxRanks];  // per rank: a device pointer valid in this process (peer memory)
 };
 size_t ep_plan_ints(int W, int E);
-cudaError_t launch_ep_plan(const int32_t* counts_all, int W, int E, int32_t* plan, cudaStream_t st);
+cudaError_t launch_ep_plan(const int32_t* counts_all, int W, int E, long long recv_capacity, int32_t* plan,
+                           int* status, cudaStream_t st);
 // Every rank holds T tokens: receive buffers W*T*k rows, return buffers T*k.
 cudaError_t launch_ep_dispatch(const void* x, const int32_t* perm_tok, const int32_t* plan, int W, int E, int k,
                                int rank, int T, size_t row_bytes, const EpPeers& recv, int num_sms, int* status,

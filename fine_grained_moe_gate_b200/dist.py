@@ -11,6 +11,8 @@ the biases stay bit-identical without ever being sent.
 """
 from __future__ import annotations
 
+import math
+
 import torch
 
 
@@ -91,34 +93,40 @@ def local_experts(p: dict, rank: int, world: int) -> dict:
     return {"w1": p["w1"][e0:e1], "w3": p["w3"][e0:e1], "w2": p["w2"][e0:e1]}
 
 
+def ep_capacity(cfg, world: int, factor: float | None = None) -> int:
+    """Rows of every rank's receive buffer.  None: W*T*k, the most that can
+    ever arrive (every rank sending all its rows to one owner).  A factor f
+    gives ceil(f*T*k) (at most W*T*k): with the bias keeping the load near
+    k/E per expert an owner receives about T*k rows per step, so f = 2 leaves
+    room for a 2x imbalance; a step that would need more is refused on the
+    device (moe_ep_plan) instead of dropping rows."""
+    full = world * cfg.T * cfg.k
+    if factor is None:
+        return full
+    return max(1, min(full, int(math.ceil(factor * cfg.T * cfg.k))))
+
+
 class EPBuffers:
     """One rank's per-step device buffers for ep_forward_steps.  `recv` and
     `back` are the buffers peers store into: allocate them where peers can
-    reach them (symmetric memory across GPUs; any allocation on one GPU)."""
+    reach them (symmetric memory across GPUs; any allocation on one GPU).
+    `capacity` rows (ep_capacity) size the receive buffer and the
+    intermediate h of the received rows; the expert outputs overwrite the
+    received rows in place (they are read by the up projection only, which
+    runs first, and the next step's stores come after this step's return)."""
 
-    def __init__(self, cfg, world: int, device, recv=None, back=None):
+    def __init__(self, cfg, world: int, device, recv=None, back=None, capacity: int | None = None):
         T, k, d, E, I = cfg.T, cfg.k, cfg.d, cfg.E, cfg.I
         dt = cfg.torch_dtype
-        cap = world * T * k                          # receive capacity: every rank sends all its rows here
+        cap = ep_capacity(cfg, world) if capacity is None else int(capacity)
+        self.capacity = cap
         i32 = torch.int32
         self.recv = recv if recv is not None else torch.empty((cap, d), dtype=dt, device=device)
+        if self.recv.shape[0] < cap:
+            raise ValueError(f"receive buffer holds {self.recv.shape[0]} rows, capacity {cap}")
         self.back = back if back is not None else torch.empty((T * k, d), dtype=dt, device=device)
         self.h_recv = torch.empty((cap, I), dtype=dt, device=device)
-        self.y_recv = torch.empty((cap, d), dtype=dt, device=device)
-        self.idx = torch.empty((T, k), dtype=i32, device=device)
-        self.w = torch.empty((T, k), dtype=torch.float32, device=device)
-        self.counts = torch.empty(E, dtype=i32, device=device)
-        self.offsets = torch.empty(E + 1, dtype=i32, device=device)
-        self.perm = torch.empty(T * k, dtype=i32, device=device)
-        self.inv = torch.empty(T * k, dtype=i32, device=device)
-        self.recv_offsets = torch.empty(E // world + 1, dtype=i32, device=device)
-        self.hs = torch.empty((T, max(1, cfg.S * cfg.Is)), dtype=dt, device=device)
-        self.shared_out = torch.empty((T, d), dtype=dt, device=device) if cfg.S > 0 else None
-        self.y = torch.empty((T, d), dtype=dt, device=device)
-        self.flag = torch.zeros(1, dtype=torch.float32, device=device)
-        self._pws = None
-        self._plan = None
-
+        self.y_recv = self.recv
     def scratch(self, moe, sh, world):
         if self._pws is None:
             self._pws = torch.empty(max(moe.moe_permute_workspace_size(sh), 256), dtype=torch.uint8,
@@ -142,13 +150,13 @@ def ep_forward_steps(moe, cfg, rank: int, world: int, x, p: dict, bufs: EPBuffer
     sh = shape_of(cfg)
     Epr = cfg.E // world
     # the GEMMs on the receive buffer: this rank's experts, rows by offsets,
-    # capacity W*T*k rows (k = 1 so that the local expert count may be < k)
-    sh_local = MoEShape(world * cfg.T * cfg.k, cfg.d, Epr, 1, cfg.I, 0, cfg.Is, sh.dtype)
+    # bufs.capacity rows (k = 1 so that the local expert count may be < k)
+    sh_local = MoEShape(bufs.capacity, cfg.d, Epr, 1, cfg.I, 0, cfg.Is, sh.dtype)
     pws, plan = bufs.scratch(moe, sh, world)
     moe.moe_route(x, p["w_gate"], p["bias"], sh, bufs.idx, bufs.w, bufs.counts, None, stream)
     counts_all = yield ("counts", bufs.counts)
     moe.moe_permute(x, bufs.idx, bufs.counts, sh, None, bufs.offsets, bufs.perm, bufs.inv, pws, stream)
-    moe.moe_ep_plan(counts_all, world, rank, sh, plan, bufs.recv_offsets, stream)
+    moe.moe_ep_plan(counts_all, world, rank, sh, bufs.capacity, plan, bufs.recv_offsets, stream)
     moe.moe_ep_dispatch(x, bufs.perm, plan, world, rank, sh, recv_ptrs, stream)
     yield ("barrier",)
     moe.moe_ffn_up(bufs.recv, bufs.recv_offsets, p["w1"], p["w3"], None, None, None, sh_local, bufs.h_recv, None,
@@ -182,14 +190,16 @@ def ep_forward(moe, cfg, rank: int, world: int, x, p: dict, bufs: EPBuffers, rec
             return stop.value
 
 
-def ep_symmetric_buffers(cfg, world: int, device, group_name: str):
+def ep_symmetric_buffers(cfg, world: int, device, group_name: str, capacity: int | None = None):
     """Receive and return buffers in symmetric memory, with every rank's
     device pointers (torch.distributed._symmetric_memory; NVLink peers).
-    Returns (recv, back, recv_ptrs, back_ptrs).  Not run on more than one GPU
-    in this build."""
+    capacity: receive rows (ep_capacity; default W*T*k).  Returns (recv,
+    back, recv_ptrs, back_ptrs).  Not run on more than one GPU in this
+    build."""
     import torch.distributed._symmetric_memory as symm_mem
     T, k, d = cfg.T, cfg.k, cfg.d
-    recv = symm_mem.empty((world * T * k, d), dtype=cfg.torch_dtype, device=device)
+    cap = ep_capacity(cfg, world) if capacity is None else int(capacity)
+    recv = symm_mem.empty((cap, d), dtype=cfg.torch_dtype, device=device)
     back = symm_mem.empty((T * k, d), dtype=cfg.torch_dtype, device=device)
     hr = symm_mem.rendezvous(recv, group_name)
     hb = symm_mem.rendezvous(back, group_name)

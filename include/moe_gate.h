@@ -371,14 +371,20 @@ MOE_API moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, cons
  * A receive buffer holds its experts in order, each expert's rows by source
  * rank, each source's rows by token: the rows, and so the results, of the
  * single-GPU layer over the ranks' concatenated batch (same routing).
- * Receive buffers need W*T*k rows of capacity at most; return buffers T*k.
+ * recv_capacity: rows every rank's receive buffer holds (the same on all
+ * ranks).  W*T*k can never overflow; with the load balanced by the bias a
+ * small multiple of T*k is enough.  If the step's counts would send more
+ * rows to some owner than that, the plan records it and reports
+ * MOE_ERR_DEVICE_CHECK, and moe_ep_dispatch / moe_ep_return with that plan
+ * store nothing (no row is dropped silently).  Return buffers hold T*k rows.
  * recv_bufs / back_bufs: host arrays of W device pointers valid in the
  * calling process (peer memory, e.g. IPC or symmetric memory; on one GPU
  * plain allocations).  bf16 and fp32 rows; MOE_FP8_E4M3 is unsupported.
  * -------------------------------------------------------------------------*/
 MOE_API size_t moe_ep_plan_size(int32_t world, moe_shape sh);  /* bytes; 0 if invalid */
-MOE_API moe_status moe_ep_plan(const int32_t* counts_all, int32_t world, int32_t rank, moe_shape sh, int32_t* plan,
-                               int32_t* recv_offsets, void* stream);  /* recv_offsets [E/W+1]: this rank's */
+MOE_API moe_status moe_ep_plan(const int32_t* counts_all, int32_t world, int32_t rank, moe_shape sh,
+                               int64_t recv_capacity, int32_t* plan, int32_t* recv_offsets,
+                               void* stream);  /* recv_offsets [E/W+1]: this rank's */
 MOE_API moe_status moe_ep_dispatch(const void* x, const int32_t* perm_tok, const int32_t* plan, int32_t world,
                                    int32_t rank, moe_shape sh, void* const* recv_bufs, void* stream);
 MOE_API moe_status moe_ep_return(const void* y_recv, const int32_t* plan, int32_t world, int32_t rank,

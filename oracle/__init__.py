@@ -61,6 +61,8 @@ def _load():
         lib.orc_permute.restype = i
         lib.orc_expert_accumulate.argtypes = [P, i, P, P, P, P, P, i, i, i, P]
         lib.orc_finalize.argtypes = [P, ctypes.c_size_t, i, P]
+        lib.orc_expert_up.argtypes = [P, i, P, P, i, i, i, P]
+        lib.orc_expert_down.argtypes = [P, i, P, i, i, i, P]
         lib.orc_layer_output.argtypes = [P, P, P, P, P, P, P, P, P, i, i, i, i, i, i, i, i, P]
         lib.orc_e4m3_encode_array.argtypes = [P, ctypes.c_size_t, P]
         lib.orc_e4m3_decode_array.argtypes = [P, ctypes.c_size_t, P]
@@ -158,6 +160,31 @@ def expert_accumulate(x_rows, dest, wts, w1, w3, w2, yacc):
     assert yacc.dtype == np.float64 and yacc.flags.c_contiguous
     _load().orc_expert_accumulate(_ptr(x_rows), n, _ptr(dest), _ptr(wts), _ptr(w1), _ptr(w3), _ptr(w2),
                                   d, I, dt, _ptr(yacc))
+
+
+def expert_up(x_rows, w1, w3) -> np.ndarray:
+    """h [n][I] = round(silu(x W1^T) * (x W3^T)), the dot products in double,
+    rounded once to x's dtype (float32, or bf16 bits as uint16)."""
+    x_rows, w1, w3 = _c(x_rows), _c(w1), _c(w3)
+    dt = _dtype_code(x_rows)
+    assert _dtype_code(w1) == dt and _dtype_code(w3) == dt
+    n, d = x_rows.shape
+    I = w1.shape[0]
+    h = np.empty((n, I), x_rows.dtype)
+    _load().orc_expert_up(_ptr(x_rows), n, _ptr(w1), _ptr(w3), d, I, dt, _ptr(h))
+    return h
+
+
+def expert_down(h_rows, w2) -> np.ndarray:
+    """o [n][d] = h W2^T in double (not rounded); h [n][K], W2 [d][K]."""
+    h_rows, w2 = _c(h_rows), _c(w2)
+    dt = _dtype_code(h_rows)
+    assert _dtype_code(w2) == dt
+    n, K = h_rows.shape
+    d = w2.shape[0]
+    o = np.empty((n, d), np.float64)
+    _load().orc_expert_down(_ptr(h_rows), n, _ptr(w2), d, K, dt, _ptr(o))
+    return o
 
 
 def finalize(yacc: np.ndarray, like_dtype) -> np.ndarray:

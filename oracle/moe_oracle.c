@@ -237,6 +237,32 @@ void orc_expert_accumulate(const void* x_rows, int n, const int32_t* dest, const
     }
 }
 
+/* The two halves of one expert's SwiGLU MLP, for checking the grouped GEMMs
+ * one projection at a time [P2 DeepSeekMoE sketch: each expert an MLP over
+ * the tokens routed to it; SwiGLU without biases].  The arithmetic is that of
+ * orc_expert_accumulate, split at h.
+ * orc_expert_up:   h[r][c] = round_dtype( silu(a) * g ),
+ *                  a = sum_i W1[c][i] x[r][i], g = sum_i W3[c][i] x[r][i] (double)
+ *                  x_rows [n][d], W1/W3 [I][d], h [n][I] in dtype.
+ * orc_expert_down: o[r][j] = sum_c W2[j][c] h[r][c]  (double, not rounded)
+ *                  h_rows [n][K], W2 [d][K] in dtype, o [n][d] double. */
+void orc_expert_up(const void* x_rows, int n, const void* w1, const void* w3, int d, int I, int dtype, void* h_out) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int c = 0; c < I; ++c) {
+        for (int r = 0; r < n; ++r) {
+            double a = dot_rows(w1, (size_t)c * d, x_rows, (size_t)r * d, dtype, d);
+            double g = dot_rows(w3, (size_t)c * d, x_rows, (size_t)r * d, dtype, d);
+            store_elem(h_out, dtype, (size_t)r * I + c, round_to_dtype(a / (1.0 + exp(-a)) * g, dtype));
+        }
+    }
+}
+
+void orc_expert_down(const void* h_rows, int n, const void* w2, int d, int K, int dtype, double* o_out) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int j = 0; j < d; ++j)
+        for (int r = 0; r < n; ++r) o_out[(size_t)r * d + j] = dot_rows(w2, (size_t)j * K, h_rows, (size_t)r * K, dtype, K);
+}
+
 /* Round the double accumulator to the output dtype once
  * [P2 DeepSeekMoE sketch: shared_out + routed_out]. */
 void orc_finalize(const double* yacc, size_t n, int dtype, void* y_out) {

@@ -155,3 +155,65 @@ def setup(cfg: MoEConfig, step: int = 0):
     p = make_layer(cfg, DEV)
     x = make_tokens(cfg, DEV, step)
     return moe.shape_of(cfg), p, x
+
+
+def oracle_terms(p, x, idx, w, tokens, S):
+    """The oracle's layer output for the given token rows, kept in double,
+    and the magnitude of the terms it sums: y = shared + sum_j w_j o_j and
+    M = |shared| + sum_j w_j |o_j| (DeepSeekMoE sketch: shared_out +
+    routed_out).  Each expert's two projections come from the oracle's
+    expert_up / expert_down, one expert's weights at a time."""
+    tokens = np.asarray(tokens)
+    n = len(tokens)
+    d = x.shape[1]
+    xs = to_numpy(x[torch.as_tensor(tokens, device=x.device)])
+    sh = np.zeros((n, d), np.float64)
+    for s in range(S):
+        h = oracle.expert_up(xs, to_numpy(p["ws1"][s]), to_numpy(p["ws3"][s]))
+        sh += oracle.expert_down(h, to_numpy(p["ws2"][s]))
+    y = sh.copy()
+    mag = np.abs(sh)
+    idx_np = idx.cpu().numpy()[tokens]
+    w_np = w.cpu().numpy()[tokens]
+    for e in np.unique(idx_np):
+        ii, jj = np.nonzero(idx_np == e)
+        o = oracle.expert_down(oracle.expert_up(xs[ii], to_numpy(p["w1"][e]), to_numpy(p["w3"][e])),
+                               to_numpy(p["w2"][e]))
+        wt = w_np[ii, jj].astype(np.float64)[:, None]
+        np.add.at(y, ii, wt * o)
+        np.add.at(mag, ii, wt * np.abs(o))
+    return y, mag
+
+
+def check_layer_elementwise(y_gpu: torch.Tensor, y_ref_f64: np.ndarray, mag: np.ndarray):
+    """bf16 layer output, element by element.  The GPU rounds each expert
+    output (y_perm) and the shared output to bf16 before the weighted sum
+    (each within 2^-8 of its value) and rounds y once more; the oracle rounds
+    y once.  So |y_gpu - y_ref| <= 2^-8 (M + 2|y|) <= 2^-7 (|y_ref| + M), M the
+    terms' magnitude from ``oracle_terms``."""
+    got = as_f64(y_gpu)
+    ref = to_f64_rows(oracle.finalize(y_ref_f64, np.uint16))
+    bound = 2.0 ** -7 * (np.abs(ref) + mag) + 1e-6
+    bad = np.abs(got - ref) > bound
+    if bad.any():
+        r, c = np.argwhere(bad)[0]
+        raise AssertionError(f"{int(bad.sum())} elements beyond the bf16 bound, first at row {r} col {c}: "
+                             f"got {got[r, c]}, oracle {ref[r, c]}, bound {bound[r, c]}")
+    return rel_fro(got, ref)
+
+
+def check_bf16_close(got: np.ndarray, ref: np.ndarray, what: str):
+    """A bf16 result rounded once from an fp32 tensor-core accumulation,
+    against the oracle's double result rounded once (or not at all): the two
+    may fall on either side of a bf16 rounding boundary (one ulp, <= 2^-7
+    |ref|), and the fp32 accumulation of K products adds far less than 2^-10
+    of the rows' RMS at these sizes."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    bound = 2.0 ** -7 * np.abs(ref) + 2.0 ** -10 * rms + 1e-12
+    bad = np.abs(got - ref) > bound
+    if bad.any():
+        r, c = np.argwhere(bad)[0]
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} elements beyond the bf16 bound, first at "
+                             f"[{r}][{c}]: got {got[r, c]}, oracle {ref[r, c]}, bound {bound[r, c]}")

@@ -150,7 +150,9 @@ def test_ep_checks(L):
     assert L.moe_ep_dispatch(c(FAKE), c(FAKE), c(FAKE), 4, 0, sh, bad, None) == INVALID
     odd = (ctypes.c_void_p * 4)(FAKE, FAKE + 8, FAKE, FAKE)
     assert L.moe_ep_return(c(FAKE), c(FAKE), 4, 1, sh, odd, None) == ALIGN
-    assert L.moe_ep_plan(c(FAKE), 4, 5, sh, c(FAKE), None, None) == INVALID
+    assert L.moe_ep_plan(c(FAKE), 4, 5, sh, 1024, c(FAKE), None, None) == INVALID          # rank out of range
+    assert L.moe_ep_plan(c(FAKE), 4, 1, sh, 0, c(FAKE), None, None) == INVALID             # no receive capacity
+    assert L.moe_ep_plan(c(FAKE), 4, 1, sh, 1 << 31, c(FAKE), None, None) == INVALID       # beyond int32 rows
 
 
 def test_bias_update_checks(L):

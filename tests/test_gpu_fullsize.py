@@ -1,22 +1,107 @@
-"""GPU parity at the workloads' full sizes, through moe_layer_forward (the
-call the bench times): routing, counts and the bias step are checked for
-every token (injected mode), the kernel's affinities and the layer output on
-sampled tokens the oracle computes one by one."""
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+bench times: routing, counts and the bias step are checked for every token
+(injected mode), the kernel's affinities on sampled tokens, the grouped
+GEMMs' outputs element by element over whole experts (the most-loaded one,
+a median one, the last one and the shared set), and the layer output element
+by element on sampled tokens the oracle computes one by one."""
 import numpy as np
 import pytest
 import torch
 
 import fine_grained_moe_gate_b200 as moe
 import oracle
-from fine_grained_moe_gate_b200.inputs import CONFIGS, make_layer, make_tokens
+from fine_grained_moe_gate_b200.inputs import CONFIGS, make_layer, make_tokens, to_numpy
 
-from gpu_harness import (DEV, as_f64, check_route_parity, check_status, layer_forward, oracle_rows, rel_fro, route,
-                         to_f64_rows)
+from gpu_harness import (DEV, as_f64, check_bf16_close, check_layer_elementwise, check_route_parity, check_status,
+                         layer_forward, oracle_rows, oracle_terms, permute, rel_fro, route, to_f64_rows)
 
 pytestmark = pytest.mark.gpu
 
 
-def _full_check(cfg, p, x, n_sample, seed, s_tol="auto"):
+def _rows_to_check(r0, r1, dense_limit):
+    """Every row of [r0, r1) when there are at most dense_limit of them; else
+    every 7th row and the last 16, which still reaches every 256-row token tile."""
+    if r1 - r0 <= dense_limit:
+        return np.arange(r0, r1)
+    return np.unique(np.concatenate([np.arange(r0, r1, 7), np.arange(max(r0, r1 - 16), r1)]))
+
+
+def _feature_subset(total, tile, offs):
+    """A few output features of every `tile`-wide feature tile, at the given
+    offsets inside the tile (chosen to reach both CTAs of a pair and every
+    TMEM lane quarter of each)."""
+    f = np.concatenate([t + np.asarray(offs) for t in range(0, total, tile)])
+    return f[f < total]
+
+
+UP_OFFS = (0, 17, 40, 63, 64, 81, 104, 127)        # 128-feature up tiles: 64 per CTA, 32 per lane quarter
+DOWN_OFFS = (0, 45, 100, 127, 128, 160, 201, 255)   # 256-feature down tiles: 128 per CTA
+
+
+def _projection_checks(cfg, p, x, idx, counts, y_layer, w):
+    """moe_permute, moe_ffn_up, moe_ffn_down and moe_combine as the bench
+    calls them.  For the most-loaded expert, a median-loaded one, the last
+    expert with rows and the shared set: h (gate/up + SwiGLU epilogue)
+    against the oracle's up projection of the same token rows, and y_perm /
+    shared_out (down) against the oracle's down projection of the GPU's own h
+    (so that each launch is judged alone), element by element.  Small
+    experts are checked in full; large ones on every 7th row and a feature
+    subset that reaches every tile."""
+    sh = moe.shape_of(cfg)
+    T, k, d, I, S, Is = cfg.T, cfg.k, cfg.d, cfg.I, cfg.S, cfg.Is
+    x_perm, offsets, perm, inv = permute(sh, x, idx, counts)
+    h = torch.empty((T * k, I), dtype=x.dtype, device=DEV)
+    hs = torch.empty((T, S * Is), dtype=x.dtype, device=DEV)
+    moe.moe_ffn_up(x_perm, offsets, p["w1"], p["w3"], x, p["ws1"], p["ws3"], sh, h, hs)
+    y_perm = torch.empty((T * k, d), dtype=x.dtype, device=DEV)
+    shared_out = torch.empty((T, d), dtype=x.dtype, device=DEV)
+    moe.moe_ffn_down(h, offsets, p["w2"], hs, p["ws2"], sh, y_perm, shared_out)
+    y = torch.empty((T, d), dtype=x.dtype, device=DEV)
+    moe.moe_combine(y_perm, w, inv, shared_out, sh, y)
+    torch.cuda.synchronize()
+    check_status()
+    assert torch.equal(y.view(torch.int16), y_layer.view(torch.int16))   # the staged calls are the layer
+    c = counts.cpu().numpy()
+    off = offsets.cpu().numpy()
+    nz = np.nonzero(c)[0]
+    by_load = nz[np.argsort(c[nz], kind="stable")]
+    picks = sorted({int(by_load[-1]), int(by_load[len(by_load) // 2]), int(nz[-1])})
+    fu_all, fd_all = np.arange(I), np.arange(d)
+    for e in picks:
+        r0, r1 = int(off[e]), int(off[e + 1])
+        rows = _rows_to_check(r0, r1, 2048)
+        fu = fu_all if r1 - r0 <= 512 else _feature_subset(I, 128, UP_OFFS)
+        fd = fd_all if r1 - r0 <= 320 else _feature_subset(d, 256, DOWN_OFFS)
+        rt = torch.as_tensor(rows, device=DEV)
+        xr = to_numpy(x_perm[rt])
+        h_ref = oracle.expert_up(xr, to_numpy(p["w1"][e][torch.as_tensor(fu, device=DEV)]),
+                                 to_numpy(p["w3"][e][torch.as_tensor(fu, device=DEV)]))
+        check_bf16_close(as_f64(h[rt][:, torch.as_tensor(fu, device=DEV)]), to_f64_rows(h_ref),
+                         f"{cfg.name} h of expert {e} ({r1 - r0} rows)")
+        o_ref = oracle.expert_down(to_numpy(h[rt]), to_numpy(p["w2"][e][torch.as_tensor(fd, device=DEV)]))
+        check_bf16_close(as_f64(y_perm[rt][:, torch.as_tensor(fd, device=DEV)]), o_ref,
+                         f"{cfg.name} y_perm of expert {e} ({r1 - r0} rows)")
+    if S > 0:
+        rows = _rows_to_check(0, T, 640) if T > 640 else np.arange(T)
+        rt = torch.as_tensor(rows, device=DEV)
+        fu = _feature_subset(Is, 128, UP_OFFS)
+        fd = _feature_subset(d, 256, DOWN_OFFS)
+        xr = to_numpy(x[rt])
+        hs_rows = hs[rt]
+        o_ref = np.zeros((len(rows), len(fd)), np.float64)
+        for s in range(S):
+            h_ref = oracle.expert_up(xr, to_numpy(p["ws1"][s][torch.as_tensor(fu, device=DEV)]),
+                                     to_numpy(p["ws3"][s][torch.as_tensor(fu, device=DEV)]))
+            check_bf16_close(as_f64(hs_rows[:, torch.as_tensor(s * Is + fu, device=DEV)]), to_f64_rows(h_ref),
+                             f"{cfg.name} hs of shared expert {s}")
+            o_ref += oracle.expert_down(to_numpy(hs_rows[:, s * Is:(s + 1) * Is]),
+                                        to_numpy(p["ws2"][s][torch.as_tensor(fd, device=DEV)]))
+        check_bf16_close(as_f64(shared_out[rt][:, torch.as_tensor(fd, device=DEV)]), o_ref,
+                         f"{cfg.name} shared_out")
+    return picks
+
+
+def _full_check(cfg, p, x, n_sample, seed, s_tol="auto", projections=False):
     sh = moe.shape_of(cfg)
     y, idx, w, counts = layer_forward(sh, p, x)
     check_status()
@@ -26,10 +111,11 @@ def _full_check(cfg, p, x, n_sample, seed, s_tol="auto"):
     rows = np.sort(rng.choice(cfg.T, size=min(64, cfg.T), replace=False))
     check_route_parity(x, p["w_gate"], p["bias"], cfg.k, idx, w, counts, aff, s_tol, self_rows=rows)
     assert int(counts.sum()) == cfg.T * cfg.k       # no dropped tokens
-    tokens = np.sort(rng.choice(cfg.T, size=n_sample, replace=False))
-    ref = to_f64_rows(oracle_rows(p, x, idx, w, tokens, cfg.S))
-    got = as_f64(y[torch.as_tensor(tokens, device=DEV)])
-    err = rel_fro(got, ref)
+    if projections:
+        _projection_checks(cfg, p, x, idx, counts, y, w)
+    tokens = np.sort(rng.choice(cfg.T, size=min(n_sample, cfg.T), replace=False))
+    y_ref, mag = oracle_terms(p, x, idx, w, tokens, cfg.S)
+    err = check_layer_elementwise(y[torch.as_tensor(tokens, device=DEV)], y_ref, mag)
     assert err <= 5e-3, err
     return y, idx, w, counts
 
@@ -46,7 +132,7 @@ def v3_layer():
 def test_v3_prefill_full(v3_layer):
     cfg, p = v3_layer
     x = make_tokens(cfg, DEV)
-    _full_check(cfg, p, x, n_sample=6, seed=2)
+    _full_check(cfg, p, x, n_sample=64, seed=2, projections=True)
 
 
 def test_v3_decode_calls(v3_layer):
@@ -55,7 +141,7 @@ def test_v3_decode_calls(v3_layer):
     cfg = CONFIGS["v3_decode"]
     for call in (0, 1, 999):
         x = make_tokens(cfg, DEV, call)
-        _full_check(cfg, p, x, n_sample=4, seed=call)
+        _full_check(cfg, p, x, n_sample=64 if call == 0 else 16, seed=call, projections=call == 0)
 
 
 def test_small_bf16_full_and_ten_steps():
@@ -67,7 +153,7 @@ def test_small_bf16_full_and_ten_steps():
     for step in range(cfg.steps):
         x = make_tokens(cfg, DEV, step)
         if step in (0, cfg.steps - 1):
-            y, idx, w, counts = _full_check(cfg, p, x, n_sample=24, seed=step)
+            y, idx, w, counts = _full_check(cfg, p, x, n_sample=64, seed=step, projections=step == 0)
         else:
             y, idx, w, counts = layer_forward(sh, p, x)
         ridx, rw, rc, aff = route(sh, x, p["w_gate"], p["bias"])
@@ -91,7 +177,7 @@ def test_skew_stress_routing_and_sampled_output():
     for step in range(5):
         x = make_tokens(cfg, DEV, step)
         if step == 0:
-            y, idx, w, counts = _full_check(cfg, p, x, n_sample=3, seed=4)
+            y, idx, w, counts = _full_check(cfg, p, x, n_sample=64, seed=4, projections=True)
             c = counts.cpu().numpy()
             assert c.max() > 8 * c.mean()    # the workload really is skewed
         else:

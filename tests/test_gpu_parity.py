@@ -16,8 +16,8 @@ import fine_grained_moe_gate_b200 as moe
 import oracle
 from fine_grained_moe_gate_b200.inputs import CONFIGS, make_layer, make_tokens, to_numpy
 
-from gpu_harness import (DEV, as_f64, check_route_parity, check_status, grouped_swiglu, layer_forward, oracle_rows,
-                         permute, rel_fro, route, to_f64_rows)
+from gpu_harness import (DEV, as_f64, check_layer_elementwise, check_route_parity, check_status, grouped_swiglu,
+                         layer_forward, oracle_rows, oracle_terms, permute, rel_fro, route, to_f64_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -340,6 +340,9 @@ def test_layer_bf16_against_oracle(shape):
                               n["ws3"], n["ws2"])
     err = rel_fro(as_f64(y), to_f64_rows(ref))
     assert err <= 5e-3, err
+    # element by element, every token: within the bf16 bound the roundings allow
+    y_ref, mag = oracle_terms(p, x, idx, w, np.arange(cfg.T), cfg.S)
+    check_layer_elementwise(y, y_ref, mag)
 
 
 def test_layer_is_deterministic():

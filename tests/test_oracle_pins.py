@@ -370,3 +370,34 @@ def test_layer_routed_mixture_masked_loop(oracle_lib):
             slot = (it[mask] == e).nonzero(as_tuple=True)[1]
             ref[mask] += wt[mask, slot].unsqueeze(-1) * _swiglu64(P["x"][mask], P["w1"][e], P["w3"][e], P["w2"][e])
     assert _rel_fro(y, ref.numpy()) < 2e-7
+
+
+def test_expert_up_down_against_float64_library(oracle_lib):
+    """The two projections of one expert (DeepSeekMoE sketch: one SwiGLU MLP
+    per expert): expert_up against torch float64 silu(x W1^T) * (x W3^T)
+    rounded once to bf16; expert_down against a float64 matmul of the same
+    h.  A transposed weight or a swapped W1/W3 fails these (W1 != W3)."""
+    n, d, I = 7, 40, 24
+    p = _layer_inputs(n, d, 1, I, 1, 8, 6, torch.bfloat16)
+    nb = _np(p)
+    h = oracle.expert_up(nb["x"], nb["w1"][0], nb["w3"][0])
+    P = {k_: v.double() for k_, v in p.items()}
+    ref = (torch.nn.functional.silu(P["x"] @ P["w1"][0].T) * (P["x"] @ P["w3"][0].T)).to(torch.bfloat16)
+    got = torch.from_numpy(h.view(np.int16)).view(torch.bfloat16)
+    diff = (got.double() - ref.double()).abs()
+    # float64 sums in another order may land on the other side of a bf16
+    # rounding boundary: at most one ulp, and rarely
+    assert (diff <= 2.0 ** -7 * ref.double().abs() + 1e-30).all()
+    assert (diff > 0).float().mean() < 0.01
+    swapped = oracle.expert_up(nb["x"], nb["w3"][0], nb["w1"][0])
+    assert not np.array_equal(swapped, h)
+    o = oracle.expert_down(h, nb["w2"][0])
+    ref_o = got.double() @ P["w2"][0].T
+    assert np.allclose(o, ref_o.numpy(), rtol=1e-12, atol=1e-12)
+    # fp32 layer: the split equals the fused accumulation exactly
+    pf = _np(_layer_inputs(n, d, 1, I, 1, 8, 7))
+    yacc = np.zeros((n, d), np.float64)
+    oracle.expert_accumulate(pf["x"], np.arange(n, dtype=np.int32), np.ones(n), pf["w1"][0], pf["w3"][0],
+                             pf["w2"][0], yacc)
+    o32 = oracle.expert_down(oracle.expert_up(pf["x"], pf["w1"][0], pf["w3"][0]), pf["w2"][0])
+    assert np.array_equal(o32, yacc)

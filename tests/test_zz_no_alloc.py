@@ -55,6 +55,25 @@ def test_permute_noalloc_matches_permute_on_consecutive_calls():
         assert int(got[1][-1]) == cfg.T * cfg.k
 
 
+def test_permute_noalloc_largest_accepted_problem():
+    """ceil(T/128) * E = 256 * 256 = 65536 counters: exactly the built-in
+    scratch's capacity, so the size check's edge is exercised; the result is
+    still bit-identical to moe_permute with a caller workspace, twice."""
+    cfg = CONFIGS["v3_prefill"].scaled(T=32768, d=64, E=256, k=2)
+    sh, x, idx, counts = _routing(cfg)
+    ref = _outputs(cfg, x)
+    ws = torch.empty(max(moe.moe_permute_workspace_size(sh), 256), dtype=torch.uint8, device=DEV)
+    moe.moe_permute(x, idx, counts, sh, *ref, ws)
+    for _ in range(2):
+        got = _outputs(cfg, x)
+        moe.moe_permute_noalloc(x, idx, counts, sh, *got)
+        torch.cuda.synchronize()
+        assert moe.moe_get_last_error() == 0
+        assert torch.equal(got[0].view(torch.int16), ref[0].view(torch.int16)), "x_perm differs"
+        for a, b, name in zip(got[1:], ref[1:], ("offsets", "perm_tok", "inv_row")):
+            assert torch.equal(a, b), f"{name} differs"
+
+
 def test_permute_noalloc_rejects_problems_beyond_its_scratch():
     cfg = CONFIGS["v3_prefill"].scaled(T=32768 + 128, d=64, E=256, k=2)   # needs 65792 counters > 65536
     sh = moe.shape_of(cfg)
