@@ -69,6 +69,11 @@ def _load():
         lib.orc_quantize_rows_fp8.argtypes = [P, i, ctypes.c_long, i, i, P, P]
         lib.orc_expert_up_fp8.argtypes = [P, P, i, P, P, P, P, i, i, P]
         lib.orc_expert_down_fp8.argtypes = [P, P, i, P, P, i, i, i, P]
+        lib.orc_mx_exponent.argtypes = [ctypes.c_double]
+        lib.orc_mx_exponent.restype = i
+        lib.orc_quantize_mx.argtypes = [P, i, ctypes.c_long, i, i, P, P]
+        lib.orc_expert_up_mx.argtypes = [P, P, i, P, P, P, P, i, i, P]
+        lib.orc_expert_down_mx.argtypes = [P, P, i, P, P, i, i, i, P]
         _lib = lib
     return _lib
 
@@ -327,5 +332,119 @@ def layer_output_fp8(x, idx, w, q: dict) -> np.ndarray:
                           q["w3s"][e * I:(e + 1) * I])
         hq, hsc = quantize_rows_fp8(h)
         o = expert_down_fp8(hq, hsc, q["w2q"][e], q["w2s"][e * d:(e + 1) * d])
+        yacc[t] += w[t, j].astype(np.float64)[:, None] * o
+    return finalize(yacc, x.dtype)
+
+
+# ------------------------------------------------- FP8 experts, per-tile scales
+#
+# Tiles of 32 consecutive elements of a row along the contraction dimension,
+# each with a power-of-two scale 2^e (e the smallest integer with
+# amax <= 448 * 2^e), stored as the byte e + 127; codes E4M3(v * 2^-e).
+# Pages: "DeepSeek V3 From Scratch", "The idea" (fine-grained quantization
+# tiles); crackai.dev "DeepSeek-V3", "How It Works" (per-tile scaling).
+
+MX_TILE = 32
+
+
+def mx_exponent(amax: float) -> int:
+    """Smallest e in [-127, 127] with amax <= 448 * 2^e (0 for amax = 0)."""
+    return int(_load().orc_mx_exponent(float(amax)))
+
+
+def quantize_mx(a: np.ndarray, nseg: int = 1):
+    """Per-tile E4M3 quantization.  ``a`` is [rows][K] (bf16 bits as uint16,
+    or float32) or [nseg][rows][kseg] (rows span all blocks, K = nseg*kseg).
+    Returns (codes with a's shape, exponent bytes uint8 [rows][K/32])."""
+    a = _c(a)
+    dt = _dtype_code(a)
+    if a.ndim == 3:
+        if a.shape[0] != nseg:
+            raise ValueError("nseg must equal the number of column blocks")
+        rows, kseg = a.shape[1], a.shape[2]
+    else:
+        if nseg != 1:
+            raise ValueError("a blocked matrix is passed as [nseg][rows][kseg]")
+        rows, kseg = a.shape
+    if kseg % MX_TILE:
+        raise ValueError("the row length of each block must be a multiple of 32")
+    q = np.empty(a.shape, np.uint8)
+    eb = np.empty((rows, nseg * kseg // MX_TILE), np.uint8)
+    _load().orc_quantize_mx(_ptr(a), dt, rows, kseg, nseg, _ptr(q), _ptr(eb))
+    return q, eb
+
+
+def mx_dequantize(q: np.ndarray, eb: np.ndarray) -> np.ndarray:
+    """Values (float64) of row-major codes [rows][K] with exponent bytes [rows][K/32]."""
+    v = fp8_decode(q)
+    scale = np.ldexp(1.0, eb.astype(np.int64) - 127)
+    return v * np.repeat(scale, MX_TILE, axis=1)
+
+
+def expert_up_mx(xq, xe, w1q, w1e, w3q, w3e) -> np.ndarray:
+    """h = bf16(silu(a) * g), a and g tile-scaled E4M3 dot products; bf16 bits [n][I]."""
+    xq, w1q, w3q = _c(xq, np.uint8), _c(w1q, np.uint8), _c(w3q, np.uint8)
+    xe, w1e, w3e = _c(xe, np.uint8), _c(w1e, np.uint8), _c(w3e, np.uint8)
+    n, d = xq.shape
+    I = w1q.shape[0]
+    h = np.empty((n, I), np.uint16)
+    _load().orc_expert_up_mx(_ptr(xq), _ptr(xe), n, _ptr(w1q), _ptr(w1e), _ptr(w3q), _ptr(w3e), d, I, _ptr(h))
+    return h
+
+
+def expert_down_mx(hq, he, w2q, w2e) -> np.ndarray:
+    """o [n][d] (float64), tile-scaled E4M3 products of h rows and W2 rows.
+    w2q is [d][K] or [nseg][d][kseg] (blocks joined along K) with w2e [d][K/32]."""
+    hq, w2q = _c(hq, np.uint8), _c(w2q, np.uint8)
+    he, w2e = _c(he, np.uint8), _c(w2e, np.uint8)
+    n = hq.shape[0]
+    if w2q.ndim == 3:
+        nseg, d, kseg = w2q.shape
+    else:
+        nseg, (d, kseg) = 1, w2q.shape
+    o = np.empty((n, d), np.float64)
+    _load().orc_expert_down_mx(_ptr(hq), _ptr(he), n, _ptr(w2q), _ptr(w2e), d, kseg, nseg, _ptr(o))
+    return o
+
+
+def quantize_weights_mx(p: dict) -> dict:
+    """Per-tile quantization of a layer's expert weights (numpy, bf16 bits):
+    W1/W3 [E][I][d] and W2 [E][d][I] per row, shared Ws1/Ws3 [S][Is][d] per
+    row, Ws2 [S][d][Is] per row d across the S blocks.  Codes under w1q, ...
+    exponent bytes under w1e, ... ([rows][K/32], rows = E*I, E*d, ...)."""
+    out = {}
+    for key in ("w1", "w3", "w2", "ws1", "ws3"):
+        a = p[key]
+        q, eb = quantize_mx(a.reshape(-1, a.shape[-1]))
+        out[key + "q"], out[key + "e"] = q.reshape(a.shape), eb
+    ws2 = p["ws2"]
+    q, eb = quantize_mx(ws2, nseg=ws2.shape[0])
+    out["ws2q"], out["ws2e"] = q, eb
+    return out
+
+
+def layer_output_mx(x, idx, w, q: dict) -> np.ndarray:
+    """Whole layer with tile-scaled FP8 experts for given routing: x (bf16
+    bits) [T][d] quantized by tiles; each routed expert e: h = up(x rows), h
+    quantized by tiles, o = down(h), y += w * o; shared: h over the S*Is
+    concatenated features, quantized by tiles, o = down over the concatenated
+    K.  y in bf16 bits."""
+    T, d = x.shape
+    E, I, _ = q["w1q"].shape
+    S, Is, _ = q["ws1q"].shape
+    xq, xe = quantize_mx(x)
+    yacc = np.zeros((T, d), np.float64)
+    if S > 0:
+        hs = expert_up_mx(xq, xe, q["ws1q"].reshape(S * Is, d), q["ws1e"], q["ws3q"].reshape(S * Is, d), q["ws3e"])
+        hq, he = quantize_mx(hs)
+        yacc += expert_down_mx(hq, he, q["ws2q"], q["ws2e"])
+    for e in range(E):
+        t, j = np.nonzero(idx == e)
+        if len(t) == 0:
+            continue
+        h = expert_up_mx(xq[t], xe[t], q["w1q"][e], q["w1e"][e * I:(e + 1) * I], q["w3q"][e],
+                         q["w3e"][e * I:(e + 1) * I])
+        hq, he = quantize_mx(h)
+        o = expert_down_mx(hq, he, q["w2q"][e], q["w2e"][e * d:(e + 1) * d])
         yacc[t] += w[t, j].astype(np.float64)[:, None] * o
     return finalize(yacc, x.dtype)

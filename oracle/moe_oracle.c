@@ -455,3 +455,107 @@ void orc_expert_down_fp8(const uint8_t* hq, const float* hs, int n, const uint8_
         }
     }
 }
+
+/* ---- FP8 (E4M3) experts with per-tile scaling ----------------------------
+ * [P1 "The idea": FP8 mixed precision with fine-grained quantization tiles;
+ *  P5 "How It Works": FP8 training with per-tile scaling; P4 "FP8 Formats":
+ *  E4M3 for weights and activations.]  The pages fix neither the tile nor
+ * the scale arithmetic.  Read here as: a tile is 32 consecutive elements of
+ * one row along the contraction dimension (weights: along the input features
+ * of each output row; activations: along the features of each token row),
+ * and its scale is a power of two, 2^e with e the smallest integer such that
+ * the tile's largest magnitude fits the E4M3 range (amax <= 448 * 2^e), so no
+ * element saturates.  Codes are E4M3(v * 2^-e).  The scale of a tile is kept
+ * as its exponent byte e + 127.  A dot product then sums, tile by tile,
+ * 2^(e_a + e_b) * sum_{i in tile} dec(qa_i) dec(qb_i). */
+
+#define ORC_MX_TILE 32
+
+/* Smallest e in [-127, 127] with amax <= 448 * 2^e (0 for an all-zero tile;
+ * -127 for tiles whose amax is below 448 * 2^-127). */
+int orc_mx_exponent(double amax) {
+    if (!(amax > 0.0)) return 0;
+    int e = -127;
+    while (e < 127 && amax > ldexp(448.0, e)) ++e;
+    return e;
+}
+
+/* Tile quantization of a matrix with `rows` rows of K = nseg * kseg columns,
+ * stored as [nseg][rows][kseg] (nseg = 1: plain row major); kseg % 32 == 0.
+ * q has src's layout; ebyte [rows][K / 32] holds e + 127 of tile b of row r
+ * at r * (K / 32) + b, tiles numbered along the whole row. */
+void orc_quantize_mx(const void* src, int dtype, long rows, int kseg, int nseg, uint8_t* q, uint8_t* ebyte) {
+    int K = kseg * nseg, nb = K / ORC_MX_TILE;
+    #pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        for (int b = 0; b < nb; ++b) {
+            double amax = 0.0;
+            for (int c = b * ORC_MX_TILE; c < (b + 1) * ORC_MX_TILE; ++c) {
+                double v = fabs(load_elem(src, dtype, seg_index(r, c, rows, kseg)));
+                if (v > amax) amax = v;
+            }
+            int e = orc_mx_exponent(amax);
+            ebyte[(size_t)r * nb + b] = (uint8_t)(e + 127);
+            for (int c = b * ORC_MX_TILE; c < (b + 1) * ORC_MX_TILE; ++c) {
+                size_t i = seg_index(r, c, rows, kseg);
+                q[i] = orc_e4m3_encode((float)(load_elem(src, dtype, i) * ldexp(1.0, -e)));
+            }
+        }
+    }
+}
+
+/* sum over the K/32 tiles of 2^(ea + eb) * sum_i dec(qa_i) dec(qb_i), in
+ * double; a and b are rows of K codes whose tile exponent bytes are ea, eb. */
+static double mx_dot(const uint8_t* qa, const uint8_t* ea, const uint8_t* qb, const uint8_t* eb, int K,
+                     size_t (*bidx)(const void*, int), const void* bctx) {
+    const double* val = e4m3_values();
+    double acc = 0.0;
+    for (int b = 0; b < K / ORC_MX_TILE; ++b) {
+        double s = 0.0;
+        for (int i = b * ORC_MX_TILE; i < (b + 1) * ORC_MX_TILE; ++i)
+            s += val[qa[i]] * val[qb[bidx ? bidx(bctx, i) : (size_t)i]];
+        acc += ldexp(s, ((int)ea[b] - 127) + ((int)eb[b] - 127));
+    }
+    return acc;
+}
+
+/* Gate/up of one FP8 expert on n token rows quantized by tiles:
+ *   a[r][c] = mx_dot(xq[r], W1q[c]),  g[r][c] = mx_dot(xq[r], W3q[c])  (double)
+ *   h[r][c] = bf16(silu(a) * g)
+ * xq [n][d] with xe [n][d/32]; w1q/w3q [I][d] with w1e/w3e [I][d/32]. */
+void orc_expert_up_mx(const uint8_t* xq, const uint8_t* xe, int n, const uint8_t* w1q, const uint8_t* w1e,
+                      const uint8_t* w3q, const uint8_t* w3e, int d, int I, uint16_t* h) {
+    int nb = d / ORC_MX_TILE;
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (int c = 0; c < I; ++c) {
+        for (int r = 0; r < n; ++r) {
+            const uint8_t* xr = xq + (size_t)r * d;
+            const uint8_t* xer = xe + (size_t)r * nb;
+            double a = mx_dot(xr, xer, w1q + (size_t)c * d, w1e + (size_t)c * nb, d, NULL, NULL);
+            double g = mx_dot(xr, xer, w3q + (size_t)c * d, w3e + (size_t)c * nb, d, NULL, NULL);
+            h[(size_t)r * I + c] = float_to_bf16_bits((float)(a / (1.0 + exp(-a)) * g));
+        }
+    }
+}
+
+/* Down projection of one FP8 expert on n rows of h quantized by tiles:
+ *   o[r][j] = mx_dot(hq[r], W2q(j, .))  (double)
+ * hq [n][K] with he [n][K/32]; W2q is [d][K] stored as nseg blocks of kseg
+ * columns ([nseg][d][kseg], K = nseg * kseg) with w2e [d][K/32] (tiles
+ * numbered along the whole row, as orc_quantize_mx gives them). */
+struct mx_seg_ctx { long rows; int kseg; long j; };
+static size_t mx_seg_col(const void* ctx, int c) {
+    const struct mx_seg_ctx* s = (const struct mx_seg_ctx*)ctx;
+    return seg_index(s->j, c, s->rows, s->kseg);
+}
+void orc_expert_down_mx(const uint8_t* hq, const uint8_t* he, int n, const uint8_t* w2q, const uint8_t* w2e, int d,
+                        int kseg, int nseg, double* o) {
+    int K = kseg * nseg, nb = K / ORC_MX_TILE;
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (int j = 0; j < d; ++j) {
+        struct mx_seg_ctx ctx = {d, kseg, j};
+        for (int r = 0; r < n; ++r)
+            o[(size_t)r * d + j] = mx_dot(hq + (size_t)r * K, he + (size_t)r * nb, w2q, w2e + (size_t)j * nb, K,
+                                          mx_seg_col, &ctx);
+    }
+}
