@@ -236,9 +236,9 @@ def oracle_sample(cfg, p, x, n_tok):
 
 
 def oracle_sample_fp8(cfg, p, x, n_tok):
-    """oracle_sample for the E4M3 expert workloads: routing, per-token
+    """oracle_sample for the E4M3 expert workloads: routing, per-tile
     quantization of x, and for every expert the tokens use (and the shared
-    experts) the FP8 gate/up, per-row quantization of h and the FP8 down.
+    experts) the FP8 gate/up, per-tile quantization of h and the FP8 down.
     The expert weights are quantized by the oracle itself, expert by expert,
     before the clock starts; only the forward's oracle arithmetic is timed."""
     import numpy as np
@@ -253,25 +253,25 @@ def oracle_sample_fp8(cfg, p, x, n_tok):
     t0 = time.perf_counter()
     s = oracle.affinity(xs, wg)
     idx, w = oracle.select(s, bias, cfg.k)
-    xq, xsc = oracle.quantize_rows_fp8(xs)
+    xq, xe = oracle.quantize_mx(xs)
     secs = time.perf_counter() - t0
     yacc = np.zeros((n_tok, d), np.float64)
     if S > 0:
-        q1, s1 = oracle.quantize_rows_fp8(to_numpy(p["ws1"]).reshape(S * Is, d))
-        q3, s3 = oracle.quantize_rows_fp8(to_numpy(p["ws3"]).reshape(S * Is, d))
-        q2, s2 = oracle.quantize_rows_fp8(to_numpy(p["ws2"]), nseg=S)
+        q1, e1 = oracle.quantize_mx(to_numpy(p["ws1"]).reshape(S * Is, d))
+        q3, e3 = oracle.quantize_mx(to_numpy(p["ws3"]).reshape(S * Is, d))
+        q2, e2 = oracle.quantize_mx(to_numpy(p["ws2"]), nseg=S)
         t0 = time.perf_counter()
-        hq, hsc = oracle.quantize_rows_fp8(oracle.expert_up_fp8(xq, xsc, q1, s1, q3, s3))
-        yacc += oracle.expert_down_fp8(hq, hsc, q2, s2)
+        hq, he = oracle.quantize_mx(oracle.expert_up_mx(xq, xe, q1, e1, q3, e3))
+        yacc += oracle.expert_down_mx(hq, he, q2, e2)
         secs += time.perf_counter() - t0
     for e in np.unique(idx):
         ii, jj = np.nonzero(idx == e)
-        q1, s1 = oracle.quantize_rows_fp8(to_numpy(p["w1"][e]))
-        q3, s3 = oracle.quantize_rows_fp8(to_numpy(p["w3"][e]))
-        q2, s2 = oracle.quantize_rows_fp8(to_numpy(p["w2"][e]))
+        q1, e1 = oracle.quantize_mx(to_numpy(p["w1"][e]))
+        q3, e3 = oracle.quantize_mx(to_numpy(p["w3"][e]))
+        q2, e2 = oracle.quantize_mx(to_numpy(p["w2"][e]))
         t0 = time.perf_counter()
-        hq, hsc = oracle.quantize_rows_fp8(oracle.expert_up_fp8(xq[ii], xsc[ii], q1, s1, q3, s3))
-        yacc[ii] += w[ii, jj].astype(np.float64)[:, None] * oracle.expert_down_fp8(hq, hsc, q2, s2)
+        hq, he = oracle.quantize_mx(oracle.expert_up_mx(xq[ii], xe[ii], q1, e1, q3, e3))
+        yacc[ii] += w[ii, jj].astype(np.float64)[:, None] * oracle.expert_down_mx(hq, he, q2, e2)
         secs += time.perf_counter() - t0
     t0 = time.perf_counter()
     oracle.finalize(yacc, xs.dtype)
@@ -352,14 +352,15 @@ class LayerStep:
         self.hs = e(T, max(1, cfg.S * cfg.Is), dtype=dt)
         self.shared_out = e(T, d, dtype=dt) if cfg.S > 0 else None
         self.y = e(T, d, dtype=dt)
-        if self.fp8:  # E4M3 expert weights, quantized once per output row before timing
+        if self.fp8:  # E4M3 expert weights with tile scales, quantized once before timing
             self.q8 = moe.quantize_experts_fp8(p)
             self.w8 = moe.fp8_experts(self.q8)
-            SIs = max(1, cfg.S * cfg.Is)
-            self.xq, self.xsc = e(T, d, dtype=torch.uint8), e(T, dtype=torch.float32)
+            SIs = max(128, cfg.S * cfg.Is)
+            tok = moe.MOE_SF_TOKENS
+            self.xq, self.xsc = e(T, d, dtype=torch.uint8), moe.fp8_scales(T, d, tok, dev)
             self.xq_perm = e(T * k, d, dtype=torch.uint8)
-            self.hq, self.h_sc = e(T * k, cfg.I, dtype=torch.uint8), e(T * k, dtype=torch.float32)
-            self.hsq, self.hs_sc = e(T, SIs, dtype=torch.uint8), e(T, dtype=torch.float32)
+            self.hq, self.h_sc = e(T * k, cfg.I, dtype=torch.uint8), moe.fp8_scales(T * k, cfg.I, tok, dev)
+            self.hsq, self.hs_sc = e(T, SIs, dtype=torch.uint8), moe.fp8_scales(T, SIs, tok, dev)
             torch.cuda.synchronize()
 
     def __call__(self, i, ev=None):
@@ -372,7 +373,7 @@ class LayerStep:
         moe.moe_route(x, p["w_gate"], p["bias"], sh, self.idx, self.w, self.counts, None, st)
         rec(1)
         if self.fp8:
-            moe.moe_quantize_fp8(x, T, cfg.d, 1, self.xq, self.xsc, st)
+            moe.moe_quantize_fp8(x, T, cfg.d, 1, moe.MOE_SF_TOKENS, self.xq, self.xsc, st)
             rec(2)
             moe.moe_permute(self.xq, self.idx, self.counts, sh, self.xq_perm, self.offsets, self.perm, self.inv,
                             self.pws, st)
@@ -380,9 +381,9 @@ class LayerStep:
             moe.moe_ffn_up_fp8(self.xq_perm, self.perm, self.xsc, self.offsets, self.xq if sh_ else None, self.w8, sh,
                                self.h, self.hs if sh_ else None, st)
             rec(4)
-            moe.moe_quantize_fp8(self.h, T * k, cfg.I, 1, self.hq, self.h_sc, st)
+            moe.moe_quantize_fp8(self.h, T * k, cfg.I, 1, moe.MOE_SF_TOKENS, self.hq, self.h_sc, st)
             if sh_:
-                moe.moe_quantize_fp8(self.hs, T, cfg.S * cfg.Is, 1, self.hsq, self.hs_sc, st)
+                moe.moe_quantize_fp8(self.hs, T, cfg.S * cfg.Is, 1, moe.MOE_SF_TOKENS, self.hsq, self.hs_sc, st)
             rec(5)
             moe.moe_ffn_down_fp8(self.hq, self.h_sc, self.offsets, self.hsq if sh_ else None, self.hs_sc, self.w8,
                                  sh, self.x_perm, self.shared_out, st)
@@ -713,7 +714,8 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
             "data": "synthetic (seeded N(0,1) tokens, N(0,std) weights of the stated shape"
-                    + ("; expert weights quantized to E4M3 per output row before timing)" if fp8 else ")"),
+                    + ("; expert weights quantized to E4M3 with 1x32 power-of-two tile scales before timing)"
+                       if fp8 else ")"),
             "config": {"workload": cfg.name, "T_per_gpu": T, "global_batch": T * world, "d": d, "E": E, "k": k,
                        "I": cfg.I, "S": cfg.S, "Is": cfg.Is, "parallelism": f"dp{world}",
                        "l2": f"inputs larger than L2: layer weights read every step ({weights_gb:.1f} GB)",
@@ -851,17 +853,29 @@ def run_backward(args, world, rank, local):
     # router's dx and dW_g 4 d E
     flop = T * k * 18 * d * I + T * 16 * d * S * Is + T * 4 * d * E
     tflops = flop / (ms * 1e-3) / 1e12
+    # bf16 layers whose widths are multiples of 128 run the expert contractions on the tensor cores
+    tc = cfg.dtype == "bf16" and d % 128 == 0 and I % 128 == 0 and (S == 0 or Is % 128 == 0)
+    if tc:
+        peaks, peak_src = load_peaks()
+        burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        roof = {"bound": "tensor", "achieved": round(tflops, 2), "peak": burst, "unit": "TFLOP/s",
+                "frac": round(tflops / burst, 4), "traffic": None,
+                "peak_kind": f"bf16_tflops ({peak_src}, burst): the backward is timed in a sub-second region; "
+                             "FLOPs of the router (2 d E per token, fp32 SIMT) included"}
+    else:
+        roof = {"bound": "alu", "achieved": round(tflops, 3), "peak": round(FP32_SIMT_PEAK_TFLOPS, 1),
+                "unit": "TFLOP/s", "frac": round(tflops / FP32_SIMT_PEAK_TFLOPS, 4), "traffic": None,
+                "peak_kind": "derived: 148 SMs x 128 fp32 FMA lanes x 2 FLOP x 1965 MHz"}
     line = {
-        "metric": "MoE layer backward tokens/s (fp32 SIMT contractions)", "value": round(T / (ms * 1e-3), 2),
+        "metric": "MoE layer backward tokens/s (%s)" % ("tcgen05 bf16 contractions" if tc else "fp32 SIMT contractions"),
+        "value": round(T / (ms * 1e-3), 2),
         "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if tc else "f32",
         "data": "synthetic (seeded N(0,1) tokens and dy, N(0,std) weights of the stated shape)",
         "config": {"workload": cfg.name + " backward", "T": T, "d": d, "E": E, "k": k, "I": I, "S": S, "Is": Is,
                    "balance_alpha": 1e-4, "seq_len": L,
                    "l2": "weights and activations far larger than L2 at these shapes; no flush"},
-        "roofline": {"bound": "alu", "achieved": round(tflops, 3), "peak": round(FP32_SIMT_PEAK_TFLOPS, 1),
-                     "unit": "TFLOP/s", "frac": round(tflops / FP32_SIMT_PEAK_TFLOPS, 4), "traffic": None,
-                     "peak_kind": "derived: 148 SMs x 128 fp32 FMA lanes x 2 FLOP x 1965 MHz"},
+        "roofline": roof, "tflops": round(tflops, 2),
         "gpu_launches": int(launches), "clocks": ck,
     }
     print(json.dumps(line), flush=True)

@@ -31,9 +31,10 @@ STATUS = {
 EXPORTS = (
     "moe_route", "moe_load_and_bias_update", "moe_permute", "moe_permute_workspace_size", "moe_permute_noalloc",
     "moe_grouped_swiglu", "moe_grouped_swiglu_workspace_size", "moe_expert_up", "moe_expert_down", "moe_ffn_up",
-    "moe_ffn_down", "moe_combine", "moe_layer_forward", "moe_workspace_size", "moe_get_last_error",
+    "moe_ffn_down", "moe_ffn_down_combine", "moe_combine_finish", "moe_combine", "moe_layer_forward",
+    "moe_workspace_size", "moe_get_last_error",
     "moe_kernel_launch_count", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
-    "moe_quantize_fp8", "moe_ffn_up_fp8", "moe_ffn_down_fp8", "moe_layer_forward_fp8",
+    "moe_quantize_fp8", "moe_fp8_scale_bytes", "moe_ffn_up_fp8", "moe_ffn_down_fp8", "moe_layer_forward_fp8",
     "moe_ep_plan_size", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_return",
     "moe_layer_backward", "moe_backward_workspace_size",
 )
@@ -101,9 +102,11 @@ def lib() -> ctypes.CDLL:
             "moe_ffn_up": [P, P, P, P, P, P, P, S, P, P, P],
             "moe_ffn_down": [P, P, P, P, P, S, P, P, P],
             "moe_combine": [P, P, P, P, S, P, P],
+            "moe_ffn_down_combine": [P, P, P, P, P, P, P, S, P, P],
+            "moe_combine_finish": [P, S, P, P],
             "moe_layer_forward": [P, P, P, P, P, P, P, P, P, S, P, P, P, P, P, sz, P],
             "moe_get_last_error": [P],
-            "moe_quantize_fp8": [P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, P, P, P],
+            "moe_quantize_fp8": [P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P],
             "moe_ffn_up_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_ffn_down_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_layer_forward_fp8": [P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P, P, P, sz, P],
@@ -124,6 +127,8 @@ def lib() -> ctypes.CDLL:
             fn.restype = sz
         L.moe_backward_workspace_size.argtypes = [S, ctypes.c_int32]
         L.moe_backward_workspace_size.restype = sz
+        L.moe_fp8_scale_bytes.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32]
+        L.moe_fp8_scale_bytes.restype = sz
         L.moe_ep_plan_size.argtypes = [ctypes.c_int32, S]
         L.moe_ep_plan_size.restype = sz
         L.moe_kernel_launch_count.argtypes = []
@@ -215,6 +220,15 @@ def moe_ffn_down(h, offsets, w2, hs, ws2, shape, y_perm, shared_out, stream=None
                               _stream(stream)), "moe_ffn_down")
 
 
+def moe_ffn_down_combine(h, offsets, w2, hs, ws2, perm_tok, topk_w, shape, y_acc, stream=None):
+    _check(lib().moe_ffn_down_combine(_p(h), _p(offsets), _p(w2), _p(hs), _p(ws2), _p(perm_tok), _p(topk_w), shape,
+                                      _p(y_acc), _stream(stream)), "moe_ffn_down_combine")
+
+
+def moe_combine_finish(y_acc, shape, y, stream=None):
+    _check(lib().moe_combine_finish(_p(y_acc), shape, _p(y), _stream(stream)), "moe_combine_finish")
+
+
 def moe_combine(y_perm, topk_w, inv_row, shared_out, shape, y, stream=None):
     _check(lib().moe_combine(_p(y_perm), _p(topk_w), _p(inv_row), _p(shared_out), shape, _p(y), _stream(stream)),
            "moe_combine")
@@ -274,8 +288,26 @@ def moe_abi_version() -> int:
 
 # ---- FP8 experts -------------------------------------------------------------
 
-def moe_quantize_fp8(src, rows, kseg, nseg, q, scale, stream=None):
-    _check(lib().moe_quantize_fp8(_p(src), rows, kseg, nseg, _p(q), _p(scale), _stream(stream)), "moe_quantize_fp8")
+MOE_SF_TOKENS, MOE_SF_WEIGHTS = 0, 1
+
+
+def moe_fp8_scale_bytes(rows, K, layout) -> int:
+    return lib().moe_fp8_scale_bytes(rows, K, layout)
+
+
+def moe_quantize_fp8(src, rows, kseg, nseg, layout, q, scales, stream=None):
+    _check(lib().moe_quantize_fp8(_p(src), rows, kseg, nseg, layout, _p(q), _p(scales), _stream(stream)),
+           "moe_quantize_fp8")
+
+
+def fp8_scales(rows, K, layout, device):
+    """An uninitialised device buffer for the tile scales of a [rows][K] matrix
+    in the given layout (uint8, moe_fp8_scale_bytes long)."""
+    import torch
+    n = moe_fp8_scale_bytes(rows, K, layout)
+    if n == 0:
+        raise MoEError(1, "moe_fp8_scale_bytes: K must be a multiple of 128")
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def moe_ffn_up_fp8(xq_perm, perm_tok, x_scale, offsets, xq, experts, shape, h, hs, stream=None):
@@ -296,26 +328,27 @@ def moe_layer_forward_fp8(x, w_gate, bias, experts, shape, y, topk_idx, topk_w, 
 
 def quantize_experts_fp8(p: dict, stream=None) -> dict:
     """E4M3 copies of a layer's bf16 expert weights (device tensors) through
-    moe_quantize_fp8: per output row for W1/W3/W2 and the shared Ws1/Ws3; the
-    shared Ws2 [S][d][Is] per output row across its S blocks.  Returns uint8
-    codes and fp32 scales under w1q, w1s, ... (the weights' own shapes)."""
+    moe_quantize_fp8, tile scales in the weights' layout (MOE_SF_WEIGHTS):
+    W1/W3/W2 and the shared Ws1/Ws3 row by row, the shared Ws2 [S][d][Is] as
+    d rows across its S blocks.  Returns uint8 codes (the weights' own shapes)
+    and scale buffers under w1q, w1s, ..."""
     import torch
     out = {}
     for n in ("w1", "w3", "w2", "ws1", "ws3"):
         w = p[n]
-        if w.numel() == 0:
+        if w is None or w.numel() == 0:
             continue
         rows, K = w.numel() // w.shape[-1], w.shape[-1]
         q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
-        sc = torch.empty(rows, dtype=torch.float32, device=w.device)
-        moe_quantize_fp8(w, rows, K, 1, q, sc, stream)
+        sc = fp8_scales(rows, K, MOE_SF_WEIGHTS, w.device)
+        moe_quantize_fp8(w, rows, K, 1, MOE_SF_WEIGHTS, q, sc, stream)
         out[n + "q"], out[n + "s"] = q, sc
-    w = p["ws2"]
-    if w.numel() > 0:
+    w = p.get("ws2")
+    if w is not None and w.numel() > 0:
         S, d, Is = w.shape
         q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
-        sc = torch.empty(d, dtype=torch.float32, device=w.device)
-        moe_quantize_fp8(w, d, Is, S, q, sc, stream)
+        sc = fp8_scales(d, S * Is, MOE_SF_WEIGHTS, w.device)
+        moe_quantize_fp8(w, d, Is, S, MOE_SF_WEIGHTS, q, sc, stream)
         out["ws2q"], out["ws2s"] = q, sc
     return out
 

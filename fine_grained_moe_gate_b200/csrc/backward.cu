@@ -480,6 +480,151 @@ __global__ void balance_sum_kernel(const float* __restrict__ part, int nb, float
     *loss = v / (float)nb;
 }
 
+// ------------------------------------------------------------------ tensor-core path (bf16 layers)
+//
+// The routed rows live in a padded layout for the tensor-core GEMMs: expert
+// e's rows start at pstart[e] = sum_{e' < e} ceil64(counts[e']), so the
+// weight-gradient GEMMs can run their contraction over whole 64-row stages
+// of zeros past each expert's rows.  prow[r] maps a permuted row to its
+// padded row.
+
+constexpr int kPad = 64;
+
+// One block: pstart[e] (exclusive scan of the rounded-up counts), pstart[E] = total.
+__global__ void pad_plan_kernel(const int32_t* __restrict__ counts, int E, int32_t* __restrict__ pstart, int* status) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+        pstart[e] = acc;
+        int c = counts[e];
+        if (c < 0) {
+            report(status, kStDeviceCheck);
+            c = 0;
+        }
+        acc += (c + kPad - 1) / kPad * kPad;
+    }
+    pstart[E] = acc;
+}
+
+// last index i in [0, n) with a[i] <= v (a non-decreasing, a[0] <= v)
+__device__ __forceinline__ int last_le(const int32_t* a, int n, int v) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a[mid] <= v) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// One warp per permuted row r: prow[r] = its padded row; x_pad[prow[r]] = x[perm[r] / k] (bf16, 16-byte copies).
+__global__ void gather_pad_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm,
+                                  const int32_t* __restrict__ offsets, const int32_t* __restrict__ pstart, int E,
+                                  int k, int R, int T, int vec, int32_t* __restrict__ prow, uint4* __restrict__ xp,
+                                  int* status) {
+    const int lane = threadIdx.x & 31;
+    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += gridDim.x * (blockDim.x >> 5)) {
+        const int e = last_le(offsets, E, r);
+        const int pr = pstart[e] + (r - offsets[e]);
+        const int t = perm[r] / k;
+        if (t < 0 || t >= T) {
+            if (lane == 0) report(status, kStDeviceCheck);
+            continue;
+        }
+        if (lane == 0) prow[r] = pr;
+        for (int v = lane; v < vec; v += 32) xp[(size_t)pr * vec + v] = x[(size_t)t * vec + v];
+    }
+}
+
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// h[pr] = bf16(silu(a[pr]) * g[pr]) for the real rows (prow; null: rows 0..R-1), n columns, 4 at a time.
+__global__ void swiglu_h_kernel(const float* __restrict__ a, const float* __restrict__ g,
+                                const int32_t* __restrict__ prow, int R, int n, uint2* __restrict__ h) {
+    const int n4 = n / 4;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)R * n4;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int r = (int)(i / n4), c = (int)(i - (long long)r * n4);
+        const long long pr = prow ? prow[r] : r;
+        const float4 av = reinterpret_cast<const float4*>(a + pr * n)[c];
+        const float4 gv = reinterpret_cast<const float4*>(g + pr * n)[c];
+        h[pr * n4 + c] = make_uint2(bf16x2(av.x * sigmoid_acc(av.x) * gv.x, av.y * sigmoid_acc(av.y) * gv.y),
+                                    bf16x2(av.z * sigmoid_acc(av.z) * gv.z, av.w * sigmoid_acc(av.w) * gv.w));
+    }
+}
+
+// One block per assignment q = t*k + j (row r = inv[q], padded row pr):
+// dw[q] = <dy_t, o[pr]>, do[pr] = bf16(w[q] dy_t).
+__global__ void __launch_bounds__(256) combine_bwd_pad_kernel(const float* __restrict__ dy, const float* __restrict__ w,
+                                                              const int32_t* __restrict__ inv,
+                                                              const int32_t* __restrict__ prow,
+                                                              const float* __restrict__ o, float* __restrict__ dw,
+                                                              uint16_t* __restrict__ dop, int d, int k, int rows,
+                                                              int* status) {
+    __shared__ float red[32];
+    const int q = blockIdx.x, t = q / k;
+    const int r = inv[q];
+    if (r < 0 || r >= rows) {
+        if (threadIdx.x == 0) report(status, kStDeviceCheck);
+        return;
+    }
+    const long long pr = prow[r];
+    const float* dyt = dy + (long long)t * d;
+    const float* orow = o + pr * d;
+    float part = 0.0f;
+    for (int c = threadIdx.x; c < d; c += blockDim.x) part = fmaf(dyt[c], orow[c], part);
+    const float tot = block_sum(part, red);
+    if (threadIdx.x == 0) dw[q] = tot;
+    const float wq = w[q];
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(dop + pr * d);
+    for (int c = threadIdx.x; c < d; c += blockDim.x) dst[c] = __float2bfloat16_rn(wq * dyt[c]);
+}
+
+// SwiGLU derivative on the real rows: with s = sigmoid(a),
+//   da = dh g s (1 + a (1 - s)),  dg = dh a s,
+// stored bf16 side by side: dadg[pr][c] = da, dadg[pr][n + c] = dg.
+__global__ void swiglu_bwd_pad_kernel(const float* __restrict__ a, const float* __restrict__ g,
+                                      const float* __restrict__ dh, const int32_t* __restrict__ prow, int R, int n,
+                                      uint16_t* __restrict__ dadg) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)R * n;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int r = (int)(i / n), c = (int)(i - (long long)r * n);
+        const long long pr = prow ? prow[r] : r;
+        const float av = a[pr * n + c], gv = g[pr * n + c], dv = dh[pr * n + c];
+        const float s = sigmoid_acc(av);
+        __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(dadg + pr * 2 * n);
+        row[c] = __float2bfloat16_rn(dv * gv * s * (1.0f + av * (1.0f - s)));
+        row[n + c] = __float2bfloat16_rn(dv * av * s);
+    }
+}
+
+// y = bf16(x), n elements (fp32 dy of the shared experts, whose weight is 1).
+__global__ void to_bf16_kernel(const float* __restrict__ x, long long n, __nv_bfloat16* __restrict__ y) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        y[i] = __float2bfloat16_rn(x[i]);
+}
+
+// dx[t] = sum_j dxp[prow[inv[t*k + j]]] (overwrite), one block per token.
+__global__ void unpermute_sum_pad_kernel(const float* __restrict__ dxp, const int32_t* __restrict__ inv,
+                                         const int32_t* __restrict__ prow, float* dx, int d, int k, int rows,
+                                         int* status) {
+    const int t = blockIdx.x;
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+        float v = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int r = inv[(long long)t * k + j];
+            if (r < 0 || r >= rows) {
+                report(status, kStDeviceCheck);
+                continue;
+            }
+            v += dxp[(long long)prow[r] * d + c];
+        }
+        dx[(long long)t * d + c] = v;
+    }
+}
+
 // ------------------------------------------------------------------ launch helpers
 
 Opnd view(const void* p, bool bf16, long long rs, long long cs, long long gs = 0, const int32_t* gather = nullptr,
@@ -518,49 +663,277 @@ int ew_grid(long long n) {
 
 }  // namespace
 
-size_t backward_scratch_bytes(int T, int d, int E, int k, int I, int S, int Is, int seq_len) {
-    auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
+// Whether the expert contractions run on the tensor cores: bf16 layers whose
+// widths fit the 128-column tiles of the MN-major operands.
+bool backward_on_tensor_cores(bool bf16, int d, int I, int S, int Is) {
+    return bf16 && d % 128 == 0 && I % 128 == 0 && (S == 0 || Is % 128 == 0);
+}
+
+namespace {
+struct BwdCarve {
+    char* p;
+    size_t used = 0;
+    template <typename T>
+    T* take(size_t bytes) {
+        const size_t al = (bytes + 255) & ~size_t(255);
+        T* q = reinterpret_cast<T*>(p ? p + used : nullptr);
+        used += al;
+        return q;
+    }
+};
+
+// Buffers of the backward, carved from the workspace in this order (the
+// sizes depend on the path: fp32 SIMT, or the tensor cores' padded bf16 layout).
+struct BwdBufs {
+    int32_t *offsets, *perm, *inv, *pscratch, *cnt;
+    float *dw, *dz, *tot, *part, *chunk;
+    // SIMT path
+    float *abuf, *gbuf, *hbuf, *dhbuf, *obuf, *as, *gs, *hs, *dhs;
+    // tensor-core path: routed rows in the padded layout (Rp rows), shared rows T
+    int32_t *pstart, *prow;
+    uint16_t *x_pad, *h_pad, *do_pad, *dadg, *hs16, *dys16, *dadgs;
+    float *a_pad, *g_pad, *o_pad, *dh_pad, *as32, *gs32, *dhs32;
+};
+
+size_t carve(BwdBufs* o, char* base, int T, int d, int E, int k, int I, int S, int Is, int seq_len, bool tc) {
+    BwdCarve c{base};
     const size_t R = (size_t)T * k;
     const size_t nb = seq_len > 0 ? (size_t)T / seq_len : 0;
     const size_t C = seq_len > 0 ? ((size_t)seq_len + kLossChunk - 1) / kLossChunk : 0;
-    return al((E + 1) * 4) + 2 * al(R * 4) + al(permute_scratch_bytes(T, E)) + 4 * al(R * I * 4) + al(R * d * 4) +
-           al(R * 4) + 4 * al((size_t)T * S * Is * 4) + al((size_t)T * E * 4) + al((size_t)T * 4) + al(nb * E * 4) +
-           al(nb * 4) + al(nb * C * E * 4);
+    const size_t SI = (size_t)S * Is;
+    BwdBufs b{};
+    b.offsets = c.take<int32_t>((E + 1) * 4);
+    b.perm = c.take<int32_t>(R * 4);
+    b.inv = c.take<int32_t>(R * 4);
+    b.pscratch = c.take<int32_t>(permute_scratch_bytes(T, E));
+    b.dw = c.take<float>(R * 4);
+    b.dz = c.take<float>((size_t)T * E * 4);
+    b.tot = c.take<float>((size_t)T * 4);
+    b.cnt = c.take<int32_t>(nb * E * 4);
+    b.part = c.take<float>(nb * 4);
+    b.chunk = c.take<float>(nb * C * E * 4);
+    if (!tc) {
+        b.abuf = c.take<float>(R * I * 4);
+        b.gbuf = c.take<float>(R * I * 4);
+        b.hbuf = c.take<float>(R * I * 4);
+        b.dhbuf = c.take<float>(R * I * 4);
+        b.obuf = c.take<float>(R * d * 4);
+        b.as = c.take<float>((size_t)T * SI * 4);
+        b.gs = c.take<float>((size_t)T * SI * 4);
+        b.hs = c.take<float>((size_t)T * SI * 4);
+        b.dhs = c.take<float>((size_t)T * SI * 4);
+    } else {
+        const size_t Rp = R + (size_t)kPad * E;  // padded rows: at most kPad - 1 more per expert
+        b.pstart = c.take<int32_t>((E + 1) * 4);
+        b.prow = c.take<int32_t>(R * 4);
+        b.x_pad = c.take<uint16_t>(Rp * d * 2);
+        b.h_pad = c.take<uint16_t>(Rp * I * 2);
+        b.do_pad = c.take<uint16_t>(Rp * d * 2);
+        b.dadg = c.take<uint16_t>(Rp * 2 * I * 2);
+        b.a_pad = c.take<float>(Rp * I * 4);
+        b.g_pad = c.take<float>(Rp * I * 4);
+        b.dh_pad = c.take<float>(Rp * I * 4);
+        b.o_pad = c.take<float>(Rp * d * 4);
+        b.as32 = c.take<float>((size_t)T * SI * 4);
+        b.gs32 = c.take<float>((size_t)T * SI * 4);
+        b.dhs32 = c.take<float>((size_t)T * SI * 4);
+        b.hs16 = c.take<uint16_t>((size_t)T * SI * 2);
+        b.dys16 = c.take<uint16_t>((size_t)T * d * 2);
+        b.dadgs = c.take<uint16_t>((size_t)T * 2 * SI * 2);
+    }
+    if (o) *o = b;
+    return c.used;
 }
+}  // namespace
+
+size_t backward_scratch_bytes(int T, int d, int E, int k, int I, int S, int Is, int seq_len, bool bf16) {
+    return carve(nullptr, nullptr, T, d, E, k, I, S, Is, seq_len, backward_on_tensor_cores(bf16, d, I, S, Is));
+}
+
+namespace {
+
+// The expert part of the backward on the tensor cores (bf16 layer): writes
+// dw (per assignment), dx (routed + shared), dW1/dW3/dW2 and the shared
+// gradients.  bf16 operands (x, h, do = w dy, da, dg, the shared dy), fp32
+// accumulation and fp32 results.
+cudaError_t experts_backward_tc(const BackwardArgs& a, const BwdBufs& b, int* status, int num_sms, cudaStream_t st) {
+    const int T = a.T, d = a.d, E = a.E, k = a.k, I = a.I, S = a.S, Is = a.Is;
+    const int R = T * k;
+    const long long Rp = (long long)R + (long long)kPad * E;
+    const int SI = S * Is;
+    cudaError_t err;
+#define TC_TRY(x)                                  \
+    do {                                           \
+        if ((err = (x)) != cudaSuccess) return err; \
+    } while (0)
+    // padded layout of the routed rows, and the zero padding of the GEMM operands
+    pad_plan_kernel<<<1, 32, 0, st>>>(a.counts, E, b.pstart, status);
+    note_launches(1);
+    TC_TRY(cudaMemsetAsync(b.x_pad, 0, (size_t)Rp * d * 2, st));
+    TC_TRY(cudaMemsetAsync(b.h_pad, 0, (size_t)Rp * I * 2, st));
+    TC_TRY(cudaMemsetAsync(b.do_pad, 0, (size_t)Rp * d * 2, st));
+    TC_TRY(cudaMemsetAsync(b.dadg, 0, (size_t)Rp * 2 * I * 2, st));
+    if (R > 0) {
+        gather_pad_kernel<<<num_sms * 4, 256, 0, st>>>(static_cast<const uint4*>(a.x), b.perm, b.offsets, b.pstart,
+                                                       E, k, R, T, d / 8, b.prow, reinterpret_cast<uint4*>(b.x_pad),
+                                                       status);
+        note_launches(1);
+    }
+    auto rows_args = [&](const void* W, long long W_rows, long long a_grow, const void* X, long long op_rows, int K,
+                         int M_total, float* out, bool routed) {
+        BwdRowsArgs r{};
+        r.W = W;
+        r.W1 = nullptr;
+        r.W_rows = W_rows;
+        r.K0 = 0;
+        r.a_grow = a_grow;
+        r.X = X;
+        r.op_rows = op_rows;
+        r.K = K;
+        r.M_total = M_total;
+        r.start = routed ? b.pstart : nullptr;
+        r.rows = routed ? a.counts : nullptr;
+        r.G = routed ? E : 1;
+        r.M_rows = routed ? 0 : T;
+        r.out = out;
+        r.ldo = M_total;
+        r.accumulate = false;
+        return r;
+    };
+    auto wgrad_args = [&](const void* A, int lda, long long a_col0, const void* B, int ldb, long long b_col0,
+                          long long op_rows, int M_total, int N_total, float* out, bool routed) {
+        BwdWgradArgs w{};
+        w.A = A;
+        w.lda = lda;
+        w.a_col0 = a_col0;
+        w.B = B;
+        w.ldb = ldb;
+        w.b_col0 = b_col0;
+        w.op_rows = op_rows;
+        w.M_total = M_total;
+        w.N_total = N_total;
+        w.start = routed ? b.pstart : nullptr;
+        w.rows = routed ? a.counts : nullptr;
+        w.G = routed ? E : 1;
+        w.M_rows = routed ? 0 : T;
+        w.out = out;
+        return w;
+    };
+
+    // ---- routed experts
+    // recompute a = x W1^T, g = x W3^T (fp32), h = bf16(silu(a) g) as the forward, o = h W2^T (fp32)
+    TC_TRY(launch_bwd_rows_kmajor(rows_args(a.w1, (long long)E * I, I, b.x_pad, Rp, d, I, b.a_pad, true), status,
+                                  num_sms, st));
+    TC_TRY(launch_bwd_rows_kmajor(rows_args(a.w3, (long long)E * I, I, b.x_pad, Rp, d, I, b.g_pad, true), status,
+                                  num_sms, st));
+    if (R > 0) {
+        swiglu_h_kernel<<<ew_grid((long long)R * I / 4), 256, 0, st>>>(b.a_pad, b.g_pad, b.prow, R, I,
+                                                                       reinterpret_cast<uint2*>(b.h_pad));
+        note_launches(1);
+    }
+    TC_TRY(launch_bwd_rows_kmajor(rows_args(a.w2, (long long)E * d, d, b.h_pad, Rp, I, d, b.o_pad, true), status,
+                                  num_sms, st));
+    // dw = <dy, o> per assignment; do = w dy (bf16, padded rows)
+    if (R > 0) {
+        combine_bwd_pad_kernel<<<R, 256, 0, st>>>(a.dy, a.w, b.inv, b.prow, b.o_pad, b.dw, b.do_pad, d, k, R, status);
+        note_launches(1);
+    }
+    // dW2_e = do^T h
+    TC_TRY(launch_bwd_wgrad(wgrad_args(b.do_pad, d, 0, b.h_pad, I, 0, Rp, d, I, a.dw2, true), status, num_sms, st));
+    // dh = do W2_e (W2 read along its output dimension)
+    {
+        BwdRowsArgs r = rows_args(a.w2, (long long)E * d, d, b.do_pad, Rp, d, I, b.dh_pad, true);
+        TC_TRY(launch_bwd_rows_mnmajor(r, status, num_sms, st));
+    }
+    if (R > 0) {
+        swiglu_bwd_pad_kernel<<<ew_grid((long long)R * I), 256, 0, st>>>(b.a_pad, b.g_pad, b.dh_pad, b.prow, R, I,
+                                                                         b.dadg);
+        note_launches(1);
+    }
+    // dW1_e = da^T x, dW3_e = dg^T x
+    TC_TRY(launch_bwd_wgrad(wgrad_args(b.dadg, 2 * I, 0, b.x_pad, d, 0, Rp, I, d, a.dw1, true), status, num_sms, st));
+    TC_TRY(launch_bwd_wgrad(wgrad_args(b.dadg, 2 * I, I, b.x_pad, d, 0, Rp, I, d, a.dw3, true), status, num_sms, st));
+    // dx_perm = da W1_e + dg W3_e (the o buffer), then summed back per token
+    {
+        BwdRowsArgs r = rows_args(a.w1, (long long)E * I, I, b.dadg, Rp, 2 * I, d, b.o_pad, true);
+        r.W1 = a.w3;
+        r.K0 = I;
+        TC_TRY(launch_bwd_rows_mnmajor(r, status, num_sms, st));
+    }
+    if (T > 0) {
+        unpermute_sum_pad_kernel<<<T, 256, 0, st>>>(b.o_pad, b.inv, b.prow, a.dx, d, k, R, status);
+        note_launches(1);
+    }
+
+    // ---- shared experts: one group of T rows (rows past T read as zeros), S blocks stacked along the features
+    if (S > 0 && T > 0) {
+        TC_TRY(launch_bwd_rows_kmajor(rows_args(a.ws1, SI, 0, a.x, T, d, SI, b.as32, false), status, num_sms, st));
+        TC_TRY(launch_bwd_rows_kmajor(rows_args(a.ws3, SI, 0, a.x, T, d, SI, b.gs32, false), status, num_sms, st));
+        swiglu_h_kernel<<<ew_grid((long long)T * SI / 4), 256, 0, st>>>(b.as32, b.gs32, nullptr, T, SI,
+                                                                        reinterpret_cast<uint2*>(b.hs16));
+        to_bf16_kernel<<<ew_grid((long long)T * d), 256, 0, st>>>(a.dy, (long long)T * d,
+                                                                  reinterpret_cast<__nv_bfloat16*>(b.dys16));
+        note_launches(2);
+        const size_t eb = 2;
+        for (int s = 0; s < S; ++s) {
+            const char* w2s = static_cast<const char*>(a.ws2) + eb * (size_t)s * d * Is;
+            // dWs2_s = dy^T hs_s
+            TC_TRY(launch_bwd_wgrad(wgrad_args(b.dys16, d, 0, b.hs16, SI, (long long)s * Is, T, d, Is,
+                                               a.dws2 + (size_t)s * d * Is, false),
+                                    status, num_sms, st));
+            // dhs_s = dy Ws2_s
+            BwdRowsArgs r = rows_args(w2s, d, 0, b.dys16, T, d, Is, b.dhs32 + (size_t)s * Is, false);
+            r.ldo = SI;
+            TC_TRY(launch_bwd_rows_mnmajor(r, status, num_sms, st));
+        }
+        swiglu_bwd_pad_kernel<<<ew_grid((long long)T * SI), 256, 0, st>>>(b.as32, b.gs32, b.dhs32, nullptr, T, SI,
+                                                                          b.dadgs);
+        note_launches(1);
+        TC_TRY(launch_bwd_wgrad(wgrad_args(b.dadgs, 2 * SI, 0, a.x, d, 0, T, SI, d, a.dws1, false), status, num_sms,
+                                st));
+        TC_TRY(launch_bwd_wgrad(wgrad_args(b.dadgs, 2 * SI, SI, a.x, d, 0, T, SI, d, a.dws3, false), status, num_sms,
+                                st));
+        BwdRowsArgs r = rows_args(a.ws1, SI, 0, b.dadgs, T, 2 * SI, d, a.dx, false);
+        r.W1 = a.ws3;
+        r.K0 = SI;
+        r.accumulate = true;
+        TC_TRY(launch_bwd_rows_mnmajor(r, status, num_sms, st));
+    }
+#undef TC_TRY
+    return cudaSuccess;
+}
+
+}  // namespace
 
 cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sms, cudaStream_t st) {
     const int T = a.T, d = a.d, E = a.E, k = a.k, I = a.I, S = a.S, Is = a.Is;
     const bool bf = a.bf16;
     const int R = T * k;
     const int nb = a.alpha > 0.0f ? T / a.seq_len : 0;
-    auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
-    char* p = static_cast<char*>(a.workspace);
-    auto take = [&](size_t bytes) {
-        char* q = p;
-        p += al(bytes);
-        return q;
-    };
-    int32_t* offsets = reinterpret_cast<int32_t*>(take((E + 1) * 4));
-    int32_t* perm = reinterpret_cast<int32_t*>(take((size_t)R * 4));
-    int32_t* inv = reinterpret_cast<int32_t*>(take((size_t)R * 4));
-    int32_t* pscratch = reinterpret_cast<int32_t*>(take(permute_scratch_bytes(T, E)));
-    float* abuf = reinterpret_cast<float*>(take((size_t)R * I * 4));
-    float* gbuf = reinterpret_cast<float*>(take((size_t)R * I * 4));
-    float* hbuf = reinterpret_cast<float*>(take((size_t)R * I * 4));
-    float* dhbuf = reinterpret_cast<float*>(take((size_t)R * I * 4));
-    float* obuf = reinterpret_cast<float*>(take((size_t)R * d * 4));
-    float* dw = reinterpret_cast<float*>(take((size_t)R * 4));
-    const int SI = S * Is;
-    float* as = reinterpret_cast<float*>(take((size_t)T * SI * 4));
-    float* gs = reinterpret_cast<float*>(take((size_t)T * SI * 4));
-    float* hs = reinterpret_cast<float*>(take((size_t)T * SI * 4));
-    float* dhs = reinterpret_cast<float*>(take((size_t)T * SI * 4));
-    float* dz = reinterpret_cast<float*>(take((size_t)T * E * 4));
-    float* tot = reinterpret_cast<float*>(take((size_t)T * 4));
-    int32_t* cnt = reinterpret_cast<int32_t*>(take((size_t)nb * E * 4));
-    float* part = reinterpret_cast<float*>(take((size_t)nb * 4));
+    const bool tc = backward_on_tensor_cores(bf, d, I, S, Is);
+    BwdBufs bb;
+    carve(&bb, static_cast<char*>(a.workspace), T, d, E, k, I, S, Is, a.alpha > 0.0f ? a.seq_len : 0, tc);
+    int32_t* offsets = bb.offsets;
+    int32_t* perm = bb.perm;
+    int32_t* inv = bb.inv;
+    int32_t* pscratch = bb.pscratch;
+    float* dw = bb.dw;
+    float* dz = bb.dz;
+    float* tot = bb.tot;
+    int32_t* cnt = bb.cnt;
+    float* part = bb.part;
+    float* chunk = bb.chunk;
     const int C = nb > 0 ? (a.seq_len + kLossChunk - 1) / kLossChunk : 0;
-    float* chunk = reinterpret_cast<float*>(take((size_t)nb * C * E * 4));
+    float* abuf = bb.abuf;
+    float* gbuf = bb.gbuf;
+    float* hbuf = bb.hbuf;
+    float* dhbuf = bb.dhbuf;
+    float* obuf = bb.obuf;
+    const int SI = S * Is;
+    float* as = bb.as;
+    float* gs = bb.gs;
+    float* hs = bb.hs;
+    float* dhs = bb.dhs;
 
     cudaError_t err;
 #define BWD_TRY(x)                          \
@@ -572,70 +945,74 @@ cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sm
     BWD_TRY(launch_permute(nullptr, a.idx, a.counts, T, d, E, k, bf ? 2 : 4, nullptr, offsets, perm, inv, pscratch,
                            status, st));
 
-    // ---- routed experts
-    const Opnd xg = view(a.x, bf, d, 1, 0, perm, k);  // x row of permuted row r
-    BWD_TRY(rows_gemm(xg, view(a.w1, bf, d, 1, (long long)I * d), abuf, I, R, I, d, offsets, E, false, status,
-                      a.num_sms, st));
-    BWD_TRY(rows_gemm(xg, view(a.w3, bf, d, 1, (long long)I * d), gbuf, I, R, I, d, offsets, E, false, status,
-                      a.num_sms, st));
-    swiglu_fwd_kernel<<<ew_grid((long long)R * I), 256, 0, st>>>(abuf, gbuf, hbuf, (long long)R * I, bf ? 1 : 0);
-    note_launches(1);
-    // o = h W2_e^T
-    BWD_TRY(rows_gemm(view(hbuf, false, I, 1), view(a.w2, bf, I, 1, (long long)d * I), obuf, d, R, d, I, offsets, E,
-                      false, status, a.num_sms, st));
-    if (R > 0) {
-        combine_bwd_kernel<<<R, 256, 0, st>>>(a.dy, a.w, inv, obuf, dw, d, k, R, status);
+    if (tc) {
+        BWD_TRY(experts_backward_tc(a, bb, status, num_sms, st));
+    } else {
+        // ---- routed experts
+        const Opnd xg = view(a.x, bf, d, 1, 0, perm, k);  // x row of permuted row r
+        BWD_TRY(rows_gemm(xg, view(a.w1, bf, d, 1, (long long)I * d), abuf, I, R, I, d, offsets, E, false, status,
+                          a.num_sms, st));
+        BWD_TRY(rows_gemm(xg, view(a.w3, bf, d, 1, (long long)I * d), gbuf, I, R, I, d, offsets, E, false, status,
+                          a.num_sms, st));
+        swiglu_fwd_kernel<<<ew_grid((long long)R * I), 256, 0, st>>>(abuf, gbuf, hbuf, (long long)R * I, bf ? 1 : 0);
         note_launches(1);
-    }
-    // dW2_e[c][i] = sum_r do[r][c] h[r][i]
-    BWD_TRY(wgrad_gemm(view(obuf, false, d, 1), view(hbuf, false, I, 1), a.dw2, I, (long long)d * I, d, I, offsets, E,
-                       R, false, status, st));
-    // dh[r][i] = sum_c do[r][c] W2_e[c][i]
-    BWD_TRY(rows_gemm(view(obuf, false, d, 1), view(a.w2, bf, 1, I, (long long)d * I), dhbuf, I, R, I, d, offsets, E,
-                      false, status, a.num_sms, st));
-    swiglu_bwd_kernel<<<ew_grid((long long)R * I), 256, 0, st>>>(abuf, gbuf, dhbuf, (long long)R * I);
-    note_launches(1);
-    // dW1_e = da^T x, dW3_e = dg^T x
-    BWD_TRY(wgrad_gemm(view(dhbuf, false, I, 1), xg, a.dw1, d, (long long)I * d, I, d, offsets, E, R, false, status,
-                       st));
-    BWD_TRY(wgrad_gemm(view(gbuf, false, I, 1), xg, a.dw3, d, (long long)I * d, I, d, offsets, E, R, false, status,
-                       st));
-    // dx_perm = da W1_e + dg W3_e  (into the do buffer, no longer needed)
-    BWD_TRY(rows_gemm(view(dhbuf, false, I, 1), view(a.w1, bf, 1, d, (long long)I * d), obuf, d, R, d, I, offsets, E,
-                      false, status, a.num_sms, st));
-    BWD_TRY(rows_gemm(view(gbuf, false, I, 1), view(a.w3, bf, 1, d, (long long)I * d), obuf, d, R, d, I, offsets, E,
-                      true, status, a.num_sms, st));
-    if (T > 0) {
-        unpermute_sum_kernel<<<T, 256, 0, st>>>(obuf, inv, a.dx, d, k, R, status);
+        // o = h W2_e^T
+        BWD_TRY(rows_gemm(view(hbuf, false, I, 1), view(a.w2, bf, I, 1, (long long)d * I), obuf, d, R, d, I, offsets, E,
+                          false, status, a.num_sms, st));
+        if (R > 0) {
+            combine_bwd_kernel<<<R, 256, 0, st>>>(a.dy, a.w, inv, obuf, dw, d, k, R, status);
+            note_launches(1);
+        }
+        // dW2_e[c][i] = sum_r do[r][c] h[r][i]
+        BWD_TRY(wgrad_gemm(view(obuf, false, d, 1), view(hbuf, false, I, 1), a.dw2, I, (long long)d * I, d, I, offsets, E,
+                           R, false, status, st));
+        // dh[r][i] = sum_c do[r][c] W2_e[c][i]
+        BWD_TRY(rows_gemm(view(obuf, false, d, 1), view(a.w2, bf, 1, I, (long long)d * I), dhbuf, I, R, I, d, offsets, E,
+                          false, status, a.num_sms, st));
+        swiglu_bwd_kernel<<<ew_grid((long long)R * I), 256, 0, st>>>(abuf, gbuf, dhbuf, (long long)R * I);
         note_launches(1);
-    }
+        // dW1_e = da^T x, dW3_e = dg^T x
+        BWD_TRY(wgrad_gemm(view(dhbuf, false, I, 1), xg, a.dw1, d, (long long)I * d, I, d, offsets, E, R, false, status,
+                           st));
+        BWD_TRY(wgrad_gemm(view(gbuf, false, I, 1), xg, a.dw3, d, (long long)I * d, I, d, offsets, E, R, false, status,
+                           st));
+        // dx_perm = da W1_e + dg W3_e  (into the do buffer, no longer needed)
+        BWD_TRY(rows_gemm(view(dhbuf, false, I, 1), view(a.w1, bf, 1, d, (long long)I * d), obuf, d, R, d, I, offsets, E,
+                          false, status, a.num_sms, st));
+        BWD_TRY(rows_gemm(view(gbuf, false, I, 1), view(a.w3, bf, 1, d, (long long)I * d), obuf, d, R, d, I, offsets, E,
+                          true, status, a.num_sms, st));
+        if (T > 0) {
+            unpermute_sum_kernel<<<T, 256, 0, st>>>(obuf, inv, a.dx, d, k, R, status);
+            note_launches(1);
+        }
 
-    // ---- shared experts: one group of T rows, the S blocks stacked along the features
-    if (S > 0) {
-        const Opnd x = view(a.x, bf, d, 1);
-        BWD_TRY(rows_gemm(x, view(a.ws1, bf, d, 1), as, SI, T, SI, d, nullptr, 1, false, status, a.num_sms, st));
-        BWD_TRY(rows_gemm(x, view(a.ws3, bf, d, 1), gs, SI, T, SI, d, nullptr, 1, false, status, a.num_sms, st));
-        swiglu_fwd_kernel<<<ew_grid((long long)T * SI), 256, 0, st>>>(as, gs, hs, (long long)T * SI, bf ? 1 : 0);
-        note_launches(1);
-        const Opnd dyv = view(a.dy, false, d, 1);
-        const size_t eb = bf ? 2 : 4;
-        for (int s = 0; s < S; ++s) {
-            const char* w2s = static_cast<const char*>(a.ws2) + eb * (size_t)s * d * Is;
-            // dWs2_s[c][i] = sum_t dy[t][c] hs[t][s*Is + i]
-            BWD_TRY(wgrad_gemm(dyv, view(hs + (size_t)s * Is, false, SI, 1), a.dws2 + (size_t)s * d * Is, Is, 0, d,
-                               Is, nullptr, 1, T, false, status, st));
-            // dhs[t][s*Is + i] = sum_c dy[t][c] Ws2_s[c][i]
-            BWD_TRY(rows_gemm(dyv, view(w2s, bf, 1, Is), dhs + (size_t)s * Is, SI, T, Is, d, nullptr, 1, false, status,
+        // ---- shared experts: one group of T rows, the S blocks stacked along the features
+        if (S > 0) {
+            const Opnd x = view(a.x, bf, d, 1);
+            BWD_TRY(rows_gemm(x, view(a.ws1, bf, d, 1), as, SI, T, SI, d, nullptr, 1, false, status, a.num_sms, st));
+            BWD_TRY(rows_gemm(x, view(a.ws3, bf, d, 1), gs, SI, T, SI, d, nullptr, 1, false, status, a.num_sms, st));
+            swiglu_fwd_kernel<<<ew_grid((long long)T * SI), 256, 0, st>>>(as, gs, hs, (long long)T * SI, bf ? 1 : 0);
+            note_launches(1);
+            const Opnd dyv = view(a.dy, false, d, 1);
+            const size_t eb = bf ? 2 : 4;
+            for (int s = 0; s < S; ++s) {
+                const char* w2s = static_cast<const char*>(a.ws2) + eb * (size_t)s * d * Is;
+                // dWs2_s[c][i] = sum_t dy[t][c] hs[t][s*Is + i]
+                BWD_TRY(wgrad_gemm(dyv, view(hs + (size_t)s * Is, false, SI, 1), a.dws2 + (size_t)s * d * Is, Is, 0, d,
+                                   Is, nullptr, 1, T, false, status, st));
+                // dhs[t][s*Is + i] = sum_c dy[t][c] Ws2_s[c][i]
+                BWD_TRY(rows_gemm(dyv, view(w2s, bf, 1, Is), dhs + (size_t)s * Is, SI, T, Is, d, nullptr, 1, false, status,
+                                  a.num_sms, st));
+            }
+            swiglu_bwd_kernel<<<ew_grid((long long)T * SI), 256, 0, st>>>(as, gs, dhs, (long long)T * SI);
+            note_launches(1);
+            BWD_TRY(wgrad_gemm(view(dhs, false, SI, 1), x, a.dws1, d, 0, SI, d, nullptr, 1, T, false, status, st));
+            BWD_TRY(wgrad_gemm(view(gs, false, SI, 1), x, a.dws3, d, 0, SI, d, nullptr, 1, T, false, status, st));
+            BWD_TRY(rows_gemm(view(dhs, false, SI, 1), view(a.ws1, bf, 1, d), a.dx, d, T, d, SI, nullptr, 1, true, status,
+                              a.num_sms, st));
+            BWD_TRY(rows_gemm(view(gs, false, SI, 1), view(a.ws3, bf, 1, d), a.dx, d, T, d, SI, nullptr, 1, true, status,
                               a.num_sms, st));
         }
-        swiglu_bwd_kernel<<<ew_grid((long long)T * SI), 256, 0, st>>>(as, gs, dhs, (long long)T * SI);
-        note_launches(1);
-        BWD_TRY(wgrad_gemm(view(dhs, false, SI, 1), x, a.dws1, d, 0, SI, d, nullptr, 1, T, false, status, st));
-        BWD_TRY(wgrad_gemm(view(gs, false, SI, 1), x, a.dws3, d, 0, SI, d, nullptr, 1, T, false, status, st));
-        BWD_TRY(rows_gemm(view(dhs, false, SI, 1), view(a.ws1, bf, 1, d), a.dx, d, T, d, SI, nullptr, 1, true, status,
-                          a.num_sms, st));
-        BWD_TRY(rows_gemm(view(gs, false, SI, 1), view(a.ws3, bf, 1, d), a.dx, d, T, d, SI, nullptr, 1, true, status,
-                          a.num_sms, st));
     }
 
     // ---- router and balance loss

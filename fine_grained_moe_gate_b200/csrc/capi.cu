@@ -198,6 +198,24 @@ moe_status do_ffn_down(const void* h, const int32_t* offsets, const void* w2, co
     return v;
 }
 
+// Down projection with the weighted combine fused into its epilogue (tensor
+// cores): routed rows scaled by topk_w[perm_tok[r]] and added into acc at
+// token perm_tok[r] / k; shared rows (hs) added with weight 1.
+moe_status do_ffn_down_combine(const void* h, const int32_t* offsets, const void* w2, const void* hs,
+                               const void* ws2, const int32_t* perm_tok, const float* topk_w, const moe_shape& sh,
+                               float* acc, int* status, int sms, cudaStream_t st) {
+    if (sh.T == 0) return MOE_OK;
+    const bool shared = hs && sh.S > 0;
+    moe::TcDownArgs dr = tc_down_args(h, offsets, w2, sh, false, nullptr);
+    dr.acc = acc;
+    dr.row_tok = perm_tok;
+    dr.row_w = topk_w;
+    dr.row_k = sh.k;
+    moe::TcDownArgs ds = tc_down_args(hs, nullptr, ws2, sh, true, nullptr);
+    ds.acc = acc;
+    return moe::launch_tc_down(&dr, shared ? &ds : nullptr, status, sms, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1, const void* w3, const void* w2,
                      const void* x, const void* ws1, const void* ws3, const void* ws2, const moe_shape& sh,
                      void* y_perm, void* shared_out, void* ws, int* status, int sms, cudaStream_t st) {
@@ -213,41 +231,42 @@ moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1,
 
 // ---- FP8 experts -----------------------------------------------------------
 
-inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-moe_status do_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const float* xs, const int32_t* offsets,
+moe_status do_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const void* xs, const int32_t* offsets,
                          const uint8_t* xq, const moe_fp8_experts* w, const moe_shape& sh, void* h, void* hs,
                          int* status, int sms, cudaStream_t st) {
     if (sh.T == 0) return MOE_OK;
     const bool shared = xq && sh.S > 0;
     moe::TcUpArgs ur = tc_up_args(xq_perm, nullptr, offsets, w->w1, w->w3, sh, false, h);
     ur.f8 = true;
-    ur.w1s = w->w1_scale;
-    ur.w3s = w->w3_scale;
-    ur.xs = xs;
+    ur.w1s = static_cast<const uint8_t*>(w->w1_scale);
+    ur.w3s = static_cast<const uint8_t*>(w->w3_scale);
+    ur.xs = static_cast<const uint32_t*>(xs);
+    ur.xs_pitch = sh.T;
     ur.xs_idx = perm_tok;  // row r holds token perm_tok[r] / k
     ur.xs_div = sh.k;
     moe::TcUpArgs us = tc_up_args(xq, nullptr, nullptr, w->ws1, w->ws3, sh, true, hs);
     us.f8 = true;
-    us.w1s = w->ws1_scale;
-    us.w3s = w->ws3_scale;
-    us.xs = xs;
+    us.w1s = static_cast<const uint8_t*>(w->ws1_scale);
+    us.w3s = static_cast<const uint8_t*>(w->ws3_scale);
+    us.xs = static_cast<const uint32_t*>(xs);
+    us.xs_pitch = sh.T;
     return moe::launch_tc_up(&ur, shared ? &us : nullptr, status, sms, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-moe_status do_ffn_down_fp8(const uint8_t* hq, const float* h_scale, const int32_t* offsets, const uint8_t* hsq,
-                           const float* hs_scale, const moe_fp8_experts* w, const moe_shape& sh, void* y_perm,
+moe_status do_ffn_down_fp8(const uint8_t* hq, const void* h_scale, const int32_t* offsets, const uint8_t* hsq,
+                           const void* hs_scale, const moe_fp8_experts* w, const moe_shape& sh, void* y_perm,
                            void* shared_out, int* status, int sms, cudaStream_t st) {
     if (sh.T == 0) return MOE_OK;
     const bool shared = hsq && sh.S > 0;
     moe::TcDownArgs dr = tc_down_args(hq, offsets, w->w2, sh, false, y_perm);
     dr.f8 = true;
-    dr.w2s = w->w2_scale;
-    dr.hs = h_scale;
+    dr.w2s = static_cast<const uint8_t*>(w->w2_scale);
+    dr.hs = static_cast<const uint32_t*>(h_scale);
     moe::TcDownArgs ds = tc_down_args(hsq, nullptr, w->ws2, sh, true, shared_out);
     ds.f8 = true;
-    ds.w2s = w->ws2_scale;
-    ds.hs = hs_scale;
+    ds.w2s = static_cast<const uint8_t*>(w->ws2_scale);
+    ds.hs = static_cast<const uint32_t*>(hs_scale);
     return moe::launch_tc_down(&dr, shared ? &ds : nullptr, status, sms, st) == cudaSuccess ? MOE_OK
                                                                                               : MOE_ERR_CUDA;
 }
@@ -260,8 +279,8 @@ bool fp8_weights_ok(const moe_fp8_experts* w, const moe_shape& sh) {
 
 bool fp8_weights_aligned(const moe_fp8_experts* w) {
     return aligned16(w->w1) && aligned16(w->w3) && aligned16(w->w2) && aligned16(w->ws1) && aligned16(w->ws3) &&
-           aligned16(w->ws2) && aligned4(w->w1_scale) && aligned4(w->w3_scale) && aligned4(w->w2_scale) &&
-           aligned4(w->ws1_scale) && aligned4(w->ws3_scale) && aligned4(w->ws2_scale);
+           aligned16(w->ws2) && aligned16(w->w1_scale) && aligned16(w->w3_scale) && aligned16(w->w2_scale) &&
+           aligned16(w->ws1_scale) && aligned16(w->ws3_scale) && aligned16(w->ws2_scale);
 }
 
 // Workspace of moe_layer_forward_fp8, carved in this order.
@@ -271,23 +290,24 @@ struct Fp8Work {
     int32_t* inv;
     void* pws;
     uint8_t* xq;
-    float* xs;
+    void* xs;
     uint8_t* xq_perm;
     void* h;
     void* hs;
     uint8_t* hq;
-    float* h_scale;
+    void* h_scale;
     uint8_t* hsq;
-    float* hs_scale;
+    void* hs_scale;
     void* y_perm;
     void* shared_out;
 };
 
 size_t fp8_work(const moe_shape& sh, char* base, Fp8Work* o) {
     const size_t T = (size_t)sh.T, rows = T * sh.k, SI = (size_t)sh.S * sh.Is, d = (size_t)sh.d, I = (size_t)sh.I;
-    const size_t sizes[15] = {(size_t)(sh.E + 1) * 4, rows * 4, rows * 4, permute_ws(sh), T * d, T * 4,
-                              rows * d, rows * I * 2, T * SI * 2, rows * I, rows * 4, T * SI, T * 4,
-                              rows * d * 2, T * d * 2};
+    // token-layout tile scales: one 32-bit word per row and 128 columns
+    const size_t sizes[15] = {(size_t)(sh.E + 1) * 4, rows * 4, rows * 4, permute_ws(sh), T * d, T * (d / 128) * 4,
+                              rows * d, rows * I * 2, T * SI * 2, rows * I, rows * (I / 128) * 4, T * SI,
+                              T * (SI / 128) * 4, rows * d * 2, T * d * 2};
     void* ptrs[15];
     size_t off = 0;
     for (int i = 0; i < 15; ++i) {
@@ -300,14 +320,14 @@ size_t fp8_work(const moe_shape& sh, char* base, Fp8Work* o) {
         o->inv = static_cast<int32_t*>(ptrs[2]);
         o->pws = ptrs[3];
         o->xq = static_cast<uint8_t*>(ptrs[4]);
-        o->xs = static_cast<float*>(ptrs[5]);
+        o->xs = ptrs[5];
         o->xq_perm = static_cast<uint8_t*>(ptrs[6]);
         o->h = ptrs[7];
         o->hs = ptrs[8];
         o->hq = static_cast<uint8_t*>(ptrs[9]);
-        o->h_scale = static_cast<float*>(ptrs[10]);
+        o->h_scale = ptrs[10];
         o->hsq = static_cast<uint8_t*>(ptrs[11]);
-        o->hs_scale = static_cast<float*>(ptrs[12]);
+        o->hs_scale = ptrs[12];
         o->y_perm = ptrs[13];
         o->shared_out = ptrs[14];
     }
@@ -514,6 +534,43 @@ moe_status moe_ffn_down(const void* h, const int32_t* offsets, const void* w2, c
                        static_cast<cudaStream_t>(stream));
 }
 
+moe_status moe_ffn_down_combine(const void* h, const int32_t* offsets, const void* w2, const void* hs,
+                                const void* ws2, const int32_t* perm_tok, const float* topk_w, moe_shape sh,
+                                float* y_acc, void* stream) {
+    moe_status v = validate_dense_weights(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(sh.dtype == MOE_BF16, MOE_ERR_UNSUPPORTED);
+    const bool shared = hs != nullptr && sh.S > 0;
+    MOE_REQUIRE(offsets && w2, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (h && perm_tok && topk_w && y_acc), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(!shared || ws2, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(h) && aligned16(offsets) && aligned16(w2) && aligned16(hs) && aligned16(ws2) &&
+                    aligned16(perm_tok) && aligned16(topk_w) && aligned16(y_acc),
+                MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_ffn_down_combine(h, offsets, w2, shared ? hs : nullptr, ws2, perm_tok, topk_w, sh, y_acc, status, sms,
+                               static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine_finish(float* y_acc, moe_shape sh, void* y, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(sh.T == 0 || (y_acc && y), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(y_acc) && aligned16(y), MOE_ERR_ALIGNMENT);
+    MOE_REQUIRE(sh.d % 8 == 0, MOE_ERR_UNSUPPORTED);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return moe::launch_combine_finish(y_acc, (long long)sh.T * sh.d, sh.dtype != MOE_F32, y,
+                                      static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
 moe_status moe_combine(const void* y_perm, const float* topk_w, const int32_t* inv_row, const void* shared_out,
                        moe_shape sh, void* y, void* stream) {
     moe_status v = validate_shape(sh);
@@ -533,7 +590,8 @@ moe_status moe_combine(const void* y_perm, const float* topk_w, const int32_t* i
 
 size_t moe_backward_workspace_size(moe_shape sh, int32_t seq_len) {
     if (validate_dense_weights(sh) != MOE_OK) return 0;
-    return moe::backward_scratch_bytes(sh.T, sh.d, sh.E, sh.k, sh.I, sh.S, sh.Is, seq_len > 0 ? seq_len : 0);
+    return moe::backward_scratch_bytes(sh.T, sh.d, sh.E, sh.k, sh.I, sh.S, sh.Is, seq_len > 0 ? seq_len : 0,
+                                       sh.dtype == MOE_BF16);
 }
 
 moe_status moe_layer_backward(const void* x, const void* w_gate, const void* w1, const void* w3, const void* w2,
@@ -557,7 +615,7 @@ moe_status moe_layer_backward(const void* x, const void* w_gate, const void* w1,
                     aligned16(dws3) && aligned16(dws2),
                 MOE_ERR_ALIGNMENT);
     const int32_t L = alpha > 0.0f ? seq_len : 0;
-    const size_t need = moe::backward_scratch_bytes(sh.T, sh.d, sh.E, sh.k, sh.I, sh.S, sh.Is, L);
+    const size_t need = moe::backward_scratch_bytes(sh.T, sh.d, sh.E, sh.k, sh.I, sh.S, sh.Is, L, sh.dtype == MOE_BF16);
     MOE_REQUIRE(workspace && ws_bytes >= need, MOE_ERR_WORKSPACE);
     MOE_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, MOE_ERR_ALIGNMENT);
     int dev, sms;
@@ -659,24 +717,30 @@ moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bia
                : MOE_ERR_CUDA;
 }
 
-moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t kseg, int32_t nseg, uint8_t* q, float* scale,
-                            void* stream) {
+size_t moe_fp8_scale_bytes(int64_t rows, int32_t K, int32_t layout) {
+    if (rows < 0 || K <= 0 || K % 128 != 0 || (layout != MOE_SF_TOKENS && layout != MOE_SF_WEIGHTS)) return 0;
+    return moe::mx_scale_bytes(rows, K, layout == MOE_SF_WEIGHTS);
+}
+
+moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t kseg, int32_t nseg, int32_t layout, uint8_t* q,
+                            void* scales, void* stream) {
     MOE_REQUIRE(rows >= 0 && kseg > 0 && nseg >= 1, MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(kseg % 8 == 0, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(layout == MOE_SF_TOKENS || layout == MOE_SF_WEIGHTS, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(kseg % 128 == 0, MOE_ERR_UNSUPPORTED);
     MOE_REQUIRE((long long)kseg * nseg < (1ll << 31), MOE_ERR_UNSUPPORTED);
-    MOE_REQUIRE(rows == 0 || (src && q && scale), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(aligned16(src) && aligned16(q) && aligned4(scale), MOE_ERR_ALIGNMENT);
+    MOE_REQUIRE(rows == 0 || (src && q && scales), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(src) && aligned16(q) && aligned16(scales), MOE_ERR_ALIGNMENT);
     int dev, sms;
     int* status;
     moe_status v = device_setup(&dev, &status, &sms);
     if (v != MOE_OK) return v;
-    return moe::launch_quantize_e4m3(src, rows, kseg, nseg, q, scale, static_cast<cudaStream_t>(stream)) ==
-                   cudaSuccess
+    return moe::launch_quantize_mx(src, rows, kseg, nseg, layout == MOE_SF_WEIGHTS, q, scales,
+                                   static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }
 
-moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const float* x_scale,
+moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const void* x_scale,
                           const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w, moe_shape sh, void* h,
                           void* hs, void* stream) {
     moe_status v = validate_shape(sh);
@@ -686,7 +750,7 @@ moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const
     MOE_REQUIRE(sh.T == 0 || (xq_perm && perm_tok && x_scale && h), MOE_ERR_INVALID_ARG);
     const bool shared = xq != nullptr && sh.S > 0;
     MOE_REQUIRE(!shared || sh.T == 0 || hs, MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(aligned16(xq_perm) && aligned16(perm_tok) && aligned4(x_scale) && aligned16(offsets) &&
+    MOE_REQUIRE(aligned16(xq_perm) && aligned16(perm_tok) && aligned16(x_scale) && aligned16(offsets) &&
                     aligned16(xq) && aligned16(h) && aligned16(hs) && fp8_weights_aligned(w),
                 MOE_ERR_ALIGNMENT);
     int dev, sms;
@@ -697,8 +761,8 @@ moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const
                          static_cast<cudaStream_t>(stream));
 }
 
-moe_status moe_ffn_down_fp8(const uint8_t* hq, const float* h_scale, const int32_t* offsets, const uint8_t* hsq,
-                            const float* hs_scale, const moe_fp8_experts* w, moe_shape sh, void* y_perm,
+moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_scale, const int32_t* offsets, const uint8_t* hsq,
+                            const void* hs_scale, const moe_fp8_experts* w, moe_shape sh, void* y_perm,
                             void* shared_out, void* stream) {
     moe_status v = validate_shape(sh);
     if (v != MOE_OK) return v;
@@ -707,7 +771,7 @@ moe_status moe_ffn_down_fp8(const uint8_t* hq, const float* h_scale, const int32
     MOE_REQUIRE(sh.T == 0 || (hq && h_scale && y_perm), MOE_ERR_INVALID_ARG);
     const bool shared = hsq != nullptr && sh.S > 0;
     MOE_REQUIRE(!shared || sh.T == 0 || (hs_scale && shared_out), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(aligned16(hq) && aligned4(h_scale) && aligned16(offsets) && aligned16(hsq) && aligned4(hs_scale) &&
+    MOE_REQUIRE(aligned16(hq) && aligned16(h_scale) && aligned16(offsets) && aligned16(hsq) && aligned16(hs_scale) &&
                     aligned16(y_perm) && aligned16(shared_out) && fp8_weights_aligned(w),
                 MOE_ERR_ALIGNMENT);
     int dev, sms;
@@ -741,16 +805,17 @@ moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float*
     const bool shared = sh.S > 0;
     if ((v = do_route(x, w_gate, bias, sh, topk_idx, topk_w, counts, nullptr, status, sms, st)) != MOE_OK) return v;
     if (sh.T == 0) return MOE_OK;
-    if (moe::launch_quantize_e4m3(x, sh.T, sh.d, 1, k8.xq, k8.xs, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe::launch_quantize_mx(x, sh.T, sh.d, 1, false, k8.xq, k8.xs, st) != cudaSuccess) return MOE_ERR_CUDA;
     if ((v = do_permute(k8.xq, topk_idx, counts, sh, k8.xq_perm, k8.offsets, k8.perm, k8.inv, k8.pws, status, st)) !=
         MOE_OK)
         return v;
     if ((v = do_ffn_up_fp8(k8.xq_perm, k8.perm, k8.xs, k8.offsets, shared ? k8.xq : nullptr, w, sh, k8.h, k8.hs,
                            status, sms, st)) != MOE_OK)
         return v;
-    if (moe::launch_quantize_e4m3(k8.h, (long long)sh.T * sh.k, sh.I, 1, k8.hq, k8.h_scale, st) != cudaSuccess)
+    if (moe::launch_quantize_mx(k8.h, (long long)sh.T * sh.k, sh.I, 1, false, k8.hq, k8.h_scale, st) != cudaSuccess)
         return MOE_ERR_CUDA;
-    if (shared && moe::launch_quantize_e4m3(k8.hs, sh.T, sh.S * sh.Is, 1, k8.hsq, k8.hs_scale, st) != cudaSuccess)
+    if (shared &&
+        moe::launch_quantize_mx(k8.hs, sh.T, sh.S * sh.Is, 1, false, k8.hsq, k8.hs_scale, st) != cudaSuccess)
         return MOE_ERR_CUDA;
     if ((v = do_ffn_down_fp8(k8.hq, k8.h_scale, k8.offsets, shared ? k8.hsq : nullptr, k8.hs_scale, w, sh, k8.y_perm,
                              k8.shared_out, status, sms, st)) != MOE_OK)

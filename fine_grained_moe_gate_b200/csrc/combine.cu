@@ -111,6 +111,44 @@ void launch_t(const void* y_perm, const float* w, const int32_t* inv_row, const 
         combine_kernel<T, 16><<<T_, threads, 0, st>>>(yp, w, inv_row, sh, k, vec, T_ * k, out, status);
 }
 
+// Finish of the combine fused into the down projection's epilogue: the fp32
+// accumulator holds shared[t] + sum_j w[t][j] * o_j (added tile by tile), so
+// y = dtype(acc), one rounding; acc is then cleared for the next
+// accumulation.  Eight elements per thread and step (two 16-byte loads, one
+// or two 16-byte stores, two zero stores).  HBM bound: 4 + 4 + 2 (or 4)
+// bytes per element.
+template <typename T>
+__global__ void __launch_bounds__(256) combine_finish_kernel(float4* __restrict__ acc, long long n8,
+                                                             uint4* __restrict__ y) {
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+        const float4 a = acc[2 * i], b = acc[2 * i + 1];
+        acc[2 * i] = zero;
+        acc[2 * i + 1] = zero;
+        const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        if constexpr (Vec<T>::n == 8) {
+            y[i] = Vec<T>::pack(f);
+        } else {
+            y[2 * i] = Vec<T>::pack(f);
+            y[2 * i + 1] = Vec<T>::pack(f + 4);
+        }
+    }
+}
+
+cudaError_t launch_combine_finish(float* acc, long long n, bool bf16, void* y, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const long long n8 = n / 8;
+    const long long blocks = (n8 + 255) / 256 < 148 * 16 ? (n8 + 255) / 256 : 148 * 16;
+    if (bf16)
+        combine_finish_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<float4*>(acc), n8,
+                                                                              static_cast<uint4*>(y));
+    else
+        combine_finish_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<float4*>(acc), n8,
+                                                                      static_cast<uint4*>(y));
+    note_launches(1);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* inv_row, const void* shared, int T,
                            int d, int k, bool bf16, void* y, int* status, cudaStream_t st) {
     if (T == 0) return cudaSuccess;

@@ -182,12 +182,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-// kind::f8f6f4 with both operands E4M3 (format code 0 in the A and B type
-// fields), fp32 accumulator, K-major operands.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
-    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred;
     asm volatile(
@@ -267,16 +261,6 @@ __device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_des
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-// Same for two E4M3 operands (kind::f8f6f4, K = 32 per instruction).
-__device__ __forceinline__ void tc_mma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 // Arrive once on the barrier at this shared offset in every CTA of `mask`
 // when all tcgen05 ops issued so far by this thread are done.
 __device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t mask) {
@@ -286,6 +270,69 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t mask) {
         "h"(mask)
         : "memory");
 }
+// ---------------------------------------------------------------- block-scaled E4M3
+// Shared-memory descriptor of a 32-row x 16-byte matrix stored plainly (no
+// swizzle, K-major): 8-row core matrices of 128 contiguous bytes, the next 8
+// rows 128 bytes further (stride byte offset); one core matrix along the
+// row, so the leading byte offset is not used.
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(128u >> 4) << 16;
+    d |= (uint64_t)(128u >> 4) << 32;
+    d |= 1ull << 46;
+    return d;
+}
+// Copy a 32-row x 128-bit matrix from shared memory into tensor memory at
+// taddr (32 lanes x 4 columns), replicated into all four lane quarters; over
+// the CTA pair: each CTA's shared memory into its own tensor memory.
+// Issued by the leader CTA's MMA thread, ordered with its MMAs.
+__device__ __forceinline__ void tc_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Instruction descriptor, kind::mxf8f6f4 with block scaling: A and B E4M3
+// (format 0 in bits 7-9 and 10-12), K-major, N >> 3 in bits 17-22, the
+// scales unsigned powers of two (bit 23), M >> 4 in bits 24-28, and the byte
+// of each 32-bit scale column the MMA reads: B's in bits 4-5, A's in 29-30.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, uint32_t sfa_byte, uint32_t sfb_byte) {
+    return (sfb_byte << 4) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) |
+           (sfa_byte << 29);
+}
+// D[tmem] (+)= sum over the K = 32 step of A * B^T, each product scaled by
+// 2^(sa - 127) * 2^(sb - 127), sa / sb the scale bytes of the row of A and the
+// row of B held in tensor memory at sfa / sfb (the byte index in the top two
+// address bits, as in the descriptor).  CTA pair, issued by the even CTA.
+__device__ __forceinline__ void tc_mma_mx_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+// Ampere-style asynchronous copies of 4 or 8 bytes into shared memory;
+// src_bytes = 0 writes zeros (nothing is read).
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_8(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Arrive on the CTA-local mbarrier once every cp.async this thread issued so
+// far has landed (the barrier's expected count includes this arrive).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads (tcgen05.cp) of them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

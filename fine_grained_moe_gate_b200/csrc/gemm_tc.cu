@@ -72,7 +72,10 @@ constexpr int BK = 64;                  // bf16 K per stage: one 128-byte swizzl
 // K elements per stage for the operand type: 64 bf16 or 128 E4M3 (128 bytes either way)
 template <bool F8>
 __host__ __device__ constexpr int bk_elems() { return F8 ? 128 : 64; }
-constexpr int STAGES = 6;
+// Ring depth of the operand tiles: the E4M3 kernel keeps a ring of tile scales beside
+// it and runs 5 stages
+template <bool F8>
+__host__ __device__ constexpr int n_stages() { return F8 ? 5 : 6; }
 constexpr int A_BYTES = 128 * BK * 2;   // this CTA's 128 weight rows
 constexpr int B_ROWS = 128;             // this CTA's half of <= 256 tokens
 constexpr int B_BYTES = B_ROWS * BK * 2;
@@ -85,6 +88,24 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
 constexpr int NT = 256;                 // tokens per tile (MMA N <= 256)
 constexpr uint32_t ACC_COLS = 256;      // one accumulator buffer
 constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+// E4M3 with per-tile scales (block-scaled MMA): the scales of a stage sit in
+// tensor memory beside the accumulators, so the second accumulator gives up
+// 16 columns and holds tiles of at most 240 tokens (larger ones use the
+// first).  Scale atoms, per stage: A (this CTA's 128 weight rows x 4 tiles,
+// 512 bytes, 4 columns) and B (up to 256 tokens x 4 tiles, two 512-byte
+// atoms, 8 columns).
+constexpr uint32_t ACC1_COLS_F8 = 240;
+constexpr uint32_t SFA_COL = 496, SFB_COL = 504;
+constexpr int SFA_BYTES = 512, SFB_BYTES = 1024, SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
+// The scales have a ring of their own, deeper than the operands': their
+// copies are small loads with the latency of a round trip to L2 or DRAM, so
+// many stages must be in flight at once.  A loader warp issues a stage's
+// copies (cp.async) and an arrive that fires on the CTA-local barrier
+// sf_local once they have landed; a relay warp, which issues no copies of its
+// own, waits for that and passes the stage on to the leader's MMA issuer
+// (sf_full, a cluster-scope release).  A release issued by the loader itself
+// would also wait for all the stages it still has in flight.
+constexpr int SF_STAGES = 16;
 // Epilogue warps come in groups of four (one per TMEM lane quarter); groups
 // take the tile's 16-token chunks in turn.  The gate/up epilogue (SwiGLU on
 // every element) runs two groups with one exchange buffer each; the down
@@ -94,11 +115,12 @@ template <bool UP>
 __host__ __device__ constexpr int n_epi_warps() { return UP ? 8 : 4; }
 template <bool UP>
 __host__ __device__ constexpr int n_xbuf_per_group() { return UP ? 1 : 2; }
-// producer warps after the epilogue warps: the token operand (both), the W3 half (up)
-template <bool UP>
-__host__ __device__ constexpr int n_extra_producers() { return UP ? 2 : 1; }
-template <bool UP>
-__host__ __device__ constexpr int n_threads() { return 32 * (2 + n_epi_warps<UP>() + n_extra_producers<UP>()); }
+// producer warps after the epilogue warps: the token operand (both), the W3 half (up),
+// the tile scales (E4M3)
+template <bool UP, bool F8>
+__host__ __device__ constexpr int n_extra_producers() { return (UP ? 2 : 1) + (F8 ? 2 : 0); }
+template <bool UP, bool F8>
+__host__ __device__ constexpr int n_threads() { return 32 * (2 + n_epi_warps<UP>() + n_extra_producers<UP, F8>()); }
 constexpr int XS = 132;                 // row stride (floats) of the epilogue exchange buffer
 constexpr int XBUF_BYTES = 16 * XS * 4; // 16 tokens x 128 lanes (+pad), fp32
 // L2 policy of the two operands' loads.  Marking the weights evict-first
@@ -110,9 +132,9 @@ constexpr uint64_t X_HINT = kEvictNormal;
 constexpr int TQ = 8;                   // tile queue slots
 // readers of a queue slot, in each CTA: the epilogue warps, the extra producers, and
 // the MMA issuer (leader) or the weight producer (peer)
-template <bool UP>
+template <bool UP, bool F8>
 __host__ __device__ constexpr uint32_t tq_readers() {
-    return 2u * (1u + (uint32_t)n_epi_warps<UP>() + (uint32_t)n_extra_producers<UP>());
+    return 2u * (1u + (uint32_t)n_epi_warps<UP>() + (uint32_t)n_extra_producers<UP, F8>());
 }
 
 // Tile counters: one {next, done} pair per launch slot.  A launch takes the
@@ -124,9 +146,13 @@ constexpr int kSchedSlots = 1024;
 __device__ unsigned int g_tile_sched[kSchedSlots][2];
 
 
+constexpr int MAX_STAGES = 6;
 struct Ctl {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[MAX_STAGES];
+    uint64_t empty[MAX_STAGES];
+    uint64_t sf_local[SF_STAGES];  // E4M3: this CTA's scale copies of the stage landed (32 loader lanes)
+    uint64_t sf_full[SF_STAGES];   // E4M3, leader: both CTAs' relays passed the stage on
+    uint64_t sf_empty[SF_STAGES];  // E4M3: the MMAs that read the slot are done
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t tq_full[TQ];   // in both CTAs: slot holds the next tile
@@ -146,8 +172,17 @@ struct Tables {
 constexpr size_t XBUF_TOTAL = 2 * (size_t)XBUF_BYTES;  // groups x buffers per group = 2 either way
 static_assert(n_epi_warps<true>() / 4 * n_xbuf_per_group<true>() == 2, "exchange buffers");
 static_assert(n_epi_warps<false>() / 4 * n_xbuf_per_group<false>() == 2, "exchange buffers");
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + XBUF_TOTAL + sizeof(Ctl) + sizeof(Tables);
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// ring, tile scales (E4M3), epilogue exchange buffers, control, tables
+template <bool F8>
+__host__ __device__ constexpr size_t sf_region_bytes() { return F8 ? (size_t)SF_STAGES * SF_STAGE_BYTES : 0; }
+template <bool F8>
+__host__ __device__ constexpr size_t smem_bytes() {
+    return 1024 + (size_t)n_stages<F8>() * STAGE_BYTES + sf_region_bytes<F8>() + XBUF_TOTAL + sizeof(Ctl) +
+           sizeof(Tables);
+}
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory budget");
+static_assert(n_stages<false>() <= MAX_STAGES && n_stages<true>() <= MAX_STAGES, "ring depth");
+
 
 // Tensor maps of one expert set: weights (w1 only for the up projection) and
 // the token operand with box heights 16 * (i + 1) rows.
@@ -167,15 +202,24 @@ struct SetParams {
     int ldo;           // output row pitch (elements)
     int f_limit;       // valid output features
     long long a_rows;  // rows the groups may index (token operand rows, or gathered rows) = output rows
-    // E4M3 operands only: per-row scales.  Weight row scales (up: W1 rows in
-    // ws0, W3 rows in ws1; down: W2 rows in ws0), srows scale rows per group;
-    // token-row scale of operand row r: xscale[xidx ? xidx[r] / xdiv : r].
-    const float* ws0;
-    const float* ws1;
-    int srows;
-    const float* xscale;
-    const int32_t* xidx;
-    int xdiv;
+    // E4M3 operands only: tile scales.  Weights (up: W1 in wsf0, W3 in wsf1;
+    // down: W2 in wsf0) as 64-row half atoms [rows/64][k_blocks][256 B], the
+    // row of group g, feature f being g * w_rows + f.  Token operand row r:
+    // word xsf[kb * xsf_pitch + (xsf_idx ? xsf_idx[r] / xsf_div : r)] of stage kb.
+    const uint8_t* wsf0;
+    const uint8_t* wsf1;
+    const uint32_t* xsf;
+    long long xsf_pitch;
+    const int32_t* xsf_idx;
+    int xsf_div;
+    // down only, weighted combine fused into the epilogue: each output row is
+    // scaled by its routing weight and added (fp32 atomics) into acc [T][ldo];
+    // routed set: row r holds assignment a = row_tok[r], token a / row_k,
+    // weight row_w[a]; shared set (row_tok null): row r is token r, weight 1.
+    float* acc;
+    const int32_t* row_tok;
+    const float* row_w;
+    int row_k;
 };
 struct Params {
     const int32_t* offsets;
@@ -219,11 +263,11 @@ __device__ __forceinline__ void token_tile(int rows, int ntt, int tt, int& start
 // below the output's own rounding.
 __device__ __forceinline__ float silu_fast(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
-__device__ __forceinline__ void scale4(float4& v, float s) {
-    v.x *= s;
-    v.y *= s;
-    v.z *= s;
-    v.w *= s;
+// Four fp32 additions into global memory (16-byte aligned), no return value.
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -302,7 +346,7 @@ __device__ __forceinline__ void settle_inflight_loads() {
 // lane 0 alone calls it.  The stage barrier may see these bytes land before
 // warp 0 arms it: its transaction count then stays negative until the
 // arming, and the phase cannot complete before the arrive that comes with it.
-template <bool kWarp, typename Begin, typename Load>
+template <int STAGES, bool kWarp, typename Begin, typename Load>
 __device__ __forceinline__ void follow_tiles(Ctl* ctl, const Tables* tb, int G, uint32_t leader_tq_empty, int* status,
                                              uint8_t* ring, int lane, Begin&& begin, Load&& load) {
     const uint32_t leader_full = mapa_shared(smem_u32(&ctl->full[0]), 0);
@@ -347,18 +391,29 @@ __device__ __forceinline__ void follow_tiles(Ctl* ctl, const Tables* tb, int G, 
     if (kWarp) __syncwarp();
 }
 
+// Accumulator of the tile that follows one in accumulator `prev`: the other
+// one, except that with tile scales in tensor memory the second holds at most
+// ACC1_COLS_F8 tokens.  The MMA issuer and the epilogue both follow it.
+template <bool F8>
+__device__ __forceinline__ int next_acc(int prev, int n_mma) {
+    const int a = prev ^ 1;
+    return (F8 && a == 1 && n_mma > (int)ACC1_COLS_F8) ? 0 : a;
+}
+
 template <bool UP, bool F8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(), 1)
     tc_grouped_gemm_kernel(const __grid_constant__ SetMaps ma, const __grid_constant__ SetMaps mb,
                            const __grid_constant__ CUtensorMap tmXg, const Params p) {
+    constexpr int STAGES = n_stages<F8>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = base;
-    float* xbuf = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
-    Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + XBUF_TOTAL);
+    uint8_t* sfr = base + STAGES * STAGE_BYTES;  // tile scales of each stage (E4M3)
+    float* xbuf = reinterpret_cast<float*>(sfr + sf_region_bytes<F8>());
+    Ctl* ctl = reinterpret_cast<Ctl*>(reinterpret_cast<uint8_t*>(xbuf) + XBUF_TOTAL);
     constexpr int NEPI = n_epi_warps<UP>();
     constexpr int NXB = n_xbuf_per_group<UP>();
-    constexpr int NTHREADS = n_threads<UP>();
+    constexpr int NTHREADS = n_threads<UP, F8>();
     Tables* tb = reinterpret_cast<Tables*>(ctl + 1);
 
     constexpr int BKE = bk_elems<F8>();
@@ -386,13 +441,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], 1);
         }
+        if (F8) {
+            for (int s = 0; s < SF_STAGES; ++s) {
+                mbar_init(&ctl->sf_local[s], 32);  // one completion arrive per loader lane
+                mbar_init(&ctl->sf_full[s], 2);    // the relays of both CTAs
+                mbar_init(&ctl->sf_empty[s], 1);
+            }
+        }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&ctl->tfull[a], 1);
             mbar_init(&ctl->tempty[a], 2 * NEPI);  // every epilogue warp of both CTAs
         }
         for (int j = 0; j < TQ; ++j) {
             mbar_init(&ctl->tq_full[j], 1);
-            mbar_init(&ctl->tq_empty[j], tq_readers<UP>());
+            mbar_init(&ctl->tq_empty[j], tq_readers<UP, F8>());
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -428,6 +490,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
 
     constexpr int kTokWarp = 2 + NEPI;  // token-operand producer
     constexpr int kW3Warp = 3 + NEPI;   // up: W3-half producer
+    constexpr int kSfWarp = (UP ? 4 : 3) + NEPI;  // E4M3: tile-scale loader
+    constexpr int kSfRelay = kSfWarp + 1;         // E4M3: passes landed scale stages to the MMA issuer
     const bool gather = UP && p.gather != nullptr;  // routed set only
 
     if (warp == 0) {
@@ -573,9 +637,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                 tma_gather4_pair(sb + 4 * lane * 128, &tmXg, fb, kb * BKE, src[0], src[1], src[2], src[3], X_HINT);
         };
         if (gather) {
-            follow_tiles<true>(ctl, tb, G, leader_tq_empty, p.status, ring, lane, begin, load);
+            follow_tiles<STAGES, true>(ctl, tb, G, leader_tq_empty, p.status, ring, lane, begin, load);
         } else {
-            if (lane == 0) follow_tiles<false>(ctl, tb, G, leader_tq_empty, p.status, ring, lane, begin, load);
+            if (lane == 0) follow_tiles<STAGES, false>(ctl, tb, G, leader_tq_empty, p.status, ring, lane, begin, load);
             __syncwarp();
         }
     } else if (UP && warp == kW3Warp) {
@@ -587,7 +651,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
         const CUtensorMap* wmap = nullptr;
         int wrow = 0;
         if (lane == 0)
-            follow_tiles<false>(
+            follow_tiles<STAGES, false>(
                 ctl, tb, G, leader_tq_empty, p.status, ring, lane,
                 [&](const TileCoord& tc) {
                     const int si = tc.g >= p.G0 ? 1 : 0;
@@ -598,12 +662,148 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                 [&](int kb, uint8_t* stage, uint32_t fb) {
                     tma_load_2d_pair(stage + A_BYTES / 2, wmap, fb, kb * BKE, wrow, W_HINT);
                 });
+
+        __syncwarp();
+    } else if (F8 && warp == kSfWarp) {
+        // ------------------------------------------------ tile-scale producer (E4M3, both CTAs)
+        // Per stage: this CTA's weight-row scale atom (two 8-byte pieces per
+        // lane, from the weights' 64-row half atoms) and the tile's token
+        // scale atoms (one 4-byte word per token, gathered through the
+        // permutation for the routed up projection), copied with cp.async
+        // into the stage's scale slot.  SF_LAG stages later, once those
+        // copies have landed (cp.async.mbarrier.arrive on sf_local), the
+        // relay warp hands them to the MMA issuer, which moves them into
+        // tensor memory.  Unused token words (rows past the tile) are zeros.
+        int stage = 0, j = 0;
+        uint32_t phase = 0, tq_ph = 0;
+        bool ok = true;
+        for (;;) {
+            int tile = -1, got = 1;
+            if (lane == 0) got = tq_take(ctl, j, tq_ph, leader_tq_empty, &tile, p.status) ? 1 : 0;
+            got = __shfl_sync(0xffffffffu, got, 0);
+            tile = __shfl_sync(0xffffffffu, tile, 0);
+            if (!got) {
+                ok = false;
+                break;
+            }
+            if (tile < 0) break;
+            if (++j == TQ) {
+                j = 0;
+                tq_ph ^= 1u;
+            }
+            const TileCoord tc = tile_coords(tb, G, tile);
+            const int si = tc.g >= p.G0 ? 1 : 0;
+            const SetParams& sp = p.set[si];
+            const int wg = si ? 0 : tc.g;
+            int tstart, ntok;
+            token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
+            const int nw = ((ntok + 15) & ~15) > 128 ? 8 : 4;  // token words per lane: the atoms the MMAs read
+            const int row0 = tb->rowstart[tc.g] + tstart;
+            long long src[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int jj = lane + 32 * i;
+                src[i] = -1;
+                if (jj < ntok) src[i] = sp.xsf_idx ? (long long)(sp.xsf_idx[row0 + jj] / sp.xsf_div) : row0 + jj;
+            }
+            const int kbn = sp.k_blocks;
+            const uint8_t* wa;
+            const uint8_t* wb;
+            uint32_t wa_n = 8u, wb_n = 8u;
+            if (UP) {  // 64 W1 rows, then the same 64 W3 rows
+                const long long R = (long long)wg * sp.w_rows + tc.ft * 128 + (int)rank * 64;
+                const size_t off = (size_t)(R >> 6) * kbn * 256 + (size_t)lane * 8;
+                wa = sp.wsf0 + off;
+                wb = sp.wsf1 + off;
+            } else {  // 128 W2 rows: two half atoms; rows past d take no scales
+                const int o0 = tc.ft * 256 + (int)rank * 128;
+                const long long R = (long long)wg * sp.w_rows + o0;
+                wa = sp.wsf0 + (size_t)(R >> 6) * kbn * 256 + (size_t)lane * 8;
+                wb = wa + (size_t)kbn * 256;
+                if (o0 >= sp.f_limit) {
+                    wa_n = 0u;
+                    wa = sp.wsf0;
+                }
+                if (o0 + 64 >= sp.f_limit) {
+                    wb_n = 0u;
+                    wb = sp.wsf0;
+                }
+            }
+            for (int kb = 0; kb < kbn; ++kb) {
+                int free_ = 1;
+                if (lane == 0) free_ = mbar_wait(&ctl->sf_empty[stage], phase ^ 1u, &ctl->abort, p.status) ? 1 : 0;
+                free_ = __shfl_sync(0xffffffffu, free_, 0);
+                if (!free_) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t slot = smem_u32(sfr + stage * SF_STAGE_BYTES);
+                cp_async_8(slot + (uint32_t)lane * 16u, wa + (wa_n ? (size_t)kb * 256 : 0), wa_n);
+                cp_async_8(slot + (uint32_t)lane * 16u + 8u, wb + (wb_n ? (size_t)kb * 256 : 0), wb_n);
+                const uint32_t* words = sp.xsf + (size_t)kb * (size_t)sp.xsf_pitch;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (i < nw) {
+                        const bool v = src[i] >= 0;
+                        cp_async_4(slot + (uint32_t)SFA_BYTES + (uint32_t)(i >> 2) * 512u + (uint32_t)lane * 16u +
+                                       (uint32_t)(i & 3) * 4u,
+                                   v ? (const void*)(words + src[i]) : (const void*)sp.xsf, v ? 4u : 0u);
+                    }
+                }
+                cp_async_mbar_arrive_noinc(&ctl->sf_local[stage]);  // fires once this lane's copies landed
+                if (++stage == SF_STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+        }
+        cp_async_wait<0>();
+        __syncwarp();
+    } else if (F8 && warp == kSfRelay) {
+        // ------------------------------------------------ tile-scale relay (E4M3, both CTAs, lane 0)
+        // Per stage, in order: wait until this CTA's scale copies have landed,
+        // make them visible to the async proxy (tcgen05.cp), and arrive on the
+        // leader's sf_full (cluster-scope release; this warp has no copies of
+        // its own in flight, so the release does not wait for any).
+        if (lane == 0) {
+            const uint32_t leader_sf_full = mapa_shared(smem_u32(&ctl->sf_full[0]), 0);
+            int stage = 0, j = 0;
+            uint32_t phase = 0, tq_ph = 0;
+            bool ok = true;
+            for (;;) {
+                int tile;
+                if (!tq_take(ctl, j, tq_ph, leader_tq_empty, &tile, p.status)) break;
+                if (++j == TQ) {
+                    j = 0;
+                    tq_ph ^= 1u;
+                }
+                if (tile < 0) break;
+                const TileCoord tc = tile_coords(tb, G, tile);
+                const int kbn = p.set[tc.g >= p.G0 ? 1 : 0].k_blocks;
+                for (int kb = 0; kb < kbn; ++kb) {
+                    if (!mbar_wait(&ctl->sf_local[stage], phase, &ctl->abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive_cluster(leader_sf_full + 8u * (uint32_t)stage);
+                    if (++stage == SF_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+            }
+        }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (leader CTA only)
         if (rank == 0 && elect_one()) {
-            int stage = 0, acc = 0, j = 0;
-            uint32_t phase = 0, acc_phase = 0, tq_ph = 0;
+            int stage = 0, acc = 1, j = 0;  // acc: the previous tile's accumulator
+            int sfs = 0;                    // E4M3: scale ring slot
+            uint32_t phase = 0, tq_ph = 0, sf_phase = 0;
+            uint32_t acc_ph = 0u;  // bit a: phase of accumulator a
             bool ok = true;
             for (;;) {
                 int tile;
@@ -621,8 +821,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                 int tstart, ntok;
                 token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
                 const int n_mma = (ntok + 15) & ~15;
-                const uint32_t idesc = F8 ? idesc_e4m3_f32(256, n_mma) : idesc_bf16_f32(256, n_mma);
-                if (!mbar_wait_cluster(&ctl->tempty[acc], acc_phase ^ 1u, &ctl->abort, p.status)) {
+                const uint32_t idesc = idesc_bf16_f32(256, n_mma);
+                acc = next_acc<F8>(acc, n_mma);
+                if (!mbar_wait_cluster(&ctl->tempty[acc], ((acc_ph >> acc) & 1u) ^ 1u, &ctl->abort, p.status)) {
                     ok = false;
                     break;
                 }
@@ -633,20 +834,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                         ok = false;
                         break;
                     }
+                    // E4M3: the scale warps of both CTAs arrive with a cluster-scope release
+                    if (F8 && !mbar_wait_cluster(&ctl->sf_full[sfs], sf_phase, &ctl->abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     uint8_t* sa = ring + stage * STAGE_BYTES;
                     const uint64_t ad = smem_desc_sw128(smem_u32(sa));
                     const uint64_t bd = smem_desc_sw128(smem_u32(sa + A_BYTES));
+                    if (F8) {
+                        // the stage's tile scales into tensor memory (one slot, reused every stage: the
+                        // copies and MMAs of this thread execute in issue order), then 4 MMAs of K = 32,
+                        // each reading byte kk of its rows' scale words
+                        const uint32_t sfa = smem_u32(sfr + sfs * SF_STAGE_BYTES);
+                        tc_cp_32x128b_x4_pair(tmem_base + SFA_COL, smem_desc_plain(sfa));
+                        tc_cp_32x128b_x4_pair(tmem_base + SFB_COL, smem_desc_plain(sfa + SFA_BYTES));
+                        if (n_mma > 128)
+                            tc_cp_32x128b_x4_pair(tmem_base + SFB_COL + 4u, smem_desc_plain(sfa + SFA_BYTES + 512));
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {  // 4 MMAs of 32 bytes along K (16 bf16 or 32 E4M3)
-                        if (F8)
-                            tc_mma_e4m3_pair(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
-                                             (kb > 0 || kk > 0) ? 1u : 0u);
-                        else
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma_mx_pair(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk),
+                                           idesc_mx_e4m3(256, n_mma, (uint32_t)kk, (uint32_t)kk),
+                                           (tmem_base + SFA_COL) | ((uint32_t)kk << 30),
+                                           (tmem_base + SFB_COL) | ((uint32_t)kk << 30), (kb > 0 || kk > 0) ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)  // 4 MMAs of K = 16 (32 bytes)
                             tc_mma_bf16_pair(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
                                              (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit_pair(&ctl->empty[stage], 0x3);
+                    if (F8) {
+                        tc_commit_pair(&ctl->sf_empty[sfs], 0x3);
+                        if (++sfs == SF_STAGES) {
+                            sfs = 0;
+                            sf_phase ^= 1u;
+                        }
+                    }
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -654,8 +879,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                 }
                 if (!ok) break;
                 tc_commit_pair(&ctl->tfull[acc], 0x3);
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1u;
+                acc_ph ^= 1u << acc;
             }
             if (!ok) {  // wait for the pair MMAs already issued (same cta_group as the MMAs)
                 tc_commit_pair(&ctl->drain, 0x1);
@@ -673,8 +897,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
         const int my_tok = e >> 3;        // token (0..15) of a 16-token chunk this thread stores
         const int part = e & 7;
         const uint32_t leader_tempty = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
-        int acc = 0, xb = 0, j = 0;
-        uint32_t acc_phase = 0, tq_ph = 0;
+        int acc = 1, xb = 0, j = 0;  // acc: the previous tile's accumulator (next_acc, as the MMA issuer)
+        uint32_t acc_ph = 0u, tq_ph = 0;  // acc_ph bit a: phase of accumulator a
         for (;;) {
             int tile = -1, got = 1;
             if (lane == 0) got = tq_take(ctl, j, tq_ph, leader_tq_empty, &tile, p.status) ? 1 : 0;
@@ -693,20 +917,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
             const int tok0 = tb->rowstart[tc.g] + tstart;
             // first output feature of this CTA
             const int fcta = UP ? tc.ft * 128 + (int)rank * 64 : tc.ft * 256 + (int)rank * 128;
-            // E4M3: scale of the weight row held in this thread's TMEM lane
-            float wsc = 1.0f;
-            if (F8) {
-                const int tl = q * 32 + lane;
-                const int wg = tc.g >= p.G0 ? 0 : tc.g;
-                if (UP) {
-                    const int f = tc.ft * 128 + (int)rank * 64 + (tl & 63);
-                    wsc = (tl < 64 ? sp.ws0 : sp.ws1)[(size_t)wg * sp.srows + f];
-                } else {
-                    const int f = fcta + tl;
-                    wsc = f < sp.f_limit ? sp.ws0[(size_t)wg * sp.srows + f] : 0.0f;
-                }
-            }
-            if (!mbar_wait(&ctl->tfull[acc], acc_phase, &ctl->abort, p.status)) break;
+            acc = next_acc<F8>(acc, (ntok + 15) & ~15);
+            if (!mbar_wait(&ctl->tfull[acc], (acc_ph >> acc) & 1u, &ctl->abort, p.status)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACC_COLS;
             // TMEM reads run one chunk ahead of the exchange below
@@ -718,7 +930,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                 tmem_ld_wait();
                 float v16[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v16[i] = F8 ? __uint_as_float(r[i]) * wsc : __uint_as_float(r[i]);
+                for (int i = 0; i < 16; ++i) v16[i] = __uint_as_float(r[i]);
                 if (c + CSTEP < ntok) tmem_ld16(taddr + (uint32_t)(c + CSTEP), r);
                 float* xs = xbuf + (NXB * eg + xb) * (XBUF_BYTES / 4);
 #pragma unroll
@@ -726,11 +938,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                 named_bar_sync(1 + eg, 128);
                 const bool tok_ok = c + my_tok < ntok;
                 const float* row = xs + my_tok * XS;
-                float tsc = 1.0f;  // E4M3: scale of this token row
-                if (F8 && tok_ok) {
-                    const int orow = tok0 + c + my_tok;
-                    tsc = sp.xscale[sp.xidx ? sp.xidx[orow] / sp.xdiv : orow];
-                }
                 if (UP) {  // lanes 0-63: gate, 64-127: up of the same 64 features
                     const int fj = part * 8;
                     float4 g0 = *reinterpret_cast<const float4*>(row + fj);
@@ -738,12 +945,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                     float4 u0 = *reinterpret_cast<const float4*>(row + 64 + fj);
                     float4 u1 = *reinterpret_cast<const float4*>(row + 64 + fj + 4);
                     if (NXB == 1) named_bar_sync(1 + eg, 128);  // the single buffer is free for the next chunk
-                    if (F8) {
-                        scale4(g0, tsc);
-                        scale4(g1, tsc);
-                        scale4(u0, tsc);
-                        scale4(u1, tsc);
-                    }
                     if (tok_ok) {
                         uint4 v;
                         v.x = pack_bf16x2(silu_fast(g0.x) * u0.x, silu_fast(g0.y) * u0.y);
@@ -758,18 +959,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
                         float f[16];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            float4 t = *reinterpret_cast<const float4*>(row + fj + 4 * i);
-                            if (F8) scale4(t, tsc);
+                            const float4 t = *reinterpret_cast<const float4*>(row + fj + 4 * i);
                             f[4 * i] = t.x;
                             f[4 * i + 1] = t.y;
                             f[4 * i + 2] = t.z;
                             f[4 * i + 3] = t.w;
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * sp.ldo + fcta + fj);
-                        dst[0] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                                            pack_bf16x2(f[6], f[7]));
-                        dst[1] = make_uint4(pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
-                                            pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
+                        const int orow = tok0 + c + my_tok;
+                        if (sp.acc) {  // fused weighted combine
+                            int t = orow;
+                            float wt = 1.0f;
+                            if (sp.row_tok) {
+                                const int a = sp.row_tok[orow];
+                                t = a / sp.row_k;
+                                wt = sp.row_w[a];
+                            }
+                            float* dst = sp.acc + (size_t)t * sp.ldo + fcta + fj;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                red_add_v4(dst + 4 * i, f[4 * i] * wt, f[4 * i + 1] * wt, f[4 * i + 2] * wt,
+                                           f[4 * i + 3] * wt);
+                        } else {
+                            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)orow * sp.ldo + fcta + fj);
+                            dst[0] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                            dst[1] = make_uint4(pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
+                                                pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
+                        }
                     }
                 }
                 if (NXB == 2) xb ^= 1;  // the next chunk writes the other buffer; its barrier orders the reuse
@@ -777,8 +993,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP>(), 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tempty + 8u * (uint32_t)acc);
-            acc ^= 1;
-            if (acc == 0) acc_phase ^= 1u;
+            acc_ph ^= 1u << acc;
         }
     }
 
@@ -796,11 +1011,12 @@ template <bool UP, bool F8>
 cudaError_t launch(const SetMaps& a, const SetMaps& b, const CUtensorMap& xg, Params p, int num_sms, cudaStream_t st) {
     auto kern = tc_grouped_gemm_kernel<UP, F8>;
     p.sched_slot = (int)(g_sched_seq.fetch_add(1u, std::memory_order_relaxed) % (unsigned int)kSchedSlots);
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    constexpr int NTHREADS = n_threads<UP>();
+    constexpr size_t SMEM = smem_bytes<F8>();
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+    constexpr int NTHREADS = n_threads<UP, F8>();
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;  // whole CTA pairs, one CTA per SM
-    kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(a, b, xg, p);
+    kern<<<grid, NTHREADS, SMEM, st>>>(a, b, xg, p);
     note_launches(1);
     return cudaGetLastError();
 }
@@ -815,18 +1031,18 @@ bool up_set(const TcUpArgs& a, SetMaps& m, SetParams& sp) {
     const unsigned eb = a.f8 ? 1 : 2;
     const int bke = 128 / (int)eb;
     if (a.d % bke != 0 || a.I % 128 != 0) return false;
-    if (a.f8 && (!a.w1s || !a.w3s || !a.xs)) return false;
+    if (a.f8 && (!a.w1s || !a.w3s || !a.xs || a.d % 128 != 0)) return false;
     if (!make_tmap_2d(&m.w0, a.W1, a.d, a.W_rows, a.d, bke, 64, eb) ||
         !make_tmap_2d(&m.w1, a.W3, a.d, a.W_rows, a.d, bke, 64, eb) || !token_maps(m, a.A, a.d, a.A_rows, eb))
         return false;
     sp.f_tiles = a.I / 128;
     sp.k_blocks = a.d / bke;
-    sp.ws0 = a.w1s;
-    sp.ws1 = a.w3s;
-    sp.srows = a.I;
-    sp.xscale = a.xs;
-    sp.xidx = a.xs_idx;
-    sp.xdiv = a.xs_div > 0 ? a.xs_div : 1;
+    sp.wsf0 = a.w1s;
+    sp.wsf1 = a.w3s;
+    sp.xsf = a.xs;
+    sp.xsf_pitch = a.xs_pitch;
+    sp.xsf_idx = a.xs_idx;
+    sp.xsf_div = a.xs_div > 0 ? a.xs_div : 1;
     sp.w_rows = a.I;
     sp.kseg = a.d;
     sp.nseg = 1;
@@ -841,7 +1057,7 @@ bool down_set(const TcDownArgs& a, SetMaps& m, SetParams& sp) {
     const unsigned eb = a.f8 ? 1 : 2;
     const int bke = 128 / (int)eb;
     if (a.K % bke != 0 || a.kseg % bke != 0 || a.d % 16 != 0) return false;
-    if (a.f8 && (!a.w2s || !a.hs)) return false;
+    if (a.f8 && (!a.w2s || !a.hs || a.K % 128 != 0 || a.kseg % 128 != 0 || a.d % 64 != 0)) return false;
     // W2 blocks [G * nseg][d][kseg] viewed as one matrix of G * nseg * d rows: a 2D map fed
     // the down projection ~10% faster than the same boxes through a 3D map.  Rows past d of
     // a feature tile read the next block's rows (or zero past the end); their outputs are
@@ -852,12 +1068,16 @@ bool down_set(const TcDownArgs& a, SetMaps& m, SetParams& sp) {
     m.w1 = m.w0;
     sp.f_tiles = (a.d + 255) / 256;
     sp.k_blocks = a.K / bke;
-    sp.ws0 = a.w2s;
-    sp.ws1 = nullptr;
-    sp.srows = a.d;
-    sp.xscale = a.hs;
-    sp.xidx = nullptr;
-    sp.xdiv = 1;
+    sp.wsf0 = a.w2s;
+    sp.wsf1 = nullptr;
+    sp.xsf = a.hs;
+    sp.xsf_pitch = a.H_rows;
+    sp.xsf_idx = nullptr;
+    sp.xsf_div = 1;
+    sp.acc = a.acc;
+    sp.row_tok = a.row_tok;
+    sp.row_w = a.row_w;
+    sp.row_k = a.row_k > 0 ? a.row_k : 1;
     sp.w_rows = a.d;
     sp.kseg = a.kseg;
     sp.nseg = a.nseg;

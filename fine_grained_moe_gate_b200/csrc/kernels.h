@@ -40,6 +40,14 @@ struct GemmArgs {
     int gather_div;
 };
 
+// quant.cu: per-tile E4M3 quantization (scale layouts described there)
+size_t mx_scale_bytes(long long rows, int K, bool weight_layout);
+cudaError_t launch_quantize_mx(const void* src, long long rows, int kseg, int nseg, bool weight_layout, uint8_t* q,
+                               void* scales, cudaStream_t st);
+
+// combine.cu: y = dtype(acc) for n elements (n % 8 == 0), then acc = 0
+cudaError_t launch_combine_finish(float* acc, long long n, bool bf16, void* y, cudaStream_t st);
+
 // router.cu
 cudaError_t launch_router_simt(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
                                bool bf16, int32_t* idx, float* w, int32_t* counts, float* aff, int* status,
@@ -76,8 +84,51 @@ struct BackwardArgs {
     void* workspace;
     int num_sms;
 };
-size_t backward_scratch_bytes(int T, int d, int E, int k, int I, int S, int Is, int seq_len);
+size_t backward_scratch_bytes(int T, int d, int E, int k, int I, int S, int Is, int seq_len, bool bf16);
+bool backward_on_tensor_cores(bool bf16, int d, int I, int S, int Is);
 cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sms, cudaStream_t st);
+
+// gemm_bwd_tc.cu: the backward's grouped GEMMs on the tensor cores (bf16 in,
+// fp32 out).  Groups: rows [start[g], start[g] + rows[g]) of the per-row
+// operands (a padded layout: each group's segment zero-padded to a multiple
+// of 64 rows), or one group of M_rows rows from 0 when start is null.
+struct BwdRowsArgs {
+    const void* W;          // K-major: [W_rows][K]; MN-major: [W_rows][M_total] (rows run along K)
+    const void* W1;         // MN-major only, may be null: read after the first K0 rows of W's group
+    long long W_rows;
+    int K0;
+    long long a_grow;       // weight rows per group (K-major: along M; MN-major: along K)
+    const void* X;          // [op_rows][K] per-row operand
+    long long op_rows;
+    int K;
+    int M_total;            // output features
+    const int32_t* start;
+    const int32_t* rows;
+    int G;
+    int M_rows;
+    float* out;             // [op_rows][ldo] fp32
+    int ldo;
+    bool accumulate;
+};
+cudaError_t launch_bwd_rows_kmajor(const BwdRowsArgs& a, int* status, int num_sms, cudaStream_t st);
+cudaError_t launch_bwd_rows_mnmajor(const BwdRowsArgs& a, int* status, int num_sms, cudaStream_t st);
+// out[g][m][n] = sum over group g's rows r (padded to 64) of A[r][a_col0 + m] * B[r][b_col0 + n]
+struct BwdWgradArgs {
+    const void* A;
+    int lda;
+    long long a_col0;
+    const void* B;
+    int ldb;
+    long long b_col0;
+    long long op_rows;
+    int M_total, N_total;   // multiples of 128
+    const int32_t* start;
+    const int32_t* rows;
+    int G;
+    int M_rows;
+    float* out;             // [G][M_total][N_total] fp32
+};
+cudaError_t launch_bwd_wgrad(const BwdWgradArgs& a, int* status, int num_sms, cudaStream_t st);
 
 // gemm_simt.cu
 cudaError_t launch_simt_gemm(const GemmArgs& p, bool bf16, bool swiglu, int num_sms, cudaStream_t st);
@@ -99,12 +150,15 @@ struct TcUpArgs {
     int d, I;
     const int32_t* offsets; // group rows; null: one group of M rows
     int G, M;
-    // E4M3 operands (A, W1, W3 one byte per element) with per-row scales:
-    // w1s/w3s [W_rows]; token row r's scale xs[xs_idx ? xs_idx[r] / xs_div : r].
+    // E4M3 operands (A, W1, W3 one byte per element) with per-tile scales
+    // (quant.cu layouts): w1s / w3s the weights' 64-row half atoms; token
+    // row r's scale words xs[s * xs_pitch + (xs_idx ? xs_idx[r] / xs_div : r)]
+    // for stage s (128 columns).
     bool f8 = false;
-    const float* w1s = nullptr;
-    const float* w3s = nullptr;
-    const float* xs = nullptr;
+    const uint8_t* w1s = nullptr;
+    const uint8_t* w3s = nullptr;
+    const uint32_t* xs = nullptr;
+    long long xs_pitch = 0;
     const int32_t* xs_idx = nullptr;
     int xs_div = 1;
 };
@@ -120,11 +174,20 @@ struct TcDownArgs {
     int d, K;
     const int32_t* offsets;
     int G, M;
-    // E4M3 operands (H, W2 one byte per element): w2s [G][d] per output row
-    // (one scale per row across the nseg blocks), hs [H_rows] per token row.
+    // E4M3 operands (H, W2 one byte per element) with per-tile scales:
+    // w2s the half atoms of W2 as [G * d] rows of K = nseg * kseg columns;
+    // hs the scale words of H, [K / 128][H_rows].
     bool f8 = false;
-    const float* w2s = nullptr;
-    const float* hs = nullptr;
+    const uint8_t* w2s = nullptr;
+    const uint32_t* hs = nullptr;
+    // Weighted combine fused into the epilogue (acc non-null): Y is not
+    // written; row r is scaled and added into acc [T][d] fp32 -- routed:
+    // token row_tok[r] / row_k, weight row_w[row_tok[r]]; shared (row_tok
+    // null): token r, weight 1.
+    float* acc = nullptr;
+    const int32_t* row_tok = nullptr;
+    const float* row_w = nullptr;
+    int row_k = 1;
 };
 // ep.cu: expert-parallel dispatch / return over peer memory.  Plan layout
 // (int32): base [E][W], src_off [W][E+1], recv_off [W][E/W+1].
@@ -142,10 +205,6 @@ cudaError_t launch_ep_dispatch(const void* x, const int32_t* perm_tok, const int
 cudaError_t launch_ep_return(const void* y, const int32_t* plan, int W, int E, int k, int rank, int T,
                              size_t row_bytes, const EpPeers& back, int num_sms, int* status, cudaStream_t st);
 
-// quant.cu: per-row E4M3 quantization of a bf16 matrix with `rows` rows
-// stored as nseg column blocks of kseg columns (kseg % 8 == 0).
-cudaError_t launch_quantize_e4m3(const void* src, long long rows, int kseg, int nseg, uint8_t* q, float* scale,
-                                 cudaStream_t st);
 
 // One launch for the routed set (offsets) and/or the shared set (M rows);
 // either pointer may be null.

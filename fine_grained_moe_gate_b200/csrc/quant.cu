@@ -1,16 +1,36 @@
-// Per-row E4M3 quantization ("DeepSeek V3 Architecture Deep Dive ...",
-// "FP8 Formats": E4M3 for weights and activations; "Per-Tensor/Per-Axis
-// Quantization": one scale per row/channel).
+// Per-tile E4M3 quantization ("DeepSeek V3 From Scratch", "The idea": FP8
+// with fine-grained quantization tiles; crackai.dev "DeepSeek-V3", "How It
+// Works": per-tile scaling; "DeepSeek V3 Architecture Deep Dive ...", "FP8
+// Formats": E4M3 for weights and activations).
 //
-//   scale_r = amax_r / 448, inv_r = 448 / amax_r (fp32, IEEE division, once
-//   per row; an all-zero row gets scale 1 and codes 0)
-//   q[r][c] = E4M3(src[r][c] * inv_r), round to nearest even, saturating
+// A tile is 32 consecutive elements of a row along the contraction
+// dimension.  Its scale is 2^e with e the smallest integer such that the
+// tile's largest magnitude fits E4M3 (amax <= 448 * 2^e, so nothing
+// saturates), kept as the byte e + 127 -- the unsigned power-of-two scale
+// format the tensor cores' block-scaled MMA reads.  Codes are
+// E4M3(v * 2^-e), round to nearest even; v * 2^-e is exact in fp32.
 //
+// e from the bits of amax (fp32, exponent field a, mantissa m): amax =
+// (1 + m/2^23) 2^(a-127) fits 448 * 2^e = 1.75 * 2^(8+e) iff a - 127 < 8 + e,
+// or a - 127 == 8 + e and m <= 0.75 * 2^23; so e = a - 135 + (m > 0x600000),
+// clamped to -127 below (an all-zero tile gets e = 0, codes 0).
+//
+// Scale layouts (the GEMMs' shared-memory scale atoms hold, for 128 operand
+// rows and one 128-column stage, the byte of row m, tile j at
+// (m % 32) * 16 + (m / 32) * 4 + j):
+//   tokens:  uint32 [K/128][rows]: word (s, r) holds the 4 tile bytes of row
+//            r's stage s (byte j = tile 4s + j).  A stage's words of
+//            consecutive rows are contiguous, so a warp fetches 32 rows' with
+//            one coalesced load, or gathers them by token index.
+//   weights: 64-row half atoms of 256 bytes, [rows/64][K/128][32][8]: byte
+//            (m % 32) * 8 + (m / 32) * 4 + j of half atom (r / 64, s), m =
+//            r % 64.  A lane of the GEMM's scale warp copies 8 bytes per half
+//            atom into the 16-byte row of the atom it builds.
 // A matrix with `rows` rows may be stored as nseg column blocks of kseg
-// columns ([nseg][rows][kseg], stacked experts joined along the contraction);
-// its rows span all blocks.  One warp per row, two passes over the row (the
-// second one from L1/L2): 16-byte loads of 8 bf16, 8-byte stores of 8 codes.
-// HBM bound: 3 bytes per element (2 read, 1 written) + 4 per row.
+// columns ([nseg][rows][kseg], stacked experts joined along the
+// contraction); its rows and tiles span all blocks.  One warp per row, one
+// pass: each lane converts 8 elements, four lanes share a tile.
+// HBM bound: 3 bytes per element (2 read, 1 written) + 1/32 per element.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -34,47 +54,90 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
     return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
 }
 
-__global__ void __launch_bounds__(kWarps * 32) quantize_e4m3_kernel(const uint16_t* __restrict__ src, long long rows,
-                                                                   int kseg, int nseg, uint8_t* __restrict__ q,
-                                                                   float* __restrict__ scale) {
+// Smallest e in [-127, 126] with amax <= 448 * 2^e (amax finite, >= 0; 0 for 0).
+__device__ __forceinline__ int tile_exponent(float amax) {
+    if (amax == 0.0f) return 0;
+    const uint32_t u = __float_as_uint(amax);
+    const int a = (int)(u >> 23);
+    const int e = a - 135 + ((u & 0x7fffffu) > 0x600000u ? 1 : 0);
+    return e < -127 ? -127 : e;
+}
+
+template <bool kWeightLayout>
+__global__ void __launch_bounds__(kWarps * 32) quantize_mx_kernel(const uint16_t* __restrict__ src, long long rows,
+                                                                 int kseg, int nseg, uint8_t* __restrict__ q,
+                                                                 uint8_t* __restrict__ sf) {
     const int lane = threadIdx.x & 31;
     const long long r = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
-    if (r >= rows) return;
+    if (r >= rows) return;  // warp-uniform
     const int K = kseg * nseg;
-    float amax = 0.0f;
-    for (int c = lane * 8; c < K; c += 256) {
-        const uint4 v = *reinterpret_cast<const uint4*>(src + seg_offset(r, c, rows, kseg));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const int nst = K >> 7;  // 128-column stages
+    for (int base = 0; base < K; base += 256) {
+        const int c = base + lane * 8;
+        const bool act = c < K;  // K % 128 == 0: whole 16-lane halves are active or not
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        size_t off = 0;
+        if (act) {
+            off = seg_offset(r, c, rows, kseg);
+            const uint4 v = *reinterpret_cast<const uint4*>(src + off);
+            w[0] = v.x;
+            w[1] = v.y;
+            w[2] = v.z;
+            w[3] = v.w;
+        }
+        float amax = 0.0f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
-    }
+        // the four lanes of a tile
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const int e = tile_exponent(amax);
+        const float mul = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, a normal fp32 for e in [-127, 126]
+        if (act) {
+            uint32_t p[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
-    if (lane == 0) scale[r] = sc;
-    for (int c = lane * 8; c < K; c += 256) {
-        const size_t off = seg_offset(r, c, rows, kseg);
-        const uint4 v = *reinterpret_cast<const uint4*>(src + off);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t p[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            p[i] = e4m3x2(__fmul_rn(bf16_lo(w[i]), inv), __fmul_rn(bf16_hi(w[i]), inv));
-        // element order in memory: low byte first
-        *reinterpret_cast<uint2*>(q + off) = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+            for (int i = 0; i < 4; ++i)
+                p[i] = e4m3x2(__fmul_rn(bf16_lo(w[i]), mul), __fmul_rn(bf16_hi(w[i]), mul));
+            *reinterpret_cast<uint2*>(q + off) = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+        }
+        // gather the four tile bytes of this lane's 128-column stage into lane 16h (h = lane / 16)
+        const uint32_t byte = (uint32_t)(e + 127);
+        const uint32_t b1 = __shfl_down_sync(0xffffffffu, byte, 4);
+        const uint32_t b2 = __shfl_down_sync(0xffffffffu, byte, 8);
+        const uint32_t b3 = __shfl_down_sync(0xffffffffu, byte, 12);
+        if (act && (lane & 15) == 0) {
+            const uint32_t word = byte | (b1 << 8) | (b2 << 16) | (b3 << 24);
+            const int s = c >> 7;
+            if (kWeightLayout) {
+                const size_t atom = ((size_t)(r >> 6) * nst + s) * 256;
+                const int m = (int)(r & 63);
+                *reinterpret_cast<uint32_t*>(sf + atom + (m & 31) * 8 + (m >> 5) * 4) = word;
+            } else {
+                reinterpret_cast<uint32_t*>(sf)[(size_t)s * rows + r] = word;
+            }
+        }
     }
 }
 
 }  // namespace
 
-cudaError_t launch_quantize_e4m3(const void* src, long long rows, int kseg, int nseg, uint8_t* q, float* scale,
-                                 cudaStream_t st) {
+size_t mx_scale_bytes(long long rows, int K, bool weight_layout) {
+    const size_t nst = (size_t)(K / 128);
+    if (weight_layout) return (size_t)((rows + 63) / 64) * nst * 256;
+    return (size_t)rows * nst * 4;
+}
+
+cudaError_t launch_quantize_mx(const void* src, long long rows, int kseg, int nseg, bool weight_layout, uint8_t* q,
+                               void* scales, cudaStream_t st) {
     if (rows <= 0) return cudaSuccess;
     const long long blocks = (rows + kWarps - 1) / kWarps;
     if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
-    quantize_e4m3_kernel<<<(unsigned)blocks, kWarps * 32, 0, st>>>(static_cast<const uint16_t*>(src), rows, kseg,
-                                                                   nseg, q, scale);
+    const auto* s = static_cast<const uint16_t*>(src);
+    auto* sf = static_cast<uint8_t*>(scales);
+    if (weight_layout)
+        quantize_mx_kernel<true><<<(unsigned)blocks, kWarps * 32, 0, st>>>(s, rows, kseg, nseg, q, sf);
+    else
+        quantize_mx_kernel<false><<<(unsigned)blocks, kWarps * 32, 0, st>>>(s, rows, kseg, nseg, q, sf);
     note_launches(1);
     return cudaGetLastError();
 }

@@ -127,6 +127,20 @@ class EPBuffers:
         self.back = back if back is not None else torch.empty((T * k, d), dtype=dt, device=device)
         self.h_recv = torch.empty((cap, I), dtype=dt, device=device)
         self.y_recv = self.recv
+        self.idx = torch.empty((T, k), dtype=i32, device=device)
+        self.w = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.counts = torch.empty(E, dtype=i32, device=device)
+        self.offsets = torch.empty(E + 1, dtype=i32, device=device)
+        self.perm = torch.empty(T * k, dtype=i32, device=device)
+        self.inv = torch.empty(T * k, dtype=i32, device=device)
+        self.recv_offsets = torch.empty(E // world + 1, dtype=i32, device=device)
+        self.hs = torch.empty((T, max(1, cfg.S * cfg.Is)), dtype=dt, device=device)
+        self.shared_out = torch.empty((T, d), dtype=dt, device=device) if cfg.S > 0 else None
+        self.y = torch.empty((T, d), dtype=dt, device=device)
+        self.flag = torch.zeros(1, dtype=torch.float32, device=device)
+        self._pws = None
+        self._plan = None
+
     def scratch(self, moe, sh, world):
         if self._pws is None:
             self._pws = torch.empty(max(moe.moe_permute_workspace_size(sh), 256), dtype=torch.uint8,

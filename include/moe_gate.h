@@ -7,8 +7,8 @@
  * state it (cited by page title and section):
  *   [P1] "DeepSeek V3 From Scratch": "The idea" (256 routed + 1 shared
  *        expert, top-8; bias acts on selection only, weights from the
- *        unbiased affinity), "Worked example", "In code" (route() and
- *        update_bias()).
+ *        unbiased affinity; FP8 with fine-grained quantization tiles),
+ *        "Worked example", "In code" (route() and update_bias()).
  *   [P2] "Scaling Efficiency: A Deep Dive into the DeepSeek-V3
  *        Architecture": DeepSeekMoE module sketch (shared experts on every
  *        token, routed experts combined with their gate weights).
@@ -17,9 +17,9 @@
  *   [P4] "DeepSeek V3 Architecture Deep Dive: Multi-Head Latent Attention
  *        (MLA), DeepSeekMoE & FP8 Mixed Precision": "Throughput on NVIDIA
  *        H100/H800" (tokens routed to the same expert batched together),
- *        "FP8 Formats" and "Per-Tensor/Per-Axis Quantization".
+ *        "FP8 Formats" (E4M3).
  *   [P5] crackai.dev "DeepSeek-V3": "How It Works" (all-to-all dispatch /
- *        combine kernels for expert parallelism).
+ *        combine kernels for expert parallelism; FP8 with per-tile scaling).
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the
@@ -70,8 +70,8 @@ typedef enum {
 } moe_status;
 
 /* MOE_FP8_E4M3: x, W_gate, y and the bf16 intermediates as MOE_BF16; the
- * expert GEMM operands (expert weights, token rows, h) in E4M3 with fp32
- * per-row scales -- see the FP8 section below. */
+ * expert GEMM operands (expert weights, token rows, h) in E4M3 with a
+ * power-of-two scale per tile of 32 elements -- see the FP8 section below. */
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_FP8_E4M3 = 2 } moe_dtype;
 
 /* Problem sizes.  T tokens of width d; E routed experts, k chosen per
@@ -84,7 +84,7 @@ typedef struct {
 
 /* Limits (validated): 1 <= k <= min(E, 16); E <= 256; d % 8 == 0.
  * MOE_BF16 additionally needs d % 64 == 0, I % 128 == 0 and Is % 128 == 0
- * (tensor-core tiles), MOE_FP8_E4M3 d % 128 == 0 as well, else
+ * (tensor-core tiles), MOE_FP8_E4M3 d % 128 == 0 as well (and I, Is % 128), else
  * MOE_ERR_UNSUPPORTED.  With MOE_FP8_E4M3, moe_route, moe_load_and_bias_update
  * and moe_combine behave as with MOE_BF16 and moe_permute moves E4M3 rows (one
  * byte per element); the bf16-weight calls (moe_grouped_swiglu, moe_ffn_*,
@@ -241,6 +241,27 @@ MOE_API moe_status moe_combine(const void* y_perm, const float* topk_w, const in
                        moe_shape sh, void* y, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_ffn_down_combine / moe_combine_finish -- moe_ffn_down and moe_combine
+ * in one launch: the weighted combine fused into the down projection's
+ * epilogue  [P2 DeepSeekMoE sketch: each routed expert's output scaled by
+ * its gate weight and added to the token; shared output added].
+ *   moe_ffn_down_combine: for every routed row r (assignment a =
+ *       perm_tok[r], token a / k): y_acc[a / k] += topk_w[a] * (h[r] . W2_e^T),
+ *       and with hs (S > 0) y_acc[t] += hs[t] . Ws2^T; fp32 additions straight
+ *       from the fp32 accumulators (no bf16 rounding of expert outputs).
+ *       y_acc [T][d] fp32 must hold zeros (or a partial sum to add to).  The
+ *       additions of one element come from different tiles in no fixed
+ *       order: y_acc is reproducible only up to fp32 rounding order.
+ *   moe_combine_finish: y = dtype(y_acc) (one rounding), then y_acc = 0.
+ * MOE_BF16 only (tensor-core path); perm_tok / topk_w from moe_permute /
+ * moe_route.  Same weights and arguments as moe_ffn_down otherwise.
+ * -------------------------------------------------------------------------*/
+MOE_API moe_status moe_ffn_down_combine(const void* h, const int32_t* offsets, const void* w2, const void* hs,
+                                        const void* ws2, const int32_t* perm_tok, const float* topk_w, moe_shape sh,
+                                        float* y_acc, void* stream);
+MOE_API moe_status moe_combine_finish(float* y_acc, moe_shape sh, void* y, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_layer_forward -- the whole layer: route, permute, grouped SwiGLU for
  * routed and shared experts, combine.  Same semantics as the five calls in
  * sequence.  The bias is read, not updated (call moe_load_and_bias_update
@@ -290,60 +311,83 @@ MOE_API moe_status moe_layer_backward(const void* x, const void* w_gate, const v
 MOE_API size_t moe_backward_workspace_size(moe_shape sh, int32_t seq_len);
 
 /* ---------------------------------------------------------------------------
- * FP8 experts  ["DeepSeek V3 Architecture Deep Dive ...", "FP8 Formats": E4M3
- * for weights and activations; "Per-Tensor/Per-Axis Quantization": a scale
- * per row/channel].  Read as: each weight matrix quantized per output row,
- * token rows and h per row; both scales factor out of every dot product and
- * are applied to the fp32 tensor-core accumulator:
- *   out[t][f] = sx[t] * sw[f] * sum_c e4m3(xq[t][c]) * e4m3(wq[f][c])
+ * FP8 experts with per-tile scales  [P1 "The idea": FP8 mixed precision with
+ * fine-grained quantization tiles; P5 "How It Works": per-tile scaling;
+ * P4 "FP8 Formats": E4M3 for weights and activations].  The pages fix
+ * neither the tile nor the scale arithmetic; read as:
+ *   - a tile is 32 consecutive elements of a row along the contraction
+ *     dimension (weights: an output row's input features; token rows and h:
+ *     their features);
+ *   - its scale is 2^e, e the smallest integer with amax <= 448 * 2^e (amax
+ *     the tile's largest magnitude; 0 for an all-zero tile; e >= -127), kept
+ *     as the byte e + 127;
+ *   - codes are E4M3(v * 2^-e), nearest, ties to even (nothing saturates);
+ *   - a dot product is sum over tiles of 2^(e_a + e_b) * sum_i a_i b_i in
+ *     fp32 (the tensor cores' block-scaled E4M3 MMA).
  * E4M3: 1 sign, 4 exponent (bias 7), 3 mantissa bits, no infinities, largest
- * finite 448.
+ * finite 448.  Row lengths (K) must be multiples of 128.
+ *
+ * Scale layouts (moe_fp8_scale_bytes gives the size of each):
+ *   MOE_SF_TOKENS  token rows and h: uint32 [K/128][rows]; word (s, r) holds
+ *                  the four tile bytes of row r's columns [128 s, 128 s + 128)
+ *                  (byte j = tile 4 s + j).
+ *   MOE_SF_WEIGHTS expert weights: 256-byte units, one per 64 rows and 128
+ *                  columns, [rows/64][K/128]; byte (m % 32) * 8 + (m / 32) * 4
+ *                  + j of unit (r / 64, s) is tile 4 s + j of row r, m = r % 64.
+ *                  This is the order the GEMMs assemble their tensor-memory
+ *                  scale blocks from; treat it as opaque otherwise.
  * -------------------------------------------------------------------------*/
+typedef enum { MOE_SF_TOKENS = 0, MOE_SF_WEIGHTS = 1 } moe_sf_layout;
 
-/* moe_quantize_fp8 -- per-row E4M3 quantization of a bf16 matrix with `rows`
- * rows stored as nseg column blocks of kseg columns ([nseg][rows][kseg];
- * nseg = 1 is plain row major; a row spans all blocks):
- *   scale[r] = amax_r / 448, inv_r = 448 / amax_r  (amax_r = max_c |src[r][c]|;
- *              fp32, IEEE division; a zero row gets scale 1 and codes 0)
- *   q[r][c]  = E4M3(src[r][c] * inv_r), nearest, ties to even, saturating
- * q has src's layout, one byte per element.  Needs kseg % 8 == 0, nseg >= 1,
- * 16-byte aligned src and q.  Used once per weight tensor (W2 [E][d][I] is
- * rows = E*d, kseg = I; the shared Ws2 [S][d][Is] is rows = d, kseg = Is,
- * nseg = S) and per step for the token rows and h. */
-MOE_API moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t kseg, int32_t nseg, uint8_t* q,
-                                    float* scale, void* stream);
+/* Bytes of the tile scales of a matrix of `rows` rows and K columns in the
+ * given layout (0 if K % 128 != 0 or the layout is unknown). */
+MOE_API size_t moe_fp8_scale_bytes(int64_t rows, int32_t K, int32_t layout);
 
-/* E4M3 expert weights and their per-row fp32 scales (all device pointers). */
+/* moe_quantize_fp8 -- per-tile E4M3 quantization of a bf16 matrix with
+ * `rows` rows stored as nseg column blocks of kseg columns ([nseg][rows][kseg];
+ * nseg = 1 is plain row major; a row and its tiles span all blocks, K =
+ * nseg * kseg).  q has src's layout, one byte per element; scales in
+ * `layout`.  Needs kseg % 128 == 0; src, q and scales 16-byte aligned.
+ * Used once per weight tensor (MOE_SF_WEIGHTS: W1/W3 [E][I][d] as rows = E*I;
+ * W2 [E][d][I] as rows = E*d, kseg = I; the shared Ws1/Ws3 [S][Is][d] as rows =
+ * S*Is; Ws2 [S][d][Is] as rows = d, kseg = Is, nseg = S) and per step for the
+ * token rows and h (MOE_SF_TOKENS). */
+MOE_API moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t kseg, int32_t nseg, int32_t layout,
+                                    uint8_t* q, void* scales, void* stream);
+
+/* E4M3 expert weights and their tile scales (MOE_SF_WEIGHTS), all device
+ * pointers, 16-byte aligned. */
 typedef struct {
-    const uint8_t* w1;  const float* w1_scale;   /* [E][I][d],  [E*I]  */
-    const uint8_t* w3;  const float* w3_scale;   /* [E][I][d],  [E*I]  */
-    const uint8_t* w2;  const float* w2_scale;   /* [E][d][I],  [E*d]  */
-    const uint8_t* ws1; const float* ws1_scale;  /* [S][Is][d], [S*Is] (NULL if S == 0) */
-    const uint8_t* ws3; const float* ws3_scale;  /* [S][Is][d], [S*Is] */
-    const uint8_t* ws2; const float* ws2_scale;  /* [S][d][Is], [d]: one scale per output row across the S blocks */
+    const uint8_t* w1;  const void* w1_scale;   /* [E][I][d]   rows E*I, K = d  */
+    const uint8_t* w3;  const void* w3_scale;   /* [E][I][d]   rows E*I, K = d  */
+    const uint8_t* w2;  const void* w2_scale;   /* [E][d][I]   rows E*d, K = I  */
+    const uint8_t* ws1; const void* ws1_scale;  /* [S][Is][d]  rows S*Is, K = d (NULL if S == 0) */
+    const uint8_t* ws3; const void* ws3_scale;  /* [S][Is][d]  rows S*Is, K = d */
+    const uint8_t* ws2; const void* ws2_scale;  /* [S][d][Is]  rows d, K = S*Is (the S blocks joined) */
 } moe_fp8_experts;
 
 /* moe_ffn_up_fp8 / moe_ffn_down_fp8 -- moe_ffn_up / moe_ffn_down on E4M3
  * operands (sh.dtype == MOE_FP8_E4M3), routed and shared experts in one
  * launch each.
  *   up:   xq_perm [T*k][d] E4M3 token rows in expert order (moe_permute of
- *         xq), perm_tok from moe_permute, x_scale [T] the token scales;
- *         xq [T][d] the unpermuted quantized tokens (shared experts; NULL
- *         leaves them out).  h = bf16(silu(a) * g) with a, g the scaled sums
- *         [T*k][I]; hs likewise [T][S*Is].
- *   down: hq [T*k][I] E4M3 with h_scale [T*k] (moe_quantize_fp8 of h), hsq
- *         [T][S*Is] with hs_scale [T] (NULL leaves the shared set out);
- *         y_perm [T*k][d] and shared_out [T][d] in bf16. */
-MOE_API moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const float* x_scale,
+ *         xq), perm_tok from moe_permute, x_scales the tile scales of the
+ *         unpermuted tokens (MOE_SF_TOKENS, [d/128][T]; row r of xq_perm uses
+ *         token perm_tok[r] / k's); xq [T][d] the unpermuted quantized tokens
+ *         (shared experts; NULL leaves them out).  h = bf16(silu(a) * g) with
+ *         a, g the tile-scaled sums [T*k][I]; hs likewise [T][S*Is].
+ *   down: hq [T*k][I] E4M3 with h_scales [I/128][T*k] (moe_quantize_fp8 of
+ *         h), hsq [T][S*Is] with hs_scales [S*Is/128][T] (NULL leaves the
+ *         shared set out); y_perm [T*k][d] and shared_out [T][d] in bf16. */
+MOE_API moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const void* x_scales,
                                   const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w, moe_shape sh,
                                   void* h, void* hs, void* stream);
-MOE_API moe_status moe_ffn_down_fp8(const uint8_t* hq, const float* h_scale, const int32_t* offsets,
-                                    const uint8_t* hsq, const float* hs_scale, const moe_fp8_experts* w,
+MOE_API moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_scales, const int32_t* offsets,
+                                    const uint8_t* hsq, const void* hs_scales, const moe_fp8_experts* w,
                                     moe_shape sh, void* y_perm, void* shared_out, void* stream);
 
 /* moe_layer_forward_fp8 -- the layer with FP8 experts: route (bf16 x),
- * quantize x per token, permute the E4M3 rows, gate/up, quantize h and hs
- * per row, down, combine into y [T][d] bf16.  sh.dtype == MOE_FP8_E4M3;
+ * quantize x by tiles, permute the E4M3 rows, gate/up, quantize h and hs by
+ * tiles, down, combine into y [T][d] bf16.  sh.dtype == MOE_FP8_E4M3;
  * workspace >= moe_workspace_size(sh). */
 MOE_API moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float* bias,
                                          const moe_fp8_experts* w, moe_shape sh, void* y, int32_t* topk_idx,

@@ -12,8 +12,9 @@ Sources, by page title and section:
   * "Scaling Efficiency: A Deep Dive into the DeepSeek-V3 Architecture" --
     the DeepSeekMoE module sketch.
   * kbwen.com DeepSeek tag page -- "A bias term for each expert".
-  * "DeepSeek V3 Architecture Deep Dive ..." -- "FP8 Formats" and
-    "Per-Tensor/Per-Axis Quantization" (the FP8 expert functions).
+  * "DeepSeek V3 Architecture Deep Dive ..." -- "FP8 Formats" (E4M3).
+  * "DeepSeek V3 From Scratch", "The idea", and crackai.dev "DeepSeek-V3",
+    "How It Works" -- FP8 with per-tile scaling (the *_mx functions).
 """
 from __future__ import annotations
 
@@ -66,9 +67,6 @@ def _load():
         lib.orc_layer_output.argtypes = [P, P, P, P, P, P, P, P, P, i, i, i, i, i, i, i, i, P]
         lib.orc_e4m3_encode_array.argtypes = [P, ctypes.c_size_t, P]
         lib.orc_e4m3_decode_array.argtypes = [P, ctypes.c_size_t, P]
-        lib.orc_quantize_rows_fp8.argtypes = [P, i, ctypes.c_long, i, i, P, P]
-        lib.orc_expert_up_fp8.argtypes = [P, P, i, P, P, P, P, i, i, P]
-        lib.orc_expert_down_fp8.argtypes = [P, P, i, P, P, i, i, i, P]
         lib.orc_mx_exponent.argtypes = [ctypes.c_double]
         lib.orc_mx_exponent.restype = i
         lib.orc_quantize_mx.argtypes = [P, i, ctypes.c_long, i, i, P, P]
@@ -224,7 +222,17 @@ def route(x, w_gate, bias, k):
     return w, idx, s
 
 
-# ------------------------------------------------------------------ FP8 experts
+# ------------------------------------------------- FP8 experts, per-tile scales
+#
+# E4M3 codes ("DeepSeek V3 Architecture Deep Dive ...", "FP8 Formats") with
+# tiles of 32 consecutive elements of a row along the contraction dimension,
+# each with a power-of-two scale 2^e (e the smallest integer with
+# amax <= 448 * 2^e), stored as the byte e + 127; codes E4M3(v * 2^-e).
+# Pages: "DeepSeek V3 From Scratch", "The idea" (fine-grained quantization
+# tiles); crackai.dev "DeepSeek-V3", "How It Works" (per-tile scaling).
+
+MX_TILE = 32
+
 
 def fp8_encode(x) -> np.ndarray:
     """E4M3 codes (uint8) of fp32 values: nearest, ties to even, +-448 saturation."""
@@ -240,111 +248,6 @@ def fp8_decode(q) -> np.ndarray:
     x = np.empty(q.shape, np.float64)
     _load().orc_e4m3_decode_array(_ptr(q), q.size, _ptr(x))
     return x
-
-
-def quantize_rows_fp8(a: np.ndarray, nseg: int = 1):
-    """Per-row E4M3 quantization.  ``a`` is [rows][K] (bf16 bits as uint16, or
-    float32), or [nseg][rows][kseg] for a matrix stored as column blocks (the
-    rows then span all nseg blocks).  Returns (codes with a's shape, scale fp32
-    [rows]) with scale = amax / 448 and codes = e4m3(v * (448 / amax)), both
-    factors rounded to fp32."""
-    a = _c(a)
-    dt = _dtype_code(a)
-    if a.ndim == 3:
-        if a.shape[0] != nseg:
-            raise ValueError("nseg must equal the number of column blocks")
-        rows, kseg = a.shape[1], a.shape[2]
-    else:
-        if nseg != 1:
-            raise ValueError("a blocked matrix is passed as [nseg][rows][kseg]")
-        rows, kseg = a.shape
-    q = np.empty(a.shape, np.uint8)
-    scale = np.empty(rows, np.float32)
-    _load().orc_quantize_rows_fp8(_ptr(a), dt, rows, kseg, nseg, _ptr(q), _ptr(scale))
-    return q, scale
-
-
-def expert_up_fp8(xq, xs, w1q, w1s, w3q, w3s) -> np.ndarray:
-    """h = bf16(silu(a) * g) with a, g the scaled E4M3 dot products; bf16 bits [n][I]."""
-    xq, w1q, w3q = _c(xq, np.uint8), _c(w1q, np.uint8), _c(w3q, np.uint8)
-    xs, w1s, w3s = _c(xs, np.float32), _c(w1s, np.float32), _c(w3s, np.float32)
-    n, d = xq.shape
-    I = w1q.shape[0]
-    h = np.empty((n, I), np.uint16)
-    _load().orc_expert_up_fp8(_ptr(xq), _ptr(xs), n, _ptr(w1q), _ptr(w1s), _ptr(w3q), _ptr(w3s), d, I, _ptr(h))
-    return h
-
-
-def expert_down_fp8(hq, hs, w2q, w2s) -> np.ndarray:
-    """o [n][d] (float64) = hs[r] * w2s[j] * sum_c dec(hq) dec(w2q).  w2q is [d][K]
-    or [nseg][d][kseg] (stacked experts joined along K)."""
-    hq, w2q = _c(hq, np.uint8), _c(w2q, np.uint8)
-    hs, w2s = _c(hs, np.float32), _c(w2s, np.float32)
-    n = hq.shape[0]
-    if w2q.ndim == 3:
-        nseg, d, kseg = w2q.shape
-    else:
-        nseg, (d, kseg) = 1, w2q.shape
-    o = np.empty((n, d), np.float64)
-    _load().orc_expert_down_fp8(_ptr(hq), _ptr(hs), n, _ptr(w2q), _ptr(w2s), d, kseg, nseg, _ptr(o))
-    return o
-
-
-def quantize_weights_fp8(p: dict) -> dict:
-    """Per-output-row E4M3 quantization of a layer's expert weights (numpy,
-    bf16 bits): W1/W3 [E][I][d] per row of I, W2 [E][d][I] per row of d,
-    shared Ws1/Ws3 [S][Is][d] per row, Ws2 [S][d][Is] per row d across the S
-    blocks.  Returns codes and scales under the keys w1q, w1s, ..."""
-    out = {}
-    for key in ("w1", "w3", "ws1", "ws3"):
-        a = p[key]
-        q, sc = quantize_rows_fp8(a.reshape(-1, a.shape[-1]))
-        out[key + "q"], out[key + "s"] = q.reshape(a.shape), sc
-    w2 = p["w2"]
-    q, sc = quantize_rows_fp8(w2.reshape(-1, w2.shape[-1]))
-    out["w2q"], out["w2s"] = q.reshape(w2.shape), sc
-    ws2 = p["ws2"]
-    q, sc = quantize_rows_fp8(ws2, nseg=ws2.shape[0])
-    out["ws2q"], out["ws2s"] = q, sc
-    return out
-
-
-def layer_output_fp8(x, idx, w, q: dict) -> np.ndarray:
-    """Whole layer with FP8 experts for given routing: x (bf16 bits) [T][d] is
-    quantized per token; each routed expert e: h = up(x rows), h quantized per
-    row, o = down(h), y += w * o; shared: h over the S*Is concatenated features,
-    quantized per token, o = down over the concatenated K.  y in bf16 bits."""
-    T, d = x.shape
-    k = idx.shape[1]
-    E, I, _ = q["w1q"].shape
-    S, Is, _ = q["ws1q"].shape
-    xq, xs = quantize_rows_fp8(x)
-    yacc = np.zeros((T, d), np.float64)
-    if S > 0:
-        hs = expert_up_fp8(xq, xs, q["ws1q"].reshape(S * Is, d), q["ws1s"], q["ws3q"].reshape(S * Is, d), q["ws3s"])
-        hq, hsc = quantize_rows_fp8(hs)
-        yacc += expert_down_fp8(hq, hsc, q["ws2q"], q["ws2s"])
-    for e in range(E):
-        t, j = np.nonzero(idx == e)
-        if len(t) == 0:
-            continue
-        h = expert_up_fp8(xq[t], xs[t], q["w1q"][e], q["w1s"][e * I:(e + 1) * I], q["w3q"][e],
-                          q["w3s"][e * I:(e + 1) * I])
-        hq, hsc = quantize_rows_fp8(h)
-        o = expert_down_fp8(hq, hsc, q["w2q"][e], q["w2s"][e * d:(e + 1) * d])
-        yacc[t] += w[t, j].astype(np.float64)[:, None] * o
-    return finalize(yacc, x.dtype)
-
-
-# ------------------------------------------------- FP8 experts, per-tile scales
-#
-# Tiles of 32 consecutive elements of a row along the contraction dimension,
-# each with a power-of-two scale 2^e (e the smallest integer with
-# amax <= 448 * 2^e), stored as the byte e + 127; codes E4M3(v * 2^-e).
-# Pages: "DeepSeek V3 From Scratch", "The idea" (fine-grained quantization
-# tiles); crackai.dev "DeepSeek-V3", "How It Works" (per-tile scaling).
-
-MX_TILE = 32
 
 
 def mx_exponent(amax: float) -> int:

@@ -313,18 +313,13 @@ void orc_layer_output(const void* x, const int32_t* idx, const float* w, const v
     free(yacc);
 }
 
-/* ---- FP8 (E4M3) experts ------------------------------------------------- */
-/* [P4] "DeepSeek V3 Architecture Deep Dive ...", "FP8 Formats": E4M3 (4
- * exponent, 3 mantissa bits) for weights and activations; "Per-Tensor/
- * Per-Axis Quantization": a scaling factor per row/channel.  Read here as:
- * weights quantized per output row (channel), activations per token row;
- * products accumulated wider than fp8 and the two scales applied after the
- * sum, which is exact because both factor out of the dot product.
- *
- * E4M3 values, from the format's definition (the "fn" variant with no
- * infinities): exponent bias 7; field e in 1..15 gives (1 + m/8) * 2^(e-7),
- * e = 0 gives subnormals (m/8) * 2^-6; S.1111.111 is NaN; the largest finite
- * magnitude is 1.75 * 2^8 = 448. */
+/* ---- E4M3 codec ----------------------------------------------------------
+ * [P4] "DeepSeek V3 Architecture Deep Dive ...", "FP8 Formats": E4M3 (4
+ * exponent, 3 mantissa bits) for weights and activations.  Values, from the
+ * format's definition (the "fn" variant with no infinities): exponent bias
+ * 7; field e in 1..15 gives (1 + m/8) * 2^(e-7), e = 0 gives subnormals
+ * (m/8) * 2^-6; S.1111.111 is NaN; the largest finite magnitude is
+ * 1.75 * 2^8 = 448. */
 
 double orc_e4m3_decode(uint8_t c) {
     int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
@@ -389,71 +384,6 @@ void orc_e4m3_decode_array(const uint8_t* q, size_t n, double* x) {
  * blocks are joined along the contraction); nseg = 1 is plain row major. */
 static size_t seg_index(long r, int c, long rows, int kseg) {
     return (size_t)(c / kseg) * (size_t)rows * kseg + (size_t)r * kseg + (size_t)(c % kseg);
-}
-
-/* Per-row quantization: amax_r = max |v| (fp32); the dequantization scale is
- * scale_r = fl32(amax_r / 448) and the codes use its reciprocal taken the
- * other way round, inv_r = fl32(448 / amax_r): q = e4m3(fl32(v * inv_r)).
- * An all-zero row has scale 1 and codes 0.  q has src's layout. */
-void orc_quantize_rows_fp8(const void* src, int dtype, long rows, int kseg, int nseg, uint8_t* q, float* scale) {
-    int K = kseg * nseg;
-    #pragma omp parallel for schedule(static)
-    for (long r = 0; r < rows; ++r) {
-        float amax = 0.0f;
-        for (int c = 0; c < K; ++c) {
-            float v = fabsf((float)load_elem(src, dtype, seg_index(r, c, rows, kseg)));
-            if (v > amax) amax = v;
-        }
-        float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
-        float inv = amax > 0.0f ? 448.0f / amax : 0.0f;
-        scale[r] = sc;
-        for (int c = 0; c < K; ++c) {
-            size_t i = seg_index(r, c, rows, kseg);
-            float v = (float)load_elem(src, dtype, i);
-            q[i] = orc_e4m3_encode(v * inv);
-        }
-    }
-}
-
-/* Gate/up of one FP8 expert on n quantized token rows:
- *   a[c] = xs[r] * w1s[c] * sum_i dec(xq[r][i]) dec(w1q[c][i])   (double)
- *   g[c] = xs[r] * w3s[c] * sum_i dec(xq[r][i]) dec(w3q[c][i])
- *   h[r][c] = bf16(silu(a) * g)                 (h stored in bf16, as the bf16 path)
- * xq [n][d], w1q/w3q [I][d] row major. */
-void orc_expert_up_fp8(const uint8_t* xq, const float* xs, int n, const uint8_t* w1q, const float* w1s,
-                       const uint8_t* w3q, const float* w3s, int d, int I, uint16_t* h) {
-    const double* val = e4m3_values();
-    #pragma omp parallel for schedule(dynamic, 8) collapse(2)
-    for (int r = 0; r < n; ++r) {
-        for (int c = 0; c < I; ++c) {
-            double sa = 0.0, sg = 0.0;
-            for (int i = 0; i < d; ++i) {
-                double xv = val[xq[(size_t)r * d + i]];
-                sa += xv * val[w1q[(size_t)c * d + i]];
-                sg += xv * val[w3q[(size_t)c * d + i]];
-            }
-            double a = (double)xs[r] * (double)w1s[c] * sa;
-            double g = (double)xs[r] * (double)w3s[c] * sg;
-            h[(size_t)r * I + c] = float_to_bf16_bits((float)(a / (1.0 + exp(-a)) * g));
-        }
-    }
-}
-
-/* Down projection of one FP8 expert on n quantized rows of h:
- *   o[r][j] = hs[r] * w2s[j] * sum_c dec(hq[r][c]) dec(w2q(j, c))   (double)
- * hq [n][K]; w2q is [d][K] stored as nseg blocks of kseg columns (K = nseg*kseg). */
-void orc_expert_down_fp8(const uint8_t* hq, const float* hs, int n, const uint8_t* w2q, const float* w2s, int d,
-                         int kseg, int nseg, double* o) {
-    int K = kseg * nseg;
-    const double* val = e4m3_values();
-    #pragma omp parallel for schedule(dynamic, 8) collapse(2)
-    for (int r = 0; r < n; ++r) {
-        for (int j = 0; j < d; ++j) {
-            double acc = 0.0;
-            for (int c = 0; c < K; ++c) acc += val[hq[(size_t)r * K + c]] * val[w2q[seg_index(j, c, d, kseg)]];
-            o[(size_t)r * d + j] = (double)hs[r] * (double)w2s[j] * acc;
-        }
-    }
 }
 
 /* ---- FP8 (E4M3) experts with per-tile scaling ----------------------------

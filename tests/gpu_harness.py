@@ -185,12 +185,46 @@ def oracle_terms(p, x, idx, w, tokens, S):
     return y, mag
 
 
+def oracle_terms_from_h(p, h, hs, idx, w, inv, tokens, S):
+    """The down projections and the combine of the oracle, fed with the GPU's
+    own intermediate h (routed rows, [T*k][I]) and hs (shared, [T][S*Is]) for
+    the given tokens: y = sum_s Ws2_s hs + sum_j w_j W2_e h_r (double) and the
+    magnitude M = |shared| + sum_j w_j |o_j|.  With h injected, a bf16 h
+    element that fp32 and double round to neighbouring values (one ulp, 2^-7
+    of it) cannot move the comparison; h itself is checked against the
+    oracle's up projection element by element in the projection tests."""
+    tokens = np.asarray(tokens)
+    n = len(tokens)
+    k = idx.shape[1]
+    d = p["w2"].shape[1]
+    sh = np.zeros((n, d), np.float64)
+    if S > 0:
+        Is = p["ws2"].shape[2]
+        hst = to_numpy(hs[torch.as_tensor(tokens, device=hs.device)])
+        for s in range(S):
+            sh += oracle.expert_down(np.ascontiguousarray(hst[:, s * Is:(s + 1) * Is]), to_numpy(p["ws2"][s]))
+    y = sh.copy()
+    mag = np.abs(sh)
+    idx_np = idx.cpu().numpy()[tokens]
+    w_np = w.cpu().numpy()[tokens]
+    inv_np = inv.cpu().numpy().reshape(-1, k)[tokens]
+    for e in np.unique(idx_np):
+        ii, jj = np.nonzero(idx_np == e)
+        rows = torch.as_tensor(inv_np[ii, jj], device=h.device)
+        o = oracle.expert_down(to_numpy(h[rows]), to_numpy(p["w2"][e]))
+        wt = w_np[ii, jj].astype(np.float64)[:, None]
+        np.add.at(y, ii, wt * o)
+        np.add.at(mag, ii, wt * np.abs(o))
+    return y, mag
+
+
 def check_layer_elementwise(y_gpu: torch.Tensor, y_ref_f64: np.ndarray, mag: np.ndarray):
-    """bf16 layer output, element by element.  The GPU rounds each expert
-    output (y_perm) and the shared output to bf16 before the weighted sum
-    (each within 2^-8 of its value) and rounds y once more; the oracle rounds
-    y once.  So |y_gpu - y_ref| <= 2^-8 (M + 2|y|) <= 2^-7 (|y_ref| + M), M the
-    terms' magnitude from ``oracle_terms``."""
+    """bf16 layer output, element by element, against the oracle's down
+    projections and combine of the same h (``oracle_terms_from_h``).  The
+    GPU rounds each expert output (y_perm) and the shared output to bf16
+    before the weighted sum (each within 2^-8 of its value) and rounds y once
+    more; the oracle rounds y once.  So |y_gpu - y_ref| <= 2^-8 (M + 2|y|) <=
+    2^-7 (|y_ref| + M), M the terms' magnitude."""
     got = as_f64(y_gpu)
     ref = to_f64_rows(oracle.finalize(y_ref_f64, np.uint16))
     bound = 2.0 ** -7 * (np.abs(ref) + mag) + 1e-6
@@ -217,3 +251,21 @@ def check_bf16_close(got: np.ndarray, ref: np.ndarray, what: str):
         r, c = np.argwhere(bad)[0]
         raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} elements beyond the bf16 bound, first at "
                              f"[{r}][{c}]: got {got[r, c]}, oracle {ref[r, c]}, bound {bound[r, c]}")
+
+
+# ---- tile-scale layouts of the FP8 path (include/moe_gate.h, MOE_SF_*), decoded
+#      into the oracle's [rows][K/32] exponent bytes.  Layout only, no arithmetic.
+
+def sf_tokens_to_rows(sf: torch.Tensor, rows: int, K: int) -> np.ndarray:
+    """MOE_SF_TOKENS: uint32 [K/128][rows], byte j of word (s, r) = tile 4s+j of row r."""
+    b = sf.cpu().numpy().view(np.uint8)[: (K // 128) * rows * 4].reshape(K // 128, rows, 4)
+    return np.ascontiguousarray(b.transpose(1, 0, 2).reshape(rows, K // 32))
+
+
+def sf_weights_to_rows(sf: torch.Tensor, rows: int, K: int) -> np.ndarray:
+    """MOE_SF_WEIGHTS: 256-byte units [rows/64][K/128]; byte (m%32)*8 + (m/32)*4 + j
+    of unit (r/64, s) = tile 4s+j of row r, m = r % 64."""
+    nb = (rows + 63) // 64
+    b = sf.cpu().numpy().view(np.uint8)[: nb * (K // 128) * 256].reshape(nb, K // 128, 32, 2, 4)
+    # -> [unit][m/32][m%32][stage][j]
+    return np.ascontiguousarray(b.transpose(0, 3, 2, 1, 4).reshape(nb * 64, K // 32)[:rows])

@@ -10,13 +10,19 @@ Pages cited (title, section):
       no gradient; the complementary sequence-wise balance loss).
 
 Bar: every gradient within a relative Frobenius error of 2e-5 (fp32 layer) or
-2e-4 (bf16 layer) of the oracle's, and elementwise within 1e-3 of the
-gradient's largest magnitude.  Inputs are exact in both; the kernel
-accumulates in fp32 (relative error ~ K * 2^-24 on the longest sums, K <= a
-few hundred here) against the oracle's float64; in bf16 layers both round
-the recomputed h to bf16, and an h within fp32 error of a rounding boundary
-may land on the other neighbour (2^-8 of one element).  Gradients of experts
-no token chose are exactly zero.
+2e-4 (bf16 layer on the fp32 SIMT path) of the oracle's, and elementwise
+within 1e-3 of the gradient's largest magnitude.  Inputs are exact in both;
+the kernel accumulates in fp32 (relative error ~ K * 2^-24 on the longest
+sums, K <= a few hundred here) against the oracle's float64; in bf16 layers
+both round the recomputed h to bf16, and an h within fp32 error of a
+rounding boundary may land on the other neighbour (2^-8 of one element).
+bf16 layers whose widths are multiples of 128 run their contractions on the
+tensor cores with bf16 operands: do = w dy, da, dg (and dy for the shared
+experts) are rounded to bf16 (relative error up to 2^-9 each, about 1e-3
+RMS, carried into every gradient built from them, twice for dx), so there
+the bar is the forward's bf16 one: 5e-3 relative Frobenius, elementwise 5e-3
+of the largest magnitude.  Gradients of experts no token chose are exactly
+zero on both paths.
 """
 import numpy as np
 import pytest
@@ -71,14 +77,25 @@ def _run(cfg, alpha=0.0, seq_len=0, bias=None):
     return got, ref, float(loss.item()), idx.cpu().numpy()
 
 
-def _check(got, ref, tol):
+def _tensor_cores(c):
+    """The tensor-core path: bf16 and every width a multiple of 128."""
+    return c["dtype"] == "bf16" and c["d"] % 128 == 0 and c["I"] % 128 == 0 and (c["S"] == 0 or c["Is"] % 128 == 0)
+
+
+def _tols(c):
+    if c["dtype"] == "f32":
+        return 2e-5, 1e-3
+    return (5e-3, 5e-3) if _tensor_cores(c) else (2e-4, 1e-3)
+
+
+def _check(got, ref, tol, elem=1e-3):
     for n in NAMES:
         if got[n] is None:
             continue
         g, r = got[n], ref[n]
         assert np.all(np.isfinite(g)), n
         assert rel_fro(g, r) < tol, (n, rel_fro(g, r))
-        assert np.max(np.abs(g - r)) <= 1e-3 * max(np.max(np.abs(r)), 1e-30), n
+        assert np.max(np.abs(g - r)) <= elem * max(np.max(np.abs(r)), 1e-30), (n, np.max(np.abs(g - r)))
 
 
 CASES = {
@@ -86,6 +103,12 @@ CASES = {
     "bf16_ragged_two_shared": dict(dtype="bf16", T=200, d=192, E=16, k=4, I=256, S=2, Is=128),
     "bf16_no_shared": dict(dtype="bf16", T=130, d=64, E=12, k=3, I=128, S=0, Is=128),
     "f32": dict(dtype="f32", T=50, d=40, E=6, k=3, I=24, S=1, Is=16),
+    # tensor-core path: ragged experts, two shared experts, partial 256-wide tiles
+    # (d, I = 384), experts of several 256-row token tiles and 64-row stages
+    "tc_ragged_two_shared": dict(dtype="bf16", T=200, d=256, E=16, k=4, I=256, S=2, Is=128),
+    "tc_wide": dict(dtype="bf16", T=300, d=384, E=8, k=2, I=384, S=1, Is=256),
+    "tc_big_experts": dict(dtype="bf16", T=600, d=256, E=4, k=2, I=256, S=1, Is=128),
+    "tc_no_shared": dict(dtype="bf16", T=130, d=128, E=12, k=3, I=128, S=0, Is=128),
 }
 
 
@@ -97,7 +120,7 @@ def test_backward_matches_oracle(name, alpha):
                                        **c)
     L = 10 if c["T"] % 10 == 0 else c["T"]
     got, ref, loss, _ = _run(cfg, alpha=alpha, seq_len=L if alpha > 0 else 0)
-    _check(got, ref, 2e-5 if c["dtype"] == "f32" else 2e-4)
+    _check(got, ref, *_tols(c))
     if alpha > 0:
         assert abs(loss - ref["balance_loss"]) <= 1e-5 * abs(ref["balance_loss"])
     else:
@@ -115,7 +138,7 @@ def test_backward_unchosen_experts_get_zero_gradient():
     assert set(np.unique(idx)) <= {0, 1, 2, 3}
     for n in ("dw1", "dw3", "dw2"):
         assert np.all(got[n][4:] == 0.0), n
-    _check(got, ref, 2e-4)
+    _check(got, ref, *_tols(dict(dtype="bf16", d=128, I=128, S=1, Is=128)))
 
 
 def test_backward_pages_balance_weight_and_long_sequence():
@@ -123,7 +146,7 @@ def test_backward_pages_balance_weight_and_long_sequence():
     cfg = CONFIGS["small_bf16"].scaled(name="bwd_seq", T=256, d=128, E=32, k=4, I=128, S=1, Is=128, w_std=0.05,
                                        bias_kind="uniform", bias_range=0.02, seed=5)
     got, ref, loss, _ = _run(cfg, alpha=1e-4, seq_len=256)
-    _check(got, ref, 2e-4)
+    _check(got, ref, *_tols(dict(dtype="bf16", d=128, I=128, S=1, Is=128)))
     assert abs(loss - ref["balance_loss"]) <= 1e-5 * abs(ref["balance_loss"])
 
 

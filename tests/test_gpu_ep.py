@@ -6,10 +6,10 @@ dispatch/combine kernels).
 
 Bars: every rank's layer output against the CPU oracle's layer over the
 ranks' concatenated batch with the ranks' own routing (relative Frobenius
-5e-3 bf16 / 1e-5 fp32, and bf16 element by element within the rounding
-bound); and, bit for bit, the single-GPU layer over the same batch -- the
-receive buffers hold each expert's rows in the single-GPU permutation's
-order, so the same tiles compute the same sums.
+5e-3 bf16 / 1e-5 fp32); and, bit for bit, the single-GPU layer over the same
+batch -- the receive buffers hold each expert's rows in the single-GPU
+permutation's order, so the same tiles compute the same sums (the
+single-GPU kernels are checked element by element in the parity tests).
 """
 import numpy as np
 import pytest
@@ -21,7 +21,7 @@ from fine_grained_moe_gate_b200.inputs import CONFIGS, make_layer, make_tokens
 
 import oracle
 from fine_grained_moe_gate_b200.inputs import to_numpy
-from gpu_harness import DEV, as_f64, check_layer_elementwise, check_status, oracle_terms, rel_fro, to_f64_rows
+from gpu_harness import DEV, as_f64, check_status, rel_fro, to_f64_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -76,9 +76,6 @@ def _oracle_check(cfg, world, p, xs, bufs, outs):
                               n["ws3"], n["ws2"])
     err = rel_fro(as_f64(got), to_f64_rows(ref))
     assert err <= (5e-3 if cfg.dtype == "bf16" else 1e-5), err
-    if cfg.dtype == "bf16":
-        y_ref, mag = oracle_terms(p, x, idx, w, np.arange(x.shape[0]), cfg.S)
-        check_layer_elementwise(got, y_ref, mag)
 
 
 def _single_gpu(cfg, world, p, xs, bufs):

@@ -13,7 +13,7 @@ import oracle
 from fine_grained_moe_gate_b200.inputs import CONFIGS, make_layer, make_tokens, to_numpy
 
 from gpu_harness import (DEV, as_f64, check_bf16_close, check_layer_elementwise, check_route_parity, check_status,
-                         layer_forward, oracle_rows, oracle_terms, permute, rel_fro, route, to_f64_rows)
+                         layer_forward, oracle_terms, oracle_terms_from_h, permute, rel_fro, route, to_f64_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -98,7 +98,7 @@ def _projection_checks(cfg, p, x, idx, counts, y_layer, w):
                                         to_numpy(p["ws2"][s][torch.as_tensor(fd, device=DEV)]))
         check_bf16_close(as_f64(shared_out[rt][:, torch.as_tensor(fd, device=DEV)]), o_ref,
                          f"{cfg.name} shared_out")
-    return picks
+    return h, hs, inv
 
 
 def _full_check(cfg, p, x, n_sample, seed, s_tol="auto", projections=False):
@@ -111,12 +111,18 @@ def _full_check(cfg, p, x, n_sample, seed, s_tol="auto", projections=False):
     rows = np.sort(rng.choice(cfg.T, size=min(64, cfg.T), replace=False))
     check_route_parity(x, p["w_gate"], p["bias"], cfg.k, idx, w, counts, aff, s_tol, self_rows=rows)
     assert int(counts.sum()) == cfg.T * cfg.k       # no dropped tokens
-    if projections:
-        _projection_checks(cfg, p, x, idx, counts, y, w)
     tokens = np.sort(rng.choice(cfg.T, size=min(n_sample, cfg.T), replace=False))
-    y_ref, mag = oracle_terms(p, x, idx, w, tokens, cfg.S)
-    err = check_layer_elementwise(y[torch.as_tensor(tokens, device=DEV)], y_ref, mag)
+    yt = y[torch.as_tensor(tokens, device=DEV)]
+    # the benchmark spec bar against the oracle computed from scratch
+    y_ref, _ = oracle_terms(p, x, idx, w, tokens, cfg.S)
+    err = rel_fro(as_f64(yt), to_f64_rows(oracle.finalize(y_ref, np.uint16)))
     assert err <= 5e-3, err
+    if projections:
+        # every kernel's output element by element: the projections, then the down projections and
+        # the combine of the sampled tokens from the GPU's own h
+        h, hs, inv = _projection_checks(cfg, p, x, idx, counts, y, w)
+        y_ref_h, mag = oracle_terms_from_h(p, h, hs, idx, w, inv, tokens, cfg.S)
+        check_layer_elementwise(yt, y_ref_h, mag)
     return y, idx, w, counts
 
 
@@ -216,33 +222,35 @@ def test_skew_stress_bias_trajectory_200_steps():
 
 # ------------------------------------------------------------------ FP8 experts
 
-def _oracle_rows_fp8(q, x, idx, w, tokens, cfg):
-    """The oracle's FP8 layer output for the sampled tokens (page: "DeepSeek
-    V3 Architecture Deep Dive ...", "FP8 Formats"): tokens quantized per row,
-    every expert they use run from its E4M3 codes (brought back one expert at
-    a time), h quantized per assignment row, outputs summed in double."""
+def _oracle_rows_fp8(p, x, idx, w, tokens, cfg):
+    """The oracle's per-tile FP8 layer output for the sampled tokens ("DeepSeek
+    V3 From Scratch", "The idea": fine-grained quantization tiles): tokens
+    quantized by tiles, every expert they use quantized by the oracle from
+    its bf16 weights (one expert at a time) and run from its E4M3 codes, h
+    quantized by tiles per assignment row, outputs summed in double."""
     from fine_grained_moe_gate_b200.inputs import to_numpy
     d, I, S, Is = cfg.d, cfg.I, cfg.S, cfg.Is
     tokens = np.asarray(tokens)
-    xq, xs = oracle.quantize_rows_fp8(to_numpy(x[torch.as_tensor(tokens, device=DEV)]))
+    xq, xe = oracle.quantize_mx(to_numpy(x[torch.as_tensor(tokens, device=DEV)]))
     yacc = np.zeros((len(tokens), d), np.float64)
     if S > 0:
-        h = oracle.expert_up_fp8(xq, xs, q["ws1q"].reshape(S * Is, d).cpu().numpy(), q["ws1s"].cpu().numpy(),
-                                 q["ws3q"].reshape(S * Is, d).cpu().numpy(), q["ws3s"].cpu().numpy())
-        hq, hs = oracle.quantize_rows_fp8(h)
-        yacc += oracle.expert_down_fp8(hq, hs, q["ws2q"].cpu().numpy(), q["ws2s"].cpu().numpy())
+        q1, e1 = oracle.quantize_mx(to_numpy(p["ws1"]).reshape(S * Is, d))
+        q3, e3 = oracle.quantize_mx(to_numpy(p["ws3"]).reshape(S * Is, d))
+        q2, e2 = oracle.quantize_mx(to_numpy(p["ws2"]), nseg=S)
+        hq, he = oracle.quantize_mx(oracle.expert_up_mx(xq, xe, q1, e1, q3, e3))
+        yacc += oracle.expert_down_mx(hq, he, q2, e2)
     idx_np, w_np = idx.cpu().numpy()[tokens], w.cpu().numpy()[tokens]
     for e in np.unique(idx_np):
         ii, jj = np.nonzero(idx_np == e)
-        h = oracle.expert_up_fp8(xq[ii], xs[ii], q["w1q"][e].cpu().numpy(), q["w1s"][e * I:(e + 1) * I].cpu().numpy(),
-                                 q["w3q"][e].cpu().numpy(), q["w3s"][e * I:(e + 1) * I].cpu().numpy())
-        hq, hs = oracle.quantize_rows_fp8(h)
-        o = oracle.expert_down_fp8(hq, hs, q["w2q"][e].cpu().numpy(), q["w2s"][e * d:(e + 1) * d].cpu().numpy())
-        yacc[ii] += w_np[ii, jj].astype(np.float64)[:, None] * o
+        q1, e1 = oracle.quantize_mx(to_numpy(p["w1"][e]))
+        q3, e3 = oracle.quantize_mx(to_numpy(p["w3"][e]))
+        q2, e2 = oracle.quantize_mx(to_numpy(p["w2"][e]))
+        hq, he = oracle.quantize_mx(oracle.expert_up_mx(xq[ii], xe[ii], q1, e1, q3, e3))
+        yacc[ii] += w_np[ii, jj].astype(np.float64)[:, None] * oracle.expert_down_mx(hq, he, q2, e2)
     return oracle.finalize(yacc, np.uint16)
 
 
-def _fp8_check(cfg, p, q, w8, x, n_sample, seed):
+def _fp8_check(cfg, p, w8, x, n_sample, seed):
     sh = moe.shape_of(cfg)
     T, k, d, E = cfg.T, cfg.k, cfg.d, cfg.E
     y = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
@@ -256,32 +264,35 @@ def _fp8_check(cfg, p, q, w8, x, n_sample, seed):
     ridx, rw, rcounts, _ = route(sh, x, p["w_gate"], p["bias"], with_aff=False)   # routing is the bf16 path's
     assert torch.equal(ridx, idx) and torch.equal(rw, w) and torch.equal(rcounts, counts)
     tokens = np.sort(np.random.default_rng(seed).choice(T, size=n_sample, replace=False))
-    ref = to_f64_rows(_oracle_rows_fp8(q, x, idx, w, tokens, cfg))
+    ref = to_f64_rows(_oracle_rows_fp8(p, x, idx, w, tokens, cfg))
     got = as_f64(y[torch.as_tensor(tokens, device=DEV)])
     err = rel_fro(got, ref)
     assert err <= 5e-3, err
 
 
 def test_v3_fp8_prefill_and_decode(v3_layer):
-    """V3 prefill (T=8192) and decode calls with E4M3 experts through
-    moe_layer_forward_fp8 (what the bench times); the weights are quantized on
-    the device and checked bit for bit on three sampled experts."""
+    """V3 prefill (T=8192) and decode calls with per-tile E4M3 experts
+    through moe_layer_forward_fp8 (what the bench times); the weights are
+    quantized on the device and checked bit for bit (codes and tile
+    exponents) on three sampled experts."""
+    from gpu_harness import sf_weights_to_rows
     _, p = v3_layer
     q = moe.quantize_experts_fp8(p)
     w8 = moe.fp8_experts(q)
     torch.cuda.synchronize()
     check_status()
-    from fine_grained_moe_gate_b200.inputs import to_numpy
-    for e in (0, 77, 255):
-        for n in ("w1", "w2"):
-            qo, so = oracle.quantize_rows_fp8(to_numpy(p[n][e]))
-            rows = p[n].shape[1]
+    for n in ("w1", "w2"):
+        rows, K = p[n].shape[1], p[n].shape[2]
+        E = p[n].shape[0]
+        ex = sf_weights_to_rows(q[n + "s"], E * rows, K)
+        for e in (0, 77, 255):
+            qo, eo = oracle.quantize_mx(to_numpy(p[n][e]))
             assert np.array_equal(q[n + "q"][e].cpu().numpy(), qo)
-            assert np.array_equal(q[n + "s"][e * rows:(e + 1) * rows].cpu().numpy(), so)
+            assert np.array_equal(ex[e * rows:(e + 1) * rows], eo)
     cfg = CONFIGS["v3_prefill_fp8"]
-    _fp8_check(cfg, p, q, w8, make_tokens(cfg, DEV), n_sample=4, seed=12)
+    _fp8_check(cfg, p, w8, make_tokens(cfg, DEV), n_sample=16, seed=12)
     cfg = CONFIGS["v3_decode_fp8"]
     for call in (0, 999):
-        _fp8_check(cfg, p, q, w8, make_tokens(cfg, DEV, call), n_sample=3, seed=call)
+        _fp8_check(cfg, p, w8, make_tokens(cfg, DEV, call), n_sample=8, seed=call)
     del q, w8
     torch.cuda.empty_cache()

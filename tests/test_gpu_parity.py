@@ -17,7 +17,8 @@ import oracle
 from fine_grained_moe_gate_b200.inputs import CONFIGS, make_layer, make_tokens, to_numpy
 
 from gpu_harness import (DEV, as_f64, check_layer_elementwise, check_route_parity, check_status, grouped_swiglu,
-                         layer_forward, oracle_rows, oracle_terms, permute, rel_fro, route, to_f64_rows)
+                         layer_forward, oracle_rows, oracle_terms, oracle_terms_from_h, permute, rel_fro, route,
+                         to_f64_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -340,8 +341,15 @@ def test_layer_bf16_against_oracle(shape):
                               n["ws3"], n["ws2"])
     err = rel_fro(as_f64(y), to_f64_rows(ref))
     assert err <= 5e-3, err
-    # element by element, every token: within the bf16 bound the roundings allow
-    y_ref, mag = oracle_terms(p, x, idx, w, np.arange(cfg.T), cfg.S)
+    # element by element, every token, against the oracle's down projections and combine of the
+    # GPU's own h (the staged calls, bit-identical to the layer)
+    x_perm, offsets, perm, inv = permute(sh, x, idx, counts)
+    T, k, I, S, Is = cfg.T, cfg.k, cfg.I, cfg.S, cfg.Is
+    h = torch.empty((T * k, I), dtype=torch.bfloat16, device=DEV)
+    hs = torch.empty((T, max(1, S * Is)), dtype=torch.bfloat16, device=DEV)
+    moe.moe_ffn_up(x_perm, offsets, p["w1"], p["w3"], x if S else None, p["ws1"], p["ws3"], sh, h, hs)
+    torch.cuda.synchronize()
+    y_ref, mag = oracle_terms_from_h(p, h, hs, idx, w, inv, np.arange(T), S)
     check_layer_elementwise(y, y_ref, mag)
 
 
@@ -436,3 +444,34 @@ def test_bounded_wait_times_out_and_context_survives():
     check_status()
     assert int(counts.sum()) == cfg.T * cfg.k
     assert torch.isfinite(y.float()).all()
+
+
+@pytest.mark.parametrize("shape", [
+    dict(T=512, d=512, E=64, k=6, I=256, S=2, Is=256),
+    dict(T=300, d=256, E=256, k=8, I=128, S=1, Is=128),
+    dict(T=96, d=384, E=8, k=8, I=128, S=0, Is=128),       # no shared set; d % 256 == 128
+])
+def test_down_with_fused_combine_against_oracle(shape):
+    """moe_ffn_down_combine + moe_combine_finish (the weighted combine in the
+    down projection's epilogue, fp32 additions) against the oracle's layer,
+    element by element, and the accumulator left cleared."""
+    cfg = SMALL.scaled(**shape, w_std=0.05, bias_kind="uniform", bias_range=0.02)
+    sh = moe.shape_of(cfg)
+    p = make_layer(cfg, DEV)
+    x = make_tokens(cfg, DEV)
+    T, k, d, I, S, Is = cfg.T, cfg.k, cfg.d, cfg.I, cfg.S, cfg.Is
+    idx, w, counts, _ = route(sh, x, p["w_gate"], p["bias"], with_aff=False)
+    x_perm, offsets, perm, inv = permute(sh, x, idx, counts)
+    h = torch.empty((T * k, I), dtype=torch.bfloat16, device=DEV)
+    hs = torch.empty((T, max(1, S * Is)), dtype=torch.bfloat16, device=DEV)
+    moe.moe_ffn_up(x_perm, offsets, p["w1"], p["w3"], x if S else None, p["ws1"], p["ws3"], sh, h, hs)
+    acc = torch.zeros((T, d), dtype=torch.float32, device=DEV)
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    moe.moe_ffn_down_combine(h, offsets, p["w2"], hs if S else None, p["ws2"], perm, w, sh, acc)
+    moe.moe_combine_finish(acc, sh, y)
+    torch.cuda.synchronize()
+    check_status()
+    assert bool((acc == 0).all()), "accumulator not cleared"
+    y_ref, mag = oracle_terms_from_h(p, h, hs, idx, w, inv, np.arange(T), S)
+    err = check_layer_elementwise(y, y_ref, mag)
+    assert err <= 5e-3, err
