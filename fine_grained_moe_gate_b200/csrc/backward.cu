@@ -584,19 +584,31 @@ __global__ void __launch_bounds__(256) combine_bwd_pad_kernel(const float* __res
 
 // SwiGLU derivative on the real rows: with s = sigmoid(a),
 //   da = dh g s (1 + a (1 - s)),  dg = dh a s,
-// stored bf16 side by side: dadg[pr][c] = da, dadg[pr][n + c] = dg.
+// stored bf16 side by side: dadg[pr][c] = da, dadg[pr][n + c] = dg.  Four
+// columns per thread (n % 4 == 0): 16-byte loads, 8-byte stores.
 __global__ void swiglu_bwd_pad_kernel(const float* __restrict__ a, const float* __restrict__ g,
                                       const float* __restrict__ dh, const int32_t* __restrict__ prow, int R, int n,
                                       uint16_t* __restrict__ dadg) {
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)R * n;
+    const int n4 = n / 4;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)R * n4;
          i += (long long)gridDim.x * blockDim.x) {
-        const int r = (int)(i / n), c = (int)(i - (long long)r * n);
+        const int r = (int)(i / n4), c = (int)(i - (long long)r * n4);
         const long long pr = prow ? prow[r] : r;
-        const float av = a[pr * n + c], gv = g[pr * n + c], dv = dh[pr * n + c];
-        const float s = sigmoid_acc(av);
-        __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(dadg + pr * 2 * n);
-        row[c] = __float2bfloat16_rn(dv * gv * s * (1.0f + av * (1.0f - s)));
-        row[n + c] = __float2bfloat16_rn(dv * av * s);
+        const float4 av = reinterpret_cast<const float4*>(a + pr * n)[c];
+        const float4 gv = reinterpret_cast<const float4*>(g + pr * n)[c];
+        const float4 dv = reinterpret_cast<const float4*>(dh + pr * n)[c];
+        const float al[4] = {av.x, av.y, av.z, av.w}, gl[4] = {gv.x, gv.y, gv.z, gv.w},
+                    dl[4] = {dv.x, dv.y, dv.z, dv.w};
+        float da[4], dg[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float s = sigmoid_acc(al[u]);
+            da[u] = dl[u] * gl[u] * s * (1.0f + al[u] * (1.0f - s));
+            dg[u] = dl[u] * al[u] * s;
+        }
+        uint2* row = reinterpret_cast<uint2*>(dadg + pr * 2 * n);
+        row[c] = make_uint2(bf16x2(da[0], da[1]), bf16x2(da[2], da[3]));
+        row[n4 + c] = make_uint2(bf16x2(dg[0], dg[1]), bf16x2(dg[2], dg[3]));
     }
 }
 
@@ -691,7 +703,7 @@ struct BwdBufs {
     float *abuf, *gbuf, *hbuf, *dhbuf, *obuf, *as, *gs, *hs, *dhs;
     // tensor-core path: routed rows in the padded layout (Rp rows), shared rows T
     int32_t *pstart, *prow;
-    uint16_t *x_pad, *h_pad, *do_pad, *dadg, *hs16, *dys16, *dadgs;
+    uint16_t *x_pad, *h_pad, *do_pad, *dadg, *hs16, *dys16, *dadgs, *dz16;
     float *a_pad, *g_pad, *o_pad, *dh_pad, *as32, *gs32, *dhs32;
 };
 
@@ -740,6 +752,7 @@ size_t carve(BwdBufs* o, char* base, int T, int d, int E, int k, int I, int S, i
         b.hs16 = c.take<uint16_t>((size_t)T * SI * 2);
         b.dys16 = c.take<uint16_t>((size_t)T * d * 2);
         b.dadgs = c.take<uint16_t>((size_t)T * 2 * SI * 2);
+        b.dz16 = c.take<uint16_t>((size_t)T * E * 2);
     }
     if (o) *o = b;
     return c.used;
@@ -846,8 +859,8 @@ cudaError_t experts_backward_tc(const BackwardArgs& a, const BwdBufs& b, int* st
         TC_TRY(launch_bwd_rows_mnmajor(r, status, num_sms, st));
     }
     if (R > 0) {
-        swiglu_bwd_pad_kernel<<<ew_grid((long long)R * I), 256, 0, st>>>(b.a_pad, b.g_pad, b.dh_pad, b.prow, R, I,
-                                                                         b.dadg);
+        swiglu_bwd_pad_kernel<<<ew_grid((long long)R * I / 4), 256, 0, st>>>(b.a_pad, b.g_pad, b.dh_pad, b.prow, R,
+                                                                             I, b.dadg);
         note_launches(1);
     }
     // dW1_e = da^T x, dW3_e = dg^T x
@@ -886,8 +899,8 @@ cudaError_t experts_backward_tc(const BackwardArgs& a, const BwdBufs& b, int* st
             r.ldo = SI;
             TC_TRY(launch_bwd_rows_mnmajor(r, status, num_sms, st));
         }
-        swiglu_bwd_pad_kernel<<<ew_grid((long long)T * SI), 256, 0, st>>>(b.as32, b.gs32, b.dhs32, nullptr, T, SI,
-                                                                          b.dadgs);
+        swiglu_bwd_pad_kernel<<<ew_grid((long long)T * SI / 4), 256, 0, st>>>(b.as32, b.gs32, b.dhs32, nullptr, T,
+                                                                              SI, b.dadgs);
         note_launches(1);
         TC_TRY(launch_bwd_wgrad(wgrad_args(b.dadgs, 2 * SI, 0, a.x, d, 0, T, SI, d, a.dws1, false), status, num_sms,
                                 st));
@@ -1031,12 +1044,58 @@ cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sm
             balance_sum_kernel<<<1, 32, 0, st>>>(part, nb, a.loss);
             note_launches(3);
         }
-        // dx += dz W_g;  dW_g = dz^T x
-        BWD_TRY(rows_gemm(view(dz, false, E, 1), view(a.w_gate, bf, 1, d), a.dx, d, T, d, E, nullptr, 1, true, status,
-                          a.num_sms, st));
+        // dx += dz W_g;  dW_g = dz^T x.  On the tensor-core path with dz in bf16: dW_g whenever E % 8 == 0
+        // (16-byte rows of dz), dx when E % 64 == 0 (whole 64-column stages of the contraction).
+        if (tc && E % 8 == 0) {
+            to_bf16_kernel<<<ew_grid((long long)T * E), 256, 0, st>>>(dz, (long long)T * E,
+                                                                      reinterpret_cast<__nv_bfloat16*>(bb.dz16));
+            note_launches(1);
+        }
+        if (tc && E % 64 == 0) {
+            BwdRowsArgs r{};
+            r.W = a.w_gate;
+            r.W1 = nullptr;
+            r.W_rows = E;
+            r.K0 = 0;
+            r.a_grow = 0;
+            r.X = bb.dz16;
+            r.op_rows = T;
+            r.K = E;
+            r.M_total = d;
+            r.start = nullptr;
+            r.rows = nullptr;
+            r.G = 1;
+            r.M_rows = T;
+            r.out = a.dx;
+            r.ldo = d;
+            r.accumulate = true;
+            BWD_TRY(launch_bwd_rows_mnmajor(r, status, num_sms, st));
+        } else {
+            BWD_TRY(rows_gemm(view(dz, false, E, 1), view(a.w_gate, bf, 1, d), a.dx, d, T, d, E, nullptr, 1, true,
+                              status, a.num_sms, st));
+        }
     }
-    BWD_TRY(wgrad_gemm(view(dz, false, E, 1), view(a.x, bf, d, 1), a.dw_gate, d, 0, E, d, nullptr, 1, T, false, status,
-                       st));
+    if (tc && E % 8 == 0 && T > 0) {
+        BwdWgradArgs w{};
+        w.A = bb.dz16;
+        w.lda = E;
+        w.a_col0 = 0;
+        w.B = a.x;
+        w.ldb = d;
+        w.b_col0 = 0;
+        w.op_rows = T;
+        w.M_total = E;
+        w.N_total = d;
+        w.start = nullptr;
+        w.rows = nullptr;
+        w.G = 1;
+        w.M_rows = T;
+        w.out = a.dw_gate;
+        BWD_TRY(launch_bwd_wgrad(w, status, num_sms, st));
+    } else {
+        BWD_TRY(wgrad_gemm(view(dz, false, E, 1), view(a.x, bf, d, 1), a.dw_gate, d, 0, E, d, nullptr, 1, T, false,
+                           status, st));
+    }
     if (a.loss && nb == 0) BWD_TRY(cudaMemsetAsync(a.loss, 0, sizeof(float), st));
 #undef BWD_TRY
     return cudaSuccess;

@@ -111,6 +111,19 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr) {
     return d;
 }
 
+// 32 lanes x 32 bits, 32 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
@@ -423,26 +436,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACC_COLS;
             const int mcta = ti.m0 + (int)rank * 128;  // this CTA's first M row
             if (WG) {
-                // D[m][n]: lane = m, column = n; each thread stores 16 fp32 of its row per chunk
+                // D[m][n]: lane = m, column = n; each thread stores its row 32 columns at a time (128
+                // contiguous bytes), the TMEM read of the next 32 columns in flight meanwhile
                 const int m = mcta + q * 32 + lane;
                 float* dst = p.out + (size_t)t.g * p.out_gstride + (size_t)m * p.ldo + ti.n0;
                 const bool row_ok = m < p.M_total;
-                for (int c = 0; c < ti.ntok; c += 16) {
-                    uint32_t r[16];
+                // two register sets in turn (the loop is unrolled by two so that both stay in registers)
+                uint32_t r0[32], r1[32];
+                const auto store32 = [&](int c, const uint32_t (&v)[32]) {
+                    if (!row_ok) return;
+                    float4* d4 = reinterpret_cast<float4*>(dst + c);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        d4[i] = ti.kb > 0 ? make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]))
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                };
+                if (ti.kb > 0) tmem_ld32(taddr, r0);
+                for (int c = 0; c < ti.ntok; c += 64) {  // ntok is a multiple of 128
                     if (ti.kb > 0) {
-                        tmem_ld16(taddr + (uint32_t)c, r);
                         tmem_ld_wait();
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) r[i] = 0u;
+                        tmem_ld32(taddr + (uint32_t)(c + 32), r1);
                     }
-                    if (row_ok) {
-                        float4* d4 = reinterpret_cast<float4*>(dst + c);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                    store32(c, r0);
+                    if (ti.kb > 0) {
+                        tmem_ld_wait();
+                        if (c + 64 < ti.ntok) tmem_ld32(taddr + (uint32_t)(c + 64), r0);
                     }
+                    store32(c + 32, r1);
                 }
             } else {
                 // D[m][token]: 16-token chunks through shared memory, token-major fp32 rows
@@ -569,7 +590,8 @@ cudaError_t launch_bwd_rows_mnmajor(const BwdRowsArgs& a, int* status, int num_s
 //   A: [op_rows][lda] bf16, B: [op_rows][ldb] bf16, out: [G][M_total][N_total] fp32.
 cudaError_t launch_bwd_wgrad(const BwdWgradArgs& a, int* status, int num_sms, cudaStream_t st) {
     Maps m{};
-    if (a.M_total % 128 != 0 || a.N_total % 128 != 0) return cudaErrorInvalidValue;
+    // M: the 64-wide boxes past M_total read zeros and those rows are not stored; N: whole 128-column halves
+    if (a.M_total % 8 != 0 || a.N_total % 128 != 0) return cudaErrorInvalidValue;
     // the boxes start at column a_col0 + m (b_col0 + n): a view that begins there keeps the 16-byte rule
     const uint16_t* A = static_cast<const uint16_t*>(a.A) + a.a_col0;
     const uint16_t* B = static_cast<const uint16_t*>(a.B) + a.b_col0;
