@@ -57,7 +57,7 @@ if ROOT not in sys.path:
 METRIC = "MoE layer fwd tokens/s (V3-shaped, bf16) and % of BF16 tensor / HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES = ["route", "permute", "ffn_up", "ffn_down", "combine", "bias_update"]
-# E4M3 expert workloads: token rows and h are quantized per row in the step
+# E4M3 expert workloads: token rows and h are quantized (1x32 tiles) in the step
 STAGES_FP8 = ["route", "quant_x", "permute", "ffn_up", "quant_h", "ffn_down", "combine", "bias_update"]
 DOMINANT = "ffn_up"
 WORKLOADS = ["v3_prefill", "v3_decode", "small_bf16", "skew_stress", "tiny_fp32", "v3_prefill_fp8",
@@ -76,6 +76,8 @@ def parse_args():
     ap.add_argument("--cpu-tokens", type=int, default=0, help="oracle sample size (0: per-workload default)")
     ap.add_argument("--T", type=int, default=0, help="override tokens per GPU (profiling slices)")
     ap.add_argument("--E", type=int, default=0, help="override routed experts (profiling slices)")
+    ap.add_argument("--I", type=int, default=0,
+                    help="override the expert width I = Is (profiling slices: the router at full size in little memory)")
     ap.add_argument("--no-extra", action="store_true",
                     help="v3_prefill only: skip the decode and skew workloads of the default line")
     ap.add_argument("--decode-calls", type=int, default=1000, help="decode workload: timed calls (fresh x each)")
@@ -320,6 +322,8 @@ def workload(args):
         over["T"] = args.T
     if args.E:
         over["E"] = args.E
+    if args.I:
+        over["I"] = over["Is"] = args.I
     if over:
         tag = ",".join(f"{k}={v}" for k, v in over.items())
         cfg = cfg.scaled(name=f"{cfg.name}[{tag}]", **over)
@@ -699,7 +703,7 @@ def run_ours(args, world, rank, local):
 
     # ---- the other workloads of the default line (decode-shaped, skewed routing)
     extras = {}
-    if not args.no_extra and args.workload == "v3_prefill" and not (args.T or args.E):
+    if not args.no_extra and args.workload == "v3_prefill" and not (args.T or args.E or args.I):
         del step, xs
         p.clear()
         torch.cuda.empty_cache()

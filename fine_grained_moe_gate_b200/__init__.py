@@ -64,7 +64,7 @@ def shape_of(cfg, T: int | None = None) -> MoEShape:
 
 
 class MoEFp8Experts(ctypes.Structure):
-    """moe_fp8_experts: E4M3 expert weights and their per-row fp32 scales."""
+    """moe_fp8_experts: E4M3 expert weights and their 1x32-tile power-of-two scales (weight layout)."""
     _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "w1_scale", "w3", "w3_scale", "w2", "w2_scale",
                                                "ws1", "ws1_scale", "ws3", "ws3_scale", "ws2", "ws2_scale")]
 

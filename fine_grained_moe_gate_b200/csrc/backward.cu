@@ -555,31 +555,40 @@ __global__ void swiglu_h_kernel(const float* __restrict__ a, const float* __rest
     }
 }
 
-// One block per assignment q = t*k + j (row r = inv[q], padded row pr):
-// dw[q] = <dy_t, o[pr]>, do[pr] = bf16(w[q] dy_t).
+// One warp per assignment q = t*k + j (row r = inv[q], padded row pr):
+// dw[q] = <dy_t, o[pr]>, do[pr] = bf16(w[q] dy_t).  d % 4 == 0: 16-byte
+// loads, 8-byte stores.
 __global__ void __launch_bounds__(256) combine_bwd_pad_kernel(const float* __restrict__ dy, const float* __restrict__ w,
                                                               const int32_t* __restrict__ inv,
                                                               const int32_t* __restrict__ prow,
                                                               const float* __restrict__ o, float* __restrict__ dw,
                                                               uint16_t* __restrict__ dop, int d, int k, int rows,
-                                                              int* status) {
-    __shared__ float red[32];
-    const int q = blockIdx.x, t = q / k;
+                                                              int nq, int* status) {
+    const int lane = threadIdx.x & 31;
+    const int q = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (q >= nq) return;  // warp-uniform
+    const int t = q / k;
     const int r = inv[q];
     if (r < 0 || r >= rows) {
-        if (threadIdx.x == 0) report(status, kStDeviceCheck);
+        if (lane == 0) report(status, kStDeviceCheck);
         return;
     }
     const long long pr = prow[r];
-    const float* dyt = dy + (long long)t * d;
-    const float* orow = o + pr * d;
-    float part = 0.0f;
-    for (int c = threadIdx.x; c < d; c += blockDim.x) part = fmaf(dyt[c], orow[c], part);
-    const float tot = block_sum(part, red);
-    if (threadIdx.x == 0) dw[q] = tot;
+    const float4* dyt = reinterpret_cast<const float4*>(dy + (long long)t * d);
+    const float4* orow = reinterpret_cast<const float4*>(o + pr * d);
+    uint2* dst = reinterpret_cast<uint2*>(dop + pr * d);
     const float wq = w[q];
-    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(dop + pr * d);
-    for (int c = threadIdx.x; c < d; c += blockDim.x) dst[c] = __float2bfloat16_rn(wq * dyt[c]);
+    const int d4 = d / 4;
+    float part = 0.0f;
+#pragma unroll 4
+    for (int c = lane; c < d4; c += 32) {
+        const float4 y = dyt[c], v = orow[c];
+        part = fmaf(y.x, v.x, fmaf(y.y, v.y, fmaf(y.z, v.z, fmaf(y.w, v.w, part))));
+        dst[c] = make_uint2(bf16x2(wq * y.x, wq * y.y), bf16x2(wq * y.z, wq * y.w));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (lane == 0) dw[q] = part;
 }
 
 // SwiGLU derivative on the real rows: with s = sigmoid(a),
@@ -618,22 +627,38 @@ __global__ void to_bf16_kernel(const float* __restrict__ x, long long n, __nv_bf
         y[i] = __float2bfloat16_rn(x[i]);
 }
 
-// dx[t] = sum_j dxp[prow[inv[t*k + j]]] (overwrite), one block per token.
-__global__ void unpermute_sum_pad_kernel(const float* __restrict__ dxp, const int32_t* __restrict__ inv,
-                                         const int32_t* __restrict__ prow, float* dx, int d, int k, int rows,
-                                         int* status) {
-    const int t = blockIdx.x;
-    for (int c = threadIdx.x; c < d; c += blockDim.x) {
-        float v = 0.0f;
+// dx[t] = sum_j dxp[prow[inv[t*k + j]]] (overwrite, j in order), one warp
+// per token; d % 4 == 0: 16-byte loads and stores.
+__global__ void __launch_bounds__(256) unpermute_sum_pad_kernel(const float* __restrict__ dxp,
+                                                                const int32_t* __restrict__ inv,
+                                                                const int32_t* __restrict__ prow, float* dx, int d,
+                                                                int k, int rows, int T, int* status) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;  // warp-uniform
+    // padded row of assignment j in lane j (k <= 32); -1: a corrupt inverse entry, skipped
+    long long my_row = -1;
+    if (lane < k) {
+        const int r = inv[(long long)t * k + lane];
+        if (r < 0 || r >= rows)
+            report(status, kStDeviceCheck);
+        else
+            my_row = prow[r];
+    }
+    const int d4 = d / 4;
+    float4* out = reinterpret_cast<float4*>(dx + (long long)t * d);
+    for (int c = lane; c < d4; c += 32) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
-            const int r = inv[(long long)t * k + j];
-            if (r < 0 || r >= rows) {
-                report(status, kStDeviceCheck);
-                continue;
-            }
-            v += dxp[(long long)prow[r] * d + c];
+            const long long pr = __shfl_sync(0xffffffffu, my_row, j);
+            if (pr < 0) continue;
+            const float4 x = reinterpret_cast<const float4*>(dxp + pr * d)[c];
+            v.x += x.x;
+            v.y += x.y;
+            v.z += x.z;
+            v.w += x.w;
         }
-        dx[(long long)t * d + c] = v;
+        out[c] = v;
     }
 }
 
@@ -848,7 +873,8 @@ cudaError_t experts_backward_tc(const BackwardArgs& a, const BwdBufs& b, int* st
                                   num_sms, st));
     // dw = <dy, o> per assignment; do = w dy (bf16, padded rows)
     if (R > 0) {
-        combine_bwd_pad_kernel<<<R, 256, 0, st>>>(a.dy, a.w, b.inv, b.prow, b.o_pad, b.dw, b.do_pad, d, k, R, status);
+        combine_bwd_pad_kernel<<<(R + 7) / 8, 256, 0, st>>>(a.dy, a.w, b.inv, b.prow, b.o_pad, b.dw, b.do_pad, d, k,
+                                                            R, R, status);
         note_launches(1);
     }
     // dW2_e = do^T h
@@ -874,7 +900,7 @@ cudaError_t experts_backward_tc(const BackwardArgs& a, const BwdBufs& b, int* st
         TC_TRY(launch_bwd_rows_mnmajor(r, status, num_sms, st));
     }
     if (T > 0) {
-        unpermute_sum_pad_kernel<<<T, 256, 0, st>>>(b.o_pad, b.inv, b.prow, a.dx, d, k, R, status);
+        unpermute_sum_pad_kernel<<<(T + 7) / 8, 256, 0, st>>>(b.o_pad, b.inv, b.prow, a.dx, d, k, R, T, status);
         note_launches(1);
     }
 

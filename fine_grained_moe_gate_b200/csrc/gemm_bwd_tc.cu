@@ -80,6 +80,7 @@ struct Maps {
     CUtensorMap a0, a1;   // A: the weights (rows) or the per-row matrix (wgrad); a1: dx's W3
     CUtensorMap b;        // wgrad: MN-major B
     CUtensorMap bx[NXBOX];  // rows: K-major token boxes
+    CUtensorMap o;        // wgrad: the fp32 output [G][M_total][N_total], stored in 32 x 32 boxes
 };
 
 struct BwdParams {
@@ -436,24 +437,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACC_COLS;
             const int mcta = ti.m0 + (int)rank * 128;  // this CTA's first M row
             if (WG) {
-                // D[m][n]: lane = m, column = n; each thread stores its row 32 columns at a time (128
-                // contiguous bytes), the TMEM read of the next 32 columns in flight meanwhile
-                const int m = mcta + q * 32 + lane;
-                float* dst = p.out + (size_t)t.g * p.out_gstride + (size_t)m * p.ldo + ti.n0;
-                const bool row_ok = m < p.M_total;
-                // two register sets in turn (the loop is unrolled by two so that both stay in registers)
+                // D[m][n]: lane = m, column = n.  Per 32 columns the warp's 32 x 32 block goes through its
+                // 4 KB of shared memory (128-byte swizzled rows: 16-byte chunk j of row r at j ^ (r % 8))
+                // and leaves as one TMA store, whole 128-byte lines; rows past M_total are clipped by the
+                // map.  The TMEM read of the next 32 columns is in flight meanwhile.
+                float* sb = xbuf + (warp - 2) * 1024;
+                float4* srow = reinterpret_cast<float4*>(sb + lane * 32);
+                const int mq = mcta + q * 32;
                 uint32_t r0[32], r1[32];
                 const auto store32 = [&](int c, const uint32_t (&v)[32]) {
-                    if (!row_ok) return;
-                    float4* d4 = reinterpret_cast<float4*>(dst + c);
+                    if (lane == 0) bulk_wait_group_read<0>();  // the previous box has left shared memory
+                    __syncwarp();
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
-                        d4[i] = ti.kb > 0 ? make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]))
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                        srow[i ^ (lane & 7)] =
+                            ti.kb > 0 ? make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                    __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&mp.o, sb, ti.n0 + c, mq, t.g);
+                        bulk_commit_group();
+                    }
                 };
-                if (ti.kb > 0) tmem_ld32(taddr, r0);
-                for (int c = 0; c < ti.ntok; c += 64) {  // ntok is a multiple of 128
+                const bool live = mq < p.M_total;  // warp-uniform: a block wholly past M_total is not stored
+                if (live && ti.kb > 0) tmem_ld32(taddr, r0);
+                for (int c = 0; live && c < ti.ntok; c += 64) {  // ntok is a multiple of 128
                     if (ti.kb > 0) {
                         tmem_ld_wait();
                         tmem_ld32(taddr + (uint32_t)(c + 32), r1);
@@ -505,6 +515,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
     }
 
+    if (WG && warp >= 2 && warp < 2 + NEPI && lane == 0) bulk_wait_group<0>();  // the output boxes are written
     tc_fence_before();
     cluster_sync_all();
     if (warp == 1) {
@@ -601,6 +612,10 @@ cudaError_t launch_bwd_wgrad(const BwdWgradArgs& a, int* status, int num_sms, cu
         return cudaErrorInvalidValue;
     m.a1 = m.a0;
     for (int b = 0; b < NXBOX; ++b) m.bx[b] = m.b;
+    if ((reinterpret_cast<uintptr_t>(a.out) & 15u) ||
+        !make_tmap_3d_f32(&m.o, a.out, a.N_total, a.M_total, a.G, a.N_total, (unsigned long long)a.M_total * a.N_total,
+                          32, 32))
+        return cudaErrorInvalidValue;
     BwdParams p{};
     p.G = a.G;
     p.start = a.start;

@@ -242,6 +242,12 @@ struct TileCoord {
     int g, ft, tt;
 };
 
+// Tile order inside a group: the token tiles of a feature tile run back to
+// back, so the clusters that share a weight tile read it at about the same
+// time and DRAM sees it once.  (Running the feature tiles of a token tile back
+// to back instead, for groups with more token tiles than feature tiles, cut
+// the V3 gate/up DRAM reads from 18.4 to 17.5 GB but measured 2% slower there
+// and 12% slower on the skewed batch.)
 __device__ __forceinline__ TileCoord tile_coords(const Tables* tb, int G, int tile) {
     int lo = 0, hi = G - 1;
     while (lo < hi) {  // last group whose first tile is <= tile (never an empty one)
@@ -334,14 +340,6 @@ __device__ __forceinline__ bool tq_take(Ctl* ctl, int j, uint32_t ph, uint32_t l
     *tile = t;
     mbar_arrive_relaxed_cluster(leader_tq_empty + 8u * (uint32_t)j);
     return true;
-}
-
-// After an abort, wait (bounded) for TMA loads this thread issued to land
-// before the CTA releases its shared memory.
-__device__ __forceinline__ void settle_inflight_loads() {
-    const uint64_t t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 200000ull) {
-    }
 }
 
 // A producer other than warp 0: follows the tile queue; per tile, begin(tc)

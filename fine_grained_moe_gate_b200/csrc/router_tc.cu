@@ -2,12 +2,15 @@
 // "In code", route(); "The idea"): gate GEMM + sigmoid + bias-shifted top-k
 // + unbiased renormalised weights + load histogram in one kernel.
 //
-// A tile = 128 tokens.  All E (<= 256) experts fit one tcgen05 MMA: the
-// accumulator is 128 TMEM lanes (tokens) x E columns (experts), fp32.  The
-// K loop over d streams x and W_gate through a 4-stage TMA ring.  Small
-// batches split K over a cluster of up to 8 CTAs per tile (one CTA per tile
-// read all of W_gate alone, 3.7 MB at V3 through one SM); the scores only
-// leave shared memory for the caller's optional affinity output.
+// A tile = 128 tokens in one CTA, or 256 tokens in a CTA pair.  All E (<= 256)
+// experts fit one tcgen05 MMA: each CTA's accumulator is 128 TMEM lanes
+// (tokens) x E columns (experts), fp32.  The K loop over d streams x and
+// W_gate through a TMA ring.  Every token tile reads all of W_gate (3.7 MB at
+// V3) from L2, so large batches run the 2-SM form (cta_group::2, M = 256):
+// each CTA of a pair loads its 128 tokens and half of W_gate's rows, which
+// halves the gate re-reads per token.  Small batches split K over a cluster of
+// CTAs (or pairs) per tile so that enough SMs take part; the scores only leave
+// shared memory for the caller's optional affinity output.
 #include "common.cuh"
 #include "kernels.h"
 #include "tmap.h"
@@ -16,17 +19,32 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int BM = 128, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_STRIDE = 256 * BK * 2;  // room for N <= 256 rows
-constexpr int NTHREADS = 192;
-constexpr int RING_BYTES = STAGES * (A_BYTES + B_STRIDE);
+// One CTA holds all N <= 256 rows of W_gate per stage (4 stages); a CTA of a
+// pair holds N/2 <= 128 rows (6 stages).  Both rings take 192 KB.
+template <bool PAIR>
+__host__ __device__ constexpr int ring_stages() {
+    return PAIR ? 6 : 4;
+}
+template <bool PAIR>
+__host__ __device__ constexpr int b_stride() {
+    return (PAIR ? 128 : 256) * BK * 2;
+}
+constexpr int MAX_STAGES = 6;
+constexpr int RING_BYTES = 4 * (A_BYTES + 256 * BK * 2);
+static_assert(ring_stages<true>() * (A_BYTES + b_stride<true>()) == RING_BYTES, "both rings take the same room");
+// Warps: 0 loads the token boxes (and arms the stage barrier), 6 the W_gate
+// boxes (one issuing thread paces a TMA ring, so two share it), 1 issues the
+// MMAs; after the K loop all eight read the accumulator and finish tokens.
+constexpr int NTHREADS = 256;
+constexpr int kWarpB = 6;
 constexpr int PS = kMaxExperts + 4;  // row stride (floats) of the score buffers
 constexpr int PART_BYTES = BM * PS * 4;
 
 struct Ctl {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[MAX_STAGES];
+    uint64_t empty[MAX_STAGES];
     uint64_t tfull;
     uint64_t drain;
     uint32_t tmem_base;
@@ -49,18 +67,24 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t cluster_addr) {
     return v;
 }
 
-// Split K: the C CTAs of a cluster share one 128-token tile, CTA c running
-// the MMA over its slice of d; the slices' fp32 partial scores are summed in
-// the fixed order c = 0..C-1 through distributed shared memory (deterministic
-// for a given C), CTA c then finishes tokens [c*128/C, (c+1)*128/C) with C
-// threads per token, each taking every C-th expert, whose top-k lists are
-// merged with warp shuffles.  C = 1 is the plain one-CTA tile.
-template <int KMAX, int C>
+// Split K: the C CTAs (or CTA pairs) of a cluster share one token tile, CTA
+// (pair) c running the MMA over its slice of d; the slices' fp32 partial
+// scores are summed in the fixed order c = 0..C-1 through distributed shared
+// memory (deterministic for a given C), CTA c then finishes tokens
+// [c*128/C, (c+1)*128/C) of its 128 with C threads per token, each taking
+// every C-th expert, whose top-k lists are merged with warp shuffles.  C = 1
+// is the plain tile.  PAIR: a cluster of 2C CTAs, ranks 2c and 2c + 1 forming
+// the pair of slice c; the even CTA issues the MMAs, the odd one holds tokens
+// 128..255 of the tile and W_gate rows [N/2, N).
+template <int KMAX, int C, bool PAIR>
 __global__ void __launch_bounds__(NTHREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ bias, int T, int E, int n_pad, uint32_t tmem_cols, int k_blocks,
                      int k, int32_t* __restrict__ idx, float* __restrict__ w, int32_t* __restrict__ counts,
                      float* __restrict__ aff, int* status) {
+    constexpr int STAGES = ring_stages<PAIR>();
+    constexpr int BSTR = b_stride<PAIR>();
+    constexpr int CL = PAIR ? 2 * C : C;  // CTAs per cluster
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sA = base;
@@ -70,9 +94,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const size_t ring_or_scores = RING_BYTES > SCORE_BYTES ? RING_BYTES : SCORE_BYTES;
     Ctl* ctl = reinterpret_cast<Ctl*>(base + ring_or_scores);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int crank = C > 1 ? (int)cluster_ctarank() : 0;
-    const int t0 = (blockIdx.x / C) * BM;
-    const int kb0 = crank * k_blocks / C, kb1 = (crank + 1) * k_blocks / C;
+    const int crank = CL > 1 ? (int)cluster_ctarank() : 0;
+    const int half = PAIR ? (crank & 1) : 0;        // which 128 tokens of a pair's tile
+    const int slice = PAIR ? (crank >> 1) : crank;  // K slice
+    const uint32_t leader = (uint32_t)(crank - half);
+    const uint16_t pair_mask = (uint16_t)(3u << leader);
+    const int t0 = (blockIdx.x / CL) * (PAIR ? 2 * BM : BM) + half * BM;
+    const int kb0 = slice * k_blocks / C, kb1 = (slice + 1) * k_blocks / C;
+    const int n_rows = PAIR ? n_pad / 2 : n_pad;  // W_gate rows this CTA loads per stage
 
     for (int e = tid; e < E; e += NTHREADS) {
         ctl->bias[e] = bias[e];
@@ -89,19 +118,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(&ctl->tmem_base, tmem_cols);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(&ctl->tmem_base, tmem_cols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&ctl->tmem_base, tmem_cols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR)
+        cluster_sync_all();  // the leader's barriers are initialised before the peer's loads count on them
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
-    const uint32_t stage_tx = (uint32_t)(A_BYTES + n_pad * BK * 2);
+    // bytes landing on a stage's full barrier: both CTAs' parts for a pair
+    const uint32_t stage_tx = (uint32_t)(PAIR ? 2 : 1) * (uint32_t)(A_BYTES + n_rows * BK * 2);
 
-    if (warp == 0) {
+    if (warp == 0 || warp == kWarpB) {
+        // token boxes (warp 0, which also arms the stage barrier) or W_gate boxes
+        const bool tok = warp == 0;
         if (elect_one()) {
-            tma_prefetch_desc(&tmX);
-            tma_prefetch_desc(&tmW);
+            tma_prefetch_desc(tok ? &tmX : &tmW);
+            const uint32_t leader_full = PAIR ? mapa_shared(smem_u32(&ctl->full[0]), leader) : 0u;
             int stage = 0;
             uint32_t phase = 0, issued = 0, iss_phase = 0;
             bool ok = true;
@@ -110,10 +150,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     ok = false;
                     break;
                 }
-                uint64_t* fb = &ctl->full[stage];
-                mbar_arrive_expect_tx(fb, stage_tx);
-                tma_load_2d(sA + stage * A_BYTES, &tmX, fb, kb * BK, t0, kEvictFirst);
-                tma_load_2d(sB + stage * B_STRIDE, &tmW, fb, kb * BK, 0, kEvictLast);
+                if (PAIR) {
+                    if (tok && half == 0) mbar_arrive_expect_tx(&ctl->full[stage], stage_tx);
+                    const uint32_t fb = leader_full + 8u * (uint32_t)stage;
+                    if (tok)
+                        tma_load_2d_pair(sA + stage * A_BYTES, &tmX, fb, kb * BK, t0, kEvictFirst);
+                    else
+                        tma_load_2d_pair(sB + stage * BSTR, &tmW, fb, kb * BK, half * n_rows, kEvictLast);
+                } else {
+                    uint64_t* fb = &ctl->full[stage];
+                    if (tok) {
+                        mbar_arrive_expect_tx(fb, stage_tx);
+                        tma_load_2d(sA + stage * A_BYTES, &tmX, fb, kb * BK, t0, kEvictFirst);
+                    } else {
+                        tma_load_2d(sB + stage * BSTR, &tmW, fb, kb * BK, 0, kEvictLast);
+                    }
+                }
                 issued |= 1u << stage;
                 iss_phase = (iss_phase & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) {
@@ -122,14 +174,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             }
             if (!ok) {
-                for (int s = 0; s < STAGES; ++s)
-                    if ((issued >> s) & 1u) mbar_wait_drain(&ctl->full[s], (iss_phase >> s) & 1u);
+                if (PAIR) {
+                    settle_inflight_loads();
+                } else {
+                    for (int s = 0; s < STAGES; ++s)
+                        if ((issued >> s) & 1u) mbar_wait_drain(&ctl->full[s], (iss_phase >> s) & 1u);
+                }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (elect_one()) {
-            const uint32_t idesc = idesc_bf16_f32(BM, n_pad);
+        if ((!PAIR || half == 0) && elect_one()) {
+            const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * BM : BM, n_pad);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -140,26 +196,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 tc_fence_after();
                 const uint64_t ad = smem_desc_sw128(smem_u32(sA + stage * A_BYTES));
-                const uint64_t bd = smem_desc_sw128(smem_u32(sB + stage * B_STRIDE));
+                const uint64_t bd = smem_desc_sw128(smem_u32(sB + stage * BSTR));
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    tc_mma_bf16(tmem_base, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
-                                (kb > kb0 || kk > 0) ? 1u : 0u);
-                tc_commit(&ctl->empty[stage]);
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
+                    if (PAIR)
+                        tc_mma_bf16_pair(tmem_base, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, acc);
+                    else
+                        tc_mma_bf16(tmem_base, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, acc);
+                }
+                if (PAIR)
+                    tc_commit_pair(&ctl->empty[stage], pair_mask);
+                else
+                    tc_commit(&ctl->empty[stage]);
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
                 }
             }
             if (ok) {
-                tc_commit(&ctl->tfull);
+                if (PAIR)
+                    tc_commit_pair(&ctl->tfull, pair_mask);
+                else
+                    tc_commit(&ctl->tfull);
             } else {
-                tc_commit(&ctl->drain);
+                if (PAIR)
+                    tc_commit_pair(&ctl->drain, (uint16_t)(1u << leader));
+                else
+                    tc_commit(&ctl->drain);
                 mbar_wait_drain(&ctl->drain, 0);
             }
         }
         __syncwarp();
-    } else if (C == 1) {
+    } else if (C == 1 && warp >= 2 && warp < 6) {
         // whole K in this CTA: thread r owns token r and streams its scores
         // from TMEM straight into the top-k
         const int q = warp & 3;
@@ -186,14 +255,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (t < T) emit_route<KMAX>(tk, k, idx + (size_t)t * k, w + (size_t)t * k, ctl->hist, status);
         }
-    } else {
-        // partial scores of this K slice: TMEM lane r (token r) -> part[r][0..n_pad)
+    }
+    if (C > 1) {
+        // partial scores of this K slice: TMEM lane r (token r) -> part[r][0..n_pad);
+        // warp w reads lane quarter w % 4, columns of half w / 4
         const int q = warp & 3;
         const int r = q * 32 + lane;
+        const int c_mid = (n_pad >> 5) << 4;  // a multiple of 16
+        const int c_lo = warp < 4 ? 0 : c_mid, c_hi = warp < 4 ? c_mid : n_pad;
         if (mbar_wait(&ctl->tfull, 0, &ctl->abort, status)) {
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
-            for (int c = 0; c < n_pad; c += 16) {
+            for (int c = c_lo; c < c_hi; c += 16) {
                 uint32_t v[16];
                 tmem_ld16(taddr + (uint32_t)c, v);
                 tmem_ld_wait();
@@ -209,26 +282,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     if (C > 1) cluster_sync_all();  // every CTA's partial scores are complete and visible
 
-    if (C > 1 && warp >= 2) {
-        const int u = tid - 64;             // 0..127
+    if (C > 1) {
+        const int u = tid;                  // all threads of the CTA
         constexpr int TPC = BM / C;         // tokens this CTA finishes
-        const int tl0 = crank * TPC;        // its first token within the tile
+        constexpr int P = NTHREADS / TPC;   // threads per token
+        static_assert(P <= 32 && (P & (P - 1)) == 0, "a token's threads are a power-of-two group of one warp");
+        const int tl0 = slice * TPC;        // its first token within the CTA's 128
         // scores s = sigmoid(sum of the C partials in CTA order), for this CTA's
-        // tokens: 128 / TPC threads per token row, four experts per DSMEM load
+        // tokens: P threads per token row, four experts per DSMEM load
         // (rows are 16-byte aligned; columns up to n_pad >= E hold MMA results)
         float* sc = red;
         {
-            constexpr int TPR = 128 / TPC;
+            constexpr int TPR = P;
             const int rl = u / TPR, q4 = u - rl * TPR;
             const int r = tl0 + rl;
             const bool keep_aff = aff && t0 + r < T;
 #pragma unroll 4
             for (int e = 4 * q4; e < E; e += 4 * TPR) {
                 const uint32_t a = smem_u32(part + r * PS + e);
-                float4 z = ld_cluster_f32x4(mapa_shared(a, 0));
+                float4 z = ld_cluster_f32x4(mapa_shared(a, (uint32_t)half));
 #pragma unroll
                 for (int c = 1; c < C; ++c) {
-                    const float4 o = ld_cluster_f32x4(mapa_shared(a, c));
+                    const float4 o = ld_cluster_f32x4(mapa_shared(a, (uint32_t)(PAIR ? 2 * c + half : c)));
                     z.x = __fadd_rn(z.x, o.x);
                     z.y = __fadd_rn(z.y, o.y);
                     z.z = __fadd_rn(z.z, o.z);
@@ -245,17 +320,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             }
         }
-        named_bar_sync(1, 128);
-        // top-k: C threads per token, thread `sub` pushes experts sub, sub + C, ...
-        const int rl = u / C, sub = u - rl * C;
+        __syncthreads();
+        // top-k: P threads per token, thread `sub` pushes experts sub, sub + P, ...
+        const int rl = u / P, sub = u - rl * P;
         const int t = t0 + tl0 + rl;
         TopK<KMAX> tk;
         tk.init();
-        for (int e = sub; e < E; e += C) {
+        for (int e = sub; e < E; e += P) {
             const float s = sc[rl * PS + e];
             tk.push(__fadd_rn(s, ctl->bias[e]), s, e);
         }
-        {  // merge the C lists in (v desc, index asc) order
+        {  // merge the P lists in (v desc, index asc) order
             TopK<KMAX> m;
             m.init();
             int pos = 0;
@@ -273,7 +348,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 float bv = hv, bs = hs;
                 int bid = hid;
 #pragma unroll
-                for (int o = C / 2; o > 0; o >>= 1) {
+                for (int o = P / 2; o > 0; o >>= 1) {
                     const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
                     const float os = __shfl_xor_sync(0xffffffffu, bs, o);
                     const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
@@ -297,28 +372,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     for (int e = tid; e < E; e += NTHREADS)
         if (ctl->hist[e]) atomicAdd(&counts[e], ctl->hist[e]);
-    if (C > 1) cluster_sync_all();  // no CTA leaves while its partial scores may still be read
+    // no CTA leaves while its partial scores may still be read, or while its
+    // pair leader's MMAs may still read its shared memory
+    if (CL > 1) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, tmem_cols);
+        if (PAIR)
+            tmem_dealloc_pair(tmem_base, tmem_cols);
+        else
+            tmem_dealloc(tmem_base, tmem_cols);
     }
 }
 
-template <int KMAX, int C>
+template <int KMAX, int C, bool PAIR>
 cudaError_t launch_kc(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int E, int n_pad,
                       uint32_t cols, int kb, int k, int32_t* idx, float* w, int32_t* counts, float* aff, int* status,
                       cudaStream_t st) {
-    auto kern = router_tc_kernel<KMAX, C>;
+    auto kern = router_tc_kernel<KMAX, C, PAIR>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
+    constexpr int CL = PAIR ? 2 * C : C;
+    const int tile = PAIR ? 2 * BM : BM;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(((T + BM - 1) / BM) * C));
+    cfg.gridDim = dim3((unsigned)(((T + tile - 1) / tile) * CL));
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.x = CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -328,15 +410,20 @@ cudaError_t launch_kc(const CUtensorMap& tx, const CUtensorMap& tw, const float*
     return err == cudaSuccess ? cudaGetLastError() : err;
 }
 
-template <int KMAX>
+template <int KMAX, bool PAIR>
 cudaError_t launch_k(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int E, int n_pad,
                      uint32_t cols, int kb, int k, int32_t* idx, float* w, int32_t* counts, float* aff, int* status,
                      int split, cudaStream_t st) {
     switch (split) {
-        case 8: return launch_kc<KMAX, 8>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
-        case 4: return launch_kc<KMAX, 4>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
-        case 2: return launch_kc<KMAX, 2>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
-        default: return launch_kc<KMAX, 1>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
+        case 8:
+            if (!PAIR)  // a pair cluster of 16 CTAs is not portable
+                return launch_kc<KMAX, 8, false>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status,
+                                                 st);
+            return cudaErrorInvalidValue;
+        case 4: return launch_kc<KMAX, 4, PAIR>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
+        case 2: return launch_kc<KMAX, 2, PAIR>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
+        default:
+            return launch_kc<KMAX, 1, PAIR>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, st);
     }
 }
 
@@ -347,18 +434,26 @@ cudaError_t launch_router_tc(const void* x, const void* wg, const float* bias, i
                              cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     if (d % BK != 0 || E > kMaxExperts || E <= 0) return cudaErrorInvalidValue;
-    const int n_pad = (E + 15) / 16 * 16;  // MMA N: multiple of 16 for M = 128
+    const int n_pad = (E + 15) / 16 * 16;  // MMA N: a multiple of 16 (N/2 rows per CTA of a pair: 8-row atoms)
     uint32_t cols = 32;
     while (cols < (uint32_t)n_pad) cols <<= 1;  // TMEM allocation: power of two >= 32
+    // Large batches: CTA pairs of 256 tokens (half the W_gate rows per CTA);
+    // the one-CTA form only while its K split would still reach 4 or more.
+    const int tiles1 = (T + BM - 1) / BM, kb = d / BK;
+    const bool pair = T > 2 * BM && tiles1 * 4 > num_sms;
     CUtensorMap tx, tw;
-    if (!make_tmap_2d(&tx, x, d, T, d, BK, BM) || !make_tmap_2d(&tw, wg, d, E, d, BK, n_pad))
+    if (!make_tmap_2d(&tx, x, d, T, d, BK, BM) || !make_tmap_2d(&tw, wg, d, E, d, BK, pair ? n_pad / 2 : n_pad))
         return cudaErrorInvalidValue;
     // K split: as many CTAs per token tile as keep the grid within one wave of SMs
-    const int tiles = (T + BM - 1) / BM, kb = d / BK;
-    int split = 8;
-    while (split > 1 && (tiles * split > num_sms || split > kb)) split >>= 1;
-    return k <= 8 ? launch_k<8>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, split, st)
-                  : launch_k<16>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, split, st);
+    const int tiles = pair ? (T + 2 * BM - 1) / (2 * BM) : tiles1, per = pair ? 2 : 1;
+    int split = pair ? 4 : 8;  // clusters of at most 8 CTAs
+    while (split > 1 && (tiles * split * per > num_sms || split > kb)) split >>= 1;
+    if (pair)
+        return k <= 8 ? launch_k<8, true>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, split, st)
+                      : launch_k<16, true>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, split,
+                                           st);
+    return k <= 8 ? launch_k<8, false>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, split, st)
+                  : launch_k<16, false>(tx, tw, bias, T, E, n_pad, cols, kb, k, idx, w, counts, aff, status, split, st);
 }
 
 }  // namespace moe

@@ -48,4 +48,21 @@ inline bool make_tmap_2d(CUtensorMap* m, const void* base, unsigned long long co
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// rank-3 fp32 map for tiled stores: [planes][rows][cols] with row pitch
+// `ld` and plane pitch `plane` elements; box = box_cols (innermost, 32
+// floats = 128 bytes, 128-byte swizzle) x box_rows x 1.
+inline bool make_tmap_3d_f32(CUtensorMap* m, void* base, unsigned long long cols, unsigned long long rows,
+                             unsigned long long planes, unsigned long long ld, unsigned long long plane,
+                             unsigned box_cols, unsigned box_rows) {
+    auto enc = tmap_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {cols, rows, planes};
+    cuuint64_t strides[2] = {ld * 4, plane * 4};
+    cuuint32_t box[3] = {box_cols, box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace moe

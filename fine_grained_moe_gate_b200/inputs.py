@@ -13,7 +13,8 @@ from the stated distributions):
                x~N(0,1), W~N(0,0.006), bias~U(-0.01,0.01)
   v3_decode    T=64 per call, V3 shape and distributions, fresh x per call
   *_fp8        small_fp8, v3_prefill_fp8, v3_decode_fp8: the same tensors,
-               expert GEMMs in E4M3 (weights quantized per output row)
+               expert GEMMs in E4M3 (weights, tokens and h quantized in
+               1x32 tiles along the contraction, power-of-two scales)
   skew_stress  T=32768, V3 shape; x[:,0]=1 and W_g[i][0]=o_i, a per-expert
                logit offset that ranks expert popularity by a seeded
                permutation with Zipf exponent 1.2 (see ``zipf_offsets``);

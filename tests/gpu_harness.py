@@ -39,7 +39,7 @@ def route(sh, x, wg, bias, with_aff=True):
     return idx, w, counts, aff
 
 
-def affinity_tolerance(s_orc: np.ndarray, K: int, tensor_cores: bool) -> np.ndarray:
+def affinity_tolerance(s_orc: np.ndarray, K: int, tensor_cores: bool, cap: bool = True) -> np.ndarray:
     """Per-element bound on |s_kernel - s_oracle| from the arithmetic.
 
     The kernel accumulates z = x . W_g in fp32; the oracle in double (exact
@@ -50,7 +50,16 @@ def affinity_tolerance(s_orc: np.ndarray, K: int, tensor_cores: bool) -> np.ndar
                         fp32 accumulator, each may lose up to one ulp:
                         |dz| <= (K / 16) * 2^-23 * (|z| + 1)
     (|z| + 1 bounds the partial sums for these inputs).  The sigmoid scales
-    dz by s (1 - s); rounding s to fp32 adds 2^-24."""
+    dz by s (1 - s); rounding s to fp32 adds 2^-24.
+
+    With ``cap`` the bar is the smaller of that bound and a fixed one: 1e-6
+    for fp32 inputs, 4e-6 for bf16 inputs with fp32 accumulation, which is
+    what the worst-case bound gives at K ~ 1000 and |z| ~ 1; at V3's K = 7168
+    with V3's weight scale the fixed bar is the tighter one (the worst case
+    assumes every block's rounding error has the same sign).  Inputs built
+    to give large logits (the skewed workload's per-expert offsets) carry
+    proportionally larger partial sums, so their check uses the derived
+    bound alone (cap=False)."""
     s = s_orc.astype(np.float64)
     z = np.log(s / (1.0 - s))
     dsig = s * (1.0 - s)
@@ -58,14 +67,16 @@ def affinity_tolerance(s_orc: np.ndarray, K: int, tensor_cores: bool) -> np.ndar
         dz = (K / 16.0) * 2.0 ** -23 * (np.abs(z) + 1.0)
     else:
         dz = K * 2.0 ** -24 * (np.abs(z) + 1.0)
-    return dsig * dz + 2.0 ** -24
+    bound = dsig * dz + 2.0 ** -24
+    return np.minimum(bound, 4e-6 if tensor_cores else 1e-6) if cap else bound
 
 
 def check_route_parity(x, wg, bias, k, idx, w, counts, aff, s_tol, self_rows=None):
     """Injected mode: the oracle's selection on the kernel's fp32 affinities
     must match idx, w and counts bit for bit.  Self mode: the oracle's own
     affinities on ``self_rows`` within s_tol ("auto": the bound
-    ``affinity_tolerance`` derives for the input dtype)."""
+    ``affinity_tolerance`` gives for the input dtype; "derived": the same
+    without its fixed cap)."""
     aff_np = aff.cpu().numpy()
     b_np = bias.cpu().numpy()
     o_idx, o_w = oracle.select(aff_np, b_np, k)
@@ -77,8 +88,8 @@ def check_route_parity(x, wg, bias, k, idx, w, counts, aff, s_tol, self_rows=Non
     rows = np.arange(aff_np.shape[0]) if self_rows is None else np.asarray(self_rows)
     s_orc = oracle.affinity(to_numpy(x[torch.as_tensor(rows, device=x.device)]), to_numpy(wg))
     diff = np.abs(s_orc.astype(np.float64) - aff_np[rows].astype(np.float64))
-    if s_tol == "auto":
-        tol = affinity_tolerance(s_orc, x.shape[1], x.dtype == torch.bfloat16)
+    if s_tol in ("auto", "derived"):
+        tol = affinity_tolerance(s_orc, x.shape[1], x.dtype == torch.bfloat16, cap=s_tol == "auto")
     else:
         tol = np.full(diff.shape, float(s_tol))
     worst = np.unravel_index(np.argmax(diff / tol), diff.shape)

@@ -183,7 +183,8 @@ def test_skew_stress_routing_and_sampled_output():
     for step in range(5):
         x = make_tokens(cfg, DEV, step)
         if step == 0:
-            y, idx, w, counts = _full_check(cfg, p, x, n_sample=64, seed=4, projections=True)
+            # logits carry the per-expert offsets: the derived affinity bound, uncapped
+            y, idx, w, counts = _full_check(cfg, p, x, n_sample=64, seed=4, s_tol="derived", projections=True)
             c = counts.cpu().numpy()
             assert c.max() > 8 * c.mean()    # the workload really is skewed
         else:

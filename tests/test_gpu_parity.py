@@ -52,6 +52,11 @@ ROUTER_BF16 = [
     dict(T=130, d=64, E=8, k=8),          # k = E
     dict(T=64, d=256, E=32, k=12),        # k > 8 (16-wide top-k registers)
     dict(T=1, d=64, E=16, k=2),
+    # CTA-pair tiles of 256 tokens (large batches)
+    dict(T=4964, d=256, E=72, k=6),       # last pair's second CTA entirely past T; N/2 = 40 rows per CTA
+    dict(T=8192, d=1024, E=256, k=8),     # V3 routing width, K split over 2 pairs
+    dict(T=6000, d=192, E=24, k=4),       # uneven K slices (3 blocks over 2 pairs), N = 32
+    dict(T=20000, d=128, E=256, k=12),    # k > 8, no K split, more pairs than one wave
 ]
 
 
@@ -63,7 +68,8 @@ def test_route_bf16_tensor_cores(c):
     x = make_tokens(cfg, DEV)
     idx, w, counts, aff = route(sh, x, p["w_gate"], p["bias"])
     check_status()
-    rows = np.arange(min(c["T"], 256))
+    # the first tile and the ragged last ones
+    rows = np.unique(np.concatenate([np.arange(min(c["T"], 256)), np.arange(max(c["T"] - 300, 0), c["T"])]))
     check_route_parity(x, p["w_gate"], p["bias"], sh.k, idx, w, counts, aff, "auto", self_rows=rows)
 
 
