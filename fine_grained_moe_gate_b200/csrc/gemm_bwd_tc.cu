@@ -43,7 +43,7 @@ namespace moe {
 namespace {
 
 constexpr int BK = 64;
-constexpr int STAGES = 6;
+constexpr int MAX_STAGES = 6;
 constexpr int A_BYTES = 128 * BK * 2;
 constexpr int B_BYTES = 128 * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -51,15 +51,29 @@ constexpr int NT = 256;
 constexpr int NXBOX = 8;  // token boxes of 16, 32, ..., 128 rows (K-major B)
 constexpr uint32_t ACC_COLS = 256;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int NEPI = 4;
-constexpr int NTHREADS = 32 * (2 + NEPI + 1);
+// The weight-gradient kind has short K loops (a group's rows) and 128 KB of
+// fp32 results per CTA and tile: it runs eight epilogue warps (each quarter
+// of TMEM lanes read by two, one per column half) and four stages; the rows
+// kind four epilogue warps and six stages.
+template <bool WG>
+__host__ __device__ constexpr int n_epi() {
+    return WG ? 8 : 4;
+}
+template <bool WG>
+__host__ __device__ constexpr int n_stages() {
+    return WG ? 4 : 6;
+}
+template <bool WG>
+__host__ __device__ constexpr int n_threads() {
+    return 32 * (3 + n_epi<WG>());
+}
 constexpr int XS = 132;
 constexpr int XBUF_BYTES = 16 * XS * 4;
 constexpr int kMaxBwdGroups = kMaxGroups + 1;
 
 struct Ctl {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[MAX_STAGES];
+    uint64_t empty[MAX_STAGES];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -72,9 +86,17 @@ struct Tables {
     int ttiles[kMaxBwdGroups];  // rows: token tiles; wgrad: 1
     int prefix[kMaxBwdGroups + 1];
 };
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 2 * (size_t)XBUF_BYTES + sizeof(Ctl) +
-                              sizeof(Tables);
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// epilogue staging: rows, two exchange buffers; wgrad, two 4 KB output boxes per epilogue warp
+template <bool WG>
+__host__ __device__ constexpr size_t xbuf_bytes() {
+    return WG ? (size_t)n_epi<WG>() * 2 * 4096 : 2 * (size_t)XBUF_BYTES;
+}
+template <bool WG>
+__host__ __device__ constexpr size_t smem_bytes() {
+    return 1024 + (size_t)n_stages<WG>() * STAGE_BYTES + xbuf_bytes<WG>() + sizeof(Ctl) + sizeof(Tables);
+}
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory budget");
+static_assert(n_stages<false>() <= MAX_STAGES && n_stages<true>() <= MAX_STAGES, "ring depth");
 
 struct Maps {
     CUtensorMap a0, a1;   // A: the weights (rows) or the per-row matrix (wgrad); a1: dx's W3
@@ -211,13 +233,16 @@ __device__ __forceinline__ TileInfo tile_info(const Tables* tb, const BwdParams&
 }
 
 template <bool AMN, bool BMN, bool WG>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<WG>(), 1)
     tc_bwd_gemm_kernel(const __grid_constant__ Maps mp, const BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = base;
+    constexpr int STAGES = n_stages<WG>();
+    constexpr int NEPI = n_epi<WG>();
+    constexpr int NTHREADS = n_threads<WG>();
     float* xbuf = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
-    Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + 2 * XBUF_BYTES);
+    Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + xbuf_bytes<WG>());
     Tables* tb = reinterpret_cast<Tables*>(ctl + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
@@ -422,7 +447,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------ epilogue (both CTAs, warps 2..5)
+        // ------------------------------------------------ epilogue (both CTAs, warps 2 .. 1 + NEPI)
         const int q = warp & 3;  // TMEM lane quarter
         const int e = tid - 64;  // 0..127
         const int my_tok = e >> 3, part = e & 7;
@@ -437,17 +462,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * ACC_COLS;
             const int mcta = ti.m0 + (int)rank * 128;  // this CTA's first M row
             if (WG) {
-                // D[m][n]: lane = m, column = n.  Per 32 columns the warp's 32 x 32 block goes through its
-                // 4 KB of shared memory (128-byte swizzled rows: 16-byte chunk j of row r at j ^ (r % 8))
-                // and leaves as one TMA store, whole 128-byte lines; rows past M_total are clipped by the
-                // map.  The TMEM read of the next 32 columns is in flight meanwhile.
-                float* sb = xbuf + (warp - 2) * 1024;
-                float4* srow = reinterpret_cast<float4*>(sb + lane * 32);
+                // D[m][n]: lane = m, column = n; warp w reads lane quarter w % 4, column half (w - 2) / 4.
+                // Per 32 columns the warp's 32 x 32 block goes through one of its two 4 KB shared-memory
+                // boxes (128-byte swizzled rows: 16-byte chunk j of row r at j ^ (r % 8)) and leaves as one
+                // TMA store, whole 128-byte lines; rows past M_total are clipped by the map.  The TMEM
+                // read of the next 32 columns and the store of the previous box run meanwhile.
+                const int ew = warp - 2;
+                const int c_lo = (ew >> 2) * 128, c_hi = min(c_lo + 128, ti.ntok);
                 const int mq = mcta + q * 32;
                 uint32_t r0[32], r1[32];
                 const auto store32 = [&](int c, const uint32_t (&v)[32]) {
-                    if (lane == 0) bulk_wait_group_read<0>();  // the previous box has left shared memory
+                    float* sb = xbuf + ew * 2048 + xb * 1024;
+                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used this box has read it
                     __syncwarp();
+                    float4* srow = reinterpret_cast<float4*>(sb + lane * 32);
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         srow[i ^ (lane & 7)] =
@@ -460,10 +488,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                         tma_store_3d(&mp.o, sb, ti.n0 + c, mq, t.g);
                         bulk_commit_group();
                     }
+                    xb ^= 1;
                 };
-                const bool live = mq < p.M_total;  // warp-uniform: a block wholly past M_total is not stored
-                if (live && ti.kb > 0) tmem_ld32(taddr, r0);
-                for (int c = 0; live && c < ti.ntok; c += 64) {  // ntok is a multiple of 128
+                const bool live = mq < p.M_total && c_lo < c_hi;  // warp-uniform: nothing of this warp's to store
+                if (live && ti.kb > 0) tmem_ld32(taddr + (uint32_t)c_lo, r0);
+                for (int c = c_lo; live && c < c_hi; c += 64) {  // the tile's columns come in multiples of 128
                     if (ti.kb > 0) {
                         tmem_ld_wait();
                         tmem_ld32(taddr + (uint32_t)(c + 32), r1);
@@ -471,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                     store32(c, r0);
                     if (ti.kb > 0) {
                         tmem_ld_wait();
-                        if (c + 64 < ti.ntok) tmem_ld32(taddr + (uint32_t)(c + 64), r0);
+                        if (c + 64 < c_hi) tmem_ld32(taddr + (uint32_t)(c + 64), r0);
                     }
                     store32(c + 32, r1);
                 }
@@ -527,10 +556,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 template <bool AMN, bool BMN, bool WG>
 cudaError_t launch_bwd(const Maps& m, const BwdParams& p, int num_sms, cudaStream_t st) {
     auto kern = tc_bwd_gemm_kernel<AMN, BMN, WG>;
+    constexpr size_t SMEM_BYTES = smem_bytes<WG>();
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     const int grid = (num_sms / 2) * 2;
-    kern<<<grid, NTHREADS, SMEM_BYTES, st>>>(m, p);
+    kern<<<grid, n_threads<WG>(), SMEM_BYTES, st>>>(m, p);
     note_launches(1);
     return cudaGetLastError();
 }

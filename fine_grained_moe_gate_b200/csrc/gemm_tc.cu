@@ -963,8 +963,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                     }
                 } else {
                     const int fj = part * 16;
-                    if (tok_ok && fcta + fj < sp.f_limit) {
-                        float f[16];
+                    const bool st_ok = tok_ok && fcta + fj < sp.f_limit;
+                    float f[16];
+                    if (st_ok) {
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const float4 t = *reinterpret_cast<const float4*>(row + fj + 4 * i);
@@ -973,6 +974,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                             f[4 * i + 2] = t.z;
                             f[4 * i + 3] = t.w;
                         }
+                    }
+                    if (NXB == 1) named_bar_sync(1 + eg, 128);  // the single buffer is free for the next chunk
+                    if (st_ok) {
                         const int orow = tok0 + c + my_tok;
                         if (sp.acc) {  // fused weighted combine
                             int t = orow;
