@@ -852,13 +852,14 @@ def run_backward(args, world, rank, local):
     if st != 0:
         raise SystemExit(f"device status {moe.STATUS.get(st, st)}")
     ms = a.elapsed_time(b) / steps
-    # FLOPs (2 per multiply-add): per routed row the recomputed a, g and o (6 d I), dh (2 d I), dx_perm
-    # (4 d I) and dW1, dW3, dW2 (6 d I) = 18 d I; per token the shared experts 16 d S Is (no o) and the
-    # router's dx and dW_g 4 d E
-    flop = T * k * 18 * d * I + T * 16 * d * S * Is + T * 4 * d * E
-    tflops = flop / (ms * 1e-3) / 1e12
     # bf16 layers whose widths are multiples of 128 run the expert contractions on the tensor cores
     tc = cfg.dtype == "bf16" and d % 128 == 0 and I % 128 == 0 and (S == 0 or Is % 128 == 0)
+    # FLOPs (2 per multiply-add): per routed row the recomputed a and g (4 d I), dh (2 d I), dx_perm
+    # (4 d I) and dW1, dW3, dW2 (6 d I) = 16 d I, plus the recomputed o (2 d I) on the SIMT path (the
+    # tensor-core path takes the combine weights' gradient from dh instead); per token the shared
+    # experts 16 d S Is and the router's dx and dW_g 4 d E
+    flop = T * k * (16 if tc else 18) * d * I + T * 16 * d * S * Is + T * 4 * d * E
+    tflops = flop / (ms * 1e-3) / 1e12
     if tc:
         peaks, peak_src = load_peaks()
         burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))

@@ -25,12 +25,17 @@
 //   (dw_tj - sum_j' dw_tj' w_tj') / sum_j' s_{t,idx_j'} (+ the balance term),
 //   dz = ds s (1 - s),  dx += dz W_g,  dW_g = dz^T x.
 //
-// Every contraction runs through two fp32 SIMT kernels over strided operand
-// views (no transposed copies): a "rows" GEMM (C[r][n] = sum_k A(r,k) B_g(n,k)
-// for the rows r of group g) and a weight-gradient GEMM whose contraction runs
-// over a group's rows (C_g[m][n] = sum_r A(r,m) B(r,n)).  Groups and tiles are
-// resolved on the device from the routing offsets.  fp32 FFMA throughout:
-// the backward is a first, exact-in-fp32 path, not yet on the tensor cores.
+// Two paths compute these.  bf16 layers whose widths are multiples of 128 run
+// every contraction on the tensor cores (gemm_bwd_tc.cu: bf16 operands, fp32
+// accumulation) over a padded row layout (each expert's rows padded to a
+// multiple of 64 with zero rows); there the routed dw comes without
+// recomputing o: with u_r = W2_e^T dy_t (the dh GEMM run on the unweighted
+// dy), dw_tj = <dy_t, W2_e h_r> = <u_r, h_r> and dh_r = w_tj u_r.  Every
+// other layer runs two fp32 SIMT kernels over strided operand views (no
+// transposed copies): a "rows" GEMM (C[r][n] = sum_k A(r,k) B_g(n,k) for the
+// rows r of group g) and a weight-gradient GEMM whose contraction runs over a
+// group's rows (C_g[m][n] = sum_r A(r,m) B(r,n)); groups and tiles are
+// resolved on the device from the routing offsets.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -556,14 +561,13 @@ __global__ void swiglu_h_kernel(const float* __restrict__ a, const float* __rest
 }
 
 // One warp per assignment q = t*k + j (row r = inv[q], padded row pr):
-// dw[q] = <dy_t, o[pr]>, do[pr] = bf16(w[q] dy_t).  d % 4 == 0: 16-byte
-// loads, 8-byte stores.
-__global__ void __launch_bounds__(256) combine_bwd_pad_kernel(const float* __restrict__ dy, const float* __restrict__ w,
-                                                              const int32_t* __restrict__ inv,
-                                                              const int32_t* __restrict__ prow,
-                                                              const float* __restrict__ o, float* __restrict__ dw,
-                                                              uint16_t* __restrict__ dop, int d, int k, int rows,
-                                                              int nq, int* status) {
+// dy_pad[pr] = bf16(dy_t), do_pad[pr] = bf16(w[q] dy_t).  d % 4 == 0:
+// 16-byte loads, 8-byte stores.
+__global__ void __launch_bounds__(256) spread_dy_pad_kernel(const float* __restrict__ dy, const float* __restrict__ w,
+                                                            const int32_t* __restrict__ inv,
+                                                            const int32_t* __restrict__ prow,
+                                                            uint16_t* __restrict__ dyp, uint16_t* __restrict__ dop,
+                                                            int d, int k, int rows, int nq, int* status) {
     const int lane = threadIdx.x & 31;
     const int q = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (q >= nq) return;  // warp-uniform
@@ -575,20 +579,62 @@ __global__ void __launch_bounds__(256) combine_bwd_pad_kernel(const float* __res
     }
     const long long pr = prow[r];
     const float4* dyt = reinterpret_cast<const float4*>(dy + (long long)t * d);
-    const float4* orow = reinterpret_cast<const float4*>(o + pr * d);
-    uint2* dst = reinterpret_cast<uint2*>(dop + pr * d);
+    uint2* dst_y = reinterpret_cast<uint2*>(dyp + pr * d);
+    uint2* dst_o = reinterpret_cast<uint2*>(dop + pr * d);
     const float wq = w[q];
     const int d4 = d / 4;
-    float part = 0.0f;
 #pragma unroll 4
     for (int c = lane; c < d4; c += 32) {
-        const float4 y = dyt[c], v = orow[c];
-        part = fmaf(y.x, v.x, fmaf(y.y, v.y, fmaf(y.z, v.z, fmaf(y.w, v.w, part))));
-        dst[c] = make_uint2(bf16x2(wq * y.x, wq * y.y), bf16x2(wq * y.z, wq * y.w));
+        const float4 y = dyt[c];
+        dst_y[c] = make_uint2(bf16x2(y.x, y.y), bf16x2(y.z, y.w));
+        dst_o[c] = make_uint2(bf16x2(wq * y.x, wq * y.y), bf16x2(wq * y.z, wq * y.w));
+    }
+}
+
+// Routed rows, one warp per row r (padded row pr = prow[r], assignment
+// q = perm[r]), from u = dy_t W2_e (fp32, the unweighted upstream gradient
+// of h): dh = w[q] u, the SwiGLU derivative as below into dadg, and the
+// combine weight's gradient dw[q] = <dy_t, o> = <u, h> with h recomputed
+// exactly as the forward rounds it (bf16(silu(a) g)).  n % 4 == 0.
+__global__ void __launch_bounds__(256) swiglu_bwd_dw_pad_kernel(const float* __restrict__ a,
+                                                                const float* __restrict__ g,
+                                                                const float* __restrict__ u,
+                                                                const int32_t* __restrict__ prow,
+                                                                const int32_t* __restrict__ perm,
+                                                                const float* __restrict__ w, int R, int n,
+                                                                uint16_t* __restrict__ dadg, float* __restrict__ dw) {
+    const int lane = threadIdx.x & 31;
+    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= R) return;  // warp-uniform
+    const long long pr = prow[r];
+    const int q = perm[r];
+    const float wq = w[q];
+    const int n4 = n / 4;
+    const float4* ar = reinterpret_cast<const float4*>(a + pr * n);
+    const float4* gr = reinterpret_cast<const float4*>(g + pr * n);
+    const float4* ur = reinterpret_cast<const float4*>(u + pr * n);
+    uint2* row = reinterpret_cast<uint2*>(dadg + pr * 2 * n);
+    float dot = 0.0f;
+    for (int c = lane; c < n4; c += 32) {
+        const float4 av = ar[c], gv = gr[c], uv = ur[c];
+        const float al[4] = {av.x, av.y, av.z, av.w}, gl[4] = {gv.x, gv.y, gv.z, gv.w},
+                    ul[4] = {uv.x, uv.y, uv.z, uv.w};
+        float da[4], dg[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const float s = sigmoid_acc(al[v]);
+            const float h = __bfloat162float(__float2bfloat16_rn(al[v] * s * gl[v]));
+            dot = fmaf(ul[v], h, dot);
+            const float dh = wq * ul[v];
+            da[v] = dh * gl[v] * s * (1.0f + al[v] * (1.0f - s));
+            dg[v] = dh * al[v] * s;
+        }
+        row[c] = make_uint2(bf16x2(da[0], da[1]), bf16x2(da[2], da[3]));
+        row[n4 + c] = make_uint2(bf16x2(dg[0], dg[1]), bf16x2(dg[2], dg[3]));
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-    if (lane == 0) dw[q] = part;
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    if (lane == 0) dw[q] = dot;
 }
 
 // SwiGLU derivative on the real rows: with s = sigmoid(a),
@@ -859,7 +905,7 @@ cudaError_t experts_backward_tc(const BackwardArgs& a, const BwdBufs& b, int* st
     };
 
     // ---- routed experts
-    // recompute a = x W1^T, g = x W3^T (fp32), h = bf16(silu(a) g) as the forward, o = h W2^T (fp32)
+    // recompute a = x W1^T, g = x W3^T (fp32), h = bf16(silu(a) g) as the forward
     TC_TRY(launch_bwd_rows_kmajor(rows_args(a.w1, (long long)E * I, I, b.x_pad, Rp, d, I, b.a_pad, true), status,
                                   num_sms, st));
     TC_TRY(launch_bwd_rows_kmajor(rows_args(a.w3, (long long)E * I, I, b.x_pad, Rp, d, I, b.g_pad, true), status,
@@ -869,24 +915,26 @@ cudaError_t experts_backward_tc(const BackwardArgs& a, const BwdBufs& b, int* st
                                                                        reinterpret_cast<uint2*>(b.h_pad));
         note_launches(1);
     }
-    TC_TRY(launch_bwd_rows_kmajor(rows_args(a.w2, (long long)E * d, d, b.h_pad, Rp, I, d, b.o_pad, true), status,
-                                  num_sms, st));
-    // dw = <dy, o> per assignment; do = w dy (bf16, padded rows)
+    // dy_t and do = w dy_t (bf16) on every assignment's padded row; dy_pad lives in the o_pad buffer,
+    // which dx_perm overwrites only after its last use.  Its padding rows are never cleared: a B row of
+    // the rows GEMM only reaches the output row of the same index, and padding rows are not stored.
+    uint16_t* dy_pad = reinterpret_cast<uint16_t*>(b.o_pad);
     if (R > 0) {
-        combine_bwd_pad_kernel<<<(R + 7) / 8, 256, 0, st>>>(a.dy, a.w, b.inv, b.prow, b.o_pad, b.dw, b.do_pad, d, k,
-                                                            R, R, status);
+        spread_dy_pad_kernel<<<(R + 7) / 8, 256, 0, st>>>(a.dy, a.w, b.inv, b.prow, dy_pad, b.do_pad, d, k, R, R,
+                                                          status);
         note_launches(1);
     }
     // dW2_e = do^T h
     TC_TRY(launch_bwd_wgrad(wgrad_args(b.do_pad, d, 0, b.h_pad, I, 0, Rp, d, I, a.dw2, true), status, num_sms, st));
-    // dh = do W2_e (W2 read along its output dimension)
+    // u = dy W2_e (W2 read along its output dimension); dh = w u.  The combine weight's gradient
+    // <dy_t, o> = <dy_t, W2_e h> = <u, h> comes with it, so o is never recomputed.
     {
-        BwdRowsArgs r = rows_args(a.w2, (long long)E * d, d, b.do_pad, Rp, d, I, b.dh_pad, true);
+        BwdRowsArgs r = rows_args(a.w2, (long long)E * d, d, dy_pad, Rp, d, I, b.dh_pad, true);
         TC_TRY(launch_bwd_rows_mnmajor(r, status, num_sms, st));
     }
     if (R > 0) {
-        swiglu_bwd_pad_kernel<<<ew_grid((long long)R * I / 4), 256, 0, st>>>(b.a_pad, b.g_pad, b.dh_pad, b.prow, R,
-                                                                             I, b.dadg);
+        swiglu_bwd_dw_pad_kernel<<<(R + 7) / 8, 256, 0, st>>>(b.a_pad, b.g_pad, b.dh_pad, b.prow, b.perm, a.w, R, I,
+                                                              b.dadg, b.dw);
         note_launches(1);
     }
     // dW1_e = da^T x, dW3_e = dg^T x
