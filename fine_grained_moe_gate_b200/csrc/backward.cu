@@ -1030,7 +1030,7 @@ cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sm
 
     // routing layout of the forward: offsets, perm_tok, inv_row (no row copy)
     BWD_TRY(launch_permute(nullptr, a.idx, a.counts, T, d, E, k, bf ? 2 : 4, nullptr, offsets, perm, inv, pscratch,
-                           status, num_sms, st));
+                           status, st));
 
     if (tc) {
         BWD_TRY(experts_backward_tc(a, bb, status, num_sms, st));

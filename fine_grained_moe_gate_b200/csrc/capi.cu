@@ -99,10 +99,9 @@ moe_status do_route(const void* x, const void* w_gate, const float* bias, const 
 }
 
 moe_status do_permute(const void* x, const int32_t* idx, const int32_t* counts, const moe_shape& sh, void* x_perm,
-                      int32_t* offsets, int32_t* perm, int32_t* inv, void* ws, int* status, int sms,
-                      cudaStream_t st) {
+                      int32_t* offsets, int32_t* perm, int32_t* inv, void* ws, int* status, cudaStream_t st) {
     cudaError_t err = moe::launch_permute(x, idx, counts, sh.T, sh.d, sh.E, sh.k, esize(sh), x_perm, offsets, perm,
-                                          inv, static_cast<int32_t*>(ws), status, sms, st);
+                                          inv, static_cast<int32_t*>(ws), status, st);
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -431,7 +430,7 @@ moe_status moe_permute(const void* x, const int32_t* topk_idx, const int32_t* co
     int* status;
     v = device_setup(&dev, &status, &sms);
     if (v != MOE_OK) return v;
-    return do_permute(x, topk_idx, counts, sh, x_perm, offsets, perm_tok, inv_row, workspace, status, sms,
+    return do_permute(x, topk_idx, counts, sh, x_perm, offsets, perm_tok, inv_row, workspace, status,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -708,8 +707,7 @@ moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bia
     void* y_perm = x_perm;  // the down projection overwrites x_perm once the up projection has read it
     if ((v = do_route(x, w_gate, bias, sh, topk_idx, topk_w, counts, nullptr, status, sms, st)) != MOE_OK) return v;
     if (sh.T == 0) return MOE_OK;
-    if ((v = do_permute(x, topk_idx, counts, sh, x_perm, offsets, perm, inv, pws, status, sms, st)) != MOE_OK)
-        return v;
+    if ((v = do_permute(x, topk_idx, counts, sh, x_perm, offsets, perm, inv, pws, status, st)) != MOE_OK) return v;
     if ((v = do_swiglu(x_perm, offsets, w1, w3, w2, sh.S > 0 ? x : nullptr, ws1, ws3, ws2, sh, y_perm, shared_out,
                        gws, status, sms, st)) != MOE_OK)
         return v;
@@ -808,8 +806,8 @@ moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float*
     if ((v = do_route(x, w_gate, bias, sh, topk_idx, topk_w, counts, nullptr, status, sms, st)) != MOE_OK) return v;
     if (sh.T == 0) return MOE_OK;
     if (moe::launch_quantize_mx(x, sh.T, sh.d, 1, false, k8.xq, k8.xs, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if ((v = do_permute(k8.xq, topk_idx, counts, sh, k8.xq_perm, k8.offsets, k8.perm, k8.inv, k8.pws, status, sms,
-                        st)) != MOE_OK)
+    if ((v = do_permute(k8.xq, topk_idx, counts, sh, k8.xq_perm, k8.offsets, k8.perm, k8.inv, k8.pws, status, st)) !=
+        MOE_OK)
         return v;
     if ((v = do_ffn_up_fp8(k8.xq_perm, k8.perm, k8.xs, k8.offsets, shared ? k8.xq : nullptr, w, sh, k8.h, k8.hs,
                            status, sms, st)) != MOE_OK)

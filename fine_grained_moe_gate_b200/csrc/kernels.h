@@ -65,7 +65,7 @@ cudaError_t launch_router_tc(const void* x, const void* wg, const float* bias, i
 size_t permute_scratch_bytes(int T, int E);
 cudaError_t launch_permute(const void* x, const int32_t* idx, const int32_t* counts, int T, int d, int E, int k,
                            size_t elem_bytes, void* x_perm, int32_t* offsets, int32_t* perm_tok, int32_t* inv_row,
-                           int32_t* scratch, int* status, int num_sms, cudaStream_t st);
+                           int32_t* scratch, int* status, cudaStream_t st);
 
 // backward.cu: the layer backward (fp32 SIMT contractions).  Pointers as in
 // moe_layer_backward; x and the weights bf16 when bf16, else fp32.

@@ -11,10 +11,8 @@
 //   3. rank:    per chunk, a bitmask of the chunk's tokens per expert; the
 //               rank of token t inside expert e is popcount of the bits
 //               below t; row = base[c][e] + rank                     (grid C)
-//   4. scatter: token t's row is read once and written to its k rows:
-//               bulk copies through shared memory, one thread per CTA
-//               issuing them (one wave of CTAs), or 16-byte vector stores
-//               when a row does not fit the bulk path          (grid T)
+//   4. scatter: token t's row is read once and written to its k rows with
+//               16-byte vector stores                                 (grid T)
 #include "common.cuh"
 #include "kernels.h"
 
@@ -165,61 +163,6 @@ __global__ void permute_scatter_kernel(const uint4* __restrict__ x, int vec_per_
     }
 }
 
-// Bulk form of the scatter: CTA b moves tokens b, b + G, ... (G CTAs).  Its
-// one issuing thread keeps up to NB - 1 row loads in flight (bulk copies into
-// NB shared-memory buffers, each with its own barrier) and, as each lands,
-// issues the row's k bulk stores to x_perm; a buffer is reloaded once the
-// stores of its previous row have read it.  Rows are whole 16-byte multiples
-// (row_bytes % 16 == 0) at 16-byte aligned addresses.  Waits are bounded: a
-// timeout reports it, waits for what was issued and returns.
-constexpr int kBulkBufs = 8;
-constexpr int kBulkSmem = 200 * 1024;
-
-__global__ void __launch_bounds__(32) permute_scatter_bulk_kernel(const uint8_t* __restrict__ x, int row_bytes,
-                                                                  int T, int k, const int32_t* __restrict__ inv_row,
-                                                                  int total_rows, uint8_t* __restrict__ xp, int nb,
-                                                                  int* status) {
-    extern __shared__ __align__(128) uint8_t sbuf[];
-    __shared__ uint64_t full[kBulkBufs];
-    __shared__ int abort_flag;
-    if (threadIdx.x != 0) return;
-    const int G = gridDim.x;
-    const int n = (T - (int)blockIdx.x + G - 1) / G;  // tokens of this CTA
-    if (n <= 0) return;
-    for (int b = 0; b < nb; ++b) mbar_init(&full[b], 1);
-    abort_flag = 0;
-    fence_mbar_init();
-    const auto token = [&](int i) { return (int)blockIdx.x + i * G; };
-    const auto load = [&](int i) {
-        const int b = i % nb;
-        mbar_arrive_expect_tx(&full[b], (uint32_t)row_bytes);
-        bulk_load(sbuf + (size_t)b * row_bytes, x + (size_t)token(i) * row_bytes, (uint32_t)row_bytes, &full[b]);
-    };
-    for (int i = 0; i < nb - 1 && i < n; ++i) load(i);
-    int i = 0;
-    for (; i < n; ++i) {
-        const int b = i % nb;
-        if (!mbar_wait(&full[b], (uint32_t)((i / nb) & 1), &abort_flag, status)) break;
-        const int t = token(i);
-        const uint8_t* src = sbuf + (size_t)b * row_bytes;
-        for (int j = 0; j < k; ++j) {
-            const int r = inv_row[(size_t)t * k + j];
-            if ((unsigned)r >= (unsigned)total_rows) continue;
-            bulk_store(xp + (size_t)r * row_bytes, src, (uint32_t)row_bytes);
-        }
-        bulk_commit_group();
-        // the buffer of row i - 1 takes row i + nb - 1 once its stores have read it
-        if (i + nb - 1 < n) {
-            bulk_wait_group_read<1>();
-            load(i + nb - 1);
-        }
-    }
-    if (i < n) {  // timed out: let the loads already issued land before the CTA's shared memory goes
-        for (int j = i; j < n && j < i + nb - 1; ++j) mbar_wait_drain(&full[j % nb], (uint32_t)((j / nb) & 1));
-    }
-    bulk_wait_group<0>();
-}
-
 size_t permute_scratch_bytes(int T, int E) {
     const size_t C = (size_t)(T + kChunk - 1) / kChunk;
     return C * (size_t)E * sizeof(int32_t);
@@ -227,7 +170,7 @@ size_t permute_scratch_bytes(int T, int E) {
 
 cudaError_t launch_permute(const void* x, const int32_t* idx, const int32_t* counts, int T, int d, int E, int k,
                            size_t elem_bytes, void* x_perm, int32_t* offsets, int32_t* perm_tok, int32_t* inv_row,
-                           int32_t* scratch, int* status, int num_sms, cudaStream_t st) {
+                           int32_t* scratch, int* status, cudaStream_t st) {
     const int C = (T + kChunk - 1) / kChunk;
     int launched = 0;
     if (C > 0) {
@@ -241,20 +184,7 @@ cudaError_t launch_permute(const void* x, const int32_t* idx, const int32_t* cou
         permute_rank_kernel<<<C, 256, (size_t)E * kChunkWords * sizeof(uint32_t), st>>>(idx, T, k, E, scratch,
                                                                                           perm_tok, inv_row);
         ++launched;
-        const size_t row_bytes = (size_t)d * elem_bytes;
-        if (x && x_perm && row_bytes % 16 == 0 && row_bytes * 2 <= (size_t)kBulkSmem) {
-            int nb = (int)((size_t)kBulkSmem / row_bytes);
-            nb = nb > kBulkBufs ? kBulkBufs : nb;
-            const size_t smem = (size_t)nb * row_bytes;
-            cudaError_t e = cudaFuncSetAttribute(permute_scatter_bulk_kernel,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            const int grid = T < num_sms ? T : num_sms;
-            permute_scatter_bulk_kernel<<<grid, 32, smem, st>>>(static_cast<const uint8_t*>(x), (int)row_bytes, T, k,
-                                                                inv_row, T * k, static_cast<uint8_t*>(x_perm), nb,
-                                                                status);
-            ++launched;
-        } else if (x && x_perm) {
+        if (x && x_perm) {
             const int vec = (int)((size_t)d * elem_bytes / 16);
             // a block size that divides the row's vectors in U = 4 passes when one does
             int threads = 128;
