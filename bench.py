@@ -57,8 +57,8 @@ if ROOT not in sys.path:
 METRIC = "MoE layer fwd tokens/s (V3-shaped, bf16) and % of BF16 tensor / HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES = ["route", "permute", "ffn_up", "ffn_down", "combine", "bias_update"]
-# E4M3 expert workloads: token rows and h are quantized (1x32 tiles) in the step
-STAGES_FP8 = ["route", "quant_x", "permute", "ffn_up", "quant_h", "ffn_down", "combine", "bias_update"]
+# E4M3 expert workloads: the token rows are quantized (1x32 tiles) in the step, h in the gate/up epilogue
+STAGES_FP8 = ["route", "quant_x", "permute", "ffn_up", "ffn_down", "combine", "bias_update"]
 DOMINANT = "ffn_up"
 WORKLOADS = ["v3_prefill", "v3_decode", "small_bf16", "skew_stress", "tiny_fp32", "v3_prefill_fp8",
              "v3_decode_fp8", "small_fp8"]
@@ -352,8 +352,9 @@ class LayerStep:
         self.offsets, self.perm, self.inv = e(E + 1), e(T * k), e(T * k)
         self.pws = e(max(moe.moe_permute_workspace_size(self.sh), 256), dtype=torch.uint8)
         self.x_perm = e(T * k, d, dtype=dt)   # x_perm, then y_perm
-        self.h = e(T * k, cfg.I, dtype=dt)
-        self.hs = e(T, max(1, cfg.S * cfg.Is), dtype=dt)
+        if not self.fp8:  # (E4M3: h leaves the gate/up launch already quantized)
+            self.h = e(T * k, cfg.I, dtype=dt)
+            self.hs = e(T, max(1, cfg.S * cfg.Is), dtype=dt)
         self.shared_out = e(T, d, dtype=dt) if cfg.S > 0 else None
         self.y = e(T, d, dtype=dt)
         if self.fp8:  # E4M3 expert weights with tile scales, quantized once before timing
@@ -382,16 +383,13 @@ class LayerStep:
             moe.moe_permute(self.xq, self.idx, self.counts, sh, self.xq_perm, self.offsets, self.perm, self.inv,
                             self.pws, st)
             rec(3)
-            moe.moe_ffn_up_fp8(self.xq_perm, self.perm, self.xsc, self.offsets, self.xq if sh_ else None, self.w8, sh,
-                               self.h, self.hs if sh_ else None, st)
+            moe.moe_ffn_up_fp8_quant(self.xq_perm, self.perm, self.xsc, self.offsets, self.xq if sh_ else None,
+                                     self.w8, sh, self.hq, self.h_sc, self.hsq if sh_ else None,
+                                     self.hs_sc if sh_ else None, st)
             rec(4)
-            moe.moe_quantize_fp8(self.h, T * k, cfg.I, 1, moe.MOE_SF_TOKENS, self.hq, self.h_sc, st)
-            if sh_:
-                moe.moe_quantize_fp8(self.hs, T, cfg.S * cfg.Is, 1, moe.MOE_SF_TOKENS, self.hsq, self.hs_sc, st)
-            rec(5)
             moe.moe_ffn_down_fp8(self.hq, self.h_sc, self.offsets, self.hsq if sh_ else None, self.hs_sc, self.w8,
                                  sh, self.x_perm, self.shared_out, st)
-            j = 6
+            j = 5
         else:
             moe.moe_permute(x, self.idx, self.counts, sh, self.x_perm, self.offsets, self.perm, self.inv, self.pws, st)
             rec(2)

@@ -34,7 +34,8 @@ EXPORTS = (
     "moe_ffn_down", "moe_ffn_down_combine", "moe_combine_finish", "moe_combine", "moe_layer_forward",
     "moe_workspace_size", "moe_get_last_error",
     "moe_kernel_launch_count", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
-    "moe_quantize_fp8", "moe_fp8_scale_bytes", "moe_ffn_up_fp8", "moe_ffn_down_fp8", "moe_layer_forward_fp8",
+    "moe_quantize_fp8", "moe_fp8_scale_bytes", "moe_ffn_up_fp8", "moe_ffn_up_fp8_quant", "moe_ffn_down_fp8",
+    "moe_layer_forward_fp8",
     "moe_ep_plan_size", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_return",
     "moe_layer_backward", "moe_backward_workspace_size",
 )
@@ -108,6 +109,7 @@ def lib() -> ctypes.CDLL:
             "moe_get_last_error": [P],
             "moe_quantize_fp8": [P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P],
             "moe_ffn_up_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
+            "moe_ffn_up_fp8_quant": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P, P, P],
             "moe_ffn_down_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_layer_forward_fp8": [P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P, P, P, sz, P],
             "moe_ep_plan": [P, ctypes.c_int32, ctypes.c_int32, S, ctypes.c_int64, P, P, P],
@@ -313,6 +315,13 @@ def fp8_scales(rows, K, layout, device):
 def moe_ffn_up_fp8(xq_perm, perm_tok, x_scale, offsets, xq, experts, shape, h, hs, stream=None):
     _check(lib().moe_ffn_up_fp8(_p(xq_perm), _p(perm_tok), _p(x_scale), _p(offsets), _p(xq), ctypes.byref(experts),
                                 shape, _p(h), _p(hs), _stream(stream)), "moe_ffn_up_fp8")
+
+
+def moe_ffn_up_fp8_quant(xq_perm, perm_tok, x_scale, offsets, xq, experts, shape, hq, h_scale, hsq, hs_scale,
+                         stream=None):
+    _check(lib().moe_ffn_up_fp8_quant(_p(xq_perm), _p(perm_tok), _p(x_scale), _p(offsets), _p(xq),
+                                      ctypes.byref(experts), shape, _p(hq), _p(h_scale), _p(hsq), _p(hs_scale),
+                                      _stream(stream)), "moe_ffn_up_fp8_quant")
 
 
 def moe_ffn_down_fp8(hq, h_scale, offsets, hsq, hs_scale, experts, shape, y_perm, shared_out, stream=None):

@@ -234,7 +234,8 @@ moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1,
 
 moe_status do_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const void* xs, const int32_t* offsets,
                          const uint8_t* xq, const moe_fp8_experts* w, const moe_shape& sh, void* h, void* hs,
-                         int* status, int sms, cudaStream_t st) {
+                         int* status, int sms, cudaStream_t st, uint8_t* hq = nullptr, void* h_scales = nullptr,
+                         uint8_t* hsq = nullptr, void* hs_scales = nullptr) {
     if (sh.T == 0) return MOE_OK;
     const bool shared = xq && sh.S > 0;
     moe::TcUpArgs ur = tc_up_args(xq_perm, nullptr, offsets, w->w1, w->w3, sh, false, h);
@@ -245,12 +246,16 @@ moe_status do_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const 
     ur.xs_pitch = sh.T;
     ur.xs_idx = perm_tok;  // row r holds token perm_tok[r] / k
     ur.xs_div = sh.k;
+    ur.hq = hq;
+    ur.hq_sf = static_cast<uint32_t*>(h_scales);
     moe::TcUpArgs us = tc_up_args(xq, nullptr, nullptr, w->ws1, w->ws3, sh, true, hs);
     us.f8 = true;
     us.w1s = static_cast<const uint8_t*>(w->ws1_scale);
     us.w3s = static_cast<const uint8_t*>(w->ws3_scale);
     us.xs = static_cast<const uint32_t*>(xs);
     us.xs_pitch = sh.T;
+    us.hq = hsq;
+    us.hq_sf = static_cast<uint32_t*>(hs_scales);
     return moe::launch_tc_up(&ur, shared ? &us : nullptr, status, sms, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -761,6 +766,29 @@ moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const
                          static_cast<cudaStream_t>(stream));
 }
 
+moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const int32_t* perm_tok, const void* x_scale,
+                                const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w, moe_shape sh,
+                                uint8_t* hq, void* h_scales, uint8_t* hsq, void* hs_scales, void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(is_fp8(sh), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(offsets && fp8_weights_ok(w, sh), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (xq_perm && perm_tok && x_scale && hq && h_scales), MOE_ERR_INVALID_ARG);
+    const bool shared = xq != nullptr && sh.S > 0;
+    MOE_REQUIRE(!shared || sh.T == 0 || (hsq && hs_scales), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(xq_perm) && aligned16(perm_tok) && aligned16(x_scale) && aligned16(offsets) &&
+                    aligned16(xq) && aligned16(hq) && aligned16(h_scales) && aligned16(hsq) && aligned16(hs_scales) &&
+                    fp8_weights_aligned(w),
+                MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return do_ffn_up_fp8(xq_perm, perm_tok, x_scale, offsets, shared ? xq : nullptr, w, sh, nullptr, nullptr, status,
+                         sms, static_cast<cudaStream_t>(stream), hq, h_scales, shared ? hsq : nullptr,
+                         shared ? hs_scales : nullptr);
+}
+
 moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_scale, const int32_t* offsets, const uint8_t* hsq,
                             const void* hs_scale, const moe_fp8_experts* w, moe_shape sh, void* y_perm,
                             void* shared_out, void* stream) {
@@ -809,14 +837,11 @@ moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float*
     if ((v = do_permute(k8.xq, topk_idx, counts, sh, k8.xq_perm, k8.offsets, k8.perm, k8.inv, k8.pws, status, st)) !=
         MOE_OK)
         return v;
-    if ((v = do_ffn_up_fp8(k8.xq_perm, k8.perm, k8.xs, k8.offsets, shared ? k8.xq : nullptr, w, sh, k8.h, k8.hs,
-                           status, sms, st)) != MOE_OK)
+    // gate/up with h (and hs) quantized by tiles in its epilogue
+    if ((v = do_ffn_up_fp8(k8.xq_perm, k8.perm, k8.xs, k8.offsets, shared ? k8.xq : nullptr, w, sh, nullptr, nullptr,
+                           status, sms, st, k8.hq, k8.h_scale, shared ? k8.hsq : nullptr,
+                           shared ? k8.hs_scale : nullptr)) != MOE_OK)
         return v;
-    if (moe::launch_quantize_mx(k8.h, (long long)sh.T * sh.k, sh.I, 1, false, k8.hq, k8.h_scale, st) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    if (shared &&
-        moe::launch_quantize_mx(k8.hs, sh.T, sh.S * sh.Is, 1, false, k8.hsq, k8.hs_scale, st) != cudaSuccess)
-        return MOE_ERR_CUDA;
     if ((v = do_ffn_down_fp8(k8.hq, k8.h_scale, k8.offsets, shared ? k8.hsq : nullptr, k8.hs_scale, w, sh, k8.y_perm,
                              k8.shared_out, status, sms, st)) != MOE_OK)
         return v;

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -281,6 +282,27 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t mask) {
         : "memory");
 }
 // ---------------------------------------------------------------- block-scaled E4M3
+// Per-tile E4M3 quantization ("DeepSeek V3 From Scratch", "The idea": FP8 with
+// fine-grained quantization tiles): a tile of 32 values gets the scale 2^e with
+// e the smallest integer such that its largest magnitude fits E4M3 (amax <=
+// 448 * 2^e), kept as the byte e + 127.  From the bits of amax (exponent field
+// a, mantissa m): amax fits 448 * 2^e = 1.75 * 2^(8+e) iff a - 127 < 8 + e, or
+// a - 127 == 8 + e and m <= 0.75 * 2^23; so e = a - 135 + (m > 0x600000),
+// clamped to -127 (an all-zero tile gets e = 0).
+__device__ __forceinline__ int mx_tile_exponent(float amax) {
+    if (amax == 0.0f) return 0;
+    const uint32_t u = __float_as_uint(amax);
+    const int a = (int)(u >> 23);
+    const int e = a - 135 + ((u & 0x7fffffu) > 0x600000u ? 1 : 0);
+    return e < -127 ? -127 : e;
+}
+// 2^-e for e in [-127, 126], a normal fp32.
+__device__ __forceinline__ float mx_inv_scale(int e) { return __uint_as_float((uint32_t)(127 - e) << 23); }
+// Two E4M3 codes (round to nearest even, saturating), a in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
 // Shared-memory descriptor of a 32-row x 16-byte matrix stored plainly (no
 // swizzle, K-major): 8-row core matrices of 128 contiguous bytes, the next 8
 // rows 128 bytes further (stride byte offset); one core matrix along the

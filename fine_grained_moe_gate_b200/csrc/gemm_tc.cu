@@ -111,6 +111,10 @@ constexpr int SFA_BYTES = 512, SFB_BYTES = 1024, SF_STAGE_BYTES = SFA_BYTES + SF
 constexpr int SF_STAGES = 16;
 constexpr int SF_GROUP = 8;
 constexpr int SF_GROUPS = SF_STAGES / SF_GROUP;
+// Relay warps: with two, each passes on every other group, so one group's
+// release overlaps the wait for the next (measured no faster than one on the
+// V3 and small E4M3 shapes; one is kept).
+constexpr int SF_RELAYS = 1;
 // Epilogue warps come in groups of four (one per TMEM lane quarter); groups
 // take the tile's 16-token chunks in turn.  The gate/up epilogue (SwiGLU on
 // every element) runs two groups with one exchange buffer each; the down
@@ -123,7 +127,7 @@ __host__ __device__ constexpr int n_xbuf_per_group() { return UP ? 1 : 2; }
 // producer warps after the epilogue warps: the token operand (both), the W3 half (up),
 // the tile scales (E4M3)
 template <bool UP, bool F8>
-__host__ __device__ constexpr int n_extra_producers() { return (UP ? 2 : 1) + (F8 ? 2 : 0); }
+__host__ __device__ constexpr int n_extra_producers() { return (UP ? 2 : 1) + (F8 ? 1 + SF_RELAYS : 0); }
 template <bool UP, bool F8>
 __host__ __device__ constexpr int n_threads() { return 32 * (2 + n_epi_warps<UP>() + n_extra_producers<UP, F8>()); }
 constexpr int XS = 132;                 // row stride (floats) of the epilogue exchange buffer
@@ -225,6 +229,12 @@ struct SetParams {
     const int32_t* row_tok;
     const float* row_w;
     int row_k;
+    // up, E4M3 only, optional: h leaves as E4M3 codes q_out [rows][ldo] with
+    // token-layout tile scales q_sf (word (s, r) at q_sf[s * q_rows + r]),
+    // exactly what quantizing the bf16 h would give; out is then unused.
+    uint8_t* q_out;
+    uint32_t* q_sf;
+    long long q_rows;
 };
 struct Params {
     const int32_t* offsets;
@@ -763,13 +773,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
         }
         cp_async_wait<0>();
         __syncwarp();
-    } else if (F8 && warp == kSfRelay) {
+    } else if (F8 && warp >= kSfRelay && warp < kSfRelay + SF_RELAYS) {
         // ------------------------------------------------ tile-scale relay (E4M3, both CTAs, lane 0)
         // Stages in order, counted across tiles: wait until this CTA's scale
         // copies of the stage have landed; after every SF_GROUP stages (and
         // after the last one) arrive on the leader's sf_full of the group
         // (cluster-scope release; this warp has no copies of its own in
-        // flight, so the release waits for none).
+        // flight, so the release waits for none).  Relay r takes the groups
+        // g with g % SF_RELAYS == r.
+        const int relay = warp - kSfRelay;
         if (lane == 0) {
             const uint32_t leader_sf_full = mapa_shared(smem_u32(&ctl->sf_full[0]), 0);
             int j = 0;
@@ -790,6 +802,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                 const TileCoord tc = tile_coords(tb, G, tile);
                 const int kbn = p.set[tc.g >= p.G0 ? 1 : 0].k_blocks;
                 for (int kb = 0; kb < kbn; ++kb, ++n) {
+                    if ((int)((n / SF_GROUP) % SF_RELAYS) != relay) continue;
                     const int s = (int)(n % SF_STAGES);
                     if (!mbar_wait(&ctl->sf_local[s], (uint32_t)((n / SF_STAGES) & 1), &ctl->abort, p.status)) {
                         ok = false;
@@ -800,7 +813,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                 }
                 if (!ok) break;
             }
-            if (ok && n % SF_GROUP != 0)  // the last, partial group
+            if (ok && n % SF_GROUP != 0 && (int)((n / SF_GROUP) % SF_RELAYS) == relay)  // the last, partial group
                 mbar_arrive_cluster(leader_sf_full + 8u * (uint32_t)((n / SF_GROUP) % SF_GROUPS));
         }
         __syncwarp();
@@ -953,7 +966,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                     float4 u0 = *reinterpret_cast<const float4*>(row + 64 + fj);
                     float4 u1 = *reinterpret_cast<const float4*>(row + 64 + fj + 4);
                     if (NXB == 1) named_bar_sync(1 + eg, 128);  // the single buffer is free for the next chunk
-                    if (tok_ok) {
+                    if (F8 && sp.q_out) {
+                        // h rounded to bf16 (as the plain output), then its 1x32 tiles to E4M3: the four lanes
+                        // of a token's 32 features share the tile's largest magnitude
+                        float hv[8] = {silu_fast(g0.x) * u0.x, silu_fast(g0.y) * u0.y, silu_fast(g0.z) * u0.z,
+                                       silu_fast(g0.w) * u0.w, silu_fast(g1.x) * u1.x, silu_fast(g1.y) * u1.y,
+                                       silu_fast(g1.z) * u1.z, silu_fast(g1.w) * u1.w};
+                        float amax = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            hv[i] = __bfloat162float(__float2bfloat16_rn(hv[i]));
+                            amax = fmaxf(amax, fabsf(hv[i]));
+                        }
+                        if (!tok_ok) amax = 0.0f;
+                        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                        const int ex = mx_tile_exponent(amax);
+                        const float mul = mx_inv_scale(ex);
+                        const uint32_t sbyte = (uint32_t)(ex + 127);
+                        const uint32_t sother = __shfl_xor_sync(0xffffffffu, sbyte, 4);  // the CTA's other tile
+                        if (tok_ok) {
+                            const size_t orow = (size_t)(tok0 + c + my_tok);
+                            const uint32_t c0 = e4m3x2(__fmul_rn(hv[0], mul), __fmul_rn(hv[1], mul)) |
+                                                (e4m3x2(__fmul_rn(hv[2], mul), __fmul_rn(hv[3], mul)) << 16);
+                            const uint32_t c1 = e4m3x2(__fmul_rn(hv[4], mul), __fmul_rn(hv[5], mul)) |
+                                                (e4m3x2(__fmul_rn(hv[6], mul), __fmul_rn(hv[7], mul)) << 16);
+                            *reinterpret_cast<uint2*>(sp.q_out + orow * sp.ldo + fcta + fj) = make_uint2(c0, c1);
+                            if (part == 0) {  // tiles fcta / 32 and the next: bytes j, j + 1 of the stage word
+                                uint8_t* wd = reinterpret_cast<uint8_t*>(sp.q_sf + (size_t)(fcta >> 7) * sp.q_rows + orow);
+                                *reinterpret_cast<uint16_t*>(wd + ((fcta & 127) >> 5)) = (uint16_t)(sbyte | (sother << 8));
+                            }
+                        }
+                    } else if (tok_ok) {
                         uint4 v;
                         v.x = pack_bf16x2(silu_fast(g0.x) * u0.x, silu_fast(g0.y) * u0.y);
                         v.y = pack_bf16x2(silu_fast(g0.z) * u0.z, silu_fast(g0.w) * u0.w);
@@ -1062,6 +1106,10 @@ bool up_set(const TcUpArgs& a, SetMaps& m, SetParams& sp) {
     sp.ldo = a.I;
     sp.f_limit = a.I;
     sp.a_rows = a.gather ? a.gather_rows : a.A_rows;
+    sp.q_out = a.f8 ? a.hq : nullptr;
+    sp.q_sf = a.f8 ? a.hq_sf : nullptr;
+    sp.q_rows = a.A_rows;
+    if (sp.q_out && !sp.q_sf) return false;
     return true;
 }
 

@@ -161,6 +161,10 @@ struct TcUpArgs {
     long long xs_pitch = 0;
     const int32_t* xs_idx = nullptr;
     int xs_div = 1;
+    // E4M3, optional: write h as E4M3 codes hq [A_rows][I] with token-layout
+    // tile scales hq_sf ([I/128][A_rows] words) instead of bf16 H.
+    uint8_t* hq = nullptr;
+    uint32_t* hq_sf = nullptr;
 };
 // Down projection: Y[r][:] = H[r] . W2_g^T, W2_g = [d][K] (K = I), or for
 // the shared group S stacked [d][Is] blocks contracted over K = S * Is.

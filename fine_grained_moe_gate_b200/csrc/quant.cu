@@ -10,10 +10,8 @@
 // format the tensor cores' block-scaled MMA reads.  Codes are
 // E4M3(v * 2^-e), round to nearest even; v * 2^-e is exact in fp32.
 //
-// e from the bits of amax (fp32, exponent field a, mantissa m): amax =
-// (1 + m/2^23) 2^(a-127) fits 448 * 2^e = 1.75 * 2^(8+e) iff a - 127 < 8 + e,
-// or a - 127 == 8 + e and m <= 0.75 * 2^23; so e = a - 135 + (m > 0x600000),
-// clamped to -127 below (an all-zero tile gets e = 0, codes 0).
+// e comes from the bits of amax (mx_tile_exponent, common.cuh); an all-zero
+// tile gets e = 0 and codes 0.
 //
 // Scale layouts (the GEMMs' shared-memory scale atoms hold, for 128 operand
 // rows and one 128-column stage, the byte of row m, tile j at
@@ -49,19 +47,6 @@ __device__ __forceinline__ size_t seg_offset(long long r, int c, long long rows,
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Two codes, a in the low byte (the lower address once stored).
-__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-}
-
-// Smallest e in [-127, 126] with amax <= 448 * 2^e (amax finite, >= 0; 0 for 0).
-__device__ __forceinline__ int tile_exponent(float amax) {
-    if (amax == 0.0f) return 0;
-    const uint32_t u = __float_as_uint(amax);
-    const int a = (int)(u >> 23);
-    const int e = a - 135 + ((u & 0x7fffffu) > 0x600000u ? 1 : 0);
-    return e < -127 ? -127 : e;
-}
 
 template <bool kWeightLayout>
 __global__ void __launch_bounds__(kWarps * 32) quantize_mx_kernel(const uint16_t* __restrict__ src, long long rows,
@@ -91,8 +76,8 @@ __global__ void __launch_bounds__(kWarps * 32) quantize_mx_kernel(const uint16_t
         // the four lanes of a tile
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        const int e = tile_exponent(amax);
-        const float mul = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, a normal fp32 for e in [-127, 126]
+        const int e = mx_tile_exponent(amax);
+        const float mul = mx_inv_scale(e);  // 2^-e
         if (act) {
             uint32_t p[4];
 #pragma unroll

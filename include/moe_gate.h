@@ -381,13 +381,26 @@ typedef struct {
 MOE_API moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const void* x_scales,
                                   const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w, moe_shape sh,
                                   void* h, void* hs, void* stream);
+/* moe_ffn_up_fp8_quant -- moe_ffn_up_fp8 with h and hs leaving the launch
+ * already quantized for moe_ffn_down_fp8: the epilogue rounds h to bf16 as
+ * moe_ffn_up_fp8 writes it, then quantizes each 1x32 tile as
+ * moe_quantize_fp8 does (MOE_SF_TOKENS layout), so hq / h_scales ([T*k][I]
+ * E4M3, [I/128][T*k] words) and hsq / hs_scales ([T][S*Is], [S*Is/128][T])
+ * equal moe_ffn_up_fp8 followed by moe_quantize_fp8, bit for bit, without
+ * the bf16 h round trip through HBM.  Pointers 16-byte aligned; hsq and
+ * hs_scales are needed when xq is given and S > 0.  Errors as moe_ffn_up_fp8. */
+MOE_API moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const int32_t* perm_tok, const void* x_scales,
+                                        const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w,
+                                        moe_shape sh, uint8_t* hq, void* h_scales, uint8_t* hsq, void* hs_scales,
+                                        void* stream);
 MOE_API moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_scales, const int32_t* offsets,
                                     const uint8_t* hsq, const void* hs_scales, const moe_fp8_experts* w,
                                     moe_shape sh, void* y_perm, void* shared_out, void* stream);
 
 /* moe_layer_forward_fp8 -- the layer with FP8 experts: route (bf16 x),
- * quantize x by tiles, permute the E4M3 rows, gate/up, quantize h and hs by
- * tiles, down, combine into y [T][d] bf16.  sh.dtype == MOE_FP8_E4M3;
+ * quantize x by tiles, permute the E4M3 rows, gate/up with h and hs
+ * quantized by tiles in its epilogue (moe_ffn_up_fp8_quant), down, combine
+ * into y [T][d] bf16.  sh.dtype == MOE_FP8_E4M3;
  * workspace >= moe_workspace_size(sh). */
 MOE_API moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float* bias,
                                          const moe_fp8_experts* w, moe_shape sh, void* y, int32_t* topk_idx,

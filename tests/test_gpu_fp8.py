@@ -145,6 +145,18 @@ def _staged(cfg, sh, p, x, q, w8):
     check_status()
     hq, h_sc = _quant(h, T * k, I)
     hsq, hs_sc = _quant(hs, T, S * Is) if S > 0 else (None, None)
+    # the same gate/up with h quantized in its epilogue: bit-identical codes and scales (buffers poisoned, so
+    # every byte must be written)
+    fq = torch.full_like(hq, 0xAB)
+    fsc = torch.full_like(h_sc, 0xAB)
+    fsq = torch.full_like(hsq, 0xAB) if S > 0 else None
+    fssc = torch.full_like(hs_sc, 0xAB) if S > 0 else None
+    moe.moe_ffn_up_fp8_quant(xq_perm, perm, xs, offsets, xq if S > 0 else None, w8, sh, fq, fsc, fsq, fssc)
+    torch.cuda.synchronize()
+    check_status()
+    assert torch.equal(fq, hq) and torch.equal(fsc, h_sc), "fused h quantization"
+    if S > 0:
+        assert torch.equal(fsq, hsq) and torch.equal(fssc, hs_sc), "fused hs quantization"
     y_perm = torch.empty((T * k, d), dtype=torch.bfloat16, device=DEV)
     shared_out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV) if S > 0 else None
     moe.moe_ffn_down_fp8(hq, h_sc, offsets, hsq, hs_sc, w8, sh, y_perm, shared_out)
