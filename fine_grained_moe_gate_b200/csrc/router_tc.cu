@@ -36,8 +36,15 @@ constexpr int RING_BYTES = 4 * (A_BYTES + 256 * BK * 2);
 static_assert(ring_stages<true>() * (A_BYTES + b_stride<true>()) == RING_BYTES, "both rings take the same room");
 // Warps: 0 loads the token boxes (and arms the stage barrier), 6 the W_gate
 // boxes (one issuing thread paces a TMA ring, so two share it), 1 issues the
-// MMAs; after the K loop all eight read the accumulator and finish tokens.
-constexpr int NTHREADS = 256;
+// MMAs; after the K loop all warps read the accumulator and finish tokens.
+// The sigmoid and the top-k of that finish are latency bound, so the pair
+// form, whose finish takes as long as its K loop at V3, runs 16 warps (V3
+// routing 55.3 -> 51.2 us against 8); the one-CTA form keeps 8 (16 measured
+// 10% slower on the small and decode shapes).
+template <bool PAIR>
+__host__ __device__ constexpr int n_threads() {
+    return PAIR ? 512 : 256;
+}
 constexpr int kWarpB = 6;
 constexpr int PS = kMaxExperts + 4;  // row stride (floats) of the score buffers
 constexpr int PART_BYTES = BM * PS * 4;
@@ -77,7 +84,7 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t cluster_addr) {
 // the pair of slice c; the even CTA issues the MMAs, the odd one holds tokens
 // 128..255 of the tile and W_gate rows [N/2, N).
 template <int KMAX, int C, bool PAIR>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(n_threads<PAIR>(), 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ bias, int T, int E, int n_pad, uint32_t tmem_cols, int k_blocks,
                      int k, int32_t* __restrict__ idx, float* __restrict__ w, int32_t* __restrict__ counts,
@@ -85,6 +92,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     constexpr int STAGES = ring_stages<PAIR>();
     constexpr int BSTR = b_stride<PAIR>();
     constexpr int CL = PAIR ? 2 * C : C;  // CTAs per cluster
+    constexpr int NTHREADS = n_threads<PAIR>();
+    constexpr int NWARPS = NTHREADS / 32;
+    static_assert(NWARPS % 4 == 0 && NWARPS >= 8, "whole TMEM lane quarters per warp group");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sA = base;
@@ -258,11 +268,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     if (C > 1) {
         // partial scores of this K slice: TMEM lane r (token r) -> part[r][0..n_pad);
-        // warp w reads lane quarter w % 4, columns of half w / 4
+        // warp w reads lane quarter w % 4, column chunk w / 4 of NWARPS / 4 (multiples of 16)
         const int q = warp & 3;
         const int r = q * 32 + lane;
-        const int c_mid = (n_pad >> 5) << 4;  // a multiple of 16
-        const int c_lo = warp < 4 ? 0 : c_mid, c_hi = warp < 4 ? c_mid : n_pad;
+        constexpr int NCH = NWARPS / 4;
+        const int ch = warp >> 2, n16 = n_pad >> 4;
+        const int c_lo = (n16 * ch / NCH) << 4, c_hi = (n16 * (ch + 1) / NCH) << 4;
         if (mbar_wait(&ctl->tfull, 0, &ctl->abort, status)) {
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
@@ -395,7 +406,7 @@ cudaError_t launch_kc(const CUtensorMap& tx, const CUtensorMap& tw, const float*
     const int tile = PAIR ? 2 * BM : BM;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(((T + tile - 1) / tile) * CL));
-    cfg.blockDim = dim3(NTHREADS);
+    cfg.blockDim = dim3(n_threads<PAIR>());
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
