@@ -364,6 +364,7 @@ class LayerStep:
             tok = moe.MOE_SF_TOKENS
             self.xq, self.xsc = e(T, d, dtype=torch.uint8), moe.fp8_scales(T, d, tok, dev)
             self.xq_perm = e(T * k, d, dtype=torch.uint8)
+            self.xsc_perm = moe.fp8_scales(T * k, d, tok, dev)
             self.hq, self.h_sc = e(T * k, cfg.I, dtype=torch.uint8), moe.fp8_scales(T * k, cfg.I, tok, dev)
             self.hsq, self.hs_sc = e(T, SIs, dtype=torch.uint8), moe.fp8_scales(T, SIs, tok, dev)
             torch.cuda.synchronize()
@@ -383,7 +384,8 @@ class LayerStep:
             moe.moe_permute(self.xq, self.idx, self.counts, sh, self.xq_perm, self.offsets, self.perm, self.inv,
                             self.pws, st)
             rec(3)
-            moe.moe_ffn_up_fp8_quant(self.xq_perm, self.perm, self.xsc, self.offsets, self.xq if sh_ else None,
+            moe.moe_permute_fp8_scales(self.xsc, self.perm, sh, self.xsc_perm, st)
+            moe.moe_ffn_up_fp8_quant(self.xq_perm, self.xsc_perm, self.offsets, self.xq if sh_ else None, self.xsc,
                                      self.w8, sh, self.hq, self.h_sc, self.hsq if sh_ else None,
                                      self.hs_sc if sh_ else None, st)
             rec(4)

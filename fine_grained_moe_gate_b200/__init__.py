@@ -34,7 +34,8 @@ EXPORTS = (
     "moe_ffn_down", "moe_ffn_down_combine", "moe_combine_finish", "moe_combine", "moe_layer_forward",
     "moe_workspace_size", "moe_get_last_error",
     "moe_kernel_launch_count", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
-    "moe_quantize_fp8", "moe_fp8_scale_bytes", "moe_ffn_up_fp8", "moe_ffn_up_fp8_quant", "moe_ffn_down_fp8",
+    "moe_quantize_fp8", "moe_fp8_scale_bytes", "moe_permute_fp8_scales", "moe_ffn_up_fp8", "moe_ffn_up_fp8_quant",
+    "moe_ffn_down_fp8",
     "moe_layer_forward_fp8",
     "moe_ep_plan_size", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_return",
     "moe_layer_backward", "moe_backward_workspace_size",
@@ -110,6 +111,7 @@ def lib() -> ctypes.CDLL:
             "moe_quantize_fp8": [P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P],
             "moe_ffn_up_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_ffn_up_fp8_quant": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P, P, P],
+            "moe_permute_fp8_scales": [P, P, S, P, P],
             "moe_ffn_down_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_layer_forward_fp8": [P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P, P, P, sz, P],
             "moe_ep_plan": [P, ctypes.c_int32, ctypes.c_int32, S, ctypes.c_int64, P, P, P],
@@ -317,9 +319,14 @@ def moe_ffn_up_fp8(xq_perm, perm_tok, x_scale, offsets, xq, experts, shape, h, h
                                 shape, _p(h), _p(hs), _stream(stream)), "moe_ffn_up_fp8")
 
 
-def moe_ffn_up_fp8_quant(xq_perm, perm_tok, x_scale, offsets, xq, experts, shape, hq, h_scale, hsq, hs_scale,
+def moe_permute_fp8_scales(x_scale, perm_tok, shape, xs_perm, stream=None):
+    _check(lib().moe_permute_fp8_scales(_p(x_scale), _p(perm_tok), shape, _p(xs_perm), _stream(stream)),
+           "moe_permute_fp8_scales")
+
+
+def moe_ffn_up_fp8_quant(xq_perm, xs_perm, offsets, xq, x_scale, experts, shape, hq, h_scale, hsq, hs_scale,
                          stream=None):
-    _check(lib().moe_ffn_up_fp8_quant(_p(xq_perm), _p(perm_tok), _p(x_scale), _p(offsets), _p(xq),
+    _check(lib().moe_ffn_up_fp8_quant(_p(xq_perm), _p(xs_perm), _p(offsets), _p(xq), _p(x_scale),
                                       ctypes.byref(experts), shape, _p(hq), _p(h_scale), _p(hsq), _p(hs_scale),
                                       _stream(stream)), "moe_ffn_up_fp8_quant")
 

@@ -235,17 +235,24 @@ moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1,
 moe_status do_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const void* xs, const int32_t* offsets,
                          const uint8_t* xq, const moe_fp8_experts* w, const moe_shape& sh, void* h, void* hs,
                          int* status, int sms, cudaStream_t st, uint8_t* hq = nullptr, void* h_scales = nullptr,
-                         uint8_t* hsq = nullptr, void* hs_scales = nullptr) {
+                         uint8_t* hsq = nullptr, void* hs_scales = nullptr, const void* xs_perm = nullptr) {
     if (sh.T == 0) return MOE_OK;
     const bool shared = xq && sh.S > 0;
     moe::TcUpArgs ur = tc_up_args(xq_perm, nullptr, offsets, w->w1, w->w3, sh, false, h);
     ur.f8 = true;
     ur.w1s = static_cast<const uint8_t*>(w->w1_scale);
     ur.w3s = static_cast<const uint8_t*>(w->w3_scale);
-    ur.xs = static_cast<const uint32_t*>(xs);
-    ur.xs_pitch = sh.T;
-    ur.xs_idx = perm_tok;  // row r holds token perm_tok[r] / k
-    ur.xs_div = sh.k;
+    if (xs_perm) {  // scale words already in xq_perm's row order: contiguous per stage
+        ur.xs = static_cast<const uint32_t*>(xs_perm);
+        ur.xs_pitch = (long long)sh.T * sh.k;
+        ur.xs_idx = nullptr;
+        ur.xs_div = 1;
+    } else {
+        ur.xs = static_cast<const uint32_t*>(xs);
+        ur.xs_pitch = sh.T;
+        ur.xs_idx = perm_tok;  // row r holds token perm_tok[r] / k
+        ur.xs_div = sh.k;
+    }
     ur.hq = hq;
     ur.hq_sf = static_cast<uint32_t*>(h_scales);
     moe::TcUpArgs us = tc_up_args(xq, nullptr, nullptr, w->ws1, w->ws3, sh, true, hs);
@@ -297,8 +304,7 @@ struct Fp8Work {
     uint8_t* xq;
     void* xs;
     uint8_t* xq_perm;
-    void* h;
-    void* hs;
+    void* xs_perm;  // the scale words of xq_perm's rows
     uint8_t* hq;
     void* h_scale;
     uint8_t* hsq;
@@ -310,12 +316,12 @@ struct Fp8Work {
 size_t fp8_work(const moe_shape& sh, char* base, Fp8Work* o) {
     const size_t T = (size_t)sh.T, rows = T * sh.k, SI = (size_t)sh.S * sh.Is, d = (size_t)sh.d, I = (size_t)sh.I;
     // token-layout tile scales: one 32-bit word per row and 128 columns
-    const size_t sizes[15] = {(size_t)(sh.E + 1) * 4, rows * 4, rows * 4, permute_ws(sh), T * d, T * (d / 128) * 4,
-                              rows * d, rows * I * 2, T * SI * 2, rows * I, rows * (I / 128) * 4, T * SI,
+    const size_t sizes[14] = {(size_t)(sh.E + 1) * 4, rows * 4, rows * 4, permute_ws(sh), T * d, T * (d / 128) * 4,
+                              rows * d, rows * (d / 128) * 4, rows * I, rows * (I / 128) * 4, T * SI,
                               T * (SI / 128) * 4, rows * d * 2, T * d * 2};
-    void* ptrs[15];
+    void* ptrs[14];
     size_t off = 0;
-    for (int i = 0; i < 15; ++i) {
+    for (int i = 0; i < 14; ++i) {
         ptrs[i] = base ? base + off : nullptr;
         off += align256(sizes[i]);
     }
@@ -327,14 +333,13 @@ size_t fp8_work(const moe_shape& sh, char* base, Fp8Work* o) {
         o->xq = static_cast<uint8_t*>(ptrs[4]);
         o->xs = ptrs[5];
         o->xq_perm = static_cast<uint8_t*>(ptrs[6]);
-        o->h = ptrs[7];
-        o->hs = ptrs[8];
-        o->hq = static_cast<uint8_t*>(ptrs[9]);
-        o->h_scale = ptrs[10];
-        o->hsq = static_cast<uint8_t*>(ptrs[11]);
-        o->hs_scale = ptrs[12];
-        o->y_perm = ptrs[13];
-        o->shared_out = ptrs[14];
+        o->xs_perm = ptrs[7];
+        o->hq = static_cast<uint8_t*>(ptrs[8]);
+        o->h_scale = ptrs[9];
+        o->hsq = static_cast<uint8_t*>(ptrs[10]);
+        o->hs_scale = ptrs[11];
+        o->y_perm = ptrs[12];
+        o->shared_out = ptrs[13];
     }
     return off;
 }
@@ -766,17 +771,34 @@ moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const
                          static_cast<cudaStream_t>(stream));
 }
 
-moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const int32_t* perm_tok, const void* x_scale,
-                                const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w, moe_shape sh,
+moe_status moe_permute_fp8_scales(const void* x_scales, const int32_t* perm_tok, moe_shape sh, void* xs_perm,
+                                  void* stream) {
+    moe_status v = validate_shape(sh);
+    if (v != MOE_OK) return v;
+    MOE_REQUIRE(is_fp8(sh), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (x_scales && perm_tok && xs_perm), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x_scales) && aligned16(perm_tok) && aligned16(xs_perm), MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return moe::launch_permute_mx_scales(x_scales, perm_tok, sh.k, sh.T, sh.d, xs_perm, status,
+                                         static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const void* xs_perm, const int32_t* offsets,
+                                const uint8_t* xq, const void* x_scale, const moe_fp8_experts* w, moe_shape sh,
                                 uint8_t* hq, void* h_scales, uint8_t* hsq, void* hs_scales, void* stream) {
     moe_status v = validate_shape(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(is_fp8(sh), MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(offsets && fp8_weights_ok(w, sh), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(sh.T == 0 || (xq_perm && perm_tok && x_scale && hq && h_scales), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (xq_perm && xs_perm && hq && h_scales), MOE_ERR_INVALID_ARG);
     const bool shared = xq != nullptr && sh.S > 0;
-    MOE_REQUIRE(!shared || sh.T == 0 || (hsq && hs_scales), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(aligned16(xq_perm) && aligned16(perm_tok) && aligned16(x_scale) && aligned16(offsets) &&
+    MOE_REQUIRE(!shared || sh.T == 0 || (x_scale && hsq && hs_scales), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(xq_perm) && aligned16(xs_perm) && aligned16(x_scale) && aligned16(offsets) &&
                     aligned16(xq) && aligned16(hq) && aligned16(h_scales) && aligned16(hsq) && aligned16(hs_scales) &&
                     fp8_weights_aligned(w),
                 MOE_ERR_ALIGNMENT);
@@ -784,9 +806,9 @@ moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const int32_t* perm_tok,
     int* status;
     v = device_setup(&dev, &status, &sms);
     if (v != MOE_OK) return v;
-    return do_ffn_up_fp8(xq_perm, perm_tok, x_scale, offsets, shared ? xq : nullptr, w, sh, nullptr, nullptr, status,
+    return do_ffn_up_fp8(xq_perm, nullptr, x_scale, offsets, shared ? xq : nullptr, w, sh, nullptr, nullptr, status,
                          sms, static_cast<cudaStream_t>(stream), hq, h_scales, shared ? hsq : nullptr,
-                         shared ? hs_scales : nullptr);
+                         shared ? hs_scales : nullptr, xs_perm);
 }
 
 moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_scale, const int32_t* offsets, const uint8_t* hsq,
@@ -837,10 +859,13 @@ moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float*
     if ((v = do_permute(k8.xq, topk_idx, counts, sh, k8.xq_perm, k8.offsets, k8.perm, k8.inv, k8.pws, status, st)) !=
         MOE_OK)
         return v;
-    // gate/up with h (and hs) quantized by tiles in its epilogue
-    if ((v = do_ffn_up_fp8(k8.xq_perm, k8.perm, k8.xs, k8.offsets, shared ? k8.xq : nullptr, w, sh, nullptr, nullptr,
+    // the token scale words in the permuted rows' order, then gate/up with h (and hs) quantized by tiles in its
+    // epilogue
+    if (moe::launch_permute_mx_scales(k8.xs, k8.perm, sh.k, sh.T, sh.d, k8.xs_perm, status, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if ((v = do_ffn_up_fp8(k8.xq_perm, nullptr, k8.xs, k8.offsets, shared ? k8.xq : nullptr, w, sh, nullptr, nullptr,
                            status, sms, st, k8.hq, k8.h_scale, shared ? k8.hsq : nullptr,
-                           shared ? k8.hs_scale : nullptr)) != MOE_OK)
+                           shared ? k8.hs_scale : nullptr, k8.xs_perm)) != MOE_OK)
         return v;
     if ((v = do_ffn_down_fp8(k8.hq, k8.h_scale, k8.offsets, shared ? k8.hsq : nullptr, k8.hs_scale, w, sh, k8.y_perm,
                              k8.shared_out, status, sms, st)) != MOE_OK)

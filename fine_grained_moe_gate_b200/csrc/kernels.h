@@ -41,6 +41,9 @@ struct GemmArgs {
 };
 
 // quant.cu: per-tile E4M3 quantization (scale layouts described there)
+// out [K/128][T*k] words = the token-layout scales xs [K/128][T] of the rows of a permutation (row r: token perm[r] / k).
+cudaError_t launch_permute_mx_scales(const void* xs, const int32_t* perm, int k, long long T, int K, void* out,
+                                     int* status, cudaStream_t st);
 size_t mx_scale_bytes(long long rows, int K, bool weight_layout);
 cudaError_t launch_quantize_mx(const void* src, long long rows, int kseg, int nseg, bool weight_layout, uint8_t* q,
                                void* scales, cudaStream_t st);

@@ -104,7 +104,40 @@ __global__ void __launch_bounds__(kWarps * 32) quantize_mx_kernel(const uint16_t
     }
 }
 
+// Token-layout scale words of the rows of a permutation: out[s][r] =
+// xs[s][perm[r] / k] (row r of xq_perm holds token perm[r] / k), so that the
+// GEMM reads a stage's words of consecutive rows with coalesced loads.
+__global__ void permute_mx_scales_kernel(const uint32_t* __restrict__ xs, const int32_t* __restrict__ perm, int k,
+                                         long long T, long long rows, int nst, uint32_t* __restrict__ out,
+                                         int* status) {
+    const long long n = rows * nst;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const int s = (int)(i / rows);
+        const long long r = i - (long long)s * rows;
+        const long long t = perm[r] / k;
+        if (t < 0 || t >= T) {
+            report(status, kStDeviceCheck);
+            continue;
+        }
+        out[i] = xs[(size_t)s * T + t];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_permute_mx_scales(const void* xs, const int32_t* perm, int k, long long T, int K, void* out,
+                                     int* status, cudaStream_t st) {
+    const long long rows = T * k;
+    const int nst = K / 128;
+    if (rows <= 0 || nst <= 0) return cudaSuccess;
+    const long long n = rows * nst;
+    long long blocks = (n + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    permute_mx_scales_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint32_t*>(xs), perm, k, T, rows, nst,
+                                                               static_cast<uint32_t*>(out), status);
+    note_launches(1);
+    return cudaGetLastError();
+}
 
 size_t mx_scale_bytes(long long rows, int K, bool weight_layout) {
     const size_t nst = (size_t)(K / 128);

@@ -381,16 +381,28 @@ typedef struct {
 MOE_API moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const void* x_scales,
                                   const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w, moe_shape sh,
                                   void* h, void* hs, void* stream);
-/* moe_ffn_up_fp8_quant -- moe_ffn_up_fp8 with h and hs leaving the launch
- * already quantized for moe_ffn_down_fp8: the epilogue rounds h to bf16 as
- * moe_ffn_up_fp8 writes it, then quantizes each 1x32 tile as
- * moe_quantize_fp8 does (MOE_SF_TOKENS layout), so hq / h_scales ([T*k][I]
- * E4M3, [I/128][T*k] words) and hsq / hs_scales ([T][S*Is], [S*Is/128][T])
- * equal moe_ffn_up_fp8 followed by moe_quantize_fp8, bit for bit, without
- * the bf16 h round trip through HBM.  Pointers 16-byte aligned; hsq and
- * hs_scales are needed when xq is given and S > 0.  Errors as moe_ffn_up_fp8. */
-MOE_API moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const int32_t* perm_tok, const void* x_scales,
-                                        const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w,
+/* moe_permute_fp8_scales -- the token-layout tile scales of the permuted
+ * rows: xs_perm [d/128][T*k] 32-bit words with word (s, r) = word (s,
+ * perm_tok[r] / k) of x_scales [d/128][T] (MOE_SF_TOKENS layout of the
+ * unpermuted E4M3 tokens; perm_tok from moe_permute).  sh.dtype ==
+ * MOE_FP8_E4M3; pointers 16-byte aligned.  A perm_tok entry outside the batch
+ * reports MOE_ERR_DEVICE_CHECK and leaves its word unwritten. */
+MOE_API moe_status moe_permute_fp8_scales(const void* x_scales, const int32_t* perm_tok, moe_shape sh, void* xs_perm,
+                                          void* stream);
+
+/* moe_ffn_up_fp8_quant -- the gate/up launch of moe_ffn_up_fp8 with h and hs
+ * leaving it already quantized for moe_ffn_down_fp8, and the token scales
+ * read in row order: xs_perm [d/128][T*k] the scales of xq_perm's rows
+ * (moe_permute_fp8_scales), x_scales [d/128][T] those of xq (shared experts;
+ * unused when xq is NULL).  The epilogue rounds h to bf16 as moe_ffn_up_fp8
+ * writes it, then quantizes each 1x32 tile as moe_quantize_fp8 does
+ * (MOE_SF_TOKENS layout), so hq / h_scales ([T*k][I] E4M3, [I/128][T*k]
+ * words) and hsq / hs_scales ([T][S*Is], [S*Is/128][T]) equal moe_ffn_up_fp8
+ * followed by moe_quantize_fp8, bit for bit, without the bf16 h round trip
+ * through HBM.  Pointers 16-byte aligned; x_scales, hsq and hs_scales are
+ * needed when xq is given and S > 0.  Errors as moe_ffn_up_fp8. */
+MOE_API moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const void* xs_perm, const int32_t* offsets,
+                                        const uint8_t* xq, const void* x_scales, const moe_fp8_experts* w,
                                         moe_shape sh, uint8_t* hq, void* h_scales, uint8_t* hsq, void* hs_scales,
                                         void* stream);
 MOE_API moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_scales, const int32_t* offsets,
@@ -398,8 +410,9 @@ MOE_API moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_scales, con
                                     moe_shape sh, void* y_perm, void* shared_out, void* stream);
 
 /* moe_layer_forward_fp8 -- the layer with FP8 experts: route (bf16 x),
- * quantize x by tiles, permute the E4M3 rows, gate/up with h and hs
- * quantized by tiles in its epilogue (moe_ffn_up_fp8_quant), down, combine
+ * quantize x by tiles, permute the E4M3 rows and their scale words, gate/up
+ * with h and hs quantized by tiles in its epilogue (moe_ffn_up_fp8_quant),
+ * down, combine
  * into y [T][d] bf16.  sh.dtype == MOE_FP8_E4M3;
  * workspace >= moe_workspace_size(sh). */
 MOE_API moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float* bias,

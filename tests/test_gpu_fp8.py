@@ -151,9 +151,16 @@ def _staged(cfg, sh, p, x, q, w8):
     fsc = torch.full_like(h_sc, 0xAB)
     fsq = torch.full_like(hsq, 0xAB) if S > 0 else None
     fssc = torch.full_like(hs_sc, 0xAB) if S > 0 else None
-    moe.moe_ffn_up_fp8_quant(xq_perm, perm, xs, offsets, xq if S > 0 else None, w8, sh, fq, fsc, fsq, fssc)
+    xs_perm = torch.full_like(moe.fp8_scales(T * k, d, TOK, DEV), 0xAB)
+    moe.moe_permute_fp8_scales(xs, perm, sh, xs_perm)
+    moe.moe_ffn_up_fp8_quant(xq_perm, xs_perm, offsets, xq if S > 0 else None, xs if S > 0 else None, w8, sh, fq, fsc,
+                             fsq, fssc)
     torch.cuda.synchronize()
     check_status()
+    # the permuted scale words are the unpermuted tokens' words, row by row
+    words = xs.view(torch.int32).view(d // 128, T).cpu().numpy()
+    assert np.array_equal(xs_perm.view(torch.int32).view(d // 128, T * k).cpu().numpy(),
+                          words[:, perm.cpu().numpy() // k]), "permuted scales"
     assert torch.equal(fq, hq) and torch.equal(fsc, h_sc), "fused h quantization"
     if S > 0:
         assert torch.equal(fsq, hsq) and torch.equal(fssc, hs_sc), "fused hs quantization"
