@@ -511,6 +511,29 @@ __global__ void pad_plan_kernel(const int32_t* __restrict__ counts, int E, int32
     pstart[E] = acc;
 }
 
+// Zero the padding rows of group g (rows [pstart[g] + count, pstart[g + 1]))
+// in every padded operand the weight-gradient contractions run over: the
+// real rows are all written by their producers, so only these need clearing.
+// One block per group; each matrix's rows are whole 16-byte vectors.
+struct PadZero {
+    uint4* p[4];
+    int vec[4];  // 16-byte vectors per row
+};
+__global__ void pad_zero_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ pstart, int E,
+                                PadZero z) {
+    const int g = blockIdx.x;
+    if (g >= E) return;
+    const int c = counts[g] < 0 ? 0 : counts[g];
+    const long long r0 = (long long)pstart[g] + c, r1 = pstart[g + 1];
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const long long n = (r1 - r0) * z.vec[m];
+        uint4* base = z.p[m] + r0 * z.vec[m];
+        for (long long i = threadIdx.x; i < n; i += blockDim.x) base[i] = zero;
+    }
+}
+
 // last index i in [0, n) with a[i] <= v (a non-decreasing, a[0] <= v)
 __device__ __forceinline__ int last_le(const int32_t* a, int n, int v) {
     int lo = 0, hi = n - 1;
@@ -853,10 +876,13 @@ cudaError_t experts_backward_tc(const BackwardArgs& a, const BwdBufs& b, int* st
     // padded layout of the routed rows, and the zero padding of the GEMM operands
     pad_plan_kernel<<<1, 32, 0, st>>>(a.counts, E, b.pstart, status);
     note_launches(1);
-    TC_TRY(cudaMemsetAsync(b.x_pad, 0, (size_t)Rp * d * 2, st));
-    TC_TRY(cudaMemsetAsync(b.h_pad, 0, (size_t)Rp * I * 2, st));
-    TC_TRY(cudaMemsetAsync(b.do_pad, 0, (size_t)Rp * d * 2, st));
-    TC_TRY(cudaMemsetAsync(b.dadg, 0, (size_t)Rp * 2 * I * 2, st));
+    {
+        PadZero z{{reinterpret_cast<uint4*>(b.x_pad), reinterpret_cast<uint4*>(b.h_pad),
+                    reinterpret_cast<uint4*>(b.do_pad), reinterpret_cast<uint4*>(b.dadg)},
+                   {d / 8, I / 8, d / 8, 2 * I / 8}};
+        pad_zero_kernel<<<E, 256, 0, st>>>(a.counts, b.pstart, E, z);
+        note_launches(1);
+    }
     if (R > 0) {
         gather_pad_kernel<<<num_sms * 4, 256, 0, st>>>(static_cast<const uint4*>(a.x), b.perm, b.offsets, b.pstart,
                                                        E, k, R, T, d / 8, b.prow, reinterpret_cast<uint4*>(b.x_pad),
