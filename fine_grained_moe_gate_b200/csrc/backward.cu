@@ -448,31 +448,53 @@ __global__ void router_bwd_kernel(const float* __restrict__ s, const int32_t* __
     }
 }
 
-constexpr int kLossChunk = 64;  // tokens per partial sum of the balance loss
+constexpr int kLossChunk = 32;  // tokens per partial sum of the balance loss
 
-// Block (c, b): chunk[b][c][i] = sum over tokens t of chunk c of sequence b of s_ti / tot_t.
+// Block (c, b): chunk[b][c][i] = sum over tokens t of chunk c of sequence b of s_ti / tot_t.  The block's
+// threads form G = blockDim.x / E groups (E <= blockDim.x); group g sums the tokens t0 + g, t0 + g + G, ...
+// of the chunk, and the G partial sums are added in group order (deterministic for a given block size).
 __global__ void balance_chunk_kernel(const float* __restrict__ s, const float* __restrict__ tot, int L, int E,
                                      int C, float* __restrict__ chunk) {
+    extern __shared__ float gpart[];  // [G][E]
     const int b = blockIdx.y, c = blockIdx.x;
     const int t0 = b * L + c * kLossChunk, t1 = min((b + 1) * L, t0 + kLossChunk);
-    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+    const int G = blockDim.x / E;
+    const int g = threadIdx.x / E, i = threadIdx.x - g * E;
+    if (g < G) {
         float P = 0.0f;
-        for (int t = t0; t < t1; ++t) P += s[(long long)t * E + i] / tot[t];
-        chunk[((long long)b * C + c) * E + i] = P;
+        for (int t = t0 + g; t < t1; t += G) P += s[(long long)t * E + i] / tot[t];
+        gpart[g * E + i] = P;
+    }
+    __syncthreads();
+    if (threadIdx.x < E) {
+        float P = 0.0f;
+        for (int q = 0; q < G; ++q) P += gpart[q * E + threadIdx.x];
+        chunk[((long long)b * C + c) * E + threadIdx.x] = P;
     }
 }
 
-// One block per sequence b: part[b] = alpha * sum_i f_bi P_bi, the chunks summed in order.
+// One block per sequence b: part[b] = alpha * sum_i f_bi P_bi, the chunks summed in order: G = blockDim.x / E
+// groups each add a contiguous run of chunks, then the runs are added in order.
 __global__ void balance_part_kernel(const float* __restrict__ chunk, const int32_t* __restrict__ cnt, float alpha,
                                     int L, int E, int k, int C, float* __restrict__ part) {
+    extern __shared__ float gpart[];  // [G][E]
     __shared__ float red[32];
     const int b = blockIdx.x;
     const float fscale = (float)E / ((float)k * (float)L);
-    float v = 0.0f;
-    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+    const int G = blockDim.x / E;
+    const int g = threadIdx.x / E, i = threadIdx.x - g * E;
+    if (g < G) {
+        const int c0 = g * C / G, c1 = (g + 1) * C / G;
         float P = 0.0f;
-        for (int c = 0; c < C; ++c) P += chunk[((long long)b * C + c) * E + i];
-        v += fscale * (float)cnt[(long long)b * E + i] * (P / (float)L);
+        for (int c = c0; c < c1; ++c) P += chunk[((long long)b * C + c) * E + i];
+        gpart[g * E + i] = P;
+    }
+    __syncthreads();
+    float v = 0.0f;
+    if (threadIdx.x < E) {
+        float P = 0.0f;
+        for (int q = 0; q < G; ++q) P += gpart[q * E + threadIdx.x];
+        v = fscale * (float)cnt[(long long)b * E + threadIdx.x] * (P / (float)L);
     }
     v = block_sum(v, red);
     if (threadIdx.x == 0) part[b] = alpha * v;
@@ -1139,8 +1161,9 @@ cudaError_t launch_layer_backward(const BackwardArgs& a, int* status, int num_sm
                                                         nb, T, E, k, dz, tot, status);
         note_launches(1);
         if (nb > 0 && a.loss) {
-            balance_chunk_kernel<<<dim3((unsigned)C, (unsigned)nb), 256, 0, st>>>(a.s, tot, a.seq_len, E, C, chunk);
-            balance_part_kernel<<<nb, 256, 0, st>>>(chunk, cnt, a.alpha, a.seq_len, E, k, C, part);
+            const size_t gsm = (size_t)(256 / E) * E * sizeof(float);  // E <= 256
+            balance_chunk_kernel<<<dim3((unsigned)C, (unsigned)nb), 256, gsm, st>>>(a.s, tot, a.seq_len, E, C, chunk);
+            balance_part_kernel<<<nb, 256, gsm, st>>>(chunk, cnt, a.alpha, a.seq_len, E, k, C, part);
             balance_sum_kernel<<<1, 32, 0, st>>>(part, nb, a.loss);
             note_launches(3);
         }
