@@ -44,7 +44,7 @@ def _projection_checks(cfg, p, x, idx, counts, y_layer, w):
     expert with rows and the shared set: h (gate/up + SwiGLU epilogue)
     against the oracle's up projection of the same token rows, and y_perm /
     shared_out (down) against the oracle's down projection of the GPU's own h
-    (so that each launch is judged alone), element by element.  Small
+    (so that each launch is checked alone), element by element.  Small
     experts are checked in full; large ones on every 7th row and a feature
     subset that reaches every tile."""
     sh = moe.shape_of(cfg)
@@ -113,7 +113,7 @@ def _full_check(cfg, p, x, n_sample, seed, s_tol="auto", projections=False):
     assert int(counts.sum()) == cfg.T * cfg.k       # no dropped tokens
     tokens = np.sort(rng.choice(cfg.T, size=min(n_sample, cfg.T), replace=False))
     yt = y[torch.as_tensor(tokens, device=DEV)]
-    # the benchmark spec bar against the oracle computed from scratch
+    # the layer bar (5e-3 relative Frobenius for bf16) against the oracle computed from scratch
     y_ref, _ = oracle_terms(p, x, idx, w, tokens, cfg.S)
     err = rel_fro(as_f64(yt), to_f64_rows(oracle.finalize(y_ref, np.uint16)))
     assert err <= 5e-3, err
