@@ -213,3 +213,18 @@ def test_backward_binding_marshals_and_raises(L):
         moe.moe_layer_backward(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, sh, FAKE, FAKE, FAKE, FAKE, FAKE, -1.0,
                                0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, ws, stream=0)
     assert ei.value.status == INVALID
+
+
+def test_fp8_scale_and_fused_up_checks(L):
+    c = ctypes.c_void_p
+    sh8 = shape(d=256, I=128, Is=128, dtype=moe.MOE_FP8_E4M3)
+    # moe_permute_fp8_scales(x_scales, perm_tok, sh, xs_perm, stream)
+    assert L.moe_permute_fp8_scales(c(FAKE), c(FAKE), shape(), c(FAKE), None) == INVALID   # not an E4M3 shape
+    assert L.moe_permute_fp8_scales(None, c(FAKE), sh8, c(FAKE), None) == INVALID
+    assert L.moe_permute_fp8_scales(c(FAKE), c(FAKE), sh8, c(FAKE + 4), None) == ALIGN
+    # moe_ffn_up_fp8_quant(xq_perm, xs_perm, offsets, xq, x_scales, w, sh, hq, h_scales, hsq, hs_scales, stream)
+    w8 = moe.MoEFp8Experts()
+    assert L.moe_ffn_up_fp8_quant(c(FAKE), c(FAKE), c(FAKE), None, None, ctypes.byref(w8), shape(), c(FAKE), c(FAKE),
+                                  None, None, None) == INVALID                              # not an E4M3 shape
+    assert L.moe_ffn_up_fp8_quant(c(FAKE), c(FAKE), c(FAKE), None, None, ctypes.byref(w8), sh8, c(FAKE), c(FAKE),
+                                  None, None, None) == INVALID                              # no expert weights
