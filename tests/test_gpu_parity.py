@@ -57,6 +57,7 @@ ROUTER_BF16 = [
     dict(T=8192, d=1024, E=256, k=8),     # V3 routing width, K split over 2 pairs
     dict(T=6000, d=192, E=24, k=4),       # uneven K slices (3 blocks over 2 pairs), N = 32
     dict(T=20000, d=128, E=256, k=12),    # k > 8, no K split, more pairs than one wave
+    dict(T=5000, d=128, E=8, k=2),        # the smallest pair MMA: N = 16, 8 W_gate rows per CTA
 ]
 
 
