@@ -364,9 +364,10 @@ class LayerStep:
             tok = moe.MOE_SF_TOKENS
             self.xq, self.xsc = e(T, d, dtype=torch.uint8), moe.fp8_scales(T, d, tok, dev)
             self.xq_perm = e(T * k, d, dtype=torch.uint8)
-            self.xsc_perm = moe.fp8_scales(T * k, d, tok, dev)
-            self.hq, self.h_sc = e(T * k, cfg.I, dtype=torch.uint8), moe.fp8_scales(T * k, cfg.I, tok, dev)
-            self.hsq, self.hs_sc = e(T, SIs, dtype=torch.uint8), moe.fp8_scales(T, SIs, tok, dev)
+            # token scales as the GEMMs' tile images: x's routed and shared tiles, h's and hs's
+            self.x_img, self.xsh_img = moe.fp8_tile_images(T * k, E, d, dev), moe.fp8_tile_images(T, 1, d, dev)
+            self.hq, self.h_img = e(T * k, cfg.I, dtype=torch.uint8), moe.fp8_tile_images(T * k, E, cfg.I, dev)
+            self.hsq, self.hs_img = e(T, SIs, dtype=torch.uint8), moe.fp8_tile_images(T, 1, SIs, dev)
             torch.cuda.synchronize()
 
     def __call__(self, i, ev=None):
@@ -384,12 +385,14 @@ class LayerStep:
             moe.moe_permute(self.xq, self.idx, self.counts, sh, self.xq_perm, self.offsets, self.perm, self.inv,
                             self.pws, st)
             rec(3)
-            moe.moe_permute_fp8_scales(self.xsc, self.perm, sh, self.xsc_perm, st)
-            moe.moe_ffn_up_fp8_quant(self.xq_perm, self.xsc_perm, self.offsets, self.xq if sh_ else None, self.xsc,
-                                     self.w8, sh, self.hq, self.h_sc, self.hsq if sh_ else None,
-                                     self.hs_sc if sh_ else None, st)
+            moe.moe_fp8_tile_scales(self.xsc, T, cfg.d, self.perm, k, self.offsets, cfg.E, T * k, self.x_img, st)
+            if sh_:
+                moe.moe_fp8_tile_scales(self.xsc, T, cfg.d, None, 1, None, 1, T, self.xsh_img, st)
+            moe.moe_ffn_up_fp8_quant(self.xq_perm, self.x_img, self.offsets, self.xq if sh_ else None, self.xsh_img,
+                                     self.w8, sh, self.hq, self.h_img, self.hsq if sh_ else None,
+                                     self.hs_img if sh_ else None, st)
             rec(4)
-            moe.moe_ffn_down_fp8(self.hq, self.h_sc, self.offsets, self.hsq if sh_ else None, self.hs_sc, self.w8,
+            moe.moe_ffn_down_fp8(self.hq, self.h_img, self.offsets, self.hsq if sh_ else None, self.hs_img, self.w8,
                                  sh, self.x_perm, self.shared_out, st)
             j = 5
         else:

@@ -34,8 +34,8 @@ EXPORTS = (
     "moe_ffn_down", "moe_ffn_down_combine", "moe_combine_finish", "moe_combine", "moe_layer_forward",
     "moe_workspace_size", "moe_get_last_error",
     "moe_kernel_launch_count", "moe_selftest_bounded_wait", "moe_status_string", "moe_abi_version",
-    "moe_quantize_fp8", "moe_fp8_scale_bytes", "moe_permute_fp8_scales", "moe_ffn_up_fp8", "moe_ffn_up_fp8_quant",
-    "moe_ffn_down_fp8",
+    "moe_quantize_fp8", "moe_fp8_scale_bytes", "moe_fp8_tile_scales", "moe_fp8_tile_scale_bytes", "moe_ffn_up_fp8",
+    "moe_ffn_up_fp8_quant", "moe_ffn_down_fp8",
     "moe_layer_forward_fp8",
     "moe_ep_plan_size", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_return",
     "moe_layer_backward", "moe_backward_workspace_size",
@@ -66,17 +66,18 @@ def shape_of(cfg, T: int | None = None) -> MoEShape:
 
 
 class MoEFp8Experts(ctypes.Structure):
-    """moe_fp8_experts: E4M3 expert weights and their 1x32-tile power-of-two scales (weight layout)."""
-    _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "w1_scale", "w3", "w3_scale", "w2", "w2_scale",
-                                               "ws1", "ws1_scale", "ws3", "ws3_scale", "ws2", "ws2_scale")]
+    """moe_fp8_experts: E4M3 expert weights and their 1x32-tile power-of-two
+    scales (W1/W3 scales in one gate/up buffer, W2 in 128-row atoms)."""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "w3", "w13_scale", "w2", "w2_scale",
+                                               "ws1", "ws3", "ws13_scale", "ws2", "ws2_scale")]
 
 
 def fp8_experts(q: dict) -> MoEFp8Experts:
-    """MoEFp8Experts from a dict of device tensors with keys w1q, w1s, ... (the
-    layout of ``quantize_experts_fp8``).  The tensors must outlive its use."""
-    f = {}
-    for n in ("w1", "w3", "w2", "ws1", "ws3", "ws2"):
-        f[n] = _p(q.get(n + "q"))
+    """MoEFp8Experts from a dict of device tensors with keys w1q, w3q, w13s,
+    w2q, w2s, ... (the layout of ``quantize_experts_fp8``).  The tensors must
+    outlive its use."""
+    f = {n: _p(q.get(n + "q")) for n in ("w1", "w3", "w2", "ws1", "ws3", "ws2")}
+    for n in ("w13", "w2", "ws13", "ws2"):
         f[n + "_scale"] = _p(q.get(n + "s"))
     return MoEFp8Experts(**f)
 
@@ -111,7 +112,8 @@ def lib() -> ctypes.CDLL:
             "moe_quantize_fp8": [P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, P],
             "moe_ffn_up_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_ffn_up_fp8_quant": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P, P, P],
-            "moe_permute_fp8_scales": [P, P, S, P, P],
+            "moe_fp8_tile_scales": [P, ctypes.c_int64, ctypes.c_int32, P, ctypes.c_int32, P, ctypes.c_int32,
+                                    ctypes.c_int64, P, P],
             "moe_ffn_down_fp8": [P, P, P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P],
             "moe_layer_forward_fp8": [P, P, P, ctypes.POINTER(MoEFp8Experts), S, P, P, P, P, P, sz, P],
             "moe_ep_plan": [P, ctypes.c_int32, ctypes.c_int32, S, ctypes.c_int64, P, P, P],
@@ -133,6 +135,8 @@ def lib() -> ctypes.CDLL:
         L.moe_backward_workspace_size.restype = sz
         L.moe_fp8_scale_bytes.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32]
         L.moe_fp8_scale_bytes.restype = sz
+        L.moe_fp8_tile_scale_bytes.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32]
+        L.moe_fp8_tile_scale_bytes.restype = sz
         L.moe_ep_plan_size.argtypes = [ctypes.c_int32, S]
         L.moe_ep_plan_size.restype = sz
         L.moe_kernel_launch_count.argtypes = []
@@ -292,7 +296,7 @@ def moe_abi_version() -> int:
 
 # ---- FP8 experts -------------------------------------------------------------
 
-MOE_SF_TOKENS, MOE_SF_WEIGHTS = 0, 1
+MOE_SF_TOKENS, MOE_SF_WEIGHTS, MOE_SF_GATE, MOE_SF_UP = 0, 1, 2, 3
 
 
 def moe_fp8_scale_bytes(rows, K, layout) -> int:
@@ -314,25 +318,39 @@ def fp8_scales(rows, K, layout, device):
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-def moe_ffn_up_fp8(xq_perm, perm_tok, x_scale, offsets, xq, experts, shape, h, hs, stream=None):
-    _check(lib().moe_ffn_up_fp8(_p(xq_perm), _p(perm_tok), _p(x_scale), _p(offsets), _p(xq), ctypes.byref(experts),
+def moe_fp8_tile_scale_bytes(rows, groups, K) -> int:
+    return lib().moe_fp8_tile_scale_bytes(rows, groups, K)
+
+
+def fp8_tile_images(rows, groups, K, device):
+    """An uninitialised device buffer for the token tile images of `rows`
+    operand rows in `groups` groups with K columns (uint8)."""
+    import torch
+    n = moe_fp8_tile_scale_bytes(rows, groups, K)
+    if n == 0:
+        raise MoEError(1, "moe_fp8_tile_scale_bytes: K must be a multiple of 128, 1 <= groups <= 256")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def moe_fp8_tile_scales(src, src_rows, K, row_of, row_div, offsets, groups, rows, tiles, stream=None):
+    _check(lib().moe_fp8_tile_scales(_p(src), src_rows, K, _p(row_of), row_div, _p(offsets), groups, rows, _p(tiles),
+                                     _stream(stream)), "moe_fp8_tile_scales")
+
+
+def moe_ffn_up_fp8(xq_perm, x_tiles, offsets, xq, xsh_tiles, experts, shape, h, hs, stream=None):
+    _check(lib().moe_ffn_up_fp8(_p(xq_perm), _p(x_tiles), _p(offsets), _p(xq), _p(xsh_tiles), ctypes.byref(experts),
                                 shape, _p(h), _p(hs), _stream(stream)), "moe_ffn_up_fp8")
 
 
-def moe_permute_fp8_scales(x_scale, perm_tok, shape, xs_perm, stream=None):
-    _check(lib().moe_permute_fp8_scales(_p(x_scale), _p(perm_tok), shape, _p(xs_perm), _stream(stream)),
-           "moe_permute_fp8_scales")
-
-
-def moe_ffn_up_fp8_quant(xq_perm, xs_perm, offsets, xq, x_scale, experts, shape, hq, h_scale, hsq, hs_scale,
+def moe_ffn_up_fp8_quant(xq_perm, x_tiles, offsets, xq, xsh_tiles, experts, shape, hq, h_tiles, hsq, hs_tiles,
                          stream=None):
-    _check(lib().moe_ffn_up_fp8_quant(_p(xq_perm), _p(xs_perm), _p(offsets), _p(xq), _p(x_scale),
-                                      ctypes.byref(experts), shape, _p(hq), _p(h_scale), _p(hsq), _p(hs_scale),
+    _check(lib().moe_ffn_up_fp8_quant(_p(xq_perm), _p(x_tiles), _p(offsets), _p(xq), _p(xsh_tiles),
+                                      ctypes.byref(experts), shape, _p(hq), _p(h_tiles), _p(hsq), _p(hs_tiles),
                                       _stream(stream)), "moe_ffn_up_fp8_quant")
 
 
-def moe_ffn_down_fp8(hq, h_scale, offsets, hsq, hs_scale, experts, shape, y_perm, shared_out, stream=None):
-    _check(lib().moe_ffn_down_fp8(_p(hq), _p(h_scale), _p(offsets), _p(hsq), _p(hs_scale), ctypes.byref(experts),
+def moe_ffn_down_fp8(hq, h_tiles, offsets, hsq, hs_tiles, experts, shape, y_perm, shared_out, stream=None):
+    _check(lib().moe_ffn_down_fp8(_p(hq), _p(h_tiles), _p(offsets), _p(hsq), _p(hs_tiles), ctypes.byref(experts),
                                   shape, _p(y_perm), _p(shared_out), _stream(stream)), "moe_ffn_down_fp8")
 
 
@@ -344,21 +362,30 @@ def moe_layer_forward_fp8(x, w_gate, bias, experts, shape, y, topk_idx, topk_w, 
 
 def quantize_experts_fp8(p: dict, stream=None) -> dict:
     """E4M3 copies of a layer's bf16 expert weights (device tensors) through
-    moe_quantize_fp8, tile scales in the weights' layout (MOE_SF_WEIGHTS):
-    W1/W3/W2 and the shared Ws1/Ws3 row by row, the shared Ws2 [S][d][Is] as
-    d rows across its S blocks.  Returns uint8 codes (the weights' own shapes)
-    and scale buffers under w1q, w1s, ..."""
+    moe_quantize_fp8: W1 and W3 (Ws1 and Ws3) with their scales in one gate/up
+    buffer (MOE_SF_GATE, MOE_SF_UP), W2 in 128-row atoms (MOE_SF_WEIGHTS), the
+    shared Ws2 [S][d][Is] as d rows across its S blocks.  Returns uint8 codes
+    (the weights' own shapes) under w1q, w3q, w2q, ... and scale buffers under
+    w13s, w2s, ws13s, ws2s."""
     import torch
     out = {}
-    for n in ("w1", "w3", "w2", "ws1", "ws3"):
-        w = p[n]
-        if w is None or w.numel() == 0:
+    for a, b in (("w1", "w3"), ("ws1", "ws3")):
+        w1, w3 = p.get(a), p.get(b)
+        if w1 is None or w1.numel() == 0:
             continue
-        rows, K = w.numel() // w.shape[-1], w.shape[-1]
-        q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
-        sc = fp8_scales(rows, K, MOE_SF_WEIGHTS, w.device)
-        moe_quantize_fp8(w, rows, K, 1, MOE_SF_WEIGHTS, q, sc, stream)
-        out[n + "q"], out[n + "s"] = q, sc
+        rows, K = w1.numel() // w1.shape[-1], w1.shape[-1]
+        sc = fp8_scales(rows, K, MOE_SF_GATE, w1.device)
+        for n, w, lay in ((a, w1, MOE_SF_GATE), (b, w3, MOE_SF_UP)):
+            q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+            moe_quantize_fp8(w, rows, K, 1, lay, q, sc, stream)
+            out[n + "q"] = q
+        out[a[:-1] + "13s"] = sc
+    w = p["w2"]
+    rows, K = w.numel() // w.shape[-1], w.shape[-1]
+    q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    sc = fp8_scales(rows, K, MOE_SF_WEIGHTS, w.device)
+    moe_quantize_fp8(w, rows, K, 1, MOE_SF_WEIGHTS, q, sc, stream)
+    out["w2q"], out["w2s"] = q, sc
     w = p.get("ws2")
     if w is not None and w.numel() > 0:
         S, d, Is = w.shape

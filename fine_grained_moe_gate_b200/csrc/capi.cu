@@ -232,67 +232,58 @@ moe_status do_swiglu(const void* x_perm, const int32_t* offsets, const void* w1,
 // ---- FP8 experts -----------------------------------------------------------
 
 
-moe_status do_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const void* xs, const int32_t* offsets,
-                         const uint8_t* xq, const moe_fp8_experts* w, const moe_shape& sh, void* h, void* hs,
-                         int* status, int sms, cudaStream_t st, uint8_t* hq = nullptr, void* h_scales = nullptr,
-                         uint8_t* hsq = nullptr, void* hs_scales = nullptr, const void* xs_perm = nullptr) {
+moe_status do_ffn_up_fp8(const uint8_t* xq_perm, const void* x_tiles, const int32_t* offsets, const uint8_t* xq,
+                         const void* xsh_tiles, const moe_fp8_experts* w, const moe_shape& sh, void* h, void* hs,
+                         int* status, int sms, cudaStream_t st, uint8_t* hq = nullptr, void* h_tiles = nullptr,
+                         uint8_t* hsq = nullptr, void* hs_tiles = nullptr) {
     if (sh.T == 0) return MOE_OK;
     const bool shared = xq && sh.S > 0;
     moe::TcUpArgs ur = tc_up_args(xq_perm, nullptr, offsets, w->w1, w->w3, sh, false, h);
     ur.f8 = true;
-    ur.w1s = static_cast<const uint8_t*>(w->w1_scale);
-    ur.w3s = static_cast<const uint8_t*>(w->w3_scale);
-    if (xs_perm) {  // scale words already in xq_perm's row order: contiguous per stage
-        ur.xs = static_cast<const uint32_t*>(xs_perm);
-        ur.xs_pitch = (long long)sh.T * sh.k;
-        ur.xs_idx = nullptr;
-        ur.xs_div = 1;
-    } else {
-        ur.xs = static_cast<const uint32_t*>(xs);
-        ur.xs_pitch = sh.T;
-        ur.xs_idx = perm_tok;  // row r holds token perm_tok[r] / k
-        ur.xs_div = sh.k;
-    }
+    ur.w13s = static_cast<const uint8_t*>(w->w13_scale);
+    ur.xs = static_cast<const uint32_t*>(x_tiles);
+    ur.xs_tiles = moe::mx_tile_images((long long)sh.T * sh.k, sh.E);
     ur.hq = hq;
-    ur.hq_sf = static_cast<uint32_t*>(h_scales);
+    ur.hq_img = static_cast<uint32_t*>(h_tiles);
     moe::TcUpArgs us = tc_up_args(xq, nullptr, nullptr, w->ws1, w->ws3, sh, true, hs);
     us.f8 = true;
-    us.w1s = static_cast<const uint8_t*>(w->ws1_scale);
-    us.w3s = static_cast<const uint8_t*>(w->ws3_scale);
-    us.xs = static_cast<const uint32_t*>(xs);
-    us.xs_pitch = sh.T;
+    us.w13s = static_cast<const uint8_t*>(w->ws13_scale);
+    us.xs = static_cast<const uint32_t*>(xsh_tiles);
+    us.xs_tiles = moe::mx_tile_images(sh.T, 1);
     us.hq = hsq;
-    us.hq_sf = static_cast<uint32_t*>(hs_scales);
+    us.hq_img = static_cast<uint32_t*>(hs_tiles);
     return moe::launch_tc_up(&ur, shared ? &us : nullptr, status, sms, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-moe_status do_ffn_down_fp8(const uint8_t* hq, const void* h_scale, const int32_t* offsets, const uint8_t* hsq,
-                           const void* hs_scale, const moe_fp8_experts* w, const moe_shape& sh, void* y_perm,
+moe_status do_ffn_down_fp8(const uint8_t* hq, const void* h_tiles, const int32_t* offsets, const uint8_t* hsq,
+                           const void* hs_tiles, const moe_fp8_experts* w, const moe_shape& sh, void* y_perm,
                            void* shared_out, int* status, int sms, cudaStream_t st) {
     if (sh.T == 0) return MOE_OK;
     const bool shared = hsq && sh.S > 0;
     moe::TcDownArgs dr = tc_down_args(hq, offsets, w->w2, sh, false, y_perm);
     dr.f8 = true;
     dr.w2s = static_cast<const uint8_t*>(w->w2_scale);
-    dr.hs = static_cast<const uint32_t*>(h_scale);
+    dr.hs = static_cast<const uint32_t*>(h_tiles);
+    dr.hs_tiles = moe::mx_tile_images((long long)sh.T * sh.k, sh.E);
     moe::TcDownArgs ds = tc_down_args(hsq, nullptr, w->ws2, sh, true, shared_out);
     ds.f8 = true;
     ds.w2s = static_cast<const uint8_t*>(w->ws2_scale);
-    ds.hs = static_cast<const uint32_t*>(hs_scale);
+    ds.hs = static_cast<const uint32_t*>(hs_tiles);
+    ds.hs_tiles = moe::mx_tile_images(sh.T, 1);
     return moe::launch_tc_down(&dr, shared ? &ds : nullptr, status, sms, st) == cudaSuccess ? MOE_OK
                                                                                               : MOE_ERR_CUDA;
 }
 
 bool fp8_weights_ok(const moe_fp8_experts* w, const moe_shape& sh) {
-    if (!w || !w->w1 || !w->w3 || !w->w2 || !w->w1_scale || !w->w3_scale || !w->w2_scale) return false;
-    if (sh.S > 0 && (!w->ws1 || !w->ws3 || !w->ws2 || !w->ws1_scale || !w->ws3_scale || !w->ws2_scale)) return false;
+    if (!w || !w->w1 || !w->w3 || !w->w2 || !w->w13_scale || !w->w2_scale) return false;
+    if (sh.S > 0 && (!w->ws1 || !w->ws3 || !w->ws2 || !w->ws13_scale || !w->ws2_scale)) return false;
     return true;
 }
 
 bool fp8_weights_aligned(const moe_fp8_experts* w) {
     return aligned16(w->w1) && aligned16(w->w3) && aligned16(w->w2) && aligned16(w->ws1) && aligned16(w->ws3) &&
-           aligned16(w->ws2) && aligned16(w->w1_scale) && aligned16(w->w3_scale) && aligned16(w->w2_scale) &&
-           aligned16(w->ws1_scale) && aligned16(w->ws3_scale) && aligned16(w->ws2_scale);
+           aligned16(w->ws2) && aligned16(w->w13_scale) && aligned16(w->w2_scale) && aligned16(w->ws13_scale) &&
+           aligned16(w->ws2_scale);
 }
 
 // Workspace of moe_layer_forward_fp8, carved in this order.
@@ -304,24 +295,33 @@ struct Fp8Work {
     uint8_t* xq;
     void* xs;
     uint8_t* xq_perm;
-    void* xs_perm;  // the scale words of xq_perm's rows
+    void* x_tiles;    // token images of xq_perm's tiles
+    void* xsh_tiles;  // token images of xq's tiles (shared experts)
     uint8_t* hq;
-    void* h_scale;
+    void* h_tiles;
     uint8_t* hsq;
-    void* hs_scale;
+    void* hs_tiles;
     void* y_perm;
     void* shared_out;
 };
 
+// Bytes of the token images of `rows` rows in `groups` groups, K columns.
+size_t tile_image_bytes(long long rows, int groups, int K) {
+    return (size_t)moe::mx_tile_images(rows, groups) * (size_t)(K / 128) * 1024;
+}
+
 size_t fp8_work(const moe_shape& sh, char* base, Fp8Work* o) {
     const size_t T = (size_t)sh.T, rows = T * sh.k, SI = (size_t)sh.S * sh.Is, d = (size_t)sh.d, I = (size_t)sh.I;
-    // token-layout tile scales: one 32-bit word per row and 128 columns
-    const size_t sizes[14] = {(size_t)(sh.E + 1) * 4, rows * 4, rows * 4, permute_ws(sh), T * d, T * (d / 128) * 4,
-                              rows * d, rows * (d / 128) * 4, rows * I, rows * (I / 128) * 4, T * SI,
-                              T * (SI / 128) * 4, rows * d * 2, T * d * 2};
-    void* ptrs[14];
+    const bool S = sh.S > 0;
+    // token-layout tile scales of x: one 32-bit word per row and 128 columns
+    const size_t sizes[15] = {(size_t)(sh.E + 1) * 4, rows * 4, rows * 4, permute_ws(sh), T * d, T * (d / 128) * 4,
+                              rows * d, tile_image_bytes((long long)rows, sh.E, sh.d),
+                              S ? tile_image_bytes(sh.T, 1, sh.d) : 0, rows * I,
+                              tile_image_bytes((long long)rows, sh.E, sh.I), T * SI,
+                              S ? tile_image_bytes(sh.T, 1, (int)SI) : 0, rows * d * 2, T * d * 2};
+    void* ptrs[15];
     size_t off = 0;
-    for (int i = 0; i < 14; ++i) {
+    for (int i = 0; i < 15; ++i) {
         ptrs[i] = base ? base + off : nullptr;
         off += align256(sizes[i]);
     }
@@ -333,13 +333,14 @@ size_t fp8_work(const moe_shape& sh, char* base, Fp8Work* o) {
         o->xq = static_cast<uint8_t*>(ptrs[4]);
         o->xs = ptrs[5];
         o->xq_perm = static_cast<uint8_t*>(ptrs[6]);
-        o->xs_perm = ptrs[7];
-        o->hq = static_cast<uint8_t*>(ptrs[8]);
-        o->h_scale = ptrs[9];
-        o->hsq = static_cast<uint8_t*>(ptrs[10]);
-        o->hs_scale = ptrs[11];
-        o->y_perm = ptrs[12];
-        o->shared_out = ptrs[13];
+        o->x_tiles = ptrs[7];
+        o->xsh_tiles = ptrs[8];
+        o->hq = static_cast<uint8_t*>(ptrs[9]);
+        o->h_tiles = ptrs[10];
+        o->hsq = static_cast<uint8_t*>(ptrs[11]);
+        o->hs_tiles = ptrs[12];
+        o->y_perm = ptrs[13];
+        o->shared_out = ptrs[14];
     }
     return off;
 }
@@ -728,14 +729,14 @@ moe_status moe_layer_forward(const void* x, const void* w_gate, const float* bia
 }
 
 size_t moe_fp8_scale_bytes(int64_t rows, int32_t K, int32_t layout) {
-    if (rows < 0 || K <= 0 || K % 128 != 0 || (layout != MOE_SF_TOKENS && layout != MOE_SF_WEIGHTS)) return 0;
-    return moe::mx_scale_bytes(rows, K, layout == MOE_SF_WEIGHTS);
+    if (rows < 0 || K <= 0 || K % 128 != 0 || layout < MOE_SF_TOKENS || layout > MOE_SF_UP) return 0;
+    return moe::mx_scale_bytes(rows, K, layout);
 }
 
 moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t kseg, int32_t nseg, int32_t layout, uint8_t* q,
                             void* scales, void* stream) {
     MOE_REQUIRE(rows >= 0 && kseg > 0 && nseg >= 1, MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(layout == MOE_SF_TOKENS || layout == MOE_SF_WEIGHTS, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(layout >= MOE_SF_TOKENS && layout <= MOE_SF_UP, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(kseg % 128 == 0, MOE_ERR_UNSUPPORTED);
     MOE_REQUIRE((long long)kseg * nseg < (1ll << 31), MOE_ERR_UNSUPPORTED);
     MOE_REQUIRE(rows == 0 || (src && q && scales), MOE_ERR_INVALID_ARG);
@@ -744,91 +745,97 @@ moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t kseg, int32_t
     int* status;
     moe_status v = device_setup(&dev, &status, &sms);
     if (v != MOE_OK) return v;
-    return moe::launch_quantize_mx(src, rows, kseg, nseg, layout == MOE_SF_WEIGHTS, q, scales,
+    return moe::launch_quantize_mx(src, rows, kseg, nseg, layout, q, scales, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+size_t moe_fp8_tile_scale_bytes(int64_t rows, int32_t groups, int32_t K) {
+    if (rows < 0 || groups < 1 || groups > moe::kMaxGroups || K <= 0 || K % 128 != 0) return 0;
+    return tile_image_bytes(rows, groups, K);
+}
+
+moe_status moe_fp8_tile_scales(const void* src, int64_t src_rows, int32_t K, const int32_t* row_of, int32_t row_div,
+                               const int32_t* offsets, int32_t groups, int64_t rows, void* tiles, void* stream) {
+    MOE_REQUIRE(src_rows >= 0 && rows >= 0 && K > 0 && row_div >= 1, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(groups >= 1 && groups <= moe::kMaxGroups && (offsets || groups == 1), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(K % 128 == 0, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(rows < (1ll << 31) && src_rows < (1ll << 31), MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(rows == 0 || (src && tiles), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(src) && aligned16(row_of) && aligned16(offsets) && aligned16(tiles), MOE_ERR_ALIGNMENT);
+    int dev, sms;
+    int* status;
+    moe_status v = device_setup(&dev, &status, &sms);
+    if (v != MOE_OK) return v;
+    return moe::launch_tile_scales(src, src_rows, K, row_of, row_div, offsets, groups, rows, tiles, status,
                                    static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }
 
-moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const void* x_scale,
-                          const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w, moe_shape sh, void* h,
-                          void* hs, void* stream) {
+moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const void* x_tiles, const int32_t* offsets, const uint8_t* xq,
+                          const void* xsh_tiles, const moe_fp8_experts* w, moe_shape sh, void* h, void* hs,
+                          void* stream) {
     moe_status v = validate_shape(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(is_fp8(sh), MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(offsets && fp8_weights_ok(w, sh), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(sh.T == 0 || (xq_perm && perm_tok && x_scale && h), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (xq_perm && x_tiles && h), MOE_ERR_INVALID_ARG);
     const bool shared = xq != nullptr && sh.S > 0;
-    MOE_REQUIRE(!shared || sh.T == 0 || hs, MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(aligned16(xq_perm) && aligned16(perm_tok) && aligned16(x_scale) && aligned16(offsets) &&
+    MOE_REQUIRE(!shared || sh.T == 0 || (xsh_tiles && hs), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(xq_perm) && aligned16(x_tiles) && aligned16(xsh_tiles) && aligned16(offsets) &&
                     aligned16(xq) && aligned16(h) && aligned16(hs) && fp8_weights_aligned(w),
                 MOE_ERR_ALIGNMENT);
     int dev, sms;
     int* status;
     v = device_setup(&dev, &status, &sms);
     if (v != MOE_OK) return v;
-    return do_ffn_up_fp8(xq_perm, perm_tok, x_scale, offsets, shared ? xq : nullptr, w, sh, h, hs, status, sms,
+    return do_ffn_up_fp8(xq_perm, x_tiles, offsets, shared ? xq : nullptr, xsh_tiles, w, sh, h, hs, status, sms,
                          static_cast<cudaStream_t>(stream));
 }
 
-moe_status moe_permute_fp8_scales(const void* x_scales, const int32_t* perm_tok, moe_shape sh, void* xs_perm,
-                                  void* stream) {
-    moe_status v = validate_shape(sh);
-    if (v != MOE_OK) return v;
-    MOE_REQUIRE(is_fp8(sh), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(sh.T == 0 || (x_scales && perm_tok && xs_perm), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(aligned16(x_scales) && aligned16(perm_tok) && aligned16(xs_perm), MOE_ERR_ALIGNMENT);
-    int dev, sms;
-    int* status;
-    v = device_setup(&dev, &status, &sms);
-    if (v != MOE_OK) return v;
-    return moe::launch_permute_mx_scales(x_scales, perm_tok, sh.k, sh.T, sh.d, xs_perm, status,
-                                         static_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? MOE_OK
-               : MOE_ERR_CUDA;
-}
-
-moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const void* xs_perm, const int32_t* offsets,
-                                const uint8_t* xq, const void* x_scale, const moe_fp8_experts* w, moe_shape sh,
-                                uint8_t* hq, void* h_scales, uint8_t* hsq, void* hs_scales, void* stream) {
+moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const void* x_tiles, const int32_t* offsets,
+                                const uint8_t* xq, const void* xsh_tiles, const moe_fp8_experts* w, moe_shape sh,
+                                uint8_t* hq, void* h_tiles, uint8_t* hsq, void* hs_tiles, void* stream) {
     moe_status v = validate_shape(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(is_fp8(sh), MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(offsets && fp8_weights_ok(w, sh), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(sh.T == 0 || (xq_perm && xs_perm && hq && h_scales), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (xq_perm && x_tiles && hq && h_tiles), MOE_ERR_INVALID_ARG);
     const bool shared = xq != nullptr && sh.S > 0;
-    MOE_REQUIRE(!shared || sh.T == 0 || (x_scale && hsq && hs_scales), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(aligned16(xq_perm) && aligned16(xs_perm) && aligned16(x_scale) && aligned16(offsets) &&
-                    aligned16(xq) && aligned16(hq) && aligned16(h_scales) && aligned16(hsq) && aligned16(hs_scales) &&
+    MOE_REQUIRE(!shared || sh.T == 0 || (xsh_tiles && hsq && hs_tiles), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(xq_perm) && aligned16(x_tiles) && aligned16(xsh_tiles) && aligned16(offsets) &&
+                    aligned16(xq) && aligned16(hq) && aligned16(h_tiles) && aligned16(hsq) && aligned16(hs_tiles) &&
                     fp8_weights_aligned(w),
                 MOE_ERR_ALIGNMENT);
     int dev, sms;
     int* status;
     v = device_setup(&dev, &status, &sms);
     if (v != MOE_OK) return v;
-    return do_ffn_up_fp8(xq_perm, nullptr, x_scale, offsets, shared ? xq : nullptr, w, sh, nullptr, nullptr, status,
-                         sms, static_cast<cudaStream_t>(stream), hq, h_scales, shared ? hsq : nullptr,
-                         shared ? hs_scales : nullptr, xs_perm);
+    return do_ffn_up_fp8(xq_perm, x_tiles, offsets, shared ? xq : nullptr, xsh_tiles, w, sh, nullptr, nullptr,
+                         status, sms, static_cast<cudaStream_t>(stream), hq, h_tiles, shared ? hsq : nullptr,
+                         shared ? hs_tiles : nullptr);
 }
 
-moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_scale, const int32_t* offsets, const uint8_t* hsq,
-                            const void* hs_scale, const moe_fp8_experts* w, moe_shape sh, void* y_perm,
+moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_tiles, const int32_t* offsets, const uint8_t* hsq,
+                            const void* hs_tiles, const moe_fp8_experts* w, moe_shape sh, void* y_perm,
                             void* shared_out, void* stream) {
     moe_status v = validate_shape(sh);
     if (v != MOE_OK) return v;
     MOE_REQUIRE(is_fp8(sh), MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(offsets && fp8_weights_ok(w, sh), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(sh.T == 0 || (hq && h_scale && y_perm), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(sh.T == 0 || (hq && h_tiles && y_perm), MOE_ERR_INVALID_ARG);
     const bool shared = hsq != nullptr && sh.S > 0;
-    MOE_REQUIRE(!shared || sh.T == 0 || (hs_scale && shared_out), MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(aligned16(hq) && aligned16(h_scale) && aligned16(offsets) && aligned16(hsq) && aligned16(hs_scale) &&
+    MOE_REQUIRE(!shared || sh.T == 0 || (hs_tiles && shared_out), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(hq) && aligned16(h_tiles) && aligned16(offsets) && aligned16(hsq) && aligned16(hs_tiles) &&
                     aligned16(y_perm) && aligned16(shared_out) && fp8_weights_aligned(w),
                 MOE_ERR_ALIGNMENT);
     int dev, sms;
     int* status;
     v = device_setup(&dev, &status, &sms);
     if (v != MOE_OK) return v;
-    return do_ffn_down_fp8(hq, h_scale, offsets, shared ? hsq : nullptr, hs_scale, w, sh, y_perm, shared_out, status,
+    return do_ffn_down_fp8(hq, h_tiles, offsets, shared ? hsq : nullptr, hs_tiles, w, sh, y_perm, shared_out, status,
                            sms, static_cast<cudaStream_t>(stream));
 }
 
@@ -855,19 +862,25 @@ moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float*
     const bool shared = sh.S > 0;
     if ((v = do_route(x, w_gate, bias, sh, topk_idx, topk_w, counts, nullptr, status, sms, st)) != MOE_OK) return v;
     if (sh.T == 0) return MOE_OK;
-    if (moe::launch_quantize_mx(x, sh.T, sh.d, 1, false, k8.xq, k8.xs, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe::launch_quantize_mx(x, sh.T, sh.d, 1, moe::kMxTokens, k8.xq, k8.xs, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
     if ((v = do_permute(k8.xq, topk_idx, counts, sh, k8.xq_perm, k8.offsets, k8.perm, k8.inv, k8.pws, status, st)) !=
         MOE_OK)
         return v;
-    // the token scale words in the permuted rows' order, then gate/up with h (and hs) quantized by tiles in its
-    // epilogue
-    if (moe::launch_permute_mx_scales(k8.xs, k8.perm, sh.k, sh.T, sh.d, k8.xs_perm, status, st) != cudaSuccess)
+    // the token images of the tiles (routed rows through the permutation, the shared experts' rows as they
+    // are), then gate/up with h (and hs) quantized by tiles in its epilogue
+    const long long rows = (long long)sh.T * sh.k;
+    if (moe::launch_tile_scales(k8.xs, sh.T, sh.d, k8.perm, sh.k, k8.offsets, sh.E, rows, k8.x_tiles, status, st) !=
+        cudaSuccess)
         return MOE_ERR_CUDA;
-    if ((v = do_ffn_up_fp8(k8.xq_perm, nullptr, k8.xs, k8.offsets, shared ? k8.xq : nullptr, w, sh, nullptr, nullptr,
-                           status, sms, st, k8.hq, k8.h_scale, shared ? k8.hsq : nullptr,
-                           shared ? k8.hs_scale : nullptr, k8.xs_perm)) != MOE_OK)
+    if (shared && moe::launch_tile_scales(k8.xs, sh.T, sh.d, nullptr, 1, nullptr, 1, sh.T, k8.xsh_tiles, status, st) !=
+                      cudaSuccess)
+        return MOE_ERR_CUDA;
+    if ((v = do_ffn_up_fp8(k8.xq_perm, k8.x_tiles, k8.offsets, shared ? k8.xq : nullptr, k8.xsh_tiles, w, sh, nullptr,
+                           nullptr, status, sms, st, k8.hq, k8.h_tiles, shared ? k8.hsq : nullptr,
+                           shared ? k8.hs_tiles : nullptr)) != MOE_OK)
         return v;
-    if ((v = do_ffn_down_fp8(k8.hq, k8.h_scale, k8.offsets, shared ? k8.hsq : nullptr, k8.hs_scale, w, sh, k8.y_perm,
+    if ((v = do_ffn_down_fp8(k8.hq, k8.h_tiles, k8.offsets, shared ? k8.hsq : nullptr, k8.hs_tiles, w, sh, k8.y_perm,
                              k8.shared_out, status, sms, st)) != MOE_OK)
         return v;
     return moe::launch_combine(k8.y_perm, topk_w, k8.inv, shared ? k8.shared_out : nullptr, sh.T, sh.d, sh.k, true, y,

@@ -303,6 +303,23 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
     return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
 }
 
+// ---------------------------------------------------------------- token tiles of the grouped GEMMs
+// A group of n rows runs as ceil(n / 256) token tiles of near-equal size (the
+// MMA's N is at most 256).  Equal sizes keep the clusters that share a weight
+// tile at the same pace.  The E4M3 token scales of a tile travel as one
+// 256-word image per 128-column stage, in the order the tensor-memory scale
+// copy reads them: token j's word at (j / 128) * 128 + (j % 32) * 4 + (j / 32) % 4.
+constexpr int kTokTile = 256;
+__host__ __device__ __forceinline__ int token_tiles(int n) { return (n + kTokTile - 1) / kTokTile; }
+__host__ __device__ __forceinline__ void token_tile_split(int rows, int ntt, int tt, int& start, int& len) {
+    const int q = rows / ntt, r = rows - q * ntt;
+    start = tt * q + (tt < r ? tt : r);
+    len = q + (tt < r ? 1 : 0);
+}
+__host__ __device__ __forceinline__ int tile_image_word(int j) {
+    return ((j >> 7) << 7) | ((j & 31) << 2) | ((j >> 5) & 3);
+}
+
 // Shared-memory descriptor of a 32-row x 16-byte matrix stored plainly (no
 // swizzle, K-major): 8-row core matrices of 128 contiguous bytes, the next 8
 // rows 128 bytes further (stride byte offset); one core matrix along the

@@ -72,10 +72,9 @@ constexpr int BK = 64;                  // bf16 K per stage: one 128-byte swizzl
 // K elements per stage for the operand type: 64 bf16 or 128 E4M3 (128 bytes either way)
 template <bool F8>
 __host__ __device__ constexpr int bk_elems() { return F8 ? 128 : 64; }
-// Ring depth of the operand tiles: the E4M3 kernel keeps a ring of tile scales beside
-// it and runs 5 stages
+// Ring depth of the operand tiles (an E4M3 stage also carries its tile scales)
 template <bool F8>
-__host__ __device__ constexpr int n_stages() { return F8 ? 5 : 6; }
+__host__ __device__ constexpr int n_stages() { return 6; }
 constexpr int A_BYTES = 128 * BK * 2;   // this CTA's 128 weight rows
 constexpr int B_ROWS = 128;             // this CTA's half of <= 256 tokens
 constexpr int B_BYTES = B_ROWS * BK * 2;
@@ -85,36 +84,19 @@ constexpr int B_BYTES = B_ROWS * BK * 2;
 // balanced tiles.
 constexpr int NXBOX = B_ROWS / 16;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
-constexpr int NT = 256;                 // tokens per tile (MMA N <= 256)
 constexpr uint32_t ACC_COLS = 256;      // one accumulator buffer
 constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
 // E4M3 with per-tile scales (block-scaled MMA): the scales of a stage sit in
 // tensor memory beside the accumulators, so the second accumulator gives up
 // 16 columns and holds tiles of at most 240 tokens (larger ones use the
-// first).  Scale atoms, per stage: A (this CTA's 128 weight rows x 4 tiles,
-// 512 bytes, 4 columns) and B (up to 256 tokens x 4 tiles, two 512-byte
-// atoms, 8 columns).
+// first).  Every ring stage has a scale slot of its own: this CTA's 128
+// weight rows x 4 tiles (one 512-byte atom, 4 columns) and the tile's token
+// image (up to 256 tokens x 4 tiles, 1024 bytes, 8 columns), both brought by
+// TMA onto the stage's full barrier, so the MMA issuer waits once per stage
+// for operands and scales alike.
 constexpr uint32_t ACC1_COLS_F8 = 240;
 constexpr uint32_t SFA_COL = 496, SFB_COL = 504;
 constexpr int SFA_BYTES = 512, SFB_BYTES = 1024, SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
-// The scales have a ring of their own, deeper than the operands': their
-// copies are small loads with the latency of a round trip to L2 or DRAM, so
-// many stages must be in flight at once.  A loader warp issues a stage's
-// copies (cp.async) and an arrive that fires on the CTA-local barrier
-// sf_local once they have landed; a relay warp, which issues no copies of its
-// own, waits for that and passes the stages on to the leader's MMA issuer in
-// groups of SF_GROUP (sf_full, one cluster-scope release per group: such a
-// release costs about a microsecond, several times an MMA stage).  A
-// release issued by the loader itself would also wait for all the stages it
-// still has in flight.  Measured on the V3 prefill shape (gate/up, E4M3):
-// groups of 1, 4 and 8 stages ran at 0.80, 1.62 and 1.71 PFLOP/s.
-constexpr int SF_STAGES = 16;
-constexpr int SF_GROUP = 8;
-constexpr int SF_GROUPS = SF_STAGES / SF_GROUP;
-// Relay warps: with two, each passes on every other group, so one group's
-// release overlaps the wait for the next (measured no faster than one on the
-// V3 and small E4M3 shapes; one is kept).
-constexpr int SF_RELAYS = 1;
 // Epilogue warps come in groups of four (one per TMEM lane quarter); groups
 // take the tile's 16-token chunks in turn.  The gate/up epilogue (SwiGLU on
 // every element) runs two groups with one exchange buffer each; the down
@@ -127,7 +109,7 @@ __host__ __device__ constexpr int n_xbuf_per_group() { return UP ? 1 : 2; }
 // producer warps after the epilogue warps: the token operand (both), the W3 half (up),
 // the tile scales (E4M3)
 template <bool UP, bool F8>
-__host__ __device__ constexpr int n_extra_producers() { return (UP ? 2 : 1) + (F8 ? 1 + SF_RELAYS : 0); }
+__host__ __device__ constexpr int n_extra_producers() { return (UP ? 2 : 1) + (F8 ? 1 : 0); }
 template <bool UP, bool F8>
 __host__ __device__ constexpr int n_threads() { return 32 * (2 + n_epi_warps<UP>() + n_extra_producers<UP, F8>()); }
 constexpr int XS = 132;                 // row stride (floats) of the epilogue exchange buffer
@@ -159,9 +141,6 @@ constexpr int MAX_STAGES = 6;
 struct Ctl {
     uint64_t full[MAX_STAGES];
     uint64_t empty[MAX_STAGES];
-    uint64_t sf_local[SF_STAGES];  // E4M3: this CTA's scale copies of the stage landed (32 loader lanes)
-    uint64_t sf_full[SF_GROUPS];   // E4M3, leader: both CTAs' relays passed a group of stages on
-    uint64_t sf_empty[SF_STAGES];  // E4M3: the MMAs that read the slot are done
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t tq_full[TQ];   // in both CTAs: slot holds the next tile
@@ -177,6 +156,7 @@ struct Tables {
     int rows[kMaxTcGroups];
     int ttiles[kMaxTcGroups];  // token tiles per group
     int fgroup[kMaxTcGroups];  // > 0: the group's tiles run in groups of this many feature tiles (see tile_coords)
+    int tbase[kMaxTcGroups];   // routed groups: index of the group's first token tile among all routed groups
     int prefix[kMaxTcGroups + 1];
 };
 // The shared set's gate/up tiles (every token x S * Is features: 32 token
@@ -191,7 +171,7 @@ static_assert(n_epi_warps<true>() / 4 * n_xbuf_per_group<true>() == 2, "exchange
 static_assert(n_epi_warps<false>() / 4 * n_xbuf_per_group<false>() == 2, "exchange buffers");
 // ring, tile scales (E4M3), epilogue exchange buffers, control, tables
 template <bool F8>
-__host__ __device__ constexpr size_t sf_region_bytes() { return F8 ? (size_t)SF_STAGES * SF_STAGE_BYTES : 0; }
+__host__ __device__ constexpr size_t sf_region_bytes() { return F8 ? (size_t)n_stages<F8>() * SF_STAGE_BYTES : 0; }
 template <bool F8>
 __host__ __device__ constexpr size_t smem_bytes() {
     return 1024 + (size_t)n_stages<F8>() * STAGE_BYTES + sf_region_bytes<F8>() + XBUF_TOTAL + sizeof(Ctl) +
@@ -201,11 +181,13 @@ static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "sh
 static_assert(n_stages<false>() <= MAX_STAGES && n_stages<true>() <= MAX_STAGES, "ring depth");
 
 
-// Tensor maps of one expert set: weights (w1 only for the up projection) and
-// the token operand with box heights 16 * (i + 1) rows.
+// Tensor maps of one expert set: weights (w1 only for the up projection),
+// the token operand with box heights 16 * (i + 1) rows, and (E4M3) the tile
+// scales.
 struct SetMaps {
     CUtensorMap w0, w1;
     CUtensorMap x[NXBOX];
+    CUtensorMap sfw, sfx;  // E4M3: weight scale atoms (512-byte rows), token images (1024-byte rows)
 };
 
 // One expert set in a launch: set 0 = the routed experts (groups [0, G0),
@@ -219,16 +201,11 @@ struct SetParams {
     int ldo;           // output row pitch (elements)
     int f_limit;       // valid output features
     long long a_rows;  // rows the groups may index (token operand rows, or gathered rows) = output rows
-    // E4M3 operands only: tile scales.  Weights (up: W1 in wsf0, W3 in wsf1;
-    // down: W2 in wsf0) as 64-row half atoms [rows/64][k_blocks][256 B], the
-    // row of group g, feature f being g * w_rows + f.  Token operand row r:
-    // word xsf[kb * xsf_pitch + (xsf_idx ? xsf_idx[r] / xsf_div : r)] of stage kb.
-    const uint8_t* wsf0;
-    const uint8_t* wsf1;
-    const uint32_t* xsf;
-    long long xsf_pitch;
-    const int32_t* xsf_idx;
-    int xsf_div;
+    // E4M3 operands only: the tile scales come through the set's scale maps
+    // (SetMaps::sfw, sfx).  Weight atom row of the CTA's rows: up, unit
+    // (g * w_rows + f) / 64 of the joint W1/W3 units; down, atom
+    // (g * w_rows + f) / 128; row y = atom row * k_blocks + kb.  Token images:
+    // row (tile image index) * k_blocks + kb.
     // down only, weighted combine fused into the epilogue: each output row is
     // scaled by its routing weight and added (fp32 atomics) into acc [T][ldo];
     // routed set: row r holds assignment a = row_tok[r], token a / row_k,
@@ -238,11 +215,12 @@ struct SetParams {
     const float* row_w;
     int row_k;
     // up, E4M3 only, optional: h leaves as E4M3 codes q_out [rows][ldo] with
-    // token-layout tile scales q_sf (word (s, r) at q_sf[s * q_rows + r]),
-    // exactly what quantizing the bf16 h would give; out is then unused.
+    // its tile scales as the down projection's token images q_img (same
+    // tiles: image of tile i, stage s at q_img + (i * ldo / 128 + s) * 256
+    // words), exactly what quantizing the bf16 h would give; out is then
+    // unused.
     uint8_t* q_out;
-    uint32_t* q_sf;
-    long long q_rows;
+    uint32_t* q_img;
 };
 struct Params {
     const int32_t* offsets;
@@ -286,13 +264,12 @@ __device__ __forceinline__ TileCoord tile_coords(const Tables* tb, int G, int ti
 }
 
 // Token tile tt of a group with `rows` tokens split into `ntt` tiles of
-// near-equal size (<= NT each).  Equal sizes keep the clusters that share a
-// weight tile at the same pace, so the weight tile is still in L2 when the
-// slower one reads it (a small tail tile would run ahead and let L2 evict).
+// near-equal size (<= kTokTile each, token_tile_split).  Equal sizes keep the
+// clusters that share a weight tile at the same pace, so the weight tile is
+// still in L2 when the slower one reads it (a small tail tile would run ahead
+// and let L2 evict).
 __device__ __forceinline__ void token_tile(int rows, int ntt, int tt, int& start, int& len) {
-    const int q = rows / ntt, r = rows - q * ntt;
-    start = tt * q + min(tt, r);
-    len = q + (tt < r ? 1 : 0);
+    token_tile_split(rows, ntt, tt, start, len);
 }
 
 // silu(a) = a / (1 + e^-a) with the hardware exponential and division: the
@@ -463,20 +440,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
         }
         tb->rowstart[g] = rows > 0 ? rs : 0;
         tb->rows[g] = rows;
-        tb->ttiles[g] = (rows + NT - 1) / NT;
+        tb->ttiles[g] = token_tiles(rows);
         tb->fgroup[g] = UP && sh ? SHARED_FGROUP : 0;
     }
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], 1);
-        }
-        if (F8) {
-            for (int s = 0; s < SF_STAGES; ++s) {
-                mbar_init(&ctl->sf_local[s], 32);  // one completion arrive per loader lane
-                mbar_init(&ctl->sf_empty[s], 1);
-            }
-            for (int g = 0; g < SF_GROUPS; ++g) mbar_init(&ctl->sf_full[g], 2);  // the relays of both CTAs
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&ctl->tfull[a], 1);
@@ -495,19 +465,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
         tmem_relinquish_pair();
     }
     __syncthreads();
-    if (warp == 0) {  // exclusive prefix of per-group tile counts
-        int carry = 0;
+    if (warp == 0) {  // exclusive prefixes of per-group tile counts: all tiles, and the token tiles
+        int carry = 0, tcarry = 0;
         for (int b = 0; b < G; b += 32) {
             const int g = b + lane;
-            const int v = g < G ? tb->ttiles[g] * p.set[g >= p.G0 ? 1 : 0].f_tiles : 0;
-            int incl = v;
+            const int tt = g < G ? tb->ttiles[g] : 0;
+            const int v = tt * p.set[g >= p.G0 ? 1 : 0].f_tiles;
+            int incl = v, tincl = tt;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += n;
+                const int tn = __shfl_up_sync(0xffffffffu, tincl, o);
+                if (lane >= o) {
+                    incl += n;
+                    tincl += tn;
+                }
             }
-            if (g < G) tb->prefix[g] = carry + incl - v;
+            if (g < G) {
+                tb->prefix[g] = carry + incl - v;
+                tb->tbase[g] = g < p.G0 ? tcarry + tincl - tt : 0;
+            }
             carry += __shfl_sync(0xffffffffu, incl, 31);
+            tcarry += __shfl_sync(0xffffffffu, tincl, 31);
         }
         if (lane == 0) tb->prefix[G] = carry;
     }
@@ -520,8 +499,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
 
     constexpr int kTokWarp = 2 + NEPI;  // token-operand producer
     constexpr int kW3Warp = 3 + NEPI;   // up: W3-half producer
-    constexpr int kSfWarp = (UP ? 4 : 3) + NEPI;  // E4M3: tile-scale loader
-    constexpr int kSfRelay = kSfWarp + 1;         // E4M3: passes landed scale stages to the MMA issuer
+    constexpr int kSfWarp = (UP ? 4 : 3) + NEPI;  // E4M3: tile-scale producer
     const bool gather = UP && p.gather != nullptr;  // routed set only
 
     if (warp == 0) {
@@ -587,7 +565,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                 token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
                 const int half = ((ntok + 15) & ~15) >> 1;
                 const int xrows = gat ? half : (half + 15) & ~15;  // token rows a CTA loads per K step
-                const uint32_t tx = 2u * ((uint32_t)A_BYTES + (uint32_t)xrows * 128u);  // both CTAs' bytes
+                // both CTAs' bytes (E4M3: with the stage's scale slot)
+                const uint32_t tx = 2u * ((uint32_t)A_BYTES + (uint32_t)xrows * 128u + (F8 ? (uint32_t)SF_STAGE_BYTES : 0u));
                 const int k_blocks = sp.k_blocks;
                 // weight box coordinates: up, this CTA's 64 W1 rows of the tile; down, its 128
                 // W2 rows, moving to the next W2 block (d rows further) every kseg columns
@@ -695,151 +674,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
 
         __syncwarp();
     } else if (F8 && warp == kSfWarp) {
-        // ------------------------------------------------ tile-scale producer (E4M3, both CTAs)
-        // Per stage: this CTA's weight-row scale atom (two 8-byte pieces per
-        // lane, from the weights' 64-row half atoms) and the tile's token
-        // scale atoms (one 4-byte word per token, gathered through the
-        // permutation for the routed up projection), copied with cp.async
-        // into the stage's scale slot.  SF_LAG stages later, once those
-        // copies have landed (cp.async.mbarrier.arrive on sf_local), the
-        // relay warp hands them to the MMA issuer, which moves them into
-        // tensor memory.  Unused token words (rows past the tile) are zeros.
-        int stage = 0, j = 0;
-        uint32_t phase = 0, tq_ph = 0;
-        bool ok = true;
-        for (;;) {
-            int tile = -1, got = 1;
-            if (lane == 0) got = tq_take(ctl, j, tq_ph, leader_tq_empty, &tile, p.status) ? 1 : 0;
-            got = __shfl_sync(0xffffffffu, got, 0);
-            tile = __shfl_sync(0xffffffffu, tile, 0);
-            if (!got) {
-                ok = false;
-                break;
-            }
-            if (tile < 0) break;
-            if (++j == TQ) {
-                j = 0;
-                tq_ph ^= 1u;
-            }
-            const TileCoord tc = tile_coords(tb, G, tile);
-            const int si = tc.g >= p.G0 ? 1 : 0;
-            const SetParams& sp = p.set[si];
-            const int wg = si ? 0 : tc.g;
-            int tstart, ntok;
-            token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
-            const int nw = ((ntok + 15) & ~15) > 128 ? 8 : 4;  // token words per lane: the atoms the MMAs read
-            const int row0 = tb->rowstart[tc.g] + tstart;
-            long long src[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int jj = lane + 32 * i;
-                src[i] = -1;
-                if (jj < ntok) src[i] = sp.xsf_idx ? (long long)(sp.xsf_idx[row0 + jj] / sp.xsf_div) : row0 + jj;
-            }
-            const int kbn = sp.k_blocks;
-            const uint8_t* wa;
-            const uint8_t* wb;
-            uint32_t wa_n = 8u, wb_n = 8u;
-            if (UP) {  // 64 W1 rows, then the same 64 W3 rows
-                const long long R = (long long)wg * sp.w_rows + tc.ft * 128 + (int)rank * 64;
-                const size_t off = (size_t)(R >> 6) * kbn * 256 + (size_t)lane * 8;
-                wa = sp.wsf0 + off;
-                wb = sp.wsf1 + off;
-            } else {  // 128 W2 rows: two half atoms; rows past d take no scales
-                const int o0 = tc.ft * 256 + (int)rank * 128;
-                const long long R = (long long)wg * sp.w_rows + o0;
-                wa = sp.wsf0 + (size_t)(R >> 6) * kbn * 256 + (size_t)lane * 8;
-                wb = wa + (size_t)kbn * 256;
-                if (o0 >= sp.f_limit) {
-                    wa_n = 0u;
-                    wa = sp.wsf0;
-                }
-                if (o0 + 64 >= sp.f_limit) {
-                    wb_n = 0u;
-                    wb = sp.wsf0;
-                }
-            }
-            for (int kb = 0; kb < kbn; ++kb) {
-                int free_ = 1;
-                if (lane == 0) free_ = mbar_wait(&ctl->sf_empty[stage], phase ^ 1u, &ctl->abort, p.status) ? 1 : 0;
-                free_ = __shfl_sync(0xffffffffu, free_, 0);
-                if (!free_) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t slot = smem_u32(sfr + stage * SF_STAGE_BYTES);
-                cp_async_8(slot + (uint32_t)lane * 16u, wa + (wa_n ? (size_t)kb * 256 : 0), wa_n);
-                cp_async_8(slot + (uint32_t)lane * 16u + 8u, wb + (wb_n ? (size_t)kb * 256 : 0), wb_n);
-                const uint32_t* words = sp.xsf + (size_t)kb * (size_t)sp.xsf_pitch;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (i < nw) {
-                        const bool v = src[i] >= 0;
-                        cp_async_4(slot + (uint32_t)SFA_BYTES + (uint32_t)(i >> 2) * 512u + (uint32_t)lane * 16u +
-                                       (uint32_t)(i & 3) * 4u,
-                                   v ? (const void*)(words + src[i]) : (const void*)sp.xsf, v ? 4u : 0u);
-                    }
-                }
-                cp_async_mbar_arrive_noinc(&ctl->sf_local[stage]);  // fires once this lane's copies landed
-                if (++stage == SF_STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            if (!ok) break;
-        }
-        cp_async_wait<0>();
-        __syncwarp();
-    } else if (F8 && warp >= kSfRelay && warp < kSfRelay + SF_RELAYS) {
-        // ------------------------------------------------ tile-scale relay (E4M3, both CTAs, lane 0)
-        // Stages in order, counted across tiles: wait until this CTA's scale
-        // copies of the stage have landed; after every SF_GROUP stages (and
-        // after the last one) arrive on the leader's sf_full of the group
-        // (cluster-scope release; this warp has no copies of its own in
-        // flight, so the release waits for none).  Relay r takes the groups
-        // g with g % SF_RELAYS == r.
-        const int relay = warp - kSfRelay;
+        // ------------------------------------------------ tile-scale producer (E4M3, both CTAs, lane 0)
+        // Per stage, into the stage's scale slot: this CTA's weight-row atom
+        // (512 bytes) and the tile's token image (1024 bytes), onto the
+        // leader's full barrier of the stage like the operand boxes.
         if (lane == 0) {
-            const uint32_t leader_sf_full = mapa_shared(smem_u32(&ctl->sf_full[0]), 0);
-            int j = 0;
-            uint32_t tq_ph = 0;
-            long long n = 0;  // stages passed on so far
-            bool ok = true;
-            for (;;) {
-                int tile;
-                if (!tq_take(ctl, j, tq_ph, leader_tq_empty, &tile, p.status)) {
-                    ok = false;
-                    break;
-                }
-                if (++j == TQ) {
-                    j = 0;
-                    tq_ph ^= 1u;
-                }
-                if (tile < 0) break;
-                const TileCoord tc = tile_coords(tb, G, tile);
-                const int kbn = p.set[tc.g >= p.G0 ? 1 : 0].k_blocks;
-                for (int kb = 0; kb < kbn; ++kb, ++n) {
-                    if ((int)((n / SF_GROUP) % SF_RELAYS) != relay) continue;
-                    const int s = (int)(n % SF_STAGES);
-                    if (!mbar_wait(&ctl->sf_local[s], (uint32_t)((n / SF_STAGES) & 1), &ctl->abort, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    if ((n + 1) % SF_GROUP == 0)
-                        mbar_arrive_cluster(leader_sf_full + 8u * (uint32_t)((n / SF_GROUP) % SF_GROUPS));
-                }
-                if (!ok) break;
+            if (p.G0 > 0) {
+                tma_prefetch_desc(&ma.sfw);
+                tma_prefetch_desc(&ma.sfx);
             }
-            if (ok && n % SF_GROUP != 0 && (int)((n / SF_GROUP) % SF_RELAYS) == relay)  // the last, partial group
-                mbar_arrive_cluster(leader_sf_full + 8u * (uint32_t)((n / SF_GROUP) % SF_GROUPS));
+            if (p.has_shared) {
+                tma_prefetch_desc(&mb.sfw);
+                tma_prefetch_desc(&mb.sfx);
+            }
+            const CUtensorMap* wmap = nullptr;
+            const CUtensorMap* xmap = nullptr;
+            int wy = 0, xy = 0;
+            follow_tiles<STAGES, false>(
+                ctl, tb, G, leader_tq_empty, p.status, ring, lane,
+                [&](const TileCoord& tc) {
+                    const int si = tc.g >= p.G0 ? 1 : 0;
+                    const SetParams& sp = p.set[si];
+                    wmap = &(si ? mb : ma).sfw;
+                    xmap = &(si ? mb : ma).sfx;
+                    const int wg = si ? 0 : tc.g;
+                    const long long f0 = UP ? (long long)wg * sp.w_rows + tc.ft * 128 + (int)rank * 64
+                                            : (long long)wg * sp.w_rows + tc.ft * 256 + (int)rank * 128;
+                    wy = (int)((UP ? f0 >> 6 : f0 >> 7) * sp.k_blocks);
+                    xy = ((si ? 0 : tb->tbase[tc.g]) + tc.tt) * sp.k_blocks;
+                    return sp.k_blocks;
+                },
+                [&](int kb, uint8_t* stage, uint32_t fb) {
+                    uint8_t* slot = sfr + (size_t)((stage - ring) / STAGE_BYTES) * SF_STAGE_BYTES;
+                    tma_load_2d_pair(slot, wmap, fb, 0, wy + kb, W_HINT);
+                    tma_load_2d_pair(slot + SFA_BYTES, xmap, fb, 0, xy + kb, X_HINT);
+                });
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (leader CTA only)
         if (rank == 0 && elect_one()) {
             int stage = 0, acc = 1, j = 0;  // acc: the previous tile's accumulator
-            int sfs = 0;                    // E4M3: scale ring slot
-            long long sfn = 0;              // E4M3: scale stages consumed
             uint32_t phase = 0, tq_ph = 0;
             uint32_t acc_ph = 0u;  // bit a: phase of accumulator a
             bool ok = true;
@@ -872,13 +747,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                         ok = false;
                         break;
                     }
-                    // E4M3: the relays of both CTAs pass the scales on in groups of SF_GROUP stages
-                    if (F8 && sfn % SF_GROUP == 0 &&
-                        !mbar_wait_cluster(&ctl->sf_full[(sfn / SF_GROUP) % SF_GROUPS],
-                                           (uint32_t)((sfn / SF_STAGES) & 1), &ctl->abort, p.status)) {
-                        ok = false;
-                        break;
-                    }
                     tc_fence_after();
                     uint8_t* sa = ring + stage * STAGE_BYTES;
                     const uint64_t ad = smem_desc_sw128(smem_u32(sa));
@@ -887,7 +755,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                         // the stage's tile scales into tensor memory (one slot, reused every stage: the
                         // copies and MMAs of this thread execute in issue order), then 4 MMAs of K = 32,
                         // each reading byte kk of its rows' scale words
-                        const uint32_t sfa = smem_u32(sfr + sfs * SF_STAGE_BYTES);
+                        const uint32_t sfa = smem_u32(sfr + stage * SF_STAGE_BYTES);
                         tc_cp_32x128b_x4_pair(tmem_base + SFA_COL, smem_desc_plain(sfa));
                         tc_cp_32x128b_x4_pair(tmem_base + SFB_COL, smem_desc_plain(sfa + SFA_BYTES));
                         if (n_mma > 128)
@@ -905,11 +773,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                                              (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit_pair(&ctl->empty[stage], 0x3);
-                    if (F8) {
-                        tc_commit_pair(&ctl->sf_empty[sfs], 0x3);
-                        ++sfn;
-                        if (++sfs == SF_STAGES) sfs = 0;
-                    }
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -953,6 +816,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
             int tstart, ntok;
             token_tile(tb->rows[tc.g], tb->ttiles[tc.g], tc.tt, tstart, ntok);
             const int tok0 = tb->rowstart[tc.g] + tstart;
+            const int qimg = (tc.g >= p.G0 ? 0 : tb->tbase[tc.g]) + tc.tt;  // E4M3 h: the tile's scale image
             // first output feature of this CTA
             const int fcta = UP ? tc.ft * 128 + (int)rank * 64 : tc.ft * 256 + (int)rank * 128;
             acc = next_acc<F8>(acc, (ntok + 15) & ~15);
@@ -1009,10 +873,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                             const uint32_t c1 = e4m3x2(__fmul_rn(hv[4], mul), __fmul_rn(hv[5], mul)) |
                                                 (e4m3x2(__fmul_rn(hv[6], mul), __fmul_rn(hv[7], mul)) << 16);
                             *reinterpret_cast<uint2*>(sp.q_out + orow * sp.ldo + fcta + fj) = make_uint2(c0, c1);
-                            if (part == 0) {  // tiles fcta / 32 and the next: bytes j, j + 1 of the stage word
-                                uint8_t* wd = reinterpret_cast<uint8_t*>(sp.q_sf + (size_t)(fcta >> 7) * sp.q_rows + orow);
-                                *reinterpret_cast<uint16_t*>(wd + ((fcta & 127) >> 5)) = (uint16_t)(sbyte | (sother << 8));
-                            }
+                        }
+                        if (part == 0) {  // tiles fcta / 32 and the next: bytes j, j + 1 of the token's stage word
+                            // (tokens of the last chunk past the tile get scale 1: the down MMA's padding columns)
+                            uint8_t* wd = reinterpret_cast<uint8_t*>(
+                                sp.q_img + ((size_t)qimg * (size_t)(sp.ldo >> 7) + (size_t)(fcta >> 7)) * 256u +
+                                tile_image_word(c + my_tok));
+                            *reinterpret_cast<uint16_t*>(wd + ((fcta & 127) >> 5)) = (uint16_t)(sbyte | (sother << 8));
                         }
                     } else if (tok_ok) {
                         uint4 v;
@@ -1104,18 +971,15 @@ bool up_set(const TcUpArgs& a, SetMaps& m, SetParams& sp) {
     const unsigned eb = a.f8 ? 1 : 2;
     const int bke = 128 / (int)eb;
     if (a.d % bke != 0 || a.I % 128 != 0) return false;
-    if (a.f8 && (!a.w1s || !a.w3s || !a.xs || a.d % 128 != 0)) return false;
+    if (a.f8 && (!a.w13s || !a.xs || a.xs_tiles <= 0 || a.d % 128 != 0 || a.W_rows % 64 != 0)) return false;
     if (!make_tmap_2d(&m.w0, a.W1, a.d, a.W_rows, a.d, bke, 64, eb) ||
         !make_tmap_2d(&m.w1, a.W3, a.d, a.W_rows, a.d, bke, 64, eb) || !token_maps(m, a.A, a.d, a.A_rows, eb))
         return false;
     sp.f_tiles = a.I / 128;
     sp.k_blocks = a.d / bke;
-    sp.wsf0 = a.w1s;
-    sp.wsf1 = a.w3s;
-    sp.xsf = a.xs;
-    sp.xsf_pitch = a.xs_pitch;
-    sp.xsf_idx = a.xs_idx;
-    sp.xsf_div = a.xs_div > 0 ? a.xs_div : 1;
+    if (a.f8 && (!make_tmap_rows_u32(&m.sfw, a.w13s, SFA_BYTES / 4, (unsigned long long)(a.W_rows / 64) * sp.k_blocks) ||
+                 !make_tmap_rows_u32(&m.sfx, a.xs, SFB_BYTES / 4, (unsigned long long)a.xs_tiles * sp.k_blocks)))
+        return false;
     sp.w_rows = a.I;
     sp.kseg = a.d;
     sp.nseg = 1;
@@ -1124,9 +988,8 @@ bool up_set(const TcUpArgs& a, SetMaps& m, SetParams& sp) {
     sp.f_limit = a.I;
     sp.a_rows = a.gather ? a.gather_rows : a.A_rows;
     sp.q_out = a.f8 ? a.hq : nullptr;
-    sp.q_sf = a.f8 ? a.hq_sf : nullptr;
-    sp.q_rows = a.A_rows;
-    if (sp.q_out && !sp.q_sf) return false;
+    sp.q_img = a.f8 ? a.hq_img : nullptr;
+    if (sp.q_out && !sp.q_img) return false;
     return true;
 }
 
@@ -1134,7 +997,8 @@ bool down_set(const TcDownArgs& a, SetMaps& m, SetParams& sp) {
     const unsigned eb = a.f8 ? 1 : 2;
     const int bke = 128 / (int)eb;
     if (a.K % bke != 0 || a.kseg % bke != 0 || a.d % 16 != 0) return false;
-    if (a.f8 && (!a.w2s || !a.hs || a.K % 128 != 0 || a.kseg % 128 != 0 || a.d % 64 != 0)) return false;
+    if (a.f8 && (!a.w2s || !a.hs || a.hs_tiles <= 0 || a.K % 128 != 0 || a.kseg % 128 != 0 || a.d % 128 != 0))
+        return false;
     // W2 blocks [G * nseg][d][kseg] viewed as one matrix of G * nseg * d rows: a 2D map fed
     // the down projection ~10% faster than the same boxes through a 3D map.  Rows past d of
     // a feature tile read the next block's rows (or zero past the end); their outputs are
@@ -1145,12 +1009,9 @@ bool down_set(const TcDownArgs& a, SetMaps& m, SetParams& sp) {
     m.w1 = m.w0;
     sp.f_tiles = (a.d + 255) / 256;
     sp.k_blocks = a.K / bke;
-    sp.wsf0 = a.w2s;
-    sp.wsf1 = nullptr;
-    sp.xsf = a.hs;
-    sp.xsf_pitch = a.H_rows;
-    sp.xsf_idx = nullptr;
-    sp.xsf_div = 1;
+    if (a.f8 && (!make_tmap_rows_u32(&m.sfw, a.w2s, SFA_BYTES / 4, (unsigned long long)a.G * a.d / 128 * sp.k_blocks) ||
+                 !make_tmap_rows_u32(&m.sfx, a.hs, SFB_BYTES / 4, (unsigned long long)a.hs_tiles * sp.k_blocks)))
+        return false;
     sp.acc = a.acc;
     sp.row_tok = a.row_tok;
     sp.row_w = a.row_w;

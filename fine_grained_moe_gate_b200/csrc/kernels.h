@@ -41,12 +41,19 @@ struct GemmArgs {
 };
 
 // quant.cu: per-tile E4M3 quantization (scale layouts described there)
-// out [K/128][T*k] words = the token-layout scales xs [K/128][T] of the rows of a permutation (row r: token perm[r] / k).
-cudaError_t launch_permute_mx_scales(const void* xs, const int32_t* perm, int k, long long T, int K, void* out,
-                                     int* status, cudaStream_t st);
-size_t mx_scale_bytes(long long rows, int K, bool weight_layout);
-cudaError_t launch_quantize_mx(const void* src, long long rows, int kseg, int nseg, bool weight_layout, uint8_t* q,
+enum MxLayout { kMxTokens = 0, kMxWeights = 1, kMxGate = 2, kMxUp = 3 };
+size_t mx_scale_bytes(long long rows, int K, int layout);
+cudaError_t launch_quantize_mx(const void* src, long long rows, int kseg, int nseg, int layout, uint8_t* q,
                                void* scales, cudaStream_t st);
+// Token images of the grouped GEMMs' tiles: groups [offsets[g], offsets[g+1])
+// (offsets null: one group of `rows` rows); tile images in group order, row
+// j of a tile taking the token-layout words of src row row_of[r] / row_div
+// (row_of null: r itself) of src [K/128][src_rows].  max_tiles bounds the
+// images written (mx_tile_images).
+long long mx_tile_images(long long rows, int groups);
+cudaError_t launch_tile_scales(const void* src, long long src_rows, int K, const int32_t* row_of, int row_div,
+                               const int32_t* offsets, int groups, long long rows, void* out, int* status,
+                               cudaStream_t st);
 
 // combine.cu: y = dtype(acc) for n elements (n % 8 == 0), then acc = 0
 cudaError_t launch_combine_finish(float* acc, long long n, bool bf16, void* y, cudaStream_t st);
@@ -154,20 +161,19 @@ struct TcUpArgs {
     const int32_t* offsets; // group rows; null: one group of M rows
     int G, M;
     // E4M3 operands (A, W1, W3 one byte per element) with per-tile scales
-    // (quant.cu layouts): w1s / w3s the weights' 64-row half atoms; token
-    // row r's scale words xs[s * xs_pitch + (xs_idx ? xs_idx[r] / xs_div : r)]
-    // for stage s (128 columns).
+    // (quant.cu layouts): w13s the joint W1/W3 scale units ([W_rows / 64][d /
+    // 128] x 512 bytes); xs the token images of the groups' tiles ([xs_tiles][d
+    // / 128] x 1024 bytes, image i for the i-th token tile over the groups in
+    // order).
     bool f8 = false;
-    const uint8_t* w1s = nullptr;
-    const uint8_t* w3s = nullptr;
+    const uint8_t* w13s = nullptr;
     const uint32_t* xs = nullptr;
-    long long xs_pitch = 0;
-    const int32_t* xs_idx = nullptr;
-    int xs_div = 1;
-    // E4M3, optional: write h as E4M3 codes hq [A_rows][I] with token-layout
-    // tile scales hq_sf ([I/128][A_rows] words) instead of bf16 H.
+    long long xs_tiles = 0;
+    // E4M3, optional: write h as E4M3 codes hq [A_rows][I] with its tile
+    // scales as the down projection's token images hq_img ([tiles][I / 128] x
+    // 1024 bytes, the same tiles) instead of bf16 H.
     uint8_t* hq = nullptr;
-    uint32_t* hq_sf = nullptr;
+    uint32_t* hq_img = nullptr;
 };
 // Down projection: Y[r][:] = H[r] . W2_g^T, W2_g = [d][K] (K = I), or for
 // the shared group S stacked [d][Is] blocks contracted over K = S * Is.
@@ -181,12 +187,14 @@ struct TcDownArgs {
     int d, K;
     const int32_t* offsets;
     int G, M;
-    // E4M3 operands (H, W2 one byte per element) with per-tile scales:
-    // w2s the half atoms of W2 as [G * d] rows of K = nseg * kseg columns;
-    // hs the scale words of H, [K / 128][H_rows].
+    // E4M3 operands (H, W2 one byte per element) with per-tile scales: w2s
+    // the 128-row atoms of W2 as [G * d] rows of K = nseg * kseg columns
+    // ([G * d / 128][K / 128] x 512 bytes); hs the token images of H's tiles
+    // ([hs_tiles][K / 128] x 1024 bytes).
     bool f8 = false;
     const uint8_t* w2s = nullptr;
     const uint32_t* hs = nullptr;
+    long long hs_tiles = 0;
     // Weighted combine fused into the epilogue (acc non-null): Y is not
     // written; row r is scaled and added into acc [T][d] fp32 -- routed:
     // token row_tok[r] / row_k, weight row_w[row_tok[r]]; shared (row_tok

@@ -13,17 +13,20 @@
 // e comes from the bits of amax (mx_tile_exponent, common.cuh); an all-zero
 // tile gets e = 0 and codes 0.
 //
-// Scale layouts (the GEMMs' shared-memory scale atoms hold, for 128 operand
-// rows and one 128-column stage, the byte of row m, tile j at
-// (m % 32) * 16 + (m / 32) * 4 + j):
+// Scale layouts (the GEMMs' scale atoms hold, for 128 operand rows and one
+// 128-column stage, the byte of row m, tile j at (m % 32) * 16 + (m / 32) * 4
+// + j: the order the tensor-memory scale copy reads them):
 //   tokens:  uint32 [K/128][rows]: word (s, r) holds the 4 tile bytes of row
-//            r's stage s (byte j = tile 4s + j).  A stage's words of
-//            consecutive rows are contiguous, so a warp fetches 32 rows' with
-//            one coalesced load, or gathers them by token index.
-//   weights: 64-row half atoms of 256 bytes, [rows/64][K/128][32][8]: byte
-//            (m % 32) * 8 + (m / 32) * 4 + j of half atom (r / 64, s), m =
-//            r % 64.  A lane of the GEMM's scale warp copies 8 bytes per half
-//            atom into the 16-byte row of the atom it builds.
+//            r's stage s (byte j = tile 4s + j).
+//   weights: 512-byte atoms [rows/128][K/128], row r at m = r % 128 of atom
+//            (r / 128, s): the down projection's A rows, one atom per stage.
+//   gate/up: W1 and W3 in one buffer of 512-byte units [rows/64][K/128];
+//            row r of W1 at m = r % 64 of unit (r / 64, s), row r of W3 at
+//            m = 64 + r % 64: the gate/up A rows of a CTA (64 W1 rows, then
+//            the same 64 W3 rows), one unit per stage.
+//   token images (per tile of the grouped GEMMs, launch_tile_scales): 256
+//            words per tile and stage, word tile_image_word(j) for the tile's
+//            row j, zero past its rows.
 // A matrix with `rows` rows may be stored as nseg column blocks of kseg
 // columns ([nseg][rows][kseg], stacked experts joined along the
 // contraction); its rows and tiles span all blocks.  One warp per row, one
@@ -48,7 +51,7 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 
-template <bool kWeightLayout>
+template <int kLayout>
 __global__ void __launch_bounds__(kWarps * 32) quantize_mx_kernel(const uint16_t* __restrict__ src, long long rows,
                                                                  int kseg, int nseg, uint8_t* __restrict__ q,
                                                                  uint8_t* __restrict__ sf) {
@@ -93,69 +96,122 @@ __global__ void __launch_bounds__(kWarps * 32) quantize_mx_kernel(const uint16_t
         if (act && (lane & 15) == 0) {
             const uint32_t word = byte | (b1 << 8) | (b2 << 16) | (b3 << 24);
             const int s = c >> 7;
-            if (kWeightLayout) {
-                const size_t atom = ((size_t)(r >> 6) * nst + s) * 256;
-                const int m = (int)(r & 63);
-                *reinterpret_cast<uint32_t*>(sf + atom + (m & 31) * 8 + (m >> 5) * 4) = word;
-            } else {
+            if (kLayout == kMxTokens) {
                 reinterpret_cast<uint32_t*>(sf)[(size_t)s * rows + r] = word;
+            } else {
+                const int sh = kLayout == kMxWeights ? 7 : 6;  // rows per atom: 128, or 64 of each matrix
+                const int m = (int)(r & ((1 << sh) - 1)) + (kLayout == kMxUp ? 64 : 0);
+                const size_t atom = ((size_t)(r >> sh) * nst + s) * 512;
+                *reinterpret_cast<uint32_t*>(sf + atom + (m & 31) * 16 + (m >> 5) * 4) = word;
             }
         }
     }
 }
 
-// Token-layout scale words of the rows of a permutation: out[s][r] =
-// xs[s][perm[r] / k] (row r of xq_perm holds token perm[r] / k), so that the
-// GEMM reads a stage's words of consecutive rows with coalesced loads.
-__global__ void permute_mx_scales_kernel(const uint32_t* __restrict__ xs, const int32_t* __restrict__ perm, int k,
-                                         long long T, long long rows, int nst, uint32_t* __restrict__ out,
-                                         int* status) {
-    const long long n = rows * nst;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-        const int s = (int)(i / rows);
-        const long long r = i - (long long)s * rows;
-        const long long t = perm[r] / k;
-        if (t < 0 || t >= T) {
-            report(status, kStDeviceCheck);
-            continue;
-        }
-        out[i] = xs[(size_t)s * T + t];
+// Token images of the tiles of a grouped GEMM (one block per image): the
+// block finds its group and token tile from the group sizes (the GEMMs'
+// split, token_tile_split), then writes the tile's 256-word image of every
+// stage.  Blocks past the last tile clear their slot, so the whole buffer is
+// written.
+__global__ void __launch_bounds__(256) tile_scales_kernel(const uint32_t* __restrict__ src, long long src_rows,
+                                                          int nst, const int32_t* __restrict__ row_of, int row_div,
+                                                          const int32_t* __restrict__ offsets, int G, long long rows,
+                                                          uint32_t* __restrict__ out, int* status) {
+    __shared__ int s_first[kMaxGroups + 1];  // first image of each group
+    __shared__ int s_g;
+    const int tid = threadIdx.x;
+    // tile counts, then an exclusive scan over the groups (one warp)
+    for (int g = tid; g < G; g += blockDim.x) {
+        const long long n = offsets ? (long long)offsets[g + 1] - offsets[g] : rows;
+        s_first[g] = n > 0 ? token_tiles((int)n) : 0;
     }
+    __syncthreads();
+    if (tid < 32) {
+        int carry = 0;
+        for (int b = 0; b < G; b += 32) {
+            const int g = b + tid;
+            const int v = g < G ? s_first[g] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (tid >= o) incl += n;
+            }
+            if (g < G) s_first[g] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (tid == 0) s_first[G] = carry;
+    }
+    __syncthreads();
+    const int img = blockIdx.x;
+    if (img >= s_first[G]) {  // block-uniform: an image slot past the last tile is cleared
+        for (int s = 0; s < nst; ++s) out[((size_t)img * nst + s) * 256 + tid] = 0u;
+        return;
+    }
+    for (int g = tid; g < G; g += blockDim.x)
+        if (s_first[g] <= img && img < s_first[g + 1]) s_g = g;
+    __syncthreads();
+    const int g = s_g;
+    const long long r0 = offsets ? offsets[g] : 0;
+    const int n = (int)(offsets ? (long long)offsets[g + 1] - r0 : rows);
+    int start, len;
+    token_tile_split(n, s_first[g + 1] - s_first[g], img - s_first[g], start, len);
+    const int j = tid;
+    long long sr = -1;
+    if (j < len) {
+        const long long r = r0 + start + j;
+        if (r >= 0 && r < rows) sr = row_of ? (long long)row_of[r] / row_div : r;
+        if (sr < 0 || sr >= src_rows) {  // rows outside the operand, or a row index outside src
+            report(status, kStDeviceCheck);
+            sr = -1;
+        }
+    }
+    uint32_t* dst = out + (size_t)img * nst * 256 + tile_image_word(j);
+    for (int s = 0; s < nst; ++s) dst[(size_t)s * 256] = sr >= 0 ? src[(size_t)s * src_rows + sr] : 0u;
 }
 
 }  // namespace
 
-cudaError_t launch_permute_mx_scales(const void* xs, const int32_t* perm, int k, long long T, int K, void* out,
-                                     int* status, cudaStream_t st) {
-    const long long rows = T * k;
+long long mx_tile_images(long long rows, int groups) { return rows / kTokTile + groups; }
+
+cudaError_t launch_tile_scales(const void* src, long long src_rows, int K, const int32_t* row_of, int row_div,
+                               const int32_t* offsets, int groups, long long rows, void* out, int* status,
+                               cudaStream_t st) {
     const int nst = K / 128;
-    if (rows <= 0 || nst <= 0) return cudaSuccess;
-    const long long n = rows * nst;
-    long long blocks = (n + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
-    permute_mx_scales_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint32_t*>(xs), perm, k, T, rows, nst,
-                                                               static_cast<uint32_t*>(out), status);
+    if (rows <= 0 || nst <= 0 || groups <= 0) return cudaSuccess;
+    if (groups > kMaxGroups) return cudaErrorInvalidValue;
+    const long long blocks = mx_tile_images(rows, groups);
+    if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
+    tile_scales_kernel<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const uint32_t*>(src), src_rows, nst, row_of,
+                                                        row_div > 0 ? row_div : 1, offsets, groups, rows,
+                                                        static_cast<uint32_t*>(out), status);
     note_launches(1);
     return cudaGetLastError();
 }
 
-size_t mx_scale_bytes(long long rows, int K, bool weight_layout) {
+size_t mx_scale_bytes(long long rows, int K, int layout) {
     const size_t nst = (size_t)(K / 128);
-    if (weight_layout) return (size_t)((rows + 63) / 64) * nst * 256;
+    if (layout == kMxWeights) return (size_t)((rows + 127) / 128) * nst * 512;
+    if (layout == kMxGate || layout == kMxUp) return (size_t)((rows + 63) / 64) * nst * 512;
     return (size_t)rows * nst * 4;
 }
 
-cudaError_t launch_quantize_mx(const void* src, long long rows, int kseg, int nseg, bool weight_layout, uint8_t* q,
+cudaError_t launch_quantize_mx(const void* src, long long rows, int kseg, int nseg, int layout, uint8_t* q,
                                void* scales, cudaStream_t st) {
     if (rows <= 0) return cudaSuccess;
     const long long blocks = (rows + kWarps - 1) / kWarps;
     if (blocks > 0x7fffffffll) return cudaErrorInvalidValue;
     const auto* s = static_cast<const uint16_t*>(src);
     auto* sf = static_cast<uint8_t*>(scales);
-    if (weight_layout)
-        quantize_mx_kernel<true><<<(unsigned)blocks, kWarps * 32, 0, st>>>(s, rows, kseg, nseg, q, sf);
-    else
-        quantize_mx_kernel<false><<<(unsigned)blocks, kWarps * 32, 0, st>>>(s, rows, kseg, nseg, q, sf);
+    const unsigned nb = (unsigned)blocks;
+    constexpr int nt = kWarps * 32;
+    switch (layout) {
+        case kMxTokens: quantize_mx_kernel<kMxTokens><<<nb, nt, 0, st>>>(s, rows, kseg, nseg, q, sf); break;
+        case kMxWeights: quantize_mx_kernel<kMxWeights><<<nb, nt, 0, st>>>(s, rows, kseg, nseg, q, sf); break;
+        case kMxGate: quantize_mx_kernel<kMxGate><<<nb, nt, 0, st>>>(s, rows, kseg, nseg, q, sf); break;
+        case kMxUp: quantize_mx_kernel<kMxUp><<<nb, nt, 0, st>>>(s, rows, kseg, nseg, q, sf); break;
+        default: return cudaErrorInvalidValue;
+    }
     note_launches(1);
     return cudaGetLastError();
 }

@@ -48,6 +48,21 @@ inline bool make_tmap_2d(CUtensorMap* m, const void* base, unsigned long long co
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// rank-2 map over `rows` rows of `words` 32-bit words each (contiguous), one
+// row per box, no swizzle: the E4M3 scale atoms and token images (512 or
+// 1024 bytes), copied as they lie.  Out-of-bounds rows fill 0.
+inline bool make_tmap_rows_u32(CUtensorMap* m, const void* base, unsigned words, unsigned long long rows) {
+    auto enc = tmap_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {words, rows};
+    cuuint64_t strides[1] = {(cuuint64_t)words * 4};
+    cuuint32_t box[2] = {words, 1};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // rank-3 fp32 map for tiled stores: [planes][rows][cols] with row pitch
 // `ld` and plane pitch `plane` elements; box = box_cols (innermost, 32
 // floats = 128 bytes, 128-byte swizzle) x box_rows x 1.

@@ -331,16 +331,31 @@ MOE_API size_t moe_backward_workspace_size(moe_shape sh, int32_t seq_len);
  *   MOE_SF_TOKENS  token rows and h: uint32 [K/128][rows]; word (s, r) holds
  *                  the four tile bytes of row r's columns [128 s, 128 s + 128)
  *                  (byte j = tile 4 s + j).
- *   MOE_SF_WEIGHTS expert weights: 256-byte units, one per 64 rows and 128
- *                  columns, [rows/64][K/128]; byte (m % 32) * 8 + (m / 32) * 4
- *                  + j of unit (r / 64, s) is tile 4 s + j of row r, m = r % 64.
- *                  This is the order the GEMMs assemble their tensor-memory
- *                  scale blocks from; treat it as opaque otherwise.
+ *   MOE_SF_WEIGHTS W2 and Ws2: 512-byte atoms, one per 128 rows and 128
+ *                  columns, [rows/128][K/128]; byte (m % 32) * 16 + (m / 32) *
+ *                  4 + j of atom (r / 128, s) is tile 4 s + j of row r, m =
+ *                  r % 128.
+ *   MOE_SF_GATE,   W1 and W3 (Ws1 and Ws3) share ONE buffer of 512-byte
+ *   MOE_SF_UP      units, one per 64 rows and 128 columns, [rows/64][K/128];
+ *                  byte (m % 32) * 16 + (m / 32) * 4 + j of unit (r / 64, s)
+ *                  is tile 4 s + j of row r of W1 (MOE_SF_GATE, m = r % 64)
+ *                  or of W3 (MOE_SF_UP, m = 64 + r % 64): quantize W1 with
+ *                  MOE_SF_GATE and W3 with MOE_SF_UP into the same buffer.
+ * These are the orders in which the GEMMs copy the scales of 128 operand rows
+ * into tensor memory; treat them as opaque otherwise.
+ *
+ * Token tile images (moe_fp8_tile_scales): the grouped GEMMs run each group
+ * of n rows as ceil(n / 256) token tiles of near-equal size (tile t has q +
+ * (t < r) rows, q = n / tiles, r = n % tiles) and read the token scales of a
+ * tile as one image of 256 uint32 words per 128 columns: [tiles][K/128][256],
+ * the tiles of all groups in order; the word of the tile's row j sits at
+ * (j / 128) * 128 + (j % 32) * 4 + (j / 32) % 4, zeros past its rows.
  * -------------------------------------------------------------------------*/
-typedef enum { MOE_SF_TOKENS = 0, MOE_SF_WEIGHTS = 1 } moe_sf_layout;
+typedef enum { MOE_SF_TOKENS = 0, MOE_SF_WEIGHTS = 1, MOE_SF_GATE = 2, MOE_SF_UP = 3 } moe_sf_layout;
 
 /* Bytes of the tile scales of a matrix of `rows` rows and K columns in the
- * given layout (0 if K % 128 != 0 or the layout is unknown). */
+ * given layout (0 if K % 128 != 0 or the layout is unknown; MOE_SF_GATE and
+ * MOE_SF_UP give the size of the joint buffer). */
 MOE_API size_t moe_fp8_scale_bytes(int64_t rows, int32_t K, int32_t layout);
 
 /* moe_quantize_fp8 -- per-tile E4M3 quantization of a bf16 matrix with
@@ -348,71 +363,79 @@ MOE_API size_t moe_fp8_scale_bytes(int64_t rows, int32_t K, int32_t layout);
  * nseg = 1 is plain row major; a row and its tiles span all blocks, K =
  * nseg * kseg).  q has src's layout, one byte per element; scales in
  * `layout`.  Needs kseg % 128 == 0; src, q and scales 16-byte aligned.
- * Used once per weight tensor (MOE_SF_WEIGHTS: W1/W3 [E][I][d] as rows = E*I;
- * W2 [E][d][I] as rows = E*d, kseg = I; the shared Ws1/Ws3 [S][Is][d] as rows =
- * S*Is; Ws2 [S][d][Is] as rows = d, kseg = Is, nseg = S) and per step for the
- * token rows and h (MOE_SF_TOKENS). */
+ * Used once per weight tensor (W1 / W3 [E][I][d] as rows = E*I with
+ * MOE_SF_GATE / MOE_SF_UP into one buffer; W2 [E][d][I] as rows = E*d, kseg =
+ * I, MOE_SF_WEIGHTS; the shared Ws1 / Ws3 [S][Is][d] as rows = S*Is likewise;
+ * Ws2 [S][d][Is] as rows = d, kseg = Is, nseg = S) and per step for the token
+ * rows and h (MOE_SF_TOKENS). */
 MOE_API moe_status moe_quantize_fp8(const void* src, int64_t rows, int32_t kseg, int32_t nseg, int32_t layout,
                                     uint8_t* q, void* scales, void* stream);
 
-/* E4M3 expert weights and their tile scales (MOE_SF_WEIGHTS), all device
- * pointers, 16-byte aligned. */
+/* Bytes of the token tile images of `rows` operand rows in `groups` groups
+ * (1 <= groups <= 256) with K columns: room for rows / 256 + groups tiles. */
+MOE_API size_t moe_fp8_tile_scale_bytes(int64_t rows, int32_t groups, int32_t K);
+
+/* moe_fp8_tile_scales -- the token tile images of a grouped GEMM's token
+ * operand of `rows` rows: groups [offsets[g], offsets[g+1]) (offsets NULL:
+ * one group of all rows, groups = 1); operand row r takes the MOE_SF_TOKENS
+ * words of row row_of[r] / row_div of src [K/128][src_rows] (row_of NULL:
+ * row r).  Routed gate/up: src = the tokens' scales [d/128][T], row_of =
+ * perm_tok, row_div = k, offsets from moe_permute, groups = E, rows = T*k;
+ * shared experts: offsets NULL, rows = T; down from moe_quantize_fp8's h
+ * scales: row_of NULL.  tiles: moe_fp8_tile_scale_bytes(rows, groups, K)
+ * bytes, all of it written.  Pointers 16-byte aligned.  A row outside
+ * [0, rows) or a source row outside src reports MOE_ERR_DEVICE_CHECK (its
+ * word is left 0). */
+MOE_API moe_status moe_fp8_tile_scales(const void* src, int64_t src_rows, int32_t K, const int32_t* row_of,
+                                       int32_t row_div, const int32_t* offsets, int32_t groups, int64_t rows,
+                                       void* tiles, void* stream);
+
+/* E4M3 expert weights and their tile scales, all device pointers, 16-byte
+ * aligned. */
 typedef struct {
-    const uint8_t* w1;  const void* w1_scale;   /* [E][I][d]   rows E*I, K = d  */
-    const uint8_t* w3;  const void* w3_scale;   /* [E][I][d]   rows E*I, K = d  */
-    const uint8_t* w2;  const void* w2_scale;   /* [E][d][I]   rows E*d, K = I  */
-    const uint8_t* ws1; const void* ws1_scale;  /* [S][Is][d]  rows S*Is, K = d (NULL if S == 0) */
-    const uint8_t* ws3; const void* ws3_scale;  /* [S][Is][d]  rows S*Is, K = d */
-    const uint8_t* ws2; const void* ws2_scale;  /* [S][d][Is]  rows d, K = S*Is (the S blocks joined) */
+    const uint8_t* w1;  const uint8_t* w3;  const void* w13_scale;    /* [E][I][d] each, rows E*I, K = d;
+                                                                        MOE_SF_GATE / MOE_SF_UP, one buffer */
+    const uint8_t* w2;  const void* w2_scale;                         /* [E][d][I] rows E*d, K = I; MOE_SF_WEIGHTS */
+    const uint8_t* ws1; const uint8_t* ws3; const void* ws13_scale;   /* [S][Is][d], rows S*Is, K = d (NULL if S == 0) */
+    const uint8_t* ws2; const void* ws2_scale;                        /* [S][d][Is] rows d, K = S*Is (blocks joined) */
 } moe_fp8_experts;
 
-/* moe_ffn_up_fp8 / moe_ffn_down_fp8 -- moe_ffn_up / moe_ffn_down on E4M3
- * operands (sh.dtype == MOE_FP8_E4M3), routed and shared experts in one
- * launch each.
- *   up:   xq_perm [T*k][d] E4M3 token rows in expert order (moe_permute of
- *         xq), perm_tok from moe_permute, x_scales the tile scales of the
- *         unpermuted tokens (MOE_SF_TOKENS, [d/128][T]; row r of xq_perm uses
- *         token perm_tok[r] / k's); xq [T][d] the unpermuted quantized tokens
- *         (shared experts; NULL leaves them out).  h = bf16(silu(a) * g) with
- *         a, g the tile-scaled sums [T*k][I]; hs likewise [T][S*Is].
- *   down: hq [T*k][I] E4M3 with h_scales [I/128][T*k] (moe_quantize_fp8 of
- *         h), hsq [T][S*Is] with hs_scales [S*Is/128][T] (NULL leaves the
- *         shared set out); y_perm [T*k][d] and shared_out [T][d] in bf16. */
-MOE_API moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const int32_t* perm_tok, const void* x_scales,
-                                  const int32_t* offsets, const uint8_t* xq, const moe_fp8_experts* w, moe_shape sh,
+/* moe_ffn_up_fp8 / moe_ffn_up_fp8_quant / moe_ffn_down_fp8 -- moe_ffn_up /
+ * moe_ffn_down on E4M3 operands (sh.dtype == MOE_FP8_E4M3), routed and shared
+ * experts in one launch each.  Token scales come as tile images
+ * (moe_fp8_tile_scales) of the same offsets:
+ *   up:    xq_perm [T*k][d] E4M3 token rows in expert order (moe_permute of
+ *          xq) with x_tiles; xq [T][d] the unpermuted quantized tokens with
+ *          xsh_tiles (shared experts; xq NULL leaves them out).  h =
+ *          bf16(silu(a) * g) with a, g the tile-scaled sums [T*k][I]; hs
+ *          likewise [T][S*Is].
+ *   quant: the same launch with h and hs leaving it quantized for the down
+ *          projection: the epilogue rounds h to bf16 as moe_ffn_up_fp8 writes
+ *          it, then quantizes each 1x32 tile as moe_quantize_fp8 does, so hq
+ *          [T*k][I] / hsq [T][S*Is] equal the codes of that h, and h_tiles /
+ *          hs_tiles its scales as tile images (equal to moe_fp8_tile_scales of
+ *          moe_quantize_fp8's scales at every tile row; rows past a tile up to
+ *          a multiple of 16 hold scale byte 127, the rest is not written),
+ *          without the bf16 h round trip through HBM.
+ *   down:  hq [T*k][I] with h_tiles, hsq [T][S*Is] with hs_tiles (NULL leaves
+ *          the shared set out); y_perm [T*k][d] and shared_out [T][d] bf16.
+ * Image buffers: moe_fp8_tile_scale_bytes(T*k, E, K) (routed) and (T, 1, K)
+ * (shared).  Pointers 16-byte aligned. */
+MOE_API moe_status moe_ffn_up_fp8(const uint8_t* xq_perm, const void* x_tiles, const int32_t* offsets,
+                                  const uint8_t* xq, const void* xsh_tiles, const moe_fp8_experts* w, moe_shape sh,
                                   void* h, void* hs, void* stream);
-/* moe_permute_fp8_scales -- the token-layout tile scales of the permuted
- * rows: xs_perm [d/128][T*k] 32-bit words with word (s, r) = word (s,
- * perm_tok[r] / k) of x_scales [d/128][T] (MOE_SF_TOKENS layout of the
- * unpermuted E4M3 tokens; perm_tok from moe_permute).  sh.dtype ==
- * MOE_FP8_E4M3; pointers 16-byte aligned.  A perm_tok entry outside the batch
- * reports MOE_ERR_DEVICE_CHECK and leaves its word unwritten. */
-MOE_API moe_status moe_permute_fp8_scales(const void* x_scales, const int32_t* perm_tok, moe_shape sh, void* xs_perm,
-                                          void* stream);
-
-/* moe_ffn_up_fp8_quant -- the gate/up launch of moe_ffn_up_fp8 with h and hs
- * leaving it already quantized for moe_ffn_down_fp8, and the token scales
- * read in row order: xs_perm [d/128][T*k] the scales of xq_perm's rows
- * (moe_permute_fp8_scales), x_scales [d/128][T] those of xq (shared experts;
- * unused when xq is NULL).  The epilogue rounds h to bf16 as moe_ffn_up_fp8
- * writes it, then quantizes each 1x32 tile as moe_quantize_fp8 does
- * (MOE_SF_TOKENS layout), so hq / h_scales ([T*k][I] E4M3, [I/128][T*k]
- * words) and hsq / hs_scales ([T][S*Is], [S*Is/128][T]) equal moe_ffn_up_fp8
- * followed by moe_quantize_fp8, bit for bit, without the bf16 h round trip
- * through HBM.  Pointers 16-byte aligned; x_scales, hsq and hs_scales are
- * needed when xq is given and S > 0.  Errors as moe_ffn_up_fp8. */
-MOE_API moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const void* xs_perm, const int32_t* offsets,
-                                        const uint8_t* xq, const void* x_scales, const moe_fp8_experts* w,
-                                        moe_shape sh, uint8_t* hq, void* h_scales, uint8_t* hsq, void* hs_scales,
+MOE_API moe_status moe_ffn_up_fp8_quant(const uint8_t* xq_perm, const void* x_tiles, const int32_t* offsets,
+                                        const uint8_t* xq, const void* xsh_tiles, const moe_fp8_experts* w,
+                                        moe_shape sh, uint8_t* hq, void* h_tiles, uint8_t* hsq, void* hs_tiles,
                                         void* stream);
-MOE_API moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_scales, const int32_t* offsets,
-                                    const uint8_t* hsq, const void* hs_scales, const moe_fp8_experts* w,
+MOE_API moe_status moe_ffn_down_fp8(const uint8_t* hq, const void* h_tiles, const int32_t* offsets,
+                                    const uint8_t* hsq, const void* hs_tiles, const moe_fp8_experts* w,
                                     moe_shape sh, void* y_perm, void* shared_out, void* stream);
 
 /* moe_layer_forward_fp8 -- the layer with FP8 experts: route (bf16 x),
- * quantize x by tiles, permute the E4M3 rows and their scale words, gate/up
- * with h and hs quantized by tiles in its epilogue (moe_ffn_up_fp8_quant),
- * down, combine
+ * quantize x by tiles, permute the E4M3 rows, the token tile images,
+ * gate/up with h and hs quantized by tiles in its epilogue
+ * (moe_ffn_up_fp8_quant), down, combine
  * into y [T][d] bf16.  sh.dtype == MOE_FP8_E4M3;
  * workspace >= moe_workspace_size(sh). */
 MOE_API moe_status moe_layer_forward_fp8(const void* x, const void* w_gate, const float* bias,

@@ -273,10 +273,68 @@ def sf_tokens_to_rows(sf: torch.Tensor, rows: int, K: int) -> np.ndarray:
     return np.ascontiguousarray(b.transpose(1, 0, 2).reshape(rows, K // 32))
 
 
-def sf_weights_to_rows(sf: torch.Tensor, rows: int, K: int) -> np.ndarray:
-    """MOE_SF_WEIGHTS: 256-byte units [rows/64][K/128]; byte (m%32)*8 + (m/32)*4 + j
-    of unit (r/64, s) = tile 4s+j of row r, m = r % 64."""
-    nb = (rows + 63) // 64
-    b = sf.cpu().numpy().view(np.uint8)[: nb * (K // 128) * 256].reshape(nb, K // 128, 32, 2, 4)
-    # -> [unit][m/32][m%32][stage][j]
-    return np.ascontiguousarray(b.transpose(0, 3, 2, 1, 4).reshape(nb * 64, K // 32)[:rows])
+def sf_weights_to_rows(sf: torch.Tensor, rows: int, K: int, layout: int = moe.MOE_SF_WEIGHTS) -> np.ndarray:
+    """MOE_SF_WEIGHTS: 512-byte atoms [rows/128][K/128]; byte (m%32)*16 + (m/32)*4 + j
+    of atom (r/128, s) = tile 4s+j of row r, m = r % 128.
+    MOE_SF_GATE / MOE_SF_UP: 512-byte units [rows/64][K/128] shared by W1 and W3;
+    row r of W1 at m = r % 64, of W3 at m = 64 + r % 64."""
+    per = 128 if layout == moe.MOE_SF_WEIGHTS else 64
+    nb = (rows + per - 1) // per
+    b = sf.cpu().numpy().view(np.uint8)[: nb * (K // 128) * 512].reshape(nb, K // 128, 32, 4, 4)
+    if layout == moe.MOE_SF_GATE:
+        b = b[:, :, :, 0:2]
+    elif layout == moe.MOE_SF_UP:
+        b = b[:, :, :, 2:4]
+    # -> [atom][m/32][m%32][stage][j]
+    return np.ascontiguousarray(b.transpose(0, 3, 2, 1, 4).reshape(nb * per, K // 32)[:rows])
+
+
+def token_tile_split(n: int, ntt: int, tt: int):
+    """Rows (start, length) of token tile tt of a group of n rows in ntt near-equal tiles."""
+    q, r = divmod(n, ntt)
+    return tt * q + min(tt, r), q + (1 if tt < r else 0)
+
+
+def _tiles(offsets, rows):
+    """(first row, rows) of every token tile, groups in order (offsets None: one group)."""
+    bounds = [(0, rows)] if offsets is None else list(zip(offsets[:-1], offsets[1:]))
+    out = []
+    for a, b in bounds:
+        n = int(b) - int(a)
+        if n <= 0:
+            continue
+        ntt = -(-n // 256)
+        for tt in range(ntt):
+            st, ln = token_tile_split(n, ntt, tt)
+            out.append((int(a) + st, ln))
+    return out
+
+
+_IMG_POS = np.array([((j >> 7) << 7) | ((j & 31) << 2) | ((j >> 5) & 3) for j in range(256)])
+
+
+def tile_images_expected(words: np.ndarray, offsets, rows: int, nbytes: int) -> np.ndarray:
+    """The token image buffer (uint32, nbytes long) for per-row scale words [rows][K/128]:
+    the images of all tiles, zeros past each tile's rows and after the last tile."""
+    nst = words.shape[1]
+    out = np.zeros(nbytes // 4, np.uint32)
+    for i, (r0, ln) in enumerate(_tiles(offsets, rows)):
+        img = out[i * nst * 256:(i + 1) * nst * 256].reshape(nst, 256)
+        img[:, _IMG_POS[:ln]] = words[r0:r0 + ln].T
+    return out
+
+
+def tile_images_to_rows(tiles: torch.Tensor, offsets, rows: int, K: int, pad_byte=None) -> np.ndarray:
+    """Per-row tile exponent bytes [rows][K/32] read back from token images; with
+    pad_byte, also checks that the rows of each tile's last 16-row chunk past the
+    tile hold that byte in every scale."""
+    nst = K // 128
+    w = tiles.cpu().numpy().view(np.uint32)
+    out = np.zeros((rows, nst), np.uint32)
+    for i, (r0, ln) in enumerate(_tiles(offsets, rows)):
+        img = w[i * nst * 256:(i + 1) * nst * 256].reshape(nst, 256)
+        out[r0:r0 + ln] = img[:, _IMG_POS[:ln]].T
+        if pad_byte is not None:
+            pad = img[:, _IMG_POS[ln:(ln + 15) // 16 * 16]]
+            assert (pad == pad_byte * 0x01010101).all(), f"tile {i}: padding rows' scales"
+    return np.ascontiguousarray(out.view(np.uint8).reshape(rows, nst * 4))

@@ -216,13 +216,27 @@ def test_backward_binding_marshals_and_raises(L):
 
 
 def test_fp8_scale_and_fused_up_checks(L):
+    """The FP8 scale helpers and the fused gate/up validate before touching the device."""
     c = ctypes.c_void_p
     sh8 = shape(d=256, I=128, Is=128, dtype=moe.MOE_FP8_E4M3)
-    # moe_permute_fp8_scales(x_scales, perm_tok, sh, xs_perm, stream)
-    assert L.moe_permute_fp8_scales(c(FAKE), c(FAKE), shape(), c(FAKE), None) == INVALID   # not an E4M3 shape
-    assert L.moe_permute_fp8_scales(None, c(FAKE), sh8, c(FAKE), None) == INVALID
-    assert L.moe_permute_fp8_scales(c(FAKE), c(FAKE), sh8, c(FAKE + 4), None) == ALIGN
-    # moe_ffn_up_fp8_quant(xq_perm, xs_perm, offsets, xq, x_scales, w, sh, hq, h_scales, hsq, hs_scales, stream)
+    # scale buffer sizes: token words, 128-row atoms, the joint gate/up units, token tile images
+    assert moe.moe_fp8_scale_bytes(200, 256, moe.MOE_SF_TOKENS) == 200 * 2 * 4
+    assert moe.moe_fp8_scale_bytes(200, 256, moe.MOE_SF_WEIGHTS) == 2 * 2 * 512
+    assert moe.moe_fp8_scale_bytes(200, 256, moe.MOE_SF_GATE) == moe.moe_fp8_scale_bytes(200, 256, moe.MOE_SF_UP) \
+        == 4 * 2 * 512
+    assert moe.moe_fp8_scale_bytes(200, 256, 4) == 0 and moe.moe_fp8_scale_bytes(200, 200, moe.MOE_SF_TOKENS) == 0
+    assert moe.moe_fp8_tile_scale_bytes(1000, 8, 256) == (1000 // 256 + 8) * 2 * 1024
+    assert moe.moe_fp8_tile_scale_bytes(1000, 0, 256) == 0 and moe.moe_fp8_tile_scale_bytes(1000, 257, 256) == 0
+    assert moe.moe_fp8_tile_scale_bytes(1000, 8, 200) == 0
+    # moe_fp8_tile_scales(src, src_rows, K, row_of, row_div, offsets, groups, rows, tiles, stream)
+    tiles = L.moe_fp8_tile_scales
+    assert tiles(c(FAKE), 100, 256, None, 1, None, 2, 100, c(FAKE), None) == INVALID       # groups need offsets
+    assert tiles(c(FAKE), 100, 256, c(FAKE), 2, c(FAKE), 257, 100, c(FAKE), None) == INVALID  # more than 256 groups
+    assert tiles(c(FAKE), 100, 256, None, 0, None, 1, 100, c(FAKE), None) == INVALID       # row_div 0
+    assert tiles(None, 100, 256, None, 1, None, 1, 100, c(FAKE), None) == INVALID
+    assert tiles(c(FAKE), 100, 200, None, 1, None, 1, 100, c(FAKE), None) == UNSUPPORTED   # K % 128 != 0
+    assert tiles(c(FAKE), 100, 256, None, 1, None, 1, 100, c(FAKE + 4), None) == ALIGN
+    # moe_ffn_up_fp8_quant(xq_perm, x_tiles, offsets, xq, xsh_tiles, w, sh, hq, h_tiles, hsq, hs_tiles, stream)
     w8 = moe.MoEFp8Experts()
     assert L.moe_ffn_up_fp8_quant(c(FAKE), c(FAKE), c(FAKE), None, None, ctypes.byref(w8), shape(), c(FAKE), c(FAKE),
                                   None, None, None) == INVALID                              # not an E4M3 shape

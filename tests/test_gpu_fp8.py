@@ -22,11 +22,11 @@ import oracle
 from fine_grained_moe_gate_b200.inputs import CONFIGS, make_layer, make_tokens, to_numpy
 
 from gpu_harness import (DEV, as_f64, check_status, permute, rel_fro, route, sf_tokens_to_rows, sf_weights_to_rows,
-                         to_f64_rows)
+                         tile_images_expected, tile_images_to_rows, to_f64_rows)
 
 pytestmark = pytest.mark.gpu
 
-TOK, WGT = moe.MOE_SF_TOKENS, moe.MOE_SF_WEIGHTS
+TOK, WGT, GATE, UP = moe.MOE_SF_TOKENS, moe.MOE_SF_WEIGHTS, moe.MOE_SF_GATE, moe.MOE_SF_UP
 
 
 @pytest.fixture(autouse=True)
@@ -50,10 +50,10 @@ def _quant(src: torch.Tensor, rows, kseg, nseg=1, layout=TOK):
 
 
 def _exps(sc, rows, K, layout):
-    return sf_tokens_to_rows(sc, rows, K) if layout == TOK else sf_weights_to_rows(sc, rows, K)
+    return sf_tokens_to_rows(sc, rows, K) if layout == TOK else sf_weights_to_rows(sc, rows, K, layout)
 
 
-@pytest.mark.parametrize("layout", [TOK, WGT], ids=["tokens", "weights"])
+@pytest.mark.parametrize("layout", [TOK, WGT, GATE, UP], ids=["tokens", "weights", "gate", "up"])
 @pytest.mark.parametrize("rows,K,std", [(37, 256, 0.05), (9, 7168, 1.0), (300, 2048, 3e-3), (128, 128, 100.0),
                                         (5, 10240, 0.5), (64, 1408, 2.0)])
 def test_quantize_tiles_bit_exact(layout, rows, K, std):
@@ -112,11 +112,11 @@ def test_weight_quantization_matches_oracle():
     cfg, sh, p, x, q, _ = _case()
     qo = _oracle_weights(p, cfg)
     E, I, d, S, Is = cfg.E, cfg.I, cfg.d, cfg.S, cfg.Is
-    geo = {"w1": (E * I, d), "w3": (E * I, d), "w2": (E * d, I), "ws1": (S * Is, d), "ws3": (S * Is, d),
-           "ws2": (d, S * Is)}
-    for n, (rows, K) in geo.items():
+    geo = {"w1": (E * I, d, "w13s", GATE), "w3": (E * I, d, "w13s", UP), "w2": (E * d, I, "w2s", WGT),
+           "ws1": (S * Is, d, "ws13s", GATE), "ws3": (S * Is, d, "ws13s", UP), "ws2": (d, S * Is, "ws2s", WGT)}
+    for n, (rows, K, key, lay) in geo.items():
         assert np.array_equal(q[n + "q"].cpu().numpy(), qo[n + "q"]), n
-        assert np.array_equal(sf_weights_to_rows(q[n + "s"], rows, K), qo[n + "e"]), n
+        assert np.array_equal(sf_weights_to_rows(q[key], rows, K, lay), qo[n + "e"]), n
 
 
 def _bf16_close(got: torch.Tensor, ref_bits_or_f64: np.ndarray, what: str):
@@ -132,43 +132,69 @@ def _bf16_close(got: torch.Tensor, ref_bits_or_f64: np.ndarray, what: str):
     assert rel_fro(g, r) < 2e-3, what
 
 
+def _images(sc, src_rows, K, rows, offsets=None, groups=1, row_of=None, row_div=1, poison=False):
+    """Token tile images of a token-layout scale buffer through moe_fp8_tile_scales."""
+    t = moe.fp8_tile_images(rows, groups, K, DEV)
+    if poison:
+        t.fill_(0xAB)
+    moe.moe_fp8_tile_scales(sc, src_rows, K, row_of, row_div, offsets, groups, rows, t)
+    return t
+
+
 def _staged(cfg, sh, p, x, q, w8):
-    """Route, quantize x, permute, gate/up, quantize h, down -- through the C ABI."""
-    T, k, d, I, S, Is = cfg.T, cfg.k, cfg.d, cfg.I, cfg.S, cfg.Is
+    """Route, quantize x, permute, tile images, gate/up, quantize h, down -- through the C ABI."""
+    T, k, d, I, S, Is, E = cfg.T, cfg.k, cfg.d, cfg.I, cfg.S, cfg.Is, cfg.E
     idx, w, counts, _ = route(sh, x, p["w_gate"], p["bias"], with_aff=False)
     xq, xs = _quant(x, T, d)
     xq_perm, offsets, perm, inv = permute(sh, xq, idx, counts)
+    x_tiles = _images(xs, T, d, T * k, offsets, E, perm, k, poison=True)
+    xsh_tiles = _images(xs, T, d, T, poison=True) if S > 0 else None
+    torch.cuda.synchronize()
+    check_status()
+    # the images hold the unpermuted tokens' words, row by row, zeros elsewhere (every byte written)
+    off_np = offsets.cpu().numpy()
+    words = xs.view(torch.int32).view(d // 128, T).cpu().numpy().view(np.uint32).T
+    exp = tile_images_expected(words[perm.cpu().numpy() // k], off_np, T * k, x_tiles.numel())
+    assert np.array_equal(x_tiles.cpu().numpy().view(np.uint32), exp), "routed token images"
+    if S > 0:
+        assert np.array_equal(xsh_tiles.cpu().numpy().view(np.uint32),
+                              tile_images_expected(words, None, T, xsh_tiles.numel())), "shared token images"
     h = torch.empty((T * k, I), dtype=torch.bfloat16, device=DEV)
     hs = torch.empty((T, S * Is), dtype=torch.bfloat16, device=DEV) if S > 0 else None
-    moe.moe_ffn_up_fp8(xq_perm, perm, xs, offsets, xq if S > 0 else None, w8, sh, h, hs)
+    moe.moe_ffn_up_fp8(xq_perm, x_tiles, offsets, xq if S > 0 else None, xsh_tiles, w8, sh, h, hs)
     torch.cuda.synchronize()
     check_status()
     hq, h_sc = _quant(h, T * k, I)
     hsq, hs_sc = _quant(hs, T, S * Is) if S > 0 else (None, None)
-    # the same gate/up with h quantized in its epilogue: bit-identical codes and scales (buffers poisoned, so
-    # every byte must be written)
+    h_tiles = _images(h_sc, T * k, I, T * k, offsets, E)
+    hs_tiles = _images(hs_sc, T, S * Is, T) if S > 0 else None
+    # the same gate/up with h quantized in its epilogue: bit-identical codes, and images holding the same
+    # scales at every tile row (buffers poisoned, so every code byte must be written)
     fq = torch.full_like(hq, 0xAB)
-    fsc = torch.full_like(h_sc, 0xAB)
+    fimg = torch.full_like(h_tiles, 0xAB)
     fsq = torch.full_like(hsq, 0xAB) if S > 0 else None
-    fssc = torch.full_like(hs_sc, 0xAB) if S > 0 else None
-    xs_perm = torch.full_like(moe.fp8_scales(T * k, d, TOK, DEV), 0xAB)
-    moe.moe_permute_fp8_scales(xs, perm, sh, xs_perm)
-    moe.moe_ffn_up_fp8_quant(xq_perm, xs_perm, offsets, xq if S > 0 else None, xs if S > 0 else None, w8, sh, fq, fsc,
-                             fsq, fssc)
+    fsimg = torch.full_like(hs_tiles, 0xAB) if S > 0 else None
+    moe.moe_ffn_up_fp8_quant(xq_perm, x_tiles, offsets, xq if S > 0 else None, xsh_tiles, w8, sh, fq, fimg, fsq,
+                             fsimg)
     torch.cuda.synchronize()
     check_status()
-    # the permuted scale words are the unpermuted tokens' words, row by row
-    words = xs.view(torch.int32).view(d // 128, T).cpu().numpy()
-    assert np.array_equal(xs_perm.view(torch.int32).view(d // 128, T * k).cpu().numpy(),
-                          words[:, perm.cpu().numpy() // k]), "permuted scales"
-    assert torch.equal(fq, hq) and torch.equal(fsc, h_sc), "fused h quantization"
+    assert torch.equal(fq, hq), "fused h quantization: codes"
+    assert np.array_equal(tile_images_to_rows(fimg, off_np, T * k, I, pad_byte=0x7F),
+                          sf_tokens_to_rows(h_sc, T * k, I)), "fused h quantization: scales"
     if S > 0:
-        assert torch.equal(fsq, hsq) and torch.equal(fssc, hs_sc), "fused hs quantization"
+        assert torch.equal(fsq, hsq), "fused hs quantization: codes"
+        assert np.array_equal(tile_images_to_rows(fsimg, None, T, S * Is, pad_byte=0x7F),
+                              sf_tokens_to_rows(hs_sc, T, S * Is)), "fused hs quantization: scales"
     y_perm = torch.empty((T * k, d), dtype=torch.bfloat16, device=DEV)
     shared_out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV) if S > 0 else None
-    moe.moe_ffn_down_fp8(hq, h_sc, offsets, hsq, hs_sc, w8, sh, y_perm, shared_out)
+    moe.moe_ffn_down_fp8(hq, h_tiles, offsets, hsq, hs_tiles, w8, sh, y_perm, shared_out)
+    # the down projection from the fused images (poison past each tile's padded rows) is the same
+    y2 = torch.empty_like(y_perm)
+    s2 = torch.empty_like(shared_out) if S > 0 else None
+    moe.moe_ffn_down_fp8(fq, fimg, offsets, fsq, fsimg, w8, sh, y2, s2)
     torch.cuda.synchronize()
     check_status()
+    assert torch.equal(y2, y_perm) and (S == 0 or torch.equal(s2, shared_out)), "down from the fused images"
     return dict(idx=idx, w=w, counts=counts, xq=xq, xs=xs, xq_perm=xq_perm, offsets=offsets, perm=perm, inv=inv,
                 h=h, hs=hs, hq=hq, h_sc=h_sc, hsq=hsq, hs_sc=hs_sc, y_perm=y_perm, shared_out=shared_out)
 

@@ -275,17 +275,18 @@ def test_v3_fp8_prefill_and_decode(v3_layer):
     """V3 prefill (T=8192) and decode calls with per-tile E4M3 experts
     through moe_layer_forward_fp8 (what the bench times); the weights are
     quantized on the device and checked bit for bit (codes and tile
-    exponents) on three sampled experts."""
+    exponents of W1, W3 and W2) on three sampled experts."""
     from gpu_harness import sf_weights_to_rows
     _, p = v3_layer
     q = moe.quantize_experts_fp8(p)
     w8 = moe.fp8_experts(q)
     torch.cuda.synchronize()
     check_status()
-    for n in ("w1", "w2"):
+    for n, key, lay in (("w1", "w13s", moe.MOE_SF_GATE), ("w3", "w13s", moe.MOE_SF_UP),
+                        ("w2", "w2s", moe.MOE_SF_WEIGHTS)):
         rows, K = p[n].shape[1], p[n].shape[2]
         E = p[n].shape[0]
-        ex = sf_weights_to_rows(q[n + "s"], E * rows, K)
+        ex = sf_weights_to_rows(q[key], E * rows, K, lay)
         for e in (0, 77, 255):
             qo, eo = oracle.quantize_mx(to_numpy(p[n][e]))
             assert np.array_equal(q[n + "q"][e].cpu().numpy(), qo)
