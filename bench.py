@@ -486,9 +486,9 @@ def roofline_records(step, stage_ms, peaks, peak_src, dominant_ms=None):
         touched.append(int((step.counts > 0).sum().item()))
     n_touched = statistics.mean(touched)
     esz = {"bf16": 2, "fp8": 1}.get(cfg.dtype, 4)
-    if step.fp8:  # E4M3 weights and token rows in, bf16 h out
-        bytes_per_launch = (n_touched * 2 * cfg.I * d + 2 * SIs * d + T * k * d + T * d) + \
-            (T * k * cfg.I + T * SIs) * 2
+    if step.fp8:  # E4M3 codes (weights and token rows in, h out), each with one scale byte per 32
+        bytes_per_launch = (n_touched * 2 * cfg.I * d + 2 * SIs * d + T * k * d + T * d + T * k * cfg.I +
+                            T * SIs) * 33 // 32
     else:
         bytes_per_launch = (n_touched * 2 * cfg.I * d + T * k * (d + cfg.I) + 2 * SIs * d + T * (d + SIs)) * esz
     hbm_gbs = bytes_per_launch / (dom_ms / 1e3) / 1e9
