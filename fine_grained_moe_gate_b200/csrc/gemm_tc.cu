@@ -99,19 +99,22 @@ constexpr uint32_t SFA_COL = 496, SFB_COL = 504;
 constexpr int SFA_BYTES = 512, SFB_BYTES = 1024, SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
 // Epilogue warps come in groups of four (one per TMEM lane quarter); groups
 // take the tile's 16-token chunks in turn.  The gate/up epilogue (SwiGLU on
-// every element) runs two groups with one exchange buffer each; the down
-// epilogue, a plain conversion, one group with two buffers.  On short-K
-// tiles (d = 2048, E4M3) the single group paced the whole kernel.
-template <bool UP>
-__host__ __device__ constexpr int n_epi_warps() { return UP ? 8 : 4; }
-template <bool UP>
-__host__ __device__ constexpr int n_xbuf_per_group() { return UP ? 1 : 2; }
+// every element) runs two groups with one exchange buffer each.  The bf16
+// down epilogue, a plain conversion, runs one group with two buffers: a
+// second group there took issue slots from the producer lanes and measured
+// 10% slower on the V3 down projection.  The E4M3 down projection (16 K steps
+// of 128 per tile at I = 2048) runs two groups: with one, its epilogue paced
+// the launch (the MMA issuer waited for a free accumulator 28% of its time).
+template <bool UP, bool F8>
+__host__ __device__ constexpr int n_epi_warps() { return UP || F8 ? 8 : 4; }
+template <bool UP, bool F8>
+__host__ __device__ constexpr int n_xbuf_per_group() { return UP || F8 ? 1 : 2; }
 // producer warps after the epilogue warps: the token operand (both), the W3 half (up),
 // the tile scales (E4M3)
 template <bool UP, bool F8>
 __host__ __device__ constexpr int n_extra_producers() { return (UP ? 2 : 1) + (F8 ? 1 : 0); }
 template <bool UP, bool F8>
-__host__ __device__ constexpr int n_threads() { return 32 * (2 + n_epi_warps<UP>() + n_extra_producers<UP, F8>()); }
+__host__ __device__ constexpr int n_threads() { return 32 * (2 + n_epi_warps<UP, F8>() + n_extra_producers<UP, F8>()); }
 constexpr int XS = 132;                 // row stride (floats) of the epilogue exchange buffer
 constexpr int XBUF_BYTES = 16 * XS * 4; // 16 tokens x 128 lanes (+pad), fp32
 // L2 policy of the two operands' loads.  Marking the weights evict-first
@@ -125,7 +128,7 @@ constexpr int TQ = 8;                   // tile queue slots
 // the MMA issuer (leader) or the weight producer (peer)
 template <bool UP, bool F8>
 __host__ __device__ constexpr uint32_t tq_readers() {
-    return 2u * (1u + (uint32_t)n_epi_warps<UP>() + (uint32_t)n_extra_producers<UP, F8>());
+    return 2u * (1u + (uint32_t)n_epi_warps<UP, F8>() + (uint32_t)n_extra_producers<UP, F8>());
 }
 
 // Tile counters: one {next, done} pair per launch slot.  A launch takes the
@@ -167,8 +170,10 @@ struct Tables {
 // DRAM reads 18.4 -> 17.3 GB, the skewed batch's gate/up 4.5% faster.
 constexpr int SHARED_FGROUP = 8;
 constexpr size_t XBUF_TOTAL = 2 * (size_t)XBUF_BYTES;  // groups x buffers per group = 2 either way
-static_assert(n_epi_warps<true>() / 4 * n_xbuf_per_group<true>() == 2, "exchange buffers");
-static_assert(n_epi_warps<false>() / 4 * n_xbuf_per_group<false>() == 2, "exchange buffers");
+static_assert(n_epi_warps<true, false>() / 4 * n_xbuf_per_group<true, false>() == 2, "exchange buffers");
+static_assert(n_epi_warps<true, true>() / 4 * n_xbuf_per_group<true, true>() == 2, "exchange buffers");
+static_assert(n_epi_warps<false, false>() / 4 * n_xbuf_per_group<false, false>() == 2, "exchange buffers");
+static_assert(n_epi_warps<false, true>() / 4 * n_xbuf_per_group<false, true>() == 2, "exchange buffers");
 // ring, tile scales (E4M3), epilogue exchange buffers, control, tables
 template <bool F8>
 __host__ __device__ constexpr size_t sf_region_bytes() { return F8 ? (size_t)n_stages<F8>() * SF_STAGE_BYTES : 0; }
@@ -417,8 +422,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
     uint8_t* sfr = base + STAGES * STAGE_BYTES;  // tile scales of each stage (E4M3)
     float* xbuf = reinterpret_cast<float*>(sfr + sf_region_bytes<F8>());
     Ctl* ctl = reinterpret_cast<Ctl*>(reinterpret_cast<uint8_t*>(xbuf) + XBUF_TOTAL);
-    constexpr int NEPI = n_epi_warps<UP>();
-    constexpr int NXB = n_xbuf_per_group<UP>();
+    constexpr int NEPI = n_epi_warps<UP, F8>();
+    constexpr int NXB = n_xbuf_per_group<UP, F8>();
     constexpr int NTHREADS = n_threads<UP, F8>();
     Tables* tb = reinterpret_cast<Tables*>(ctl + 1);
 
