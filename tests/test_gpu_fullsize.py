@@ -271,11 +271,90 @@ def _fp8_check(cfg, p, w8, x, n_sample, seed):
     assert err <= 5e-3, err
 
 
+def _fp8_projection_checks(cfg, p, w8, x):
+    """The E4M3 stages as the bench calls them (quantize x, permute, token tile
+    images, gate/up with h quantized in its epilogue, down), at full size.
+    For the most-loaded expert, a median one, the last one with rows and the
+    shared set: h from moe_ffn_up_fp8 (bf16) element by element against the
+    oracle's up projection of the same E4M3 rows and scales; the fused
+    launch's codes and tile scales bit for bit against the oracle's
+    quantization of that h; y_perm / shared_out element by element against
+    the oracle's down projection of the fused launch's own codes and scales
+    (each launch checked alone)."""
+    from gpu_harness import sf_tokens_to_rows, tile_images_to_rows
+    sh = moe.shape_of(cfg)
+    T, k, d, E, I, S, Is = cfg.T, cfg.k, cfg.d, cfg.E, cfg.I, cfg.S, cfg.Is
+    TOK = moe.MOE_SF_TOKENS
+    idx, w, counts, _ = route(sh, x, p["w_gate"], p["bias"], with_aff=False)
+    xq = torch.empty((T, d), dtype=torch.uint8, device=DEV)
+    xs = moe.fp8_scales(T, d, TOK, DEV)
+    moe.moe_quantize_fp8(x, T, d, 1, TOK, xq, xs)
+    xq_perm, offsets, perm, inv = permute(sh, xq, idx, counts)
+    x_img, xsh_img = moe.fp8_tile_images(T * k, E, d, DEV), moe.fp8_tile_images(T, 1, d, DEV)
+    moe.moe_fp8_tile_scales(xs, T, d, perm, k, offsets, E, T * k, x_img)
+    moe.moe_fp8_tile_scales(xs, T, d, None, 1, None, 1, T, xsh_img)
+    h = torch.empty((T * k, I), dtype=torch.bfloat16, device=DEV)
+    hs = torch.empty((T, S * Is), dtype=torch.bfloat16, device=DEV)
+    moe.moe_ffn_up_fp8(xq_perm, x_img, offsets, xq, xsh_img, w8, sh, h, hs)
+    hq = torch.empty((T * k, I), dtype=torch.uint8, device=DEV)
+    hsq = torch.empty((T, S * Is), dtype=torch.uint8, device=DEV)
+    h_img, hs_img = moe.fp8_tile_images(T * k, E, I, DEV), moe.fp8_tile_images(T, 1, S * Is, DEV)
+    moe.moe_ffn_up_fp8_quant(xq_perm, x_img, offsets, xq, xsh_img, w8, sh, hq, h_img, hsq, hs_img)
+    y_perm = torch.empty((T * k, d), dtype=torch.bfloat16, device=DEV)
+    shared_out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    moe.moe_ffn_down_fp8(hq, h_img, offsets, hsq, hs_img, w8, sh, y_perm, shared_out)
+    torch.cuda.synchronize()
+    check_status()
+    off = offsets.cpu().numpy()
+    xq_o, xe_o = oracle.quantize_mx(to_numpy(x))
+    assert np.array_equal(xq.cpu().numpy(), xq_o) and np.array_equal(sf_tokens_to_rows(xs, T, d), xe_o)
+    perm_np = perm.cpu().numpy()
+    he_all = tile_images_to_rows(h_img, off, T * k, I)
+    c = counts.cpu().numpy()
+    nz = np.nonzero(c)[0]
+    by_load = nz[np.argsort(c[nz], kind="stable")]
+    picks = sorted({int(by_load[-1]), int(by_load[len(by_load) // 2]), int(nz[-1])})
+    for e in picks:
+        r0, r1 = int(off[e]), int(off[e + 1])
+        rows = _rows_to_check(r0, r1, 2048)
+        fu = np.arange(I) if r1 - r0 <= 512 else _feature_subset(I, 128, UP_OFFS)
+        fd = np.arange(d) if r1 - r0 <= 320 else _feature_subset(d, 256, DOWN_OFFS)
+        rt = torch.as_tensor(rows, device=DEV)
+        tok = perm_np[rows] // k
+        q1, e1 = oracle.quantize_mx(to_numpy(p["w1"][e]))
+        q3, e3 = oracle.quantize_mx(to_numpy(p["w3"][e]))
+        q2, e2 = oracle.quantize_mx(to_numpy(p["w2"][e]))
+        h_ref = oracle.expert_up_mx(xq_o[tok], xe_o[tok], q1[fu], e1[fu], q3[fu], e3[fu])
+        check_bf16_close(as_f64(h[rt][:, torch.as_tensor(fu, device=DEV)]), to_f64_rows(h_ref),
+                         f"{cfg.name} h of expert {e} ({r1 - r0} rows)")
+        hq_o, he_o = oracle.quantize_mx(to_numpy(h[rt]))
+        assert np.array_equal(hq[rt].cpu().numpy(), hq_o), f"fused h codes of expert {e}"
+        assert np.array_equal(he_all[rows], he_o), f"fused h scales of expert {e}"
+        o_ref = oracle.expert_down_mx(hq_o, he_o, q2[fd], e2[fd])
+        check_bf16_close(as_f64(y_perm[rt][:, torch.as_tensor(fd, device=DEV)]), o_ref,
+                         f"{cfg.name} y_perm of expert {e} ({r1 - r0} rows)")
+    rows = _rows_to_check(0, T, 640) if T > 640 else np.arange(T)
+    rt = torch.as_tensor(rows, device=DEV)
+    fu = _feature_subset(S * Is, 128, UP_OFFS)
+    fd = _feature_subset(d, 256, DOWN_OFFS)
+    q1, e1 = oracle.quantize_mx(to_numpy(p["ws1"]).reshape(S * Is, d))
+    q3, e3 = oracle.quantize_mx(to_numpy(p["ws3"]).reshape(S * Is, d))
+    q2, e2 = oracle.quantize_mx(to_numpy(p["ws2"]), nseg=S)
+    h_ref = oracle.expert_up_mx(xq_o[rows], xe_o[rows], q1[fu], e1[fu], q3[fu], e3[fu])
+    check_bf16_close(as_f64(hs[rt][:, torch.as_tensor(fu, device=DEV)]), to_f64_rows(h_ref), f"{cfg.name} hs")
+    hsq_o, hse_o = oracle.quantize_mx(to_numpy(hs[rt]))
+    assert np.array_equal(hsq[rt].cpu().numpy(), hsq_o), "fused hs codes"
+    assert np.array_equal(tile_images_to_rows(hs_img, None, T, S * Is)[rows], hse_o), "fused hs scales"
+    o_ref = oracle.expert_down_mx(hsq_o, hse_o, q2[:, fd], e2[fd])   # q2 [S][d][Is], K joined over the blocks
+    check_bf16_close(as_f64(shared_out[rt][:, torch.as_tensor(fd, device=DEV)]), o_ref, f"{cfg.name} shared_out")
+
+
 def test_v3_fp8_prefill_and_decode(v3_layer):
     """V3 prefill (T=8192) and decode calls with per-tile E4M3 experts
     through moe_layer_forward_fp8 (what the bench times); the weights are
     quantized on the device and checked bit for bit (codes and tile
-    exponents of W1, W3 and W2) on three sampled experts."""
+    exponents of W1, W3 and W2) on three sampled experts; the prefill
+    batch's stages also expert by expert (_fp8_projection_checks)."""
     from gpu_harness import sf_weights_to_rows
     _, p = v3_layer
     q = moe.quantize_experts_fp8(p)
@@ -293,6 +372,7 @@ def test_v3_fp8_prefill_and_decode(v3_layer):
             assert np.array_equal(ex[e * rows:(e + 1) * rows], eo)
     cfg = CONFIGS["v3_prefill_fp8"]
     _fp8_check(cfg, p, w8, make_tokens(cfg, DEV), n_sample=16, seed=12)
+    _fp8_projection_checks(cfg, p, w8, make_tokens(cfg, DEV))
     cfg = CONFIGS["v3_decode_fp8"]
     for call in (0, 999):
         _fp8_check(cfg, p, w8, make_tokens(cfg, DEV, call), n_sample=8, seed=call)
