@@ -73,7 +73,7 @@ constexpr int BK = 64;                  // bf16 K per stage: one 128-byte swizzl
 template <bool F8>
 __host__ __device__ constexpr int bk_elems() { return F8 ? 128 : 64; }
 // Ring depth of the operand tiles (an E4M3 stage also carries its tile scales)
-template <bool F8>
+template <bool UP, bool F8>
 __host__ __device__ constexpr int n_stages() { return 6; }
 constexpr int A_BYTES = 128 * BK * 2;   // this CTA's 128 weight rows
 constexpr int B_ROWS = 128;             // this CTA's half of <= 256 tokens
@@ -175,15 +175,19 @@ static_assert(n_epi_warps<true, true>() / 4 * n_xbuf_per_group<true, true>() == 
 static_assert(n_epi_warps<false, false>() / 4 * n_xbuf_per_group<false, false>() == 2, "exchange buffers");
 static_assert(n_epi_warps<false, true>() / 4 * n_xbuf_per_group<false, true>() == 2, "exchange buffers");
 // ring, tile scales (E4M3), epilogue exchange buffers, control, tables
-template <bool F8>
-__host__ __device__ constexpr size_t sf_region_bytes() { return F8 ? (size_t)n_stages<F8>() * SF_STAGE_BYTES : 0; }
-template <bool F8>
+template <bool UP, bool F8>
+__host__ __device__ constexpr size_t sf_region_bytes() { return F8 ? (size_t)n_stages<UP, F8>() * SF_STAGE_BYTES : 0; }
+template <bool UP, bool F8>
 __host__ __device__ constexpr size_t smem_bytes() {
-    return 1024 + (size_t)n_stages<F8>() * STAGE_BYTES + sf_region_bytes<F8>() + XBUF_TOTAL + sizeof(Ctl) +
+    return 1024 + (size_t)n_stages<UP, F8>() * STAGE_BYTES + sf_region_bytes<UP, F8>() + XBUF_TOTAL + sizeof(Ctl) +
            sizeof(Tables);
 }
-static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory budget");
-static_assert(n_stages<false>() <= MAX_STAGES && n_stages<true>() <= MAX_STAGES, "ring depth");
+static_assert(smem_bytes<false, false>() <= 232448 && smem_bytes<false, true>() <= 232448 &&
+                  smem_bytes<true, false>() <= 232448 && smem_bytes<true, true>() <= 232448,
+              "shared memory budget");
+static_assert(n_stages<false, false>() <= MAX_STAGES && n_stages<false, true>() <= MAX_STAGES &&
+                  n_stages<true, false>() <= MAX_STAGES && n_stages<true, true>() <= MAX_STAGES,
+              "ring depth");
 
 
 // Tensor maps of one expert set: weights (w1 only for the up projection),
@@ -415,12 +419,12 @@ template <bool UP, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(), 1)
     tc_grouped_gemm_kernel(const __grid_constant__ SetMaps ma, const __grid_constant__ SetMaps mb,
                            const __grid_constant__ CUtensorMap tmXg, const Params p) {
-    constexpr int STAGES = n_stages<F8>();
+    constexpr int STAGES = n_stages<UP, F8>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = base;
     uint8_t* sfr = base + STAGES * STAGE_BYTES;  // tile scales of each stage (E4M3)
-    float* xbuf = reinterpret_cast<float*>(sfr + sf_region_bytes<F8>());
+    float* xbuf = reinterpret_cast<float*>(sfr + sf_region_bytes<UP, F8>());
     Ctl* ctl = reinterpret_cast<Ctl*>(reinterpret_cast<uint8_t*>(xbuf) + XBUF_TOTAL);
     constexpr int NEPI = n_epi_warps<UP, F8>();
     constexpr int NXB = n_xbuf_per_group<UP, F8>();
@@ -956,7 +960,7 @@ template <bool UP, bool F8>
 cudaError_t launch(const SetMaps& a, const SetMaps& b, const CUtensorMap& xg, Params p, int num_sms, cudaStream_t st) {
     auto kern = tc_grouped_gemm_kernel<UP, F8>;
     p.sched_slot = (int)(g_sched_seq.fetch_add(1u, std::memory_order_relaxed) % (unsigned int)kSchedSlots);
-    constexpr size_t SMEM = smem_bytes<F8>();
+    constexpr size_t SMEM = smem_bytes<UP, F8>();
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
     constexpr int NTHREADS = n_threads<UP, F8>();
     if (err != cudaSuccess) return err;
