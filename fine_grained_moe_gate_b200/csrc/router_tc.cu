@@ -332,14 +332,36 @@ __global__ void __launch_bounds__(n_threads<PAIR>(), 1)
             }
         }
         __syncthreads();
-        // top-k: P threads per token, thread `sub` pushes experts sub, sub + P, ...
+        // top-k: P threads per token, thread `sub` takes experts sub, sub + P, ...
         const int rl = u / P, sub = u - rl * P;
         const int t = t0 + tl0 + rl;
         TopK<KMAX> tk;
         tk.init();
-        for (int e = sub; e < E; e += P) {
-            const float s = sc[rl * PS + e];
-            tk.push(__fadd_rn(s, ctl->bias[e]), s, e);
+        if (P >= k && E <= 32 * P) {
+            // The P threads' largest v are P >= k distinct experts, so the k-th
+            // largest v of the token is at least their minimum: experts below it
+            // cannot be chosen.  Each thread marks its experts at or above it in a
+            // bit mask and pushes only those, in expert order; without the mask
+            // the warp ran the insertion for every expert that any lane inserted.
+            float vmax = -FLT_MAX;
+            for (int e = sub; e < E; e += P) vmax = fmaxf(vmax, __fadd_rn(sc[rl * PS + e], ctl->bias[e]));
+            float th = vmax;
+#pragma unroll
+            for (int o = P / 2; o > 0; o >>= 1) th = fminf(th, __shfl_xor_sync(0xffffffffu, th, o));
+            uint32_t mask = 0u;
+            for (int e = sub, j = 0; e < E; e += P, ++j)
+                if (__fadd_rn(sc[rl * PS + e], ctl->bias[e]) >= th) mask |= 1u << j;
+            while (mask) {
+                const int e = sub + (__ffs(mask) - 1) * P;
+                mask &= mask - 1u;
+                const float s = sc[rl * PS + e];
+                tk.push(__fadd_rn(s, ctl->bias[e]), s, e);
+            }
+        } else {
+            for (int e = sub; e < E; e += P) {
+                const float s = sc[rl * PS + e];
+                tk.push(__fadd_rn(s, ctl->bias[e]), s, e);
+            }
         }
         {  // merge the P lists in (v desc, index asc) order
             TopK<KMAX> m;
