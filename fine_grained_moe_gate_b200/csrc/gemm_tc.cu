@@ -1,5 +1,5 @@
 // Grouped expert GEMMs on the sm_100a tensor cores (2-SM tcgen05 MMA, TMEM,
-// TMA) for the bf16 layer ("Scaling Efficiency: A Deep Dive into the
+// TMA) for bf16 and block-scaled E4M3 experts ("Scaling Efficiency: A Deep Dive into the
 // DeepSeek-V3 Architecture", DeepSeekMoE sketch: one MLP per expert over the
 // tokens routed to it; "DeepSeek V3 Architecture Deep Dive ...", "Throughput
 // on NVIDIA H100/H800": tokens of one expert batched together).
@@ -34,7 +34,7 @@
 // find them in L2, and the last tiles spread over the clusters that are free.
 // Per expert, token tiles are walked fastest, then feature tiles.
 //
-// Warp roles per CTA (up: 12 warps, down: 7):
+// Warp roles per CTA (bf16 up: 12 warps, down: 7; E4M3 up: 13, down: 12):
 //   warp 0      weight producer (one lane), both CTAs: loads this CTA's
 //               weight rows (up: the W1 half), completion counted on the
 //               leader CTA's stage barrier, which the leader's lane arms with
@@ -45,7 +45,7 @@
 //               tile's loads).
 //   warp 1      TMEM owner (paired allocation); in the leader (even) CTA one
 //               lane issues the MMAs and commits to both CTAs' barriers.
-//   warps 2..   epilogue (up: 8 warps, down: 4): tcgen05.ld 32 lanes x 16
+//   warps 2..   epilogue (up and E4M3 down: 8 warps, bf16 down: 4): tcgen05.ld 32 lanes x 16
 //               tokens into shared memory, SwiGLU / bf16 conversion,
 //               token-major vector stores.  Two 256-column TMEM accumulators
 //               let the epilogue of one tile overlap the main loop of the next.
@@ -55,7 +55,9 @@
 //               long as the unit takes to accept its bytes, so one thread
 //               issuing all of a stage's loads left the tensor pipe waiting;
 //               spreading a stage's loads over warps measured the up
-//               projection 13-15% and the V3 step 7% faster.
+//               projection 13-15% and the V3 step 7% faster.  E4M3: one
+//               more warp loads each stage's tile scales (weight atom and
+//               token image) onto the same stage barrier.
 // Every wait is bounded (common.cuh); on a timeout the CTA raises its abort
 // flag, drains what it issued, frees TMEM and exits (the peer then times out
 // on its next wait and does the same).
