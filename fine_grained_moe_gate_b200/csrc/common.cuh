@@ -221,9 +221,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive on an mbarrier given by its shared::cluster address (local or peer).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+// Relaxed arrive on an mbarrier given by its shared::cluster address (local or
+// peer): no memory ordering.
+// For signals whose data is ordered by other means (a tile index delivered by
+// st.async, tensor memory read with tcgen05.ld and tcgen05.wait::ld before
+// the arrive, then tcgen05.fence::before_thread_sync).
+__device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 // Tiled TMA loads for a 2-SM MMA: data land in this CTA's shared memory,
 // completion bytes are counted on the barrier at `bar_cluster` (the pair

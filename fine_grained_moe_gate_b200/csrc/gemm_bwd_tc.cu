@@ -538,7 +538,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<WG>(), 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(leader_tempty + 8u * (uint32_t)acc);
+            // the accumulator's tcgen05.ld have completed (wait::ld above): a relaxed arrive frees it (a
+            // cluster-scope release here cost about 1 us per tile and warp)
+            if (lane == 0) mbar_arrive_relaxed_cluster(leader_tempty + 8u * (uint32_t)acc);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }

@@ -341,9 +341,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_ba
                  "r"(bytes)
                  : "memory");
 }
-__device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
-}
 
 // Reader side of the tile queue: wait for slot j, take its tile, free the
 // slot for the leader's producer.  Returns false on a timeout or abort.
@@ -943,7 +940,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(leader_tempty + 8u * (uint32_t)acc);
+            // the accumulator's tcgen05.ld have completed (wait::ld above): a relaxed arrive frees it (a
+            // cluster-scope release here cost about 1 us per tile and warp)
+            if (lane == 0) mbar_arrive_relaxed_cluster(leader_tempty + 8u * (uint32_t)acc);
             acc_ph ^= 1u << acc;
         }
     }
