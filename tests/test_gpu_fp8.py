@@ -276,6 +276,57 @@ def test_layer_forward_fp8_equals_staged_calls_and_oracle():
     assert rel_fro(as_f64(y), to_f64_rows(y_o)) < 5e-3
 
 
+@pytest.mark.parametrize("sizes", [
+    [0, 256, 257, 0, 1, 512, 513, 100],     # empty groups, exactly one and two tiles, a tile of one row
+    [3000],                                  # one group of 12 tiles of 250
+    [1] * 64,                                # 64 single-row groups
+    [255, 0, 0, 767, 1280],                  # tiles of 255, 256 and 256
+], ids=["mixed", "one_group", "single_rows", "wide"])
+@pytest.mark.parametrize("gather", [False, True], ids=["rows", "gathered"])
+def test_token_tile_images_bit_exact(sizes, gather):
+    """moe_fp8_tile_scales against images built on the host from the same words and the tile split (a group of n
+    rows as ceil(n/256) near-equal tiles), every byte of the buffer; with a row index and a divisor (as perm_tok / k
+    for the routed rows) the words come from the indexed source rows."""
+    G = len(sizes)
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    rows = int(off[-1])
+    K, k = 384, 3
+    src_rows = rows if not gather else (rows + k - 1) // k + 5
+    g = np.random.default_rng(rows + G)
+    words = g.integers(0, 2 ** 32, size=(K // 128, src_rows), dtype=np.uint64).astype(np.uint32)
+    src = torch.as_tensor(words.view(np.int32), device=DEV)
+    row_of = None
+    src_row = np.arange(rows)
+    if gather:
+        idx = g.permutation(rows).astype(np.int32) % (src_rows * k)
+        row_of = torch.as_tensor(idx, device=DEV)
+        src_row = idx // k
+    tiles = _images(src, src_rows, K, rows, torch.as_tensor(off, device=DEV), G, row_of, k if gather else 1,
+                    poison=True)
+    torch.cuda.synchronize()
+    check_status()
+    exp = tile_images_expected(words.T[src_row], off, rows, tiles.numel())
+    assert np.array_equal(tiles.cpu().numpy().view(np.uint32), exp)
+
+
+def test_token_tile_images_device_check():
+    """A group reaching past the operand's rows, or a row index past the source, reports MOE_ERR_DEVICE_CHECK
+    (its words stay 0) instead of reading out of bounds."""
+    K = 128
+    src = torch.zeros((1, 64), dtype=torch.int32, device=DEV)
+    off = torch.as_tensor(np.array([0, 40, 80], np.int32), device=DEV)     # 80 rows claimed, 64 given
+    t = moe.fp8_tile_images(64, 2, K, DEV)
+    moe.moe_fp8_tile_scales(src, 64, K, None, 1, off, 2, 64, t)
+    torch.cuda.synchronize()
+    assert moe.moe_get_last_error() == 6  # MOE_ERR_DEVICE_CHECK
+    bad = torch.as_tensor(np.array([0, 1, 999, 3], np.int32), device=DEV)  # row 2 points past the 64 source rows
+    t = moe.fp8_tile_images(4, 1, K, DEV)
+    moe.moe_fp8_tile_scales(src, 64, K, bad, 1, None, 1, 4, t)
+    torch.cuda.synchronize()
+    assert moe.moe_get_last_error() == 6  # MOE_ERR_DEVICE_CHECK
+    check_status()
+
+
 def test_fp8_rejected_by_bf16_weight_calls():
     cfg, sh, p, x, q, w8 = _case(T=16)
     ws = torch.empty(1 << 20, dtype=torch.uint8, device=DEV)
