@@ -28,9 +28,11 @@
 // Two paths compute these.  bf16 layers whose widths are multiples of 128 run
 // every contraction on the tensor cores (gemm_bwd_tc.cu: bf16 operands, fp32
 // accumulation) over a padded row layout (each expert's rows padded to a
-// multiple of 64 with zero rows); there the routed dw comes without
-// recomputing o: with u_r = W2_e^T dy_t (the dh GEMM run on the unweighted
-// dy), dw_tj = <dy_t, W2_e h_r> = <u_r, h_r> and dh_r = w_tj u_r.  Every
+// multiple of 64 with zero rows); there a, g and h are recomputed by one
+// launch of the forward's gate/up kernel (the forward's own h, with the fp32
+// a and g beside it), and the routed dw comes without recomputing o: with
+// u_r = W2_e^T dy_t (the dh GEMM run on the unweighted dy),
+// dw_tj = <dy_t, W2_e h_r> = <u_r, h_r> and dh_r = w_tj u_r.  Every
 // other layer runs two fp32 SIMT kernels over strided operand views (no
 // transposed copies): a "rows" GEMM (C[r][n] = sum_k A(r,k) B_g(n,k) for the
 // rows r of group g) and a weight-gradient GEMM whose contraction runs over a
@@ -590,21 +592,6 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// h[pr] = bf16(silu(a[pr]) * g[pr]) for the real rows (prow; null: rows 0..R-1), n columns, 4 at a time.
-__global__ void swiglu_h_kernel(const float* __restrict__ a, const float* __restrict__ g,
-                                const int32_t* __restrict__ prow, int R, int n, uint2* __restrict__ h) {
-    const int n4 = n / 4;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)R * n4;
-         i += (long long)gridDim.x * blockDim.x) {
-        const int r = (int)(i / n4), c = (int)(i - (long long)r * n4);
-        const long long pr = prow ? prow[r] : r;
-        const float4 av = reinterpret_cast<const float4*>(a + pr * n)[c];
-        const float4 gv = reinterpret_cast<const float4*>(g + pr * n)[c];
-        h[pr * n4 + c] = make_uint2(bf16x2(av.x * sigmoid_acc(av.x) * gv.x, av.y * sigmoid_acc(av.y) * gv.y),
-                                    bf16x2(av.z * sigmoid_acc(av.z) * gv.z, av.w * sigmoid_acc(av.w) * gv.w));
-    }
-}
-
 // One warp per assignment q = t*k + j (row r = inv[q], padded row pr):
 // dy_pad[pr] = bf16(dy_t), do_pad[pr] = bf16(w[q] dy_t).  d % 4 == 0:
 // 16-byte loads, 8-byte stores.
@@ -952,17 +939,42 @@ cudaError_t experts_backward_tc(const BackwardArgs& a, const BwdBufs& b, int* st
         return w;
     };
 
-    // ---- routed experts
-    // recompute a = x W1^T, g = x W3^T (fp32), h = bf16(silu(a) g) as the forward
-    TC_TRY(launch_bwd_rows_kmajor(rows_args(a.w1, (long long)E * I, I, b.x_pad, Rp, d, I, b.a_pad, true), status,
-                                  num_sms, st));
-    TC_TRY(launch_bwd_rows_kmajor(rows_args(a.w3, (long long)E * I, I, b.x_pad, Rp, d, I, b.g_pad, true), status,
-                                  num_sms, st));
-    if (R > 0) {
-        swiglu_h_kernel<<<ew_grid((long long)R * I / 4), 256, 0, st>>>(b.a_pad, b.g_pad, b.prow, R, I,
-                                                                       reinterpret_cast<uint2*>(b.h_pad));
-        note_launches(1);
+    // ---- recompute, routed and shared experts in one launch of the forward's gate/up GEMM: a = x W1^T and
+    // g = x W3^T (fp32) beside h = bf16(silu(a) g), the very h the forward computed.  The routed groups are the
+    // padded segments (pstart), whose zero padding rows give a = g = h = 0; the shared set is one group of T rows.
+    {
+        TcUpArgs ur{};
+        ur.A = b.x_pad;
+        ur.A_rows = Rp;
+        ur.gather_div = 1;
+        ur.W1 = a.w1;
+        ur.W3 = a.w3;
+        ur.W_rows = (long long)E * I;
+        ur.H = b.h_pad;
+        ur.d = d;
+        ur.I = I;
+        ur.offsets = b.pstart;
+        ur.G = E;
+        ur.pre_a = b.a_pad;
+        ur.pre_g = b.g_pad;
+        TcUpArgs us{};
+        us.A = a.x;
+        us.A_rows = T;
+        us.gather_div = 1;
+        us.W1 = a.ws1;
+        us.W3 = a.ws3;
+        us.W_rows = (long long)S * Is;
+        us.H = b.hs16;
+        us.d = d;
+        us.I = S * Is;
+        us.G = 1;
+        us.M = T;
+        us.pre_a = b.as32;
+        us.pre_g = b.gs32;
+        TC_TRY(launch_tc_up(R > 0 ? &ur : nullptr, S > 0 && T > 0 ? &us : nullptr, status, num_sms, st));
     }
+
+    // ---- routed experts
     // dy_t and do = w dy_t (bf16) on every assignment's padded row; dy_pad lives in the o_pad buffer,
     // which dx_perm overwrites only after its last use.  Its padding rows are never cleared: a B row of
     // the rows GEMM only reaches the output row of the same index, and padding rows are not stored.
@@ -1002,13 +1014,10 @@ cudaError_t experts_backward_tc(const BackwardArgs& a, const BwdBufs& b, int* st
 
     // ---- shared experts: one group of T rows (rows past T read as zeros), S blocks stacked along the features
     if (S > 0 && T > 0) {
-        TC_TRY(launch_bwd_rows_kmajor(rows_args(a.ws1, SI, 0, a.x, T, d, SI, b.as32, false), status, num_sms, st));
-        TC_TRY(launch_bwd_rows_kmajor(rows_args(a.ws3, SI, 0, a.x, T, d, SI, b.gs32, false), status, num_sms, st));
-        swiglu_h_kernel<<<ew_grid((long long)T * SI / 4), 256, 0, st>>>(b.as32, b.gs32, nullptr, T, SI,
-                                                                        reinterpret_cast<uint2*>(b.hs16));
+        // (as, gs and hs came with the recompute launch above)
         to_bf16_kernel<<<ew_grid((long long)T * d), 256, 0, st>>>(a.dy, (long long)T * d,
                                                                   reinterpret_cast<__nv_bfloat16*>(b.dys16));
-        note_launches(2);
+        note_launches(1);
         const size_t eb = 2;
         for (int s = 0; s < S; ++s) {
             const char* w2s = static_cast<const char*>(a.ws2) + eb * (size_t)s * d * Is;

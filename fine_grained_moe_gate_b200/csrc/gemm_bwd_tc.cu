@@ -9,14 +9,16 @@
 // every per-row operand, and every group's segment is padded with zero rows
 // up to a multiple of 64 (the rows past rows[g] are never written).
 //
-//   rows (input-gradient / recompute): out[r][m] (+)= sum_k A_g(m, k) B(r, k)
-//     for the rows r of group g -- the weight of the group is the MMA's M
-//     operand (256 of its output features per CTA pair), the group's rows the
-//     N operand (token tiles of <= 256 rows, as in the forward).  A is read
-//     K-major (a = x W1^T, g = x W3^T, o = h W2^T: the weights' natural
-//     [out][in] layout) or MN-major (dh = do W2, dx = da W1 + dg W3: the
-//     weights read along their output dimension, no transposed copy); for dx
-//     the contraction runs over W1's rows and then W3's (two tensor maps).
+//   rows (input gradients): out[r][m] (+)= sum_k A_g(m, k) B(r, k) for the
+//     rows r of group g -- the weight of the group is the MMA's M operand
+//     (256 of its output features per CTA pair), the group's rows the N
+//     operand (token tiles of <= 256 rows, as in the forward).  A is read
+//     MN-major (u = dy W2, dx = da W1 + dg W3: the weights read along their
+//     output dimension from their natural [out][in] layout, no transposed
+//     copy); for dx the contraction runs over W1's rows and then W3's (two
+//     tensor maps).  The template keeps the K-major form of A as well; the
+//     recompute of a = x W1^T and g = x W3^T, which read it so, runs in the
+//     forward's gate/up kernel instead (h comes out of the same launch).
 //   wgrad (weight gradients): out_g[m][n] = sum_{r in g} A(r, m) B(r, n) --
 //     M and N the weight's two dimensions (256 x 256 tiles per CTA pair), the
 //     contraction over the group's padded rows (64 per stage, the zero rows
@@ -568,35 +570,6 @@ cudaError_t launch_bwd(const Maps& m, const BwdParams& p, int num_sms, cudaStrea
 }
 
 }  // namespace
-
-// rows kind, A K-major: out[r][m] (+)= sum_k W[g * a_grow + m][k] * X[r][k]
-//   W: [Wrows][K] bf16, X: [op_rows][K] bf16, out: [op_rows][ldo] fp32.
-cudaError_t launch_bwd_rows_kmajor(const BwdRowsArgs& a, int* status, int num_sms, cudaStream_t st) {
-    Maps m{};
-    if (a.K % BK != 0 || a.M_total % 16 != 0) return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&m.a0, a.W, a.K, a.W_rows, a.K, 64, 128) || !make_tmap_2d(&m.a1, a.W, a.K, a.W_rows, a.K, 64, 128))
-        return cudaErrorInvalidValue;
-    for (int b = 0; b < NXBOX; ++b)
-        if (!make_tmap_2d(&m.bx[b], a.X, a.K, a.op_rows, a.K, 64, 16 * (b + 1))) return cudaErrorInvalidValue;
-    m.b = m.a0;
-    BwdParams p{};
-    p.G = a.G;
-    p.start = a.start;
-    p.rows = a.rows;
-    p.M_rows = a.M_rows;
-    p.op_rows = a.op_rows;
-    p.M_total = a.M_total;
-    p.m_tiles = (a.M_total + 255) / 256;
-    p.n_tiles = 1;
-    p.k_blocks = a.K / BK;
-    p.k_split = 0;
-    p.a_grow = a.a_grow;
-    p.out = a.out;
-    p.ldo = a.ldo;
-    p.accumulate = a.accumulate ? 1 : 0;
-    p.status = status;
-    return launch_bwd<false, false, false>(m, p, num_sms, st);
-}
 
 // rows kind, A MN-major: out[r][m] (+)= sum_k W(k, m) X[r][k] with W(k, m) =
 //   W0[g * a_grow + k][m] for k < K0, then W1[g * a_grow + k - K0][m];

@@ -232,6 +232,10 @@ struct SetParams {
     // unused.
     uint8_t* q_out;
     uint32_t* q_img;
+    // up, bf16 only, optional: the fp32 pre-activations (gate rows into a_out,
+    // up rows into g_out, [rows][ldo]) beside h.
+    float* a_out;
+    float* g_out;
 };
 struct Params {
     const int32_t* offsets;
@@ -896,6 +900,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(n_threads<UP, F8>(),
                         v.z = pack_bf16x2(silu_fast(g1.x) * u1.x, silu_fast(g1.y) * u1.y);
                         v.w = pack_bf16x2(silu_fast(g1.z) * u1.z, silu_fast(g1.w) * u1.w);
                         *reinterpret_cast<uint4*>(out + (size_t)(tok0 + c + my_tok) * sp.ldo + fcta + fj) = v;
+                        if (!F8 && sp.a_out) {
+                            const size_t o = (size_t)(tok0 + c + my_tok) * sp.ldo + fcta + fj;
+                            float4* ad = reinterpret_cast<float4*>(sp.a_out + o);
+                            float4* gd = reinterpret_cast<float4*>(sp.g_out + o);
+                            ad[0] = g0;
+                            ad[1] = g1;
+                            gd[0] = u0;
+                            gd[1] = u1;
+                        }
                     }
                 } else {
                     const int fj = part * 16;
@@ -1000,6 +1013,9 @@ bool up_set(const TcUpArgs& a, SetMaps& m, SetParams& sp) {
     sp.q_out = a.f8 ? a.hq : nullptr;
     sp.q_img = a.f8 ? a.hq_img : nullptr;
     if (sp.q_out && !sp.q_img) return false;
+    sp.a_out = a.f8 ? nullptr : a.pre_a;
+    sp.g_out = a.f8 ? nullptr : a.pre_g;
+    if (!sp.a_out != !sp.g_out) return false;
     return true;
 }
 

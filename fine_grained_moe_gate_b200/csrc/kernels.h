@@ -120,7 +120,6 @@ struct BwdRowsArgs {
     int ldo;
     bool accumulate;
 };
-cudaError_t launch_bwd_rows_kmajor(const BwdRowsArgs& a, int* status, int num_sms, cudaStream_t st);
 cudaError_t launch_bwd_rows_mnmajor(const BwdRowsArgs& a, int* status, int num_sms, cudaStream_t st);
 // out[g][m][n] = sum over group g's rows r (padded to 64) of A[r][a_col0 + m] * B[r][b_col0 + n]
 struct BwdWgradArgs {
@@ -174,6 +173,11 @@ struct TcUpArgs {
     // 1024 bytes, the same tiles) instead of bf16 H.
     uint8_t* hq = nullptr;
     uint32_t* hq_img = nullptr;
+    // bf16 only, optional: also write the fp32 pre-activations a = W1 . x
+    // (pre_a) and g = W3 . x (pre_g), [A_rows][I] each, beside h (the
+    // backward's recompute).
+    float* pre_a = nullptr;
+    float* pre_g = nullptr;
 };
 // Down projection: Y[r][:] = H[r] . W2_g^T, W2_g = [d][K] (K = I), or for
 // the shared group S stacked [d][Is] blocks contracted over K = S * Is.
