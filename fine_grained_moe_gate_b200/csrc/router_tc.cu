@@ -249,6 +249,16 @@ __global__ void __launch_bounds__(n_threads<PAIR>(), 1)
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
             TopK<KMAX> tk;
             tk.init();
+            // Scores into shared memory (the operand ring is free now), column e of token r at
+            // sbuf[e * BM + r], with the maxima of v = s + b over the KMAX expert classes e % KMAX: those
+            // are KMAX >= k distinct experts, so the token's k-th largest v is at least their minimum and
+            // experts below it cannot be chosen.  The pushes then take only the experts at or above it,
+            // popped from a bit mask in expert order (pushing every expert ran the sorted-list insertion
+            // for the whole warp whenever one lane needed it).
+            float* sbuf = part;
+            float gmax[KMAX];
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) gmax[j] = -FLT_MAX;
             for (int c = 0; c < n_pad; c += 16) {
                 uint32_t v[16];
                 tmem_ld16(taddr + (uint32_t)c, v);
@@ -258,9 +268,25 @@ __global__ void __launch_bounds__(n_threads<PAIR>(), 1)
                     const int e = c + i;
                     if (e < E) {
                         const float s = sigmoid_f32(__uint_as_float(v[i]));
-                        tk.push(__fadd_rn(s, ctl->bias[e]), s, e);
+                        sbuf[e * BM + r] = s;
+                        gmax[i % KMAX] = fmaxf(gmax[i % KMAX], __fadd_rn(s, ctl->bias[e]));
                         if (aff && t < T) aff[(size_t)t * E + e] = s;
                     }
+                }
+            }
+            float th = gmax[0];
+#pragma unroll
+            for (int j = 1; j < KMAX; ++j) th = fminf(th, gmax[j]);
+            if (E < KMAX) th = -FLT_MAX;  // a class without experts: no bound
+            for (int e0 = 0; e0 < E; e0 += 32) {
+                uint32_t mask = 0u;
+                for (int i = 0; i < 32 && e0 + i < E; ++i)
+                    if (__fadd_rn(sbuf[(e0 + i) * BM + r], ctl->bias[e0 + i]) >= th) mask |= 1u << i;
+                while (mask) {
+                    const int e = e0 + __ffs(mask) - 1;
+                    mask &= mask - 1u;
+                    const float s = sbuf[e * BM + r];
+                    tk.push(__fadd_rn(s, ctl->bias[e]), s, e);
                 }
             }
             if (t < T) emit_route<KMAX>(tk, k, idx + (size_t)t * k, w + (size_t)t * k, ctl->hist, status);
